@@ -1,0 +1,355 @@
+/*
+ * CPU oracle for the quantized linear layer Y = dequant(Xq) . dequant(Wq)^T.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or constant with the CUDA path, and the CUDA path never
+ * calls it.
+ *
+ * It is deliberately plain and slow: every step is the textbook definition,
+ * written out, in exact integer or fp64 arithmetic.
+ *
+ * Sources (article "Building a High-Performance and Portable vLLM Linear
+ * Backend with Helion", as summarised and translated on the pages it was
+ * published on):
+ *   - formats: "Put algorithm selection inside the search space" (three
+ *     formats: FP8_Dynamic per-token activation / per-channel weight scales;
+ *     W8A8_INT8 with the same granularity; Block_FP8 with 1x128 activation
+ *     and 128x128 weight scales), and the "Alcance" (scope) list of the
+ *     Spanish translation, which restates the same three formats.
+ *   - every variant (Standard, Split-K, Swap-AB) computes the same product;
+ *     only the accumulation path differs ("Put algorithm selection inside
+ *     the search space"; the matmul listing under "Codigo").
+ *   - scale formula (absmax/448 for e4m3, absmax/127 for int8), round to
+ *     nearest even and saturation: the workload definitions this library is
+ *     measured on, since the pages only name "dynamic" per-token scaling.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *   - all-zero row/group/block: amax is clamped to at least 1e-12f before the
+ *     division, so the scale is tiny but finite and every code is +-0.
+ *   - the scale is the correctly rounded fp32 quotient amax/qmax; a value's
+ *     code is taken from the correctly rounded fp32 quotient x/s.
+ *   - e4m3 keeps the sign of zero (-0 -> 0x80); NaN -> 0x7F.
+ *   - int8 is symmetric: codes are clamped to [-127, 127].
+ *
+ * Parity pins for every function here live in tests/test_oracle_*.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_E4M3_MAX 448.0
+#define ORC_INT8_MAX 127.0
+#define ORC_AMAX_FLOOR 1e-12f
+
+enum { ORC_E4M3 = 0, ORC_INT8 = 1 };
+
+/* ------------------------------------------------------------------ */
+/* bf16 input                                                          */
+/* ------------------------------------------------------------------ */
+
+/* A bf16 value is the upper half of an IEEE binary32. */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* OCP FP8 E4M3 ("fn" variant): 1 sign bit, 4 exponent bits with bias 7,  */
+/* 3 mantissa bits, no infinities, NaN = S.1111.111, max finite 448.   */
+/* ------------------------------------------------------------------ */
+
+/* Value of a code, straight from the bit fields. */
+double orc_e4m3_decode(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, 1 - 7); /* subnormal: 0.m * 2^(1-bias) */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/*
+ * Nearest e4m3 code to v.  Ties go to the code with an even mantissa (its
+ * lowest bit clear).  Magnitudes above 448 saturate to 448.  The sign of zero
+ * is kept.  The search runs over the ordered positive finite codes 0..0x7E,
+ * whose values increase with the code.
+ */
+uint8_t orc_e4m3_encode(double v)
+{
+    uint8_t sign, lo, hi, best;
+    double a, dlo, dhi;
+    if (isnan(v))
+        return 0x7F;
+    sign = signbit(v) ? 0x80 : 0x00;
+    a = fabs(v);
+    if (a >= ORC_E4M3_MAX)
+        return (uint8_t)(sign | 0x7E);
+    /* bisection for the last code whose value is <= a */
+    lo = 0;
+    hi = 0x7E;
+    while (hi - lo > 1) {
+        uint8_t mid = (uint8_t)((lo + hi) / 2);
+        if (orc_e4m3_decode(mid) <= a)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    if (orc_e4m3_decode(hi) <= a)
+        lo = hi;
+    hi = (uint8_t)(lo < 0x7E ? lo + 1 : lo);
+    dlo = a - orc_e4m3_decode(lo);
+    dhi = orc_e4m3_decode(hi) - a;
+    if (dlo < dhi)
+        best = lo;
+    else if (dhi < dlo)
+        best = hi;
+    else
+        best = (lo & 1) ? hi : lo; /* exact tie: even mantissa */
+    return (uint8_t)(sign | best);
+}
+
+/* Round half to even to an integer, then clamp to the symmetric int8 range. */
+int8_t orc_int8_encode(double v)
+{
+    double r = floor(v);
+    double frac = v - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))
+        r += 1.0;
+    if (r > ORC_INT8_MAX)
+        r = ORC_INT8_MAX;
+    if (r < -ORC_INT8_MAX)
+        r = -ORC_INT8_MAX;
+    return (int8_t)r;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dynamic quantization of one group of values that share one scale.  */
+/* ------------------------------------------------------------------ */
+
+/* Correctly rounded fp32 quotient a/b of two fp32 values: the fp64 quotient
+ * carries more than 2*24+2 bits, so rounding it to fp32 is exact rounding. */
+static float div_rn_f32(float a, float b)
+{
+    return (float)((double)a / (double)b);
+}
+
+/*
+ * Quantize `count` bf16 values read with stride pattern (rows of `len`
+ * contiguous values, `nrows` rows, row pitch `pitch`) to one scale.
+ * qtype ORC_E4M3 writes uint8 codes; ORC_INT8 writes int8 codes.
+ * Returns the scale.
+ */
+static float quant_group(const uint16_t *x, long nrows, long len, long pitch,
+                         int qtype, void *q, long qpitch)
+{
+    float amax = 0.0f, s;
+    double qmax = (qtype == ORC_E4M3) ? ORC_E4M3_MAX : ORC_INT8_MAX;
+    long r, k;
+    for (r = 0; r < nrows; r++)
+        for (k = 0; k < len; k++) {
+            float a = fabsf(bf16_to_float(x[r * pitch + k]));
+            if (a > amax)
+                amax = a;
+        }
+    if (amax < ORC_AMAX_FLOOR)
+        amax = ORC_AMAX_FLOOR;
+    s = div_rn_f32(amax, (float)qmax);
+    for (r = 0; r < nrows; r++)
+        for (k = 0; k < len; k++) {
+            float v = div_rn_f32(bf16_to_float(x[r * pitch + k]), s);
+            if (qtype == ORC_E4M3)
+                ((uint8_t *)q)[r * qpitch + k] = orc_e4m3_encode(v);
+            else
+                ((int8_t *)q)[r * qpitch + k] = orc_int8_encode(v);
+        }
+    return s;
+}
+
+/* Per-row (per-token activation, or per-output-channel weight) scaling:
+ * x [rows, K] bf16 -> q [rows, K], s [rows]. */
+void orc_quant_rows(const uint16_t *x, long rows, long K, int qtype, void *q,
+                    float *s)
+{
+    long r;
+    for (r = 0; r < rows; r++) {
+        void *qrow = (qtype == ORC_E4M3) ? (void *)((uint8_t *)q + r * K)
+                                         : (void *)((int8_t *)q + r * K);
+        s[r] = quant_group(x + r * K, 1, K, K, qtype, qrow, K);
+    }
+}
+
+/* 1 x G activation groups: x [M, K] -> e4m3 q [M, K], s [M, K/G]. */
+void orc_quant_groups(const uint16_t *x, long M, long K, long G, uint8_t *q,
+                      float *s)
+{
+    long m, g, ng = K / G;
+    for (m = 0; m < M; m++)
+        for (g = 0; g < ng; g++)
+            s[m * ng + g] = quant_group(x + m * K + g * G, 1, G, K, ORC_E4M3,
+                                        q + m * K + g * G, K);
+}
+
+/* B x B weight blocks: w [N, K] -> e4m3 q [N, K], s [N/B, K/B]. */
+void orc_quant_blocks(const uint16_t *w, long N, long K, long B, uint8_t *q,
+                      float *s)
+{
+    long nb, kb, nbs = N / B, kbs = K / B;
+    for (nb = 0; nb < nbs; nb++)
+        for (kb = 0; kb < kbs; kb++)
+            s[nb * kbs + kb] =
+                quant_group(w + nb * B * K + kb * B, B, B, K, ORC_E4M3,
+                            q + nb * B * K + kb * B, K);
+}
+
+/* ------------------------------------------------------------------ */
+/* GEMM in exact integer arithmetic                                    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Every e4m3 value is an integer multiple of 2^-9 (the smallest subnormal),
+ * and 448 * 2^9 = 229376 < 2^18, so code -> value * 2^9 is an exact integer
+ * and a product of two codes is an exact integer times 2^-18.  Sums over
+ * K <= 2^15 terms stay below 2^51, so int64 holds them exactly.
+ */
+static int64_t e4m3_as_int(uint8_t code)
+{
+    return (int64_t)ldexp(orc_e4m3_decode(code), 9);
+}
+
+static int64_t code_int(const void *q, long idx, int qtype)
+{
+    if (qtype == ORC_E4M3)
+        return e4m3_as_int(((const uint8_t *)q)[idx]);
+    return (int64_t)((const int8_t *)q)[idx];
+}
+
+/* Unit of the integer accumulator: 2^-18 for e4m3 x e4m3, 1 for int8. */
+static double acc_unit(int qtype)
+{
+    return qtype == ORC_E4M3 ? ldexp(1.0, -18) : 1.0;
+}
+
+/*
+ * Exact dot product of row a of A [*, K] with row b of B [*, K] over the
+ * index range [k0, k1).  `absacc` (nullable) receives sum |a_k b_k|.
+ */
+static int64_t dot_range(const void *A, long a, const void *B, long b, long K,
+                         long k0, long k1, int qtype, int64_t *absacc)
+{
+    int64_t acc = 0, aacc = 0;
+    long k;
+    for (k = k0; k < k1; k++) {
+        int64_t p = code_int(A, a * K + k, qtype) * code_int(B, b * K + k, qtype);
+        acc += p;
+        aacc += p < 0 ? -p : p;
+    }
+    if (absacc)
+        *absacc = aacc;
+    return acc;
+}
+
+/*
+ * Per-row scaled product (FP8_Dynamic and W8A8_INT8):
+ *   acc[m,n] = sum_k Xq[m,k] Wq[n,k]              (exact)
+ *   y[m,n]   = acc[m,n] * unit * sx[m] * sw[n]    (fp64)
+ *   bound[m,n] = sum_k |x^_k| |w^_k|              (fp64, dequantized)
+ * A and B are both K-major: Xq [M, K], Wq [N, K].  acc/bound nullable.
+ */
+void orc_gemm_rowscaled(const void *xq, const float *sx, const void *wq,
+                        const float *sw, long M, long N, long K, int qtype,
+                        double *y, double *bound, int64_t *acc)
+{
+    long n;
+    double unit = acc_unit(qtype);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < N; n++) {
+        long m;
+        for (m = 0; m < M; m++) {
+            int64_t aabs;
+            int64_t a = dot_range(xq, m, wq, n, K, 0, K, qtype, &aabs);
+            double scale = (double)sx[m] * (double)sw[n];
+            y[m * N + n] = (double)a * unit * scale;
+            if (bound)
+                bound[m * N + n] = (double)aabs * unit * scale;
+            if (acc)
+                acc[m * N + n] = a;
+        }
+    }
+}
+
+/*
+ * Block-scaled product (Block_FP8): one exact partial sum per G-wide K block,
+ * each weighted by its own activation-group scale and weight-block scale:
+ *   y[m,n] = sum_kb acc_kb[m,n] * 2^-18 * sx[m,kb] * sw[n/G, kb]
+ * sx [M, K/G], sw [N/G, K/G].  bound nullable.
+ */
+void orc_gemm_blockscaled(const uint8_t *xq, const float *sx,
+                          const uint8_t *wq, const float *sw, long M, long N,
+                          long K, long G, double *y, double *bound)
+{
+    long n, kbs = K / G;
+    double unit = acc_unit(ORC_E4M3);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < N; n++) {
+        long m, kb;
+        for (m = 0; m < M; m++) {
+            double s = 0.0, b = 0.0;
+            for (kb = 0; kb < kbs; kb++) {
+                int64_t aabs;
+                int64_t a = dot_range(xq, m, wq, n, K, kb * G, (kb + 1) * G,
+                                      ORC_E4M3, &aabs);
+                double scale =
+                    (double)sx[m * kbs + kb] * (double)sw[(n / G) * kbs + kb];
+                s += (double)a * unit * scale;
+                b += (double)aabs * unit * scale;
+            }
+            y[m * N + n] = s;
+            if (bound)
+                bound[m * N + n] = b;
+        }
+    }
+}
+
+/*
+ * Split-K partition of one exact dot product: K is cut into `splits`
+ * contiguous chunks of ceil(K/splits) elements (the last may be short or
+ * empty) and the chunk sums are added.  In exact arithmetic the result is
+ * the same for every split count; the tests pin that.
+ */
+int64_t orc_dot_split(const void *xq, long m, const void *wq, long n, long K,
+                      int qtype, long splits)
+{
+    long chunk = (K + splits - 1) / splits, s;
+    int64_t total = 0;
+    for (s = 0; s < splits; s++) {
+        long k0 = s * chunk, k1 = k0 + chunk;
+        if (k0 >= K)
+            break;
+        if (k1 > K)
+            k1 = K;
+        total += dot_range(xq, m, wq, n, K, k0, k1, qtype, NULL);
+    }
+    return total;
+}
+
+/* Number of OpenMP threads the GEMMs above run on (1 without OpenMP). */
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
