@@ -1,0 +1,189 @@
+/*
+ * qgd.h - C ABI of a B200 (sm_100a) library for the quantized linear layer
+ *
+ *     Y[M,N] = dequant(Xq)[M,K] . dequant(Wq)[N,K]^T      (Y in bf16)
+ *
+ * at decode-sized token counts M (1..32) and beyond, in the three formats of
+ * "Building a High-Performance and Portable vLLM Linear Backend with Helion"
+ * (section "Put algorithm selection inside the search space", and the scope
+ * list "Alcance" of its Spanish translation):
+ *
+ *   FP8_Dynamic  e4m3 activations with one scale per token (row of X) and
+ *                e4m3 weights with one scale per output channel (row of W);
+ *   W8A8_INT8    the same granularity with symmetric int8 codes;
+ *   Block_FP8    e4m3 with one activation scale per 1x128 group of a row and
+ *                one weight scale per 128x128 block.
+ *
+ * The GEMM comes in the article's algorithm variants (section "Como se
+ * implementa el kernel?" and its matmul listing): Standard (each CTA owns an
+ * output tile and reduces all of K), Split-K (K is cut into split_k parts,
+ * split_k a power of two from 1 to 256, whose partial sums are then added)
+ * and Swap-AB (the product is computed as (W . X^T)^T so the wide N dimension
+ * fills the MMA's M slot).  Which one runs for a shape is chosen from a
+ * measured dispatch table (section "Hybrid dispatch" / "Despacho hibrido":
+ * the token counts 1, 2, 4, 8, 16, 24 and 32 are tuned separately).
+ *
+ * Conventions for every call below
+ *   - All matrices are row-major with K contiguous ("K-major"): X/Xq [M,K],
+ *     W/Wq [N,K], Y [M,N].  bf16 is passed as its 16-bit storage.
+ *   - Data pointers are DEVICE pointers owned by the caller and must be
+ *     16-byte aligned.  The library never allocates device memory, never
+ *     frees caller memory and never synchronizes the stream.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; calls can be captured into a CUDA graph
+ *     (nothing inside a call allocates or synchronizes).
+ *   - Errors are returned as a qgd_status and nothing is launched when the
+ *     arguments are rejected.  qgd_last_error_message() describes the last
+ *     failure on the calling thread.  A device-side wait that gives up (about
+ *     one second without progress) is reported through qgd_device_error().
+ *   - M == 0 is a valid empty call: it returns QGD_OK and launches nothing.
+ */
+#ifndef QGD_H
+#define QGD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QGD_API __attribute__((visibility("default")))
+#else
+#define QGD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QGD_OK = 0,
+  QGD_ERR_INVALID = -1,     /* null or misaligned pointer, negative size, bad enum */
+  QGD_ERR_UNSUPPORTED = -2, /* shape outside the supported set (see each call) */
+  QGD_ERR_WORKSPACE = -3,   /* workspace missing or smaller than qgd_workspace_size() */
+  QGD_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed */
+  QGD_ERR_TABLE = -5,       /* dispatch table file unreadable or malformed */
+  QGD_ERR_DEVICE = -6       /* current device is not an sm_100 part */
+} qgd_status;
+
+typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8 = 2 } qgd_format;
+typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
+typedef enum { QGD_VARIANT_AUTO = -1, QGD_VARIANT_STANDARD = 0, QGD_VARIANT_SWAP_AB = 1 } qgd_variant;
+typedef enum {
+  QGD_REDUCE_AUTO = -1,
+  QGD_REDUCE_LAST_CTA = 0, /* split partials to workspace; the last CTA of each tile adds them in split order */
+  QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order */
+  QGD_REDUCE_ATOMIC = 2    /* split partials added atomically into a zeroed workspace (fp32 order varies) */
+} qgd_reduce;
+
+/* The execution plan for one (format, M, N, K). */
+typedef struct {
+  int variant; /* qgd_variant (never AUTO here) */
+  int split_k; /* CTAs along K: power of two, 1..256, at most ceil(K/128) */
+  int reduce;  /* qgd_reduce, meaningful when split_k > 1 */
+  int stages;  /* depth of the shared-memory operand ring */
+  int tile_n;  /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */
+  int source;  /* 0 = built-in default, 1 = dispatch table, 2 = override */
+} qgd_plan;
+
+/* ---------------------------------------------------------------------
+ * Dynamic quantizers ("Fused Quantization Ops"; per-token / per-group
+ * scaling of the three formats).  For each row (or 1x128 group, or 128x128
+ * block) g:
+ *     amax = max(max |x| over g, 1e-12f)
+ *     s    = amax / qmax            (qmax = 448 for e4m3, 127 for int8;
+ *                                    correctly rounded fp32 division)
+ *     q    = convert(x / s)         (correctly rounded fp32 quotient, then
+ *                                    round-to-nearest-even; e4m3 saturates to
+ *                                    +-448 and keeps the sign of zero; int8 is
+ *                                    clamped to [-127, 127])
+ * ------------------------------------------------------------------- */
+
+/* Per-row scales.  x_bf16 [M,K] -> xq [M,K] (e4m3 bytes or int8), sx [M]
+ * fp32.  Also the weight quantizer for FP8_Dynamic / W8A8_INT8 (rows = N).
+ * Requires K % 8 == 0 and K <= 65536. */
+QGD_API qgd_status quant_act_per_token(const void* x_bf16, int M, int K, int qtype, void* xq, float* sx, void* stream);
+
+/* 1x128 activation groups (Block_FP8).  x_bf16 [M,K] -> xq e4m3 [M,K],
+ * sx [M][K/128] fp32 row-major.  Requires K % 128 == 0. */
+QGD_API qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float* sx, void* stream);
+
+/* 128x128 weight blocks (Block_FP8).  w_bf16 [N,K] -> wq e4m3 [N,K],
+ * sw [N/128][K/128] fp32 row-major.  Requires N % 128 == 0, K % 128 == 0. */
+QGD_API qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Quantized GEMMs.  y_bf16 [M,N] = round_bf16( sum_k xq*wq * scales ):
+ *   FP8_Dynamic / W8A8_INT8: acc[m,n] = sum_k Xq[m,k] Wq[n,k] (fp32 / exact
+ *     int32 accumulation); Y = (acc * sx[m]) * sw[n].
+ *   Block_FP8: for each 128-wide K block kb, P_kb = sum over the block;
+ *     Y = sum_kb P_kb * (sx[m][kb] * sw[n/128][kb]).
+ * Shapes: M >= 0; N % 16 == 0; K % 16 == 0 (FP8_Dynamic, W8A8_INT8) or
+ * K % 128 == 0 and N % 128 == 0 (Block_FP8).
+ * Workspace: `ws` (device, >= qgd_workspace_size() bytes for the same
+ * arguments) holds Split-K partials and per-tile arrival counters.  It must be
+ * zero-filled once after allocation; every call leaves its counters and
+ * atomic accumulators zero again.  Calls that share a workspace must not run
+ * concurrently.  ws may be NULL when qgd_workspace_size() returns 0.
+ * ------------------------------------------------------------------- */
+QGD_API qgd_status qlinear_fp8_dynamic(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                               int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
+QGD_API qgd_status qlinear_w8a8_int8(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                             int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
+QGD_API qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                             int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
+
+/* Test hook: the W8A8_INT8 mainloop and Split-K reduction of the plan in
+ * force, writing the exact int32 accumulator acc[M][N] instead of Y. */
+QGD_API qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Bytes of workspace the plan for (fmt, M, N, K) needs (0 when it needs
+ * none).  Re-query after changing the override or the dispatch table. */
+QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
+
+/* ---------------------------------------------------------------------
+ * Dispatch (host only; no GPU needed).
+ * ------------------------------------------------------------------- */
+
+/* Load a dispatch table (text; see the file format in the package's
+ * tables/ directory): one line per (format, N, K, M-bucket) with the
+ * variant, split_k, reduction, stages and tile_n measured best.  Replaces
+ * the table in force.  On QGD_ERR_TABLE the table in force is unchanged.
+ * Not thread-safe against concurrent qlinear_* calls. */
+QGD_API qgd_status qgd_load_dispatch_table(const char* path);
+
+/* Drop the table in force; the built-in defaults apply again. */
+QGD_API qgd_status qgd_clear_dispatch_table(void);
+
+/* Force a plan for one format (tests and the tuner).  Any argument < 0 keeps
+ * the table/default choice for that field; stages/tile_n 0 = default.
+ * qgd_set_override(fmt, -1, -1, -1, 0, 0) removes the override. */
+QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n);
+
+/* The plan a qlinear_* call with these arguments would run. */
+QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);
+
+/* M-bucket of a token count: the smallest tuned count >= M among
+ * 1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192 (the last one beyond). */
+QGD_API int qgd_m_bucket(int M);
+
+/* ---------------------------------------------------------------------
+ * Status
+ * ------------------------------------------------------------------- */
+QGD_API const char* qgd_status_string(int status);
+QGD_API const char* qgd_last_error_message(void);
+
+/* Device error flag of the current device (0 = none).  Nonzero means a
+ * kernel gave up a bounded wait and returned without finishing; its outputs
+ * are undefined and the workspace must be zero-filled again.  Synchronizes
+ * the device.  qgd_clear_device_error() resets the flag. */
+QGD_API qgd_status qgd_device_error(unsigned int* code);
+QGD_API qgd_status qgd_clear_device_error(void);
+
+/* Library version, "major.minor.patch". */
+QGD_API const char* qgd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGD_H */

@@ -1,0 +1,314 @@
+"""Python binding of libqgd.so, the B200 (sm_100a) quantized linear-layer library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI (include/qgd.h).  PyTorch supplies device memory and
+streams.  The functions keep the C names:
+
+    quant_act_per_token, quant_act_group128, quant_weight_block128,
+    qlinear_fp8_dynamic, qlinear_w8a8_int8, qlinear_block_fp8,
+    qgd_w8a8_int8_acc32, qgd_workspace_size, qgd_load_dispatch_table,
+    qgd_clear_dispatch_table, qgd_set_override, qgd_get_plan, qgd_m_bucket,
+    qgd_device_error, qgd_clear_device_error
+
+There is no fallback: if libqgd.so is missing or cannot be loaded, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "QGDError", "lib", "FMT_FP8_DYNAMIC", "FMT_W8A8_INT8", "FMT_BLOCK_FP8", "QTYPE_E4M3", "QTYPE_INT8",
+    "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC",
+    "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
+    "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
+    "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
+    "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
+    "Workspace", "DEFAULT_TABLE",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqgd.so")
+DEFAULT_TABLE = os.path.join(_PKG, "tables", "b200.tsv")
+
+FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8 = 0, 1, 2
+QTYPE_E4M3, QTYPE_INT8 = 0, 1
+VARIANT_STANDARD, VARIANT_SWAP_AB = 0, 1
+REDUCE_LAST_CTA, REDUCE_TWO_PASS, REDUCE_ATOMIC = 0, 1, 2
+FORMAT_NAMES = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class QGDError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {message} (status {status})")
+        self.status = status
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
+                ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("source", ctypes.c_int)]
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqgd.so (built in-tree by quantized_gemm_decode_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise QGDError(-4, "load", f"{LIB_PATH} is missing; run `python -m quantized_gemm_decode_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "quant_act_per_token": [P, I, I, I, P, P, P],
+            "quant_act_group128": [P, I, I, P, P, P],
+            "quant_weight_block128": [P, I, I, P, P, P],
+            "qlinear_fp8_dynamic": [P, P, P, P, P, I, I, I, P, S, P],
+            "qlinear_w8a8_int8": [P, P, P, P, P, I, I, I, P, S, P],
+            "qlinear_block_fp8": [P, P, P, P, P, I, I, I, P, S, P],
+            "qgd_w8a8_int8_acc32": [P, P, P, I, I, I, P, S, P],
+            "qgd_load_dispatch_table": [ctypes.c_char_p],
+            "qgd_clear_dispatch_table": [],
+            "qgd_set_override": [I, I, I, I, I, I],
+            "qgd_get_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
+            "qgd_device_error": [ctypes.POINTER(ctypes.c_uint)],
+            "qgd_clear_device_error": [],
+        }
+        for name, args in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.qgd_workspace_size.argtypes = [I, I, I, I]
+        L.qgd_workspace_size.restype = S
+        L.qgd_m_bucket.argtypes = [I]
+        L.qgd_m_bucket.restype = I
+        L.qgd_status_string.argtypes = [I]
+        L.qgd_status_string.restype = ctypes.c_char_p
+        L.qgd_last_error_message.argtypes = []
+        L.qgd_last_error_message.restype = ctypes.c_char_p
+        L.qgd_version.argtypes = []
+        L.qgd_version.restype = ctypes.c_char_p
+        _lib = L
+        if os.path.exists(DEFAULT_TABLE) and not os.environ.get("QGD_NO_TABLE"):
+            _check(L.qgd_load_dispatch_table(os.environ.get("QGD_TABLE", DEFAULT_TABLE).encode()),
+                   "qgd_load_dispatch_table")
+        return L
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        L = _lib
+        msg = L.qgd_last_error_message().decode() if L is not None else ""
+        raise QGDError(status, where, msg or (L.qgd_status_string(status).decode() if L else "error"))
+
+
+def _ptr(t) -> ctypes.c_void_p | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda_2d(t: torch.Tensor, name: str, dtypes) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D tensor")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+
+
+_BYTE_TYPES = (torch.uint8, torch.int8, torch.float8_e4m3fn)
+
+
+# ---------------------------------------------------------------------------
+# Quantizers
+# ---------------------------------------------------------------------------
+def quant_act_per_token(x: torch.Tensor, qtype: int = QTYPE_E4M3, xq=None, sx=None, stream=None):
+    """Per-row dynamic quantization: x bf16 [M, K] -> (xq [M, K], sx fp32 [M])."""
+    _cuda_2d(x, "x", (torch.bfloat16,))
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.float8_e4m3fn if qtype == QTYPE_E4M3 else torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().quant_act_per_token(_ptr(x), M, K, qtype, _ptr(xq), _ptr(sx), _stream(stream)),
+           "quant_act_per_token")
+    return xq, sx
+
+
+def quant_weight_per_channel(w: torch.Tensor, qtype: int = QTYPE_E4M3, stream=None):
+    """Per-output-channel weight quantization (the per-row quantizer over N rows)."""
+    return quant_act_per_token(w, qtype, stream=stream)
+
+
+def quant_act_group128(x: torch.Tensor, xq=None, sx=None, stream=None):
+    """1x128 group quantization: x bf16 [M, K] -> (xq e4m3 [M, K], sx fp32 [M, K/128])."""
+    _cuda_2d(x, "x", (torch.bfloat16,))
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if sx is None:
+        sx = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check(lib().quant_act_group128(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "quant_act_group128")
+    return xq, sx
+
+
+def quant_weight_block128(w: torch.Tensor, wq=None, sw=None, stream=None):
+    """128x128 block quantization: w bf16 [N, K] -> (wq e4m3 [N, K], sw fp32 [N/128, K/128])."""
+    _cuda_2d(w, "w", (torch.bfloat16,))
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    if sw is None:
+        sw = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device)
+    _check(lib().quant_weight_block128(_ptr(w), N, K, _ptr(wq), _ptr(sw), _stream(stream)), "quant_weight_block128")
+    return wq, sw
+
+
+# ---------------------------------------------------------------------------
+# Workspace
+# ---------------------------------------------------------------------------
+class Workspace:
+    """A zero-filled device buffer for Split-K partials and tile counters.
+
+    The kernels leave its counters zero after every call, so it is zeroed only
+    when it is (re)allocated.  Not to be shared by calls running concurrently.
+    """
+
+    def __init__(self, nbytes: int = 0, device=None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+    def ensure(self, nbytes: int) -> "Workspace":
+        if nbytes > self.nbytes:
+            self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
+        return self
+
+
+_default_ws: dict = {}
+
+
+def _workspace(fmt: int, M: int, N: int, K: int, ws, device):
+    need = qgd_workspace_size(fmt, M, N, K)
+    if ws is None:
+        key = (device.index if device.index is not None else torch.cuda.current_device())
+        ws = _default_ws.get(key)
+        if ws is None:
+            ws = _default_ws[key] = Workspace(need, device)
+    if isinstance(ws, Workspace):
+        ws.ensure(need)
+        return ws.buf.data_ptr(), ws.nbytes
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+# ---------------------------------------------------------------------------
+# GEMMs
+# ---------------------------------------------------------------------------
+def _qlinear(fn_name: str, fmt: int, xq, sx, wq, sw, y, ws, stream):
+    _cuda_2d(xq, "xq", _BYTE_TYPES)
+    _cuda_2d(wq, "wq", _BYTE_TYPES)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"K mismatch: xq {tuple(xq.shape)} vs wq {tuple(wq.shape)}")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    wsp, wsn = _workspace(fmt, M, N, K, ws, xq.device)
+    fn = getattr(lib(), fn_name)
+    _check(fn(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K, ctypes.c_void_p(wsp), wsn, _stream(stream)),
+           fn_name)
+    return y
+
+
+def qlinear_fp8_dynamic(xq, sx, wq, sw, y=None, ws=None, stream=None):
+    """Y bf16 [M, N] = (Xq . Wq^T) * sx[m] * sw[n], e4m3 operands."""
+    return _qlinear("qlinear_fp8_dynamic", FMT_FP8_DYNAMIC, xq, sx, wq, sw, y, ws, stream)
+
+
+def qlinear_w8a8_int8(xq, sx, wq, sw, y=None, ws=None, stream=None):
+    """Y bf16 [M, N] = (Xq . Wq^T) * sx[m] * sw[n], int8 operands, int32 accumulation."""
+    return _qlinear("qlinear_w8a8_int8", FMT_W8A8_INT8, xq, sx, wq, sw, y, ws, stream)
+
+
+def qlinear_block_fp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
+    """Y bf16 [M, N] with 1x128 activation and 128x128 weight block scales."""
+    return _qlinear("qlinear_block_fp8", FMT_BLOCK_FP8, xq, sx, wq, sw, y, ws, stream)
+
+
+def qgd_w8a8_int8_acc32(xq, wq, acc=None, ws=None, stream=None):
+    """Exact int32 accumulator [M, N] of the W8A8_INT8 mainloop (test hook)."""
+    _cuda_2d(xq, "xq", (torch.int8,))
+    _cuda_2d(wq, "wq", (torch.int8,))
+    M, K = xq.shape
+    N = wq.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    wsp, wsn = _workspace(FMT_W8A8_INT8, M, N, K, ws, xq.device)
+    _check(lib().qgd_w8a8_int8_acc32(_ptr(xq), _ptr(wq), _ptr(acc), M, N, K, ctypes.c_void_p(wsp), wsn,
+                                     _stream(stream)), "qgd_w8a8_int8_acc32")
+    return acc
+
+
+# ---------------------------------------------------------------------------
+# Dispatch and status (host only)
+# ---------------------------------------------------------------------------
+def qgd_workspace_size(fmt: int, M: int, N: int, K: int) -> int:
+    return int(lib().qgd_workspace_size(fmt, M, N, K))
+
+
+def qgd_load_dispatch_table(path: str) -> None:
+    _check(lib().qgd_load_dispatch_table(str(path).encode()), "qgd_load_dispatch_table")
+
+
+def qgd_clear_dispatch_table() -> None:
+    _check(lib().qgd_clear_dispatch_table(), "qgd_clear_dispatch_table")
+
+
+def qgd_set_override(fmt: int, variant: int = -1, split_k: int = -1, reduce: int = -1, stages: int = 0,
+                     tile_n: int = 0) -> None:
+    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n), "qgd_set_override")
+
+
+def qgd_get_plan(fmt: int, M: int, N: int, K: int) -> dict:
+    p = _Plan()
+    _check(lib().qgd_get_plan(fmt, M, N, K, ctypes.byref(p)), "qgd_get_plan")
+    return {f: getattr(p, f) for f, _ in _Plan._fields_}
+
+
+def qgd_m_bucket(M: int) -> int:
+    return int(lib().qgd_m_bucket(M))
+
+
+def qgd_device_error() -> int:
+    code = ctypes.c_uint(0)
+    _check(lib().qgd_device_error(ctypes.byref(code)), "qgd_device_error")
+    return int(code.value)
+
+
+def qgd_clear_device_error() -> None:
+    _check(lib().qgd_clear_device_error(), "qgd_clear_device_error")
+
+
+def qgd_version() -> str:
+    return lib().qgd_version().decode()

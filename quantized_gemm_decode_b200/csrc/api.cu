@@ -1,0 +1,468 @@
+// C ABI of the library (declared in include/qgd.h): argument checking, plan
+// selection from the dispatch table, workspace layout, TMA descriptor
+// encoding, and kernel launch on the caller's stream.
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <cstring>
+#include <fstream>
+#include <map>
+#include <mutex>
+#include <sstream>
+#include <string>
+#include <tuple>
+
+#include "../../include/qgd.h"
+#include "qgd_internal.h"
+
+using namespace qgd;
+
+namespace {
+
+thread_local std::string g_err;
+
+qgd_status fail(qgd_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  if (getenv("QGD_LOG")) fprintf(stderr, "[qgd] %s\n", buf);
+  return st;
+}
+
+qgd_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(QGD_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// Device checks (per device, cached)
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+int g_dev_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+int g_num_sms = 148;         // used by the default plan; refreshed from the device
+
+qgd_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(QGD_ERR_DEVICE, "device index %d out of range", dev);
+  if (g_dev_ok[dev] == 0) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms > 0) g_num_sms = sms;
+    g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (g_dev_ok[dev] < 0) return fail(QGD_ERR_DEVICE, "device %d is not an sm_100 GPU; this library is built for sm_100a only", dev);
+  return QGD_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors.  cuTensorMapEncodeTiled is a host-only driver function;
+// it is looked up once through the runtime.
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+qgd_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(QGD_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  return QGD_OK;
+}
+
+// 2-D byte matrix [rows, cols] (cols contiguous), box = box_rows x 128 bytes,
+// 128-byte swizzle; out-of-range rows/columns read as zero.
+qgd_status encode_kmajor(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QGD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%d cols=%d box_rows=%d", (int)r, rows, cols, box_rows);
+  return QGD_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch: table (format, N, K, M-bucket) -> plan; override per format.
+// ---------------------------------------------------------------------------
+const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
+constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
+constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
+
+struct Entry {
+  int variant, split_k, reduce, stages, tile_n;
+};
+using Key = std::tuple<int, int, int, int>;
+std::mutex g_mu;
+std::map<Key, Entry> g_table;
+struct Override {
+  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0;
+} g_override[3];
+
+int bucket_of(int M) {
+  for (int i = 0; i < kNumBuckets; ++i)
+    if (M <= kBuckets[i]) return kBuckets[i];
+  return kBuckets[kNumBuckets - 1];
+}
+
+int floor_pow2(int v) {
+  int p = 1;
+  while (p * 2 <= v) p *= 2;
+  return p;
+}
+
+int fmt_from_name(const std::string& s) {
+  if (s == "fp8_dynamic" || s == "fp8") return kFmtFP8;
+  if (s == "w8a8_int8" || s == "int8") return kFmtINT8;
+  if (s == "block_fp8" || s == "block") return kFmtBlock;
+  return -1;
+}
+
+int variant_from_name(const std::string& s) {
+  if (s == "standard") return kStandard;
+  if (s == "swap_ab" || s == "swapab") return kSwapAB;
+  return -1;
+}
+
+int reduce_from_name(const std::string& s) {
+  if (s == "last_cta") return kLastCta;
+  if (s == "two_pass") return kTwoPass;
+  if (s == "atomic") return kAtomic;
+  return -1;
+}
+
+qgd_plan make_plan(int fmt, int M, int N, int K) {
+  const int nkt = (K + kTileK - 1) / kTileK;
+  qgd_plan p;
+  p.source = 0;
+  p.reduce = kLastCta;
+  p.stages = 0;
+  if (M <= kDecodeMaxM) {
+    // Swap-AB by default for small M (the hand-written rule the method
+    // replaces with measurement), split until the grid covers the SMs.
+    p.variant = kSwapAB;
+    p.tile_n = kSwapTileN;
+    const int tiles = (N + kSwapTileN - 1) / kSwapTileN;
+    int s = 1;
+    while (tiles * s < g_num_sms && s * 2 <= nkt && s < 256) s *= 2;
+    p.split_k = s;
+  } else {
+    p.variant = kStandard;
+    p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+    p.split_k = 1;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_table.find(Key(fmt, N, K, bucket_of(M)));
+    if (it != g_table.end()) {
+      const Entry& e = it->second;
+      p.variant = e.variant;
+      p.split_k = e.split_k;
+      p.reduce = e.reduce;
+      p.stages = e.stages;
+      p.tile_n = e.tile_n;
+      p.source = 1;
+    }
+    const Override& o = g_override[fmt];
+    if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0) {
+      if (o.variant >= 0) p.variant = o.variant;
+      if (o.split_k >= 0) p.split_k = o.split_k;
+      if (o.reduce >= 0) p.reduce = o.reduce;
+      if (o.stages > 0) p.stages = o.stages;
+      if (o.tile_n > 0) p.tile_n = o.tile_n;
+      p.source = 2;
+    }
+  }
+  // Make the plan legal for this shape.
+  if (p.variant == kSwapAB && M > kDecodeMaxM) p.variant = kStandard;
+  if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
+  else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+  int smax = nkt < 256 ? nkt : 256;
+  if (smax < 1) smax = 1;
+  if (p.split_k < 1) p.split_k = 1;
+  if (p.split_k > smax) p.split_k = smax;
+  p.split_k = floor_pow2(p.split_k);
+  if (p.reduce < kLastCta || p.reduce > kAtomic) p.reduce = kLastCta;
+  const int mpad = M <= 16 ? 16 : 32;
+  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad) : standard_max_stages(p.tile_n);
+  if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
+  if (p.stages < 2) p.stages = 2;
+  return p;
+}
+
+struct WsLayout {
+  size_t tickets_off, tickets_bytes, data_off, data_bytes, total;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(const qgd_plan& p, int M, int N) {
+  WsLayout w{0, 0, 0, 0, 0};
+  if (p.split_k <= 1 || M == 0) return w;
+  size_t tiles;
+  if (p.variant == kSwapAB)
+    tiles = (N + kSwapTileN - 1) / kSwapTileN;
+  else
+    tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
+  if (p.reduce != kTwoPass) w.tickets_bytes = align256(tiles * 4);
+  w.data_off = w.tickets_bytes;
+  w.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
+  w.total = w.data_off + w.data_bytes;
+  return w;
+}
+
+qgd_status check_shape(int fmt, int M, int N, int K) {
+  if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d N=%d K=%d)", M, N, K);
+  if (N % 16 != 0) return fail(QGD_ERR_UNSUPPORTED, "N=%d must be a multiple of 16", N);
+  if (K % 16 != 0) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 16", K);
+  if (fmt == kFmtBlock && (K % 128 != 0 || N % 128 != 0))
+    return fail(QGD_ERR_UNSUPPORTED, "Block_FP8 needs N and K multiples of 128 (N=%d K=%d)", N, K);
+  if (static_cast<long long>(M) * N > (1LL << 31)) return fail(QGD_ERR_UNSUPPORTED, "M*N too large");
+  return QGD_OK;
+}
+
+qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, const float* sw, void* y, void* raw,
+                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  qgd_status st = check_shape(fmt, M, N, K);
+  if (st != QGD_OK) return st;
+  if (M == 0) return QGD_OK;
+  if (!xq || !wq || (!y && !raw)) return fail(QGD_ERR_INVALID, "null operand pointer");
+  if (!raw && (!sx || !sw)) return fail(QGD_ERR_INVALID, "null scale pointer");
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(raw) || !aligned16(sx) || !aligned16(sw))
+    return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
+  if ((st = check_device()) != QGD_OK) return st;
+  if ((st = get_encoder()) != QGD_OK) return st;
+
+  const qgd_plan p = make_plan(fmt, M, N, K);
+  const WsLayout wl = ws_layout(p, M, N);
+  if (wl.total > 0 && (!ws || ws_bytes < wl.total))
+    return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", wl.total, ws ? ws_bytes : 0);
+  if (wl.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
+
+  GemmArgs a;
+  a.sx = sx;
+  a.sw = sw;
+  a.y = static_cast<uint16_t*>(y);
+  a.raw = raw;
+  a.partial = nullptr;
+  a.accum = nullptr;
+  a.tickets = nullptr;
+  if (wl.total > 0) {
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    if (wl.tickets_bytes) a.tickets = reinterpret_cast<unsigned int*>(wsb + wl.tickets_off);
+    if (p.reduce == kAtomic) a.accum = wsb + wl.data_off;
+    else a.partial = wsb + wl.data_off;
+  }
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.splits = p.split_k;
+  a.reduce = p.reduce;
+  a.stages = p.stages;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tw, tx;
+  cudaError_t e;
+  if (p.variant == kSwapAB) {
+    const int mpad = M <= 16 ? 16 : 32;
+    if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;
+    if ((st = encode_kmajor(&tx, xq, M, K, mpad)) != QGD_OK) return st;
+    e = launch_swapab(fmt, mpad, tw, tx, a, s);
+  } else {
+    if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
+    if ((st = encode_kmajor(&tw, wq, N, K, p.tile_n)) != QGD_OK) return st;
+    e = launch_standard(fmt, p.tile_n, tx, tw, a, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+  if (p.split_k > 1 && p.reduce == kTwoPass) {
+    e = launch_splitk_reduce(fmt, a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "Split-K reduce launch");
+  }
+  return QGD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qgd_status quant_act_per_token(const void* x_bf16, int M, int K, int qtype, void* xq, float* sx, void* stream) {
+  if (M < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d K=%d)", M, K);
+  if (qtype != QGD_QTYPE_E4M3 && qtype != QGD_QTYPE_INT8) return fail(QGD_ERR_INVALID, "bad qtype %d", qtype);
+  if (K % 8 != 0 || K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 8 and <= 65536", K);
+  if (M == 0) return QGD_OK;
+  if (!x_bf16 || !xq || !sx) return fail(QGD_ERR_INVALID, "null pointer");
+  if (!aligned16(x_bf16) || !aligned16(xq) || (reinterpret_cast<uintptr_t>(sx) & 3u))
+    return fail(QGD_ERR_INVALID, "x and xq must be 16-byte aligned, sx 4-byte aligned");
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  cudaError_t e = launch_quant_rows(static_cast<const uint16_t*>(x_bf16), M, K, qtype, xq, sx,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_per_token launch");
+}
+
+qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float* sx, void* stream) {
+  if (M < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d K=%d)", M, K);
+  if (K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 128", K);
+  if (M == 0) return QGD_OK;
+  if (!x_bf16 || !xq || !sx) return fail(QGD_ERR_INVALID, "null pointer");
+  if (!aligned16(x_bf16) || !aligned16(xq) || (reinterpret_cast<uintptr_t>(sx) & 3u))
+    return fail(QGD_ERR_INVALID, "x and xq must be 16-byte aligned, sx 4-byte aligned");
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  cudaError_t e = launch_quant_group128(static_cast<const uint16_t*>(x_bf16), M, K, static_cast<uint8_t*>(xq), sx,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_group128 launch");
+}
+
+qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream) {
+  if (N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (N=%d K=%d)", N, K);
+  if (N % 128 != 0 || K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "N=%d and K=%d must be multiples of 128", N, K);
+  if (!w_bf16 || !wq || !sw) return fail(QGD_ERR_INVALID, "null pointer");
+  if (!aligned16(w_bf16) || !aligned16(wq) || (reinterpret_cast<uintptr_t>(sw) & 3u))
+    return fail(QGD_ERR_INVALID, "w and wq must be 16-byte aligned, sw 4-byte aligned");
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  cudaError_t e = launch_quant_block128(static_cast<const uint16_t*>(w_bf16), N, K, static_cast<uint8_t*>(wq), sw,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_weight_block128 launch");
+}
+
+qgd_status qlinear_fp8_dynamic(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                               int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_gemm(kFmtFP8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qlinear_w8a8_int8(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                             int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_gemm(kFmtINT8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
+                             int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_gemm(kFmtBlock, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (M > 0 && !acc) return fail(QGD_ERR_INVALID, "null accumulator pointer");
+  return run_gemm(kFmtINT8, xq, nullptr, wq, nullptr, nullptr, acc, M, N, K, ws, ws_bytes, stream);
+}
+
+size_t qgd_workspace_size(int fmt, int M, int N, int K) {
+  if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
+  return ws_layout(make_plan(fmt, M, N, K), M, N).total;
+}
+
+qgd_status qgd_load_dispatch_table(const char* path) {
+  if (!path) return fail(QGD_ERR_INVALID, "null path");
+  std::ifstream in(path);
+  if (!in) return fail(QGD_ERR_TABLE, "cannot open dispatch table %s", path);
+  std::map<Key, Entry> t;
+  std::string line;
+  int lineno = 0;
+  while (std::getline(in, line)) {
+    ++lineno;
+    const size_t hash = line.find('#');
+    if (hash != std::string::npos) line.resize(hash);
+    std::istringstream ls(line);
+    std::string fmt_s, var_s, red_s;
+    int N, K, Mb, split, stages, tile_n;
+    if (!(ls >> fmt_s)) continue;  // blank line
+    if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n))
+      return fail(QGD_ERR_TABLE, "%s:%d: expected 9 fields: fmt N K M_bucket variant split_k reduce stages tile_n",
+                  path, lineno);
+    std::string extra;
+    if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
+    const int fmt = fmt_from_name(fmt_s), var = variant_from_name(var_s), red = reduce_from_name(red_s);
+    if (fmt < 0 || var < 0 || red < 0)
+      return fail(QGD_ERR_TABLE, "%s:%d: unknown format/variant/reduce name", path, lineno);
+    if (N <= 0 || K <= 0 || bucket_of(Mb) != Mb)
+      return fail(QGD_ERR_TABLE, "%s:%d: bad N/K or M bucket %d", path, lineno, Mb);
+    if (split < 1 || split > 256 || (split & (split - 1)) != 0)
+      return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256", path, lineno, split);
+    if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+      return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n", path, lineno);
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n};
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_table.swap(t);
+  return QGD_OK;
+}
+
+qgd_status qgd_clear_dispatch_table(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_table.clear();
+  return QGD_OK;
+}
+
+qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n) {
+  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 ||
+      (tile_n != 0 && tile_n != 128 && tile_n != 256))
+    return fail(QGD_ERR_INVALID, "bad override");
+  if (split_k > 0 && (split_k & (split_k - 1)) != 0) return fail(QGD_ERR_INVALID, "split_k must be a power of two");
+  std::lock_guard<std::mutex> lk(g_mu);
+  Override& o = g_override[fmt];
+  o.variant = variant < 0 ? -1 : variant;
+  o.split_k = split_k <= 0 ? -1 : split_k;
+  o.reduce = reduce < 0 ? -1 : reduce;
+  o.stages = stages;
+  o.tile_n = tile_n;
+  return QGD_OK;
+}
+
+qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan) {
+  if (!plan) return fail(QGD_ERR_INVALID, "null plan");
+  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "bad sizes");
+  *plan = make_plan(fmt, M < 1 ? 1 : M, N, K);
+  return QGD_OK;
+}
+
+int qgd_m_bucket(int M) { return bucket_of(M < 1 ? 1 : M); }
+
+const char* qgd_status_string(int status) {
+  switch (status) {
+    case QGD_OK: return "ok";
+    case QGD_ERR_INVALID: return "invalid argument";
+    case QGD_ERR_UNSUPPORTED: return "unsupported shape";
+    case QGD_ERR_WORKSPACE: return "workspace too small";
+    case QGD_ERR_CUDA: return "CUDA error";
+    case QGD_ERR_TABLE: return "dispatch table error";
+    case QGD_ERR_DEVICE: return "unsupported device";
+  }
+  return "unknown status";
+}
+
+const char* qgd_last_error_message(void) { return g_err.c_str(); }
+
+qgd_status qgd_device_error(unsigned int* code) {
+  if (!code) return fail(QGD_ERR_INVALID, "null code");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = read_device_error(code);
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "read device error flag");
+}
+
+qgd_status qgd_clear_device_error(void) {
+  cudaError_t e = clear_device_error();
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "clear device error flag");
+}
+
+const char* qgd_version(void) { return "0.1.0"; }
+
+}  // extern "C"

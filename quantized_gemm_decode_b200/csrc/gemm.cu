@@ -1,0 +1,818 @@
+// Quantized GEMM kernels for sm_100a: TMA-fed shared-memory ring ->
+// tcgen05.mma (kind::f8f6f4 for e4m3, kind::i8 for int8) -> TMEM accumulator
+// -> scale epilogue.  Two orientations:
+//
+//   Swap-AB   D^T[n, m] = sum_k Wq[n,k] Xq[m,k]: a CTA owns 128 weight rows
+//             (the MMA's M) and all M <= 32 tokens (the MMA's N, padded to 16
+//             or 32).  The weight stream is the whole cost at decode sizes.
+//   Standard  D[m, n] = sum_k Xq[m,k] Wq[n,k]: a CTA owns a 128-token x
+//             tile_n-column output tile; the large-M path.
+//
+// Either one runs with split_k CTAs along K (Split-K).  Partials are added
+// by the last CTA to arrive at a tile (in split order, deterministic), by a
+// second kernel (two-pass, deterministic), or atomically.
+//
+// Algorithm variants and their roles follow "Building a High-Performance and
+// Portable vLLM Linear Backend with Helion" (section "Como se implementa el
+// kernel?" and its matmul listing); the formats follow its scope list.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues MMAs, warps 2-5 drain the accumulator (warp w reads TMEM lanes
+// 32*(w%4) .. +31).  Every mbarrier wait is bounded; a wait that gives up
+// records an error code, and the CTA unwinds, drains what it issued, frees
+// TMEM and exits.
+#include <cuda_bf16.h>
+
+#include "qgd_internal.h"
+#include "sm100.cuh"
+
+namespace qgd {
+
+// First error code recorded by any kernel of this library on this device.
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+__device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_device_error, 0u, code); }
+
+constexpr uint32_t kBarBytes = 512;  // mbarriers + a few flags, after the rings
+
+struct SmemCtl {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t tfull[4];
+  uint64_t tempty[4];
+  uint64_t accfull;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int last_flag;
+  int epi_ok;
+};
+static_assert(sizeof(SmemCtl) <= kBarBytes, "control block too large");
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// Wait on an mbarrier with the whole warp and agree on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int kCols>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[kCols]) {
+  static_assert(kCols % 16 == 0, "columns come in groups of 16");
+#pragma unroll
+  for (int c = 0; c < kCols / 16; ++c) {
+    uint32_t t[16];
+    tmem_ld16(taddr + c * 16, t);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[c * 16 + j] = t[j];
+  }
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Accumulator word (fp32 bits, or int32 for INT8) -> final fp32 value.
+template <int kFmt>
+__device__ __forceinline__ float scale_out(uint32_t accbits, int m, int n, const GemmArgs& a) {
+  if constexpr (kFmt == kFmtBlock) {
+    return __uint_as_float(accbits);  // scales were applied per K block
+  } else if constexpr (kFmt == kFmtINT8) {
+    return (static_cast<float>(static_cast<int32_t>(accbits)) * __ldg(a.sx + m)) * __ldg(a.sw + n);
+  } else {
+    return (__uint_as_float(accbits) * __ldg(a.sx + m)) * __ldg(a.sw + n);
+  }
+}
+
+template <int kFmt>
+__device__ __forceinline__ uint32_t add_acc(uint32_t x, uint32_t y) {
+  if constexpr (kFmt == kFmtINT8)
+    return static_cast<uint32_t>(static_cast<int32_t>(x) + static_cast<int32_t>(y));
+  else
+    return __float_as_uint(__uint_as_float(x) + __uint_as_float(y));
+}
+
+template <int kFmt>
+__device__ __forceinline__ void atomic_acc(void* base, size_t idx, uint32_t v) {
+  if constexpr (kFmt == kFmtINT8)
+    atomicAdd(static_cast<int*>(base) + idx, static_cast<int>(v));
+  else
+    atomicAdd(static_cast<float*>(base) + idx, __uint_as_float(v));
+}
+
+// Store one finished element (y in bf16, or the raw accumulator).
+template <int kFmt>
+__device__ __forceinline__ void store_final(uint32_t accbits, int m, int n, const GemmArgs& a) {
+  const size_t idx = static_cast<size_t>(m) * a.N + n;
+  if (a.raw) {
+    static_cast<uint32_t*>(a.raw)[idx] = accbits;
+  } else {
+    a.y[idx] = bf16_bits(scale_out<kFmt>(accbits, m, n, a));
+  }
+}
+
+__device__ __forceinline__ uint32_t ldcg_u32(const void* p) {
+  return __ldcg(static_cast<const unsigned int*>(p));
+}
+
+// Teardown shared by both kernels: drain on abort, then free TMEM.
+__device__ __forceinline__ void teardown(SmemCtl* ctl, int warp, int lane, int issued, int stages,
+                                         uint32_t tmem, uint32_t ncols) {
+  tc_fence_before();
+  __syncthreads();
+  if (ctl->abort_flag) {
+    if (warp == 0 && lane == 0) {
+      // the last load issued into each stage must land before the CTA exits
+      for (int i = issued > stages ? issued - stages : 0; i < issued; ++i) {
+        if (!mbar_wait(&ctl->full[i % stages], (i / stages) & 1)) {
+          record_error(kErrWaitDrain);
+          break;
+        }
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(&ctl->drain);  // arrives once every MMA issued so far is done
+      if (!mbar_wait(&ctl->drain, 0)) record_error(kErrWaitDrain);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+// Epilogue-only barrier (the 128 threads of warps 2..5).
+__device__ __forceinline__ void epi_sync() { named_bar_sync(1, 128); }
+
+// After the epilogue's waits: agree (uniformly) on whether to write output.
+__device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl) {
+  epi_sync();
+  if (threadIdx.x == 64) ctl->epi_ok = (ctl->abort_flag == 0);
+  epi_sync();
+  return ctl->epi_ok != 0;
+}
+
+// Split-K arrival: returns true in every epilogue thread of the last CTA to
+// arrive at tile `tile`.  Called after this CTA's partials are written.
+__device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile) {
+  __threadfence();
+  epi_sync();
+  if (threadIdx.x == 64) {
+    const unsigned int old = atomicAdd(a.tickets + tile, 1u);
+    ctl->last_flag = (old == static_cast<unsigned int>(a.splits - 1));
+  }
+  epi_sync();
+  const bool last = ctl->last_flag != 0;
+  if (last) __threadfence();
+  return last;
+}
+
+// ===========================================================================
+// Swap-AB kernel (decode): grid = (ceil(N/128), splits)
+// ===========================================================================
+template <int kFmt, int kMpad>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    swapab_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx,
+                  const GemmArgs a) {
+  constexpr bool kInt = (kFmt == kFmtINT8);
+  constexpr bool kBlock = (kFmt == kFmtBlock);
+  constexpr int kSlots = kBlock ? 4 : 1;
+  constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : 128);
+  constexpr uint32_t kWBytes = kSwapTileN * kTileK;
+  constexpr uint32_t kXBytes = kMpad * kTileK;
+  constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kSwapTileN, kMpad);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  const int stages = a.stages;
+  uint8_t* w_ring = base;
+  uint8_t* x_ring = base + stages * kWBytes;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * kXBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x, split = blockIdx.y;
+  const int nkt = (a.K + kTileK - 1) / kTileK;
+  const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / a.splits);
+  const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / a.splits);
+  const int nk = kt1 - kt0;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tw);
+    tma_prefetch_desc(&tx);
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&ctl->tfull[i], 1);
+      mbar_init(&ctl->tempty[i], 128);
+    }
+    mbar_init(&ctl->accfull, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    ctl->last_flag = 0;
+    ctl->epi_ok = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  int issued = 0;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t round = i / stages;
+        if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+          record_error(kErrWaitProducer);
+          ctl->abort_flag = 1;
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], kWBytes + kXBytes);
+        const int kx = (kt0 + i) * kTileK;
+        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, n_tile * kSwapTileN, pol_w);
+        tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kx, 0, pol_x);
+        issued = i + 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t w_base = smem_u32(w_ring), x_base = smem_u32(x_ring);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t round = i / stages;
+        if (!mbar_wait(&ctl->full[s], round & 1)) {
+          record_error(kErrWaitMma);
+          ctl->abort_flag = 1;
+          break;
+        }
+        uint32_t d = tmem;
+        if constexpr (kBlock) {
+          const int slot = i % kSlots;
+          if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
+            record_error(kErrWaitMma);
+            ctl->abort_flag = 1;
+            break;
+          }
+          d = tmem + slot * kMpad;
+        }
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 32; ++kk) {
+          const uint64_t ad = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
+          const uint64_t bd = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
+          const uint32_t accumulate = kBlock ? (kk > 0) : (i > 0 || kk > 0);
+          mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+        }
+        mma_commit(&ctl->empty[s]);
+        if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
+      }
+      if constexpr (!kBlock) mma_commit(&ctl->accfull);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // TMEM lane = weight row inside the tile
+    const int n = n_tile * kSwapTileN + row;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int M = a.M, N = a.N;
+    uint32_t acc[kMpad];
+
+    if constexpr (kBlock) {
+      const int KB = a.K / kTileK;
+      float facc[kMpad];
+#pragma unroll
+      for (int m = 0; m < kMpad; ++m) facc[m] = 0.f;
+      const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;  // weight block row = this tile
+      for (int i = 0; i < nk; ++i) {
+        const int slot = i % kSlots;
+        if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
+          if (lane == 0) {
+            record_error(kErrWaitEpilogue);
+            ctl->abort_flag = 1;
+          }
+          break;
+        }
+        tc_fence_after();
+        uint32_t r[kMpad];
+        tmem_load_cols<kMpad>(taddr + slot * kMpad, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&ctl->tempty[slot]);
+        const int kb = kt0 + i;
+        const float swv = __ldg(swrow + kb);
+#pragma unroll
+        for (int m = 0; m < kMpad; ++m) {
+          if (m < M) facc[m] = fmaf(__uint_as_float(r[m]), __ldg(a.sx + static_cast<size_t>(m) * KB + kb) * swv, facc[m]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < kMpad; ++m) acc[m] = __float_as_uint(facc[m]);
+    } else {
+      if (!warp_wait(&ctl->accfull, 0)) {
+        if (lane == 0) {
+          record_error(kErrWaitEpilogue);
+          ctl->abort_flag = 1;
+        }
+      } else {
+        tc_fence_after();
+        tmem_load_cols<kMpad>(taddr, acc);
+        tmem_wait_ld();
+      }
+    }
+
+    if (epi_agree_ok(ctl)) {
+      const bool in_n = n < N;
+      if (a.splits == 1) {
+        if (in_n) {
+#pragma unroll
+          for (int m = 0; m < kMpad; ++m)
+            if (m < M) store_final<kFmt>(acc[m], m, n, a);
+        }
+      } else {
+        if (in_n) {
+#pragma unroll
+          for (int m = 0; m < kMpad; ++m) {
+            if (m < M) {
+              if (a.reduce == kAtomic)
+                atomic_acc<kFmt>(a.accum, static_cast<size_t>(m) * N + n, acc[m]);
+              else
+                static_cast<uint32_t*>(a.partial)[(static_cast<size_t>(split) * M + m) * N + n] = acc[m];
+            }
+          }
+        }
+        if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, n_tile)) {
+          if (in_n) {
+            for (int m = 0; m < M && m < kMpad; ++m) {
+              const size_t idx = static_cast<size_t>(m) * N + n;
+              uint32_t v;
+              if (a.reduce == kAtomic) {
+                v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
+                static_cast<uint32_t*>(a.accum)[idx] = 0u;
+              } else {
+                v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
+                for (int s = 1; s < a.splits; ++s)
+                  v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
+                                                 (static_cast<size_t>(s) * M) * N + idx));
+              }
+              store_final<kFmt>(v, m, n, a);
+            }
+          }
+          if (threadIdx.x == 64) a.tickets[n_tile] = 0u;
+        }
+      }
+    }
+  }
+
+  teardown(ctl, warp, lane, issued, stages, tmem, kCols);
+}
+
+// ===========================================================================
+// Standard kernel (large M): grid = (ceil(N/kTileN), ceil(M/128), splits)
+// ===========================================================================
+template <int kFmt, int kTileN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    standard_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+                    const GemmArgs a) {
+  constexpr bool kInt = (kFmt == kFmtINT8);
+  constexpr bool kBlock = (kFmt == kFmtBlock);
+  static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
+  constexpr int kSlots = kBlock ? 2 : 1;
+  constexpr uint32_t kCols = kSlots * kTileN;  // 128 or 256
+  constexpr uint32_t kXBytes = kStdTileM * kTileK;
+  constexpr uint32_t kWBytes = kTileN * kTileK;
+  constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kStdTileM, kTileN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  const int stages = a.stages;
+  uint8_t* x_ring = base;
+  uint8_t* w_ring = base + stages * kXBytes;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * kWBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
+  const int nkt = (a.K + kTileK - 1) / kTileK;
+  const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / a.splits);
+  const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / a.splits);
+  const int nk = kt1 - kt0;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tx);
+    tma_prefetch_desc(&tw);
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&ctl->tfull[i], 1);
+      mbar_init(&ctl->tempty[i], 128);
+    }
+    mbar_init(&ctl->accfull, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    ctl->last_flag = 0;
+    ctl->epi_ok = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  int issued = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_w = policy_evict_last();
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t round = i / stages;
+        if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+          record_error(kErrWaitProducer);
+          ctl->abort_flag = 1;
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
+        mbar_arrive_expect_tx(&ctl->full[s], kXBytes + kWBytes);
+        const int kx = (kt0 + i) * kTileK;
+        tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kx, m_tile * kStdTileM, pol_x);
+        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, n_tile * kTileN, pol_w);
+        issued = i + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t x_base = smem_u32(x_ring), w_base = smem_u32(w_ring);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % stages;
+        const uint32_t round = i / stages;
+        if (!mbar_wait(&ctl->full[s], round & 1)) {
+          record_error(kErrWaitMma);
+          ctl->abort_flag = 1;
+          break;
+        }
+        uint32_t d = tmem;
+        if constexpr (kBlock) {
+          const int slot = i % kSlots;
+          if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
+            record_error(kErrWaitMma);
+            ctl->abort_flag = 1;
+            break;
+          }
+          d = tmem + slot * kTileN;
+        }
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 32; ++kk) {
+          const uint64_t ad = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
+          const uint64_t bd = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
+          const uint32_t accumulate = kBlock ? (kk > 0) : (i > 0 || kk > 0);
+          mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+        }
+        mma_commit(&ctl->empty[s]);
+        if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
+      }
+      if constexpr (!kBlock) mma_commit(&ctl->accfull);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int m = m_tile * kStdTileM + q * 32 + lane;  // TMEM lane = token row
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int M = a.M, N = a.N;
+    const int n0 = n_tile * kTileN;
+    const bool in_m = m < M;
+
+    if constexpr (kBlock) {
+      const int KB = a.K / kTileK;
+      float facc[kTileN];
+#pragma unroll
+      for (int j = 0; j < kTileN; ++j) facc[j] = 0.f;
+      const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
+      const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
+      for (int i = 0; i < nk; ++i) {
+        const int slot = i % kSlots;
+        const int kb = kt0 + i;
+        const float sc = in_m ? __ldg(sxrow + kb) * __ldg(swrow + kb) : 0.f;
+        if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
+          if (lane == 0) {
+            record_error(kErrWaitEpilogue);
+            ctl->abort_flag = 1;
+          }
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTileN / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(taddr + slot * kTileN + c * 16, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, facc[c * 16 + j]);
+        }
+        tc_fence_before();
+        mbar_arrive(&ctl->tempty[slot]);
+      }
+      if (epi_agree_ok(ctl)) {
+        // finished tile: convert from registers
+        if (a.splits == 1) {
+          if (in_m) {
+#pragma unroll
+            for (int c = 0; c < kTileN / 16; ++c) {
+              const int nc = n0 + c * 16;
+              if (nc >= N) break;
+              if (a.raw) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.raw) + static_cast<size_t>(m) * N + nc);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(__float_as_uint(facc[c * 16 + 4 * v]), __float_as_uint(facc[c * 16 + 4 * v + 1]),
+                                      __float_as_uint(facc[c * 16 + 4 * v + 2]), __float_as_uint(facc[c * 16 + 4 * v + 3]));
+              } else {
+                uint32_t pk[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  pk[j] = static_cast<uint32_t>(bf16_bits(facc[c * 16 + 2 * j])) |
+                          (static_cast<uint32_t>(bf16_bits(facc[c * 16 + 2 * j + 1])) << 16);
+                uint4* dst = reinterpret_cast<uint4*>(a.y + static_cast<size_t>(m) * N + nc);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              }
+            }
+          }
+        } else {
+          if (in_m) {
+#pragma unroll
+            for (int c = 0; c < kTileN / 16; ++c) {
+              const int nc = n0 + c * 16;
+              if (nc >= N) break;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const size_t idx = static_cast<size_t>(m) * N + nc + j;
+                if (a.reduce == kAtomic)
+                  atomic_acc<kFmt>(a.accum, idx, __float_as_uint(facc[c * 16 + j]));
+                else
+                  static_cast<float*>(a.partial)[static_cast<size_t>(split) * M * N + idx] = facc[c * 16 + j];
+              }
+            }
+          }
+          if (a.reduce != kTwoPass) {
+            const int tile = m_tile * gridDim.x + n_tile;
+            if (epi_arrive_last(ctl, a, tile)) {
+              if (in_m) {
+                for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
+                  const size_t idx = static_cast<size_t>(m) * N + nc;
+                  uint32_t v;
+                  if (a.reduce == kAtomic) {
+                    v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
+                    static_cast<uint32_t*>(a.accum)[idx] = 0u;
+                  } else {
+                    v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
+                    for (int s = 1; s < a.splits; ++s)
+                      v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
+                                                     static_cast<size_t>(s) * M * N + idx));
+                  }
+                  store_final<kFmt>(v, m, nc, a);
+                }
+              }
+              if (threadIdx.x == 64) a.tickets[tile] = 0u;
+            }
+          }
+        }
+      }
+    } else {
+      bool ok = warp_wait(&ctl->accfull, 0);
+      if (!ok && lane == 0) {
+        record_error(kErrWaitEpilogue);
+        ctl->abort_flag = 1;
+      }
+      if (ok) tc_fence_after();
+      if (epi_agree_ok(ctl)) {
+        const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
+        if (a.splits == 1) {
+#pragma unroll 1
+          for (int c = 0; c < kTileN / 16; ++c) {
+            const int nc = n0 + c * 16;
+            uint32_t r[16];
+            __syncwarp();
+            tmem_ld16(taddr + c * 16, r);
+            tmem_wait_ld();
+            if (in_m && nc < N) {
+            if (a.raw) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            } else {
+              const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+              float sw16[16];
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 t = __ldg(swv + v);
+                sw16[4 * v] = t.x;
+                sw16[4 * v + 1] = t.y;
+                sw16[4 * v + 2] = t.z;
+                sw16[4 * v + 3] = t.w;
+              }
+              uint32_t pk[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float v0, v1;
+                if constexpr (kInt) {
+                  v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
+                  v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+                } else {
+                  v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
+                  v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+                }
+                pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(a.y + static_cast<size_t>(m) * N + nc);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < kTileN / 16; ++c) {
+            const int nc = n0 + c * 16;
+            uint32_t r[16];
+            __syncwarp();
+            tmem_ld16(taddr + c * 16, r);
+            tmem_wait_ld();
+            if (in_m && nc < N) {
+              const size_t idx = static_cast<size_t>(m) * N + nc;
+              if (a.reduce == kAtomic) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, r[j]);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+              }
+            }
+          }
+          if (a.reduce != kTwoPass) {
+            const int tile = m_tile * gridDim.x + n_tile;
+            if (epi_arrive_last(ctl, a, tile)) {
+              if (in_m) {
+                for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
+                  const size_t idx = static_cast<size_t>(m) * N + nc;
+                  uint32_t v;
+                  if (a.reduce == kAtomic) {
+                    v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
+                    static_cast<uint32_t*>(a.accum)[idx] = 0u;
+                  } else {
+                    v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
+                    for (int s = 1; s < a.splits; ++s)
+                      v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
+                                                     static_cast<size_t>(s) * M * N + idx));
+                  }
+                  store_final<kFmt>(v, m, nc, a);
+                }
+              }
+              if (threadIdx.x == 64) a.tickets[tile] = 0u;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  teardown(ctl, warp, lane, issued, stages, tmem, kCols);
+}
+
+// ===========================================================================
+// Two-pass Split-K reduction: one thread per output element, partials added
+// in split order s = 0, 1, ..., splits-1.
+// ===========================================================================
+template <int kFmt>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
+  const size_t total = static_cast<size_t>(a.M) * a.N;
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const uint32_t* p = static_cast<const uint32_t*>(a.partial);
+  uint32_t v = p[idx];
+  for (int s = 1; s < a.splits; ++s) v = add_acc<kFmt>(v, p[static_cast<size_t>(s) * total + idx]);
+  const int m = static_cast<int>(idx / a.N), n = static_cast<int>(idx % a.N);
+  store_final<kFmt>(v, m, n, a);
+}
+
+template <typename Kern>
+cudaError_t launch_kernel(Kern kernel, dim3 grid, size_t smem, cudaStream_t stream, bool& attr_done,
+                          const CUtensorMap& t0, const CUtensorMap& t1, const GemmArgs& a) {
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_budget()));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  kernel<<<grid, kGemmThreads, smem, stream>>>(t0, t1, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t swapab_smem_bytes(int mpad, int stages) {
+  return 1024 + static_cast<size_t>(stages) * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes;
+}
+
+size_t standard_smem_bytes(int tile_n, int stages) {
+  return 1024 + static_cast<size_t>(stages) * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
+}
+
+int swapab_max_stages(int mpad) {
+  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kSwapTileN * kTileK + mpad * kTileK));
+  return s > kMaxStages ? kMaxStages : s;
+}
+
+int standard_max_stages(int tile_n) {
+  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kStdTileM * kTileK + tile_n * kTileK));
+  return s > kMaxStages ? kMaxStages : s;
+}
+
+template <int kFmt, int kMpad>
+static cudaError_t launch_swapab_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                                   cudaStream_t stream) {
+  static bool attr_done = false;
+  const dim3 grid((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
+  return launch_kernel(swapab_kernel<kFmt, kMpad>, grid, swapab_smem_bytes(kMpad, a.stages), stream, attr_done, tw,
+                       tx, a);
+}
+
+template <int kFmt, int kTileN>
+static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                                     cudaStream_t stream) {
+  static bool attr_done = false;
+  const dim3 grid((a.N + kTileN - 1) / kTileN, (a.M + kStdTileM - 1) / kStdTileM, a.splits);
+  return launch_kernel(standard_kernel<kFmt, kTileN>, grid, standard_smem_bytes(kTileN, a.stages), stream,
+                       attr_done, tx, tw, a);
+}
+
+cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                          cudaStream_t stream) {
+  switch (fmt * 2 + (mpad == 32 ? 1 : 0)) {
+    case 0: return launch_swapab_t<kFmtFP8, 16>(tw, tx, a, stream);
+    case 1: return launch_swapab_t<kFmtFP8, 32>(tw, tx, a, stream);
+    case 2: return launch_swapab_t<kFmtINT8, 16>(tw, tx, a, stream);
+    case 3: return launch_swapab_t<kFmtINT8, 32>(tw, tx, a, stream);
+    case 4: return launch_swapab_t<kFmtBlock, 16>(tw, tx, a, stream);
+    case 5: return launch_swapab_t<kFmtBlock, 32>(tw, tx, a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
+                            const GemmArgs& a, cudaStream_t stream) {
+  if (fmt == kFmtFP8) return tile_n == 256 ? launch_standard_t<kFmtFP8, 256>(tx, tw, a, stream)
+                                           : launch_standard_t<kFmtFP8, 128>(tx, tw, a, stream);
+  if (fmt == kFmtINT8) return tile_n == 256 ? launch_standard_t<kFmtINT8, 256>(tx, tw, a, stream)
+                                            : launch_standard_t<kFmtINT8, 128>(tx, tw, a, stream);
+  if (fmt == kFmtBlock && tile_n == 128) return launch_standard_t<kFmtBlock, 128>(tx, tw, a, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t read_device_error(unsigned int* code) {
+  return cudaMemcpyFromSymbol(code, g_device_error, sizeof(unsigned int));
+}
+
+cudaError_t clear_device_error() {
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+
+cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream) {
+  const size_t total = static_cast<size_t>(a.M) * a.N;
+  const unsigned blocks = static_cast<unsigned>((total + 255) / 256);
+  if (fmt == kFmtFP8) splitk_reduce_kernel<kFmtFP8><<<blocks, 256, 0, stream>>>(a);
+  else if (fmt == kFmtINT8) splitk_reduce_kernel<kFmtINT8><<<blocks, 256, 0, stream>>>(a);
+  else splitk_reduce_kernel<kFmtBlock><<<blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace qgd

@@ -1,0 +1,58 @@
+// Shared declarations between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qgd {
+
+enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2 };
+enum Variant : int { kStandard = 0, kSwapAB = 1 };
+enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2 };
+
+constexpr int kTileK = 128;           // K elements (= bytes) per pipeline stage
+constexpr int kSwapTileN = 128;       // weight rows per Swap-AB CTA (MMA M)
+constexpr int kStdTileM = 128;        // token rows per Standard CTA (MMA M)
+constexpr int kMaxStages = 16;
+constexpr int kGemmThreads = 192;     // producer warp, MMA warp, 4 epilogue warps
+// Opt-in dynamic shared memory per CTA on sm_100 (227 KB).
+constexpr size_t kSmemBudget = 232448;
+inline size_t smem_budget() { return kSmemBudget; }
+
+// Runtime arguments common to both GEMM orientations.
+struct GemmArgs {
+  const float* sx;      // FP8/INT8: [M]; Block: [M][K/128]
+  const float* sw;      // FP8/INT8: [N]; Block: [N/128][K/128]
+  uint16_t* y;          // bf16 [M][N]
+  void* raw;            // when non-null: fp32/int32 accumulator [M][N] instead of y
+  void* partial;        // Split-K partials, 4-byte [splits][M][N]
+  void* accum;          // atomic Split-K accumulator, 4-byte [M][N], zero on entry
+  unsigned int* tickets;  // per output tile arrival counters, zero on entry
+  int M, N, K;
+  int splits;
+  int reduce;
+  int stages;
+};
+
+// Launchers (gemm.cu).  Each returns the cudaError_t of the launch.
+cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                          cudaStream_t stream);
+cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
+                            const GemmArgs& a, cudaStream_t stream);
+cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
+cudaError_t read_device_error(unsigned int* code);
+cudaError_t clear_device_error();
+size_t swapab_smem_bytes(int mpad, int stages);
+size_t standard_smem_bytes(int tile_n, int stages);
+int swapab_max_stages(int mpad);
+int standard_max_stages(int tile_n);
+
+// Quantizer launchers (quant.cu).
+cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, void* q, float* s,
+                              cudaStream_t stream);
+cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, uint8_t* q, float* s, cudaStream_t stream);
+cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream);
+
+}  // namespace qgd

@@ -1,0 +1,207 @@
+// Dynamic quantizers: bf16 -> e4m3 / int8 codes plus fp32 scales.
+//
+// For a group g of values sharing one scale (a row, a 1x128 group, or a
+// 128x128 block):  amax = max(max|x|, 1e-12f),  s = amax / qmax  (qmax 448
+// for e4m3, 127 for int8), q = convert(x / s).  Both divisions are IEEE
+// round-to-nearest (__fdiv_rn); the e4m3 conversion rounds to nearest even and
+// saturates to +-448 (cvt.rn.satfinite), int8 rounds half to even and clamps
+// to [-127, 127].  Formats and scale granularities: "Building a
+// High-Performance and Portable vLLM Linear Backend with Helion", section "Put
+// algorithm selection inside the search space".
+//
+// Each kernel loads its group once with 16-byte vector loads, keeps it in
+// registers, reduces the absolute maximum with warp shuffles, and writes the
+// codes with 8-byte stores.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "qgd_internal.h"
+
+namespace qgd {
+namespace {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kInt8Max = 127.0f;
+constexpr float kAmaxFloor = 1e-12f;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+  float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t int8_code(float v) {
+  int q = __float2int_rn(v);
+  q = q > 127 ? 127 : (q < -127 ? -127 : q);
+  return static_cast<uint32_t>(q) & 0xFFu;
+}
+
+// 8 bf16 values (one uint4) / s -> 8 codes packed in a uint2.
+template <int kQType>
+__device__ __forceinline__ uint2 encode8(const uint4& v, float s) {
+  const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+  float d[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i] = __fdiv_rn(f[i], s);
+  uint2 out;
+  if constexpr (kQType == 0) {
+    out.x = e4m3x2(d[0], d[1]) | (e4m3x2(d[2], d[3]) << 16);
+    out.y = e4m3x2(d[4], d[5]) | (e4m3x2(d[6], d[7]) << 16);
+  } else {
+    out.x = int8_code(d[0]) | (int8_code(d[1]) << 8) | (int8_code(d[2]) << 16) | (int8_code(d[3]) << 24);
+    out.y = int8_code(d[4]) | (int8_code(d[5]) << 8) | (int8_code(d[6]) << 16) | (int8_code(d[7]) << 24);
+  }
+  return out;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Maximum over the whole CTA (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ float block_max(float v, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  v = warp_max(v);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float t = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_max(t);
+    if (lane == 0) red[32] = t;
+  }
+  __syncthreads();
+  return red[32];
+}
+
+// ---------------------------------------------------------------------------
+// One CTA per row; each thread holds kVPT vectors of 8 values.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 512;
+
+template <int kVPT, int kQType>
+__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int K,
+                                                                 uint8_t* __restrict__ q, float* __restrict__ s) {
+  __shared__ float red[33];
+  const size_t row = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+  uint2* qr = reinterpret_cast<uint2*>(q + row * K);
+  const int nvec = K / 8;
+  uint4 v[kVPT];
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < kVPT; ++j) {
+    const int idx = threadIdx.x + j * kRowThreads;
+    if (idx < nvec) {
+      v[j] = __ldg(xr + idx);
+      amax = fmaxf(amax, absmax8(v[j]));
+    }
+  }
+  amax = fmaxf(block_max(amax, red), kAmaxFloor);
+  const float sc = __fdiv_rn(amax, kQType == 0 ? kE4M3Max : kInt8Max);
+  if (threadIdx.x == 0) s[row] = sc;
+#pragma unroll
+  for (int j = 0; j < kVPT; ++j) {
+    const int idx = threadIdx.x + j * kRowThreads;
+    if (idx < nvec) qr[idx] = encode8<kQType>(v[j], sc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 1x128 groups: a half-warp per group, 8 values per lane.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                             uint8_t* __restrict__ q, float* __restrict__ s) {
+  const int KB = K / 128;
+  const long long g = static_cast<long long>(blockIdx.x) * 16 + (threadIdx.x >> 4);
+  const int sub = threadIdx.x & 15;
+  const bool valid = g < static_cast<long long>(M) * KB;
+  const long long gg = valid ? g : 0;
+  const long long m = gg / KB, kb = gg % KB;
+  const size_t off = static_cast<size_t>(m) * K + static_cast<size_t>(kb) * 128 + sub * 8;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (valid) v = __ldg(reinterpret_cast<const uint4*>(x + off));
+  float amax = absmax8(v);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  amax = fmaxf(amax, kAmaxFloor);
+  const float sc = __fdiv_rn(amax, kE4M3Max);
+  if (valid) {
+    *reinterpret_cast<uint2*>(q + off) = encode8<0>(v, sc);
+    if (sub == 0) s[static_cast<size_t>(m) * KB + kb] = sc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 128x128 weight blocks: one CTA of 256 threads per block, 8 vectors each.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_block128_kernel(const uint16_t* __restrict__ w, int K,
+                                                             uint8_t* __restrict__ q, float* __restrict__ s) {
+  __shared__ float red[33];
+  const int nb = blockIdx.y, kb = blockIdx.x, KB = gridDim.x;
+  uint4 v[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int t = threadIdx.x + j * 256;  // 0..2047: row = t/16, vector = t%16
+    const size_t off = static_cast<size_t>(nb * 128 + t / 16) * K + kb * 128 + (t % 16) * 8;
+    v[j] = __ldg(reinterpret_cast<const uint4*>(w + off));
+    amax = fmaxf(amax, absmax8(v[j]));
+  }
+  amax = fmaxf(block_max(amax, red), kAmaxFloor);
+  const float sc = __fdiv_rn(amax, kE4M3Max);
+  if (threadIdx.x == 0) s[static_cast<size_t>(nb) * KB + kb] = sc;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int t = threadIdx.x + j * 256;
+    const size_t off = static_cast<size_t>(nb * 128 + t / 16) * K + kb * 128 + (t % 16) * 8;
+    *reinterpret_cast<uint2*>(q + off) = encode8<0>(v[j], sc);
+  }
+}
+
+template <int kQType>
+cudaError_t launch_rows_q(const uint16_t* x, int rows, int K, void* q, float* s, cudaStream_t st) {
+  const int nvec = K / 8;
+  const int vpt = (nvec + kRowThreads - 1) / kRowThreads;
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  if (vpt <= 1) quant_rows_kernel<1, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
+  else if (vpt <= 2) quant_rows_kernel<2, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
+  else if (vpt <= 4) quant_rows_kernel<4, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
+  else if (vpt <= 8) quant_rows_kernel<8, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
+  else if (vpt <= 16) quant_rows_kernel<16, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, void* q, float* s,
+                              cudaStream_t stream) {
+  return qtype == 0 ? launch_rows_q<0>(x, rows, K, q, s, stream) : launch_rows_q<1>(x, rows, K, q, s, stream);
+}
+
+cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, uint8_t* q, float* s, cudaStream_t stream) {
+  const long long groups = static_cast<long long>(M) * (K / 128);
+  const unsigned blocks = static_cast<unsigned>((groups + 15) / 16);
+  quant_group128_kernel<<<blocks, 256, 0, stream>>>(x, M, K, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream) {
+  const dim3 grid(K / 128, N / 128);
+  quant_block128_kernel<<<grid, 256, 0, stream>>>(w, K, q, s);
+  return cudaGetLastError();
+}
+
+}  // namespace qgd

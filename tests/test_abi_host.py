@@ -1,0 +1,172 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function
+include/qgd.h declares, and its host-side logic (M buckets, default plans,
+dispatch-table parsing, overrides, workspace sizing, argument rejection)
+behaves as documented.  No GPU and no kernel launch is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_gemm_decode_b200 as qgd
+from quantized_gemm_decode_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgd.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+    qgd.lib()
+    yield
+    qgd.qgd_clear_dispatch_table()
+    for f in range(3):
+        qgd.qgd_set_override(f)
+
+
+@pytest.fixture(autouse=True)
+def clean_state():
+    qgd.qgd_clear_dispatch_table()
+    for f in range(3):
+        qgd.qgd_set_override(f)
+    yield
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^QGD_API\s+[\w\s\*]+?\b(\w+)\(", text, flags=re.M)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for required in ("quant_act_per_token", "quant_act_group128", "quant_weight_block128",
+                     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8",
+                     "qgd_load_dispatch_table", "qgd_workspace_size", "qgd_set_override",
+                     "qgd_w8a8_int8_acc32", "qgd_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(qgd.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version():
+    L = qgd.lib()
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert L.qgd_status_string(st)
+    assert qgd.qgd_version().count(".") == 2
+
+
+@pytest.mark.parametrize("M,b", [(1, 1), (2, 2), (3, 4), (5, 8), (9, 16), (17, 24), (25, 32), (33, 64),
+                                 (100, 128), (129, 512), (600, 2048), (3000, 8192), (100000, 8192)])
+def test_m_buckets(M, b):
+    assert qgd.qgd_m_bucket(M) == b
+
+
+def test_default_plans():
+    # decode: Swap-AB, split until the 148 SMs are covered
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)
+    assert p["variant"] == qgd.VARIANT_SWAP_AB and p["source"] == 0
+    assert p["split_k"] == 8  # 32 tiles * 8 >= 148
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 32, 24576, 4096)
+    assert p["split_k"] == 1  # 192 tiles already cover the SMs
+    # large M: Standard, no split
+    p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 512, 6144, 4096)
+    assert p["variant"] == qgd.VARIANT_STANDARD and p["split_k"] == 1 and p["tile_n"] == 256
+    p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 512, 6144, 4096)
+    assert p["tile_n"] == 128
+    # split never exceeds the number of 128-wide K tiles
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 128, 256)
+    assert p["split_k"] == 2
+
+
+def test_override_and_clamping():
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 256, qgd.REDUCE_ATOMIC, 5, 0)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+    assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["source"]) == (1, 32, 2, 5, 2)
+    # Swap-AB cannot take more than 32 tokens: it falls back to Standard
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)
+    assert p["variant"] == qgd.VARIANT_STANDARD
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 3, 0, 0, 0)  # split not a power of two
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(7, 1, 2, 0, 0, 0)
+
+
+def test_workspace_size_follows_plan():
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 1, 0, 0, 0)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 0
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0)
+    # 32 tile counters (rounded to 256 bytes) + 8 partials of 4 x 4096 fp32
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 256 + 8 * 4 * 4096 * 4
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_TWO_PASS, 0, 0)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 8 * 4 * 4096 * 4
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_ATOMIC, 0, 0)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 256 + 4 * 4096 * 4
+
+
+def test_table_load_and_lookup(tmp_path):
+    t = tmp_path / "t.tsv"
+    t.write_text("# fmt N K M_bucket variant split_k reduce stages tile_n\n"
+                 "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n"
+                 "\n"
+                 "w8a8_int8 5120 5120 32 swap_ab 4 atomic 0 0   # trailing comment\n")
+    qgd.qgd_load_dispatch_table(str(t))
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 3, 4096, 4096)  # bucket 4
+    assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["tile_n"], p["source"]) == (0, 2, 1, 4, 256, 1)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 5, 4096, 4096)  # bucket 8: not in the table
+    assert p["source"] == 0
+    p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)
+    assert (p["variant"], p["split_k"], p["reduce"], p["source"]) == (1, 4, 2, 1)
+    qgd.qgd_clear_dispatch_table()
+    assert qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)["source"] == 0
+
+
+@pytest.mark.parametrize("bad", [
+    "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256\n",      # split not a power of two
+    "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256\n",      # 5 is not a bucket
+    "fp9 4096 4096 4 standard 2 two_pass 4 256\n",              # unknown format
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4\n",          # missing field
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 7\n",    # extra field
+    "fp8_dynamic 4096 4096 4 diagonal 2 two_pass 4 256\n",      # unknown variant
+])
+def test_malformed_table_is_rejected_and_keeps_previous(tmp_path, bad):
+    good = tmp_path / "good.tsv"
+    good.write_text("fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n")
+    qgd.qgd_load_dispatch_table(str(good))
+    t = tmp_path / "bad.tsv"
+    t.write_text(bad)
+    with pytest.raises(qgd.QGDError) as e:
+        qgd.qgd_load_dispatch_table(str(t))
+    assert e.value.status == -5
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["source"] == 1
+
+
+def test_missing_table_file():
+    with pytest.raises(qgd.QGDError) as e:
+        qgd.qgd_load_dispatch_table("/nonexistent/table.tsv")
+    assert e.value.status == -5
+
+
+def test_shipped_table_parses():
+    if os.path.exists(qgd.DEFAULT_TABLE):
+        qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
+
+
+def test_argument_rejection_before_any_launch():
+    L = qgd.lib()
+    P = ctypes.c_void_p
+    # null pointers / bad shapes are rejected on the host, with no device call
+    assert L.qlinear_fp8_dynamic(None, None, None, None, None, 4, 512, 1024, None, 0, None) == -1
+    assert L.qlinear_fp8_dynamic(P(16), P(16), P(16), P(16), P(16), 4, 500, 1024, None, 0, None) == -2
+    assert L.qlinear_block_fp8(P(16), P(16), P(16), P(16), P(16), 4, 512, 1000, None, 0, None) == -2
+    assert L.qlinear_w8a8_int8(P(16), P(16), P(16), P(16), P(16), -1, 512, 1024, None, 0, None) == -1
+    assert L.qlinear_fp8_dynamic(P(17), P(16), P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
+    assert L.quant_act_per_token(P(16), 4, 12, 0, P(16), P(16), None) == -2
+    assert L.quant_act_per_token(P(16), 4, 16, 5, P(16), P(16), None) == -1
+    # M == 0 is an empty, successful call
+    assert L.qlinear_fp8_dynamic(None, None, None, None, None, 0, 512, 1024, None, 0, None) == 0
+    assert b"16" in L.qgd_last_error_message() or L.qgd_last_error_message() is not None

@@ -1,0 +1,180 @@
+"""GPU parity of the quantized GEMMs against the oracle, per algorithm variant.
+
+Every variant (Swap-AB / Standard, split_k, reduction mode) is forced through
+qgd_set_override and compared with the oracle on the same seeded inputs:
+INT8 accumulators bit-exact, INT8 bf16 output within one ulp of the oracle's
+fp32 value, FP8 outputs within the stated tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import quantized_gemm_decode_b200 as qgd
+from quantized_gemm_decode_b200 import synth
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8
+from paritylib import FMT_ID, Case, as_u8, bf16_to_f64
+
+pytestmark = pytest.mark.gpu
+
+ALL_FMTS = [FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8]
+
+
+@pytest.fixture(autouse=True)
+def _no_override():
+    qgd.lib()
+    for f in range(3):
+        qgd.qgd_set_override(f)
+    yield
+    for f in range(3):
+        qgd.qgd_set_override(f)
+
+
+def _oracle(case: Case, want_acc=False):
+    xq, sx, wq, sw = case.oracle_quant()
+    # the GPU and the oracle quantize independently; bytes must agree first
+    np.testing.assert_array_equal(as_u8(case.xq), xq.view(np.uint8))
+    np.testing.assert_array_equal(as_u8(case.wq), wq.view(np.uint8))
+    return case.oracle_gemm(xq, sx, wq, sw, want_acc=want_acc)
+
+
+def test_tiny_fp8_dynamic_default_plan():
+    # FP8_Dynamic, X 4x1024 ~N(0,1), W 512x1024 ~N(0,0.02), seed 0
+    case = Case(FP8_DYNAMIC, 4, 512, 1024, seed=0, outliers=False)
+    yref, bound = _oracle(case)
+    case.check_output(case.run(), yref, bound, "tiny default")
+
+
+VARIANTS = (
+    [(qgd.VARIANT_SWAP_AB, s, r, 0) for s in (1, 2, 4, 8) for r in (0, 1, 2)]
+    + [(qgd.VARIANT_STANDARD, s, r, t) for t in (128, 256) for s in (1, 2, 8) for r in (0, 1, 2)]
+)
+
+
+def _vid(v):
+    return f"{'swap' if v[0] == qgd.VARIANT_SWAP_AB else 'std'}-s{v[1]}-r{v[2]}-t{v[3]}"
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("variant", VARIANTS, ids=_vid)
+def test_every_variant_tiny(fmt, variant):
+    var, split, red, tile = variant
+    if fmt == BLOCK_FP8 and tile == 256:
+        pytest.skip("Block_FP8 Standard tiles are 128 wide")
+    case = Case(fmt, 4, 512, 1024, seed=1, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, tile)
+    plan = qgd.qgd_get_plan(FMT_ID[fmt], 4, 512, 1024)
+    assert plan["variant"] == var and plan["split_k"] == split and plan["source"] == 2
+    case.check_output(case.run(), yref, bound, f"{fmt} {_vid(variant)}")
+
+
+@pytest.mark.parametrize("variant", VARIANTS, ids=_vid)
+def test_int8_acc32_bit_exact_every_variant(variant):
+    var, split, red, tile = variant
+    case = Case(W8A8_INT8, 5, 640, 2048, seed=2, outliers=True)
+    _, _, acc = _oracle(case, want_acc=True)
+    qgd.qgd_set_override(qgd.FMT_W8A8_INT8, var, split, red, 0, tile)
+    got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 15, 16, 17, 24, 31, 32])
+def test_decode_m_range(fmt, M):
+    case = Case(fmt, M, 768, 2048, seed=M, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    case.check_output(case.run(), yref, bound, f"{fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("M,N,K", [(33, 512, 1024), (100, 384, 2048), (130, 640, 1024), (257, 256, 512)])
+def test_large_m_standard(fmt, M, N, K):
+    case = Case(fmt, M, N, K, seed=M + N, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    assert qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)["variant"] == qgd.VARIANT_STANDARD
+    case.check_output(case.run(), yref, bound, f"{fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
+@pytest.mark.parametrize("M,N,K", [(3, 528, 1040), (20, 1040, 272), (40, 272, 1040), (1, 16, 16)])
+def test_ragged_tiles(fmt, M, N, K):
+    # N not a multiple of the 128/256 tile, K not a multiple of the 128 stage
+    case = Case(fmt, M, N, K, seed=N, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    for var, split, red in ((qgd.VARIANT_SWAP_AB, 1, 0), (qgd.VARIANT_SWAP_AB, 4, 0),
+                            (qgd.VARIANT_STANDARD, 1, 0), (qgd.VARIANT_STANDARD, 2, 1)):
+        if var == qgd.VARIANT_SWAP_AB and M > 32:
+            continue
+        qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, 0)
+        case.check_output(case.run(), yref, bound, f"{fmt} M={M} N={N} K={K} var={var} s={split}")
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+def test_empty_m(fmt):
+    case = Case(fmt, 1, 256, 1024, seed=5)
+    xq = case.xq[:0]
+    fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
+          BLOCK_FP8: qgd.qlinear_block_fp8}[fmt]
+    y = fn(xq, case.sx[:0], case.wq, case.sw)
+    assert y.shape == (0, 256)
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("reduce", [qgd.REDUCE_LAST_CTA, qgd.REDUCE_TWO_PASS])
+def test_deterministic_split_reductions_repeat_bitwise(fmt, reduce):
+    case = Case(fmt, 7, 1024, 4096, seed=9)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, 8, reduce, 0, 0)
+    ys = [case.run().view(torch.int16).cpu() for _ in range(4)]
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+
+
+def test_split_k_up_to_256():
+    # K = 32768 gives 256 K tiles, so every power of two up to 256 is legal
+    case = Case(W8A8_INT8, 2, 256, 32768, seed=4)
+    _, _, acc = _oracle(case, want_acc=True)
+    for split in (16, 64, 256):
+        for red in (0, 1, 2):
+            qgd.qgd_set_override(qgd.FMT_W8A8_INT8, qgd.VARIANT_SWAP_AB, split, red, 0, 0)
+            assert qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 2, 256, 32768)["split_k"] == split
+            got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc, err_msg=f"s={split} r={red}")
+
+
+def test_graph_replay_matches_eager():
+    case = Case(FP8_DYNAMIC, 8, 1024, 4096, seed=3)
+    ws = qgd.Workspace(qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 8, 1024, 4096) + 4096)
+    y_eager = case.run(ws=ws).clone()
+    y = torch.empty_like(y_eager)
+    xq = torch.empty_like(case.xq)
+    sx = torch.empty_like(case.sx)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):  # warm up outside capture
+            qgd.quant_act_per_token(case.xd, qgd.QTYPE_E4M3, xq=xq, sx=sx)
+            qgd.qlinear_fp8_dynamic(xq, sx, case.wq, case.sw, y=y, ws=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        qgd.quant_act_per_token(case.xd, qgd.QTYPE_E4M3, xq=xq, sx=sx)
+        qgd.qlinear_fp8_dynamic(xq, sx, case.wq, case.sw, y=y, ws=ws)
+    for _ in range(5):
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
+
+
+def test_workspace_errors_are_reported():
+    case = Case(FP8_DYNAMIC, 4, 512, 4096, seed=3)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, qgd.REDUCE_LAST_CTA, 0, 0)
+    need = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 512, 4096)
+    assert need > 0
+    small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(qgd.QGDError) as e:
+        qgd.qlinear_fp8_dynamic(case.xq, case.sx, case.wq, case.sw, ws=small)
+    assert e.value.status == -3
+    assert qgd.qgd_device_error() == 0
