@@ -119,9 +119,12 @@ QGD_API qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void*
  * Shapes: M >= 0; N % 16 == 0; K % 16 == 0 (FP8_Dynamic, W8A8_INT8) or
  * K % 128 == 0 and N % 128 == 0 (Block_FP8).
  * Workspace: `ws` (device, >= qgd_workspace_size() bytes for the same
- * arguments) holds Split-K partials and per-tile arrival counters.  It must be
- * zero-filled once after allocation; every call leaves its counters and
- * atomic accumulators zero again.  Calls that share a workspace must not run
+ * arguments) holds, when the plan splits K, a 64 KiB header of per-tile
+ * arrival counters followed by the Split-K partials (or the atomic
+ * accumulator, which the call zeroes itself with a memset node).  The header
+ * must be zero-filled once after allocation; every call leaves it zero again
+ * and never writes anything else there, so one workspace can serve calls of
+ * different shapes and plans.  Calls that share a workspace must not run
  * concurrently.  ws may be NULL when qgd_workspace_size() returns 0.
  * ------------------------------------------------------------------- */
 QGD_API qgd_status qlinear_fp8_dynamic(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,

@@ -99,6 +99,13 @@ qgd_status encode_kmajor(CUtensorMap* map, const void* base, int rows, int cols,
 // ---------------------------------------------------------------------------
 // Dispatch: table (format, N, K, M-bucket) -> plan; override per format.
 // ---------------------------------------------------------------------------
+// Workspace layout: a fixed header of per-tile arrival counters that every
+// call leaves zero, then the Split-K data (partials, or the atomic
+// accumulator, which is zeroed by a memset node at the start of the call).
+// No call ever writes data into the header, so calls with different shapes
+// and plans can share one workspace.
+constexpr size_t kTicketBytes = 64 * 1024;
+constexpr size_t kMaxTickets = kTicketBytes / 4;
 const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
 constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
@@ -197,6 +204,12 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.split_k > smax) p.split_k = smax;
   p.split_k = floor_pow2(p.split_k);
   if (p.reduce < kLastCta || p.reduce > kAtomic) p.reduce = kLastCta;
+  if (p.split_k > 1 && p.reduce != kTwoPass) {
+    const size_t tiles = p.variant == kSwapAB
+                             ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
+                             : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
+    if (tiles > kMaxTickets) p.reduce = kTwoPass;  // more tiles than arrival counters
+  }
   const int mpad = M <= 16 ? 16 : 32;
   const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad) : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
@@ -205,21 +218,15 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
 }
 
 struct WsLayout {
-  size_t tickets_off, tickets_bytes, data_off, data_bytes, total;
+  size_t data_off, data_bytes, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 WsLayout ws_layout(const qgd_plan& p, int M, int N) {
-  WsLayout w{0, 0, 0, 0, 0};
+  WsLayout w{0, 0, 0};
   if (p.split_k <= 1 || M == 0) return w;
-  size_t tiles;
-  if (p.variant == kSwapAB)
-    tiles = (N + kSwapTileN - 1) / kSwapTileN;
-  else
-    tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
-  if (p.reduce != kTwoPass) w.tickets_bytes = align256(tiles * 4);
-  w.data_off = w.tickets_bytes;
+  w.data_off = kTicketBytes;
   w.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
   w.total = w.data_off + w.data_bytes;
   return w;
@@ -263,7 +270,7 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.tickets = nullptr;
   if (wl.total > 0) {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
-    if (wl.tickets_bytes) a.tickets = reinterpret_cast<unsigned int*>(wsb + wl.tickets_off);
+    a.tickets = reinterpret_cast<unsigned int*>(wsb);
     if (p.reduce == kAtomic) a.accum = wsb + wl.data_off;
     else a.partial = wsb + wl.data_off;
   }
@@ -277,6 +284,10 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
   cudaError_t e;
+  if (a.accum) {
+    e = cudaMemsetAsync(a.accum, 0, static_cast<size_t>(M) * N * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (atomic Split-K accumulator)");
+  }
   if (p.variant == kSwapAB) {
     const int mpad = M <= 16 ? 16 : 32;
     if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;

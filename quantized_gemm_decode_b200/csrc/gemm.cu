@@ -368,7 +368,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               uint32_t v;
               if (a.reduce == kAtomic) {
                 v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-                static_cast<uint32_t*>(a.accum)[idx] = 0u;
               } else {
                 v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
                 for (int s = 1; s < a.splits; ++s)
@@ -590,7 +589,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                   uint32_t v;
                   if (a.reduce == kAtomic) {
                     v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-                    static_cast<uint32_t*>(a.accum)[idx] = 0u;
                   } else {
                     v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
                     for (int s = 1; s < a.splits; ++s)
@@ -686,7 +684,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                   uint32_t v;
                   if (a.reduce == kAtomic) {
                     v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-                    static_cast<uint32_t*>(a.accum)[idx] = 0u;
                   } else {
                     v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
                     for (int s = 1; s < a.splits; ++s)

@@ -29,7 +29,7 @@ struct GemmArgs {
   void* raw;            // when non-null: fp32/int32 accumulator [M][N] instead of y
   void* partial;        // Split-K partials, 4-byte [splits][M][N]
   void* accum;          // atomic Split-K accumulator, 4-byte [M][N], zero on entry
-  unsigned int* tickets;  // per output tile arrival counters, zero on entry
+  unsigned int* tickets;  // per output tile arrival counters (workspace header), zero on entry and exit
   int M, N, K;
   int splits;
   int reduce;

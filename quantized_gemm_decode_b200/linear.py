@@ -1,0 +1,104 @@
+"""A quantized linear layer built on the C ABI, with the method's hybrid
+dispatch: token counts up to 32 replay a CUDA graph captured once per M
+bucket (1, 2, 4, 8, 16, 24, 32); larger counts launch directly.
+
+Hybrid dispatch and graph replay follow "Building a High-Performance and
+Portable vLLM Linear Backend with Helion", section "Hybrid dispatch"
+("Despacho hibrido"): small shapes run under CUDA-graph replay so the CPU's
+launch cost does not eat the kernel's gain.
+"""
+from __future__ import annotations
+
+import torch
+
+import quantized_gemm_decode_b200 as qgd
+
+DECODE_BUCKETS = (1, 2, 4, 8, 16, 24, 32)
+GRAPH_MAX_M = 32
+
+_FMT = {"fp8_dynamic": qgd.FMT_FP8_DYNAMIC, "w8a8_int8": qgd.FMT_W8A8_INT8, "block_fp8": qgd.FMT_BLOCK_FP8}
+
+
+class QuantizedLinear:
+    """y = x @ W^T with W quantized once at construction and x quantized
+    dynamically on every call, both by this library's kernels."""
+
+    def __init__(self, w: torch.Tensor, fmt: str = "fp8_dynamic", wq=None, sw=None):
+        if fmt not in _FMT:
+            raise ValueError(f"unknown format {fmt}")
+        self.fmt = fmt
+        self.fmt_id = _FMT[fmt]
+        self.N, self.K = (w.shape if w is not None else wq.shape)
+        self.device = (w if w is not None else wq).device
+        if wq is None:
+            if fmt == "block_fp8":
+                wq, sw = qgd.quant_weight_block128(w)
+            else:
+                qt = qgd.QTYPE_INT8 if fmt == "w8a8_int8" else qgd.QTYPE_E4M3
+                wq, sw = qgd.quant_weight_per_channel(w, qt)
+        self.wq, self.sw = wq, sw
+        need = max(qgd.qgd_workspace_size(self.fmt_id, m, self.N, self.K) for m in DECODE_BUCKETS)
+        self.ws = qgd.Workspace(need, self.device)
+        self._graphs: dict = {}
+
+    # ---- eager path ---------------------------------------------------
+    def quantize(self, x: torch.Tensor, xq=None, sx=None):
+        if self.fmt == "block_fp8":
+            return qgd.quant_act_group128(x, xq=xq, sx=sx)
+        qt = qgd.QTYPE_INT8 if self.fmt == "w8a8_int8" else qgd.QTYPE_E4M3
+        return qgd.quant_act_per_token(x, qt, xq=xq, sx=sx)
+
+    def gemm(self, xq, sx, y=None):
+        fn = {"fp8_dynamic": qgd.qlinear_fp8_dynamic, "w8a8_int8": qgd.qlinear_w8a8_int8,
+              "block_fp8": qgd.qlinear_block_fp8}[self.fmt]
+        self.ws.ensure(qgd.qgd_workspace_size(self.fmt_id, xq.shape[0], self.N, self.K))
+        return fn(xq, sx, self.wq, self.sw, y=y, ws=self.ws)
+
+    def forward_eager(self, x: torch.Tensor, y=None) -> torch.Tensor:
+        xq, sx = self.quantize(x)
+        return self.gemm(xq, sx, y=y)
+
+    # ---- graph path ---------------------------------------------------
+    def capture(self, buckets=DECODE_BUCKETS) -> None:
+        """Capture one graph per M bucket (static input/output buffers)."""
+        for mb in buckets:
+            x = torch.zeros((mb, self.K), dtype=torch.bfloat16, device=self.device)
+            y = torch.empty((mb, self.N), dtype=torch.bfloat16, device=self.device)
+            xq = torch.empty((mb, self.K), dtype=torch.int8 if self.fmt == "w8a8_int8" else torch.float8_e4m3fn,
+                             device=self.device)
+            sx = torch.empty((mb, self.K // 128) if self.fmt == "block_fp8" else (mb,), dtype=torch.float32,
+                             device=self.device)
+            self.ws.ensure(qgd.qgd_workspace_size(self.fmt_id, mb, self.N, self.K))
+            s = torch.cuda.Stream(self.device)
+            s.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(s):
+                self.quantize(x, xq, sx)
+                self.gemm(xq, sx, y)
+            torch.cuda.current_stream(self.device).wait_stream(s)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.quantize(x, xq, sx)
+                self.gemm(xq, sx, y)
+            self._graphs[mb] = (g, x, y)
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        """Apply the layer.  M <= 32 replays the captured graph of M's bucket
+        (inputs are copied into its static buffer; x may live on the host,
+        pinned); larger M runs eagerly.  With `out` (possibly pinned host
+        memory) the result is copied there and `out` is returned."""
+        M = x.shape[0]
+        if M <= GRAPH_MAX_M and self._graphs:
+            mb = qgd.qgd_m_bucket(M)
+            g, xs, ys = self._graphs[mb]
+            xs[:M].copy_(x, non_blocking=True)
+            g.replay()
+            if out is not None:
+                out.copy_(ys[:M], non_blocking=True)
+                return out
+            return ys[:M]
+        xd = x if x.is_cuda else x.to(self.device, non_blocking=True)
+        y = self.forward_eager(xd)
+        if out is not None:
+            out.copy_(y, non_blocking=True)
+            return out
+        return y

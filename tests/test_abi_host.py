@@ -97,15 +97,23 @@ def test_override_and_clamping():
 
 
 def test_workspace_size_follows_plan():
+    hdr = 64 * 1024  # arrival-counter header
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 1, 0, 0, 0)
     assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 0
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0)
-    # 32 tile counters (rounded to 256 bytes) + 8 partials of 4 x 4096 fp32
-    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 256 + 8 * 4 * 4096 * 4
+    # header + 8 partials of 4 x 4096 fp32
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 8 * 4 * 4096 * 4
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_TWO_PASS, 0, 0)
-    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 8 * 4 * 4096 * 4
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 8 * 4 * 4096 * 4
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_ATOMIC, 0, 0)
-    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 256 + 4 * 4096 * 4
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 4 * 4096 * 4
+
+
+def test_too_many_tiles_for_counters_fall_back_to_two_pass():
+    # Standard tiles of 128 x 128 over 8192 x 262144 exceed the 16384 counters
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 2, qgd.REDUCE_LAST_CTA, 0, 128)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 8192, 262144, 4096)
+    assert p["reduce"] == qgd.REDUCE_TWO_PASS
 
 
 def test_table_load_and_lookup(tmp_path):

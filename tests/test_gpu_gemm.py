@@ -178,3 +178,19 @@ def test_workspace_errors_are_reported():
         qgd.qlinear_fp8_dynamic(case.xq, case.sx, case.wq, case.sw, ws=small)
     assert e.value.status == -3
     assert qgd.qgd_device_error() == 0
+
+
+def test_shared_workspace_across_modes_and_shapes():
+    # one workspace serves calls of different shapes and reduction modes in any
+    # order: partials never land on the arrival counters
+    ws = qgd.Workspace(64 * 1024 + 64 * 4 * 4096 * 4)
+    cases = [Case(FP8_DYNAMIC, 4, 512, 1024, seed=1), Case(W8A8_INT8, 3, 1024, 2048, seed=2),
+             Case(BLOCK_FP8, 5, 768, 4096, seed=3)]
+    refs = [_oracle(c)[:2] for c in cases]
+    for rnd in range(2):
+        for red in (qgd.REDUCE_TWO_PASS, qgd.REDUCE_LAST_CTA, qgd.REDUCE_ATOMIC, qgd.REDUCE_LAST_CTA):
+            for c, (yref, bound) in zip(cases, refs):
+                for f in range(3):
+                    qgd.qgd_set_override(f, qgd.VARIANT_SWAP_AB, 4 if rnd == 0 else 8, red, 0, 0)
+                c.check_output(c.run(ws=ws), yref, bound, f"{c.fmt} red={red} rnd={rnd}")
+    assert qgd.qgd_device_error() == 0
