@@ -1,0 +1,224 @@
+"""Measure every legal plan per (format, N, K, M-bucket) on this GPU and write
+the fastest to a dispatch table.
+
+The method tunes its GEMM per layer shape and per token count (1, 2, 4, 8,
+16, 24, 32) with the algorithm choice -- Standard, Split-K with split_k a
+power of two up to 256, Swap-AB -- inside the search space, and it measures
+candidates under CUDA-graph replay ("Building a High-Performance and
+Portable vLLM Linear Backend with Helion", sections "Put algorithm selection
+inside the search space", "Hybrid dispatch addresses runtime overhead" and
+"Autoajuste de los kernels").  Here the space is small and discrete, so it is
+searched exhaustively: variant x tile x split_k x reduction at the deepest
+pipeline, then the pipeline depth of the best few.  Each candidate is first
+checked against the split-free result (bit-exact int32 accumulators for
+W8A8_INT8, a relative bound for the fp32-accumulating formats), then timed as
+a graph of calls that cycle through at least 3x L2 of distinct weight copies.
+
+    python -m quantized_gemm_decode_b200.tune [--formats fp8_dynamic,...] [--out tables/b200.tsv]
+        [--large-m] [--resume]
+
+Tuning time is reported separately on stderr.  With --resume, keys already in
+the output file are kept and skipped.
+"""
+from __future__ import annotations
+
+import argparse
+import math
+import os
+import sys
+import time
+
+import torch
+
+import quantized_gemm_decode_b200 as qgd
+from quantized_gemm_decode_b200 import synth, workloads
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8
+
+L2_BYTES = 126 * 1024 * 1024
+FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}
+VAR_NAME = {0: "standard", 1: "swap_ab"}
+RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic"}
+
+
+def _quant_w(fmt, w):
+    if fmt == BLOCK_FP8:
+        return qgd.quant_weight_block128(w)
+    return qgd.quant_weight_per_channel(w, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
+
+
+def _quant_x(fmt, x):
+    if fmt == BLOCK_FP8:
+        return qgd.quant_act_group128(x)
+    return qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
+
+
+def candidates(fmt: str, M: int, N: int, K: int):
+    nkt = (K + 127) // 128
+    splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
+    out = []
+    if M <= 32:
+        for s in splits:
+            for r in ((0,) if s == 1 else (0, 1, 2)):
+                out.append((1, s, r, 128))
+    tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
+    for t in tiles:
+        for s in splits:
+            if M <= 32 and s > 16:
+                continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
+            for r in ((0,) if s == 1 else (0, 1, 2)):
+                out.append((0, s, r, t))
+    return out
+
+
+class Problem:
+    def __init__(self, fmt, M, N, K, seed, device):
+        self.fmt, self.M, self.N, self.K = fmt, M, N, K
+        self.fid = FMT_ID[fmt]
+        w = synth.weights(N, K, seed).to(device)
+        wq, sw = _quant_w(fmt, w)
+        del w
+        ncopies = max(2, math.ceil(3 * L2_BYTES / (N * K)))
+        self.copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(ncopies - 1)]
+        x = synth.activations(M, K, seed, outliers=(fmt != W8A8_INT8)).to(device)
+        self.xq, self.sx = _quant_x(fmt, x)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        self.ws = qgd.Workspace(0, device)
+        self.fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
+                   BLOCK_FP8: qgd.qlinear_block_fp8}[fmt]
+
+    def run(self, j=0):
+        wq, sw = self.copies[j % len(self.copies)]
+        return self.fn(self.xq, self.sx, wq, sw, y=self.y, ws=self.ws)
+
+    def acc32(self):
+        return qgd.qgd_w8a8_int8_acc32(self.xq, self.copies[0][0], ws=self.ws)
+
+    def time_plan(self, reps=10) -> float:
+        n = len(self.copies)
+        self.ws.ensure(qgd.qgd_workspace_size(self.fid, self.M, self.N, self.K))
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for j in range(n):
+                self.run(j)
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for j in range(n):
+                self.run(j)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(reps):
+            g.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        del g
+        return t0.elapsed_time(t1) / (reps * n) * 1e3  # microseconds per call
+
+
+def tune_problem(p: Problem, log=None):
+    fid = p.fid
+    qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0)
+    p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
+    ref = p.run().float().clone()
+    ref_acc = p.acc32().clone() if p.fmt == W8A8_INT8 else None
+    scale = ref.abs().max().item() + 1e-30
+    results = []
+    for var, s, r, t in candidates(p.fmt, p.M, p.N, p.K):
+        qgd.qgd_set_override(fid, var, s, r, 0, t)
+        p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
+        y = p.run().float()
+        ok = (y - ref).abs().max().item() <= 2e-2 * scale
+        if ok and ref_acc is not None:
+            ok = torch.equal(p.acc32(), ref_acc)
+        if not ok:
+            if log:
+                log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t}: differs from the split-free result")
+            continue
+        us = p.time_plan()
+        stages = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["stages"]
+        results.append((us, var, s, r, stages, t))
+    results.sort()
+    # refine the pipeline depth of the three fastest
+    refined = list(results[:3])
+    for us0, var, s, r, smax, t in results[:3]:
+        for st in (3, 4, 6, 8, 10):
+            if st >= smax:
+                continue
+            qgd.qgd_set_override(fid, var, s, r, st, t)
+            us = p.time_plan()
+            refined.append((us, var, s, r, st, t))
+    refined.sort()
+    qgd.qgd_set_override(fid)
+    return refined[0], results
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--formats", default="fp8_dynamic,w8a8_int8,block_fp8")
+    ap.add_argument("--out", default=qgd.DEFAULT_TABLE)
+    ap.add_argument("--large-m", action="store_true", help="also tune the larger-M buckets")
+    ap.add_argument("--resume", action="store_true")
+    ap.add_argument("--only-m", default=None, help="comma-separated M values to tune")
+    args = ap.parse_args(argv)
+
+    os.environ["QGD_NO_TABLE"] = "1"
+    qgd.lib()
+    qgd.qgd_clear_dispatch_table()
+    device = torch.device("cuda")
+    fmts = args.formats.split(",")
+    wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE) if w.fmt in fmts]
+    if args.large_m:
+        wls += [w for w in workloads.LARGE if w.fmt in fmts]
+    done = {}
+    if args.resume and os.path.exists(args.out):
+        for ln in open(args.out):
+            f = ln.split("#")[0].split()
+            if len(f) == 9:
+                done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
+    only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
+    t_start = time.time()
+    lines = dict(done)
+
+    def log(msg):
+        print(msg, file=sys.stderr, flush=True)
+
+    def flush():
+        tmp = args.out + ".tmp"
+        with open(tmp, "w") as f:
+            f.write("# Dispatch table for B200 (sm_100a), measured by quantized_gemm_decode_b200.tune\n")
+            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n   # us/call\n")
+            for k in sorted(lines):
+                f.write(lines[k] + "\n")
+        os.replace(tmp, args.out)
+
+    for wl in wls:
+        for (N, K) in wl.shapes:
+            for M in wl.ms:
+                if only_m and M not in only_m:
+                    continue
+                key = (wl.fmt, N, K, M)
+                if key in done:
+                    continue
+                t0 = time.time()
+                p = Problem(wl.fmt, M, N, K, wl.seed, device)
+                best, allres = tune_problem(p, log)
+                us, var, s, r, st, t = best
+                gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
+                lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t}"
+                              f"   # {us:.2f} us, {gbs:.0f} GB/s")
+                log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
+                    f"{us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, {time.time() - t0:.1f} s)")
+                del p
+                torch.cuda.empty_cache()
+                flush()
+    flush()
+    log(f"tuning wall time: {time.time() - t_start:.1f} s")
+
+
+if __name__ == "__main__":
+    main()
