@@ -139,6 +139,26 @@ QGD_API qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void
 QGD_API qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
                                size_t ws_bytes, void* stream);
 
+/* FP8_Dynamic GEMM for callers that cannot allocate device memory -- for
+ * example a caller whose stream is being captured into a CUDA graph, or an
+ * engine that hands out all device memory from pools fixed at start-up, where
+ * a cudaMalloc would fail, stall the device or break the capture.  It is
+ * qlinear_fp8_dynamic without the workspace arguments: the caller still
+ * passes inputs and output, and the Split-K scratch comes from a fixed 8 MiB
+ * array inside the library (held by every GPU that loads it until exit).
+ * The pages have no counterpart; this is an addition of this library.
+ *   - The plan is the same as qlinear_fp8_dynamic's; a plan whose Split-K
+ *     scratch exceeds 8 MiB (64 KiB of counters + partials) is rejected with
+ *     QGD_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race and give undefined results.  Each call
+ *     clears the counters it uses with a memset node, then runs the GEMM.
+ *   - Nothing is allocated or freed. */
+QGD_API qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const void* wq, const float* sw,
+                                               void* y_bf16, int M, int N, int K, void* stream);
+
 /* Bytes of workspace the plan for (fmt, M, N, K) needs (0 when it needs
  * none).  Re-query after changing the override or the dispatch table. */
 QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);

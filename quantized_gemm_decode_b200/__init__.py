@@ -26,6 +26,7 @@ __all__ = [
     "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
+    "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
     "Workspace", "DEFAULT_TABLE",
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "qlinear_w8a8_int8": [P, P, P, P, P, I, I, I, P, S, P],
             "qlinear_block_fp8": [P, P, P, P, P, I, I, I, P, S, P],
             "qgd_w8a8_int8_acc32": [P, P, P, I, I, I, P, S, P],
+            "qlinear_fp8_dynamic_noalloc": [P, P, P, P, P, I, I, I, P],
             "qgd_load_dispatch_table": [ctypes.c_char_p],
             "qgd_clear_dispatch_table": [],
             "qgd_set_override": [I, I, I, I, I, I],
@@ -254,6 +256,18 @@ def qlinear_w8a8_int8(xq, sx, wq, sw, y=None, ws=None, stream=None):
 def qlinear_block_fp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
     """Y bf16 [M, N] with 1x128 activation and 128x128 weight block scales."""
     return _qlinear("qlinear_block_fp8", FMT_BLOCK_FP8, xq, sx, wq, sw, y, ws, stream)
+
+
+def qlinear_fp8_dynamic_noalloc(xq, sx, wq, sw, y, stream=None):
+    """FP8_Dynamic GEMM into a caller-provided y, with no workspace and no
+    allocation of any kind (the library's built-in scratch is used)."""
+    _cuda_2d(xq, "xq", _BYTE_TYPES)
+    _cuda_2d(wq, "wq", _BYTE_TYPES)
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check(lib().qlinear_fp8_dynamic_noalloc(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K,
+                                             _stream(stream)), "qlinear_fp8_dynamic_noalloc")
+    return y
 
 
 def qgd_w8a8_int8_acc32(xq, wq, acc=None, ws=None, stream=None):

@@ -306,6 +306,40 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   return QGD_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Built-in scratch for qlinear_fp8_dynamic_noalloc.  Some callers cannot
+// allocate device memory (their allocator is closed after start-up, or the
+// call is being captured into a CUDA graph); they get the Split-K workspace
+// from this fixed array instead.  Every GPU that loads the library holds it
+// until the process exits.  Its first 64 KiB are the arrival-counter header
+// (zero at load, left zero by every call, and cleared again at the start of
+// each call); the rest holds Split-K partials.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device.  In host code
+// `g_noalloc_scratch` names a host-side stand-in, never the device memory, so
+// the address is looked up once per device (with that device current).
+qgd_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(QGD_ERR_DEVICE, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (built-in Split-K scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return QGD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -371,6 +405,34 @@ qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int
                                size_t ws_bytes, void* stream) {
   if (M > 0 && !acc) return fail(QGD_ERR_INVALID, "null accumulator pointer");
   return run_gemm(kFmtINT8, xq, nullptr, wq, nullptr, nullptr, acc, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const void* wq, const float* sw,
+                                       void* y_bf16, int M, int N, int K, void* stream) {
+  qgd_status st = check_shape(kFmtFP8, M, N, K);
+  if (st != QGD_OK) return st;
+  if (M == 0) return QGD_OK;
+  const qgd_plan p = make_plan(kFmtFP8, M, N, K);
+  const WsLayout wl = ws_layout(p, M, N);
+  if (wl.total > kNoAllocScratchBytes)
+    return fail(QGD_ERR_WORKSPACE,
+                "qlinear_fp8_dynamic_noalloc: this plan (split_k=%d, M=%d, N=%d) needs %zu bytes of Split-K "
+                "scratch but the built-in scratch holds %zu; use qlinear_fp8_dynamic with a workspace or a "
+                "smaller split_k",
+                p.split_k, M, N, wl.total, kNoAllocScratchBytes);
+  if ((st = check_device()) != QGD_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != QGD_OK) return st;
+  if (wl.total > 0) {
+    // the counters this call uses must start at zero whatever an earlier
+    // (possibly interrupted) call left behind
+    const size_t tiles = p.variant == kSwapAB
+                             ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
+                             : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
+    cudaError_t e = cudaMemsetAsync(scratch, 0, tiles * 4, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (built-in scratch counters)");
+  }
+  return run_gemm(kFmtFP8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, scratch, kNoAllocScratchBytes, stream);
 }
 
 size_t qgd_workspace_size(int fmt, int M, int N, int K) {
