@@ -289,7 +289,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
         rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3),
                      "gbs": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / peak_gbs, 4),
                      "tflops": round(f / (ms * 1e-3) / 1e12, 2),
-                     "plan": f"{'swap' if p['variant'] == 1 else 'std'}/s{p['split_k']}/r{p['reduce']}/st{p['stages']}"})
+                     "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
+                              f"{'pers' if p['schedule'] == 1 else 's' + str(p['split_k'])}/r{p['reduce']}/st{p['stages']}")})
     return rows
 
 
@@ -450,6 +451,29 @@ def traffic_record():
     return rec, rec
 
 
+def run_case(args):
+    """One (format, M, N, K) GEMM: `warmup` + `steps` eager calls that cycle
+    through >= 3x L2 of weight copies, then a graph-replay timing."""
+    import quantized_gemm_decode_b200 as qgd
+    from quantized_gemm_decode_b200.tune import Problem
+
+    fmt, M, N, K = args.case.split(":")
+    M, N, K = int(M), int(N), int(K)
+    qgd.lib()
+    p = Problem(fmt, M, N, K, 1001, torch.device("cuda"))
+    p.ws.ensure(qgd.qgd_workspace_size(p.fid, M, N, K))
+    for i in range(args.warmup + args.steps):
+        p.run(i)
+    torch.cuda.synchronize()
+    us = p.time_plan()
+    b = workloads.algorithmic_bytes(fmt, M, N, K)
+    pk = peaks()
+    print(json.dumps({"case": args.case, "plan": qgd.qgd_get_plan(p.fid, M, N, K), "us": round(us, 3),
+                      "gbs": round(b / (us * 1e-6) / 1e9, 1), "frac": round(b / (us * 1e-6) / 1e9 / pk["hbm_gbs"], 4),
+                      "algorithmic_bytes": b}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -461,6 +485,8 @@ def main():
                                                          "other formats, large M or CPU baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out", default=None, help="also write the JSON line to this file")
+    ap.add_argument("--case", default=None, metavar="FMT:M:N:K",
+                    help="time one GEMM shape (eager launches, for profilers) instead of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -468,6 +494,8 @@ def main():
     dist = Dist()
     if args.impl == "reference":
         return run_reference(args, dist)
+    if args.case:
+        return run_case(args)
 
     torch.cuda.set_device(dist.local)
     device = torch.device("cuda", dist.local)

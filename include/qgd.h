@@ -74,14 +74,22 @@ typedef enum {
   QGD_REDUCE_ATOMIC = 2    /* split partials added atomically into a zeroed workspace (fp32 order varies) */
 } qgd_reduce;
 
+typedef enum {
+  QGD_SCHEDULE_AUTO = -1,
+  QGD_SCHEDULE_GRID = 0,      /* one CTA per (output tile, K split): split_k CTAs along K */
+  QGD_SCHEDULE_PERSISTENT = 1 /* Swap-AB only: one CTA per SM; all (tile, 128-wide K slice) units are dealt
+                                 out in equal contiguous ranges, shared tiles finished by the last CTA */
+} qgd_schedule;
+
 /* The execution plan for one (format, M, N, K). */
 typedef struct {
-  int variant; /* qgd_variant (never AUTO here) */
-  int split_k; /* CTAs along K: power of two, 1..256, at most ceil(K/128) */
-  int reduce;  /* qgd_reduce, meaningful when split_k > 1 */
-  int stages;  /* depth of the shared-memory operand ring */
-  int tile_n;  /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */
-  int source;  /* 0 = built-in default, 1 = dispatch table, 2 = override */
+  int variant;  /* qgd_variant (never AUTO here) */
+  int split_k;  /* grid schedule: CTAs along K, power of two, 1..256, at most ceil(K/128) */
+  int reduce;   /* qgd_reduce, used when several CTAs share an output tile */
+  int stages;   /* depth of the shared-memory operand ring */
+  int tile_n;   /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */
+  int schedule; /* qgd_schedule (never AUTO here) */
+  int source;   /* 0 = built-in default, 1 = dispatch table, 2 = override */
 } qgd_plan;
 
 /* ---------------------------------------------------------------------
@@ -167,11 +175,14 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
  * Dispatch (host only; no GPU needed).
  * ------------------------------------------------------------------- */
 
-/* Load a dispatch table (text; see the file format in the package's
- * tables/ directory): one line per (format, N, K, M-bucket) with the
- * variant, split_k, reduction, stages and tile_n measured best.  Replaces
- * the table in force.  On QGD_ERR_TABLE the table in force is unchanged.
- * Not thread-safe against concurrent qlinear_* calls. */
+/* Load a dispatch table: a text file with one line per (format, N, K,
+ * M-bucket) and '#' comments,
+ *     fmt N K M_bucket variant split_k reduce stages tile_n schedule
+ * fmt in {fp8_dynamic, w8a8_int8, block_fp8}; variant in {standard, swap_ab};
+ * reduce in {last_cta, two_pass, atomic}; schedule in {grid, persistent};
+ * stages/tile_n 0 = default.  Replaces the table in force.  On
+ * QGD_ERR_TABLE the table in force is unchanged.  Not thread-safe against
+ * concurrent qlinear_* calls. */
 QGD_API qgd_status qgd_load_dispatch_table(const char* path);
 
 /* Drop the table in force; the built-in defaults apply again. */
@@ -179,8 +190,9 @@ QGD_API qgd_status qgd_clear_dispatch_table(void);
 
 /* Force a plan for one format (tests and the tuner).  Any argument < 0 keeps
  * the table/default choice for that field; stages/tile_n 0 = default.
- * qgd_set_override(fmt, -1, -1, -1, 0, 0) removes the override. */
-QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n);
+ * qgd_set_override(fmt, -1, -1, -1, 0, 0, -1) removes the override. */
+QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n,
+                                    int schedule);
 
 /* The plan a qlinear_* call with these arguments would run. */
 QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);

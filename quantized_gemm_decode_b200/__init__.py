@@ -24,6 +24,7 @@ import torch
 __all__ = [
     "QGDError", "lib", "FMT_FP8_DYNAMIC", "FMT_W8A8_INT8", "FMT_BLOCK_FP8", "QTYPE_E4M3", "QTYPE_INT8",
     "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC",
+    "SCHEDULE_GRID", "SCHEDULE_PERSISTENT",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
     "qlinear_fp8_dynamic_noalloc",
@@ -40,6 +41,7 @@ FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8 = 0, 1, 2
 QTYPE_E4M3, QTYPE_INT8 = 0, 1
 VARIANT_STANDARD, VARIANT_SWAP_AB = 0, 1
 REDUCE_LAST_CTA, REDUCE_TWO_PASS, REDUCE_ATOMIC = 0, 1, 2
+SCHEDULE_GRID, SCHEDULE_PERSISTENT = 0, 1
 FORMAT_NAMES = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2}
 
 _lock = threading.Lock()
@@ -54,7 +56,8 @@ class QGDError(RuntimeError):
 
 class _Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
-                ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("source", ctypes.c_int)]
+                ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("schedule", ctypes.c_int),
+                ("source", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -78,7 +81,7 @@ def lib() -> ctypes.CDLL:
             "qlinear_fp8_dynamic_noalloc": [P, P, P, P, P, I, I, I, P],
             "qgd_load_dispatch_table": [ctypes.c_char_p],
             "qgd_clear_dispatch_table": [],
-            "qgd_set_override": [I, I, I, I, I, I],
+            "qgd_set_override": [I, I, I, I, I, I, I],
             "qgd_get_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
             "qgd_device_error": [ctypes.POINTER(ctypes.c_uint)],
             "qgd_clear_device_error": [],
@@ -300,8 +303,10 @@ def qgd_clear_dispatch_table() -> None:
 
 
 def qgd_set_override(fmt: int, variant: int = -1, split_k: int = -1, reduce: int = -1, stages: int = 0,
-                     tile_n: int = 0) -> None:
-    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n), "qgd_set_override")
+                     tile_n: int = 0, schedule: int = -1) -> None:
+    """Force plan fields for one format; every default argument leaves that
+    field to the dispatch table / built-in default."""
+    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n, schedule), "qgd_set_override")
 
 
 def qgd_get_plan(fmt: int, M: int, N: int, K: int) -> dict:

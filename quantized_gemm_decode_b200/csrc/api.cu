@@ -111,13 +111,13 @@ constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
 
 struct Entry {
-  int variant, split_k, reduce, stages, tile_n;
+  int variant, split_k, reduce, stages, tile_n, schedule;
 };
 using Key = std::tuple<int, int, int, int>;
 std::mutex g_mu;
 std::map<Key, Entry> g_table;
 struct Override {
-  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0;
+  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1;
 } g_override[3];
 
 int bucket_of(int M) {
@@ -145,6 +145,12 @@ int variant_from_name(const std::string& s) {
   return -1;
 }
 
+int schedule_from_name(const std::string& s) {
+  if (s == "grid") return kGrid;
+  if (s == "persistent") return kPersistent;
+  return -1;
+}
+
 int reduce_from_name(const std::string& s) {
   if (s == "last_cta") return kLastCta;
   if (s == "two_pass") return kTwoPass;
@@ -158,15 +164,18 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   p.source = 0;
   p.reduce = kLastCta;
   p.stages = 0;
+  p.schedule = kGrid;
   if (M <= kDecodeMaxM) {
-    // Swap-AB by default for small M (the hand-written rule the method
-    // replaces with measurement), split until the grid covers the SMs.
+    // Decode: Swap-AB (the hand-written rule the method replaces with
+    // measurement), persistent over all (tile, K-slice) units so that every
+    // SM streams the same share of the weights.
     p.variant = kSwapAB;
     p.tile_n = kSwapTileN;
+    p.schedule = kPersistent;
     const int tiles = (N + kSwapTileN - 1) / kSwapTileN;
     int s = 1;
     while (tiles * s < g_num_sms && s * 2 <= nkt && s < 256) s *= 2;
-    p.split_k = s;
+    p.split_k = s;  // used by the grid schedule
   } else {
     p.variant = kStandard;
     p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
@@ -182,15 +191,17 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       p.reduce = e.reduce;
       p.stages = e.stages;
       p.tile_n = e.tile_n;
+      p.schedule = e.schedule;
       p.source = 1;
     }
     const Override& o = g_override[fmt];
-    if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0) {
+    if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0 || o.schedule >= 0) {
       if (o.variant >= 0) p.variant = o.variant;
       if (o.split_k >= 0) p.split_k = o.split_k;
       if (o.reduce >= 0) p.reduce = o.reduce;
       if (o.stages > 0) p.stages = o.stages;
       if (o.tile_n > 0) p.tile_n = o.tile_n;
+      if (o.schedule >= 0) p.schedule = o.schedule;
       p.source = 2;
     }
   }
@@ -198,13 +209,14 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.variant == kSwapAB && M > kDecodeMaxM) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+  if (p.variant != kSwapAB || p.schedule != kPersistent) p.schedule = kGrid;
   int smax = nkt < 256 ? nkt : 256;
   if (smax < 1) smax = 1;
   if (p.split_k < 1) p.split_k = 1;
   if (p.split_k > smax) p.split_k = smax;
   p.split_k = floor_pow2(p.split_k);
   if (p.reduce < kLastCta || p.reduce > kAtomic) p.reduce = kLastCta;
-  if (p.split_k > 1 && p.reduce != kTwoPass) {
+  if (p.reduce != kTwoPass) {
     const size_t tiles = p.variant == kSwapAB
                              ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
                              : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
@@ -217,19 +229,70 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   return p;
 }
 
-struct WsLayout {
-  size_t data_off, data_bytes, total;
-};
-
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-WsLayout ws_layout(const qgd_plan& p, int M, int N) {
-  WsLayout w{0, 0, 0};
-  if (p.split_k <= 1 || M == 0) return w;
-  w.data_off = kTicketBytes;
-  w.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
-  w.total = w.data_off + w.data_bytes;
-  return w;
+long long sk_owner(long long u, long long G, long long U) { return ((u + 1) * G - 1) / U; }
+
+// Everything a launch derives from the plan and the shape: the persistent
+// schedule's CTA count, the partial-slot geometry and the workspace layout.
+struct Exec {
+  bool persistent = false;
+  int ctas = 0;     // persistent schedule: CTAs launched
+  int maxc = 1;     // most CTAs sharing one output tile
+  int mpad = 16;    // Swap-AB: token columns per MMA (16 or 32)
+  int mstride = 4;  // Swap-AB: partial row stride in words
+  size_t tiles = 0;  // output tiles (arrival counters)
+  size_t data_off = 0, data_bytes = 0, total = 0;
+};
+
+Exec make_exec(const qgd_plan& p, int M, int N, int K) {
+  Exec e;
+  const int nkt = (K + kTileK - 1) / kTileK;
+  e.mpad = M <= 16 ? 16 : 32;
+  e.mstride = (M + 3) / 4 * 4;
+  if (M <= 0) return e;
+  if (p.variant == kSwapAB) {
+    const int n_tiles = (N + kSwapTileN - 1) / kSwapTileN;
+    e.tiles = n_tiles;
+    if (p.schedule == kPersistent) {
+      const long long U = static_cast<long long>(n_tiles) * nkt;
+      int occ = static_cast<int>(kSmemPerSM / (swapab_smem_bytes(e.mpad, p.stages) + 1024));
+      occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);  // registers allow at most 2 CTAs per SM
+      const long long cap = static_cast<long long>(g_num_sms) * occ;
+      const long long G = U < cap ? U : cap;
+      e.persistent = true;
+      e.ctas = static_cast<int>(G);
+      int maxc = 1;
+      for (int t = 0; t < n_tiles; ++t) {
+        const long long c = sk_owner(static_cast<long long>(t) * nkt + nkt - 1, G, U) -
+                            sk_owner(static_cast<long long>(t) * nkt, G, U) + 1;
+        if (c > maxc) maxc = static_cast<int>(c);
+      }
+      e.maxc = maxc;
+    } else {
+      e.maxc = p.split_k;
+    }
+    if (e.maxc > 1)
+      e.data_bytes = p.reduce == kAtomic
+                         ? align256(static_cast<size_t>(M) * N * 4)
+                         : align256(static_cast<size_t>(n_tiles) * e.maxc * kSwapTileN * e.mstride * 4);
+  } else {
+    e.maxc = p.split_k;
+    e.tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
+    if (p.split_k > 1)
+      e.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
+  }
+  if (e.data_bytes) {
+    e.data_off = kTicketBytes;
+    e.total = e.data_off + e.data_bytes;
+  }
+  return e;
+}
+
+// Programmatic dependent launch is on unless QGD_PDL=0.
+bool pdl_enabled() {
+  const char* v = getenv("QGD_PDL");
+  return !(v && v[0] == '0');
 }
 
 qgd_status check_shape(int fmt, int M, int N, int K) {
@@ -255,10 +318,10 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   if ((st = get_encoder()) != QGD_OK) return st;
 
   const qgd_plan p = make_plan(fmt, M, N, K);
-  const WsLayout wl = ws_layout(p, M, N);
-  if (wl.total > 0 && (!ws || ws_bytes < wl.total))
-    return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", wl.total, ws ? ws_bytes : 0);
-  if (wl.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
+  const Exec ex = make_exec(p, M, N, K);
+  if (ex.total > 0 && (!ws || ws_bytes < ex.total))
+    return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", ex.total, ws ? ws_bytes : 0);
+  if (ex.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
 
   GemmArgs a;
   a.sx = sx;
@@ -268,11 +331,11 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.partial = nullptr;
   a.accum = nullptr;
   a.tickets = nullptr;
-  if (wl.total > 0) {
+  if (ex.total > 0) {
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     a.tickets = reinterpret_cast<unsigned int*>(wsb);
-    if (p.reduce == kAtomic) a.accum = wsb + wl.data_off;
-    else a.partial = wsb + wl.data_off;
+    if (p.reduce == kAtomic) a.accum = wsb + ex.data_off;
+    else a.partial = wsb + ex.data_off;
   }
   a.M = M;
   a.N = N;
@@ -280,6 +343,11 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.splits = p.split_k;
   a.reduce = p.reduce;
   a.stages = p.stages;
+  a.persistent = ex.persistent ? 1 : 0;
+  a.ctas = ex.ctas;
+  a.maxc = ex.maxc;
+  a.mstride = ex.mstride;
+  a.pdl = pdl_enabled() ? 1 : 0;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
@@ -287,20 +355,21 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   if (a.accum) {
     e = cudaMemsetAsync(a.accum, 0, static_cast<size_t>(M) * N * 4, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (atomic Split-K accumulator)");
+    a.pdl = 0;  // the GEMM follows a memset, not a kernel
   }
   if (p.variant == kSwapAB) {
-    const int mpad = M <= 16 ? 16 : 32;
     if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;
-    if ((st = encode_kmajor(&tx, xq, M, K, mpad)) != QGD_OK) return st;
-    e = launch_swapab(fmt, mpad, tw, tx, a, s);
+    if ((st = encode_kmajor(&tx, xq, M, K, ex.mpad)) != QGD_OK) return st;
+    e = launch_swapab(fmt, ex.mpad, tw, tx, a, s);
   } else {
     if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
     if ((st = encode_kmajor(&tw, wq, N, K, p.tile_n)) != QGD_OK) return st;
     e = launch_standard(fmt, p.tile_n, tx, tw, a, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
-  if (p.split_k > 1 && p.reduce == kTwoPass) {
-    e = launch_splitk_reduce(fmt, a, s);
+  if (ex.maxc > 1 && p.reduce == kTwoPass) {
+    a.pdl = pdl_enabled() ? 1 : 0;
+    e = p.variant == kSwapAB ? launch_swapab_reduce(fmt, ex.mpad, a, s) : launch_splitk_reduce(fmt, a, s);
     if (e != cudaSuccess) return cuda_fail(e, "Split-K reduce launch");
   }
   return QGD_OK;
@@ -413,23 +482,20 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
   if (st != QGD_OK) return st;
   if (M == 0) return QGD_OK;
   const qgd_plan p = make_plan(kFmtFP8, M, N, K);
-  const WsLayout wl = ws_layout(p, M, N);
-  if (wl.total > kNoAllocScratchBytes)
+  const Exec ex = make_exec(p, M, N, K);
+  if (ex.total > kNoAllocScratchBytes)
     return fail(QGD_ERR_WORKSPACE,
                 "qlinear_fp8_dynamic_noalloc: this plan (split_k=%d, M=%d, N=%d) needs %zu bytes of Split-K "
                 "scratch but the built-in scratch holds %zu; use qlinear_fp8_dynamic with a workspace or a "
                 "smaller split_k",
-                p.split_k, M, N, wl.total, kNoAllocScratchBytes);
+                p.split_k, M, N, ex.total, kNoAllocScratchBytes);
   if ((st = check_device()) != QGD_OK) return st;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != QGD_OK) return st;
-  if (wl.total > 0) {
+  if (ex.total > 0) {
     // the counters this call uses must start at zero whatever an earlier
     // (possibly interrupted) call left behind
-    const size_t tiles = p.variant == kSwapAB
-                             ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
-                             : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
-    cudaError_t e = cudaMemsetAsync(scratch, 0, tiles * 4, static_cast<cudaStream_t>(stream));
+    cudaError_t e = cudaMemsetAsync(scratch, 0, ex.tiles * 4, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (built-in scratch counters)");
   }
   return run_gemm(kFmtFP8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, scratch, kNoAllocScratchBytes, stream);
@@ -437,7 +503,7 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
 
 size_t qgd_workspace_size(int fmt, int M, int N, int K) {
   if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
-  return ws_layout(make_plan(fmt, M, N, K), M, N).total;
+  return make_exec(make_plan(fmt, M, N, K), M, N, K).total;
 }
 
 qgd_status qgd_load_dispatch_table(const char* path) {
@@ -452,24 +518,26 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     const size_t hash = line.find('#');
     if (hash != std::string::npos) line.resize(hash);
     std::istringstream ls(line);
-    std::string fmt_s, var_s, red_s;
+    std::string fmt_s, var_s, red_s, sch_s;
     int N, K, Mb, split, stages, tile_n;
     if (!(ls >> fmt_s)) continue;  // blank line
-    if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n))
-      return fail(QGD_ERR_TABLE, "%s:%d: expected 9 fields: fmt N K M_bucket variant split_k reduce stages tile_n",
+    if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s))
+      return fail(QGD_ERR_TABLE,
+                  "%s:%d: expected 10 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule",
                   path, lineno);
     std::string extra;
     if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
     const int fmt = fmt_from_name(fmt_s), var = variant_from_name(var_s), red = reduce_from_name(red_s);
-    if (fmt < 0 || var < 0 || red < 0)
-      return fail(QGD_ERR_TABLE, "%s:%d: unknown format/variant/reduce name", path, lineno);
+    const int sch = schedule_from_name(sch_s);
+    if (fmt < 0 || var < 0 || red < 0 || sch < 0)
+      return fail(QGD_ERR_TABLE, "%s:%d: unknown format/variant/reduce/schedule name", path, lineno);
     if (N <= 0 || K <= 0 || bucket_of(Mb) != Mb)
       return fail(QGD_ERR_TABLE, "%s:%d: bad N/K or M bucket %d", path, lineno, Mb);
     if (split < 1 || split > 256 || (split & (split - 1)) != 0)
       return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256", path, lineno, split);
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256))
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n", path, lineno);
-    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n};
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch};
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_table.swap(t);
@@ -482,9 +550,9 @@ qgd_status qgd_clear_dispatch_table(void) {
   return QGD_OK;
 }
 
-qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n) {
+qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule) {
   if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
-  if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 ||
+  if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");
   if (split_k > 0 && (split_k & (split_k - 1)) != 0) return fail(QGD_ERR_INVALID, "split_k must be a power of two");
@@ -495,6 +563,7 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
   o.reduce = reduce < 0 ? -1 : reduce;
   o.stages = stages;
   o.tile_n = tile_n;
+  o.schedule = schedule < 0 ? -1 : schedule;
   return QGD_OK;
 }
 

@@ -23,6 +23,8 @@
 // TMEM and exits.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "qgd_internal.h"
 #include "sm100.cuh"
 
@@ -161,12 +163,12 @@ __device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl) {
 
 // Split-K arrival: returns true in every epilogue thread of the last CTA to
 // arrive at tile `tile`.  Called after this CTA's partials are written.
-__device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile) {
+__device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile, int expected) {
   __threadfence();
   epi_sync();
   if (threadIdx.x == 64) {
     const unsigned int old = atomicAdd(a.tickets + tile, 1u);
-    ctl->last_flag = (old == static_cast<unsigned int>(a.splits - 1));
+    ctl->last_flag = (old == static_cast<unsigned int>(expected - 1));
   }
   epi_sync();
   const bool last = ctl->last_flag != 0;
@@ -175,15 +177,54 @@ __device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a,
 }
 
 // ===========================================================================
-// Swap-AB kernel (decode): grid = (ceil(N/128), splits)
+// Swap-AB kernel (decode, M <= 32).
+//
+// Work is the linear sequence of units u = tile * nkt + kt (tile = 128 weight
+// rows, kt = one 128-wide K slice).  Every CTA takes a contiguous range of
+// units; the range breaks into segments, one per tile it touches.
+//   grid schedule       grid (n_tiles, split_k): CTA (t, s) owns the s-th of
+//                       split_k near-equal K ranges of tile t (Split-K).
+//   persistent schedule grid (G): CTA c owns units [c*U/G, (c+1)*U/G) of all
+//                       U units, so every SM streams the same number of
+//                       weight bytes (the Split-K partition chosen per CTA).
+// A tile whose units all belong to one CTA is written straight to Y; a tile
+// shared by several CTAs is finished by the last of them to arrive, which
+// adds the partials in contributor order (deterministic), or the partials
+// are added atomically, or by a second kernel.
 // ===========================================================================
+__device__ __forceinline__ int sk_owner(long long u, long long G, long long U) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+
+// Contributors to tile t and this CTA's index among them.
+__device__ __forceinline__ void tile_contributors(const GemmArgs& a, int t, int nkt, long long U, int cta,
+                                                  int& ncontrib, int& j) {
+  if (a.persistent) {
+    const int first = sk_owner(static_cast<long long>(t) * nkt, a.ctas, U);
+    const int last = sk_owner(static_cast<long long>(t) * nkt + nkt - 1, a.ctas, U);
+    ncontrib = last - first + 1;
+    j = cta - first;
+  } else {
+    ncontrib = a.splits;
+    j = cta;
+  }
+}
+
+template <int kMpad>
+__device__ __forceinline__ uint32_t* swap_slot(const GemmArgs& a, int t, int j, int row) {
+  return static_cast<uint32_t*>(a.partial) +
+         ((static_cast<size_t>(t) * a.maxc + j) * kSwapTileN + row) * static_cast<size_t>(a.mstride);
+}
+
 template <int kFmt, int kMpad>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     swapab_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx,
                   const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
-  constexpr int kSlots = kBlock ? 4 : 1;
+  // Block_FP8: a ring of per-K-block accumulators; otherwise one accumulator
+  // per segment, double-buffered so the next segment's MMAs overlap the drain.
+  constexpr int kSlots = kBlock ? 4 : 2;
   constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : 128);
   constexpr uint32_t kWBytes = kSwapTileN * kTileK;
   constexpr uint32_t kXBytes = kMpad * kTileK;
@@ -197,11 +238,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * kXBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, split = blockIdx.y;
   const int nkt = (a.K + kTileK - 1) / kTileK;
-  const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / a.splits);
-  const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / a.splits);
-  const int nk = kt1 - kt0;
+  const int n_tiles = (a.N + kSwapTileN - 1) / kSwapTileN;
+  const long long U = static_cast<long long>(n_tiles) * nkt;
+  long long ub, ue;
+  int cta;  // index among the contributors' numbering (persistent: CTA id; grid: split id)
+  if (a.persistent) {
+    cta = blockIdx.x;
+    ub = static_cast<long long>(blockIdx.x) * U / gridDim.x;
+    ue = static_cast<long long>(blockIdx.x + 1) * U / gridDim.x;
+  } else {
+    cta = blockIdx.y;
+    const long long t0 = static_cast<long long>(blockIdx.x) * nkt;
+    ub = t0 + static_cast<long long>(blockIdx.y) * nkt / a.splits;
+    ue = t0 + static_cast<long long>(blockIdx.y + 1) * nkt / a.splits;
+  }
+  const int nk = static_cast<int>(ue - ub);
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tw);
@@ -228,6 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();
   const uint32_t tmem = ctl->tmem_base;
   int issued = 0;
 
@@ -236,7 +289,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      for (int i = 0; i < nk; ++i) {
+      // Weights do not depend on the preceding kernel: start streaming them
+      // before waiting for it, then fetch the activations.
+      const int pre = nk < stages ? nk : stages;
+      for (int i = 0; i < pre; ++i) {
+        const long long u = ub + i;
+        mbar_arrive_expect_tx(&ctl->full[i], kWBytes + kXBytes);
+        tma_load_2d(w_ring + i * kWBytes, &tw, &ctl->full[i], static_cast<int>(u % nkt) * kTileK,
+                    static_cast<int>(u / nkt) * kSwapTileN, pol_w);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i)
+        tma_load_2d(x_ring + i * kXBytes, &tx, &ctl->full[i], static_cast<int>((ub + i) % nkt) * kTileK, 0, pol_x);
+      issued = pre;
+      for (int i = pre; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
         if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
@@ -245,9 +311,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
+        const long long u = ub + i;
+        const int kx = static_cast<int>(u % nkt) * kTileK;
         mbar_arrive_expect_tx(&ctl->full[s], kWBytes + kXBytes);
-        const int kx = (kt0 + i) * kTileK;
-        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, n_tile * kSwapTileN, pol_w);
+        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, static_cast<int>(u / nkt) * kSwapTileN, pol_w);
         tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kx, 0, pol_x);
         issued = i + 1;
       }
@@ -256,6 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t w_base = smem_u32(w_ring), x_base = smem_u32(x_ring);
+      int seg = 0;
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
@@ -264,86 +332,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ctl->abort_flag = 1;
           break;
         }
-        uint32_t d = tmem;
+        const int kt = static_cast<int>((ub + i) % nkt);
+        const bool seg_start = (i == 0) || (kt == 0);
+        const bool seg_end = (i == nk - 1) || (kt == nkt - 1);
+        int slot;
+        uint32_t slot_round;
         if constexpr (kBlock) {
-          const int slot = i % kSlots;
-          if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
+          slot = i % kSlots;
+          slot_round = i / kSlots;
+        } else {
+          slot = seg & 1;
+          slot_round = seg >> 1;
+        }
+        if (kBlock || seg_start) {
+          if (!mbar_wait(&ctl->tempty[slot], (slot_round & 1) ^ 1)) {
             record_error(kErrWaitMma);
             ctl->abort_flag = 1;
             break;
           }
-          d = tmem + slot * kMpad;
         }
         if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
         tc_fence_after();
+        const uint32_t d = tmem + slot * kMpad;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 32; ++kk) {
           const uint64_t ad = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
           const uint64_t bd = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
-          const uint32_t accumulate = kBlock ? (kk > 0) : (i > 0 || kk > 0);
+          const uint32_t accumulate = kBlock ? (kk > 0) : !(seg_start && kk == 0);
           mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
         }
         mma_commit(&ctl->empty[s]);
-        if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
+        if (kBlock || seg_end) mma_commit(&ctl->tfull[slot]);
+        if (seg_end) ++seg;
       }
-      if constexpr (!kBlock) mma_commit(&ctl->accfull);
     }
     __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
+    griddep_wait();  // scales and outputs: only after the preceding kernel is done
     const int q = warp & 3;
     const int row = q * 32 + lane;  // TMEM lane = weight row inside the tile
-    const int n = n_tile * kSwapTileN + row;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int M = a.M, N = a.N;
-    uint32_t acc[kMpad];
-
-    if constexpr (kBlock) {
-      const int KB = a.K / kTileK;
-      float facc[kMpad];
+    const int KB = a.K / kTileK;
+    const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
+    int i = 0, seg = 0;
+    while (i < nk) {
+      const long long u = ub + i;
+      const int t = static_cast<int>(u / nkt);
+      const int kt_first = static_cast<int>(u % nkt);
+      const int len = (nkt - kt_first) < (nk - i) ? (nkt - kt_first) : (nk - i);
+      const int n = t * kSwapTileN + row;
+      uint32_t acc[kMpad];
+      if constexpr (kBlock) {
+        float facc[kMpad];
 #pragma unroll
-      for (int m = 0; m < kMpad; ++m) facc[m] = 0.f;
-      const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;  // weight block row = this tile
-      for (int i = 0; i < nk; ++i) {
-        const int slot = i % kSlots;
-        if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
+        for (int m = 0; m < kMpad; ++m) facc[m] = 0.f;
+                for (int jj = 0; jj < len; ++jj) {
+          const int ii = i + jj;
+          const int slot = ii % kSlots;
+          if (!warp_wait(&ctl->tfull[slot], (ii / kSlots) & 1)) {
+            if (lane == 0) {
+              record_error(kErrWaitEpilogue);
+              ctl->abort_flag = 1;
+            }
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[kMpad];
+          tmem_load_cols<kMpad>(taddr + slot * kMpad, r);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&ctl->tempty[slot]);
+          const int kb = kt_first + jj;
+          const float swv = __ldg(a.sw + static_cast<size_t>(t) * KB + kb);  // one weight block per tile
+#pragma unroll
+          for (int m = 0; m < kMpad; ++m) {
+            if (m < M)
+              facc[m] = fmaf(__uint_as_float(r[m]), __ldg(a.sx + static_cast<size_t>(m) * KB + kb) * swv, facc[m]);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < kMpad; ++m) acc[m] = __float_as_uint(facc[m]);
+      } else {
+        const int slot = seg & 1;
+        if (!warp_wait(&ctl->tfull[slot], (seg >> 1) & 1)) {
           if (lane == 0) {
             record_error(kErrWaitEpilogue);
             ctl->abort_flag = 1;
           }
-          break;
-        }
-        tc_fence_after();
-        uint32_t r[kMpad];
-        tmem_load_cols<kMpad>(taddr + slot * kMpad, r);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&ctl->tempty[slot]);
-        const int kb = kt0 + i;
-        const float swv = __ldg(swrow + kb);
-#pragma unroll
-        for (int m = 0; m < kMpad; ++m) {
-          if (m < M) facc[m] = fmaf(__uint_as_float(r[m]), __ldg(a.sx + static_cast<size_t>(m) * KB + kb) * swv, facc[m]);
+        } else {
+          tc_fence_after();
+          tmem_load_cols<kMpad>(taddr + slot * kMpad, acc);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&ctl->tempty[slot]);
         }
       }
-#pragma unroll
-      for (int m = 0; m < kMpad; ++m) acc[m] = __float_as_uint(facc[m]);
-    } else {
-      if (!warp_wait(&ctl->accfull, 0)) {
-        if (lane == 0) {
-          record_error(kErrWaitEpilogue);
-          ctl->abort_flag = 1;
-        }
-      } else {
-        tc_fence_after();
-        tmem_load_cols<kMpad>(taddr, acc);
-        tmem_wait_ld();
-      }
-    }
+      if (!epi_agree_ok(ctl)) break;
 
-    if (epi_agree_ok(ctl)) {
       const bool in_n = n < N;
-      if (a.splits == 1) {
+      int ncontrib, jslot;
+      tile_contributors(a, t, nkt, U, cta, ncontrib, jslot);
+      if (ncontrib == 1) {
         if (in_n) {
 #pragma unroll
           for (int m = 0; m < kMpad; ++m)
@@ -351,39 +442,98 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else {
         if (in_n) {
+          if (a.reduce == kAtomic) {
 #pragma unroll
-          for (int m = 0; m < kMpad; ++m) {
-            if (m < M) {
-              if (a.reduce == kAtomic)
-                atomic_acc<kFmt>(a.accum, static_cast<size_t>(m) * N + n, acc[m]);
-              else
-                static_cast<uint32_t*>(a.partial)[(static_cast<size_t>(split) * M + m) * N + n] = acc[m];
-            }
+            for (int m = 0; m < kMpad; ++m)
+              if (m < M) atomic_acc<kFmt>(a.accum, static_cast<size_t>(m) * N + n, acc[m]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(swap_slot<kMpad>(a, t, jslot, row));
+#pragma unroll
+            for (int v = 0; v < kMpad / 4; ++v)
+              if (v < nvec) dst[v] = make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
           }
         }
-        if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, n_tile)) {
+        if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, t, ncontrib)) {
           if (in_n) {
-            for (int m = 0; m < M && m < kMpad; ++m) {
-              const size_t idx = static_cast<size_t>(m) * N + n;
-              uint32_t v;
-              if (a.reduce == kAtomic) {
-                v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-              } else {
-                v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
-                for (int s = 1; s < a.splits; ++s)
-                  v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
-                                                 (static_cast<size_t>(s) * M) * N + idx));
+            if (a.reduce == kAtomic) {
+#pragma unroll
+              for (int m = 0; m < kMpad; ++m)
+                if (m < M) store_final<kFmt>(ldcg_u32(static_cast<uint32_t*>(a.accum) + static_cast<size_t>(m) * N + n), m, n, a);
+            } else {
+              uint32_t sum[kMpad];
+              const uint4* src0 = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, 0, row));
+#pragma unroll
+              for (int v = 0; v < kMpad / 4; ++v) {
+                if (v < nvec) {
+                  const uint4 w4 = __ldcg(src0 + v);
+                  sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+                }
               }
-              store_final<kFmt>(v, m, n, a);
+              for (int jj = 1; jj < ncontrib; ++jj) {
+                const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, jj, row));
+#pragma unroll
+                for (int v = 0; v < kMpad / 4; ++v) {
+                  if (v < nvec) {
+                    const uint4 w4 = __ldcg(src + v);
+                    sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+                    sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+                    sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+                    sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+                  }
+                }
+              }
+#pragma unroll
+              for (int m = 0; m < kMpad; ++m)
+                if (m < M) store_final<kFmt>(sum[m], m, n, a);
             }
           }
-          if (threadIdx.x == 64) a.tickets[n_tile] = 0u;
+          if (threadIdx.x == 64) a.tickets[t] = 0u;
         }
       }
+      i += len;
+      ++seg;
     }
   }
 
   teardown(ctl, warp, lane, issued, stages, tmem, kCols);
+}
+
+// Two-pass reduction for the Swap-AB layout: one CTA per tile, one thread per
+// weight row; contributors' partials added in contributor order.
+template <int kFmt, int kMpad>
+__global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArgs a) {
+  griddep_wait();
+  const int t = blockIdx.x, row = threadIdx.x;
+  const int nkt = (a.K + kTileK - 1) / kTileK;
+  const long long U = static_cast<long long>((a.N + kSwapTileN - 1) / kSwapTileN) * nkt;
+  int ncontrib = a.splits, j0;
+  if (a.persistent) tile_contributors(a, t, nkt, U, 0, ncontrib, j0);
+  const int n = t * kSwapTileN + row;
+  if (ncontrib == 1 || n >= a.N) return;  // written directly by its only contributor
+  const int M = a.M, nvec = (M + 3) / 4;
+  uint32_t sum[kMpad];
+#pragma unroll
+  for (int m = 0; m < kMpad; ++m) sum[m] = 0u;
+  for (int jj = 0; jj < ncontrib; ++jj) {
+    const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, jj, row));
+#pragma unroll
+    for (int v = 0; v < kMpad / 4; ++v) {
+      if (v < nvec) {
+        const uint4 w4 = src[v];
+        if (jj == 0) {
+          sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+        } else {
+          sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+          sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+          sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+          sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kMpad; ++m)
+    if (m < M) store_final<kFmt>(sum[m], m, n, a);
 }
 
 // ===========================================================================
@@ -441,6 +591,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();
   const uint32_t tmem = ctl->tmem_base;
   int issued = 0;
 
@@ -448,6 +599,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_x = policy_evict_last();
       const uint64_t pol_w = policy_evict_last();
+      griddep_wait();  // activations come from the preceding kernel
       for (int i = 0; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
@@ -501,6 +653,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else {
+    griddep_wait();  // scales and outputs: only after the preceding kernel is done
     const int q = warp & 3;
     const int m = m_tile * kStdTileM + q * 32 + lane;  // TMEM lane = token row
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -582,7 +735,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           if (a.reduce != kTwoPass) {
             const int tile = m_tile * gridDim.x + n_tile;
-            if (epi_arrive_last(ctl, a, tile)) {
+            if (epi_arrive_last(ctl, a, tile, a.splits)) {
               if (in_m) {
                 for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
                   const size_t idx = static_cast<size_t>(m) * N + nc;
@@ -677,7 +830,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           if (a.reduce != kTwoPass) {
             const int tile = m_tile * gridDim.x + n_tile;
-            if (epi_arrive_last(ctl, a, tile)) {
+            if (epi_arrive_last(ctl, a, tile, a.splits)) {
               if (in_m) {
                 for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
                   const size_t idx = static_cast<size_t>(m) * N + nc;
@@ -710,6 +863,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ===========================================================================
 template <int kFmt>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
+  griddep_wait();
   const size_t total = static_cast<size_t>(a.M) * a.N;
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= total) return;
@@ -720,17 +874,33 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
   store_final<kFmt>(v, m, n, a);
 }
 
-template <typename Kern>
-cudaError_t launch_kernel(Kern kernel, dim3 grid, size_t smem, cudaStream_t stream, bool& attr_done,
-                          const CUtensorMap& t0, const CUtensorMap& t1, const GemmArgs& a) {
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_budget()));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
-  kernel<<<grid, kGemmThreads, smem, stream>>>(t0, t1, a);
+// Launch with dynamic shared memory and, when `pdl` is set, a programmatic
+// dependency on the preceding kernel in the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_ex(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <typename Kern>
+cudaError_t set_smem_attr(Kern kernel, bool& done) {
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_budget()));
+  if (e == cudaSuccess) done = true;
+  return e;
 }
 
 }  // namespace
@@ -757,18 +927,23 @@ template <int kFmt, int kMpad>
 static cudaError_t launch_swapab_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                                    cudaStream_t stream) {
   static bool attr_done = false;
-  const dim3 grid((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
-  return launch_kernel(swapab_kernel<kFmt, kMpad>, grid, swapab_smem_bytes(kMpad, a.stages), stream, attr_done, tw,
-                       tx, a);
+  cudaError_t e = set_smem_attr(swapab_kernel<kFmt, kMpad>, attr_done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid = a.persistent ? dim3(a.ctas, 1, 1)
+                                 : dim3((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
+  return launch_ex(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads), swapab_smem_bytes(kMpad, a.stages),
+                   stream, a.pdl != 0, tw, tx, a);
 }
 
 template <int kFmt, int kTileN>
 static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                                      cudaStream_t stream) {
   static bool attr_done = false;
+  cudaError_t e = set_smem_attr(standard_kernel<kFmt, kTileN>, attr_done);
+  if (e != cudaSuccess) return e;
   const dim3 grid((a.N + kTileN - 1) / kTileN, (a.M + kStdTileM - 1) / kStdTileM, a.splits);
-  return launch_kernel(standard_kernel<kFmt, kTileN>, grid, standard_smem_bytes(kTileN, a.stages), stream,
-                       attr_done, tx, tw, a);
+  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(kGemmThreads), standard_smem_bytes(kTileN, a.stages),
+                   stream, a.pdl != 0, tx, tw, a);
 }
 
 cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
@@ -806,10 +981,25 @@ cudaError_t clear_device_error() {
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream) {
   const size_t total = static_cast<size_t>(a.M) * a.N;
   const unsigned blocks = static_cast<unsigned>((total + 255) / 256);
-  if (fmt == kFmtFP8) splitk_reduce_kernel<kFmtFP8><<<blocks, 256, 0, stream>>>(a);
-  else if (fmt == kFmtINT8) splitk_reduce_kernel<kFmtINT8><<<blocks, 256, 0, stream>>>(a);
-  else splitk_reduce_kernel<kFmtBlock><<<blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  const bool pdl = a.pdl != 0;
+  if (fmt == kFmtFP8) return launch_ex(splitk_reduce_kernel<kFmtFP8>, dim3(blocks), dim3(256), 0, stream, pdl, a);
+  if (fmt == kFmtINT8) return launch_ex(splitk_reduce_kernel<kFmtINT8>, dim3(blocks), dim3(256), 0, stream, pdl, a);
+  return launch_ex(splitk_reduce_kernel<kFmtBlock>, dim3(blocks), dim3(256), 0, stream, pdl, a);
+}
+
+cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream) {
+  const dim3 grid((a.N + kSwapTileN - 1) / kSwapTileN);
+  const dim3 block(kSwapTileN);
+  const bool pdl = a.pdl != 0;
+  switch (fmt * 2 + (mpad == 32 ? 1 : 0)) {
+    case 0: return launch_ex(swapab_reduce_kernel<kFmtFP8, 16>, grid, block, 0, stream, pdl, a);
+    case 1: return launch_ex(swapab_reduce_kernel<kFmtFP8, 32>, grid, block, 0, stream, pdl, a);
+    case 2: return launch_ex(swapab_reduce_kernel<kFmtINT8, 16>, grid, block, 0, stream, pdl, a);
+    case 3: return launch_ex(swapab_reduce_kernel<kFmtINT8, 32>, grid, block, 0, stream, pdl, a);
+    case 4: return launch_ex(swapab_reduce_kernel<kFmtBlock, 16>, grid, block, 0, stream, pdl, a);
+    case 5: return launch_ex(swapab_reduce_kernel<kFmtBlock, 32>, grid, block, 0, stream, pdl, a);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace qgd

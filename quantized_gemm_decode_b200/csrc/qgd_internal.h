@@ -11,6 +11,7 @@ namespace qgd {
 enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2 };
 enum Variant : int { kStandard = 0, kSwapAB = 1 };
 enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2 };
+enum Schedule : int { kGrid = 0, kPersistent = 1 };
 
 constexpr int kTileK = 128;           // K elements (= bytes) per pipeline stage
 constexpr int kSwapTileN = 128;       // weight rows per Swap-AB CTA (MMA M)
@@ -19,6 +20,8 @@ constexpr int kMaxStages = 16;
 constexpr int kGemmThreads = 192;     // producer warp, MMA warp, 4 epilogue warps
 // Opt-in dynamic shared memory per CTA on sm_100 (227 KB).
 constexpr size_t kSmemBudget = 232448;
+// Shared memory per SM on sm_100 (228 KB), shared by the CTAs resident on it.
+constexpr size_t kSmemPerSM = 233472;
 inline size_t smem_budget() { return kSmemBudget; }
 
 // Runtime arguments common to both GEMM orientations.
@@ -31,9 +34,14 @@ struct GemmArgs {
   void* accum;          // atomic Split-K accumulator, 4-byte [M][N], zero on entry
   unsigned int* tickets;  // per output tile arrival counters (workspace header), zero on entry and exit
   int M, N, K;
-  int splits;
+  int splits;      // grid schedule: CTAs along K per tile
   int reduce;
   int stages;
+  int persistent;  // Swap-AB: 1 = persistent schedule over all (tile, K-slice) units
+  int ctas;        // persistent schedule: number of CTAs
+  int maxc;        // Swap-AB partial slots per tile (largest contributor count)
+  int mstride;     // Swap-AB partial row stride in words (M rounded up to 4)
+  int pdl;         // launch with a programmatic dependency on the preceding kernel
 };
 
 // Launchers (gemm.cu).  Each returns the cudaError_t of the launch.
@@ -42,6 +50,7 @@ cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtens
 cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
+cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();
 size_t swapab_smem_bytes(int mpad, int stages);

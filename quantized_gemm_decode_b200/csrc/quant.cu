@@ -14,6 +14,9 @@
 // codes with 8-byte stores.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+#include <stdlib.h>
+
+#include <utility>
 
 #include "qgd_internal.h"
 
@@ -94,6 +97,8 @@ template <int kVPT, int kQType>
 __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int K,
                                                                  uint8_t* __restrict__ q, float* __restrict__ s) {
   __shared__ float red[33];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
   const size_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
   uint2* qr = reinterpret_cast<uint2*>(q + row * K);
@@ -123,6 +128,8 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t*
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                              uint8_t* __restrict__ q, float* __restrict__ s) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
   const int KB = K / 128;
   const long long g = static_cast<long long>(blockIdx.x) * 16 + (threadIdx.x >> 4);
   const int sub = threadIdx.x & 15;
@@ -149,6 +156,8 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __r
 __global__ void __launch_bounds__(256) quant_block128_kernel(const uint16_t* __restrict__ w, int K,
                                                              uint8_t* __restrict__ q, float* __restrict__ s) {
   __shared__ float red[33];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nb = blockIdx.y, kb = blockIdx.x, KB = gridDim.x;
   uint4 v[8];
   float amax = 0.f;
@@ -170,18 +179,38 @@ __global__ void __launch_bounds__(256) quant_block128_kernel(const uint16_t* __r
   }
 }
 
+// Launch with a programmatic dependency on the preceding kernel (unless
+// QGD_PDL=0): the kernel may start early and waits in griddepcontrol.wait.
+template <typename... Params, typename... Args>
+cudaError_t launch_q(void (*kernel)(Params...), dim3 grid, dim3 block, cudaStream_t stream, Args&&... args) {
+  const char* v = getenv("QGD_PDL");
+  const bool pdl = !(v && v[0] == '0');
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int kQType>
 cudaError_t launch_rows_q(const uint16_t* x, int rows, int K, void* q, float* s, cudaStream_t st) {
   const int nvec = K / 8;
   const int vpt = (nvec + kRowThreads - 1) / kRowThreads;
   uint8_t* qb = static_cast<uint8_t*>(q);
-  if (vpt <= 1) quant_rows_kernel<1, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
-  else if (vpt <= 2) quant_rows_kernel<2, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
-  else if (vpt <= 4) quant_rows_kernel<4, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
-  else if (vpt <= 8) quant_rows_kernel<8, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
-  else if (vpt <= 16) quant_rows_kernel<16, kQType><<<rows, kRowThreads, 0, st>>>(x, K, qb, s);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  const dim3 grid(rows), block(kRowThreads);
+  if (vpt <= 1) return launch_q(quant_rows_kernel<1, kQType>, grid, block, st, x, K, qb, s);
+  if (vpt <= 2) return launch_q(quant_rows_kernel<2, kQType>, grid, block, st, x, K, qb, s);
+  if (vpt <= 4) return launch_q(quant_rows_kernel<4, kQType>, grid, block, st, x, K, qb, s);
+  if (vpt <= 8) return launch_q(quant_rows_kernel<8, kQType>, grid, block, st, x, K, qb, s);
+  if (vpt <= 16) return launch_q(quant_rows_kernel<16, kQType>, grid, block, st, x, K, qb, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -194,14 +223,12 @@ cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, voi
 cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, uint8_t* q, float* s, cudaStream_t stream) {
   const long long groups = static_cast<long long>(M) * (K / 128);
   const unsigned blocks = static_cast<unsigned>((groups + 15) / 16);
-  quant_group128_kernel<<<blocks, 256, 0, stream>>>(x, M, K, q, s);
-  return cudaGetLastError();
+  return launch_q(quant_group128_kernel, dim3(blocks), dim3(256), stream, x, M, K, q, s);
 }
 
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream) {
   const dim3 grid(K / 128, N / 128);
-  quant_block128_kernel<<<grid, 256, 0, stream>>>(w, K, q, s);
-  return cudaGetLastError();
+  return launch_q(quant_block128_kernel, grid, dim3(256), stream, w, K, q, s);
 }
 
 }  // namespace qgd

@@ -67,15 +67,18 @@ def test_m_buckets(M, b):
 
 
 def test_default_plans():
-    # decode: Swap-AB, split until the 148 SMs are covered
+    # decode: Swap-AB on the persistent schedule (grid-schedule split until
+    # the 148 SMs are covered)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)
     assert p["variant"] == qgd.VARIANT_SWAP_AB and p["source"] == 0
+    assert p["schedule"] == qgd.SCHEDULE_PERSISTENT
     assert p["split_k"] == 8  # 32 tiles * 8 >= 148
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 32, 24576, 4096)
     assert p["split_k"] == 1  # 192 tiles already cover the SMs
     # large M: Standard, no split
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 512, 6144, 4096)
     assert p["variant"] == qgd.VARIANT_STANDARD and p["split_k"] == 1 and p["tile_n"] == 256
+    assert p["schedule"] == qgd.SCHEDULE_GRID
     p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 512, 6144, 4096)
     assert p["tile_n"] == 128
     # split never exceeds the number of 128-wide K tiles
@@ -84,12 +87,14 @@ def test_default_plans():
 
 
 def test_override_and_clamping():
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 256, qgd.REDUCE_ATOMIC, 5, 0)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 256, qgd.REDUCE_ATOMIC, 5, 0, qgd.SCHEDULE_GRID)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
     assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["source"]) == (1, 32, 2, 5, 2)
-    # Swap-AB cannot take more than 32 tokens: it falls back to Standard
+    # Swap-AB cannot take more than 32 tokens: it falls back to Standard, and
+    # the persistent schedule is Swap-AB only
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, qgd.SCHEDULE_PERSISTENT)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)
-    assert p["variant"] == qgd.VARIANT_STANDARD
+    assert p["variant"] == qgd.VARIANT_STANDARD and p["schedule"] == qgd.SCHEDULE_GRID
     with pytest.raises(qgd.QGDError):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 3, 0, 0, 0)  # split not a power of two
     with pytest.raises(qgd.QGDError):
@@ -98,52 +103,81 @@ def test_override_and_clamping():
 
 def test_workspace_size_follows_plan():
     hdr = 64 * 1024  # arrival-counter header
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 1, 0, 0, 0)
+    G = qgd.SCHEDULE_GRID
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 1, 0, 0, 0, G)
     assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 0
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0)
-    # header + 8 partials of 4 x 4096 fp32
-    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 8 * 4 * 4096 * 4
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_TWO_PASS, 0, 0)
-    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 8 * 4 * 4096 * 4
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_ATOMIC, 0, 0)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0, G)
+    # header + 32 tiles x 8 splits x 128 rows x 4 tokens of fp32
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 32 * 8 * 128 * 4 * 4
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_TWO_PASS, 0, 0, G)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 32 * 8 * 128 * 4 * 4
+    # 5 tokens: rows of partials are padded to 8 words (two 16-byte vectors)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 5, 4096, 4096) == hdr + 32 * 8 * 128 * 8 * 4
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_ATOMIC, 0, 0, G)
     assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == hdr + 4 * 4096 * 4
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 2, qgd.REDUCE_LAST_CTA, 0, 128, G)
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 40, 4096, 4096) == hdr + 2 * 40 * 4096 * 4
+
+
+def _persistent_geometry(N, K, ctas):
+    """Contributors per tile when ctas CTAs share the (tile, K-slice) units."""
+    nkt, tiles = (K + 127) // 128, (N + 127) // 128
+    U = tiles * nkt
+    G = min(U, ctas)
+    owner = lambda u: ((u + 1) * G - 1) // U  # noqa: E731
+    return max(owner(t * nkt + nkt - 1) - owner(t * nkt) + 1 for t in range(tiles)), tiles
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (32, 6144, 4096), (8, 24576, 4096), (3, 4096, 12288),
+                                   (1, 256, 256), (16, 51200, 5120)])
+def test_persistent_workspace_matches_unit_partition(M, N, K):
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, qgd.REDUCE_LAST_CTA, 0, 0,
+                         qgd.SCHEDULE_PERSISTENT)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, M, N, K)
+    assert p["schedule"] == qgd.SCHEDULE_PERSISTENT
+    # the deepest pipelines leave room for one CTA per SM (148 SMs)
+    maxc, tiles = _persistent_geometry(N, K, 148)
+    mstride = (M + 3) // 4 * 4
+    want = 0 if maxc == 1 else 64 * 1024 + ((tiles * maxc * 128 * mstride * 4 + 255) // 256) * 256
+    assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, M, N, K) == want
 
 
 def test_too_many_tiles_for_counters_fall_back_to_two_pass():
     # Standard tiles of 128 x 128 over 8192 x 262144 exceed the 16384 counters
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 2, qgd.REDUCE_LAST_CTA, 0, 128)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 2, qgd.REDUCE_LAST_CTA, 0, 128, 0)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 8192, 262144, 4096)
     assert p["reduce"] == qgd.REDUCE_TWO_PASS
 
 
 def test_table_load_and_lookup(tmp_path):
     t = tmp_path / "t.tsv"
-    t.write_text("# fmt N K M_bucket variant split_k reduce stages tile_n\n"
-                 "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n"
+    t.write_text("# fmt N K M_bucket variant split_k reduce stages tile_n schedule\n"
+                 "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n"
                  "\n"
-                 "w8a8_int8 5120 5120 32 swap_ab 4 atomic 0 0   # trailing comment\n")
+                 "w8a8_int8 5120 5120 32 swap_ab 4 atomic 0 0 persistent  # trailing comment\n")
     qgd.qgd_load_dispatch_table(str(t))
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 3, 4096, 4096)  # bucket 4
     assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["tile_n"], p["source"]) == (0, 2, 1, 4, 256, 1)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 5, 4096, 4096)  # bucket 8: not in the table
     assert p["source"] == 0
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)
-    assert (p["variant"], p["split_k"], p["reduce"], p["source"]) == (1, 4, 2, 1)
+    assert (p["variant"], p["split_k"], p["reduce"], p["schedule"], p["source"]) == (1, 4, 2, 1, 1)
     qgd.qgd_clear_dispatch_table()
     assert qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)["source"] == 0
 
 
 @pytest.mark.parametrize("bad", [
-    "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256\n",      # split not a power of two
-    "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256\n",      # 5 is not a bucket
-    "fp9 4096 4096 4 standard 2 two_pass 4 256\n",              # unknown format
-    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4\n",          # missing field
-    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 7\n",    # extra field
-    "fp8_dynamic 4096 4096 4 diagonal 2 two_pass 4 256\n",      # unknown variant
+    "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256 grid\n",      # split not a power of two
+    "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256 grid\n",      # 5 is not a bucket
+    "fp9 4096 4096 4 standard 2 two_pass 4 256 grid\n",              # unknown format
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n",           # missing field
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 7\n",    # extra field
+    "fp8_dynamic 4096 4096 4 diagonal 2 two_pass 4 256 grid\n",      # unknown variant
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 stream\n",    # unknown schedule
 ])
 def test_malformed_table_is_rejected_and_keeps_previous(tmp_path, bad):
     good = tmp_path / "good.tsv"
-    good.write_text("fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n")
+    good.write_text("fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n")
     qgd.qgd_load_dispatch_table(str(good))
     t = tmp_path / "bad.tsv"
     t.write_text(bad)

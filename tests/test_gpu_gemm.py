@@ -44,36 +44,40 @@ def test_tiny_fp8_dynamic_default_plan():
     case.check_output(case.run(), yref, bound, "tiny default")
 
 
+GRID, PERSISTENT = qgd.SCHEDULE_GRID, qgd.SCHEDULE_PERSISTENT
 VARIANTS = (
-    [(qgd.VARIANT_SWAP_AB, s, r, 0) for s in (1, 2, 4, 8) for r in (0, 1, 2)]
-    + [(qgd.VARIANT_STANDARD, s, r, t) for t in (128, 256) for s in (1, 2, 8) for r in (0, 1, 2)]
+    [(qgd.VARIANT_SWAP_AB, s, r, 0, GRID) for s in (1, 2, 4, 8) for r in (0, 1, 2)]
+    + [(qgd.VARIANT_SWAP_AB, 1, r, 0, PERSISTENT) for r in (0, 1, 2)]
+    + [(qgd.VARIANT_STANDARD, s, r, t, GRID) for t in (128, 256) for s in (1, 2, 8) for r in (0, 1, 2)]
 )
 
 
 def _vid(v):
-    return f"{'swap' if v[0] == qgd.VARIANT_SWAP_AB else 'std'}-s{v[1]}-r{v[2]}-t{v[3]}"
+    sched = "pers" if v[4] == PERSISTENT else f"s{v[1]}"
+    return f"{'swap' if v[0] == qgd.VARIANT_SWAP_AB else 'std'}-{sched}-r{v[2]}-t{v[3]}"
 
 
 @pytest.mark.parametrize("fmt", ALL_FMTS)
 @pytest.mark.parametrize("variant", VARIANTS, ids=_vid)
 def test_every_variant_tiny(fmt, variant):
-    var, split, red, tile = variant
+    var, split, red, tile, sched = variant
     if fmt == BLOCK_FP8 and tile == 256:
         pytest.skip("Block_FP8 Standard tiles are 128 wide")
     case = Case(fmt, 4, 512, 1024, seed=1, outliers=True)
     yref, bound = _oracle(case)[:2]
-    qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, tile)
+    qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, tile, sched)
     plan = qgd.qgd_get_plan(FMT_ID[fmt], 4, 512, 1024)
     assert plan["variant"] == var and plan["split_k"] == split and plan["source"] == 2
+    assert plan["schedule"] == sched
     case.check_output(case.run(), yref, bound, f"{fmt} {_vid(variant)}")
 
 
 @pytest.mark.parametrize("variant", VARIANTS, ids=_vid)
 def test_int8_acc32_bit_exact_every_variant(variant):
-    var, split, red, tile = variant
+    var, split, red, tile, sched = variant
     case = Case(W8A8_INT8, 5, 640, 2048, seed=2, outliers=True)
     _, _, acc = _oracle(case, want_acc=True)
-    qgd.qgd_set_override(qgd.FMT_W8A8_INT8, var, split, red, 0, tile)
+    qgd.qgd_set_override(qgd.FMT_W8A8_INT8, var, split, red, 0, tile, sched)
     got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
@@ -102,11 +106,12 @@ def test_ragged_tiles(fmt, M, N, K):
     # N not a multiple of the 128/256 tile, K not a multiple of the 128 stage
     case = Case(fmt, M, N, K, seed=N, outliers=True)
     yref, bound = _oracle(case)[:2]
-    for var, split, red in ((qgd.VARIANT_SWAP_AB, 1, 0), (qgd.VARIANT_SWAP_AB, 4, 0),
-                            (qgd.VARIANT_STANDARD, 1, 0), (qgd.VARIANT_STANDARD, 2, 1)):
+    for var, split, red, sched in ((qgd.VARIANT_SWAP_AB, 1, 0, GRID), (qgd.VARIANT_SWAP_AB, 4, 0, GRID),
+                                   (qgd.VARIANT_SWAP_AB, 1, 0, PERSISTENT), (qgd.VARIANT_SWAP_AB, 1, 1, PERSISTENT),
+                                   (qgd.VARIANT_STANDARD, 1, 0, GRID), (qgd.VARIANT_STANDARD, 2, 1, GRID)):
         if var == qgd.VARIANT_SWAP_AB and M > 32:
             continue
-        qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, 0)
+        qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, 0, sched)
         case.check_output(case.run(), yref, bound, f"{fmt} M={M} N={N} K={K} var={var} s={split}")
 
 
@@ -122,9 +127,10 @@ def test_empty_m(fmt):
 
 @pytest.mark.parametrize("fmt", ALL_FMTS)
 @pytest.mark.parametrize("reduce", [qgd.REDUCE_LAST_CTA, qgd.REDUCE_TWO_PASS])
-def test_deterministic_split_reductions_repeat_bitwise(fmt, reduce):
+@pytest.mark.parametrize("sched", [GRID, PERSISTENT])
+def test_deterministic_split_reductions_repeat_bitwise(fmt, reduce, sched):
     case = Case(fmt, 7, 1024, 4096, seed=9)
-    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, 8, reduce, 0, 0)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, 8, reduce, 0, 0, sched)
     ys = [case.run().view(torch.int16).cpu() for _ in range(4)]
     for y in ys[1:]:
         assert torch.equal(y, ys[0])
@@ -136,7 +142,7 @@ def test_split_k_up_to_256():
     _, _, acc = _oracle(case, want_acc=True)
     for split in (16, 64, 256):
         for red in (0, 1, 2):
-            qgd.qgd_set_override(qgd.FMT_W8A8_INT8, qgd.VARIANT_SWAP_AB, split, red, 0, 0)
+            qgd.qgd_set_override(qgd.FMT_W8A8_INT8, qgd.VARIANT_SWAP_AB, split, red, 0, 0, GRID)
             assert qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 2, 256, 32768)["split_k"] == split
             got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
             torch.cuda.synchronize()
@@ -170,7 +176,7 @@ def test_graph_replay_matches_eager():
 
 def test_workspace_errors_are_reported():
     case = Case(FP8_DYNAMIC, 4, 512, 4096, seed=3)
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, qgd.REDUCE_LAST_CTA, 0, 0)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, qgd.REDUCE_LAST_CTA, 0, 0, GRID)
     need = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 512, 4096)
     assert need > 0
     small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
@@ -191,6 +197,58 @@ def test_shared_workspace_across_modes_and_shapes():
         for red in (qgd.REDUCE_TWO_PASS, qgd.REDUCE_LAST_CTA, qgd.REDUCE_ATOMIC, qgd.REDUCE_LAST_CTA):
             for c, (yref, bound) in zip(cases, refs):
                 for f in range(3):
-                    qgd.qgd_set_override(f, qgd.VARIANT_SWAP_AB, 4 if rnd == 0 else 8, red, 0, 0)
+                    qgd.qgd_set_override(f, qgd.VARIANT_SWAP_AB, 4 if rnd == 0 else 8, red, 0, 0,
+                                         GRID if rnd == 0 else PERSISTENT)
                 c.check_output(c.run(ws=ws), yref, bound, f"{c.fmt} red={red} rnd={rnd}")
     assert qgd.qgd_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("reduce", [qgd.REDUCE_LAST_CTA, qgd.REDUCE_TWO_PASS, qgd.REDUCE_ATOMIC])
+@pytest.mark.parametrize("M,N,K", [(1, 1024, 4096), (13, 384, 8192), (32, 2048, 1024), (5, 128, 25600)])
+def test_persistent_schedule_uneven_units(fmt, reduce, M, N, K):
+    # unit counts that do not divide by the CTA count: tiles shared by 1..many CTAs
+    case = Case(fmt, M, N, K, seed=N + K, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, -1, reduce, 0, 0, PERSISTENT)
+    case.check_output(case.run(), yref, bound, f"{fmt} M={M} N={N} K={K} r={reduce}")
+    if fmt == W8A8_INT8:
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+
+
+@pytest.mark.parametrize("stages", [2, 3, 5])
+def test_persistent_shallow_pipelines_two_ctas_per_sm(stages):
+    # shallow rings leave room for two CTAs per SM: more CTAs, smaller unit ranges
+    case = Case(FP8_DYNAMIC, 16, 4096, 4096, seed=stages)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, stages, 0, PERSISTENT)
+    case.check_output(case.run(), yref, bound, f"stages={stages}")
+
+
+@pytest.mark.parametrize("pdl", ["0", "1"])
+def test_chained_layers_with_and_without_programmatic_launch(monkeypatch, pdl):
+    # quantize -> GEMM -> quantize(Y) -> GEMM on one stream: the second layer
+    # reads the first layer's output, so any missing dependency shows
+    monkeypatch.setenv("QGD_PDL", pdl)
+    x = synth.activations(8, 2048, seed=31, outliers=True).cuda()
+    w1 = synth.weights(1024, 2048, seed=32).cuda()
+    w2 = synth.weights(512, 1024, seed=33).cuda()
+    wq1, sw1 = qgd.quant_weight_per_channel(w1)
+    wq2, sw2 = qgd.quant_weight_per_channel(w2)
+    ref = None
+    for rep in range(3):
+        xq, sx = qgd.quant_act_per_token(x)
+        h = qgd.qlinear_fp8_dynamic(xq, sx, wq1, sw1)
+        hq, hs = qgd.quant_act_per_token(h)
+        y = qgd.qlinear_fp8_dynamic(hq, hs, wq2, sw2)
+        torch.cuda.synchronize()
+        if ref is None:
+            # the same chain, one call at a time with a synchronize between
+            xq2, sx2 = qgd.quant_act_per_token(x); torch.cuda.synchronize()
+            h2 = qgd.qlinear_fp8_dynamic(xq2, sx2, wq1, sw1); torch.cuda.synchronize()
+            hq2, hs2 = qgd.quant_act_per_token(h2); torch.cuda.synchronize()
+            ref = qgd.qlinear_fp8_dynamic(hq2, hs2, wq2, sw2); torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"rep {rep}"

@@ -46,7 +46,7 @@ def _noalloc(case: Case, y: torch.Tensor) -> int:
 def test_noalloc_matches_workspace_entry_point_twice(split, reduce):
     case = Case(FP8_DYNAMIC, 8, 1024, 4096, seed=21)
     if split is not None:
-        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, split, reduce, 0, 0)
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, split, reduce, 0, 0, qgd.SCHEDULE_GRID)
     # the regular entry point, with a workspace the caller allocated
     ws = qgd.Workspace(qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, case.M, case.N, case.K))
     y_ref = bf16_to_f64(case.run(ws=ws))
@@ -63,7 +63,8 @@ def test_noalloc_rejects_scratch_beyond_its_size():
     # 8 splits x 32 tokens x 16384 columns of fp32 partials is 16 MiB, more
     # than the 8 MiB built-in scratch: refused before anything is launched
     case = Case(FP8_DYNAMIC, 32, 16384, 1024, seed=22)
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_LAST_CTA, 0, 0,
+                         qgd.SCHEDULE_GRID)
     y = torch.zeros((case.M, case.N), dtype=torch.bfloat16, device="cuda")
     assert _noalloc(case, y) == -3
     assert b"built-in scratch" in qgd.lib().qgd_last_error_message()
