@@ -40,35 +40,48 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """Load a build of oracle.c and declare its signatures."""
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lg = ctypes.c_long
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+    L.orc_int8_encode.restype = ctypes.c_int8
+    L.orc_int8_encode.argtypes = [ctypes.c_double]
+    L.orc_quant_rows.restype = None
+    L.orc_quant_rows.argtypes = [P, lg, lg, ctypes.c_int, P, P]
+    L.orc_quant_groups.restype = None
+    L.orc_quant_groups.argtypes = [P, lg, lg, lg, P, P]
+    L.orc_quant_blocks.restype = None
+    L.orc_quant_blocks.argtypes = [P, lg, lg, lg, P, P]
+    L.orc_gemm_rowscaled.restype = None
+    L.orc_gemm_rowscaled.argtypes = [P, P, P, P, lg, lg, lg, ctypes.c_int, P, P, P]
+    L.orc_gemm_blockscaled.restype = None
+    L.orc_gemm_blockscaled.argtypes = [P, P, P, P, lg, lg, lg, lg, P, P]
+    L.orc_dot_split.restype = ctypes.c_int64
+    L.orc_dot_split.argtypes = [P, lg, P, lg, lg, ctypes.c_int, lg]
+    L.orc_num_threads.restype = ctypes.c_int
+    L.orc_num_threads.argtypes = []
+    return L
+
+
+def compile_source(src_path: str, out_path: str) -> str:
+    """Compile a copy of oracle.c (the tests compile deliberately broken
+    copies to show that the pins catch them)."""
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+                    src_path, "-o", out_path, "-lm"], check=True)
+    return out_path
+
+
 def lib() -> ctypes.CDLL:
     global _lib
     with _lock:
         if _lib is None:
             build()
-            L = ctypes.CDLL(_LIB_PATH)
-            P = ctypes.c_void_p
-            lg = ctypes.c_long
-            L.orc_e4m3_decode.restype = ctypes.c_double
-            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
-            L.orc_e4m3_encode.restype = ctypes.c_uint8
-            L.orc_e4m3_encode.argtypes = [ctypes.c_double]
-            L.orc_int8_encode.restype = ctypes.c_int8
-            L.orc_int8_encode.argtypes = [ctypes.c_double]
-            L.orc_quant_rows.restype = None
-            L.orc_quant_rows.argtypes = [P, lg, lg, ctypes.c_int, P, P]
-            L.orc_quant_groups.restype = None
-            L.orc_quant_groups.argtypes = [P, lg, lg, lg, P, P]
-            L.orc_quant_blocks.restype = None
-            L.orc_quant_blocks.argtypes = [P, lg, lg, lg, P, P]
-            L.orc_gemm_rowscaled.restype = None
-            L.orc_gemm_rowscaled.argtypes = [P, P, P, P, lg, lg, lg, ctypes.c_int, P, P, P]
-            L.orc_gemm_blockscaled.restype = None
-            L.orc_gemm_blockscaled.argtypes = [P, P, P, P, lg, lg, lg, lg, P, P]
-            L.orc_dot_split.restype = ctypes.c_int64
-            L.orc_dot_split.argtypes = [P, lg, P, lg, lg, ctypes.c_int, lg]
-            L.orc_num_threads.restype = ctypes.c_int
-            L.orc_num_threads.argtypes = []
-            _lib = L
+            _lib = load_library(_LIB_PATH)
     return _lib
 
 
