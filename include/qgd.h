@@ -77,8 +77,10 @@ typedef enum {
 typedef enum {
   QGD_SCHEDULE_AUTO = -1,
   QGD_SCHEDULE_GRID = 0,      /* one CTA per (output tile, K split): split_k CTAs along K */
-  QGD_SCHEDULE_PERSISTENT = 1 /* Swap-AB only: one CTA per SM; all (tile, 128-wide K slice) units are dealt
-                                 out in equal contiguous ranges, shared tiles finished by the last CTA */
+  QGD_SCHEDULE_PERSISTENT = 1 /* about one CTA per SM.  Swap-AB: all (tile, 128-wide K slice) units are
+                                 dealt out in equal contiguous ranges, shared tiles finished by the last
+                                 CTA.  Standard: (tile, split) items dealt round-robin, the TMEM
+                                 accumulator double-buffered across a CTA's tiles */
 } qgd_schedule;
 
 /* The execution plan for one (format, M, N, K). */

@@ -34,7 +34,9 @@ __all__ = [
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqgd.so")
+# QGD_LIBRARY points the binding at another build of the same C ABI (for
+# example a build with developer tracing compiled in).
+LIB_PATH = os.environ.get("QGD_LIBRARY") or os.path.join(_PKG, "libqgd.so")
 DEFAULT_TABLE = os.path.join(_PKG, "tables", "b200.tsv")
 
 FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8 = 0, 1, 2

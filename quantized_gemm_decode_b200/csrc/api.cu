@@ -177,9 +177,11 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
     while (tiles * s < g_num_sms && s * 2 <= nkt && s < 256) s *= 2;
     p.split_k = s;  // used by the grid schedule
   } else {
+    // Larger M: Standard tiles, one persistent CTA per SM.
     p.variant = kStandard;
     p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
     p.split_k = 1;
+    p.schedule = kPersistent;
   }
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -209,7 +211,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.variant == kSwapAB && M > kDecodeMaxM) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
-  if (p.variant != kSwapAB || p.schedule != kPersistent) p.schedule = kGrid;
+  if (p.schedule != kPersistent) p.schedule = kGrid;
   int smax = nkt < 256 ? nkt : 256;
   if (smax < 1) smax = 1;
   if (p.split_k < 1) p.split_k = 1;
@@ -279,6 +281,17 @@ Exec make_exec(const qgd_plan& p, int M, int N, int K) {
   } else {
     e.maxc = p.split_k;
     e.tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
+    if (p.schedule == kPersistent) {
+      // (tile, split) items dealt round-robin over one CTA per SM; a 256-wide
+      // double-buffered accumulator takes all of TMEM, so one CTA per SM
+      const long long items = static_cast<long long>(e.tiles) * p.split_k;
+      int occ = static_cast<int>(kSmemPerSM / (standard_smem_bytes(p.tile_n, p.stages) + 1024));
+      occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);
+      if (p.tile_n == 256) occ = 1;
+      const long long cap = static_cast<long long>(g_num_sms) * occ;
+      e.persistent = true;
+      e.ctas = static_cast<int>(items < cap ? items : cap);
+    }
     if (p.split_k > 1)
       e.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
   }

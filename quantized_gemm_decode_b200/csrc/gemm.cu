@@ -37,6 +37,24 @@ namespace {
 
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_device_error, 0u, code); }
 
+// Developer timeline of the Swap-AB kernel: with -DQGD_TRACE each CTA stamps
+// %globaltimer at eight points (entry, set-up done, first loads issued, first
+// stage landed, last MMA committed, last accumulator read, epilogue done,
+// exit); qgd_debug_trace() copies the stamps out.  Compiled out otherwise.
+#ifdef QGD_TRACE
+constexpr int kTraceCtas = 4096;
+__device__ unsigned long long g_trace[kTraceCtas * 8];
+#define QGD_STAMP(slot)                                                             \
+  do {                                                                              \
+    const unsigned cta_ = blockIdx.x + blockIdx.y * gridDim.x;                      \
+    if (cta_ < kTraceCtas) g_trace[cta_ * 8 + (slot)] = globaltimer_ns();           \
+  } while (0)
+#else
+#define QGD_STAMP(slot) \
+  do {                  \
+  } while (0)
+#endif
+
 constexpr uint32_t kBarBytes = 512;  // mbarriers + a few flags, after the rings
 
 struct SmemCtl {
@@ -254,6 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     ue = t0 + static_cast<long long>(blockIdx.y + 1) * nkt / a.splits;
   }
   const int nk = static_cast<int>(ue - ub);
+  if (threadIdx.x == 0) QGD_STAMP(0);
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tw);
@@ -283,6 +302,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   griddep_launch_dependents();
   const uint32_t tmem = ctl->tmem_base;
   int issued = 0;
+  if (threadIdx.x == 0) QGD_STAMP(1);
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -302,6 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int i = 0; i < pre; ++i)
         tma_load_2d(x_ring + i * kXBytes, &tx, &ctl->full[i], static_cast<int>((ub + i) % nkt) * kTileK, 0, pol_x);
       issued = pre;
+      QGD_STAMP(2);
       for (int i = pre; i < nk; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
@@ -332,6 +353,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ctl->abort_flag = 1;
           break;
         }
+        if (i == 0) QGD_STAMP(3);
         const int kt = static_cast<int>((ub + i) % nkt);
         const bool seg_start = (i == 0) || (kt == 0);
         const bool seg_end = (i == nk - 1) || (kt == nkt - 1);
@@ -365,6 +387,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (kBlock || seg_end) mma_commit(&ctl->tfull[slot]);
         if (seg_end) ++seg;
       }
+      QGD_STAMP(4);
     }
     __syncwarp();
   } else {
@@ -430,6 +453,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (!epi_agree_ok(ctl)) break;
+      if (threadIdx.x == 64 && i + len >= nk) QGD_STAMP(5);
 
       const bool in_n = n < N;
       int ncontrib, jslot;
@@ -493,9 +517,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       i += len;
       ++seg;
     }
+    if (threadIdx.x == 64) QGD_STAMP(6);
   }
 
   teardown(ctl, warp, lane, issued, stages, tmem, kCols);
+  if (threadIdx.x == 32) QGD_STAMP(7);
 }
 
 // Two-pass reduction for the Swap-AB layout: one CTA per tile, one thread per
@@ -536,8 +562,56 @@ __global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArg
     if (m < M) store_final<kFmt>(sum[m], m, n, a);
 }
 
+// Last CTA of a Standard tile: add the split partials (or read the atomic
+// sum) for this thread's token row, 16 columns at a time, in split order.
+template <int kFmt, int kTileN>
+__device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0, bool in_m) {
+  if (!in_m) return;
+  const int M = a.M, N = a.N;
+  for (int nc = n0; nc < n0 + kTileN && nc < N; nc += 16) {
+    const size_t idx = static_cast<size_t>(m) * N + nc;
+    uint32_t v[16];
+    if (a.reduce == kAtomic) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.accum) + idx);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 t = __ldcg(src + q);
+        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.partial) + idx);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 t = __ldcg(src + q);
+        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+      }
+      for (int s = 1; s < a.splits; ++s) {
+        const uint4* sp = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.partial) +
+                                                         static_cast<size_t>(s) * M * N + idx);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 t = __ldcg(sp + q);
+          v[4 * q] = add_acc<kFmt>(v[4 * q], t.x);
+          v[4 * q + 1] = add_acc<kFmt>(v[4 * q + 1], t.y);
+          v[4 * q + 2] = add_acc<kFmt>(v[4 * q + 2], t.z);
+          v[4 * q + 3] = add_acc<kFmt>(v[4 * q + 3], t.w);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) store_final<kFmt>(v[j], m, nc + j, a);
+  }
+}
+
 // ===========================================================================
-// Standard kernel (large M): grid = (ceil(N/kTileN), ceil(M/128), splits)
+// Standard kernel (larger M): D[m, n] over 128 x kTileN output tiles.
+//
+// Work items are (tile, split) pairs, tiles ordered token-tile fastest so
+// CTAs running side by side share a weight tile in L2.  CTA c takes items c,
+// c + G, c + 2G, ... of the grid's G CTAs: with G = #items every CTA does
+// one item (the grid schedule, needed for Split-K), with G = #SMs the CTAs
+// persist and the TMEM accumulator is double-buffered, so the epilogue of
+// one tile overlaps the mainloop of the next.
 // ===========================================================================
 template <int kFmt, int kTileN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -546,8 +620,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
   static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
-  constexpr int kSlots = kBlock ? 2 : 1;
-  constexpr uint32_t kCols = kSlots * kTileN;  // 128 or 256
+  constexpr int kSlots = 2;                   // Block_FP8: per-K-block ring; else: per-tile double buffer
+  constexpr uint32_t kCols = kSlots * kTileN;  // 256 or 512
   constexpr uint32_t kXBytes = kStdTileM * kTileK;
   constexpr uint32_t kWBytes = kTileN * kTileK;
   constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kStdTileM, kTileN);
@@ -560,11 +634,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * kWBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
   const int nkt = (a.K + kTileK - 1) / kTileK;
-  const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / a.splits);
-  const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / a.splits);
-  const int nk = kt1 - kt0;
+  const int m_tiles = (a.M + kStdTileM - 1) / kStdTileM;
+  const int n_tiles = (a.N + kTileN - 1) / kTileN;
+  const int S = a.splits;
+  const long long items = static_cast<long long>(m_tiles) * n_tiles * S;
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tx);
@@ -596,104 +670,143 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int issued = 0;
 
   if (warp == 0) {
+    // ---------------- TMA producer: items x K slices, one ring ----------------
     if (lane == 0) {
       const uint64_t pol_x = policy_evict_last();
       const uint64_t pol_w = policy_evict_last();
       griddep_wait();  // activations come from the preceding kernel
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % stages;
-        const uint32_t round = i / stages;
-        if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
-          record_error(kErrWaitProducer);
-          ctl->abort_flag = 1;
-          break;
+      int i = 0;
+      bool stop = false;
+      for (long long w = blockIdx.x; w < items && !stop; w += gridDim.x) {
+        const int tile = static_cast<int>(w / S), split = static_cast<int>(w % S);
+        const int m_tile = tile % m_tiles, n_tile = tile / m_tiles;
+        const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
+        const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
+        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+          const int s = i % stages;
+          const uint32_t round = i / stages;
+          if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+            record_error(kErrWaitProducer);
+            ctl->abort_flag = 1;
+            stop = true;
+            break;
+          }
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->full[s], kXBytes + kWBytes);
+          tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kt * kTileK, m_tile * kStdTileM, pol_x);
+          tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kt * kTileK, n_tile * kTileN, pol_w);
+          issued = i + 1;
         }
-        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
-        mbar_arrive_expect_tx(&ctl->full[s], kXBytes + kWBytes);
-        const int kx = (kt0 + i) * kTileK;
-        tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kx, m_tile * kStdTileM, pol_x);
-        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, n_tile * kTileN, pol_w);
-        issued = i + 1;
       }
     }
   } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t x_base = smem_u32(x_ring), w_base = smem_u32(w_ring);
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % stages;
-        const uint32_t round = i / stages;
-        if (!mbar_wait(&ctl->full[s], round & 1)) {
-          record_error(kErrWaitMma);
-          ctl->abort_flag = 1;
-          break;
-        }
-        uint32_t d = tmem;
-        if constexpr (kBlock) {
-          const int slot = i % kSlots;
-          if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
+      int i = 0, li = 0;
+      bool stop = false;
+      for (long long w = blockIdx.x; w < items && !stop; w += gridDim.x, ++li) {
+        const int split = static_cast<int>(w % S);
+        const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
+        const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
+        const int buf = li & 1;
+        if constexpr (!kBlock) {
+          if (!mbar_wait(&ctl->tempty[buf], ((li >> 1) & 1) ^ 1)) {
             record_error(kErrWaitMma);
             ctl->abort_flag = 1;
             break;
           }
-          d = tmem + slot * kTileN;
         }
-        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
-        tc_fence_after();
+        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+          const int s = i % stages;
+          const uint32_t round = i / stages;
+          if (!mbar_wait(&ctl->full[s], round & 1)) {
+            record_error(kErrWaitMma);
+            ctl->abort_flag = 1;
+            stop = true;
+            break;
+          }
+          uint32_t d = tmem + buf * kTileN;
+          if constexpr (kBlock) {
+            const int slot = i % kSlots;
+            if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
+              record_error(kErrWaitMma);
+              ctl->abort_flag = 1;
+              stop = true;
+              break;
+            }
+            d = tmem + slot * kTileN;
+          }
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTileK / 32; ++kk) {
-          const uint64_t ad = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
-          const uint64_t bd = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
-          const uint32_t accumulate = kBlock ? (kk > 0) : (i > 0 || kk > 0);
-          mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+          for (int kk = 0; kk < kTileK / 32; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
+            const uint32_t accumulate = kBlock ? (kk > 0) : (kt > kt0 || kk > 0);
+            mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+          }
+          mma_commit(&ctl->empty[s]);
+          if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
         }
-        mma_commit(&ctl->empty[s]);
-        if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
+        if (stop) break;
+        if constexpr (!kBlock) mma_commit(&ctl->tfull[buf]);
       }
-      if constexpr (!kBlock) mma_commit(&ctl->accfull);
     }
     __syncwarp();
   } else {
+    // ---------------- epilogue (warps 2..5) ----------------
     griddep_wait();  // scales and outputs: only after the preceding kernel is done
     const int q = warp & 3;
-    const int m = m_tile * kStdTileM + q * 32 + lane;  // TMEM lane = token row
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int M = a.M, N = a.N;
-    const int n0 = n_tile * kTileN;
-    const bool in_m = m < M;
+    int i = 0, li = 0;
+    for (long long w = blockIdx.x; w < items; w += gridDim.x, ++li) {
+      const int tile = static_cast<int>(w / S), split = static_cast<int>(w % S);
+      const int m_tile = tile % m_tiles, n_tile = tile / m_tiles;
+      const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
+      const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
+      const int m = m_tile * kStdTileM + q * 32 + lane;  // TMEM lane = token row
+      const int n0 = n_tile * kTileN;
+      const bool in_m = m < M;
 
-    if constexpr (kBlock) {
-      const int KB = a.K / kTileK;
-      float facc[kTileN];
+      if constexpr (kBlock) {
+        const int KB = a.K / kTileK;
+        float facc[kTileN];
 #pragma unroll
-      for (int j = 0; j < kTileN; ++j) facc[j] = 0.f;
-      const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
-      const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
-      for (int i = 0; i < nk; ++i) {
-        const int slot = i % kSlots;
-        const int kb = kt0 + i;
-        const float sc = in_m ? __ldg(sxrow + kb) * __ldg(swrow + kb) : 0.f;
-        if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
-          if (lane == 0) {
-            record_error(kErrWaitEpilogue);
-            ctl->abort_flag = 1;
+        for (int j = 0; j < kTileN; ++j) facc[j] = 0.f;
+        const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
+        const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
+        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+          const int slot = i % kSlots;
+          const float sc = in_m ? __ldg(sxrow + kt) * __ldg(swrow + kt) : 0.f;
+          if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
+            if (lane == 0) {
+              record_error(kErrWaitEpilogue);
+              ctl->abort_flag = 1;
+            }
+            break;
           }
-          break;
-        }
-        tc_fence_after();
+          tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kTileN / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(taddr + slot * kTileN + c * 16, r);
-          tmem_wait_ld();
+          for (int c = 0; c < kTileN / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(taddr + slot * kTileN + c * 16, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, facc[c * 16 + j]);
+            for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, facc[c * 16 + j]);
+          }
+          tc_fence_before();
+          mbar_arrive(&ctl->tempty[slot]);
         }
-        tc_fence_before();
-        mbar_arrive(&ctl->tempty[slot]);
-      }
-      if (epi_agree_ok(ctl)) {
-        // finished tile: convert from registers
-        if (a.splits == 1) {
+        if (!epi_agree_ok(ctl)) break;
+        if (S == 1) {
           if (in_m) {
 #pragma unroll
             for (int c = 0; c < kTileN / 16; ++c) {
@@ -723,132 +836,94 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < kTileN / 16; ++c) {
               const int nc = n0 + c * 16;
               if (nc >= N) break;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const size_t idx = static_cast<size_t>(m) * N + nc + j;
-                if (a.reduce == kAtomic)
-                  atomic_acc<kFmt>(a.accum, idx, __float_as_uint(facc[c * 16 + j]));
-                else
-                  static_cast<float*>(a.partial)[static_cast<size_t>(split) * M * N + idx] = facc[c * 16 + j];
-              }
-            }
-          }
-          if (a.reduce != kTwoPass) {
-            const int tile = m_tile * gridDim.x + n_tile;
-            if (epi_arrive_last(ctl, a, tile, a.splits)) {
-              if (in_m) {
-                for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
-                  const size_t idx = static_cast<size_t>(m) * N + nc;
-                  uint32_t v;
-                  if (a.reduce == kAtomic) {
-                    v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-                  } else {
-                    v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
-                    for (int s = 1; s < a.splits; ++s)
-                      v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
-                                                     static_cast<size_t>(s) * M * N + idx));
-                  }
-                  store_final<kFmt>(v, m, nc, a);
-                }
-              }
-              if (threadIdx.x == 64) a.tickets[tile] = 0u;
-            }
-          }
-        }
-      }
-    } else {
-      bool ok = warp_wait(&ctl->accfull, 0);
-      if (!ok && lane == 0) {
-        record_error(kErrWaitEpilogue);
-        ctl->abort_flag = 1;
-      }
-      if (ok) tc_fence_after();
-      if (epi_agree_ok(ctl)) {
-        const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
-        if (a.splits == 1) {
-#pragma unroll 1
-          for (int c = 0; c < kTileN / 16; ++c) {
-            const int nc = n0 + c * 16;
-            uint32_t r[16];
-            __syncwarp();
-            tmem_ld16(taddr + c * 16, r);
-            tmem_wait_ld();
-            if (in_m && nc < N) {
-            if (a.raw) {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            } else {
-              const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
-              float sw16[16];
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const float4 t = __ldg(swv + v);
-                sw16[4 * v] = t.x;
-                sw16[4 * v + 1] = t.y;
-                sw16[4 * v + 2] = t.z;
-                sw16[4 * v + 3] = t.w;
-              }
-              uint32_t pk[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                float v0, v1;
-                if constexpr (kInt) {
-                  v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
-                  v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
-                } else {
-                  v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
-                  v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
-                }
-                pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(a.y + static_cast<size_t>(m) * N + nc);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-            }
-          }
-        } else {
-#pragma unroll 1
-          for (int c = 0; c < kTileN / 16; ++c) {
-            const int nc = n0 + c * 16;
-            uint32_t r[16];
-            __syncwarp();
-            tmem_ld16(taddr + c * 16, r);
-            tmem_wait_ld();
-            if (in_m && nc < N) {
               const size_t idx = static_cast<size_t>(m) * N + nc;
               if (a.reduce == kAtomic) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, r[j]);
+                for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, __float_as_uint(facc[c * 16 + j]));
               } else {
-                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(__float_as_uint(facc[c * 16 + 4 * v]), __float_as_uint(facc[c * 16 + 4 * v + 1]),
+                                      __float_as_uint(facc[c * 16 + 4 * v + 2]), __float_as_uint(facc[c * 16 + 4 * v + 3]));
               }
             }
           }
-          if (a.reduce != kTwoPass) {
-            const int tile = m_tile * gridDim.x + n_tile;
-            if (epi_arrive_last(ctl, a, tile, a.splits)) {
-              if (in_m) {
-                for (int nc = n0; nc < n0 + kTileN && nc < N; ++nc) {
-                  const size_t idx = static_cast<size_t>(m) * N + nc;
-                  uint32_t v;
-                  if (a.reduce == kAtomic) {
-                    v = ldcg_u32(static_cast<uint32_t*>(a.accum) + idx);
-                  } else {
-                    v = ldcg_u32(static_cast<uint32_t*>(a.partial) + idx);
-                    for (int s = 1; s < a.splits; ++s)
-                      v = add_acc<kFmt>(v, ldcg_u32(static_cast<uint32_t*>(a.partial) +
-                                                     static_cast<size_t>(s) * M * N + idx));
-                  }
-                  store_final<kFmt>(v, m, nc, a);
-                }
-              }
-              if (threadIdx.x == 64) a.tickets[tile] = 0u;
-            }
+          if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, tile, S)) {
+            std_reduce_tile<kFmt, kTileN>(a, m, n0, in_m);
+            if (threadIdx.x == 64) a.tickets[tile] = 0u;
           }
+        }
+      } else {
+        const int buf = li & 1;
+        const bool ok = warp_wait(&ctl->tfull[buf], (li >> 1) & 1);
+        if (!ok && lane == 0) {
+          record_error(kErrWaitEpilogue);
+          ctl->abort_flag = 1;
+        }
+        if (ok) tc_fence_after();
+        if (!epi_agree_ok(ctl)) break;
+        const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
+        const uint32_t tbuf = taddr + buf * kTileN;
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 16; ++c) {
+          const int nc = n0 + c * 16;
+          uint32_t r[16];
+          __syncwarp();
+          tmem_ld16(tbuf + c * 16, r);
+          tmem_wait_ld();
+          if (c == kTileN / 16 - 1) {
+            // the whole accumulator is in registers: hand the buffer back
+            tc_fence_before();
+            mbar_arrive(&ctl->tempty[buf]);
+          }
+          if (!in_m || nc >= N) continue;
+          const size_t idx = static_cast<size_t>(m) * N + nc;
+          if (S > 1) {
+            if (a.reduce == kAtomic) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, r[j]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            }
+          } else if (a.raw) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+          } else {
+            const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+            float sw16[16];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 t = __ldg(swv + v);
+              sw16[4 * v] = t.x;
+              sw16[4 * v + 1] = t.y;
+              sw16[4 * v + 2] = t.z;
+              sw16[4 * v + 3] = t.w;
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float v0, v1;
+              if constexpr (kInt) {
+                v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
+                v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+              } else {
+                v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
+                v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+              }
+              pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+        if (S > 1 && a.reduce != kTwoPass && epi_arrive_last(ctl, a, tile, S)) {
+          std_reduce_tile<kFmt, kTileN>(a, m, n0, in_m);
+          if (threadIdx.x == 64) a.tickets[tile] = 0u;
         }
       }
     }
@@ -941,7 +1016,9 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
   static bool attr_done = false;
   cudaError_t e = set_smem_attr(standard_kernel<kFmt, kTileN>, attr_done);
   if (e != cudaSuccess) return e;
-  const dim3 grid((a.N + kTileN - 1) / kTileN, (a.M + kStdTileM - 1) / kStdTileM, a.splits);
+  const long long items = static_cast<long long>((a.N + kTileN - 1) / kTileN) *
+                          ((a.M + kStdTileM - 1) / kStdTileM) * a.splits;
+  const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
   return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(kGemmThreads), standard_smem_bytes(kTileN, a.stages),
                    stream, a.pdl != 0, tx, tw, a);
 }
@@ -968,6 +1045,13 @@ cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CU
   if (fmt == kFmtBlock && tile_n == 128) return launch_standard_t<kFmtBlock, 128>(tx, tw, a, stream);
   return cudaErrorInvalidValue;
 }
+
+#ifdef QGD_TRACE
+extern "C" __attribute__((visibility("default"))) int qgd_debug_trace(unsigned long long* host, size_t count) {
+  const size_t n = count < static_cast<size_t>(kTraceCtas) * 8 ? count : static_cast<size_t>(kTraceCtas) * 8;
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)));
+}
+#endif
 
 cudaError_t read_device_error(unsigned int* code) {
   return cudaMemcpyFromSymbol(code, g_device_error, sizeof(unsigned int));

@@ -78,7 +78,7 @@ def test_default_plans():
     # large M: Standard, no split
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 512, 6144, 4096)
     assert p["variant"] == qgd.VARIANT_STANDARD and p["split_k"] == 1 and p["tile_n"] == 256
-    assert p["schedule"] == qgd.SCHEDULE_GRID
+    assert p["schedule"] == qgd.SCHEDULE_PERSISTENT
     p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 512, 6144, 4096)
     assert p["tile_n"] == 128
     # split never exceeds the number of 128-wide K tiles
@@ -90,9 +90,8 @@ def test_override_and_clamping():
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 256, qgd.REDUCE_ATOMIC, 5, 0, qgd.SCHEDULE_GRID)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
     assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["source"]) == (1, 32, 2, 5, 2)
-    # Swap-AB cannot take more than 32 tokens: it falls back to Standard, and
-    # the persistent schedule is Swap-AB only
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, qgd.SCHEDULE_PERSISTENT)
+    # Swap-AB cannot take more than 32 tokens: it falls back to Standard
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, qgd.SCHEDULE_GRID)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)
     assert p["variant"] == qgd.VARIANT_STANDARD and p["schedule"] == qgd.SCHEDULE_GRID
     with pytest.raises(qgd.QGDError):

@@ -12,7 +12,7 @@ import torch
 import quantized_gemm_decode_b200 as qgd
 from quantized_gemm_decode_b200 import synth
 from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8
-from paritylib import FMT_ID, Case, as_u8, bf16_to_f64
+from paritylib import FMT_ID, Case, as_u8, bf16_to_f64, check_fp8_tolerance, check_within_one_ulp
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +49,7 @@ VARIANTS = (
     [(qgd.VARIANT_SWAP_AB, s, r, 0, GRID) for s in (1, 2, 4, 8) for r in (0, 1, 2)]
     + [(qgd.VARIANT_SWAP_AB, 1, r, 0, PERSISTENT) for r in (0, 1, 2)]
     + [(qgd.VARIANT_STANDARD, s, r, t, GRID) for t in (128, 256) for s in (1, 2, 8) for r in (0, 1, 2)]
+    + [(qgd.VARIANT_STANDARD, s, r, t, PERSISTENT) for t in (128, 256) for s in (1, 2) for r in (0, 1, 2)]
 )
 
 
@@ -252,3 +253,24 @@ def test_chained_layers_with_and_without_programmatic_launch(monkeypatch, pdl):
             hq2, hs2 = qgd.quant_act_per_token(h2); torch.cuda.synchronize()
             ref = qgd.qlinear_fp8_dynamic(hq2, hs2, wq2, sw2); torch.cuda.synchronize()
         assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"rep {rep}"
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("M,N,K,split", [(640, 2048, 1024, 1), (300, 4096, 512, 1), (1000, 768, 2048, 2),
+                                         (2048, 1024, 768, 1)])
+def test_persistent_standard_many_tiles_per_cta(fmt, M, N, K, split):
+    # more tiles than SMs: each CTA walks several tiles through the
+    # double-buffered accumulator; checked on sampled rows with the oracle
+    case = Case(fmt, M, N, K, seed=M + K, outliers=True)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD, split, 0, 0, 0, PERSISTENT)
+    y = bf16_to_f64(case.run())
+    rows = np.unique(np.concatenate([np.arange(0, M, 97), [M - 1]]))
+    xsub = case.x[torch.from_numpy(rows)]
+    sub = Case.__new__(Case)
+    sub.fmt, sub.M, sub.N, sub.K, sub.x, sub.w = fmt, len(rows), N, K, xsub, case.w
+    xq, sx, wq, sw = sub.oracle_quant()
+    yref, bound = sub.oracle_gemm(xq, sx, wq, sw)[:2]
+    if fmt == W8A8_INT8:
+        check_within_one_ulp(y[rows], yref, f"{fmt} M={M}")
+    else:
+        check_fp8_tolerance(y[rows], yref, bound, K, f"{fmt} M={M}")
