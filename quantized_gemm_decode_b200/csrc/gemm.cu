@@ -180,18 +180,19 @@ __device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl) {
 }
 
 // Split-K arrival: returns true in every epilogue thread of the last CTA to
-// arrive at tile `tile`.  Called after this CTA's partials are written.
+// arrive at tile `tile`.  Called after this CTA's partials are written: the
+// barrier orders every epilogue thread's stores before one thread's
+// acquire-release atomic at GPU scope, and the barrier after it orders that
+// acquire before the last CTA's reads of the other partials.
 __device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile, int expected) {
-  __threadfence();
   epi_sync();
   if (threadIdx.x == 64) {
-    const unsigned int old = atomicAdd(a.tickets + tile, 1u);
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.tickets + tile) : "memory");
     ctl->last_flag = (old == static_cast<unsigned int>(expected - 1));
   }
   epi_sync();
-  const bool last = ctl->last_flag != 0;
-  if (last) __threadfence();
-  return last;
+  return ctl->last_flag != 0;
 }
 
 // ===========================================================================
@@ -234,8 +235,71 @@ __device__ __forceinline__ uint32_t* swap_slot(const GemmArgs& a, int t, int j, 
          ((static_cast<size_t>(t) * a.maxc + j) * kSwapTileN + row) * static_cast<size_t>(a.mstride);
 }
 
+// Sum of the contributors' partial rows of tile t (this thread's weight row),
+// in contributor order.  Loads are issued kBatch contributors at a time so
+// that one memory round trip serves many partials; kVec 16-byte vectors per
+// partial row (only the first nvec are live).  Contributor `own` (or -1) is
+// taken from `own_acc` instead of memory.
+template <int kFmt, int kMpad, int kVec, int kBatch>
+__device__ __forceinline__ void fixup_sum_t(const GemmArgs& a, int t, int row, int ncontrib, int nvec, int own,
+                                            const uint32_t (&own_acc)[kMpad], uint32_t (&sum)[kMpad]) {
+  static_assert(kVec * 4 <= kMpad, "vector count exceeds the accumulator");
+  for (int j0 = 0; j0 < ncontrib; j0 += kBatch) {
+    uint4 buf[kBatch][kVec];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int j = j0 + b;
+      if (j < ncontrib && j != own) {
+        const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j, row));
+#pragma unroll
+        for (int v = 0; v < kVec; ++v)
+          if (v < nvec) buf[b][v] = __ldcg(src + v);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int j = j0 + b;
+      if (j < ncontrib) {
+#pragma unroll
+        for (int v = 0; v < kVec; ++v) {
+          if (v < nvec) {
+            uint4 w4 = buf[b][v];
+            if (j == own) w4 = make_uint4(own_acc[4 * v], own_acc[4 * v + 1], own_acc[4 * v + 2], own_acc[4 * v + 3]);
+            if (j == 0) {
+              sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+            } else {
+              sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+              sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+              sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+              sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int kFmt, int kMpad>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__device__ __forceinline__ void fixup_sum(const GemmArgs& a, int t, int row, int ncontrib, int nvec, int own,
+                                       const uint32_t (&own_acc)[kMpad], uint32_t (&sum)[kMpad]) {
+  // a fixed budget of kMpad/4 16-byte loads per round trip, spent on more
+  // contributors when each partial row is short
+  // contributors when each partial row is short (M > 16 always has 5+ vectors)
+  constexpr int kV = kMpad / 4;
+  if constexpr (kMpad == 16) {
+    if (nvec == 1) fixup_sum_t<kFmt, kMpad, 1, kV>(a, t, row, ncontrib, nvec, own, own_acc, sum);
+    else if (nvec == 2) fixup_sum_t<kFmt, kMpad, 2, kV / 2>(a, t, row, ncontrib, nvec, own, own_acc, sum);
+    else fixup_sum_t<kFmt, kMpad, kV, 1>(a, t, row, ncontrib, nvec, own, own_acc, sum);
+  } else {
+    fixup_sum_t<kFmt, kMpad, kV, 1>(a, t, row, ncontrib, nvec, own, own_acc, sum);
+  }
+}
+
+// Two CTAs per SM must always fit (the persistent grid size assumes it), so
+// the register budget is capped at 65536 / (2 * 192) per thread.
+template <int kFmt, int kMpad>
+__global__ void __launch_bounds__(kGemmThreads, 2)
     swapab_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx,
                   const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
@@ -485,27 +549,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (m < M) store_final<kFmt>(ldcg_u32(static_cast<uint32_t*>(a.accum) + static_cast<size_t>(m) * N + n), m, n, a);
             } else {
               uint32_t sum[kMpad];
-              const uint4* src0 = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, 0, row));
-#pragma unroll
-              for (int v = 0; v < kMpad / 4; ++v) {
-                if (v < nvec) {
-                  const uint4 w4 = __ldcg(src0 + v);
-                  sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
-                }
-              }
-              for (int jj = 1; jj < ncontrib; ++jj) {
-                const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, jj, row));
-#pragma unroll
-                for (int v = 0; v < kMpad / 4; ++v) {
-                  if (v < nvec) {
-                    const uint4 w4 = __ldcg(src + v);
-                    sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
-                    sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
-                    sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
-                    sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
-                  }
-                }
-              }
+              fixup_sum<kFmt, kMpad>(a, t, row, ncontrib, nvec, -1, acc, sum);  // own partial re-read from L2
 #pragma unroll
               for (int m = 0; m < kMpad; ++m)
                 if (m < M) store_final<kFmt>(sum[m], m, n, a);
@@ -537,26 +581,10 @@ __global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArg
   const int n = t * kSwapTileN + row;
   if (ncontrib == 1 || n >= a.N) return;  // written directly by its only contributor
   const int M = a.M, nvec = (M + 3) / 4;
-  uint32_t sum[kMpad];
+  uint32_t sum[kMpad], none[kMpad];
 #pragma unroll
-  for (int m = 0; m < kMpad; ++m) sum[m] = 0u;
-  for (int jj = 0; jj < ncontrib; ++jj) {
-    const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, jj, row));
-#pragma unroll
-    for (int v = 0; v < kMpad / 4; ++v) {
-      if (v < nvec) {
-        const uint4 w4 = src[v];
-        if (jj == 0) {
-          sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
-        } else {
-          sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
-          sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
-          sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
-          sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
-        }
-      }
-    }
-  }
+  for (int m = 0; m < kMpad; ++m) none[m] = 0u;
+  fixup_sum<kFmt, kMpad>(a, t, row, ncontrib, nvec, -1, none, sum);
 #pragma unroll
   for (int m = 0; m < kMpad; ++m)
     if (m < M) store_final<kFmt>(sum[m], m, n, a);
