@@ -73,6 +73,10 @@ def candidates(fmt: str, M: int, N: int, K: int):
                 continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
             for r in ((0,) if s == 1 else (0, 1, 2)):
                 out.append((0, s, r, t, 0))
+        for s in (1, 2):
+            if s <= nkt:
+                for r in ((0,) if s == 1 else (0, 1)):
+                    out.append((0, s, r, t, 1))  # Standard, persistent
     return out
 
 
