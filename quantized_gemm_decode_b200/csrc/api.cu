@@ -247,7 +247,7 @@ struct Exec {
   size_t data_off = 0, data_bytes = 0, total = 0;
 };
 
-Exec make_exec(const qgd_plan& p, int M, int N, int K) {
+Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   Exec e;
   const int nkt = (K + kTileK - 1) / kTileK;
   e.mpad = M <= 16 ? 16 : 32;
@@ -282,12 +282,13 @@ Exec make_exec(const qgd_plan& p, int M, int N, int K) {
     e.maxc = p.split_k;
     e.tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
     if (p.schedule == kPersistent) {
-      // (tile, split) items dealt round-robin over one CTA per SM; a 256-wide
-      // double-buffered accumulator takes all of TMEM, so one CTA per SM
+      // (tile, split) items dealt round-robin over the SMs; a CTA whose
+      // accumulators take all 512 TMEM columns (2 x 256, or Block_FP8's
+      // 4 x 128) leaves room for no second CTA on its SM
       const long long items = static_cast<long long>(e.tiles) * p.split_k;
       int occ = static_cast<int>(kSmemPerSM / (standard_smem_bytes(p.tile_n, p.stages) + 1024));
       occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);
-      if (p.tile_n == 256) occ = 1;
+      if (p.tile_n == 256 || fmt == kFmtBlock) occ = 1;
       const long long cap = static_cast<long long>(g_num_sms) * occ;
       e.persistent = true;
       e.ctas = static_cast<int>(items < cap ? items : cap);
@@ -331,7 +332,7 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   if ((st = get_encoder()) != QGD_OK) return st;
 
   const qgd_plan p = make_plan(fmt, M, N, K);
-  const Exec ex = make_exec(p, M, N, K);
+  const Exec ex = make_exec(fmt, p, M, N, K);
   if (ex.total > 0 && (!ws || ws_bytes < ex.total))
     return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", ex.total, ws ? ws_bytes : 0);
   if (ex.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
@@ -495,7 +496,7 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
   if (st != QGD_OK) return st;
   if (M == 0) return QGD_OK;
   const qgd_plan p = make_plan(kFmtFP8, M, N, K);
-  const Exec ex = make_exec(p, M, N, K);
+  const Exec ex = make_exec(kFmtFP8, p, M, N, K);
   if (ex.total > kNoAllocScratchBytes)
     return fail(QGD_ERR_WORKSPACE,
                 "qlinear_fp8_dynamic_noalloc: this plan (split_k=%d, M=%d, N=%d) needs %zu bytes of Split-K "
@@ -516,7 +517,7 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
 
 size_t qgd_workspace_size(int fmt, int M, int N, int K) {
   if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
-  return make_exec(make_plan(fmt, M, N, K), M, N, K).total;
+  return make_exec(fmt, make_plan(fmt, M, N, K), M, N, K).total;
 }
 
 qgd_status qgd_load_dispatch_table(const char* path) {

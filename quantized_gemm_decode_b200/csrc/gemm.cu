@@ -648,8 +648,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
   static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
-  constexpr int kSlots = 2;                   // Block_FP8: per-K-block ring; else: per-tile double buffer
-  constexpr uint32_t kCols = kSlots * kTileN;  // 256 or 512
+  // Block_FP8: a ring of 4 per-K-block accumulators (the MMA runs up to three
+  // K blocks ahead of the promotion); else: a per-tile double buffer.
+  constexpr int kSlots = kBlock ? 4 : 2;
+  constexpr uint32_t kCols = kSlots * kTileN;  // 512 (Block_FP8: 4 x 128; else 2 x 256) or 256
   constexpr uint32_t kXBytes = kStdTileM * kTileK;
   constexpr uint32_t kWBytes = kTileN * kTileK;
   constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kStdTileM, kTileN);
@@ -822,13 +824,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
+          // four TMEM loads in flight per wait
 #pragma unroll
-          for (int c = 0; c < kTileN / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(taddr + slot * kTileN + c * 16, r);
+          for (int h = 0; h < kTileN / 64; ++h) {
+            uint32_t r[4][16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld16(taddr + slot * kTileN + h * 64 + c * 16, r[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, facc[c * 16 + j]);
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                facc[h * 64 + c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[h * 64 + c * 16 + j]);
           }
           tc_fence_before();
           mbar_arrive(&ctl->tempty[slot]);
