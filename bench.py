@@ -66,10 +66,15 @@ def path_bytes(fmt: str, M: int, N: int, K: int) -> int:
 # distributed plumbing (replicas only: a barrier and a max over timings)
 # ---------------------------------------------------------------------------
 class Dist:
-    def __init__(self):
+    """Replica plumbing: one process per GPU, a barrier around the timed
+    region and max/sum reductions of scalars.  NCCL on GPUs; gloo (CPU
+    tensors) for the multi-process tests."""
+
+    def __init__(self, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
 
     def init(self):
@@ -78,9 +83,15 @@ class Dist:
 
             import torch.distributed as dist
 
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"timeout": datetime.timedelta(seconds=120)}
+            if self.backend == "nccl":
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, **kw)
             self.pg = dist
+
+    def _tensor(self, v: float) -> torch.Tensor:
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        return torch.tensor([v], dtype=torch.float64, device=dev)
 
     def barrier(self):
         if self.pg:
@@ -89,20 +100,28 @@ class Dist:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = self._tensor(v)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def sum(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = self._tensor(v)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def aggregate_throughput(bytes_per_rank_step: float, ms_per_step_this_rank: float, dist: Dist) -> tuple:
+    """Whole-job GB/s of replicas: every rank's bytes over the slowest rank's
+    time.  Returns (GB/s, max ms per step)."""
+    ms = dist.max(ms_per_step_this_rank)
+    total_bytes = dist.sum(bytes_per_rank_step)
+    return total_bytes / (ms * 1e-3) / 1e9, ms
 
 
 # ---------------------------------------------------------------------------
@@ -521,9 +540,9 @@ def main():
         for _ in range(20):
             g_step.replay()
         torch.cuda.synchronize()
-    ms_step = time_graph(g_step, args.steps, 0, dist)
+    ms_step_local = time_graph(g_step, args.steps, 0, dist)
     clk = clocks.stop()
-    ms_step = dist.max(ms_step)
+    value, ms_step = aggregate_throughput(path_b, ms_step_local, dist)
 
     # ---- the dominant kernel (GEMM alone), same calls --------------------
     g_gemm = ds.capture(lambda: ds.step(gemm_only=True))
@@ -564,7 +583,6 @@ def main():
     del layers
 
     world = dist.world
-    value = path_b * world / (ms_step * 1e-3) / 1e9
     gemm_gbs = gemm_b / (ms_gemm * 1e-3) / 1e9
     launches = ds.launches_per_step() * args.steps
 
