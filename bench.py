@@ -309,7 +309,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
                      "gbs": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / peak_gbs, 4),
                      "tflops": round(f / (ms * 1e-3) / 1e12, 2),
                      "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
-                              f"{'pers' if p['schedule'] == 1 else 's' + str(p['split_k'])}/r{p['reduce']}/st{p['stages']}")})
+                              f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
+                              f"/r{p['reduce']}/st{p['stages']}")})
     return rows
 
 
@@ -606,7 +607,10 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "GEMM (swapab/standard, all calls of the sweep)",
                      "achieved": round(gemm_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gemm_gbs / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-                     "traffic": (float(traffic["dram_bytes_per_launch"]) if traffic else None),
+                     # DRAM bytes per launch: the captured case's DRAM/algorithmic ratio
+                     # times this workload's algorithmic bytes per launch
+                     "traffic": (round(float(traffic["dram_over_algorithmic"]) * gemm_b / len(ds.calls))
+                                 if traffic else None),
                      "traffic_case": (traffic.get("case") if traffic else None),
                      "avg_launch_us": round(ms_gemm * 1e3 / len(ds.calls), 3),
                      "algorithmic_bytes_per_launch": round(gemm_b / len(ds.calls))},

@@ -90,8 +90,11 @@ typedef struct {
   int reduce;   /* qgd_reduce, used when several CTAs share an output tile */
   int stages;   /* depth of the shared-memory operand ring */
   int tile_n;   /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */
-  int schedule; /* qgd_schedule (never AUTO here) */
-  int source;   /* 0 = built-in default, 1 = dispatch table, 2 = override */
+  int schedule;  /* qgd_schedule (never AUTO here) */
+  int occupancy; /* persistent schedule: CTAs per SM the grid is sized for (1 or 2).  With 1 and a
+                    ring under half the SM's shared memory, the next GEMM's CTA can be resident
+                    beside this one and stream its first weights while this one finishes */
+  int source;    /* 0 = built-in default, 1 = dispatch table, 2 = override */
 } qgd_plan;
 
 /* ---------------------------------------------------------------------
@@ -179,10 +182,10 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
 
 /* Load a dispatch table: a text file with one line per (format, N, K,
  * M-bucket) and '#' comments,
- *     fmt N K M_bucket variant split_k reduce stages tile_n schedule
+ *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy
  * fmt in {fp8_dynamic, w8a8_int8, block_fp8}; variant in {standard, swap_ab};
  * reduce in {last_cta, two_pass, atomic}; schedule in {grid, persistent};
- * stages/tile_n 0 = default.  Replaces the table in force.  On
+ * stages/tile_n/occupancy 0 = default.  Replaces the table in force.  On
  * QGD_ERR_TABLE the table in force is unchanged.  Not thread-safe against
  * concurrent qlinear_* calls. */
 QGD_API qgd_status qgd_load_dispatch_table(const char* path);
@@ -191,10 +194,10 @@ QGD_API qgd_status qgd_load_dispatch_table(const char* path);
 QGD_API qgd_status qgd_clear_dispatch_table(void);
 
 /* Force a plan for one format (tests and the tuner).  Any argument < 0 keeps
- * the table/default choice for that field; stages/tile_n 0 = default.
- * qgd_set_override(fmt, -1, -1, -1, 0, 0, -1) removes the override. */
+ * the table/default choice for that field; stages/tile_n/occupancy 0 =
+ * default.  qgd_set_override(fmt, -1, -1, -1, 0, 0, -1, 0) removes it. */
 QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n,
-                                    int schedule);
+                                    int schedule, int occupancy);
 
 /* The plan a qlinear_* call with these arguments would run. */
 QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);

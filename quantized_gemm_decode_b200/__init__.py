@@ -59,7 +59,7 @@ class QGDError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
                 ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("schedule", ctypes.c_int),
-                ("source", ctypes.c_int)]
+                ("occupancy", ctypes.c_int), ("source", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -83,7 +83,7 @@ def lib() -> ctypes.CDLL:
             "qlinear_fp8_dynamic_noalloc": [P, P, P, P, P, I, I, I, P],
             "qgd_load_dispatch_table": [ctypes.c_char_p],
             "qgd_clear_dispatch_table": [],
-            "qgd_set_override": [I, I, I, I, I, I, I],
+            "qgd_set_override": [I, I, I, I, I, I, I, I],
             "qgd_get_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
             "qgd_device_error": [ctypes.POINTER(ctypes.c_uint)],
             "qgd_clear_device_error": [],
@@ -305,10 +305,11 @@ def qgd_clear_dispatch_table() -> None:
 
 
 def qgd_set_override(fmt: int, variant: int = -1, split_k: int = -1, reduce: int = -1, stages: int = 0,
-                     tile_n: int = 0, schedule: int = -1) -> None:
+                     tile_n: int = 0, schedule: int = -1, occupancy: int = 0) -> None:
     """Force plan fields for one format; every default argument leaves that
     field to the dispatch table / built-in default."""
-    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n, schedule), "qgd_set_override")
+    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n, schedule, occupancy),
+           "qgd_set_override")
 
 
 def qgd_get_plan(fmt: int, M: int, N: int, K: int) -> dict:

@@ -111,13 +111,13 @@ constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
 
 struct Entry {
-  int variant, split_k, reduce, stages, tile_n, schedule;
+  int variant, split_k, reduce, stages, tile_n, schedule, occupancy;
 };
 using Key = std::tuple<int, int, int, int>;
 std::mutex g_mu;
 std::map<Key, Entry> g_table;
 struct Override {
-  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1;
+  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1, occupancy = 0;
 } g_override[3];
 
 int bucket_of(int M) {
@@ -165,6 +165,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   p.reduce = kLastCta;
   p.stages = 0;
   p.schedule = kGrid;
+  p.occupancy = 0;
   if (M <= kDecodeMaxM) {
     // Decode: Swap-AB (the hand-written rule the method replaces with
     // measurement), persistent over all (tile, K-slice) units so that every
@@ -194,16 +195,19 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       p.stages = e.stages;
       p.tile_n = e.tile_n;
       p.schedule = e.schedule;
+      p.occupancy = e.occupancy;
       p.source = 1;
     }
     const Override& o = g_override[fmt];
-    if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0 || o.schedule >= 0) {
+    if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0 || o.schedule >= 0 ||
+        o.occupancy > 0) {
       if (o.variant >= 0) p.variant = o.variant;
       if (o.split_k >= 0) p.split_k = o.split_k;
       if (o.reduce >= 0) p.reduce = o.reduce;
       if (o.stages > 0) p.stages = o.stages;
       if (o.tile_n > 0) p.tile_n = o.tile_n;
       if (o.schedule >= 0) p.schedule = o.schedule;
+      if (o.occupancy > 0) p.occupancy = o.occupancy;
       p.source = 2;
     }
   }
@@ -228,6 +232,18 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad) : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
+  // CTAs per SM for the persistent grid: at most what shared memory (and, for
+  // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
+  int fit = 1;
+  if (p.schedule == kPersistent) {
+    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages)
+                                               : standard_smem_bytes(p.tile_n, p.stages)) + 1024;
+    fit = static_cast<int>(kSmemPerSM / bytes);
+    fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
+    if (p.variant == kStandard && (p.tile_n == 256 || fmt == kFmtBlock)) fit = 1;  // all 512 TMEM columns
+  }
+  if (p.occupancy <= 0 || p.occupancy > fit) p.occupancy = fit;
+  if (p.schedule != kPersistent) p.occupancy = 1;
   return p;
 }
 
@@ -258,9 +274,7 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
     e.tiles = n_tiles;
     if (p.schedule == kPersistent) {
       const long long U = static_cast<long long>(n_tiles) * nkt;
-      int occ = static_cast<int>(kSmemPerSM / (swapab_smem_bytes(e.mpad, p.stages) + 1024));
-      occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);  // registers allow at most 2 CTAs per SM
-      const long long cap = static_cast<long long>(g_num_sms) * occ;
+      const long long cap = static_cast<long long>(g_num_sms) * p.occupancy;
       const long long G = U < cap ? U : cap;
       e.persistent = true;
       e.ctas = static_cast<int>(G);
@@ -286,10 +300,7 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
       // accumulators take all 512 TMEM columns (2 x 256, or Block_FP8's
       // 4 x 128) leaves room for no second CTA on its SM
       const long long items = static_cast<long long>(e.tiles) * p.split_k;
-      int occ = static_cast<int>(kSmemPerSM / (standard_smem_bytes(p.tile_n, p.stages) + 1024));
-      occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);
-      if (p.tile_n == 256 || fmt == kFmtBlock) occ = 1;
-      const long long cap = static_cast<long long>(g_num_sms) * occ;
+      const long long cap = static_cast<long long>(g_num_sms) * p.occupancy;
       e.persistent = true;
       e.ctas = static_cast<int>(items < cap ? items : cap);
     }
@@ -533,11 +544,12 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (hash != std::string::npos) line.resize(hash);
     std::istringstream ls(line);
     std::string fmt_s, var_s, red_s, sch_s;
-    int N, K, Mb, split, stages, tile_n;
+    int N, K, Mb, split, stages, tile_n, occ;
     if (!(ls >> fmt_s)) continue;  // blank line
-    if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s))
+    if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s >> occ))
       return fail(QGD_ERR_TABLE,
-                  "%s:%d: expected 10 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule",
+                  "%s:%d: expected 11 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
+                  "occupancy",
                   path, lineno);
     std::string extra;
     if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
@@ -549,9 +561,10 @@ qgd_status qgd_load_dispatch_table(const char* path) {
       return fail(QGD_ERR_TABLE, "%s:%d: bad N/K or M bucket %d", path, lineno, Mb);
     if (split < 1 || split > 256 || (split & (split - 1)) != 0)
       return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256", path, lineno, split);
-    if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256))
-      return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n", path, lineno);
-    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch};
+    if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
+        occ > 2)
+      return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ};
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_table.swap(t);
@@ -564,10 +577,11 @@ qgd_status qgd_clear_dispatch_table(void) {
   return QGD_OK;
 }
 
-qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule) {
+qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule,
+                            int occupancy) {
   if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
-      (tile_n != 0 && tile_n != 128 && tile_n != 256))
+      occupancy < 0 || occupancy > 2 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");
   if (split_k > 0 && (split_k & (split_k - 1)) != 0) return fail(QGD_ERR_INVALID, "split_k must be a power of two");
   std::lock_guard<std::mutex> lk(g_mu);
@@ -578,6 +592,7 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
   o.stages = stages;
   o.tile_n = tile_n;
   o.schedule = schedule < 0 ? -1 : schedule;
+  o.occupancy = occupancy;
   return QGD_OK;
 }
 

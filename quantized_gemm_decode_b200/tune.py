@@ -56,27 +56,28 @@ SCHED_NAME = {0: "grid", 1: "persistent"}
 
 
 def candidates(fmt: str, M: int, N: int, K: int):
-    """(variant, split_k, reduce, tile_n, schedule) tuples legal for the shape."""
+    """(variant, split_k, reduce, tile_n, schedule, occupancy) tuples legal for the shape."""
     nkt = (K + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
     out = []
     if M <= 32:
         for r in (0, 1, 2):
-            out.append((1, 1, r, 128, 1))  # Swap-AB, persistent
+            for occ in (1, 2):
+                out.append((1, 1, r, 128, 1, occ))  # Swap-AB, persistent, 1 or 2 CTAs per SM
         for s in splits:
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((1, s, r, 128, 0))
+                out.append((1, s, r, 128, 0, 0))
     tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
     for t in tiles:
         for s in splits:
             if M <= 32 and s > 16:
                 continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((0, s, r, t, 0))
+                out.append((0, s, r, t, 0, 0))
         for s in (1, 2):
             if s <= nkt:
                 for r in ((0,) if s == 1 else (0, 1)):
-                    out.append((0, s, r, t, 1))  # Standard, persistent
+                    out.append((0, s, r, t, 1, 0))  # Standard, persistent
     return out
 
 
@@ -133,14 +134,14 @@ class Problem:
 def tune_problem(p: Problem, log=None):
     fid = p.fid
     qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0,
-                         qgd.SCHEDULE_GRID)
+                         qgd.SCHEDULE_GRID, 0)
     p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
     ref = p.run().float().clone()
     ref_acc = p.acc32().clone() if p.fmt == W8A8_INT8 else None
     scale = ref.abs().max().item() + 1e-30
     results = []
-    for var, s, r, t, sch in candidates(p.fmt, p.M, p.N, p.K):
-        qgd.qgd_set_override(fid, var, s, r, 0, t, sch)
+    for var, s, r, t, sch, occ in candidates(p.fmt, p.M, p.N, p.K):
+        qgd.qgd_set_override(fid, var, s, r, 0, t, sch, occ)
         p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
         y = p.run().float()
         ok = (y - ref).abs().max().item() <= 2e-2 * scale
@@ -148,23 +149,24 @@ def tune_problem(p: Problem, log=None):
             ok = torch.equal(p.acc32(), ref_acc)
         if not ok:
             if log:
-                log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]}: "
+                log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]} occ={occ}: "
                     f"differs from the split-free result")
             continue
         us = p.time_plan()
         stages = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["stages"]
-        results.append((us, var, s, r, stages, t, sch))
+        results.append((us, var, s, r, stages, t, sch, occ))
     results.sort()
     # refine the pipeline depth of the three fastest
     refined = list(results[:3])
-    for us0, var, s, r, smax, t, sch in results[:3]:
-        for st in (2, 3, 4, 6, 8, 10):
+    for us0, var, s, r, smax, t, sch, occ in results[:3]:
+        for st in (2, 3, 4, 5, 6, 8, 10):
             if st >= smax:
                 continue
-            qgd.qgd_set_override(fid, var, s, r, st, t, sch)
+            qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ)
             p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
             us = p.time_plan()
-            refined.append((us, var, s, r, st, t, sch))
+            occ_eff = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["occupancy"]
+            refined.append((us, var, s, r, st, t, sch, occ_eff))
     refined.sort()
     qgd.qgd_set_override(fid)
     return refined[0], results
@@ -191,7 +193,7 @@ def main(argv=None):
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
             f = ln.split("#")[0].split()
-            if len(f) == 10:
+            if len(f) == 11:
                 done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
     only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
     t_start = time.time()
@@ -204,7 +206,7 @@ def main(argv=None):
         tmp = args.out + ".tmp"
         with open(tmp, "w") as f:
             f.write("# Dispatch table for B200 (sm_100a), measured by quantized_gemm_decode_b200.tune\n")
-            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule   # us/call\n")
+            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy   # us/call\n")
             for k in sorted(lines):
                 f.write(lines[k] + "\n")
         os.replace(tmp, args.out)
@@ -220,12 +222,12 @@ def main(argv=None):
                 t0 = time.time()
                 p = Problem(wl.fmt, M, N, K, wl.seed, device)
                 best, allres = tune_problem(p, log)
-                us, var, s, r, st, t, sch = best
+                us, var, s, r, st, t, sch, occ = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
-                lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]}"
-                              f"   # {us:.2f} us, {gbs:.0f} GB/s")
+                lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "
+                              f"{occ}   # {us:.2f} us, {gbs:.0f} GB/s")
                 log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
-                    f"{SCHED_NAME[sch]} {us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, "
+                    f"{SCHED_NAME[sch]} occ={occ} {us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, "
                     f"{time.time() - t0:.1f} s)")
                 del p
                 torch.cuda.empty_cache()

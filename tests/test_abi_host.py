@@ -133,7 +133,7 @@ def test_persistent_workspace_matches_unit_partition(M, N, K):
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, qgd.REDUCE_LAST_CTA, 0, 0,
                          qgd.SCHEDULE_PERSISTENT)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, M, N, K)
-    assert p["schedule"] == qgd.SCHEDULE_PERSISTENT
+    assert p["schedule"] == qgd.SCHEDULE_PERSISTENT and p["occupancy"] == 1
     # the deepest pipelines leave room for one CTA per SM (148 SMs)
     maxc, tiles = _persistent_geometry(N, K, 148)
     mstride = (M + 3) // 4 * 4
@@ -150,33 +150,34 @@ def test_too_many_tiles_for_counters_fall_back_to_two_pass():
 
 def test_table_load_and_lookup(tmp_path):
     t = tmp_path / "t.tsv"
-    t.write_text("# fmt N K M_bucket variant split_k reduce stages tile_n schedule\n"
-                 "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n"
+    t.write_text("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy\n"
+                 "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 0\n"
                  "\n"
-                 "w8a8_int8 5120 5120 32 swap_ab 4 atomic 0 0 persistent  # trailing comment\n")
+                 "w8a8_int8 5120 5120 32 swap_ab 4 atomic 3 0 persistent 2  # trailing comment\n")
     qgd.qgd_load_dispatch_table(str(t))
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 3, 4096, 4096)  # bucket 4
     assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["tile_n"], p["source"]) == (0, 2, 1, 4, 256, 1)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 5, 4096, 4096)  # bucket 8: not in the table
     assert p["source"] == 0
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)
-    assert (p["variant"], p["split_k"], p["reduce"], p["schedule"], p["source"]) == (1, 4, 2, 1, 1)
+    assert (p["variant"], p["split_k"], p["reduce"], p["schedule"], p["occupancy"], p["source"]) == (1, 4, 2, 1, 2, 1)
     qgd.qgd_clear_dispatch_table()
     assert qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 25, 5120, 5120)["source"] == 0
 
 
 @pytest.mark.parametrize("bad", [
-    "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256 grid\n",      # split not a power of two
-    "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256 grid\n",      # 5 is not a bucket
-    "fp9 4096 4096 4 standard 2 two_pass 4 256 grid\n",              # unknown format
-    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256\n",           # missing field
-    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 7\n",    # extra field
-    "fp8_dynamic 4096 4096 4 diagonal 2 two_pass 4 256 grid\n",      # unknown variant
-    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 stream\n",    # unknown schedule
+    "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256 grid 0\n",      # split not a power of two
+    "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256 grid 0\n",      # 5 is not a bucket
+    "fp9 4096 4096 4 standard 2 two_pass 4 256 grid 0\n",              # unknown format
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n",        # missing field
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 0 7\n",    # extra field
+    "fp8_dynamic 4096 4096 4 diagonal 2 two_pass 4 256 grid 0\n",      # unknown variant
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 stream 0\n",    # unknown schedule
+    "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 3\n",      # occupancy out of range
 ])
 def test_malformed_table_is_rejected_and_keeps_previous(tmp_path, bad):
     good = tmp_path / "good.tsv"
-    good.write_text("fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n")
+    good.write_text("fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid 0\n")
     qgd.qgd_load_dispatch_table(str(good))
     t = tmp_path / "bad.tsv"
     t.write_text(bad)
@@ -211,3 +212,19 @@ def test_argument_rejection_before_any_launch():
     # M == 0 is an empty, successful call
     assert L.qlinear_fp8_dynamic(None, None, None, None, None, 0, 512, 1024, None, 0, None) == 0
     assert b"16" in L.qgd_last_error_message() or L.qgd_last_error_message() is not None
+
+
+def test_persistent_occupancy_follows_shared_memory():
+    # deep rings fit one CTA per SM; shallow ones two, unless one is asked for
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 4, 0, qgd.SCHEDULE_PERSISTENT)
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["occupancy"] == 2
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 4, 0, qgd.SCHEDULE_PERSISTENT, 1)
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["occupancy"] == 1
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 10, 0, qgd.SCHEDULE_PERSISTENT, 2)
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["occupancy"] == 1  # 2 do not fit
+    # fewer CTAs share each tile with one CTA per SM: a smaller workspace
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 4, 0, qgd.SCHEDULE_PERSISTENT, 1)
+    one = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 4, 0, qgd.SCHEDULE_PERSISTENT, 2)
+    two = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+    assert 0 < one < two
