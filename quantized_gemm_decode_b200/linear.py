@@ -102,3 +102,76 @@ class QuantizedLinear:
             out.copy_(y, non_blocking=True)
             return out
         return y
+
+
+class DecodeStep:
+    """One decode step of several quantized linear layers captured as a single
+    CUDA graph, host I/O included: each layer's activations are copied from
+    pinned host memory on a copy stream (all copies issued up front), each
+    layer quantizes and multiplies on the compute stream as soon as its input
+    has landed, and each result is copied back to pinned host memory on a
+    second copy stream while the next layers compute.
+
+    `calls` is a list of (layer, M); `x_host[i]` / `y_host[i]` are pinned
+    host tensors of shape [M, K] / [M, N].  replay() runs the whole step
+    asynchronously on the current stream; synchronize before reading y_host.
+    """
+
+    def __init__(self, calls, x_host, y_host):
+        self.calls = list(calls)
+        dev = self.calls[0][0].device
+        self.x_dev, self.y_dev, self.q = [], [], []
+        for (layer, M) in self.calls:
+            self.x_dev.append(torch.empty((M, layer.K), dtype=torch.bfloat16, device=dev))
+            self.y_dev.append(torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev))
+            qdt = torch.int8 if layer.fmt == "w8a8_int8" else torch.float8_e4m3fn
+            xq = torch.empty((M, layer.K), dtype=qdt, device=dev)
+            sx = torch.empty((M, layer.K // 128) if layer.fmt == "block_fp8" else (M,), dtype=torch.float32,
+                             device=dev)
+            layer.ws.ensure(qgd.qgd_workspace_size(layer.fmt_id, M, layer.N, layer.K))
+            self.q.append((xq, sx))
+        self.x_host, self.y_host = list(x_host), list(y_host)
+        self.graph = torch.cuda.CUDAGraph()
+        main = torch.cuda.Stream(dev)
+        copy_in = torch.cuda.Stream(dev)
+        copy_out = torch.cuda.Stream(dev)
+        # warm up outside capture (loads the kernels, sizes the workspaces)
+        with torch.cuda.stream(main):
+            self._body(main, None, None)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(self.graph, stream=main):
+            self._body(main, copy_in, copy_out)
+
+    def _body(self, main, copy_in, copy_out):
+        if copy_in is None:
+            for i, (layer, M) in enumerate(self.calls):
+                self.x_dev[i].copy_(self.x_host[i], non_blocking=True)
+                xq, sx = self.q[i]
+                layer.quantize(self.x_dev[i], xq, sx)
+                layer.gemm(xq, sx, self.y_dev[i])
+                self.y_host[i].copy_(self.y_dev[i], non_blocking=True)
+            return
+        landed = []
+        copy_in.wait_stream(main)
+        copy_out.wait_stream(main)
+        with torch.cuda.stream(copy_in):
+            for i in range(len(self.calls)):
+                self.x_dev[i].copy_(self.x_host[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_in)
+                landed.append(ev)
+        for i, (layer, M) in enumerate(self.calls):
+            main.wait_event(landed[i])
+            xq, sx = self.q[i]
+            layer.quantize(self.x_dev[i], xq, sx)
+            layer.gemm(xq, sx, self.y_dev[i])
+            done = torch.cuda.Event()
+            done.record(main)
+            copy_out.wait_event(done)
+            with torch.cuda.stream(copy_out):
+                self.y_host[i].copy_(self.y_dev[i], non_blocking=True)
+        main.wait_stream(copy_in)
+        main.wait_stream(copy_out)
+
+    def replay(self):
+        self.graph.replay()
