@@ -973,15 +973,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ===========================================================================
 template <int kFmt>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
+  // four adjacent outputs per thread (N % 16 == 0 keeps them in one row);
+  // up to eight splits' partials in flight before they are added in order
   griddep_wait();
   const size_t total = static_cast<size_t>(a.M) * a.N;
-  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total) return;
-  const uint32_t* p = static_cast<const uint32_t*>(a.partial);
-  uint32_t v = p[idx];
-  for (int s = 1; s < a.splits; ++s) v = add_acc<kFmt>(v, p[static_cast<size_t>(s) * total + idx]);
+  const size_t quad = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (quad * 4 >= total) return;
+  const uint4* p = reinterpret_cast<const uint4*>(a.partial);
+  const size_t stride = total / 4;
+  uint32_t acc[4];
+  for (int s0 = 0; s0 < a.splits; s0 += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (s0 + j < a.splits) v[j] = p[static_cast<size_t>(s0 + j) * stride + quad];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (s0 + j < a.splits) {
+        if (s0 + j == 0) {
+          acc[0] = v[j].x; acc[1] = v[j].y; acc[2] = v[j].z; acc[3] = v[j].w;
+        } else {
+          acc[0] = add_acc<kFmt>(acc[0], v[j].x);
+          acc[1] = add_acc<kFmt>(acc[1], v[j].y);
+          acc[2] = add_acc<kFmt>(acc[2], v[j].z);
+          acc[3] = add_acc<kFmt>(acc[3], v[j].w);
+        }
+      }
+    }
+  }
+  const size_t idx = quad * 4;
   const int m = static_cast<int>(idx / a.N), n = static_cast<int>(idx % a.N);
-  store_final<kFmt>(v, m, n, a);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) store_final<kFmt>(acc[j], m, n + j, a);
 }
 
 // Launch with dynamic shared memory and, when `pdl` is set, a programmatic
@@ -1099,7 +1122,7 @@ cudaError_t clear_device_error() {
 
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream) {
   const size_t total = static_cast<size_t>(a.M) * a.N;
-  const unsigned blocks = static_cast<unsigned>((total + 255) / 256);
+  const unsigned blocks = static_cast<unsigned>((total / 4 + 255) / 256);
   const bool pdl = a.pdl != 0;
   if (fmt == kFmtFP8) return launch_ex(splitk_reduce_kernel<kFmtFP8>, dim3(blocks), dim3(256), 0, stream, pdl, a);
   if (fmt == kFmtINT8) return launch_ex(splitk_reduce_kernel<kFmtINT8>, dim3(blocks), dim3(256), 0, stream, pdl, a);
