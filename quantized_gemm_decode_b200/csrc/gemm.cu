@@ -38,16 +38,18 @@ namespace {
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_device_error, 0u, code); }
 
 // Developer timeline of the Swap-AB kernel: with -DQGD_TRACE each CTA stamps
-// %globaltimer at eight points (entry, set-up done, first loads issued, first
-// stage landed, last MMA committed, last accumulator read, epilogue done,
-// exit); qgd_debug_trace() copies the stamps out.  Compiled out otherwise.
+// %globaltimer at up to 16 points (entry, set-up done, first loads issued,
+// first stage landed, last MMA committed, last accumulator read, epilogue
+// done, exit, and the steps of the last segment's output);
+// qgd_debug_trace() copies the stamps out.  Compiled out otherwise.
 #ifdef QGD_TRACE
 constexpr int kTraceCtas = 4096;
-__device__ unsigned long long g_trace[kTraceCtas * 8];
+constexpr int kTraceSlots = 16;
+__device__ unsigned long long g_trace[kTraceCtas * kTraceSlots];
 #define QGD_STAMP(slot)                                                             \
   do {                                                                              \
     const unsigned cta_ = blockIdx.x + blockIdx.y * gridDim.x;                      \
-    if (cta_ < kTraceCtas) g_trace[cta_ * 8 + (slot)] = globaltimer_ns();           \
+    if (cta_ < kTraceCtas) g_trace[cta_ * kTraceSlots + (slot)] = globaltimer_ns(); \
   } while (0)
 #else
 #define QGD_STAMP(slot) \
@@ -68,6 +70,7 @@ struct SmemCtl {
   int abort_flag;
   int last_flag;
   int epi_ok;
+  float sx_s[32];  // Swap-AB, per-token formats: the M token scales, staged once
 };
 static_assert(sizeof(SmemCtl) <= kBarBytes, "control block too large");
 
@@ -134,6 +137,24 @@ __device__ __forceinline__ void store_final(uint32_t accbits, int m, int n, cons
     static_cast<uint32_t*>(a.raw)[idx] = accbits;
   } else {
     a.y[idx] = bf16_bits(scale_out<kFmt>(accbits, m, n, a));
+  }
+}
+
+// Swap-AB output of one element from on-chip operands only: token scale from
+// shared memory, channel scale prefetched into a register.  Same arithmetic
+// as scale_out: ((acc * sx[m]) * sw[n]) for the per-token formats.
+template <int kFmt>
+__device__ __forceinline__ void store_swap_final(uint32_t accbits, int m, int n, float swv, const float* sx_s,
+                                                 const GemmArgs& a) {
+  const size_t idx = static_cast<size_t>(m) * a.N + n;
+  if (a.raw) {
+    static_cast<uint32_t*>(a.raw)[idx] = accbits;
+  } else if constexpr (kFmt == kFmtBlock) {
+    a.y[idx] = bf16_bits(__uint_as_float(accbits));
+  } else if constexpr (kFmt == kFmtINT8) {
+    a.y[idx] = bf16_bits((static_cast<float>(static_cast<int32_t>(accbits)) * sx_s[m]) * swv);
+  } else {
+    a.y[idx] = bf16_bits((__uint_as_float(accbits) * sx_s[m]) * swv);
   }
 }
 
@@ -274,6 +295,37 @@ __device__ __forceinline__ void fixup_sum_t(const GemmArgs& a, int t, int row, i
               sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
             }
           }
+        }
+      }
+    }
+  }
+}
+
+// The same sum through shared memory: every contributor's partial row is
+// requested at once with cp.async into this thread's own area of `stage`
+// (no register cost while in flight), then added from shared memory in
+// contributor order.  `stage` must hold 128 * ncontrib * nvec * 16 bytes.
+template <int kFmt, int kMpad>
+__device__ __forceinline__ void fixup_sum_smem(const GemmArgs& a, int t, int row, int ncontrib, int nvec,
+                                               uint8_t* stage, uint32_t (&sum)[kMpad]) {
+  uint4* mine = reinterpret_cast<uint4*>(stage) + static_cast<size_t>(row) * ncontrib * nvec;
+  for (int j = 0; j < ncontrib; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j, row));
+    for (int v = 0; v < nvec; ++v) cp_async16(mine + j * nvec + v, src + v);
+  }
+  cp_async_wait_all();
+  for (int j = 0; j < ncontrib; ++j) {
+#pragma unroll
+    for (int v = 0; v < kMpad / 4; ++v) {
+      if (v < nvec) {
+        const uint4 w4 = mine[j * nvec + v];
+        if (j == 0) {
+          sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+        } else {
+          sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+          sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+          sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+          sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
         }
       }
     }
@@ -463,6 +515,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int M = a.M, N = a.N;
     const int KB = a.K / kTileK;
     const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
+    const bool scaled = (kFmt != kFmtBlock) && !a.raw;
+    if (scaled && threadIdx.x - 64 < static_cast<unsigned>(M)) ctl->sx_s[threadIdx.x - 64] = __ldg(a.sx + threadIdx.x - 64);
+    epi_sync();
     int i = 0, seg = 0;
     while (i < nk) {
       const long long u = ub + i;
@@ -470,6 +525,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       const int kt_first = static_cast<int>(u % nkt);
       const int len = (nkt - kt_first) < (nk - i) ? (nkt - kt_first) : (nk - i);
       const int n = t * kSwapTileN + row;
+      // the channel scale is known before the accumulator is: fetch it now
+      const float swv = (scaled && n < N) ? __ldg(a.sw + n) : 0.f;
       uint32_t acc[kMpad];
       if constexpr (kBlock) {
         float facc[kMpad];
@@ -520,14 +577,16 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       if (threadIdx.x == 64 && i + len >= nk) QGD_STAMP(5);
 
       const bool in_n = n < N;
+      const bool last_seg = i + len >= nk;
       int ncontrib, jslot;
       tile_contributors(a, t, nkt, U, cta, ncontrib, jslot);
       if (ncontrib == 1) {
         if (in_n) {
 #pragma unroll
           for (int m = 0; m < kMpad; ++m)
-            if (m < M) store_final<kFmt>(acc[m], m, n, a);
+            if (m < M) store_swap_final<kFmt>(acc[m], m, n, swv, ctl->sx_s, a);
         }
+        if (threadIdx.x == 64 && last_seg) QGD_STAMP(8);
       } else {
         if (in_n) {
           if (a.reduce == kAtomic) {
@@ -541,21 +600,33 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
               if (v < nvec) dst[v] = make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
           }
         }
+        if (threadIdx.x == 64 && last_seg) QGD_STAMP(9);
         if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, t, ncontrib)) {
+          if (threadIdx.x == 64 && last_seg) QGD_STAMP(10);
           if (in_n) {
             if (a.reduce == kAtomic) {
-#pragma unroll
+#pragma unroll 4
               for (int m = 0; m < kMpad; ++m)
-                if (m < M) store_final<kFmt>(ldcg_u32(static_cast<uint32_t*>(a.accum) + static_cast<size_t>(m) * N + n), m, n, a);
+                if (m < M)
+                  store_swap_final<kFmt>(ldcg_u32(static_cast<uint32_t*>(a.accum) + static_cast<size_t>(m) * N + n),
+                                         m, n, swv, ctl->sx_s, a);
             } else {
               uint32_t sum[kMpad];
-              fixup_sum<kFmt, kMpad>(a, t, row, ncontrib, nvec, -1, acc, sum);  // own partial re-read from L2
+              // in the CTA's last segment every ring stage has been consumed,
+              // so the ring's shared memory can stage the partials
+              const size_t ring_bytes = static_cast<size_t>(stages) * (kWBytes + kXBytes);
+              if (last_seg && static_cast<size_t>(kSwapTileN) * ncontrib * nvec * 16 <= ring_bytes)
+                fixup_sum_smem<kFmt, kMpad>(a, t, row, ncontrib, nvec, w_ring, sum);
+              else
+                fixup_sum<kFmt, kMpad>(a, t, row, ncontrib, nvec, -1, acc, sum);  // own partial re-read from L2
+              if (threadIdx.x == 64 && last_seg) QGD_STAMP(11);
 #pragma unroll
               for (int m = 0; m < kMpad; ++m)
-                if (m < M) store_final<kFmt>(sum[m], m, n, a);
+                if (m < M) store_swap_final<kFmt>(sum[m], m, n, swv, ctl->sx_s, a);
             }
           }
           if (threadIdx.x == 64) a.tickets[t] = 0u;
+          if (threadIdx.x == 64 && last_seg) QGD_STAMP(12);
         }
       }
       i += len;
@@ -1106,7 +1177,8 @@ cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CU
 
 #ifdef QGD_TRACE
 extern "C" __attribute__((visibility("default"))) int qgd_debug_trace(unsigned long long* host, size_t count) {
-  const size_t n = count < static_cast<size_t>(kTraceCtas) * 8 ? count : static_cast<size_t>(kTraceCtas) * 8;
+  const size_t cap = static_cast<size_t>(kTraceCtas) * kTraceSlots;
+  const size_t n = count < cap ? count : cap;
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)));
 }
 #endif
