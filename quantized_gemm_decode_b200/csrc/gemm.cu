@@ -189,14 +189,15 @@ __device__ __forceinline__ void teardown(SmemCtl* ctl, int warp, int lane, int i
   }
 }
 
-// Epilogue-only barrier (the 128 threads of warps 2..5).
-__device__ __forceinline__ void epi_sync() { named_bar_sync(1, 128); }
+// Epilogue-only barrier: the epilogue warps are warps 2.. of the CTA
+// (128 threads, or 256 for the Block_FP8 Standard kernel).
+__device__ __forceinline__ void epi_sync(uint32_t nthreads = 128) { named_bar_sync(1, nthreads); }
 
 // After the epilogue's waits: agree (uniformly) on whether to write output.
-__device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl) {
-  epi_sync();
+__device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl, uint32_t nthreads = 128) {
+  epi_sync(nthreads);
   if (threadIdx.x == 64) ctl->epi_ok = (ctl->abort_flag == 0);
-  epi_sync();
+  epi_sync(nthreads);
   return ctl->epi_ok != 0;
 }
 
@@ -205,14 +206,15 @@ __device__ __forceinline__ bool epi_agree_ok(SmemCtl* ctl) {
 // barrier orders every epilogue thread's stores before one thread's
 // acquire-release atomic at GPU scope, and the barrier after it orders that
 // acquire before the last CTA's reads of the other partials.
-__device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile, int expected) {
-  epi_sync();
+__device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a, int tile, int expected,
+                                                uint32_t nthreads = 128) {
+  epi_sync(nthreads);
   if (threadIdx.x == 64) {
     unsigned int old;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.tickets + tile) : "memory");
     ctl->last_flag = (old == static_cast<unsigned int>(expected - 1));
   }
-  epi_sync();
+  epi_sync(nthreads);
   return ctl->last_flag != 0;
 }
 
@@ -663,11 +665,11 @@ __global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArg
 
 // Last CTA of a Standard tile: add the split partials (or read the atomic
 // sum) for this thread's token row, 16 columns at a time, in split order.
-template <int kFmt, int kTileN>
+template <int kFmt, int kCols>
 __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0, bool in_m) {
   if (!in_m) return;
   const int M = a.M, N = a.N;
-  for (int nc = n0; nc < n0 + kTileN && nc < N; nc += 16) {
+  for (int nc = n0; nc < n0 + kCols && nc < N; nc += 16) {
     const size_t idx = static_cast<size_t>(m) * N + nc;
     uint32_t v[16];
     if (a.reduce == kAtomic) {
@@ -712,13 +714,23 @@ __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0
 // persist and the TMEM accumulator is double-buffered, so the epilogue of
 // one tile overlaps the mainloop of the next.
 // ===========================================================================
+// Threads of the Standard kernel: producer warp, MMA warp, then 4 epilogue
+// warps -- 8 for Block_FP8, whose per-K-block promotion is the busiest part
+// (two warps per TMEM lane quadrant, each taking half the columns).
+template <int kFmt>
+__host__ __device__ constexpr int std_threads() {
+  return kFmt == kFmtBlock ? 64 + 256 : kGemmThreads;
+}
+
 template <int kFmt, int kTileN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     standard_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                     const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
   static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
+  constexpr uint32_t kEpi = std_threads<kFmt>() - 64;  // epilogue threads
+  constexpr int kHalf = kBlock ? kTileN / 2 : kTileN;   // columns per epilogue thread
   // Block_FP8: a ring of 4 per-K-block accumulators (the MMA runs up to three
   // K blocks ahead of the promotion); else: a per-tile double buffer.
   constexpr int kSlots = kBlock ? 4 : 2;
@@ -750,7 +762,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&ctl->tfull[i], 1);
-      mbar_init(&ctl->tempty[i], 128);
+      mbar_init(&ctl->tempty[i], kEpi);
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
@@ -862,9 +874,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..) ----------------
     griddep_wait();  // scales and outputs: only after the preceding kernel is done
     const int q = warp & 3;
+    const int half = kBlock ? (warp - 2) / 4 : 0;  // Block_FP8: which half of the columns
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int M = a.M, N = a.N;
     int i = 0, li = 0;
@@ -874,14 +887,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
       const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
       const int m = m_tile * kStdTileM + q * 32 + lane;  // TMEM lane = token row
-      const int n0 = n_tile * kTileN;
+      const int n0 = n_tile * kTileN + half * kHalf;     // this thread's first column
       const bool in_m = m < M;
 
       if constexpr (kBlock) {
         const int KB = a.K / kTileK;
-        float facc[kTileN];
+        float facc[kHalf];
 #pragma unroll
-        for (int j = 0; j < kTileN; ++j) facc[j] = 0.f;
+        for (int j = 0; j < kHalf; ++j) facc[j] = 0.f;
         const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
         const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
         for (int kt = kt0; kt < kt1; ++kt, ++i) {
@@ -895,27 +908,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          // four TMEM loads in flight per wait
-#pragma unroll
-          for (int h = 0; h < kTileN / 64; ++h) {
+          // this thread's 64 columns: four TMEM loads per wait
+          {
             uint32_t r[4][16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld16(taddr + slot * kTileN + h * 64 + c * 16, r[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld16(taddr + slot * kTileN + half * kHalf + c * 16, r[c]);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                facc[h * 64 + c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[h * 64 + c * 16 + j]);
+              for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[c * 16 + j]);
           }
           tc_fence_before();
           mbar_arrive(&ctl->tempty[slot]);
         }
-        if (!epi_agree_ok(ctl)) break;
+        if (!epi_agree_ok(ctl, kEpi)) break;
         if (S == 1) {
           if (in_m) {
 #pragma unroll
-            for (int c = 0; c < kTileN / 16; ++c) {
+            for (int c = 0; c < kHalf / 16; ++c) {
               const int nc = n0 + c * 16;
               if (nc >= N) break;
               if (a.raw) {
@@ -939,7 +950,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
           if (in_m) {
 #pragma unroll
-            for (int c = 0; c < kTileN / 16; ++c) {
+            for (int c = 0; c < kHalf / 16; ++c) {
               const int nc = n0 + c * 16;
               if (nc >= N) break;
               const size_t idx = static_cast<size_t>(m) * N + nc;
@@ -955,8 +966,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           }
-          if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, tile, S)) {
-            std_reduce_tile<kFmt, kTileN>(a, m, n0, in_m);
+          if (a.reduce != kTwoPass && epi_arrive_last(ctl, a, tile, S, kEpi)) {
+            std_reduce_tile<kFmt, kHalf>(a, m, n0, in_m);
             if (threadIdx.x == 64) a.tickets[tile] = 0u;
           }
         }
@@ -1148,7 +1159,7 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
   const long long items = static_cast<long long>((a.N + kTileN - 1) / kTileN) *
                           ((a.M + kStdTileM - 1) / kStdTileM) * a.splits;
   const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
-  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(kGemmThreads), standard_smem_bytes(kTileN, a.stages),
+  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(std_threads<kFmt>()), standard_smem_bytes(kTileN, a.stages),
                    stream, a.pdl != 0, tx, tw, a);
 }
 
