@@ -288,9 +288,24 @@ def time_graph(g: torch.cuda.CUDAGraph, steps: int, warmup: int, dist: Dist | No
     return t0.elapsed_time(t1) / steps
 
 
+def replay_times(g: torch.cuda.CUDAGraph, reps: int, warmup: int = 3) -> list:
+    """Milliseconds of each of `reps` replays (CUDA events around each)."""
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record()
+    for i in range(reps):
+        g.replay()
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+
+
 def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
-    """GEMM-only time of each call, cycling through all weight copies of its
-    shape (at least 3x L2 of distinct weights), one graph per call."""
+    """Time of each call, cycling through all weight copies of its shape (at
+    least 3x L2 of distinct weights), one graph per call: the GEMM alone (mean
+    and p90 over replays) and the whole layer call (quantize + GEMM)."""
     rows = []
     for c in ds.calls:
         ncop = len(ds.weights[(c["N"], c["K"])])
@@ -299,19 +314,72 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
             for j in range(ncop):
                 ds.gemm(c, copy_idx=j)
 
+        def layer(c=c, ncop=ncop):
+            for j in range(ncop):
+                ds.quant(c)
+                ds.gemm(c, copy_idx=j)
+
         g = ds.capture(body)
-        ms = time_graph(g, reps, 3) / ncop
+        times = replay_times(g, reps)
+        ms = statistics.mean(times) / ncop
+        p90 = sorted(times)[int(0.9 * (len(times) - 1))] / ncop
+        del g
+        g = ds.capture(layer)
+        ms_layer = statistics.mean(replay_times(g, reps)) / ncop
         del g
         b = workloads.algorithmic_bytes(ds.fmt, c["M"], c["N"], c["K"])
         f = workloads.flops(c["M"], c["N"], c["K"])
         p = ds.qgd.qgd_get_plan(ds.fmt_id, c["M"], c["N"], c["K"])
-        rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3),
+        pb = path_bytes(ds.fmt, c["M"], c["N"], c["K"])
+        rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3), "p90_us": round(p90 * 1e3, 3),
                      "gbs": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / peak_gbs, 4),
                      "tflops": round(f / (ms * 1e-3) / 1e12, 2),
+                     "layer_us": round(ms_layer * 1e3, 3),
+                     "layer_gbs": round(pb / (ms_layer * 1e-3) / 1e9, 1),
                      "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
                               f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
-                              f"/r{p['reduce']}/st{p['stages']}")})
+                              f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}")})
     return rows
+
+
+def quant_bytes(fmt: str, M: int, K: int) -> int:
+    """Algorithmic bytes of the activation quantizer: bf16 X in, codes and scales out."""
+    return 2 * M * K + M * K + (4 * M * (K // 128) if fmt == BLOCK_FP8 else 4 * M)
+
+
+def quantizer_summary(ds: DecodeSet, reps: int = 20):
+    """The activation quantizer on its own: every call's quantizer of the
+    sweep in one graph."""
+    g = ds.capture(lambda: [ds.quant(c) for c in ds.calls])
+    ms = statistics.mean(replay_times(g, reps))
+    del g
+    b = sum(quant_bytes(ds.fmt, c["M"], c["K"]) for c in ds.calls)
+    return {"us_per_call": round(ms * 1e3 / len(ds.calls), 3), "bytes_per_step": b,
+            "gbs": round(b / (ms * 1e-3) / 1e9, 1)}
+
+
+def tensor_probe(reps: int = 3, iters: int = 8192) -> dict:
+    """Dense e4m3 / int8 tensor rate of this GPU from the library's tcgen05
+    peak probe (best of `reps` launches)."""
+    import quantized_gemm_decode_b200 as qgd
+
+    out = {}
+    for name, qt in (("e4m3_tflops", qgd.QTYPE_E4M3), ("int8_tops", qgd.QTYPE_INT8)):
+        qgd.qgd_mma_peak_probe(qt, 64)
+        best = 0.0
+        for _ in range(reps):
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            f = qgd.qgd_mma_peak_probe(qt, iters)
+            t1.record()
+            torch.cuda.synchronize()
+            best = max(best, f / (t0.elapsed_time(t1) * 1e-3) / 1e12)
+        out[name] = round(best, 1)
+    assert qgd.qgd_device_error() == 0
+    out["how"] = (f"qgd_mma_peak_probe: one CTA per SM, {iters} x 4 back-to-back tcgen05.mma (128x256x32) "
+                  f"from shared memory, best of {reps}")
+    return out
 
 
 def format_summary(ds: DecodeSet, steps: int, warmup: int, peak_gbs: float):
@@ -324,8 +392,14 @@ def format_summary(ds: DecodeSet, steps: int, warmup: int, peak_gbs: float):
             "tflops": round(flops / (ms * 1e-3) / 1e12, 3)}
 
 
-def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5):
-    """Compute-bound regime: one GEMM per (M, N, K) of the larger-M config."""
+SPEC_TENSOR_TFLOPS = 4500.0  # dense e4m3 / int8 data-sheet figure
+
+
+def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict | None = None):
+    """Compute-bound regime: one GEMM per (M, N, K) of the larger-M config.
+    frac: against 2x the measured bf16 peak (the nominal e4m3:bf16 ratio);
+    frac_probe: against the tcgen05 probe's rate for this operand type;
+    frac_spec: against the 4.5 PFLOP/s data-sheet figure."""
     import quantized_gemm_decode_b200 as qgd
 
     wl = [w for w in workloads.LARGE if w.fmt == fmt][0]
@@ -367,9 +441,15 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5):
             f = workloads.flops(M, N, K)
             t_roof = max(b / (peaks_["hbm_gbs"] * 1e9), f / (peak_tc * 1e12))
             bound = "tensor" if f / (peak_tc * 1e12) > b / (peaks_["hbm_gbs"] * 1e9) else "hbm"
-            rows.append({"M": M, "N": N, "K": K, "us": round(ms * 1e3, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1),
-                         "gbs": round(b / (ms * 1e-3) / 1e9, 1), "bound": bound,
-                         "frac": round(t_roof / (ms * 1e-3), 4)})
+            row = {"M": M, "N": N, "K": K, "us": round(ms * 1e3, 2), "tflops": round(f / (ms * 1e-3) / 1e12, 1),
+                   "gbs": round(b / (ms * 1e-3) / 1e9, 1), "bound": bound,
+                   "frac": round(t_roof / (ms * 1e-3), 4),
+                   "frac_spec": round(max(b / (peaks_["hbm_gbs"] * 1e9), f / (SPEC_TENSOR_TFLOPS * 1e12))
+                                      / (ms * 1e-3), 4)}
+            if probe:
+                pk = probe["int8_tops"] if fmt == W8A8_INT8 else probe["e4m3_tflops"]
+                row["frac_probe"] = round(max(b / (peaks_["hbm_gbs"] * 1e9), f / (pk * 1e12)) / (ms * 1e-3), 4)
+            rows.append(row)
             del x, xq, sx, y, ws, flush
         del wq, sw
         torch.cuda.empty_cache()
@@ -492,7 +572,7 @@ def run_case(args):
     for i in range(args.warmup + args.steps):
         p.run(i)
     torch.cuda.synchronize()
-    us = p.time_plan()
+    us = p.time_plan(with_quant=False)
     b = workloads.algorithmic_bytes(fmt, M, N, K)
     pk = peaks()
     print(json.dumps({"case": args.case, "plan": qgd.qgd_get_plan(p.fid, M, N, K), "us": round(us, 3),
@@ -609,6 +689,7 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "tflops": round(flops * world / (ms_step * 1e-3) / 1e12, 3),
         "frac_of_hbm_peak": round(value / world / pk["hbm_gbs"], 4),
+        "frac_of_8tbs": round(value / world / 8000.0, 4),
         "roofline": {"bound": "hbm", "kernel": "GEMM (swapab/standard, all calls of the sweep)",
                      "achieved": round(gemm_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gemm_gbs / pk["hbm_gbs"], 4), "peak_source": pk["source"],
@@ -631,16 +712,20 @@ def main():
         fmts = {}
         del g_step
         fmts[FP8_DYNAMIC] = {"workload": wl.name, "ms_per_step": round(ms_step, 5), "gbs": round(value / world, 1),
-                             "frac": round(value / world / pk["hbm_gbs"], 4)}
+                             "frac": round(value / world / pk["hbm_gbs"], 4),
+                             "quantizer": quantizer_summary(ds)}
         keep = ds
         for wl2 in (workloads.INT8_DECODE, workloads.BLOCK_DECODE):
             ds2 = DecodeSet(wl2, device, per_call_rotation=True)
             fmts[wl2.fmt] = format_summary(ds2, args.steps, args.warmup, pk["hbm_gbs"])
+            fmts[wl2.fmt]["quantizer"] = quantizer_summary(ds2)
             fmts[wl2.fmt]["per_call"] = per_call_table(ds2, pk["hbm_gbs"])
             del ds2
             torch.cuda.empty_cache()
         out["formats"] = fmts
-        out["large_m"] = {f: large_m_summary(f, device, pk) for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)}
+        probe = tensor_probe()
+        out["tensor_probe"] = probe
+        out["large_m"] = {f: large_m_summary(f, device, pk, probe=probe) for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)}
         out.update(extra)
         ds = keep
     if dist.rank == 0 and dist.world == 1 and not args.quick and not args.no_cpu_baseline:

@@ -95,6 +95,9 @@ typedef struct {
                     ring under half the SM's shared memory, the next GEMM's CTA can be resident
                     beside this one and stream its first weights while this one finishes */
   int source;    /* 0 = built-in default, 1 = dispatch table, 2 = override */
+  int k_slices;  /* Swap-AB: 128-wide K slices per pipeline stage (1 or 2); Standard: 1.  Each stage
+                    costs a fixed hand-off between the copy engine and the MMA, so one CTA per SM
+                    keeps up with HBM only with two slices (32 KB of weights) per stage */
 } qgd_plan;
 
 /* ---------------------------------------------------------------------
@@ -182,10 +185,11 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
 
 /* Load a dispatch table: a text file with one line per (format, N, K,
  * M-bucket) and '#' comments,
- *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy
+ *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy [k_slices]
  * fmt in {fp8_dynamic, w8a8_int8, block_fp8}; variant in {standard, swap_ab};
  * reduce in {last_cta, two_pass, atomic}; schedule in {grid, persistent};
- * stages/tile_n/occupancy 0 = default.  Replaces the table in force.  On
+ * stages/tile_n/occupancy/k_slices 0 (or k_slices absent) = default.
+ * Replaces the table in force.  On
  * QGD_ERR_TABLE the table in force is unchanged.  Not thread-safe against
  * concurrent qlinear_* calls. */
 QGD_API qgd_status qgd_load_dispatch_table(const char* path);
@@ -194,10 +198,10 @@ QGD_API qgd_status qgd_load_dispatch_table(const char* path);
 QGD_API qgd_status qgd_clear_dispatch_table(void);
 
 /* Force a plan for one format (tests and the tuner).  Any argument < 0 keeps
- * the table/default choice for that field; stages/tile_n/occupancy 0 =
- * default.  qgd_set_override(fmt, -1, -1, -1, 0, 0, -1, 0) removes it. */
+ * the table/default choice for that field; stages/tile_n/occupancy/k_slices
+ * 0 = default.  qgd_set_override(fmt, -1, -1, -1, 0, 0, -1, 0, 0) removes it. */
 QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n,
-                                    int schedule, int occupancy);
+                                    int schedule, int occupancy, int k_slices);
 
 /* The plan a qlinear_* call with these arguments would run. */
 QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);
@@ -218,6 +222,19 @@ QGD_API const char* qgd_last_error_message(void);
  * the device.  qgd_clear_device_error() resets the flag. */
 QGD_API qgd_status qgd_device_error(unsigned int* code);
 QGD_API qgd_status qgd_clear_device_error(void);
+
+/* ---------------------------------------------------------------------
+ * Measurement aid (no counterpart on the pages, whose roofline takes the
+ * dense tensor peak from the data sheet).  Launches one CTA per SM, each
+ * issuing `iters` groups of four back-to-back tcgen05.mma (M=128, N=256,
+ * K=32 each; kind::f8f6f4 for QGD_QTYPE_E4M3, kind::i8 for QGD_QTYPE_INT8)
+ * from zeroed operands in shared memory into one TMEM accumulator; nothing
+ * is read from or written to global memory.  The caller times the launch on
+ * `stream`; *flops (host pointer, may be NULL) receives the launch's
+ * 2*M*N*K operation count.  1 <= iters <= 200000 (about 50 ms at most), else
+ * QGD_ERR_INVALID.  A wait that gives up is reported by qgd_device_error().
+ * --------------------------------------------------------------------- */
+QGD_API qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream);
 
 /* Library version, "major.minor.patch". */
 QGD_API const char* qgd_version(void);

@@ -30,6 +30,7 @@ __all__ = [
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
+    "qgd_mma_peak_probe",
     "Workspace", "DEFAULT_TABLE",
 ]
 
@@ -59,7 +60,7 @@ class QGDError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
                 ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("schedule", ctypes.c_int),
-                ("occupancy", ctypes.c_int), ("source", ctypes.c_int)]
+                ("occupancy", ctypes.c_int), ("source", ctypes.c_int), ("k_slices", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -83,10 +84,11 @@ def lib() -> ctypes.CDLL:
             "qlinear_fp8_dynamic_noalloc": [P, P, P, P, P, I, I, I, P],
             "qgd_load_dispatch_table": [ctypes.c_char_p],
             "qgd_clear_dispatch_table": [],
-            "qgd_set_override": [I, I, I, I, I, I, I, I],
+            "qgd_set_override": [I, I, I, I, I, I, I, I, I],
             "qgd_get_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
             "qgd_device_error": [ctypes.POINTER(ctypes.c_uint)],
             "qgd_clear_device_error": [],
+            "qgd_mma_peak_probe": [I, I, ctypes.POINTER(ctypes.c_double), P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -305,10 +307,10 @@ def qgd_clear_dispatch_table() -> None:
 
 
 def qgd_set_override(fmt: int, variant: int = -1, split_k: int = -1, reduce: int = -1, stages: int = 0,
-                     tile_n: int = 0, schedule: int = -1, occupancy: int = 0) -> None:
+                     tile_n: int = 0, schedule: int = -1, occupancy: int = 0, k_slices: int = 0) -> None:
     """Force plan fields for one format; every default argument leaves that
     field to the dispatch table / built-in default."""
-    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n, schedule, occupancy),
+    _check(lib().qgd_set_override(fmt, variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices),
            "qgd_set_override")
 
 
@@ -330,6 +332,15 @@ def qgd_device_error() -> int:
 
 def qgd_clear_device_error() -> None:
     _check(lib().qgd_clear_device_error(), "qgd_clear_device_error")
+
+
+def qgd_mma_peak_probe(qtype: int = QTYPE_E4M3, iters: int = 4096, stream=None) -> float:
+    """Launch the dense tensor-core peak probe on `stream` (one CTA per SM,
+    back-to-back tcgen05.mma from shared memory) and return its FLOP count;
+    the caller times the launch."""
+    flops = ctypes.c_double(0.0)
+    _check(lib().qgd_mma_peak_probe(qtype, iters, ctypes.byref(flops), _stream(stream)), "qgd_mma_peak_probe")
+    return float(flops.value)
 
 
 def qgd_version() -> str:

@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqgd.so")
-SOURCES = ["api.cu", "gemm.cu", "quant.cu"]
+SOURCES = ["api.cu", "gemm.cu", "quant.cu", "probe.cu"]
 HEADERS = ["qgd_internal.h", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

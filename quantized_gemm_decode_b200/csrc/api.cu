@@ -5,6 +5,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <fstream>
 #include <map>
@@ -111,13 +112,13 @@ constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
 
 struct Entry {
-  int variant, split_k, reduce, stages, tile_n, schedule, occupancy;
+  int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices;
 };
 using Key = std::tuple<int, int, int, int>;
 std::mutex g_mu;
 std::map<Key, Entry> g_table;
 struct Override {
-  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1, occupancy = 0;
+  int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1, occupancy = 0, k_slices = 0;
 } g_override[3];
 
 int bucket_of(int M) {
@@ -166,6 +167,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   p.stages = 0;
   p.schedule = kGrid;
   p.occupancy = 0;
+  p.k_slices = 0;
   if (M <= kDecodeMaxM) {
     // Decode: Swap-AB (the hand-written rule the method replaces with
     // measurement), persistent over all (tile, K-slice) units so that every
@@ -196,11 +198,12 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       p.tile_n = e.tile_n;
       p.schedule = e.schedule;
       p.occupancy = e.occupancy;
+      p.k_slices = e.k_slices;
       p.source = 1;
     }
     const Override& o = g_override[fmt];
     if (o.variant >= 0 || o.split_k >= 0 || o.reduce >= 0 || o.stages > 0 || o.tile_n > 0 || o.schedule >= 0 ||
-        o.occupancy > 0) {
+        o.occupancy > 0 || o.k_slices > 0) {
       if (o.variant >= 0) p.variant = o.variant;
       if (o.split_k >= 0) p.split_k = o.split_k;
       if (o.reduce >= 0) p.reduce = o.reduce;
@@ -208,6 +211,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       if (o.tile_n > 0) p.tile_n = o.tile_n;
       if (o.schedule >= 0) p.schedule = o.schedule;
       if (o.occupancy > 0) p.occupancy = o.occupancy;
+      if (o.k_slices > 0) p.k_slices = o.k_slices;
       p.source = 2;
     }
   }
@@ -216,7 +220,11 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
   if (p.schedule != kPersistent) p.schedule = kGrid;
-  int smax = nkt < 256 ? nkt : 256;
+  // K slices per stage (Swap-AB only): 1 or 2, at most the K extent
+  if (p.variant != kSwapAB || p.k_slices < 1 || nkt < 2) p.k_slices = 1;
+  if (p.k_slices > 2) p.k_slices = 2;
+  const int nku = (nkt + p.k_slices - 1) / p.k_slices;  // K units per tile
+  int smax = nku < 256 ? nku : 256;
   if (smax < 1) smax = 1;
   if (p.split_k < 1) p.split_k = 1;
   if (p.split_k > smax) p.split_k = smax;
@@ -229,14 +237,14 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
     if (tiles > kMaxTickets) p.reduce = kTwoPass;  // more tiles than arrival counters
   }
   const int mpad = M <= 16 ? 16 : 32;
-  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad) : standard_max_stages(p.tile_n);
+  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices) : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;
   if (p.schedule == kPersistent) {
-    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages)
+    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices)
                                                : standard_smem_bytes(p.tile_n, p.stages)) + 1024;
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
@@ -271,17 +279,18 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   if (M <= 0) return e;
   if (p.variant == kSwapAB) {
     const int n_tiles = (N + kSwapTileN - 1) / kSwapTileN;
+    const int nku = (nkt + p.k_slices - 1) / p.k_slices;  // K units (stages) per tile
     e.tiles = n_tiles;
     if (p.schedule == kPersistent) {
-      const long long U = static_cast<long long>(n_tiles) * nkt;
+      const long long U = static_cast<long long>(n_tiles) * nku;
       const long long cap = static_cast<long long>(g_num_sms) * p.occupancy;
       const long long G = U < cap ? U : cap;
       e.persistent = true;
       e.ctas = static_cast<int>(G);
       int maxc = 1;
       for (int t = 0; t < n_tiles; ++t) {
-        const long long c = sk_owner(static_cast<long long>(t) * nkt + nkt - 1, G, U) -
-                            sk_owner(static_cast<long long>(t) * nkt, G, U) + 1;
+        const long long c = sk_owner(static_cast<long long>(t) * nku + nku - 1, G, U) -
+                            sk_owner(static_cast<long long>(t) * nku, G, U) + 1;
         if (c > maxc) maxc = static_cast<int>(c);
       }
       e.maxc = maxc;
@@ -372,6 +381,7 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.ctas = ex.ctas;
   a.maxc = ex.maxc;
   a.mstride = ex.mstride;
+  a.kps = p.k_slices;
   a.pdl = pdl_enabled() ? 1 : 0;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -544,15 +554,21 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (hash != std::string::npos) line.resize(hash);
     std::istringstream ls(line);
     std::string fmt_s, var_s, red_s, sch_s;
-    int N, K, Mb, split, stages, tile_n, occ;
+    int N, K, Mb, split, stages, tile_n, occ, kslices = 0;
     if (!(ls >> fmt_s)) continue;  // blank line
     if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s >> occ))
       return fail(QGD_ERR_TABLE,
-                  "%s:%d: expected 11 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
-                  "occupancy",
+                  "%s:%d: expected 11 or 12 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
+                  "occupancy [k_slices]",
                   path, lineno);
     std::string extra;
-    if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
+    if (ls >> extra) {
+      char* end = nullptr;
+      const long v = strtol(extra.c_str(), &end, 10);
+      if (*end != '\0' || v < 0 || v > 2) return fail(QGD_ERR_TABLE, "%s:%d: bad k_slices '%s'", path, lineno, extra.c_str());
+      kslices = static_cast<int>(v);
+      if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
+    }
     const int fmt = fmt_from_name(fmt_s), var = variant_from_name(var_s), red = reduce_from_name(red_s);
     const int sch = schedule_from_name(sch_s);
     if (fmt < 0 || var < 0 || red < 0 || sch < 0)
@@ -564,7 +580,7 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
         occ > 2)
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
-    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ};
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ, kslices};
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_table.swap(t);
@@ -578,10 +594,11 @@ qgd_status qgd_clear_dispatch_table(void) {
 }
 
 qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule,
-                            int occupancy) {
+                            int occupancy, int k_slices) {
   if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
-      occupancy < 0 || occupancy > 2 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+      occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
+      (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");
   if (split_k > 0 && (split_k & (split_k - 1)) != 0) return fail(QGD_ERR_INVALID, "split_k must be a power of two");
   std::lock_guard<std::mutex> lk(g_mu);
@@ -593,6 +610,7 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
   o.tile_n = tile_n;
   o.schedule = schedule < 0 ? -1 : schedule;
   o.occupancy = occupancy;
+  o.k_slices = k_slices;
   return QGD_OK;
 }
 
@@ -626,12 +644,24 @@ qgd_status qgd_device_error(unsigned int* code) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   e = read_device_error(code);
+  if (e == cudaSuccess && *code == 0) e = read_probe_error(code);
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "read device error flag");
 }
 
 qgd_status qgd_clear_device_error(void) {
   cudaError_t e = clear_device_error();
+  if (e == cudaSuccess) e = clear_probe_error();
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "clear device error flag");
+}
+
+qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream) {
+  if (qtype != QGD_QTYPE_E4M3 && qtype != QGD_QTYPE_INT8) return fail(QGD_ERR_INVALID, "bad qtype %d", qtype);
+  if (iters < 1 || iters > 200000) return fail(QGD_ERR_INVALID, "iters=%d must be in [1, 200000]", iters);
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  if (flops) *flops = mma_probe_flops(iters, g_num_sms);
+  cudaError_t e = launch_mma_probe(qtype, iters, g_num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "qgd_mma_peak_probe launch");
 }
 
 const char* qgd_version(void) { return "0.1.0"; }

@@ -40,7 +40,8 @@ __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_d
 // Developer timeline of the Swap-AB kernel: with -DQGD_TRACE each CTA stamps
 // %globaltimer at up to 16 points (entry, set-up done, first loads issued,
 // first stage landed, last MMA committed, last accumulator read, epilogue
-// done, exit, and the steps of the last segment's output);
+// done, exit, the steps of the last segment's output, and the weight loads
+// issued / the preceding kernel's completion seen before the first loads);
 // qgd_debug_trace() copies the stamps out.  Compiled out otherwise.
 #ifdef QGD_TRACE
 constexpr int kTraceCtas = 4096;
@@ -221,9 +222,11 @@ __device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a,
 // ===========================================================================
 // Swap-AB kernel (decode, M <= 32).
 //
-// Work is the linear sequence of units u = tile * nkt + kt (tile = 128 weight
-// rows, kt = one 128-wide K slice).  Every CTA takes a contiguous range of
-// units; the range breaks into segments, one per tile it touches.
+// Work is the linear sequence of units u = tile * nku + kp (tile = 128 weight
+// rows, kp = the kp-th group of a.kps consecutive 128-wide K slices, one
+// pipeline stage; nku = ceil(nkt / kps) units per tile).  Every CTA takes a
+// contiguous range of units; the range breaks into segments, one per tile it
+// touches.
 //   grid schedule       grid (n_tiles, split_k): CTA (t, s) owns the s-th of
 //                       split_k near-equal K ranges of tile t (Split-K).
 //   persistent schedule grid (G): CTA c owns units [c*U/G, (c+1)*U/G) of all
@@ -239,11 +242,11 @@ __device__ __forceinline__ int sk_owner(long long u, long long G, long long U) {
 }
 
 // Contributors to tile t and this CTA's index among them.
-__device__ __forceinline__ void tile_contributors(const GemmArgs& a, int t, int nkt, long long U, int cta,
+__device__ __forceinline__ void tile_contributors(const GemmArgs& a, int t, int nku, long long U, int cta,
                                                   int& ncontrib, int& j) {
   if (a.persistent) {
-    const int first = sk_owner(static_cast<long long>(t) * nkt, a.ctas, U);
-    const int last = sk_owner(static_cast<long long>(t) * nkt + nkt - 1, a.ctas, U);
+    const int first = sk_owner(static_cast<long long>(t) * nku, a.ctas, U);
+    const int last = sk_owner(static_cast<long long>(t) * nku + nku - 1, a.ctas, U);
     ncontrib = last - first + 1;
     j = cta - first;
   } else {
@@ -369,14 +372,18 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const int stages = a.stages;
+  const int kps = a.kps;                     // K slices per stage
+  const uint32_t stage_w = kps * kWBytes;    // weight bytes per stage
+  const uint32_t stage_x = kps * kXBytes;    // activation bytes per stage
   uint8_t* w_ring = base;
-  uint8_t* x_ring = base + stages * kWBytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * kXBytes);
+  uint8_t* x_ring = base + stages * stage_w;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * stage_x);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkt = (a.K + kTileK - 1) / kTileK;
+  const int nku = (nkt + kps - 1) / kps;
   const int n_tiles = (a.N + kSwapTileN - 1) / kSwapTileN;
-  const long long U = static_cast<long long>(n_tiles) * nkt;
+  const long long U = static_cast<long long>(n_tiles) * nku;
   long long ub, ue;
   int cta;  // index among the contributors' numbering (persistent: CTA id; grid: split id)
   if (a.persistent) {
@@ -385,9 +392,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     ue = static_cast<long long>(blockIdx.x + 1) * U / gridDim.x;
   } else {
     cta = blockIdx.y;
-    const long long t0 = static_cast<long long>(blockIdx.x) * nkt;
-    ub = t0 + static_cast<long long>(blockIdx.y) * nkt / a.splits;
-    ue = t0 + static_cast<long long>(blockIdx.y + 1) * nkt / a.splits;
+    const long long t0 = static_cast<long long>(blockIdx.x) * nku;
+    ub = t0 + static_cast<long long>(blockIdx.y) * nku / a.splits;
+    ue = t0 + static_cast<long long>(blockIdx.y + 1) * nku / a.splits;
   }
   const int nk = static_cast<int>(ue - ub);
   if (threadIdx.x == 0) QGD_STAMP(0);
@@ -432,13 +439,22 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       const int pre = nk < stages ? nk : stages;
       for (int i = 0; i < pre; ++i) {
         const long long u = ub + i;
-        mbar_arrive_expect_tx(&ctl->full[i], kWBytes + kXBytes);
-        tma_load_2d(w_ring + i * kWBytes, &tw, &ctl->full[i], static_cast<int>(u % nkt) * kTileK,
-                    static_cast<int>(u / nkt) * kSwapTileN, pol_w);
+        const int k0 = static_cast<int>(u % nku) * kps;   // first K slice of the unit
+        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+        mbar_arrive_expect_tx(&ctl->full[i], ns * (kWBytes + kXBytes));
+        for (int j = 0; j < ns; ++j)
+          tma_load_2d(w_ring + i * stage_w + j * kWBytes, &tw, &ctl->full[i], (k0 + j) * kTileK,
+                      static_cast<int>(u / nku) * kSwapTileN, pol_w);
       }
+      QGD_STAMP(13);
       griddep_wait();
-      for (int i = 0; i < pre; ++i)
-        tma_load_2d(x_ring + i * kXBytes, &tx, &ctl->full[i], static_cast<int>((ub + i) % nkt) * kTileK, 0, pol_x);
+      QGD_STAMP(14);
+      for (int i = 0; i < pre; ++i) {
+        const int k0 = static_cast<int>((ub + i) % nku) * kps;
+        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+        for (int j = 0; j < ns; ++j)
+          tma_load_2d(x_ring + i * stage_x + j * kXBytes, &tx, &ctl->full[i], (k0 + j) * kTileK, 0, pol_x);
+      }
       issued = pre;
       QGD_STAMP(2);
       for (int i = pre; i < nk; ++i) {
@@ -451,10 +467,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         }
         if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
         const long long u = ub + i;
-        const int kx = static_cast<int>(u % nkt) * kTileK;
-        mbar_arrive_expect_tx(&ctl->full[s], kWBytes + kXBytes);
-        tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kx, static_cast<int>(u / nkt) * kSwapTileN, pol_w);
-        tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kx, 0, pol_x);
+        const int k0 = static_cast<int>(u % nku) * kps;
+        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+        mbar_arrive_expect_tx(&ctl->full[s], ns * (kWBytes + kXBytes));
+        for (int j = 0; j < ns; ++j) {
+          tma_load_2d(w_ring + s * stage_w + j * kWBytes, &tw, &ctl->full[s], (k0 + j) * kTileK,
+                      static_cast<int>(u / nku) * kSwapTileN, pol_w);
+          tma_load_2d(x_ring + s * stage_x + j * kXBytes, &tx, &ctl->full[s], (k0 + j) * kTileK, 0, pol_x);
+        }
         issued = i + 1;
       }
     }
@@ -463,7 +483,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     if (lane == 0) {
       const uint32_t w_base = smem_u32(w_ring), x_base = smem_u32(x_ring);
       int seg = 0;
-      for (int i = 0; i < nk; ++i) {
+      int sl = 0;  // Block_FP8: K slices consumed so far (one TMEM slot each)
+      bool stop = false;
+      for (int i = 0; i < nk && !stop; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
         if (!mbar_wait(&ctl->full[s], round & 1)) {
@@ -472,37 +494,46 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           break;
         }
         if (i == 0) QGD_STAMP(3);
-        const int kt = static_cast<int>((ub + i) % nkt);
-        const bool seg_start = (i == 0) || (kt == 0);
-        const bool seg_end = (i == nk - 1) || (kt == nkt - 1);
-        int slot;
-        uint32_t slot_round;
-        if constexpr (kBlock) {
-          slot = i % kSlots;
-          slot_round = i / kSlots;
-        } else {
-          slot = seg & 1;
-          slot_round = seg >> 1;
-        }
-        if (kBlock || seg_start) {
-          if (!mbar_wait(&ctl->tempty[slot], (slot_round & 1) ^ 1)) {
+        const int kp = static_cast<int>((ub + i) % nku);
+        const int ns = (nkt - kp * kps) < kps ? (nkt - kp * kps) : kps;
+        const bool seg_start = (i == 0) || (kp == 0);
+        const bool seg_end = (i == nk - 1) || (kp == nku - 1);
+        if (!kBlock && seg_start) {
+          if (!mbar_wait(&ctl->tempty[seg & 1], ((seg >> 1) & 1) ^ 1)) {
             record_error(kErrWaitMma);
             ctl->abort_flag = 1;
             break;
           }
         }
-        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d = tmem + slot * kMpad;
+        for (int j = 0; j < ns; ++j) {
+          const int slot = kBlock ? sl % kSlots : (seg & 1);
+          if (kBlock && !mbar_wait(&ctl->tempty[slot], ((sl / kSlots) & 1) ^ 1)) {
+            record_error(kErrWaitMma);
+            ctl->abort_flag = 1;
+            stop = true;
+            break;
+          }
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + slot * kMpad;
 #pragma unroll
-        for (int kk = 0; kk < kTileK / 32; ++kk) {
-          const uint64_t ad = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
-          const uint64_t bd = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
-          const uint32_t accumulate = kBlock ? (kk > 0) : !(seg_start && kk == 0);
-          mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+          for (int kk = 0; kk < kTileK / 32; ++kk) {
+            const uint64_t ad = sdesc_kmajor_sw128(w_base + s * stage_w + j * kWBytes + kk * 32);
+            const uint64_t bd = sdesc_kmajor_sw128(x_base + s * stage_x + j * kXBytes + kk * 32);
+            const uint32_t accumulate = kBlock ? (kk > 0) : !(seg_start && j == 0 && kk == 0);
+            mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+          }
+          if (kBlock) {
+            mma_commit(&ctl->tfull[slot]);
+            ++sl;
+          }
         }
+        if (stop) break;
         mma_commit(&ctl->empty[s]);
-        if (kBlock || seg_end) mma_commit(&ctl->tfull[slot]);
+        if (!kBlock && seg_end) mma_commit(&ctl->tfull[seg & 1]);
         if (seg_end) ++seg;
       }
       QGD_STAMP(4);
@@ -521,11 +552,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     if (scaled && threadIdx.x - 64 < static_cast<unsigned>(M)) ctl->sx_s[threadIdx.x - 64] = __ldg(a.sx + threadIdx.x - 64);
     epi_sync();
     int i = 0, seg = 0;
+    int sl = 0;  // Block_FP8: K slices consumed so far (same sequence as the MMA issuer's)
     while (i < nk) {
       const long long u = ub + i;
-      const int t = static_cast<int>(u / nkt);
-      const int kt_first = static_cast<int>(u % nkt);
-      const int len = (nkt - kt_first) < (nk - i) ? (nkt - kt_first) : (nk - i);
+      const int t = static_cast<int>(u / nku);
+      const int kp_first = static_cast<int>(u % nku);
+      const int len = (nku - kp_first) < (nk - i) ? (nku - kp_first) : (nk - i);
       const int n = t * kSwapTileN + row;
       // the channel scale is known before the accumulator is: fetch it now
       const float swv = (scaled && n < N) ? __ldg(a.sw + n) : 0.f;
@@ -534,10 +566,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         float facc[kMpad];
 #pragma unroll
         for (int m = 0; m < kMpad; ++m) facc[m] = 0.f;
-                for (int jj = 0; jj < len; ++jj) {
-          const int ii = i + jj;
-          const int slot = ii % kSlots;
-          if (!warp_wait(&ctl->tfull[slot], (ii / kSlots) & 1)) {
+        const int kb_first = kp_first * kps;
+        const int kb_end = (kp_first + len) * kps < nkt ? (kp_first + len) * kps : nkt;
+        for (int kb = kb_first; kb < kb_end; ++kb, ++sl) {
+          const int slot = sl % kSlots;
+          if (!warp_wait(&ctl->tfull[slot], (sl / kSlots) & 1)) {
             if (lane == 0) {
               record_error(kErrWaitEpilogue);
               ctl->abort_flag = 1;
@@ -550,7 +583,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(&ctl->tempty[slot]);
-          const int kb = kt_first + jj;
           const float swv = __ldg(a.sw + static_cast<size_t>(t) * KB + kb);  // one weight block per tile
 #pragma unroll
           for (int m = 0; m < kMpad; ++m) {
@@ -581,7 +613,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       const bool in_n = n < N;
       const bool last_seg = i + len >= nk;
       int ncontrib, jslot;
-      tile_contributors(a, t, nkt, U, cta, ncontrib, jslot);
+      tile_contributors(a, t, nku, U, cta, ncontrib, jslot);
       if (ncontrib == 1) {
         if (in_n) {
 #pragma unroll
@@ -616,7 +648,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
               uint32_t sum[kMpad];
               // in the CTA's last segment every ring stage has been consumed,
               // so the ring's shared memory can stage the partials
-              const size_t ring_bytes = static_cast<size_t>(stages) * (kWBytes + kXBytes);
+              const size_t ring_bytes = static_cast<size_t>(stages) * (stage_w + stage_x);
               if (last_seg && static_cast<size_t>(kSwapTileN) * ncontrib * nvec * 16 <= ring_bytes)
                 fixup_sum_smem<kFmt, kMpad>(a, t, row, ncontrib, nvec, w_ring, sum);
               else
@@ -648,9 +680,10 @@ __global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArg
   griddep_wait();
   const int t = blockIdx.x, row = threadIdx.x;
   const int nkt = (a.K + kTileK - 1) / kTileK;
-  const long long U = static_cast<long long>((a.N + kSwapTileN - 1) / kSwapTileN) * nkt;
+  const int nku = (nkt + a.kps - 1) / a.kps;
+  const long long U = static_cast<long long>((a.N + kSwapTileN - 1) / kSwapTileN) * nku;
   int ncontrib = a.splits, j0;
-  if (a.persistent) tile_contributors(a, t, nkt, U, 0, ncontrib, j0);
+  if (a.persistent) tile_contributors(a, t, nku, U, 0, ncontrib, j0);
   const int n = t * kSwapTileN + row;
   if (ncontrib == 1 || n >= a.N) return;  // written directly by its only contributor
   const int M = a.M, nvec = (M + 3) / 4;
@@ -1120,16 +1153,16 @@ cudaError_t set_smem_attr(Kern kernel, bool& done) {
 
 }  // namespace
 
-size_t swapab_smem_bytes(int mpad, int stages) {
-  return 1024 + static_cast<size_t>(stages) * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes;
+size_t swapab_smem_bytes(int mpad, int stages, int kps) {
+  return 1024 + static_cast<size_t>(stages) * kps * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes;
 }
 
 size_t standard_smem_bytes(int tile_n, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
 }
 
-int swapab_max_stages(int mpad) {
-  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kSwapTileN * kTileK + mpad * kTileK));
+int swapab_max_stages(int mpad, int kps) {
+  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -1146,7 +1179,7 @@ static cudaError_t launch_swapab_t(const CUtensorMap& tw, const CUtensorMap& tx,
   if (e != cudaSuccess) return e;
   const dim3 grid = a.persistent ? dim3(a.ctas, 1, 1)
                                  : dim3((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
-  return launch_ex(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads), swapab_smem_bytes(kMpad, a.stages),
+  return launch_ex(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads), swapab_smem_bytes(kMpad, a.stages, a.kps),
                    stream, a.pdl != 0, tw, tx, a);
 }
 

@@ -41,6 +41,7 @@ struct GemmArgs {
   int ctas;        // persistent schedule: number of CTAs
   int maxc;        // Swap-AB partial slots per tile (largest contributor count)
   int mstride;     // Swap-AB partial row stride in words (M rounded up to 4)
+  int kps;         // Swap-AB: 128-wide K slices per pipeline stage (1 or 2)
   int pdl;         // launch with a programmatic dependency on the preceding kernel
 };
 
@@ -53,10 +54,16 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();
-size_t swapab_smem_bytes(int mpad, int stages);
+size_t swapab_smem_bytes(int mpad, int stages, int kps);
 size_t standard_smem_bytes(int tile_n, int stages);
-int swapab_max_stages(int mpad);
+int swapab_max_stages(int mpad, int kps);
 int standard_max_stages(int tile_n);
+
+// Tensor-core peak probe (probe.cu).
+cudaError_t launch_mma_probe(int qtype, int iters, int ctas, cudaStream_t stream);
+double mma_probe_flops(int iters, int ctas);
+cudaError_t read_probe_error(unsigned int* code);
+cudaError_t clear_probe_error();
 
 // Quantizer launchers (quant.cu).
 cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, void* q, float* s,

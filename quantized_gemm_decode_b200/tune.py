@@ -8,11 +8,13 @@ candidates under CUDA-graph replay ("Building a High-Performance and
 Portable vLLM Linear Backend with Helion", sections "Put algorithm selection
 inside the search space", "Hybrid dispatch addresses runtime overhead" and
 "Autoajuste de los kernels").  Here the space is small and discrete, so it is
-searched exhaustively: variant x tile x split_k x reduction at the deepest
-pipeline, then the pipeline depth of the best few.  Each candidate is first
-checked against the split-free result (bit-exact int32 accumulators for
-W8A8_INT8, a relative bound for the fp32-accumulating formats), then timed as
-a graph of calls that cycle through at least 3x L2 of distinct weight copies.
+searched exhaustively: variant x tile x split_k x reduction x schedule x
+occupancy x K slices per stage at the deepest pipeline, then the pipeline
+depth of the best few.  Each candidate is first checked against the
+split-free result (bit-exact int32 accumulators for W8A8_INT8, a relative
+bound for the fp32-accumulating formats), then timed as a graph of layer
+calls (activation quantizer + GEMM, as the layer runs) that cycle through at
+least 3x L2 of distinct weight copies.
 
     python -m quantized_gemm_decode_b200.tune [--formats fp8_dynamic,...] [--out tables/b200.tsv]
         [--large-m] [--resume]
@@ -56,28 +58,31 @@ SCHED_NAME = {0: "grid", 1: "persistent"}
 
 
 def candidates(fmt: str, M: int, N: int, K: int):
-    """(variant, split_k, reduce, tile_n, schedule, occupancy) tuples legal for the shape."""
+    """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices) tuples legal for the shape."""
     nkt = (K + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
     out = []
     if M <= 32:
-        for r in (0, 1, 2):
-            for occ in (1, 2):
-                out.append((1, 1, r, 128, 1, occ))  # Swap-AB, persistent, 1 or 2 CTAs per SM
+        for kps in ((1, 2) if nkt >= 2 else (1,)):
+            for r in (0, 1, 2):
+                for occ in (1, 2):
+                    out.append((1, 1, r, 128, 1, occ, kps))  # Swap-AB, persistent, 1 or 2 CTAs per SM
         for s in splits:
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((1, s, r, 128, 0, 0))
+                out.append((1, s, r, 128, 0, 0, 1))
+            if nkt >= 2 and s <= (nkt + 1) // 2:
+                out.append((1, s, 0, 128, 0, 0, 2))  # two K slices per stage
     tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
     for t in tiles:
         for s in splits:
             if M <= 32 and s > 16:
                 continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((0, s, r, t, 0, 0))
+                out.append((0, s, r, t, 0, 0, 1))
         for s in (1, 2):
             if s <= nkt:
                 for r in ((0,) if s == 1 else (0, 1)):
-                    out.append((0, s, r, t, 1, 0))  # Standard, persistent
+                    out.append((0, s, r, t, 1, 0, 1))  # Standard, persistent
     return out
 
 
@@ -91,6 +96,7 @@ class Problem:
         ncopies = max(2, math.ceil(3 * L2_BYTES / (N * K)))
         self.copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(ncopies - 1)]
         x = synth.activations(M, K, seed, outliers=(fmt != W8A8_INT8)).to(device)
+        self.x = x
         self.xq, self.sx = _quant_x(fmt, x)
         self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         self.ws = qgd.Workspace(0, device)
@@ -101,22 +107,34 @@ class Problem:
         wq, sw = self.copies[j % len(self.copies)]
         return self.fn(self.xq, self.sx, wq, sw, y=self.y, ws=self.ws)
 
+    def layer_call(self, j=0):
+        """What the layer runs per call: quantize the activations, then the GEMM."""
+        if self.fmt == BLOCK_FP8:
+            qgd.quant_act_group128(self.x, xq=self.xq, sx=self.sx)
+        else:
+            qgd.quant_act_per_token(self.x, qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3,
+                                    xq=self.xq, sx=self.sx)
+        return self.run(j)
+
     def acc32(self):
         return qgd.qgd_w8a8_int8_acc32(self.xq, self.copies[0][0], ws=self.ws)
 
-    def time_plan(self, reps=10) -> float:
+    def time_plan(self, reps=10, with_quant=True) -> float:
+        """Microseconds per call of a graph of n calls (layer calls, or the
+        GEMM alone), each on its own weight copy."""
         n = len(self.copies)
+        call = self.layer_call if with_quant else self.run
         self.ws.ensure(qgd.qgd_workspace_size(self.fid, self.M, self.N, self.K))
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for j in range(n):
-                self.run(j)
+                call(j)
         torch.cuda.current_stream().wait_stream(s)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for j in range(n):
-                self.run(j)
+                call(j)
         for _ in range(2):
             g.replay()
         torch.cuda.synchronize()
@@ -134,14 +152,14 @@ class Problem:
 def tune_problem(p: Problem, log=None):
     fid = p.fid
     qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0,
-                         qgd.SCHEDULE_GRID, 0)
+                         qgd.SCHEDULE_GRID, 0, 1)
     p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
     ref = p.run().float().clone()
     ref_acc = p.acc32().clone() if p.fmt == W8A8_INT8 else None
     scale = ref.abs().max().item() + 1e-30
     results = []
-    for var, s, r, t, sch, occ in candidates(p.fmt, p.M, p.N, p.K):
-        qgd.qgd_set_override(fid, var, s, r, 0, t, sch, occ)
+    for var, s, r, t, sch, occ, kps in candidates(p.fmt, p.M, p.N, p.K):
+        qgd.qgd_set_override(fid, var, s, r, 0, t, sch, occ, kps)
         p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
         y = p.run().float()
         ok = (y - ref).abs().max().item() <= 2e-2 * scale
@@ -149,24 +167,24 @@ def tune_problem(p: Problem, log=None):
             ok = torch.equal(p.acc32(), ref_acc)
         if not ok:
             if log:
-                log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]} occ={occ}: "
-                    f"differs from the split-free result")
+                log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]} occ={occ} "
+                    f"kps={kps}: differs from the split-free result")
             continue
         us = p.time_plan()
-        stages = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["stages"]
-        results.append((us, var, s, r, stages, t, sch, occ))
+        pl = qgd.qgd_get_plan(fid, p.M, p.N, p.K)
+        results.append((us, var, pl["split_k"], r, pl["stages"], t, sch, occ, pl["k_slices"]))
     results.sort()
     # refine the pipeline depth of the three fastest
     refined = list(results[:3])
-    for us0, var, s, r, smax, t, sch, occ in results[:3]:
+    for us0, var, s, r, smax, t, sch, occ, kps in results[:3]:
         for st in (2, 3, 4, 5, 6, 8, 10):
             if st >= smax:
                 continue
-            qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ)
+            qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
             p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
             us = p.time_plan()
             occ_eff = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["occupancy"]
-            refined.append((us, var, s, r, st, t, sch, occ_eff))
+            refined.append((us, var, s, r, st, t, sch, occ_eff, kps))
     refined.sort()
     qgd.qgd_set_override(fid)
     return refined[0], results
@@ -193,7 +211,7 @@ def main(argv=None):
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
             f = ln.split("#")[0].split()
-            if len(f) == 11:
+            if len(f) in (11, 12):
                 done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
     only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
     t_start = time.time()
@@ -206,7 +224,8 @@ def main(argv=None):
         tmp = args.out + ".tmp"
         with open(tmp, "w") as f:
             f.write("# Dispatch table for B200 (sm_100a), measured by quantized_gemm_decode_b200.tune\n")
-            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy   # us/call\n")
+            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy k_slices"
+                    "   # us per layer call (quantize + GEMM)\n")
             for k in sorted(lines):
                 f.write(lines[k] + "\n")
         os.replace(tmp, args.out)
@@ -222,12 +241,12 @@ def main(argv=None):
                 t0 = time.time()
                 p = Problem(wl.fmt, M, N, K, wl.seed, device)
                 best, allres = tune_problem(p, log)
-                us, var, s, r, st, t, sch, occ = best
+                us, var, s, r, st, t, sch, occ, kps = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
                 lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "
-                              f"{occ}   # {us:.2f} us, {gbs:.0f} GB/s")
+                              f"{occ} {kps}   # {us:.2f} us, {gbs:.0f} GB/s")
                 log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
-                    f"{SCHED_NAME[sch]} occ={occ} {us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, "
+                    f"{SCHED_NAME[sch]} occ={occ} kps={kps} {us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, "
                     f"{time.time() - t0:.1f} s)")
                 del p
                 torch.cuda.empty_cache()

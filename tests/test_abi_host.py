@@ -228,3 +228,65 @@ def test_persistent_occupancy_follows_shared_memory():
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 4, 0, qgd.SCHEDULE_PERSISTENT, 2)
     two = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
     assert 0 < one < two
+
+
+def test_mma_peak_probe_rejects_bad_arguments():
+    L = qgd.lib()
+    flops = ctypes.c_double(0.0)
+    assert L.qgd_mma_peak_probe(2, 16, ctypes.byref(flops), None) == -1  # qtype
+    assert L.qgd_mma_peak_probe(qgd.QTYPE_E4M3, 0, ctypes.byref(flops), None) == -1
+    assert L.qgd_mma_peak_probe(qgd.QTYPE_INT8, 200001, ctypes.byref(flops), None) == -1
+
+
+def test_k_slices_plan_field():
+    P = qgd.SCHEDULE_PERSISTENT
+    # default: one slice per stage
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)["k_slices"] == 1
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 0, 0, P, 1, 2)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)
+    assert p["k_slices"] == 2 and p["occupancy"] == 1
+    # deepest ring with two 16 KB weight slices + 2 KB activation slices per stage
+    assert p["stages"] == (232448 - 1024 - 512) // (2 * (16384 + 16 * 128))
+    # a single-slice K, or the Standard kernel, has one slice per stage
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 128)["k_slices"] == 1
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 1, 0, 0, 128, P, 0, 2)
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)["k_slices"] == 1
+    # grid Split-K counts units of two slices: at most ceil(nkt / 2) splits
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 32, 0, 0, 0, qgd.SCHEDULE_GRID, 0, 2)
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)["split_k"] == 16
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 1, 0, 0, 0, P, 1, 3)
+
+
+def test_k_slices_workspace_counts_two_slice_units():
+    P = qgd.SCHEDULE_PERSISTENT
+    hdr = 64 * 1024
+    # partial slots per tile = most CTAs sharing a tile, counted over the
+    # schedule's units: 32 tiles x 16 two-slice units, or x 32 one-slice units
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 0, 0, P, 1, 2)
+    ws2 = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, 0, 0, P, 1, 1)
+    ws1 = qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+
+    def maxc(U, G, per_tile, tiles):
+        own = lambda u: ((u + 1) * G - 1) // U
+        return max(own(t * per_tile + per_tile - 1) - own(t * per_tile) + 1 for t in range(tiles))
+
+    assert ws2 == hdr + 32 * maxc(512, 148, 16, 32) * 128 * 4 * 4
+    assert ws1 == hdr + 32 * maxc(1024, 148, 32, 32) * 128 * 4 * 4
+
+
+def test_table_k_slices_column(tmp_path):
+    t = tmp_path / "t.tsv"
+    t.write_text("fp8_dynamic 4096 4096 1 swap_ab 1 last_cta 0 0 persistent 1 2\n"
+                 "fp8_dynamic 4096 4096 2 swap_ab 1 last_cta 0 0 persistent 1\n")
+    qgd.qgd_load_dispatch_table(str(t))
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)["k_slices"] == 2
+    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 2, 4096, 4096)["k_slices"] == 1
+    bad = tmp_path / "b.tsv"
+    bad.write_text("fp8_dynamic 4096 4096 1 swap_ab 1 last_cta 0 0 persistent 1 3\n")
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_load_dispatch_table(str(bad))
+    bad.write_text("fp8_dynamic 4096 4096 1 swap_ab 1 last_cta 0 0 persistent 1 2 9\n")
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_load_dispatch_table(str(bad))

@@ -276,3 +276,38 @@ def test_persistent_standard_many_tiles_per_cta(fmt, M, N, K, split):
         check_within_one_ulp(y[rows], yref, f"{fmt} M={M}")
     else:
         check_fp8_tolerance(y[rows], yref, bound, K, f"{fmt} M={M}")
+
+
+# Two 128-wide K slices per pipeline stage (Swap-AB): units are pairs of
+# slices, and a tile with an odd slice count ends in a one-slice unit.
+TWO_SLICE_PLANS = [(GRID, 1, 0, 0), (GRID, 2, 0, 0), (GRID, 4, 1, 0), (GRID, 4, 2, 0),
+                   (PERSISTENT, -1, 0, 1), (PERSISTENT, -1, 1, 2), (PERSISTENT, -1, 2, 1), (PERSISTENT, -1, 0, 2)]
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("plan", TWO_SLICE_PLANS,
+                         ids=lambda p: f"{'pers' if p[0] == PERSISTENT else 'grid'}-s{p[1]}-r{p[2]}-o{p[3]}")
+@pytest.mark.parametrize("M,N,K", [(4, 512, 1024), (13, 384, 896), (32, 1024, 1152), (1, 2048, 4096)])
+def test_two_slices_per_stage(fmt, plan, M, N, K):
+    sched, split, red, occ = plan
+    case = Case(fmt, M, N, K, seed=M * 7 + K, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, split, red, 0, 0, sched, occ, 2)
+    p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
+    assert p["k_slices"] == 2 and p["variant"] == qgd.VARIANT_SWAP_AB
+    case.check_output(case.run(), yref, bound, f"{fmt} two slices {plan} M={M} N={N} K={K}")
+    if fmt == W8A8_INT8:
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+
+
+@pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
+@pytest.mark.parametrize("sched", [GRID, PERSISTENT])
+def test_two_slices_partial_last_slice(fmt, sched):
+    # K = 1040: nine slices, the last one 16 wide (zero-filled past K)
+    case = Case(fmt, 3, 528, 1040, seed=5, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, 2 if sched == GRID else -1, 0, 0, 0, sched, 0, 2)
+    case.check_output(case.run(), yref, bound, f"{fmt} two slices K=1040")
