@@ -5,6 +5,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <fstream>
@@ -329,6 +330,8 @@ bool pdl_enabled() {
   return !(v && v[0] == '0');
 }
 
+std::atomic<int> g_call_seq{0};  // numbers GEMM calls for the developer timeline
+
 qgd_status check_shape(int fmt, int M, int N, int K) {
   if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d N=%d K=%d)", M, N, K);
   if (N % 16 != 0) return fail(QGD_ERR_UNSUPPORTED, "N=%d must be a multiple of 16", N);
@@ -383,6 +386,7 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.mstride = ex.mstride;
   a.kps = p.k_slices;
   a.pdl = pdl_enabled() ? 1 : 0;
+  a.trace_tag = g_call_seq.fetch_add(1, std::memory_order_relaxed) & 0x7fffffff;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;

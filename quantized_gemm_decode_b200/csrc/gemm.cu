@@ -43,14 +43,28 @@ __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_d
 // done, exit, the steps of the last segment's output, and the weight loads
 // issued / the preceding kernel's completion seen before the first loads);
 // qgd_debug_trace() copies the stamps out.  Compiled out otherwise.
+// Launches are kept in a ring of kTraceLaunches (by the call's trace tag), so
+// a chain of consecutive calls can be read back on one time line; slot 15
+// holds the SM the CTA ran on.
 #ifdef QGD_TRACE
 constexpr int kTraceCtas = 4096;
 constexpr int kTraceSlots = 16;
-__device__ unsigned long long g_trace[kTraceCtas * kTraceSlots];
-#define QGD_STAMP(slot)                                                             \
-  do {                                                                              \
-    const unsigned cta_ = blockIdx.x + blockIdx.y * gridDim.x;                      \
-    if (cta_ < kTraceCtas) g_trace[cta_ * kTraceSlots + (slot)] = globaltimer_ns(); \
+constexpr int kTraceLaunches = 8;
+__device__ unsigned long long g_trace[kTraceLaunches * kTraceCtas * kTraceSlots];
+__device__ __forceinline__ unsigned long long* trace_row(const GemmArgs& a) {
+  const unsigned cta = blockIdx.x + blockIdx.y * gridDim.x;
+  if (cta >= kTraceCtas) return nullptr;
+  return g_trace + (static_cast<size_t>(a.trace_tag % kTraceLaunches) * kTraceCtas + cta) * kTraceSlots;
+}
+#define QGD_STAMP(slot)                                 \
+  do {                                                  \
+    unsigned long long* r_ = trace_row(a);              \
+    if (r_) r_[(slot)] = globaltimer_ns();              \
+    if (r_ && (slot) == 0) {                            \
+      unsigned smid_;                                   \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_)); \
+      r_[15] = smid_;                                   \
+    }                                                   \
   } while (0)
 #else
 #define QGD_STAMP(slot) \
@@ -306,31 +320,35 @@ __device__ __forceinline__ void fixup_sum_t(const GemmArgs& a, int t, int row, i
   }
 }
 
-// The same sum through shared memory: every contributor's partial row is
-// requested at once with cp.async into this thread's own area of `stage`
-// (no register cost while in flight), then added from shared memory in
-// contributor order.  `stage` must hold 128 * ncontrib * nvec * 16 bytes.
+// The same sum through shared memory: the contributors' partial rows are
+// requested with cp.async into this thread's own area of `stage` (no register
+// cost while in flight), `chunk` contributors per round trip, then added from
+// shared memory in contributor order.  `stage` holds 128 * chunk * nvec * 16
+// bytes.
 template <int kFmt, int kMpad>
-__device__ __forceinline__ void fixup_sum_smem(const GemmArgs& a, int t, int row, int ncontrib, int nvec,
+__device__ __forceinline__ void fixup_sum_smem(const GemmArgs& a, int t, int row, int ncontrib, int nvec, int chunk,
                                                uint8_t* stage, uint32_t (&sum)[kMpad]) {
-  uint4* mine = reinterpret_cast<uint4*>(stage) + static_cast<size_t>(row) * ncontrib * nvec;
-  for (int j = 0; j < ncontrib; ++j) {
-    const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j, row));
-    for (int v = 0; v < nvec; ++v) cp_async16(mine + j * nvec + v, src + v);
-  }
-  cp_async_wait_all();
-  for (int j = 0; j < ncontrib; ++j) {
+  uint4* mine = reinterpret_cast<uint4*>(stage) + static_cast<size_t>(row) * chunk * nvec;
+  for (int j0 = 0; j0 < ncontrib; j0 += chunk) {
+    const int nj = (ncontrib - j0) < chunk ? (ncontrib - j0) : chunk;
+    for (int jj = 0; jj < nj; ++jj) {
+      const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j0 + jj, row));
+      for (int v = 0; v < nvec; ++v) cp_async16(mine + jj * nvec + v, src + v);
+    }
+    cp_async_wait_all();
+    for (int jj = 0; jj < nj; ++jj) {
 #pragma unroll
-    for (int v = 0; v < kMpad / 4; ++v) {
-      if (v < nvec) {
-        const uint4 w4 = mine[j * nvec + v];
-        if (j == 0) {
-          sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
-        } else {
-          sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
-          sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
-          sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
-          sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+      for (int v = 0; v < kMpad / 4; ++v) {
+        if (v < nvec) {
+          const uint4 w4 = mine[jj * nvec + v];
+          if (j0 + jj == 0) {
+            sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+          } else {
+            sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+            sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+            sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+            sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+          }
         }
       }
     }
@@ -649,8 +667,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
               // in the CTA's last segment every ring stage has been consumed,
               // so the ring's shared memory can stage the partials
               const size_t ring_bytes = static_cast<size_t>(stages) * (stage_w + stage_x);
-              if (last_seg && static_cast<size_t>(kSwapTileN) * ncontrib * nvec * 16 <= ring_bytes)
-                fixup_sum_smem<kFmt, kMpad>(a, t, row, ncontrib, nvec, w_ring, sum);
+              const int chunk = static_cast<int>(ring_bytes / (static_cast<size_t>(kSwapTileN) * nvec * 16));
+              if (last_seg && chunk >= 1)
+                fixup_sum_smem<kFmt, kMpad>(a, t, row, ncontrib, nvec, chunk, w_ring, sum);
               else
                 fixup_sum<kFmt, kMpad>(a, t, row, ncontrib, nvec, -1, acc, sum);  // own partial re-read from L2
               if (threadIdx.x == 64 && last_seg) QGD_STAMP(11);
@@ -748,11 +767,13 @@ __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0
 // one tile overlaps the mainloop of the next.
 // ===========================================================================
 // Threads of the Standard kernel: producer warp, MMA warp, then 4 epilogue
-// warps -- 8 for Block_FP8, whose per-K-block promotion is the busiest part
-// (two warps per TMEM lane quadrant, each taking half the columns).
+// warps -- 16 for Block_FP8, whose per-K-block promotion (TMEM read, scale,
+// add) is the busiest part: four warps per TMEM lane quadrant, each taking a
+// quarter of the columns, so that enough TMEM loads are in flight.
+constexpr int kBlockEpiGroups = 4;
 template <int kFmt>
 __host__ __device__ constexpr int std_threads() {
-  return kFmt == kFmtBlock ? 64 + 256 : kGemmThreads;
+  return kFmt == kFmtBlock ? 64 + 128 * kBlockEpiGroups : kGemmThreads;
 }
 
 template <int kFmt, int kTileN>
@@ -763,7 +784,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
   constexpr bool kBlock = (kFmt == kFmtBlock);
   static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
   constexpr uint32_t kEpi = std_threads<kFmt>() - 64;  // epilogue threads
-  constexpr int kHalf = kBlock ? kTileN / 2 : kTileN;   // columns per epilogue thread
+  constexpr int kHalf = kBlock ? kTileN / kBlockEpiGroups : kTileN;  // columns per epilogue thread
   // Block_FP8: a ring of 4 per-K-block accumulators (the MMA runs up to three
   // K blocks ahead of the promotion); else: a per-tile double buffer.
   constexpr int kSlots = kBlock ? 4 : 2;
@@ -910,7 +931,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     // ---------------- epilogue (warps 2..) ----------------
     griddep_wait();  // scales and outputs: only after the preceding kernel is done
     const int q = warp & 3;
-    const int half = kBlock ? (warp - 2) / 4 : 0;  // Block_FP8: which half of the columns
+    const int half = kBlock ? (warp - 2) / 4 : 0;  // Block_FP8: which column group (of kBlockEpiGroups)
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int M = a.M, N = a.N;
     int i = 0, li = 0;
@@ -930,9 +951,12 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
         for (int j = 0; j < kHalf; ++j) facc[j] = 0.f;
         const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
         const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
+        // scales one K block ahead, so their load latency hides behind a block
+        float sc_next = (in_m && kt0 < kt1) ? __ldg(sxrow + kt0) * __ldg(swrow + kt0) : 0.f;
         for (int kt = kt0; kt < kt1; ++kt, ++i) {
           const int slot = i % kSlots;
-          const float sc = in_m ? __ldg(sxrow + kt) * __ldg(swrow + kt) : 0.f;
+          const float sc = sc_next;
+          if (kt + 1 < kt1) sc_next = in_m ? __ldg(sxrow + kt + 1) * __ldg(swrow + kt + 1) : 0.f;
           if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
             if (lane == 0) {
               record_error(kErrWaitEpilogue);
@@ -941,14 +965,14 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             break;
           }
           tc_fence_after();
-          // this thread's 64 columns: four TMEM loads per wait
+          // this thread's columns: all its TMEM loads issued before one wait
           {
-            uint32_t r[4][16];
+            uint32_t r[kHalf / 16][16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld16(taddr + slot * kTileN + half * kHalf + c * 16, r[c]);
+            for (int c = 0; c < kHalf / 16; ++c) tmem_ld16(taddr + slot * kTileN + half * kHalf + c * 16, r[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < kHalf / 16; ++c)
 #pragma unroll
               for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[c * 16 + j]);
           }
@@ -1221,7 +1245,7 @@ cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CU
 
 #ifdef QGD_TRACE
 extern "C" __attribute__((visibility("default"))) int qgd_debug_trace(unsigned long long* host, size_t count) {
-  const size_t cap = static_cast<size_t>(kTraceCtas) * kTraceSlots;
+  const size_t cap = static_cast<size_t>(kTraceLaunches) * kTraceCtas * kTraceSlots;
   const size_t n = count < cap ? count : cap;
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)));
 }

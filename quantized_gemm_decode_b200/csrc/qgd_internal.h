@@ -43,6 +43,7 @@ struct GemmArgs {
   int mstride;     // Swap-AB partial row stride in words (M rounded up to 4)
   int kps;         // Swap-AB: 128-wide K slices per pipeline stage (1 or 2)
   int pdl;         // launch with a programmatic dependency on the preceding kernel
+  int trace_tag;   // sequence number of the call (developer timeline builds file stamps by it)
 };
 
 // Launchers (gemm.cu).  Each returns the cudaError_t of the launch.
