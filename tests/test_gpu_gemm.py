@@ -226,7 +226,7 @@ def test_persistent_shallow_pipelines_one_or_two_ctas_per_sm(stages, occupancy):
     # shallow rings leave room for two CTAs per SM: sized for one or two
     case = Case(FP8_DYNAMIC, 16, 4096, 4096, seed=stages)
     yref, bound = _oracle(case)[:2]
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, stages, 0, PERSISTENT, occupancy)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, -1, 0, stages, 0, PERSISTENT, occupancy, 1)
     assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 16, 4096, 4096)["occupancy"] == occupancy
     case.check_output(case.run(), yref, bound, f"stages={stages} occupancy={occupancy}")
 
