@@ -100,6 +100,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
+// Hand a TMEM accumulator back: one arrival per warp (the barrier counts
+// warps), after every lane's reads have completed and been fenced.  One
+// shared-memory atomic per warp instead of per thread: with 128-512 epilogue
+// threads arriving on one barrier per K block, the arrivals themselves had
+// become the Block_FP8 promotion's bottleneck.
+__device__ __forceinline__ void warp_release(uint64_t* bar) {
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 template <int kCols>
 __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&r)[kCols]) {
   static_assert(kCols % 16 == 0, "columns come in groups of 16");
@@ -321,26 +332,28 @@ __device__ __forceinline__ void fixup_sum_t(const GemmArgs& a, int t, int row, i
 }
 
 // The same sum through shared memory: the contributors' partial rows are
-// requested with cp.async into this thread's own area of `stage` (no register
-// cost while in flight), `chunk` contributors per round trip, then added from
-// shared memory in contributor order.  `stage` holds 128 * chunk * nvec * 16
+// requested with cp.async (no register cost while in flight), `chunk`
+// contributors per round trip, then added from shared memory in contributor
+// order.  Vector v of contributor j for weight row `row` sits at 16-byte index
+// (j * nvec + v) * 128 + row, so a warp's 32 threads touch 32 consecutive
+// 16-byte words (no bank conflicts).  `stage` holds 128 * chunk * nvec * 16
 // bytes.
 template <int kFmt, int kMpad>
 __device__ __forceinline__ void fixup_sum_smem(const GemmArgs& a, int t, int row, int ncontrib, int nvec, int chunk,
                                                uint8_t* stage, uint32_t (&sum)[kMpad]) {
-  uint4* mine = reinterpret_cast<uint4*>(stage) + static_cast<size_t>(row) * chunk * nvec;
+  uint4* area = reinterpret_cast<uint4*>(stage);
   for (int j0 = 0; j0 < ncontrib; j0 += chunk) {
     const int nj = (ncontrib - j0) < chunk ? (ncontrib - j0) : chunk;
     for (int jj = 0; jj < nj; ++jj) {
       const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j0 + jj, row));
-      for (int v = 0; v < nvec; ++v) cp_async16(mine + jj * nvec + v, src + v);
+      for (int v = 0; v < nvec; ++v) cp_async16(area + (jj * nvec + v) * kSwapTileN + row, src + v);
     }
     cp_async_wait_all();
     for (int jj = 0; jj < nj; ++jj) {
 #pragma unroll
       for (int v = 0; v < kMpad / 4; ++v) {
         if (v < nvec) {
-          const uint4 w4 = mine[jj * nvec + v];
+          const uint4 w4 = area[(jj * nvec + v) * kSwapTileN + row];
           if (j0 + jj == 0) {
             sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
           } else {
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     }
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&ctl->tfull[i], 1);
-      mbar_init(&ctl->tempty[i], 128);
+      mbar_init(&ctl->tempty[i], 4);  // one arrival per epilogue warp
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
@@ -599,8 +612,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           uint32_t r[kMpad];
           tmem_load_cols<kMpad>(taddr + slot * kMpad, r);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&ctl->tempty[slot]);
+          warp_release(&ctl->tempty[slot]);
           const float swv = __ldg(a.sw + static_cast<size_t>(t) * KB + kb);  // one weight block per tile
 #pragma unroll
           for (int m = 0; m < kMpad; ++m) {
@@ -621,8 +633,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           tc_fence_after();
           tmem_load_cols<kMpad>(taddr + slot * kMpad, acc);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&ctl->tempty[slot]);
+          warp_release(&ctl->tempty[slot]);
         }
       }
       if (!epi_agree_ok(ctl)) break;
@@ -816,7 +827,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     }
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&ctl->tfull[i], 1);
-      mbar_init(&ctl->tempty[i], kEpi);
+      mbar_init(&ctl->tempty[i], kEpi / 32);  // one arrival per epilogue warp
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
@@ -976,8 +987,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[c * 16 + j]);
           }
-          tc_fence_before();
-          mbar_arrive(&ctl->tempty[slot]);
+          warp_release(&ctl->tempty[slot]);
         }
         if (!epi_agree_ok(ctl, kEpi)) break;
         if (S == 1) {
@@ -1048,8 +1058,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
           tmem_wait_ld();
           if (c == kTileN / 16 - 1) {
             // the whole accumulator is in registers: hand the buffer back
-            tc_fence_before();
-            mbar_arrive(&ctl->tempty[buf]);
+            warp_release(&ctl->tempty[buf]);
           }
           if (!in_m || nc >= N) continue;
           const size_t idx = static_cast<size_t>(m) * N + nc;
