@@ -71,7 +71,10 @@ typedef enum {
   QGD_REDUCE_AUTO = -1,
   QGD_REDUCE_LAST_CTA = 0, /* split partials to workspace; the last CTA of each tile adds them in split order */
   QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order */
-  QGD_REDUCE_ATOMIC = 2    /* split partials added atomically into a zeroed workspace (fp32 order varies) */
+  QGD_REDUCE_ATOMIC = 2,   /* split partials added atomically into a zeroed workspace (fp32 order varies) */
+  QGD_REDUCE_CLUSTER = 3   /* Swap-AB grid schedule, 2 <= split_k <= 8: the splits of a tile form one
+                              thread-block cluster and add their partials in split order through
+                              distributed shared memory (no workspace) */
 } qgd_reduce;
 
 typedef enum {
@@ -187,7 +190,7 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
  * M-bucket) and '#' comments,
  *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy [k_slices]
  * fmt in {fp8_dynamic, w8a8_int8, block_fp8}; variant in {standard, swap_ab};
- * reduce in {last_cta, two_pass, atomic}; schedule in {grid, persistent};
+ * reduce in {last_cta, two_pass, atomic, cluster}; schedule in {grid, persistent};
  * stages/tile_n/occupancy/k_slices 0 (or k_slices absent) = default.
  * Replaces the table in force.  On
  * QGD_ERR_TABLE the table in force is unchanged.  Not thread-safe against

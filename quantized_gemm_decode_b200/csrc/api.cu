@@ -157,6 +157,7 @@ int reduce_from_name(const std::string& s) {
   if (s == "last_cta") return kLastCta;
   if (s == "two_pass") return kTwoPass;
   if (s == "atomic") return kAtomic;
+  if (s == "cluster") return kCluster;
   return -1;
 }
 
@@ -230,7 +231,12 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.split_k < 1) p.split_k = 1;
   if (p.split_k > smax) p.split_k = smax;
   p.split_k = floor_pow2(p.split_k);
-  if (p.reduce < kLastCta || p.reduce > kAtomic) p.reduce = kLastCta;
+  if (p.reduce < kLastCta || p.reduce > kCluster) p.reduce = kLastCta;
+  // cluster Split-K: the S splits of a tile form one thread-block cluster
+  // (Swap-AB, grid schedule, 2 <= S <= 8)
+  if (p.reduce == kCluster &&
+      (p.variant != kSwapAB || p.schedule != kGrid || p.split_k < 2 || p.split_k > kMaxClusterSplit))
+    p.reduce = kLastCta;
   if (p.reduce != kTwoPass) {
     const size_t tiles = p.variant == kSwapAB
                              ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
@@ -238,14 +244,15 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
     if (tiles > kMaxTickets) p.reduce = kTwoPass;  // more tiles than arrival counters
   }
   const int mpad = M <= 16 ? 16 : 32;
-  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices) : standard_max_stages(p.tile_n);
+  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster)
+                                          : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;
   if (p.schedule == kPersistent) {
-    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices)
+    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices, false)
                                                : standard_smem_bytes(p.tile_n, p.stages)) + 1024;
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
@@ -298,7 +305,7 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
     } else {
       e.maxc = p.split_k;
     }
-    if (e.maxc > 1)
+    if (e.maxc > 1 && p.reduce != kCluster)  // the cluster reduction needs no workspace
       e.data_bytes = p.reduce == kAtomic
                          ? align256(static_cast<size_t>(M) * N * 4)
                          : align256(static_cast<size_t>(n_tiles) * e.maxc * kSwapTileN * e.mstride * 4);
@@ -600,7 +607,7 @@ qgd_status qgd_clear_dispatch_table(void) {
 qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule,
                             int occupancy, int k_slices) {
   if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
-  if (variant > 1 || reduce > 2 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
+  if (variant > 1 || reduce > 3 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
       occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");

@@ -81,6 +81,7 @@ struct SmemCtl {
   uint64_t tempty[4];
   uint64_t accfull;
   uint64_t drain;
+  uint64_t recv_bar;  // Swap-AB cluster Split-K: peers' partial rows have landed here
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
@@ -409,6 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   uint8_t* w_ring = base;
   uint8_t* x_ring = base + stages * stage_w;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * stage_x);
+  uint8_t* recv_buf = reinterpret_cast<uint8_t*>(ctl) + kBarBytes;  // cluster Split-K: 128 x kMpad words
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkt = (a.K + kTileK - 1) / kTileK;
@@ -443,6 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->recv_bar, kSwapTileN);  // cluster Split-K: one arrival per weight row of the tile
     ctl->abort_flag = 0;
     ctl->last_flag = 0;
     ctl->epi_ok = 0;
@@ -455,6 +458,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // cluster Split-K: every CTA's receive barrier is initialised before any
+  // peer can arrive on it
+  if (a.reduce == kCluster) cluster_sync_all();
   griddep_launch_dependents();
   const uint32_t tmem = ctl->tmem_base;
   int issued = 0;
@@ -650,6 +656,48 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
             if (m < M) store_swap_final<kFmt>(acc[m], m, n, swv, ctl->sx_s, a);
         }
         if (threadIdx.x == 64 && last_seg) QGD_STAMP(8);
+      } else if (a.reduce == kCluster) {
+        // Split-K inside a thread-block cluster (the grid schedule's S splits
+        // of one tile): CTA j owns weight rows [j*R, (j+1)*R) of the tile,
+        // R = 128 / S.  Every CTA writes each of its partial rows into the
+        // owner's shared memory and arrives on the owner's barrier; each owner
+        // then adds the S contributions of its rows in CTA order.
+        const int S = ncontrib;
+        const int R = kSwapTileN / S;
+        const int owner = row / R, lr = row % R;
+        const uint32_t dst = mapa_shared(smem_u32(recv_buf), static_cast<uint32_t>(owner));
+        // owner's layout: [contributor][vector][row], 16 bytes each
+#pragma unroll
+        for (int v = 0; v < kMpad / 4; ++v)
+          if (v < nvec)
+            st_cluster_v4(dst + static_cast<uint32_t>(((jslot * nvec + v) * R + lr) * 16), acc[4 * v], acc[4 * v + 1],
+                          acc[4 * v + 2], acc[4 * v + 3]);
+        mbar_arrive_remote(mapa_shared(smem_u32(&ctl->recv_bar), static_cast<uint32_t>(owner)));
+        if (!mbar_wait_cluster(&ctl->recv_bar, 0)) {
+          record_error(kErrWaitEpilogue);
+          ctl->abort_flag = 1;
+        } else {
+          const uint4* rb = reinterpret_cast<const uint4*>(recv_buf);
+          for (int idx = row; idx < R * nvec; idx += kSwapTileN) {
+            const int v = idx / R, r = idx % R;
+            uint4 s4 = rb[v * R + r];
+            for (int j = 1; j < S; ++j) {
+              const uint4 w4 = rb[(j * nvec + v) * R + r];
+              s4.x = add_acc<kFmt>(s4.x, w4.x);
+              s4.y = add_acc<kFmt>(s4.y, w4.y);
+              s4.z = add_acc<kFmt>(s4.z, w4.z);
+              s4.w = add_acc<kFmt>(s4.w, w4.w);
+            }
+            const int nn = t * kSwapTileN + jslot * R + r;
+            if (nn < N) {
+              const float swn = scaled ? __ldg(a.sw + nn) : 0.f;
+              const uint32_t vals[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (4 * v + q < M) store_swap_final<kFmt>(vals[q], 4 * v + q, nn, swn, ctl->sx_s, a);
+            }
+          }
+        }
       } else {
         if (in_n) {
           if (a.reduce == kAtomic) {
@@ -778,10 +826,10 @@ __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0
 // one tile overlaps the mainloop of the next.
 // ===========================================================================
 // Threads of the Standard kernel: producer warp, MMA warp, then 4 epilogue
-// warps -- 16 for Block_FP8, whose per-K-block promotion (TMEM read, scale,
-// add) is the busiest part: four warps per TMEM lane quadrant, each taking a
-// quarter of the columns, so that enough TMEM loads are in flight.
-constexpr int kBlockEpiGroups = 4;
+// warps -- 8 for Block_FP8, whose per-K-block promotion (TMEM read, scale,
+// add) is the busiest part: two warps per TMEM lane quadrant, each taking half
+// the columns (16 warps measured slower on B200).
+constexpr int kBlockEpiGroups = 2;
 template <int kFmt>
 __host__ __device__ constexpr int std_threads() {
   return kFmt == kFmtBlock ? 64 + 128 * kBlockEpiGroups : kGemmThreads;
@@ -1158,21 +1206,38 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
 // Launch with dynamic shared memory and, when `pdl` is set, a programmatic
 // dependency on the preceding kernel in the stream.
 template <typename... Params, typename... Args>
-cudaError_t launch_ex(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                      bool pdl, Args&&... args) {
+cudaError_t launch_ex_cluster(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              bool pdl, int cluster_y, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_y > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = static_cast<unsigned>(cluster_y);
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_ex(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      bool pdl, Args&&... args) {
+  return launch_ex_cluster(kernel, grid, block, smem, stream, pdl, 1, std::forward<Args>(args)...);
 }
 
 template <typename Kern>
@@ -1186,16 +1251,18 @@ cudaError_t set_smem_attr(Kern kernel, bool& done) {
 
 }  // namespace
 
-size_t swapab_smem_bytes(int mpad, int stages, int kps) {
-  return 1024 + static_cast<size_t>(stages) * kps * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes;
+size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster) {
+  return 1024 + static_cast<size_t>(stages) * kps * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes +
+         (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0);
 }
 
 size_t standard_smem_bytes(int tile_n, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
 }
 
-int swapab_max_stages(int mpad, int kps) {
-  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
+int swapab_max_stages(int mpad, int kps, bool cluster) {
+  const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0);
+  int s = static_cast<int>((smem_budget() - fixed) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -1212,8 +1279,10 @@ static cudaError_t launch_swapab_t(const CUtensorMap& tw, const CUtensorMap& tx,
   if (e != cudaSuccess) return e;
   const dim3 grid = a.persistent ? dim3(a.ctas, 1, 1)
                                  : dim3((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
-  return launch_ex(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads), swapab_smem_bytes(kMpad, a.stages, a.kps),
-                   stream, a.pdl != 0, tw, tx, a);
+  const bool cluster = a.reduce == kCluster;
+  return launch_ex_cluster(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads),
+                           swapab_smem_bytes(kMpad, a.stages, a.kps, cluster), stream, a.pdl != 0,
+                           cluster ? a.splits : 1, tw, tx, a);
 }
 
 template <int kFmt, int kTileN>

@@ -10,7 +10,8 @@ namespace qgd {
 
 enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2 };
 enum Variant : int { kStandard = 0, kSwapAB = 1 };
-enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2 };
+enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2, kCluster = 3 };
+constexpr int kMaxClusterSplit = 8;  // portable thread-block cluster size
 enum Schedule : int { kGrid = 0, kPersistent = 1 };
 
 constexpr int kTileK = 128;           // K elements (= bytes) per pipeline stage
@@ -55,9 +56,9 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();
-size_t swapab_smem_bytes(int mpad, int stages, int kps);
+size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster);
 size_t standard_smem_bytes(int tile_n, int stages);
-int swapab_max_stages(int mpad, int kps);
+int swapab_max_stages(int mpad, int kps, bool cluster);
 int standard_max_stages(int tile_n);
 
 // Tensor-core peak probe (probe.cu).

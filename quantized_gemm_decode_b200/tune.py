@@ -39,7 +39,7 @@ from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_IN
 L2_BYTES = 126 * 1024 * 1024
 FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}
 VAR_NAME = {0: "standard", 1: "swap_ab"}
-RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic"}
+RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
 
 
 def _quant_w(fmt, w):
@@ -72,6 +72,10 @@ def candidates(fmt: str, M: int, N: int, K: int):
                 out.append((1, s, r, 128, 0, 0, 1))
             if nkt >= 2 and s <= (nkt + 1) // 2:
                 out.append((1, s, 0, 128, 0, 0, 2))  # two K slices per stage
+            if 2 <= s <= 8:  # the splits of a tile as one thread-block cluster (DSMEM reduction)
+                out.append((1, s, 3, 128, 0, 0, 1))
+                if nkt >= 2 and s <= (nkt + 1) // 2:
+                    out.append((1, s, 3, 128, 0, 0, 2))
     tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
     for t in tiles:
         for s in splits:

@@ -290,3 +290,30 @@ def test_table_k_slices_column(tmp_path):
     bad.write_text("fp8_dynamic 4096 4096 1 swap_ab 1 last_cta 0 0 persistent 1 2 9\n")
     with pytest.raises(qgd.QGDError):
         qgd.qgd_load_dispatch_table(str(bad))
+
+
+def test_cluster_reduction_plan_rules():
+    G, P = qgd.SCHEDULE_GRID, qgd.SCHEDULE_PERSISTENT
+    C = qgd.REDUCE_CLUSTER
+    for split in (2, 4, 8):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, split, C, 0, 0, G, 0, 1)
+        p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
+        assert p["reduce"] == C and p["split_k"] == split
+        # the splits exchange partials through shared memory: no workspace
+        assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 0
+    # beyond a portable cluster, on the persistent schedule, or for Standard
+    # tiles the reduction falls back to the last-arriving CTA
+    for args in ((qgd.VARIANT_SWAP_AB, 16, C, 0, 0, G), (qgd.VARIANT_SWAP_AB, -1, C, 0, 0, P),
+                 (qgd.VARIANT_STANDARD, 4, C, 0, 128, G), (qgd.VARIANT_SWAP_AB, 1, C, 0, 0, G)):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, *args)
+        assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["reduce"] == qgd.REDUCE_LAST_CTA
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 4, 4, 0, 0, G)
+
+
+def test_table_cluster_reduce_name(tmp_path):
+    t = tmp_path / "t.tsv"
+    t.write_text("w8a8_int8 5120 5120 8 swap_ab 4 cluster 0 0 grid 0 2\n")
+    qgd.qgd_load_dispatch_table(str(t))
+    p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 8, 5120, 5120)
+    assert (p["reduce"], p["split_k"], p["k_slices"], p["source"]) == (qgd.REDUCE_CLUSTER, 4, 2, 1)

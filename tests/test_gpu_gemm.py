@@ -311,3 +311,50 @@ def test_two_slices_partial_last_slice(fmt, sched):
     yref, bound = _oracle(case)[:2]
     qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, 2 if sched == GRID else -1, 0, 0, 0, sched, 0, 2)
     case.check_output(case.run(), yref, bound, f"{fmt} two slices K=1040")
+
+
+# Split-K inside a thread-block cluster: partial rows travel through
+# distributed shared memory to the CTA that owns them.
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("split,kps", [(2, 1), (4, 1), (8, 1), (4, 2), (8, 2)])
+@pytest.mark.parametrize("M,N,K", [(1, 1024, 4096), (17, 384, 2048), (32, 2048, 1152), (5, 256, 1024)])
+def test_cluster_split_reduction(fmt, split, kps, M, N, K):
+    case = Case(fmt, M, N, K, seed=split * 31 + M, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, split, qgd.REDUCE_CLUSTER, 0, 0, GRID, 0, kps)
+    p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
+    assert p["reduce"] == qgd.REDUCE_CLUSTER and p["split_k"] == split
+    y1 = case.run()
+    case.check_output(y1, yref, bound, f"{fmt} cluster s={split} k={kps} M={M} N={N} K={K}")
+    y2 = case.run()  # fixed split order: bitwise repeatable
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    if fmt == W8A8_INT8:
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+    assert qgd.qgd_device_error() == 0
+
+
+def test_cluster_split_reduction_ragged_n_and_graph():
+    # N = 528: the last tile has 16 live weight rows; every row still reports
+    case = Case(FP8_DYNAMIC, 3, 528, 1040, seed=9, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 8, qgd.REDUCE_CLUSTER, 0, 0, GRID, 0, 1)
+    y = torch.empty((3, 528), dtype=torch.bfloat16, device="cuda")
+    call = lambda: qgd.qlinear_fp8_dynamic(case.xq, case.sx, case.wq, case.sw, y=y)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    case.check_output(y, yref, bound, "cluster ragged N under graph replay")
+    assert qgd.qgd_device_error() == 0
