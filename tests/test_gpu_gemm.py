@@ -323,7 +323,11 @@ def test_cluster_split_reduction(fmt, split, kps, M, N, K):
     yref, bound = _oracle(case)[:2]
     qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, split, qgd.REDUCE_CLUSTER, 0, 0, GRID, 0, kps)
     p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
-    assert p["reduce"] == qgd.REDUCE_CLUSTER and p["split_k"] == split
+    nku = -(-(-(-K // 128)) // kps)  # K units of kps slices: the split is at most that, a power of two
+    expect = split
+    while expect > nku:
+        expect //= 2
+    assert p["reduce"] == qgd.REDUCE_CLUSTER and p["split_k"] == expect
     y1 = case.run()
     case.check_output(y1, yref, bound, f"{fmt} cluster s={split} k={kps} M={M} N={N} K={K}")
     y2 = case.run()  # fixed split order: bitwise repeatable
