@@ -57,36 +57,55 @@ def _quant_x(fmt, x):
 SCHED_NAME = {0: "grid", 1: "persistent"}
 
 
-def candidates(fmt: str, M: int, N: int, K: int):
-    """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices) tuples legal for the shape."""
+SMEM_PER_SM = 233472  # bytes of shared memory per SM on sm_100 (228 KB)
+
+
+def two_per_sm_stages(M: int, kps: int, cluster: bool) -> int:
+    """Deepest Swap-AB ring that still lets two CTAs share an SM."""
+    mpad = 16 if M <= 16 else 32
+    per_stage = kps * (128 * 128 + mpad * 128)
+    fixed = 1024 + 512 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
+    return max(2, min(16, (SMEM_PER_SM // 2 - fixed) // per_stage))
+
+
+def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
+    """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices, stages) tuples legal for the
+    shape; stages 0 = the deepest ring.  A Swap-AB grid with more CTAs than SMs is tried at the ring
+    depth that fits two CTAs per SM, so that it runs in one wave."""
     nkt = (K + 127) // 128
+    n_tiles = (N + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
     out = []
+
+    def swap_grid(s, r, kps):
+        st = two_per_sm_stages(M, kps, r == 3) if n_tiles * s > num_sms else 0
+        out.append((1, s, r, 128, 0, 0, kps, st))
+
     if M <= 32:
         for kps in ((1, 2) if nkt >= 2 else (1,)):
             for r in (0, 1, 2):
                 for occ in (1, 2):
-                    out.append((1, 1, r, 128, 1, occ, kps))  # Swap-AB, persistent, 1 or 2 CTAs per SM
+                    out.append((1, 1, r, 128, 1, occ, kps, 0))  # Swap-AB, persistent, 1 or 2 CTAs per SM
         for s in splits:
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((1, s, r, 128, 0, 0, 1))
+                swap_grid(s, r, 1)
             if nkt >= 2 and s <= (nkt + 1) // 2:
-                out.append((1, s, 0, 128, 0, 0, 2))  # two K slices per stage
+                swap_grid(s, 0, 2)  # two K slices per stage
             if 2 <= s <= 8:  # the splits of a tile as one thread-block cluster (DSMEM reduction)
-                out.append((1, s, 3, 128, 0, 0, 1))
+                swap_grid(s, 3, 1)
                 if nkt >= 2 and s <= (nkt + 1) // 2:
-                    out.append((1, s, 3, 128, 0, 0, 2))
+                    swap_grid(s, 3, 2)
     tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
     for t in tiles:
         for s in splits:
             if M <= 32 and s > 16:
                 continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
             for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((0, s, r, t, 0, 0, 1))
+                out.append((0, s, r, t, 0, 0, 1, 0))
         for s in (1, 2):
             if s <= nkt:
                 for r in ((0,) if s == 1 else (0, 1)):
-                    out.append((0, s, r, t, 1, 0, 1))  # Standard, persistent
+                    out.append((0, s, r, t, 1, 0, 1, 0))  # Standard, persistent
     return out
 
 
@@ -162,8 +181,9 @@ def tune_problem(p: Problem, log=None):
     ref_acc = p.acc32().clone() if p.fmt == W8A8_INT8 else None
     scale = ref.abs().max().item() + 1e-30
     results = []
-    for var, s, r, t, sch, occ, kps in candidates(p.fmt, p.M, p.N, p.K):
-        qgd.qgd_set_override(fid, var, s, r, 0, t, sch, occ, kps)
+    num_sms = torch.cuda.get_device_properties(p.y.device).multi_processor_count
+    for var, s, r, t, sch, occ, kps, st0 in candidates(p.fmt, p.M, p.N, p.K, num_sms):
+        qgd.qgd_set_override(fid, var, s, r, st0, t, sch, occ, kps)
         p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
         y = p.run().float()
         ok = (y - ref).abs().max().item() <= 2e-2 * scale
