@@ -317,3 +317,26 @@ def test_table_cluster_reduce_name(tmp_path):
     qgd.qgd_load_dispatch_table(str(t))
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 8, 5120, 5120)
     assert (p["reduce"], p["split_k"], p["k_slices"], p["source"]) == (qgd.REDUCE_CLUSTER, 4, 2, 1)
+
+
+@pytest.mark.parametrize("fmt,M,N,K", [("fp8_dynamic", 1, 4096, 4096), ("w8a8_int8", 16, 34816, 5120),
+                                       ("block_fp8", 32, 5120, 25600), ("fp8_dynamic", 512, 6144, 4096)])
+def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
+    # every plan the tuner times is one the library runs as asked (no silent
+    # legalization), and a grid-schedule Swap-AB candidate with more CTAs than
+    # SMs fits two CTAs per SM
+    from quantized_gemm_decode_b200 import tune
+
+    fid = tune.FMT_ID[fmt]
+    for var, s, r, t, sch, occ, kps, st in tune.candidates(fmt, M, N, K, 148):
+        qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
+        p = qgd.qgd_get_plan(fid, M, N, K)
+        assert (p["variant"], p["reduce"], p["schedule"], p["k_slices"]) == (var, r, sch, kps), (var, s, r, sch, kps)
+        if sch == qgd.SCHEDULE_GRID:
+            assert p["split_k"] == s
+        if st:
+            assert p["stages"] == st
+            if var == qgd.VARIANT_SWAP_AB and sch == qgd.SCHEDULE_GRID:
+                mpad = 16 if M <= 16 else 32
+                smem = 1024 + st * kps * (16384 + mpad * 128) + 512 + (128 * mpad * 4 if r == 3 else 0)
+                assert 2 * (smem + 1024) <= 233472
