@@ -70,8 +70,8 @@ def two_per_sm_stages(M: int, kps: int, cluster: bool) -> int:
 
 def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
     """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices, stages) tuples legal for the
-    shape; stages 0 = the deepest ring.  A Swap-AB grid with more CTAs than SMs is tried at the ring
-    depth that fits two CTAs per SM, so that it runs in one wave."""
+    shape; stages 0 = the deepest ring.  A Swap-AB grid with more CTAs than SMs, and the persistent
+    schedule sized for two CTAs per SM, are tried at the ring depth that fits two CTAs per SM."""
     nkt = (K + 127) // 128
     n_tiles = (N + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
@@ -84,8 +84,9 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
     if M <= 32:
         for kps in ((1, 2) if nkt >= 2 else (1,)):
             for r in (0, 1, 2):
-                for occ in (1, 2):
-                    out.append((1, 1, r, 128, 1, occ, kps, 0))  # Swap-AB, persistent, 1 or 2 CTAs per SM
+                # Swap-AB, persistent: one CTA per SM at the deepest ring, or two at a ring that fits
+                out.append((1, 1, r, 128, 1, 1, kps, 0))
+                out.append((1, 1, r, 128, 1, 2, kps, two_per_sm_stages(M, kps, False)))
         for s in splits:
             for r in ((0,) if s == 1 else (0, 1, 2)):
                 swap_grid(s, r, 1)

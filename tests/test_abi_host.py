@@ -332,11 +332,13 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
         qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
         p = qgd.qgd_get_plan(fid, M, N, K)
         assert (p["variant"], p["reduce"], p["schedule"], p["k_slices"]) == (var, r, sch, kps), (var, s, r, sch, kps)
+        if sch == qgd.SCHEDULE_PERSISTENT and var == qgd.VARIANT_SWAP_AB:
+            assert p["occupancy"] == occ
         if sch == qgd.SCHEDULE_GRID:
             assert p["split_k"] == s
         if st:
             assert p["stages"] == st
-            if var == qgd.VARIANT_SWAP_AB and sch == qgd.SCHEDULE_GRID:
+            if var == qgd.VARIANT_SWAP_AB and (sch == qgd.SCHEDULE_GRID or occ == 2):
                 mpad = 16 if M <= 16 else 32
                 smem = 1024 + st * kps * (16384 + mpad * 128) + 512 + (128 * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
