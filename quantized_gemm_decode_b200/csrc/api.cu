@@ -110,7 +110,11 @@ constexpr size_t kTicketBytes = 64 * 1024;
 constexpr size_t kMaxTickets = kTicketBytes / 4;
 const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
 constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
-constexpr int kDecodeMaxM = 32;  // largest token count the Swap-AB kernel covers
+constexpr int kDecodeMaxM = 32;   // decode token counts: Swap-AB by default
+constexpr int kSwapMaxM = 128;    // largest token count the Swap-AB kernel covers (FP8_Dynamic, W8A8_INT8)
+
+// Token columns of the Swap-AB MMA (its N): the next of 16, 32, 64, 128.
+int swap_mpad(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
 struct Entry {
   int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices;
@@ -218,7 +222,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
     }
   }
   // Make the plan legal for this shape.
-  if (p.variant == kSwapAB && M > kDecodeMaxM) p.variant = kStandard;
+  if (p.variant == kSwapAB && M > (fmt == kFmtBlock ? kDecodeMaxM : kSwapMaxM)) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
   if (p.schedule != kPersistent) p.schedule = kGrid;
@@ -232,6 +236,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   if (p.split_k > smax) p.split_k = smax;
   p.split_k = floor_pow2(p.split_k);
   if (p.reduce < kLastCta || p.reduce > kCluster) p.reduce = kLastCta;
+  // the two-pass reduction kernel covers at most 32 tokens
+  if (p.variant == kSwapAB && M > kDecodeMaxM && p.reduce == kTwoPass) p.reduce = kLastCta;
   // cluster Split-K: the S splits of a tile form one thread-block cluster
   // (Swap-AB, grid schedule, 2 <= S <= 8)
   if (p.reduce == kCluster &&
@@ -243,7 +249,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
                              : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
     if (tiles > kMaxTickets) p.reduce = kTwoPass;  // more tiles than arrival counters
   }
-  const int mpad = M <= 16 ? 16 : 32;
+  const int mpad = swap_mpad(M);
   const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster)
                                           : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
@@ -273,7 +279,7 @@ struct Exec {
   bool persistent = false;
   int ctas = 0;     // persistent schedule: CTAs launched
   int maxc = 1;     // most CTAs sharing one output tile
-  int mpad = 16;    // Swap-AB: token columns per MMA (16 or 32)
+  int mpad = 16;    // Swap-AB: token columns per MMA (16, 32, 64 or 128)
   int mstride = 4;  // Swap-AB: partial row stride in words
   size_t tiles = 0;  // output tiles (arrival counters)
   size_t data_off = 0, data_bytes = 0, total = 0;
@@ -282,7 +288,7 @@ struct Exec {
 Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   Exec e;
   const int nkt = (K + kTileK - 1) / kTileK;
-  e.mpad = M <= 16 ? 16 : 32;
+  e.mpad = swap_mpad(M);
   e.mstride = (M + 3) / 4 * 4;
   if (M <= 0) return e;
   if (p.variant == kSwapAB) {

@@ -72,7 +72,7 @@ __device__ __forceinline__ unsigned long long* trace_row(const GemmArgs& a) {
   } while (0)
 #endif
 
-constexpr uint32_t kBarBytes = 512;  // mbarriers + a few flags, after the rings
+constexpr uint32_t kBarBytes = 1024;  // mbarriers, flags and staged token scales, after the rings
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
@@ -86,7 +86,7 @@ struct SmemCtl {
   int abort_flag;
   int last_flag;
   int epi_ok;
-  float sx_s[32];  // Swap-AB, per-token formats: the M token scales, staged once
+  float sx_s[128];  // Swap-AB, per-token formats: the M token scales, staged once
 };
 static_assert(sizeof(SmemCtl) <= kBarBytes, "control block too large");
 
@@ -369,6 +369,55 @@ __device__ __forceinline__ void fixup_sum_smem(const GemmArgs& a, int t, int row
   }
 }
 
+// Contributors' vectors [v0, v0 + nv) of weight row `row` of tile t, added in
+// contributor order (more than 32 tokens: one 32-token chunk of the row).
+// With chunk > 0 the drained ring stages them, `chunk` contributors per round
+// trip (same layout as fixup_sum_smem); otherwise one contributor per round
+// trip through registers.
+template <int kFmt, int kAcc, int kMpad>
+__device__ __forceinline__ void fixup_sum_range(const GemmArgs& a, int t, int row, int ncontrib, int v0, int nv,
+                                                int chunk, uint8_t* stage, uint32_t (&sum)[kAcc]) {
+  for (int j0 = 0; j0 < ncontrib; j0 += (chunk > 0 ? chunk : 1)) {
+    const int nj = chunk > 0 ? ((ncontrib - j0) < chunk ? (ncontrib - j0) : chunk) : 1;
+    uint4 buf[kAcc / 4];
+    uint4* area = reinterpret_cast<uint4*>(stage);
+    if (chunk > 0) {
+      for (int jj = 0; jj < nj; ++jj) {
+        const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j0 + jj, row)) + v0;
+        for (int v = 0; v < nv; ++v) cp_async16(area + (jj * nv + v) * kSwapTileN + row, src + v);
+      }
+      cp_async_wait_all();
+    }
+    for (int jj = 0; jj < nj; ++jj) {
+      const int j = j0 + jj;
+      if (chunk > 0) {
+#pragma unroll
+        for (int v = 0; v < kAcc / 4; ++v)
+          if (v < nv) buf[v] = area[(jj * nv + v) * kSwapTileN + row];
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(swap_slot<kMpad>(a, t, j, row)) + v0;
+#pragma unroll
+        for (int v = 0; v < kAcc / 4; ++v)
+          if (v < nv) buf[v] = __ldcg(src + v);
+      }
+#pragma unroll
+      for (int v = 0; v < kAcc / 4; ++v) {
+        if (v < nv) {
+          const uint4 w4 = buf[v];
+          if (j == 0) {
+            sum[4 * v] = w4.x; sum[4 * v + 1] = w4.y; sum[4 * v + 2] = w4.z; sum[4 * v + 3] = w4.w;
+          } else {
+            sum[4 * v] = add_acc<kFmt>(sum[4 * v], w4.x);
+            sum[4 * v + 1] = add_acc<kFmt>(sum[4 * v + 1], w4.y);
+            sum[4 * v + 2] = add_acc<kFmt>(sum[4 * v + 2], w4.z);
+            sum[4 * v + 3] = add_acc<kFmt>(sum[4 * v + 3], w4.w);
+          }
+        }
+      }
+    }
+  }
+}
+
 template <int kFmt, int kMpad>
 __device__ __forceinline__ void fixup_sum(const GemmArgs& a, int t, int row, int ncontrib, int nvec, int own,
                                        const uint32_t (&own_acc)[kMpad], uint32_t (&sum)[kMpad]) {
@@ -396,7 +445,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   // Block_FP8: a ring of per-K-block accumulators; otherwise one accumulator
   // per segment, double-buffered so the next segment's MMAs overlap the drain.
   constexpr int kSlots = kBlock ? 4 : 2;
-  constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : 128);
+  constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : (kSlots * kMpad <= 128 ? 128 : 256));
+  static_assert(!kBlock || kMpad <= 32, "Block_FP8 Swap-AB covers at most 32 tokens");
+  // the epilogue walks the accumulator row in chunks of at most 32 token columns
+  constexpr int kAcc = kMpad > 32 ? 32 : kMpad;
+  constexpr int kChunks = kMpad / kAcc;
   constexpr uint32_t kWBytes = kSwapTileN * kTileK;
   constexpr uint32_t kXBytes = kMpad * kTileK;
   constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kSwapTileN, kMpad);
@@ -586,7 +639,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int KB = a.K / kTileK;
     const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
     const bool scaled = (kFmt != kFmtBlock) && !a.raw;
-    if (scaled && threadIdx.x - 64 < static_cast<unsigned>(M)) ctl->sx_s[threadIdx.x - 64] = __ldg(a.sx + threadIdx.x - 64);
+    if (scaled)
+      for (int m = static_cast<int>(threadIdx.x) - 64; m < M; m += kSwapTileN) ctl->sx_s[m] = __ldg(a.sx + m);
     epi_sync();
     int i = 0, seg = 0;
     int sl = 0;  // Block_FP8: K slices consumed so far (same sequence as the MMA issuer's)
@@ -598,7 +652,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       const int n = t * kSwapTileN + row;
       // the channel scale is known before the accumulator is: fetch it now
       const float swv = (scaled && n < N) ? __ldg(a.sw + n) : 0.f;
-      uint32_t acc[kMpad];
+      uint32_t acc[kAcc];
+      const int slot_nb = seg & 1;  // non-Block: this segment's accumulator slot
       if constexpr (kBlock) {
         float facc[kMpad];
 #pragma unroll
@@ -629,19 +684,28 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 #pragma unroll
         for (int m = 0; m < kMpad; ++m) acc[m] = __float_as_uint(facc[m]);
       } else {
-        const int slot = seg & 1;
-        if (!warp_wait(&ctl->tfull[slot], (seg >> 1) & 1)) {
+        if (!warp_wait(&ctl->tfull[slot_nb], (seg >> 1) & 1)) {
           if (lane == 0) {
             record_error(kErrWaitEpilogue);
             ctl->abort_flag = 1;
           }
-        } else {
+        } else if constexpr (kChunks == 1) {
           tc_fence_after();
-          tmem_load_cols<kMpad>(taddr + slot * kMpad, acc);
+          tmem_load_cols<kMpad>(taddr + slot_nb * kMpad, acc);
           tmem_wait_ld();
-          warp_release(&ctl->tempty[slot]);
+          warp_release(&ctl->tempty[slot_nb]);
         }
       }
+      // More than 32 tokens: chunk cc of the accumulator row is read on demand
+      // (the slot is handed back after the last chunk).
+      auto load_chunk = [&](int cc) {
+        if constexpr (kChunks > 1) {
+          tc_fence_after();
+          tmem_load_cols<kAcc>(taddr + slot_nb * kMpad + cc * kAcc, acc);
+          tmem_wait_ld();
+          if (cc == kChunks - 1) warp_release(&ctl->tempty[slot_nb]);
+        }
+      };
       if (!epi_agree_ok(ctl)) break;
       if (threadIdx.x == 64 && i + len >= nk) QGD_STAMP(5);
 
@@ -650,10 +714,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       int ncontrib, jslot;
       tile_contributors(a, t, nku, U, cta, ncontrib, jslot);
       if (ncontrib == 1) {
-        if (in_n) {
+        for (int cc = 0; cc < kChunks; ++cc) {
+          load_chunk(cc);
+          if (in_n) {
 #pragma unroll
-          for (int m = 0; m < kMpad; ++m)
-            if (m < M) store_swap_final<kFmt>(acc[m], m, n, swv, ctl->sx_s, a);
+            for (int mm = 0; mm < kAcc; ++mm)
+              if (cc * kAcc + mm < M) store_swap_final<kFmt>(acc[mm], cc * kAcc + mm, n, swv, ctl->sx_s, a);
+          }
         }
         if (threadIdx.x == 64 && last_seg) QGD_STAMP(8);
       } else if (a.reduce == kCluster) {
@@ -667,11 +734,16 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int owner = row / R, lr = row % R;
         const uint32_t dst = mapa_shared(smem_u32(recv_buf), static_cast<uint32_t>(owner));
         // owner's layout: [contributor][vector][row], 16 bytes each
+        for (int cc = 0; cc < kChunks; ++cc) {
+          load_chunk(cc);
 #pragma unroll
-        for (int v = 0; v < kMpad / 4; ++v)
-          if (v < nvec)
-            st_cluster_v4(dst + static_cast<uint32_t>(((jslot * nvec + v) * R + lr) * 16), acc[4 * v], acc[4 * v + 1],
-                          acc[4 * v + 2], acc[4 * v + 3]);
+          for (int v = 0; v < kAcc / 4; ++v) {
+            const int vg = cc * (kAcc / 4) + v;
+            if (vg < nvec)
+              st_cluster_v4(dst + static_cast<uint32_t>(((jslot * nvec + vg) * R + lr) * 16), acc[4 * v],
+                            acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+          }
+        }
         mbar_arrive_remote(mapa_shared(smem_u32(&ctl->recv_bar), static_cast<uint32_t>(owner)));
         if (!mbar_wait_cluster(&ctl->recv_bar, 0)) {
           record_error(kErrWaitEpilogue);
@@ -699,16 +771,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           }
         }
       } else {
-        if (in_n) {
-          if (a.reduce == kAtomic) {
+        for (int cc = 0; cc < kChunks; ++cc) {
+          load_chunk(cc);
+          if (in_n) {
+            if (a.reduce == kAtomic) {
 #pragma unroll
-            for (int m = 0; m < kMpad; ++m)
-              if (m < M) atomic_acc<kFmt>(a.accum, static_cast<size_t>(m) * N + n, acc[m]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(swap_slot<kMpad>(a, t, jslot, row));
+              for (int mm = 0; mm < kAcc; ++mm)
+                if (cc * kAcc + mm < M)
+                  atomic_acc<kFmt>(a.accum, static_cast<size_t>(cc * kAcc + mm) * N + n, acc[mm]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(swap_slot<kMpad>(a, t, jslot, row)) + cc * (kAcc / 4);
 #pragma unroll
-            for (int v = 0; v < kMpad / 4; ++v)
-              if (v < nvec) dst[v] = make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+              for (int v = 0; v < kAcc / 4; ++v)
+                if (cc * (kAcc / 4) + v < nvec)
+                  dst[v] = make_uint4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+            }
           }
         }
         if (threadIdx.x == 64 && last_seg) QGD_STAMP(9);
@@ -721,7 +798,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
                 if (m < M)
                   store_swap_final<kFmt>(ldcg_u32(static_cast<uint32_t*>(a.accum) + static_cast<size_t>(m) * N + n),
                                          m, n, swv, ctl->sx_s, a);
-            } else {
+            } else if constexpr (kChunks == 1) {
               uint32_t sum[kMpad];
               // in the CTA's last segment every ring stage has been consumed,
               // so the ring's shared memory can stage the partials
@@ -735,6 +812,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 #pragma unroll
               for (int m = 0; m < kMpad; ++m)
                 if (m < M) store_swap_final<kFmt>(sum[m], m, n, swv, ctl->sx_s, a);
+            } else {
+              // more than 32 tokens: the contributors' rows, 32 tokens at a time
+              const size_t ring_bytes = static_cast<size_t>(stages) * (stage_w + stage_x);
+              for (int cc = 0; cc < kChunks; ++cc) {
+                const int v0 = cc * (kAcc / 4);
+                const int nv = (nvec - v0) < kAcc / 4 ? (nvec - v0) : kAcc / 4;
+                if (nv <= 0) break;
+                uint32_t sum[kAcc];
+                const int chunk = static_cast<int>(ring_bytes / (static_cast<size_t>(kSwapTileN) * nv * 16));
+                fixup_sum_range<kFmt, kAcc, kMpad>(a, t, row, ncontrib, v0, nv, last_seg ? chunk : 0, w_ring, sum);
+#pragma unroll
+                for (int mm = 0; mm < kAcc; ++mm)
+                  if (cc * kAcc + mm < M) store_swap_final<kFmt>(sum[mm], cc * kAcc + mm, n, swv, ctl->sx_s, a);
+              }
             }
           }
           if (threadIdx.x == 64) a.tickets[t] = 0u;
@@ -1300,13 +1391,25 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
 
 cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                           cudaStream_t stream) {
-  switch (fmt * 2 + (mpad == 32 ? 1 : 0)) {
-    case 0: return launch_swapab_t<kFmtFP8, 16>(tw, tx, a, stream);
-    case 1: return launch_swapab_t<kFmtFP8, 32>(tw, tx, a, stream);
-    case 2: return launch_swapab_t<kFmtINT8, 16>(tw, tx, a, stream);
-    case 3: return launch_swapab_t<kFmtINT8, 32>(tw, tx, a, stream);
-    case 4: return launch_swapab_t<kFmtBlock, 16>(tw, tx, a, stream);
-    case 5: return launch_swapab_t<kFmtBlock, 32>(tw, tx, a, stream);
+  if (fmt == kFmtFP8) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtFP8, 16>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtFP8, 32>(tw, tx, a, stream);
+      case 64: return launch_swapab_t<kFmtFP8, 64>(tw, tx, a, stream);
+      case 128: return launch_swapab_t<kFmtFP8, 128>(tw, tx, a, stream);
+    }
+  } else if (fmt == kFmtINT8) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtINT8, 16>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtINT8, 32>(tw, tx, a, stream);
+      case 64: return launch_swapab_t<kFmtINT8, 64>(tw, tx, a, stream);
+      case 128: return launch_swapab_t<kFmtINT8, 128>(tw, tx, a, stream);
+    }
+  } else if (fmt == kFmtBlock) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtBlock, 16>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtBlock, 32>(tw, tx, a, stream);
+    }
   }
   return cudaErrorInvalidValue;
 }
@@ -1351,6 +1454,7 @@ cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStrea
   const dim3 grid((a.N + kSwapTileN - 1) / kSwapTileN);
   const dim3 block(kSwapTileN);
   const bool pdl = a.pdl != 0;
+  if (mpad != 16 && mpad != 32) return cudaErrorInvalidValue;  // two-pass covers at most 32 tokens
   switch (fmt * 2 + (mpad == 32 ? 1 : 0)) {
     case 0: return launch_ex(swapab_reduce_kernel<kFmtFP8, 16>, grid, block, 0, stream, pdl, a);
     case 1: return launch_ex(swapab_reduce_kernel<kFmtFP8, 32>, grid, block, 0, stream, pdl, a);

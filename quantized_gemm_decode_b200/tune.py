@@ -60,12 +60,19 @@ SCHED_NAME = {0: "grid", 1: "persistent"}
 SMEM_PER_SM = 233472  # bytes of shared memory per SM on sm_100 (228 KB)
 
 
+def swap_mpad(M: int) -> int:
+    """Token columns of the Swap-AB MMA: the next of 16, 32, 64, 128."""
+    return 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+
+
 def two_per_sm_stages(M: int, kps: int, cluster: bool) -> int:
-    """Deepest Swap-AB ring that still lets two CTAs share an SM."""
-    mpad = 16 if M <= 16 else 32
+    """Deepest Swap-AB ring (at least 2 stages) that still lets two CTAs share an SM; 0 (the
+    deepest ring, one CTA per SM) when no such ring exists."""
+    mpad = swap_mpad(M)
     per_stage = kps * (128 * 128 + mpad * 128)
-    fixed = 1024 + 512 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
-    return max(2, min(16, (SMEM_PER_SM // 2 - fixed) // per_stage))
+    fixed = 1024 + 1024 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
+    st = min(16, (SMEM_PER_SM // 2 - fixed) // per_stage)
+    return st if st >= 2 else 0
 
 
 def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
@@ -81,14 +88,20 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
         st = two_per_sm_stages(M, kps, r == 3) if n_tiles * s > num_sms else 0
         out.append((1, s, r, 128, 0, 0, kps, st))
 
-    if M <= 32:
+    # Swap-AB: decode token counts, and up to 128 tokens for the per-token formats (the two-pass
+    # reduction covers at most 32)
+    swap_ok = M <= 32 or (M <= 128 and fmt != BLOCK_FP8)
+    reduces = (0, 1, 2) if M <= 32 else (0, 2)
+    if swap_ok:
         for kps in ((1, 2) if nkt >= 2 else (1,)):
-            for r in (0, 1, 2):
+            for r in reduces:
                 # Swap-AB, persistent: one CTA per SM at the deepest ring, or two at a ring that fits
                 out.append((1, 1, r, 128, 1, 1, kps, 0))
-                out.append((1, 1, r, 128, 1, 2, kps, two_per_sm_stages(M, kps, False)))
+                st2 = two_per_sm_stages(M, kps, False)
+                if st2:
+                    out.append((1, 1, r, 128, 1, 2, kps, st2))
         for s in splits:
-            for r in ((0,) if s == 1 else (0, 1, 2)):
+            for r in ((0,) if s == 1 else reduces):
                 swap_grid(s, r, 1)
             if nkt >= 2 and s <= (nkt + 1) // 2:
                 swap_grid(s, 0, 2)  # two K slices per stage

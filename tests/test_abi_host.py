@@ -90,9 +90,9 @@ def test_override_and_clamping():
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 256, qgd.REDUCE_ATOMIC, 5, 0, qgd.SCHEDULE_GRID)
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
     assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["source"]) == (1, 32, 2, 5, 2)
-    # Swap-AB cannot take more than 32 tokens: it falls back to Standard
+    # Swap-AB cannot take more than 128 tokens: it falls back to Standard
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, qgd.SCHEDULE_GRID)
-    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 129, 4096, 4096)
     assert p["variant"] == qgd.VARIANT_STANDARD and p["schedule"] == qgd.SCHEDULE_GRID
     with pytest.raises(qgd.QGDError):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 3, 0, 0, 0)  # split not a power of two
@@ -246,7 +246,7 @@ def test_k_slices_plan_field():
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)
     assert p["k_slices"] == 2 and p["occupancy"] == 1
     # deepest ring with two 16 KB weight slices + 2 KB activation slices per stage
-    assert p["stages"] == (232448 - 1024 - 512) // (2 * (16384 + 16 * 128))
+    assert p["stages"] == (232448 - 1024 - 1024) // (2 * (16384 + 16 * 128))
     # a single-slice K, or the Standard kernel, has one slice per stage
     assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 128)["k_slices"] == 1
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 1, 0, 0, 128, P, 0, 2)
@@ -320,7 +320,9 @@ def test_table_cluster_reduce_name(tmp_path):
 
 
 @pytest.mark.parametrize("fmt,M,N,K", [("fp8_dynamic", 1, 4096, 4096), ("w8a8_int8", 16, 34816, 5120),
-                                       ("block_fp8", 32, 5120, 25600), ("fp8_dynamic", 512, 6144, 4096)])
+                                       ("block_fp8", 32, 5120, 25600), ("fp8_dynamic", 512, 6144, 4096),
+                                       ("fp8_dynamic", 64, 24576, 4096), ("w8a8_int8", 128, 4096, 12288),
+                                       ("block_fp8", 64, 6144, 4096)])
 def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
     # every plan the tuner times is one the library runs as asked (no silent
     # legalization), and a grid-schedule Swap-AB candidate with more CTAs than
@@ -339,6 +341,22 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
         if st:
             assert p["stages"] == st
             if var == qgd.VARIANT_SWAP_AB and (sch == qgd.SCHEDULE_GRID or occ == 2):
-                mpad = 16 if M <= 16 else 32
-                smem = 1024 + st * kps * (16384 + mpad * 128) + 512 + (128 * mpad * 4 if r == 3 else 0)
+                mpad = tune.swap_mpad(M)
+                smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + (128 * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
+
+
+
+def test_swap_ab_up_to_128_tokens():
+    G = qgd.SCHEDULE_GRID
+    for M in (33, 64, 100, 128):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 4, qgd.REDUCE_TWO_PASS, 0, 0, G, 0, 1)
+        p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, M, 4096, 4096)
+        # Swap-AB covers up to 128 tokens; its two-pass kernel only 32, so the last CTA adds
+        assert p["variant"] == qgd.VARIANT_SWAP_AB and p["reduce"] == qgd.REDUCE_LAST_CTA
+        # partial rows are padded to 4 tokens
+        assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, M, 4096, 4096) == 64 * 1024 + 32 * 4 * 128 * (-(-M // 4) * 4) * 4
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 129, 4096, 4096)
+    assert p["variant"] == qgd.VARIANT_STANDARD
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, G, 0, 1)
+    assert qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 33, 4096, 4096)["variant"] == qgd.VARIANT_STANDARD

@@ -362,3 +362,30 @@ def test_cluster_split_reduction_ragged_n_and_graph():
     torch.cuda.synchronize()
     case.check_output(y, yref, bound, "cluster ragged N under graph replay")
     assert qgd.qgd_device_error() == 0
+
+
+# Swap-AB past the decode range (FP8_Dynamic and W8A8_INT8, up to 128 tokens):
+# the MMA's token dimension is 64 or 128 and the epilogue walks each
+# accumulator row 32 tokens at a time.
+SWAP_WIDE_PLANS = [(GRID, 1, 0, 0, 1), (GRID, 4, 0, 0, 2), (GRID, 4, 2, 0, 1), (GRID, 8, 3, 0, 1),
+                   (GRID, 4, 3, 0, 2), (PERSISTENT, -1, 0, 1, 1), (PERSISTENT, -1, 2, 1, 2), (PERSISTENT, -1, 0, 2, 1)]
+
+
+@pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
+@pytest.mark.parametrize("plan", SWAP_WIDE_PLANS,
+                         ids=lambda p: f"{'pers' if p[0] == PERSISTENT else 'grid'}-s{p[1]}-r{p[2]}-o{p[3]}-k{p[4]}")
+@pytest.mark.parametrize("M,N,K", [(33, 512, 1024), (64, 1024, 2048), (100, 384, 1152), (128, 640, 4096)])
+def test_swap_ab_wide_token_counts(fmt, plan, M, N, K):
+    sched, split, red, occ, kps = plan
+    case = Case(fmt, M, N, K, seed=M + 3 * K, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, split, red, 0, 0, sched, occ, kps)
+    p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
+    assert p["variant"] == qgd.VARIANT_SWAP_AB and p["reduce"] == red
+    case.check_output(case.run(), yref, bound, f"{fmt} swap wide {plan} M={M} N={N} K={K}")
+    if fmt == W8A8_INT8:
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+    assert qgd.qgd_device_error() == 0
