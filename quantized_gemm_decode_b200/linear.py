@@ -115,9 +115,16 @@ class DecodeStep:
     `calls` is a list of (layer, M); `x_host[i]` / `y_host[i]` are pinned
     host tensors of shape [M, K] / [M, N].  replay() runs the whole step
     asynchronously on the current stream; synchronize before reading y_host.
+
+    `join_every` groups the input copies: the compute stream waits once per
+    group of that many layers (for all of the group's copies) instead of once
+    per layer.  Every such wait is a dependency on a copy in the middle of the
+    chain of kernels, where the next kernel can no longer be launched early
+    behind the one before it.
     """
 
-    def __init__(self, calls, x_host, y_host):
+    def __init__(self, calls, x_host, y_host, join_every: int = 1):
+        self.join_every = max(1, int(join_every))
         self.calls = list(calls)
         dev = self.calls[0][0].device
         self.x_dev, self.y_dev, self.q = [], [], []
@@ -151,17 +158,20 @@ class DecodeStep:
                 layer.gemm(xq, sx, self.y_dev[i])
                 self.y_host[i].copy_(self.y_dev[i], non_blocking=True)
             return
-        landed = []
+        landed = {}
         copy_in.wait_stream(main)
         copy_out.wait_stream(main)
+        n = len(self.calls)
         with torch.cuda.stream(copy_in):
-            for i in range(len(self.calls)):
+            for i in range(n):
                 self.x_dev[i].copy_(self.x_host[i], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(copy_in)
-                landed.append(ev)
+                if (i + 1) % self.join_every == 0 or i == n - 1:
+                    ev = torch.cuda.Event()
+                    ev.record(copy_in)
+                    landed[i // self.join_every] = ev
         for i, (layer, M) in enumerate(self.calls):
-            main.wait_event(landed[i])
+            if i % self.join_every == 0:
+                main.wait_event(landed[i // self.join_every])
             xq, sx = self.q[i]
             layer.quantize(self.x_dev[i], xq, sx)
             layer.gemm(xq, sx, self.y_dev[i])
