@@ -713,8 +713,9 @@ def main():
         "e2e": {"value": round(path_b * world / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e, 4),
-                "how": "linear.DecodeStep: one graph per step; pinned host X -> device on a copy stream, "
-                       "quantize + GEMM per layer, Y -> pinned host on a second copy stream"},
+                "how": "linear.DecodeStep: one graph per step; pinned host X -> device on a copy stream "
+                       "(the compute stream joins them once per 4 layers), quantize + GEMM per layer, "
+                       "Y -> pinned host on a second copy stream"},
         "gpu_launches": launches,
         "clocks": clk,
     }

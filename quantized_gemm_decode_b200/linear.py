@@ -120,10 +120,12 @@ class DecodeStep:
     group of that many layers (for all of the group's copies) instead of once
     per layer.  Every such wait is a dependency on a copy in the middle of the
     chain of kernels, where the next kernel can no longer be launched early
-    behind the one before it.
+    behind the one before it.  On B200, over the 28 layers of the 8B-class
+    FP8 sweep, one wait per 4 layers was fastest (0.49 ms per step against
+    0.54 ms for one per layer and 0.63 ms for a single wait up front).
     """
 
-    def __init__(self, calls, x_host, y_host, join_every: int = 1):
+    def __init__(self, calls, x_host, y_host, join_every: int = 4):
         self.join_every = max(1, int(join_every))
         self.calls = list(calls)
         dev = self.calls[0][0].device
