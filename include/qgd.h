@@ -66,11 +66,15 @@ typedef enum {
 
 typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8 = 2 } qgd_format;
 typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
+/* Standard: X is the MMA's A operand (128-token tiles).  Swap-AB: Y^T = W X^T, the weight rows fill
+ * the MMA's 128-row slot and the tokens its N (16/32/64/128); up to 32 tokens for Block_FP8 and up
+ * to 128 for FP8_Dynamic / W8A8_INT8 (a plan asking for more gets Standard). */
 typedef enum { QGD_VARIANT_AUTO = -1, QGD_VARIANT_STANDARD = 0, QGD_VARIANT_SWAP_AB = 1 } qgd_variant;
 typedef enum {
   QGD_REDUCE_AUTO = -1,
   QGD_REDUCE_LAST_CTA = 0, /* split partials to workspace; the last CTA of each tile adds them in split order */
-  QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order */
+  QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order
+                              (Swap-AB: at most 32 tokens, else the last CTA adds them) */
   QGD_REDUCE_ATOMIC = 2,   /* split partials added atomically into a zeroed workspace (fp32 order varies) */
   QGD_REDUCE_CLUSTER = 3   /* Swap-AB grid schedule, 2 <= split_k <= 8: the splits of a tile form one
                               thread-block cluster and add their partials in split order through
@@ -80,7 +84,7 @@ typedef enum {
 typedef enum {
   QGD_SCHEDULE_AUTO = -1,
   QGD_SCHEDULE_GRID = 0,      /* one CTA per (output tile, K split): split_k CTAs along K */
-  QGD_SCHEDULE_PERSISTENT = 1 /* about one CTA per SM.  Swap-AB: all (tile, 128-wide K slice) units are
+  QGD_SCHEDULE_PERSISTENT = 1 /* about one CTA per SM.  Swap-AB: all (tile, K unit) units are
                                  dealt out in equal contiguous ranges, shared tiles finished by the last
                                  CTA.  Standard: (tile, split) items dealt round-robin, the TMEM
                                  accumulator double-buffered across a CTA's tiles */
@@ -96,7 +100,7 @@ typedef struct {
   int schedule;  /* qgd_schedule (never AUTO here) */
   int occupancy; /* persistent schedule: CTAs per SM the grid is sized for (1 or 2).  With 1 and a
                     ring under half the SM's shared memory, the next GEMM's CTA can be resident
-                    beside this one and stream its first weights while this one finishes */
+                    beside this one and do its set-up and first weight loads before this one ends */
   int source;    /* 0 = built-in default, 1 = dispatch table, 2 = override */
   int k_slices;  /* Swap-AB: 128-wide K slices per pipeline stage (1 or 2); Standard: 1.  Each stage
                     costs a fixed hand-off between the copy engine and the MMA, so one CTA per SM
