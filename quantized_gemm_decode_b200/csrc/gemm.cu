@@ -3,14 +3,17 @@
 // -> scale epilogue.  Two orientations:
 //
 //   Swap-AB   D^T[n, m] = sum_k Wq[n,k] Xq[m,k]: a CTA owns 128 weight rows
-//             (the MMA's M) and all M <= 32 tokens (the MMA's N, padded to 16
-//             or 32).  The weight stream is the whole cost at decode sizes.
+//             (the MMA's M) and all M tokens (the MMA's N, padded to 16, 32,
+//             64 or 128; at most 32 for Block_FP8).  The weight stream is the
+//             whole cost at decode sizes.
 //   Standard  D[m, n] = sum_k Xq[m,k] Wq[n,k]: a CTA owns a 128-token x
 //             tile_n-column output tile; the large-M path.
 //
 // Either one runs with split_k CTAs along K (Split-K).  Partials are added
 // by the last CTA to arrive at a tile (in split order, deterministic), by a
-// second kernel (two-pass, deterministic), or atomically.
+// second kernel (two-pass, deterministic), atomically, or -- Swap-AB -- by
+// the splits of a tile launched as one thread-block cluster, through
+// distributed shared memory (in split order, deterministic).
 //
 // Algorithm variants and their roles follow "Building a High-Performance and
 // Portable vLLM Linear Backend with Helion" (section "Como se implementa el
@@ -246,7 +249,7 @@ __device__ __forceinline__ bool epi_arrive_last(SmemCtl* ctl, const GemmArgs& a,
 }
 
 // ===========================================================================
-// Swap-AB kernel (decode, M <= 32).
+// Swap-AB kernel (decode token counts; up to 128 tokens for the per-token formats).
 //
 // Work is the linear sequence of units u = tile * nku + kp (tile = 128 weight
 // rows, kp = the kp-th group of a.kps consecutive 128-wide K slices, one

@@ -29,15 +29,15 @@ def test_bucket_graphs_match_eager(fmt):
         assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"M={M}"
 
 
-@pytest.mark.parametrize("join_every", [1, 2, 4])
-def test_decode_step_with_host_io_matches_eager(join_every):
+@pytest.mark.parametrize("join_every,out_every", [(1, 1), (2, 1), (4, 1), (2, 2), (1, 3)])
+def test_decode_step_with_host_io_matches_eager(join_every, out_every):
     layers = [QuantizedLinear(synth.weights(1536, 1024, seed=51).cuda(), "fp8_dynamic"),
               QuantizedLinear(synth.weights(1024, 2048, seed=52).cuda(), "w8a8_int8"),
               QuantizedLinear(synth.weights(512, 1024, seed=53).cuda(), "block_fp8")]
     ms = (4, 16, 1)
     xh = [synth.activations(m, l.K, seed=60 + i, outliers=True).pin_memory() for i, (l, m) in enumerate(zip(layers, ms))]
     yh = [torch.empty((m, l.N), dtype=torch.bfloat16).pin_memory() for l, m in zip(layers, ms)]
-    step = DecodeStep(list(zip(layers, ms)), xh, yh, join_every=join_every)
+    step = DecodeStep(list(zip(layers, ms)), xh, yh, join_every=join_every, out_every=out_every)
     for rnd in range(2):
         if rnd == 1:  # new inputs in the same pinned buffers
             for i, (l, m) in enumerate(zip(layers, ms)):
