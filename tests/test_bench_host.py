@@ -47,7 +47,7 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
 
 
 def test_decode_sweeps_match_the_configured_shapes():
-    assert workloads.FP8_DECODE.shapes == [(6144, 4096), (4096, 4096), (24576, 4096), (4096, 12288)]
+    assert list(workloads.FP8_DECODE.shapes) == [(6144, 4096), (4096, 4096), (24576, 4096), (4096, 12288)]
     assert list(workloads.FP8_DECODE.ms) == [1, 2, 4, 8, 16, 24, 32]
     for wl in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE):
         for n, k in wl.shapes:
