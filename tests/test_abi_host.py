@@ -360,3 +360,22 @@ def test_swap_ab_up_to_128_tokens():
     assert p["variant"] == qgd.VARIANT_STANDARD
     qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_SWAP_AB, 4, 0, 0, 0, G, 0, 1)
     assert qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 33, 4096, 4096)["variant"] == qgd.VARIANT_STANDARD
+
+
+def test_shipped_table_covers_every_benchmarked_shape():
+    # the shipped table parses, names only legal plans, and has an entry for every
+    # (format, N, K, M) the benchmark runs, so no benchmarked call falls back to
+    # the built-in default
+    from quantized_gemm_decode_b200 import workloads
+
+    qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
+    fid = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2}
+    for wl in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, *workloads.LARGE):
+        for (N, K) in wl.shapes:
+            for M in wl.ms:
+                p = qgd.qgd_get_plan(fid[wl.fmt], M, N, K)
+                assert p["source"] == 1, (wl.fmt, N, K, M)
+                if p["variant"] == qgd.VARIANT_SWAP_AB:
+                    assert M <= (32 if wl.fmt == "block_fp8" else 128)
+                # the workspace the plan needs is what the size query reports
+                assert qgd.qgd_workspace_size(fid[wl.fmt], M, N, K) >= 0
