@@ -304,8 +304,8 @@ def replay_times(g: torch.cuda.CUDAGraph, reps: int, warmup: int = 3) -> list:
 
 def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
     """Time of each call, cycling through all weight copies of its shape (at
-    least 3x L2 of distinct weights), one graph per call: the GEMM alone (mean
-    and p90 over replays) and the whole layer call (quantize + GEMM)."""
+    least 3x L2 of distinct weights), one graph per call: the GEMM alone (mean,
+    median and p90 over replays) and the whole layer call (quantize + GEMM)."""
     rows = []
     for c in ds.calls:
         ncop = len(ds.weights[(c["N"], c["K"])])
@@ -322,6 +322,7 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
         g = ds.capture(body)
         times = replay_times(g, reps)
         ms = statistics.mean(times) / ncop
+        med = statistics.median(times) / ncop
         p90 = sorted(times)[int(0.9 * (len(times) - 1))] / ncop
         del g
         g = ds.capture(layer)
@@ -331,7 +332,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
         f = workloads.flops(c["M"], c["N"], c["K"])
         p = ds.qgd.qgd_get_plan(ds.fmt_id, c["M"], c["N"], c["K"])
         pb = path_bytes(ds.fmt, c["M"], c["N"], c["K"])
-        rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3), "p90_us": round(p90 * 1e3, 3),
+        rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3), "median_us": round(med * 1e3, 3),
+                     "p90_us": round(p90 * 1e3, 3),
                      "gbs": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / peak_gbs, 4),
                      "tflops": round(f / (ms * 1e-3) / 1e12, 2),
                      "layer_us": round(ms_layer * 1e3, 3),
