@@ -9,7 +9,9 @@ Weights rotate over enough copies that every call streams them from HBM
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qgd|reference] [--quick]
 
-Prints one JSON line on rank 0.  Under torchrun each rank runs an independent
+Prints, on rank 0, the detail sections (per-call tables, larger-M rows, CPU
+baseline) as lines starting with 'detail ', then the result as one compact
+JSON line, always the last line of stdout.  Under torchrun each rank runs an independent
 replica on its own GPU (the path has no exchange step); the reported value
 is the bytes all ranks moved divided by the slowest rank's time.
 """
@@ -519,6 +521,128 @@ def oracle_sample(wl: workloads.Workload, budget_s: float, host_w: dict | None =
     return tot_b, tot_s, note
 
 
+def oracle_large_m_sample(fmt: str = FP8_DYNAMIC, M: int = 8192, N: int = 24576, K: int = 4096,
+                          rows: int = 16, cols: int = ORACLE_ROWS, seed: int = 1004):
+    """The oracle on a sample of one larger-M GEMM: `rows` tokens x `cols`
+    weight rows (quantize the sampled activation rows, then the product).
+    Returns the sample's seconds; the full call's time is extrapolated by the
+    ratio of output elements (every output costs the same K-long dot)."""
+    import oracle
+
+    w = synth.weights(cols, K, seed)
+    x = synth.activations(rows, K, seed, outliers=(fmt != W8A8_INT8))
+    if fmt == BLOCK_FP8:
+        wq, sw = oracle.quant_blocks(w, 128)
+        t0 = time.perf_counter()
+        xq, sx = oracle.quant_groups(x, 128)
+        oracle.gemm_blockscaled(xq, sx, wq, sw, 128)
+    else:
+        qt = oracle.INT8 if fmt == W8A8_INT8 else oracle.E4M3
+        wq, sw = oracle.quant_rows(w, qt)
+        t0 = time.perf_counter()
+        xq, sx = oracle.quant_rows(x, qt)
+        oracle.gemm_rowscaled(xq, sx, wq, sw, qt)
+    dt = time.perf_counter() - t0
+    return dt, dt * (M * N) / (rows * cols)
+
+
+def cpu_baseline_leg(wl: workloads.Workload, host_w: dict | None, budget_all: float = 10.0,
+                     budget_one: float = 5.0) -> dict:
+    """The oracle as it stands on this host's cores: the decode sweep sampled
+    on all cores and on one thread, and one larger-M call sampled (its full
+    time extrapolated, and labelled so)."""
+    import oracle
+
+    all_threads = oracle.num_threads()
+    b, s, note = oracle_sample(wl, budget_all, host_w)
+    oracle.set_num_threads(1)
+    try:
+        b1, s1, _ = oracle_sample(wl, budget_one, host_w)
+        lm1, lm1_full = oracle_large_m_sample()
+    finally:
+        oracle.set_num_threads(all_threads)
+    lm, lm_full = oracle_large_m_sample()
+    return {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": all_threads, "kind": "oracle",
+            "sample": note[:160] + f"; {s:.1f} s of oracle time",
+            "cpu_model": oracle.cpu_model(),
+            "single_thread": {"value": round(b1 / s1 / 1e9, 4), "unit": "GB/s", "cores": 1, "seconds": round(s1, 1)},
+            "large_m": {"call": "fp8_dynamic M=8192 N=24576 K=4096",
+                        "sample": f"16 tokens x {ORACLE_ROWS} weight rows",
+                        "sample_s": round(lm, 3), "sample_s_1_thread": round(lm1, 3),
+                        "full_s_extrapolated": round(lm_full, 1),
+                        "full_s_1_thread_extrapolated": round(lm1_full, 1),
+                        "label": "full times extrapolated from the sample by output count, not measured"}}
+
+
+HEADLINE_MAX_BYTES = 3500  # the result line stays far below what a log tail keeps
+
+
+def headline(out: dict) -> dict:
+    """The one-line result: the keys a reader of the run needs, compact.
+    Per-call tables and per-shape larger-M rows stay in the detail record."""
+    keep = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+            "vs_baseline", "dtype", "data", "tflops", "frac_of_hbm_peak", "frac_of_8tbs", "gpu_launches")
+    line = {k: out[k] for k in keep if k in out}
+    cfg = out.get("config", {})
+    line["config"] = {k: cfg[k] for k in ("workload", "format", "shapes", "ms", "calls_per_step", "l2", "parallelism")
+                      if k in cfg}
+    rf = out.get("roofline")
+    if rf:
+        line["roofline"] = {k: rf[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source",
+                                               "avg_launch_us", "algorithmic_bytes_per_launch") if k in rf}
+    if "e2e" in out:
+        line["e2e"] = {k: out["e2e"][k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step",
+                                                  "ms_per_step") if k in out["e2e"]}
+    if "clocks" in out:
+        line["clocks"] = {k: out["clocks"].get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "power_w_max")}
+    if "cpu_baseline" in out:
+        cb = out["cpu_baseline"]
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "cpu_model",
+                                                   "single_thread") if k in cb}
+        if "large_m" in cb:
+            lm = cb["large_m"]
+            line["cpu_baseline"]["large_m_full_s_extrapolated"] = lm.get("full_s_extrapolated")
+    if "formats" in out:
+        line["formats"] = {f: {k: v[k] for k in ("gbs", "frac", "ms_per_step") if k in v} |
+                           ({"quant_us": v["quantizer"]["us_per_call"]} if "quantizer" in v else {})
+                           for f, v in out["formats"].items()}
+    if "tensor_probe" in out:
+        line["tensor_probe"] = {k: out["tensor_probe"][k] for k in ("e4m3_tflops", "int8_tops")
+                                if k in out["tensor_probe"]}
+    if "large_m" in out:
+        summ = {}
+        for f, rows in out["large_m"].items():
+            big = [r for r in rows if r["M"] == max(x["M"] for x in rows)]
+            summ[f] = {"M": big[0]["M"] if big else None,
+                       "frac": round(statistics.mean(r["frac"] for r in big), 4) if big else None,
+                       "best_tflops": max((r["tflops"] for r in big), default=None)}
+            if big and "frac_probe" in big[0]:
+                summ[f]["frac_probe"] = round(statistics.mean(r["frac_probe"] for r in big), 4)
+        line["large_m"] = summ
+    if "detail" in out:
+        line["detail"] = out["detail"]
+    return line
+
+
+def emit(out: dict, detail_path: str | None, stream=None) -> str:
+    """Print the detail sections (lines starting 'detail '), write them to
+    `detail_path` if given, then print the headline as the last line."""
+    stream = stream or sys.stdout
+    big = {k: out[k] for k in ("per_call", "formats", "large_m", "tensor_probe", "cpu_baseline", "roofline",
+                               "e2e", "splitk_modes", "chain", "fused") if k in out}
+    for k, v in big.items():
+        stream.write(f"detail {k} {json.dumps(v)}\n")
+    if detail_path:
+        os.makedirs(os.path.dirname(os.path.abspath(detail_path)), exist_ok=True)
+        with open(detail_path, "w") as f:
+            json.dump(out, f, indent=1)
+        out = dict(out, detail=os.path.relpath(detail_path, ROOT))
+    line = json.dumps(headline(out))
+    stream.write(line + "\n")
+    stream.flush()
+    return line
+
+
 def run_reference(args, dist: Dist):
     if dist.rank != 0:
         return 0
@@ -604,6 +728,8 @@ def main():
                                                          "other formats, large M or CPU baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out", default=None, help="also write the JSON line to this file")
+    ap.add_argument("--detail-out", default=None, metavar="PATH",
+                    help="write the full record (per-call tables, larger-M rows, CPU baseline) to this JSON file")
     ap.add_argument("--case", default=None, metavar="FMT:M:N:K",
                     help="time one GEMM shape (eager launches, for profilers) instead of the workload")
     args = ap.parse_args()
@@ -742,14 +868,9 @@ def main():
         out.update(extra)
         ds = keep
     if dist.rank == 0 and dist.world == 1 and not args.quick and not args.no_cpu_baseline:
-        b, s, note = oracle_sample(wl, 15.0, ds.host_w)
-        import oracle
-
-        out["cpu_baseline"] = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-                               "kind": "oracle", "sample": note + f"; {s:.1f} s of oracle time"}
+        out["cpu_baseline"] = cpu_baseline_leg(wl, ds.host_w)
     if dist.rank == 0:
-        line = json.dumps(out)
-        print(line, flush=True)
+        line = emit(out, args.detail_out)
         if args.out:
             with open(args.out, "w") as f:
                 f.write(line + "\n")

@@ -162,23 +162,27 @@ QGD_API qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void
 QGD_API qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
                                size_t ws_bytes, void* stream);
 
-/* FP8_Dynamic GEMM for callers that cannot allocate device memory -- for
- * example a caller whose stream is being captured into a CUDA graph, or an
- * engine that hands out all device memory from pools fixed at start-up, where
- * a cudaMalloc would fail, stall the device or break the capture.  It is
- * qlinear_fp8_dynamic without the workspace arguments: the caller still
- * passes inputs and output, and the Split-K scratch comes from a fixed 8 MiB
- * array inside the library (held by every GPU that loads it until exit).
- * The pages have no counterpart; this is an addition of this library.
+/* FP8_Dynamic GEMM for callers that cannot allocate device memory while they
+ * run -- for example an inference engine that splits all device memory into
+ * fixed pools at start-up and has none left for a per-call workspace, or a
+ * latency-critical loop where a cudaMalloc may block until the device is
+ * idle.  It is qlinear_fp8_dynamic without the workspace arguments: the
+ * caller still passes inputs and output, and the Split-K scratch comes from a
+ * fixed 8 MiB array inside the library (held by every GPU that loads it until
+ * exit).  The pages have no counterpart; this is an addition of this library.
  *   - The plan is the same as qlinear_fp8_dynamic's; a plan whose Split-K
  *     scratch exceeds 8 MiB (64 KiB of counters + partials) is rejected with
  *     QGD_ERR_WORKSPACE before anything is launched.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
- *   - All calls share the one array: calls that overlap on the GPU (other
- *     streams, other threads) race and give undefined results.  Each call
- *     clears the counters it uses with a memset node, then runs the GEMM.
- *   - Nothing is allocated or freed. */
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps what the last call left in
+ *     it: calls that overlap on the GPU (other streams, other threads) race
+ *     and give undefined results.  A call that splits K first clears the
+ *     counters it uses with a memset, then runs the GEMM (launched without a
+ *     programmatic dependency, since it follows a memset).
+ *   - Nothing is allocated or freed: no cudaMalloc/cudaFree, no allocating
+ *     library routine. */
 QGD_API qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const void* wq, const float* sw,
                                                void* y_bf16, int M, int N, int K, void* stream);
 
@@ -242,6 +246,17 @@ QGD_API qgd_status qgd_clear_device_error(void);
  * QGD_ERR_INVALID.  A wait that gives up is reported by qgd_device_error().
  * --------------------------------------------------------------------- */
 QGD_API qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream);
+
+/* Test hook for the failure-detection path (the pages have no counterpart).
+ * While on (on != 0), GEMMs launched from then on in the Swap-AB orientation
+ * never signal the epilogue that an accumulator is complete -- a flag that
+ * nothing sets -- so the epilogue's bounded wait runs out after about one
+ * second.  The kernel then records error 3 (epilogue wait) for
+ * qgd_device_error(), waits for the copies and MMAs it issued, frees its
+ * tensor memory and returns without writing Y; the context stays usable.
+ * No other kernel is affected.  Host-global, for tests only; not
+ * thread-safe against concurrent qlinear_* calls.  Always QGD_OK. */
+QGD_API qgd_status qgd_test_withhold_accumulator(int on);
 
 /* Library version, "major.minor.patch". */
 QGD_API const char* qgd_version(void);

@@ -65,6 +65,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.orc_dot_split.argtypes = [P, lg, P, lg, lg, ctypes.c_int, lg]
     L.orc_num_threads.restype = ctypes.c_int
     L.orc_num_threads.argtypes = []
+    L.orc_set_num_threads.restype = ctypes.c_int
+    L.orc_set_num_threads.argtypes = [ctypes.c_int]
     return L
 
 
@@ -186,3 +188,20 @@ def dot_split(xq, m: int, wq, n: int, qtype: int, splits: int) -> int:
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+def set_num_threads(n: int) -> int:
+    """Run the GEMMs on n threads from now on; returns the count in force."""
+    return lib().orc_set_num_threads(int(n))
+
+
+def cpu_model() -> str:
+    """Model name of the host CPU (from /proc/cpuinfo), or '' if unknown."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""

@@ -353,3 +353,18 @@ int orc_num_threads(void)
     return 1;
 #endif
 }
+
+/* Run the GEMMs above on n OpenMP threads from now on (n >= 1); returns the
+ * count in force afterwards.  Only the timing of the CPU baseline uses this:
+ * the thread count changes no result (every output is one thread's sum). */
+int orc_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+    return orc_num_threads();
+}

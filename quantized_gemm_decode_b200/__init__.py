@@ -16,6 +16,7 @@ raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 
@@ -30,7 +31,7 @@ __all__ = [
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
-    "qgd_mma_peak_probe",
+    "qgd_mma_peak_probe", "qgd_test_withhold_accumulator",
     "Workspace", "DEFAULT_TABLE",
 ]
 
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
             "qgd_device_error": [ctypes.POINTER(ctypes.c_uint)],
             "qgd_clear_device_error": [],
             "qgd_mma_peak_probe": [I, I, ctypes.POINTER(ctypes.c_double), P],
+            "qgd_test_withhold_accumulator": [I],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -234,13 +236,44 @@ def _workspace(fmt: int, M: int, N: int, K: int, ws, device):
 # ---------------------------------------------------------------------------
 # GEMMs
 # ---------------------------------------------------------------------------
-def _qlinear(fn_name: str, fmt: int, xq, sx, wq, sw, y, ws, stream):
-    _cuda_2d(xq, "xq", _BYTE_TYPES)
-    _cuda_2d(wq, "wq", _BYTE_TYPES)
+def _check_operands(fmt: int, xq, sx, wq, sw, y) -> tuple:
+    """Shapes, dtypes and placement of a GEMM's operands, checked before
+    anything reaches the library (which sees only pointers and sizes).
+    Returns (M, N, K)."""
+    for t, name in ((xq, "xq"), (wq, "wq")):
+        if not isinstance(t, torch.Tensor) or t.dim() != 2:
+            raise ValueError(f"{name} must be a 2-D tensor")
     M, K = xq.shape
     N = wq.shape[0]
     if wq.shape[1] != K:
         raise ValueError(f"K mismatch: xq {tuple(xq.shape)} vs wq {tuple(wq.shape)}")
+    want_x = (torch.int8,) if fmt == FMT_W8A8_INT8 else (torch.uint8, torch.float8_e4m3fn)
+    for t, name in ((xq, "xq"), (wq, "wq")):
+        if t.dtype not in want_x:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected one of {want_x}")
+    if fmt == FMT_BLOCK_FP8:
+        sx_shape, sw_shape = (M, K // 128), (N // 128, K // 128)
+    else:
+        sx_shape, sw_shape = (M,), (N,)
+    for t, name, shape in ((sx, "sx", sx_shape), (sw, "sw", sw_shape)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 tensor")
+        if t.numel() < math.prod(shape):
+            raise ValueError(f"{name} holds {t.numel()} scales, {shape} = {math.prod(shape)} needed")
+    if y is not None:
+        if not isinstance(y, torch.Tensor) or y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) \
+                or not y.is_contiguous():
+            raise ValueError(f"y must be a contiguous bfloat16 tensor of shape {(M, N)}")
+    for t, name in ((xq, "xq"), (wq, "wq"), (sx, "sx"), (sw, "sw"), (y, "y")):
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    _cuda_2d(xq, "xq", _BYTE_TYPES)
+    _cuda_2d(wq, "wq", _BYTE_TYPES)
+    return M, N, K
+
+
+def _qlinear(fn_name: str, fmt: int, xq, sx, wq, sw, y, ws, stream):
+    M, N, K = _check_operands(fmt, xq, sx, wq, sw, y)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
     wsp, wsn = _workspace(fmt, M, N, K, ws, xq.device)
@@ -266,12 +299,13 @@ def qlinear_block_fp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
 
 
 def qlinear_fp8_dynamic_noalloc(xq, sx, wq, sw, y, stream=None):
-    """FP8_Dynamic GEMM into a caller-provided y, with no workspace and no
-    allocation of any kind (the library's built-in scratch is used)."""
-    _cuda_2d(xq, "xq", _BYTE_TYPES)
-    _cuda_2d(wq, "wq", _BYTE_TYPES)
-    M, K = xq.shape
-    N = wq.shape[0]
+    """FP8_Dynamic GEMM into a caller-provided y that allocates nothing: no
+    workspace argument, no allocation by the binding or the library (the
+    library's built-in Split-K scratch is used).  y must be a bf16 [M, N]
+    CUDA tensor; every operand is checked before the call."""
+    if y is None:
+        raise ValueError("qlinear_fp8_dynamic_noalloc writes into a caller-provided y; y is None")
+    M, N, K = _check_operands(FMT_FP8_DYNAMIC, xq, sx, wq, sw, y)
     _check(lib().qlinear_fp8_dynamic_noalloc(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K,
                                              _stream(stream)), "qlinear_fp8_dynamic_noalloc")
     return y
@@ -341,6 +375,12 @@ def qgd_mma_peak_probe(qtype: int = QTYPE_E4M3, iters: int = 4096, stream=None) 
     flops = ctypes.c_double(0.0)
     _check(lib().qgd_mma_peak_probe(qtype, iters, ctypes.byref(flops), _stream(stream)), "qgd_mma_peak_probe")
     return float(flops.value)
+
+
+def qgd_test_withhold_accumulator(on: bool) -> None:
+    """Failure-detection test hook: while on, Swap-AB GEMMs never signal a
+    finished accumulator, so their epilogue's bounded wait runs out."""
+    _check(lib().qgd_test_withhold_accumulator(1 if on else 0), "qgd_test_withhold_accumulator")
 
 
 def qgd_version() -> str:

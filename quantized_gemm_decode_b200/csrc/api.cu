@@ -344,6 +344,7 @@ bool pdl_enabled() {
 }
 
 std::atomic<int> g_call_seq{0};  // numbers GEMM calls for the developer timeline
+std::atomic<int> g_withhold_acc{0};  // qgd_test_withhold_accumulator
 
 qgd_status check_shape(int fmt, int M, int N, int K) {
   if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d N=%d K=%d)", M, N, K);
@@ -355,8 +356,11 @@ qgd_status check_shape(int fmt, int M, int N, int K) {
   return QGD_OK;
 }
 
+// follows_memset: the caller has just enqueued a memset on `stream`, so the
+// GEMM is launched without a programmatic dependency (that relaxation is
+// defined between two kernels only).
 qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, const float* sw, void* y, void* raw,
-                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream, bool follows_memset = false) {
   qgd_status st = check_shape(fmt, M, N, K);
   if (st != QGD_OK) return st;
   if (M == 0) return QGD_OK;
@@ -398,8 +402,9 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.maxc = ex.maxc;
   a.mstride = ex.mstride;
   a.kps = p.k_slices;
-  a.pdl = pdl_enabled() ? 1 : 0;
+  a.pdl = (pdl_enabled() && !follows_memset) ? 1 : 0;
   a.trace_tag = g_call_seq.fetch_add(1, std::memory_order_relaxed) & 0x7fffffff;
+  a.withhold_acc = g_withhold_acc.load(std::memory_order_relaxed);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
@@ -428,13 +433,15 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
 }
 
 // ---------------------------------------------------------------------------
-// Built-in scratch for qlinear_fp8_dynamic_noalloc.  Some callers cannot
-// allocate device memory (their allocator is closed after start-up, or the
-// call is being captured into a CUDA graph); they get the Split-K workspace
-// from this fixed array instead.  Every GPU that loads the library holds it
-// until the process exits.  Its first 64 KiB are the arrival-counter header
-// (zero at load, left zero by every call, and cleared again at the start of
-// each call); the rest holds Split-K partials.
+// Built-in scratch for qlinear_fp8_dynamic_noalloc.  Some callers must not
+// allocate device memory once they are running: an engine that carves all
+// device memory into fixed pools at start-up has none left to give, and a
+// cudaMalloc in a latency-critical loop can block until the device is idle.
+// They get the Split-K workspace from this fixed array instead.  Every GPU
+// that loads the library holds it until the process exits.  Its first 64 KiB
+// are the arrival-counter header (zero at load, left zero by every call, and
+// cleared again at the start of each call that splits K); the rest holds
+// Split-K partials.
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -550,7 +557,8 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
     cudaError_t e = cudaMemsetAsync(scratch, 0, ex.tiles * 4, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (built-in scratch counters)");
   }
-  return run_gemm(kFmtFP8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, scratch, kNoAllocScratchBytes, stream);
+  return run_gemm(kFmtFP8, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, scratch, kNoAllocScratchBytes, stream,
+                  ex.total > 0);
 }
 
 size_t qgd_workspace_size(int fmt, int M, int N, int K) {
@@ -679,6 +687,11 @@ qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream)
   if (flops) *flops = mma_probe_flops(iters, g_num_sms);
   cudaError_t e = launch_mma_probe(qtype, iters, g_num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "qgd_mma_peak_probe launch");
+}
+
+qgd_status qgd_test_withhold_accumulator(int on) {
+  g_withhold_acc.store(on ? 1 : 0, std::memory_order_relaxed);
+  return QGD_OK;
 }
 
 const char* qgd_version(void) { return "0.1.0"; }

@@ -620,13 +620,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
             mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
           }
           if (kBlock) {
-            mma_commit(&ctl->tfull[slot]);
+            if (!a.withhold_acc) mma_commit(&ctl->tfull[slot]);
             ++sl;
           }
         }
         if (stop) break;
         mma_commit(&ctl->empty[s]);
-        if (!kBlock && seg_end) mma_commit(&ctl->tfull[seg & 1]);
+        // (withhold_acc: the failure-detection test leaves the epilogue's
+        // accumulator barrier unsignalled, so its bounded wait runs out)
+        if (!kBlock && seg_end && !a.withhold_acc) mma_commit(&ctl->tfull[seg & 1]);
         if (seg_end) ++seg;
       }
       QGD_STAMP(4);

@@ -45,6 +45,7 @@ struct GemmArgs {
   int kps;         // Swap-AB: 128-wide K slices per pipeline stage (1 or 2)
   int pdl;         // launch with a programmatic dependency on the preceding kernel
   int trace_tag;   // sequence number of the call (developer timeline builds file stamps by it)
+  int withhold_acc;  // failure-detection test: Swap-AB never signals a finished accumulator
 };
 
 // Launchers (gemm.cu).  Each returns the cudaError_t of the launch.

@@ -379,3 +379,41 @@ def test_shipped_table_covers_every_benchmarked_shape():
                     assert M <= (32 if wl.fmt == "block_fp8" else 128)
                 # the workspace the plan needs is what the size query reports
                 assert qgd.qgd_workspace_size(fid[wl.fmt], M, N, K) >= 0
+
+
+def test_binding_checks_gemm_operands_before_any_launch():
+    # CPU tensors: every shape / dtype / size check runs before the device
+    # check, so each mistake is reported as what it is, and nothing reaches
+    # the library
+    import torch
+
+    M, N, K = 4, 256, 512
+    f8 = torch.float8_e4m3fn
+    xq = torch.zeros((M, K), dtype=f8)
+    wq = torch.zeros((N, K), dtype=f8)
+    sx = torch.ones(M)
+    sw = torch.ones(N)
+    y = torch.zeros((M, N), dtype=torch.bfloat16)
+    cases = [
+        (dict(wq=torch.zeros((N, K - 128), dtype=f8)), "K mismatch"),
+        (dict(sx=torch.ones(M - 1)), "sx holds"),
+        (dict(sw=torch.ones(N - 16)), "sw holds"),
+        (dict(sw=torch.ones(N, dtype=torch.float64)), "sw must be"),
+        (dict(y=torch.zeros((M, N - 16), dtype=torch.bfloat16)), "y must be"),
+        (dict(y=torch.zeros((M, N), dtype=torch.float32)), "y must be"),
+        (dict(xq=torch.zeros((M, K), dtype=torch.int8)), "xq has dtype"),
+        ({}, "must be a CUDA tensor"),
+    ]
+    for change, msg in cases:
+        args = dict(xq=xq, sx=sx, wq=wq, sw=sw, y=y) | change
+        for fn in (qgd.qlinear_fp8_dynamic, qgd.qlinear_fp8_dynamic_noalloc):
+            with pytest.raises(ValueError, match=msg):
+                fn(args["xq"], args["sx"], args["wq"], args["sw"], y=args["y"])
+    with pytest.raises(ValueError, match="y is None"):
+        qgd.qlinear_fp8_dynamic_noalloc(xq, sx, wq, sw, None)
+    # Block_FP8 scales: [M, K/128] and [N/128, K/128]
+    with pytest.raises(ValueError, match="sw holds"):
+        qgd.qlinear_block_fp8(xq, torch.ones(M, K // 128), wq, torch.ones(N // 128, K // 128 - 1), y=y)
+    # W8A8_INT8 codes are int8
+    with pytest.raises(ValueError, match="xq has dtype"):
+        qgd.qlinear_w8a8_int8(xq, sx, wq, sw, y=y)

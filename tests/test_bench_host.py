@@ -52,3 +52,66 @@ def test_decode_sweeps_match_the_configured_shapes():
     for wl in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE):
         for n, k in wl.shapes:
             assert n % 128 == 0 and k % 128 == 0
+
+
+def _fake_result():
+    """A result shaped like a full run's: three formats' per-call tables,
+    the larger-M rows, the CPU baseline, clocks and the roofline."""
+    row = {"M": 8, "N": 4096, "K": 12288, "us": 14.37, "median_us": 14.082, "p90_us": 15.1, "gbs": 3515.0,
+           "frac": 0.5371, "tflops": 56.04, "layer_us": 14.835, "layer_gbs": 3411.4, "plan": "swap/s8/r3/st2/k2"}
+    per_call = [dict(row) for _ in range(28)]
+    lrow = {"M": 8192, "N": 24576, "K": 4096, "us": 700.0, "tflops": 2300.0, "gbs": 900.0, "bound": "tensor",
+            "frac": 0.66, "frac_spec": 0.5, "plan": "std/pers1/r0/st4/k1", "frac_probe": 0.5}
+    large = {f: [dict(lrow, M=m) for m in workloads.LARGE_M for _ in range(4)] for f in workloads.FORMATS}
+    fmts = {f: {"workload": f + "_decode_sweep", "ms_per_step": 0.4, "gbs": 3400.0, "frac": 0.52,
+                "quantizer": {"us_per_call": 1.9, "bytes_per_step": 1000, "gbs": 100.0}, "per_call": per_call}
+            for f in workloads.FORMATS}
+    return {
+        "metric": bench.METRIC, "value": 3455.1, "unit": "GB/s", "n_gpus": 1, "steps": 20, "warmup": 5,
+        "ms_per_step": 0.394, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": workloads.FP8_DECODE.name, "format": FP8_DYNAMIC,
+                   "shapes": [list(s) for s in workloads.FP8_DECODE.shapes], "ms": list(workloads.FP8_DECODE.ms),
+                   "calls_per_step": 28, "graph": "one CUDA graph per step", "l2": "inputs larger than L2 " * 4,
+                   "parallelism": "replicas x1"},
+        "tflops": 20.0, "frac_of_hbm_peak": 0.53, "frac_of_8tbs": 0.43,
+        "roofline": {"bound": "hbm", "kernel": "GEMM", "achieved": 3777.0, "peak": 6545.0, "unit": "GB/s",
+                     "frac": 0.577, "peak_source": "measured", "traffic": 50_000_000, "traffic_case": "x" * 80,
+                     "avg_launch_us": 12.866, "algorithmic_bytes_per_launch": 48_590_000},
+        "e2e": {"value": 2782.0, "unit": "GB/s", "h2d_bytes_per_step": 1_000_000, "d2h_bytes_per_step": 3_000_000,
+                "ms_per_step": 0.49, "how": "y" * 200},
+        "gpu_launches": 1120, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "power_w_max": 700.0,
+                                         "samples": 40, "reasons": []},
+        "formats": fmts, "tensor_probe": {"e4m3_tflops": 4443.0, "int8_tops": 4588.0, "how": "z" * 120},
+        "large_m": large, "per_call": per_call,
+        "cpu_baseline": {"value": 0.047, "unit": "GB/s", "cores": 16, "kind": "oracle", "sample": "s" * 200,
+                         "cpu_model": "Some CPU @ 2.70GHz",
+                         "single_thread": {"value": 0.006, "unit": "GB/s", "cores": 1, "seconds": 5.0},
+                         "large_m": {"full_s_extrapolated": 4000.0, "label": "extrapolated"}},
+    }
+
+
+def test_result_line_is_compact_and_last(tmp_path):
+    import io
+    import json
+
+    detail = tmp_path / "detail.json"
+    out = io.StringIO()
+    line = bench.emit(_fake_result(), str(detail), stream=out)
+    lines = out.getvalue().splitlines()
+    assert lines[-1] == line
+    assert len(line) < bench.HEADLINE_MAX_BYTES, len(line)
+    parsed = json.loads(line)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "dtype", "config", "roofline", "e2e", "cpu_baseline", "clocks", "gpu_launches"):
+        assert k in parsed, k
+    assert parsed["value"] > 0 and parsed["config"]["workload"] == workloads.FP8_DECODE.name
+    for k in ("achieved", "peak", "frac", "traffic", "bound", "unit"):
+        assert k in parsed["roofline"]
+    assert parsed["e2e"]["h2d_bytes_per_step"] > 0 and parsed["e2e"]["d2h_bytes_per_step"] > 0
+    assert parsed["cpu_baseline"]["cores"] == 16 and parsed["cpu_baseline"]["single_thread"]["cores"] == 1
+    # every earlier line is a detail section, none of which parses as a result
+    assert all(ln.startswith("detail ") for ln in lines[:-1])
+    # the full record went to the detail file
+    full = json.loads(detail.read_text())
+    assert len(full["per_call"]) == 28 and len(full["large_m"][FP8_DYNAMIC]) == 20

@@ -3,8 +3,11 @@ benchmark times (the shipped dispatch table, no overrides).
 
 For every (N, K) of the three decode sweeps, at a few token counts, the GPU
 computes the whole Y; the oracle computes a sample of it -- all M tokens
-against the first and last 128-row bands of weight rows (whole bands, so Block_FP8's
-128 x 128 weight scales are the oracle's own) -- from the same seeded inputs,
+against 128-row bands of weight rows: the first and the last, and two
+interior bands where the plan's work partition puts CTA boundaries inside a
+tile (so tiles summed from several CTAs' partials are compared at full size),
+whole bands so Block_FP8's 128 x 128 weight scales are the oracle's own --
+from the same seeded inputs,
 quantizing them itself.  The larger-M set is sampled in both tokens and
 weight rows.  Bars as everywhere: bit-exact codes and scales, one bf16 ulp
 for W8A8_INT8, the FP8 tolerance otherwise.
@@ -95,6 +98,31 @@ def _check(fmt, y_gpu, y_ref, bound, K, what):
         check_fp8_tolerance(y_gpu, y_ref, bound, K, what)
 
 
+def _interior_bands(plan: dict, M: int, N: int, K: int) -> list:
+    """Two interior 128-row weight bands that several CTAs contribute to.
+    Persistent Swap-AB deals the (tile, K unit) units out in equal contiguous
+    ranges, CTA c taking [c*U/G, (c+1)*U/G): the first two ranges that start
+    inside a tile give the bands.  Other plans split every tile alike; the
+    bands are then one third and two thirds of the way along N."""
+    n_tiles = N // 128
+    if plan["variant"] == qgd.VARIANT_SWAP_AB and plan["schedule"] == qgd.SCHEDULE_PERSISTENT:
+        nkt = (K + 127) // 128
+        nku = (nkt + plan["k_slices"] - 1) // plan["k_slices"]
+        U = n_tiles * nku
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        G = min(U, sms * plan["occupancy"])
+        found = []
+        for c in range(1, G):
+            start = c * U // G
+            if start % nku and start // nku not in found and 0 < start // nku < n_tiles - 1:
+                found.append(start // nku)
+            if len(found) == 2:
+                return found
+        if found:
+            return found
+    return sorted({max(1, n_tiles // 3), max(1, (2 * n_tiles) // 3)} - {0, n_tiles - 1}) or [0]
+
+
 @pytest.mark.parametrize("wl,N,K,M", CASES, ids=[f"{wl.fmt}-{n}x{k}-M{m}" for wl, n, k, m in CASES])
 def test_decode_full_size_sampled(wl, N, K, M):
     w, wq, sw = _weights_for(wl, N, K)
@@ -102,13 +130,14 @@ def test_decode_full_size_sampled(wl, N, K, M):
     xq, sx = _quant_x(wl.fmt, x.cuda())
     y = bf16_to_f64(_gemm(wl.fmt, xq, sx, wq, sw))
     torch.cuda.synchronize()
-    bands = [0, N // 128 - 1]
+    plan = qgd.qgd_get_plan({FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}[wl.fmt], M, N, K)
+    bands = sorted(set([0, N // 128 - 1] + _interior_bands(plan, M, N, K)))
     rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in bands])
-    oxq, owq, y_ref, bound = _oracle_sample(wl.fmt, x, w[torch.from_numpy(rows)], (wl.fmt, N, K, "decode"))
+    oxq, owq, y_ref, bound = _oracle_sample(wl.fmt, x, w[torch.from_numpy(rows)],
+                                            (wl.fmt, N, K, "decode", tuple(bands)))
     np.testing.assert_array_equal(as_u8(xq), oxq.view(np.uint8))
     np.testing.assert_array_equal(as_u8(wq[torch.from_numpy(rows).cuda()]), owq.view(np.uint8))
-    plan = qgd.qgd_get_plan({FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}[wl.fmt], M, N, K)
-    _check(wl.fmt, y[:, rows], y_ref, bound, K, f"{wl.fmt} M={M} N={N} K={K} plan={plan}")
+    _check(wl.fmt, y[:, rows], y_ref, bound, K, f"{wl.fmt} M={M} N={N} K={K} bands={bands} plan={plan}")
 
 
 LARGE = [(wl, n, k, m) for wl in workloads.LARGE for (n, k) in wl.shapes[:2] for m in (64, 512, 2048)]
@@ -122,7 +151,7 @@ def test_large_m_full_size_sampled(wl, N, K, M):
     y = bf16_to_f64(_gemm(wl.fmt, xq, sx, wq, sw))
     torch.cuda.synchronize()
     toks = np.unique(np.concatenate([np.arange(0, M, max(1, M // 12)), [M - 1]]))
-    bands = [0, N // 128 - 1]
+    bands = [0, N // 256, N // 128 - 1]
     rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in bands])
     _, _, y_ref, bound = _oracle_sample(wl.fmt, x[torch.from_numpy(toks)], w[torch.from_numpy(rows)],
                                         (wl.fmt, N, K, "large"))

@@ -1,12 +1,14 @@
 """The FP8_Dynamic GEMM entry point that allocates nothing.
 
-Some callers cannot allocate device memory at the moment they run the layer:
-code whose stream is being captured into a CUDA graph, or a serving engine
-that carved all device memory into fixed pools at start-up.  For them
+Some callers cannot allocate device memory while they run the layer: a
+serving engine that carved all device memory into fixed pools at start-up
+has none left for a per-call workspace, and a latency-critical loop cannot
+afford a cudaMalloc that may wait for the device to go idle.  For them
 qlinear_fp8_dynamic_noalloc takes no workspace and uses a fixed scratch array
-built into the library.  These checks call it through the C ABI and hold its
-output to the regular entry point's (same plan, caller-provided workspace)
-with the FP8 tolerance the other GPU tests use, on two calls in a row.
+built into the library.  These checks call it through the C ABI, on two
+calls in a row, and hold its output both to the regular entry point's (same
+plan, caller-provided workspace) and to the oracle's, with the FP8 tolerance
+the other GPU tests use.
 
 This file is named to run last, so that a run stopping at the first failure
 has already run every other test; it sets and clears its own plan overrides,
@@ -49,13 +51,15 @@ def test_noalloc_matches_workspace_entry_point_twice(split, reduce):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, split, reduce, 0, 0, qgd.SCHEDULE_GRID)
     # the regular entry point, with a workspace the caller allocated
     ws = qgd.Workspace(qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, case.M, case.N, case.K))
-    y_ref = bf16_to_f64(case.run(ws=ws))
-    _, bound = case.oracle_gemm(*case.oracle_quant())
+    y_ws = bf16_to_f64(case.run(ws=ws))
+    yref, bound = case.oracle_gemm(*case.oracle_quant())
     for call in range(2):
         y = torch.full((case.M, case.N), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _noalloc(case, y) == 0, qgd.lib().qgd_last_error_message()
         torch.cuda.synchronize()
-        check_fp8_tolerance(bf16_to_f64(y), y_ref, bound, case.K, f"no-alloc call {call}")
+        got = bf16_to_f64(y)
+        check_fp8_tolerance(got, yref, bound, case.K, f"no-alloc call {call} vs the oracle")
+        check_fp8_tolerance(got, y_ws, bound, case.K, f"no-alloc call {call} vs the workspace entry point")
     assert qgd.qgd_device_error() == 0
 
 
