@@ -470,6 +470,83 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict |
     return rows
 
 
+def splitk_modes_table(device, ms=(1, 8, 32), reps: int = 10) -> list:
+    """The Split-K reductions side by side: for each FP8_Dynamic decode shape
+    and token count, the GEMM alone (a graph of calls over >= 3x L2 of weight
+    copies) at one split -- the shipped plan's if it splits, else 8 -- under
+    each reduction: atomic (zeroed accumulator + atomic adds, the pages'
+    scheme with fp32 partials), last arriving CTA, a second kernel, and the
+    thread-block cluster.  Same tile, ring and K slices for all four."""
+    import quantized_gemm_decode_b200 as qgd
+    from quantized_gemm_decode_b200.tune import Problem
+
+    names = {qgd.REDUCE_ATOMIC: "atomic", qgd.REDUCE_LAST_CTA: "last_cta", qgd.REDUCE_TWO_PASS: "two_pass",
+             qgd.REDUCE_CLUSTER: "cluster"}
+    rows = []
+    for (N, K) in workloads.FP8_DECODE.shapes:
+        for M in ms:
+            p = Problem(FP8_DYNAMIC, M, N, K, 1001, device)
+            base = qgd.qgd_get_plan(0, M, N, K)
+            split = base["split_k"] if (base["variant"] == 1 and base["schedule"] == 0 and base["split_k"] > 1) else 8
+            row = {"M": M, "N": N, "K": K, "split_k": split}
+            for red, name in names.items():
+                qgd.qgd_set_override(0, qgd.VARIANT_SWAP_AB, split, red, 2, 0, qgd.SCHEDULE_GRID, 1, 2)
+                pl = qgd.qgd_get_plan(0, M, N, K)
+                if pl["reduce"] != red:
+                    row[name] = None
+                    continue
+                row[name] = round(p.time_plan(reps=reps, with_quant=False), 2)
+            qgd.qgd_set_override(0)
+            rows.append(row)
+            del p
+            torch.cuda.empty_cache()
+    return rows
+
+
+def chain_table(device, reps: int = 20) -> list:
+    """The dependent decode-layer chain of one 8B-class layer (qkv -> o ->
+    gate_up -> down, FP8_Dynamic, each layer quantizing a column slice of an
+    earlier layer's output): one graph per token count, two weight copies
+    replayed alternately so every chain streams its 193 MB of weights from
+    HBM.  Microseconds per chain and the whole path's GB/s."""
+    from quantized_gemm_decode_b200.linear import LAYER_8B, DecodeChain, QuantizedLinear
+
+    shapes = workloads.SHAPES_8B
+    chains = []
+    for c in range(2):
+        layers = []
+        for i, (N, K) in enumerate(shapes):
+            w = synth.weights(N, K, 2001 + 10 * i + c).to(device)
+            layers.append(QuantizedLinear(w, FP8_DYNAMIC))
+            del w
+        chains.append(DecodeChain(layers, LAYER_8B))
+    rows = []
+    for M in workloads.DECODE_M:
+        x = synth.activations(M, shapes[0][1], 2001, outliers=True).to(device)
+        for ch in chains:
+            ch.input_buffer(M).copy_(x)
+            ch.capture(M)
+        for _ in range(3):
+            for ch in chains:
+                ch.run(M)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(reps):
+            for ch in chains:
+                ch.run(M)
+        t1.record()
+        torch.cuda.synchronize()
+        us = t0.elapsed_time(t1) * 1e3 / (2 * reps)
+        b = sum(path_bytes(FP8_DYNAMIC, M, N, K) for (N, K) in shapes)
+        rows.append({"M": M, "us_per_chain": round(us, 2), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                     "bytes_per_chain": b})
+    del chains
+    torch.cuda.empty_cache()
+    return rows
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
@@ -865,6 +942,8 @@ def main():
         probe = tensor_probe()
         out["tensor_probe"] = probe
         out["large_m"] = {f: large_m_summary(f, device, pk, probe=probe) for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)}
+        out["splitk_modes"] = splitk_modes_table(device)
+        out["chain"] = chain_table(device)
         out.update(extra)
         ds = keep
     if dist.rank == 0 and dist.world == 1 and not args.quick and not args.no_cpu_baseline:

@@ -129,6 +129,16 @@ QGD_API qgd_status quant_act_per_token(const void* x_bf16, int M, int K, int qty
  * sx [M][K/128] fp32 row-major.  Requires K % 128 == 0. */
 QGD_API qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float* sx, void* stream);
 
+/* The same two quantizers reading x rows `ldx` elements apart (ldx >= K,
+ * ldx % 8 == 0; the row starts stay 16-byte aligned), e.g. the first K
+ * columns of a wider activation such as a fused projection's output.  xq
+ * and sx are dense as above.  ldx < K or not a multiple of 8 ->
+ * QGD_ERR_INVALID. */
+QGD_API qgd_status quant_act_per_token_strided(const void* x_bf16, int M, int K, int ldx, int qtype, void* xq,
+                                               float* sx, void* stream);
+QGD_API qgd_status quant_act_group128_strided(const void* x_bf16, int M, int K, int ldx, void* xq, float* sx,
+                                              void* stream);
+
 /* 128x128 weight blocks (Block_FP8).  w_bf16 [N,K] -> wq e4m3 [N,K],
  * sw [N/128][K/128] fp32 row-major.  Requires N % 128 == 0, K % 128 == 0. */
 QGD_API qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream);

@@ -27,6 +27,7 @@ __all__ = [
     "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC", "REDUCE_CLUSTER",
     "SCHEDULE_GRID", "SCHEDULE_PERSISTENT",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
+    "quant_act_per_token_strided", "quant_act_group128_strided",
     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         sigs = {
             "quant_act_per_token": [P, I, I, I, P, P, P],
             "quant_act_group128": [P, I, I, P, P, P],
+            "quant_act_per_token_strided": [P, I, I, I, I, P, P, P],
+            "quant_act_group128_strided": [P, I, I, I, P, P, P],
             "quant_weight_block128": [P, I, I, P, P, P],
             "qlinear_fp8_dynamic": [P, P, P, P, P, I, I, I, P, S, P],
             "qlinear_w8a8_int8": [P, P, P, P, P, I, I, I, P, S, P],
@@ -151,17 +154,40 @@ _BYTE_TYPES = (torch.uint8, torch.int8, torch.float8_e4m3fn)
 # ---------------------------------------------------------------------------
 # Quantizers
 # ---------------------------------------------------------------------------
+def _activation_rows(x: torch.Tensor) -> int:
+    """Row stride (elements) of a bf16 activation: dense rows, or a view of
+    the first K columns of a wider matrix (unit column stride)."""
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    if x.stride(1) != 1 or (x.shape[0] > 1 and x.stride(0) < x.shape[1]):
+        raise ValueError("x rows must be contiguous (unit column stride, row stride >= K)")
+    return x.stride(0) if x.shape[0] > 1 else x.shape[1]
+
+
 def quant_act_per_token(x: torch.Tensor, qtype: int = QTYPE_E4M3, xq=None, sx=None, stream=None):
-    """Per-row dynamic quantization: x bf16 [M, K] -> (xq [M, K], sx fp32 [M])."""
-    _cuda_2d(x, "x", (torch.bfloat16,))
+    """Per-row dynamic quantization: x bf16 [M, K] -> (xq [M, K], sx fp32 [M]).
+    x may be a column slice of a wider matrix (rows any stride apart)."""
+    ldx = _activation_rows(x)
     M, K = x.shape
     if xq is None:
         xq = torch.empty((M, K), dtype=torch.float8_e4m3fn if qtype == QTYPE_E4M3 else torch.int8, device=x.device)
     if sx is None:
         sx = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _check(lib().quant_act_per_token(_ptr(x), M, K, qtype, _ptr(xq), _ptr(sx), _stream(stream)),
+    _check(lib().quant_act_per_token_strided(_ptr(x), M, K, ldx, qtype, _ptr(xq), _ptr(sx), _stream(stream)),
            "quant_act_per_token")
     return xq, sx
+
+
+def quant_act_per_token_strided(x: torch.Tensor, qtype: int = QTYPE_E4M3, xq=None, sx=None, stream=None):
+    """Alias of quant_act_per_token, which already takes column slices."""
+    return quant_act_per_token(x, qtype, xq=xq, sx=sx, stream=stream)
+
+
+def quant_act_group128_strided(x: torch.Tensor, xq=None, sx=None, stream=None):
+    """Alias of quant_act_group128, which already takes column slices."""
+    return quant_act_group128(x, xq=xq, sx=sx, stream=stream)
 
 
 def quant_weight_per_channel(w: torch.Tensor, qtype: int = QTYPE_E4M3, stream=None):
@@ -170,14 +196,16 @@ def quant_weight_per_channel(w: torch.Tensor, qtype: int = QTYPE_E4M3, stream=No
 
 
 def quant_act_group128(x: torch.Tensor, xq=None, sx=None, stream=None):
-    """1x128 group quantization: x bf16 [M, K] -> (xq e4m3 [M, K], sx fp32 [M, K/128])."""
-    _cuda_2d(x, "x", (torch.bfloat16,))
+    """1x128 group quantization: x bf16 [M, K] -> (xq e4m3 [M, K], sx fp32 [M, K/128]).
+    x may be a column slice of a wider matrix (rows any stride apart)."""
+    ldx = _activation_rows(x)
     M, K = x.shape
     if xq is None:
         xq = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
     if sx is None:
         sx = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
-    _check(lib().quant_act_group128(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "quant_act_group128")
+    _check(lib().quant_act_group128_strided(_ptr(x), M, K, ldx, _ptr(xq), _ptr(sx), _stream(stream)),
+           "quant_act_group128")
     return xq, sx
 
 

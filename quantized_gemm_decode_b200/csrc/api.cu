@@ -472,33 +472,45 @@ qgd_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-qgd_status quant_act_per_token(const void* x_bf16, int M, int K, int qtype, void* xq, float* sx, void* stream) {
+qgd_status quant_act_per_token_strided(const void* x_bf16, int M, int K, int ldx, int qtype, void* xq, float* sx,
+                                       void* stream) {
   if (M < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d K=%d)", M, K);
   if (qtype != QGD_QTYPE_E4M3 && qtype != QGD_QTYPE_INT8) return fail(QGD_ERR_INVALID, "bad qtype %d", qtype);
   if (K % 8 != 0 || K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 8 and <= 65536", K);
+  if (ldx < K || ldx % 8 != 0) return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
   if (M == 0) return QGD_OK;
   if (!x_bf16 || !xq || !sx) return fail(QGD_ERR_INVALID, "null pointer");
   if (!aligned16(x_bf16) || !aligned16(xq) || (reinterpret_cast<uintptr_t>(sx) & 3u))
     return fail(QGD_ERR_INVALID, "x and xq must be 16-byte aligned, sx 4-byte aligned");
   qgd_status st = check_device();
   if (st != QGD_OK) return st;
-  cudaError_t e = launch_quant_rows(static_cast<const uint16_t*>(x_bf16), M, K, qtype, xq, sx,
+  cudaError_t e = launch_quant_rows(static_cast<const uint16_t*>(x_bf16), M, K, ldx, qtype, xq, sx,
                                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_per_token launch");
 }
 
-qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float* sx, void* stream) {
+qgd_status quant_act_per_token(const void* x_bf16, int M, int K, int qtype, void* xq, float* sx, void* stream) {
+  return quant_act_per_token_strided(x_bf16, M, K, K, qtype, xq, sx, stream);
+}
+
+qgd_status quant_act_group128_strided(const void* x_bf16, int M, int K, int ldx, void* xq, float* sx,
+                                      void* stream) {
   if (M < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d K=%d)", M, K);
   if (K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 128", K);
+  if (ldx < K || ldx % 8 != 0) return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
   if (M == 0) return QGD_OK;
   if (!x_bf16 || !xq || !sx) return fail(QGD_ERR_INVALID, "null pointer");
   if (!aligned16(x_bf16) || !aligned16(xq) || (reinterpret_cast<uintptr_t>(sx) & 3u))
     return fail(QGD_ERR_INVALID, "x and xq must be 16-byte aligned, sx 4-byte aligned");
   qgd_status st = check_device();
   if (st != QGD_OK) return st;
-  cudaError_t e = launch_quant_group128(static_cast<const uint16_t*>(x_bf16), M, K, static_cast<uint8_t*>(xq), sx,
-                                        static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_quant_group128(static_cast<const uint16_t*>(x_bf16), M, K, ldx, static_cast<uint8_t*>(xq),
+                                        sx, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_group128 launch");
+}
+
+qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float* sx, void* stream) {
+  return quant_act_group128_strided(x_bf16, M, K, K, xq, sx, stream);
 }
 
 qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream) {

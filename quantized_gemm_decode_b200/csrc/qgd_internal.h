@@ -69,9 +69,11 @@ cudaError_t read_probe_error(unsigned int* code);
 cudaError_t clear_probe_error();
 
 // Quantizer launchers (quant.cu).
-cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, void* q, float* s,
+// x rows are ldx elements apart (ldx >= K); q and s are dense.
+cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int ldx, int qtype, void* q, float* s,
                               cudaStream_t stream);
-cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, uint8_t* q, float* s, cudaStream_t stream);
+cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, int ldx, uint8_t* q, float* s,
+                                  cudaStream_t stream);
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream);
 
 }  // namespace qgd

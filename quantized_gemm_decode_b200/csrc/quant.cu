@@ -94,13 +94,13 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 constexpr int kRowThreads = 512;
 
 template <int kVPT, int kQType>
-__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int K,
+__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t* __restrict__ x, int K, int ldx,
                                                                  uint8_t* __restrict__ q, float* __restrict__ s) {
   __shared__ float red[33];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
   const size_t row = blockIdx.x;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + row * K);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * static_cast<size_t>(ldx));
   uint2* qr = reinterpret_cast<uint2*>(q + row * K);
   const int nvec = K / 8;
   uint4 v[kVPT];
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(const uint16_t*
 // ---------------------------------------------------------------------------
 // 1x128 groups: a half-warp per group, 8 values per lane.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __restrict__ x, int M, int K,
+__global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __restrict__ x, int M, int K, int ldx,
                                                              uint8_t* __restrict__ q, float* __restrict__ s) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
@@ -137,8 +137,9 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __r
   const long long gg = valid ? g : 0;
   const long long m = gg / KB, kb = gg % KB;
   const size_t off = static_cast<size_t>(m) * K + static_cast<size_t>(kb) * 128 + sub * 8;
+  const size_t xoff = static_cast<size_t>(m) * ldx + static_cast<size_t>(kb) * 128 + sub * 8;
   uint4 v = make_uint4(0, 0, 0, 0);
-  if (valid) v = __ldg(reinterpret_cast<const uint4*>(x + off));
+  if (valid) v = __ldg(reinterpret_cast<const uint4*>(x + xoff));
   float amax = absmax8(v);
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -200,30 +201,32 @@ cudaError_t launch_q(void (*kernel)(Params...), dim3 grid, dim3 block, cudaStrea
 }
 
 template <int kQType>
-cudaError_t launch_rows_q(const uint16_t* x, int rows, int K, void* q, float* s, cudaStream_t st) {
+cudaError_t launch_rows_q(const uint16_t* x, int rows, int K, int ldx, void* q, float* s, cudaStream_t st) {
   const int nvec = K / 8;
   const int vpt = (nvec + kRowThreads - 1) / kRowThreads;
   uint8_t* qb = static_cast<uint8_t*>(q);
   const dim3 grid(rows), block(kRowThreads);
-  if (vpt <= 1) return launch_q(quant_rows_kernel<1, kQType>, grid, block, st, x, K, qb, s);
-  if (vpt <= 2) return launch_q(quant_rows_kernel<2, kQType>, grid, block, st, x, K, qb, s);
-  if (vpt <= 4) return launch_q(quant_rows_kernel<4, kQType>, grid, block, st, x, K, qb, s);
-  if (vpt <= 8) return launch_q(quant_rows_kernel<8, kQType>, grid, block, st, x, K, qb, s);
-  if (vpt <= 16) return launch_q(quant_rows_kernel<16, kQType>, grid, block, st, x, K, qb, s);
+  if (vpt <= 1) return launch_q(quant_rows_kernel<1, kQType>, grid, block, st, x, K, ldx, qb, s);
+  if (vpt <= 2) return launch_q(quant_rows_kernel<2, kQType>, grid, block, st, x, K, ldx, qb, s);
+  if (vpt <= 4) return launch_q(quant_rows_kernel<4, kQType>, grid, block, st, x, K, ldx, qb, s);
+  if (vpt <= 8) return launch_q(quant_rows_kernel<8, kQType>, grid, block, st, x, K, ldx, qb, s);
+  if (vpt <= 16) return launch_q(quant_rows_kernel<16, kQType>, grid, block, st, x, K, ldx, qb, s);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int qtype, void* q, float* s,
+cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int ldx, int qtype, void* q, float* s,
                               cudaStream_t stream) {
-  return qtype == 0 ? launch_rows_q<0>(x, rows, K, q, s, stream) : launch_rows_q<1>(x, rows, K, q, s, stream);
+  return qtype == 0 ? launch_rows_q<0>(x, rows, K, ldx, q, s, stream)
+                    : launch_rows_q<1>(x, rows, K, ldx, q, s, stream);
 }
 
-cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, uint8_t* q, float* s, cudaStream_t stream) {
+cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, int ldx, uint8_t* q, float* s,
+                                  cudaStream_t stream) {
   const long long groups = static_cast<long long>(M) * (K / 128);
   const unsigned blocks = static_cast<unsigned>((groups + 15) / 16);
-  return launch_q(quant_group128_kernel, dim3(blocks), dim3(256), stream, x, M, K, q, s);
+  return launch_q(quant_group128_kernel, dim3(blocks), dim3(256), stream, x, M, K, ldx, q, s);
 }
 
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream) {

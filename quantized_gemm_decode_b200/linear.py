@@ -194,3 +194,107 @@ class DecodeStep:
 
     def replay(self):
         self.graph.replay()
+
+
+# The four projections of one dense decoder layer and where each one's input
+# comes from: (name, source, input columns).  source -1 is the chain input;
+# otherwise the input is the first `input columns` columns of that earlier
+# projection's output.  The o projection reads the first 4096 columns of
+# qkv's output and down the first 12288 of gate_up's: in the model, attention
+# and the gated activation sit there, and here a column slice of the right
+# width stands in for each (neither is part of the linear layer's path).
+LAYER_8B = (("qkv", -1, 4096), ("o", 0, 4096), ("gate_up", 1, 4096), ("down", 2, 12288))
+
+
+class DecodeChain:
+    """Dependent linear layers of one decode step, captured as one CUDA graph
+    per token count: each layer dynamically quantizes its input -- a column
+    slice of an earlier layer's bf16 output, read in place through the
+    quantizer's row stride -- and runs its GEMM, so every kernel waits for the
+    one before it (the conditions of a model's forward pass, unlike
+    independent calls).
+
+    `layers` is a list of QuantizedLinear in chain order; `wiring` a list of
+    (name, source, columns) as LAYER_8B.  capture(M) builds the graph for M
+    tokens; run(M, x) copies x into the chain input and replays it; outputs(M)
+    are the layers' bf16 outputs and quantized(M) their (xq, sx) inputs.
+    """
+
+    def __init__(self, layers, wiring=LAYER_8B):
+        if len(layers) != len(wiring):
+            raise ValueError("one wiring entry per layer")
+        self.layers = list(layers)
+        self.wiring = list(wiring)
+        self.device = self.layers[0].device
+        for i, (layer, (_, src, cols)) in enumerate(zip(self.layers, self.wiring)):
+            width = self.layers[0].K if src < 0 else self.layers[src].N
+            if src >= i or cols != layer.K or cols > width:
+                raise ValueError(f"layer {i}: input of {cols} columns from source {src} does not fit")
+        self._bufs: dict = {}
+        self._graphs: dict = {}
+
+    def _buffers(self, M: int):
+        if M not in self._bufs:
+            x = torch.zeros((M, self.layers[0].K), dtype=torch.bfloat16, device=self.device)
+            ys, qs = [], []
+            for layer in self.layers:
+                ys.append(torch.empty((M, layer.N), dtype=torch.bfloat16, device=self.device))
+                qdt = torch.int8 if layer.fmt == "w8a8_int8" else torch.float8_e4m3fn
+                qs.append((torch.empty((M, layer.K), dtype=qdt, device=self.device),
+                           torch.empty((M, layer.K // 128) if layer.fmt == "block_fp8" else (M,),
+                                       dtype=torch.float32, device=self.device)))
+                layer.ws.ensure(qgd.qgd_workspace_size(layer.fmt_id, M, layer.N, layer.K))
+            self._bufs[M] = (x, ys, qs)
+        return self._bufs[M]
+
+    def _input(self, M: int, i: int) -> torch.Tensor:
+        x, ys, _ = self._buffers(M)
+        _, src, cols = self.wiring[i]
+        return x if src < 0 else ys[src][:, :cols]
+
+    def _body(self, M: int):
+        _, ys, qs = self._buffers(M)
+        for i, layer in enumerate(self.layers):
+            xq, sx = qs[i]
+            layer.quantize(self._input(M, i), xq, sx)
+            layer.gemm(xq, sx, ys[i])
+
+    def capture(self, M: int) -> None:
+        self._buffers(M)
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self._body(M)  # warm-up outside capture
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self._body(M)
+        self._graphs[M] = g
+
+    def graph(self, M: int) -> torch.cuda.CUDAGraph:
+        if M not in self._graphs:
+            self.capture(M)
+        return self._graphs[M]
+
+    def run(self, M: int, x: torch.Tensor | None = None) -> torch.Tensor:
+        """Replay the chain for M tokens (after copying x into its input) and
+        return the last layer's output buffer."""
+        g = self.graph(M)
+        if x is not None:
+            self._bufs[M][0].copy_(x, non_blocking=True)
+        g.replay()
+        return self._bufs[M][1][-1]
+
+    def input_buffer(self, M: int) -> torch.Tensor:
+        return self._buffers(M)[0]
+
+    def outputs(self, M: int) -> list:
+        return self._buffers(M)[1]
+
+    def quantized(self, M: int) -> list:
+        return self._buffers(M)[2]
+
+    def inputs(self, M: int) -> list:
+        """The bf16 input each layer quantized (views into earlier outputs)."""
+        return [self._input(M, i) for i in range(len(self.layers))]

@@ -417,3 +417,14 @@ def test_binding_checks_gemm_operands_before_any_launch():
     # W8A8_INT8 codes are int8
     with pytest.raises(ValueError, match="xq has dtype"):
         qgd.qlinear_w8a8_int8(xq, sx, wq, sw, y=y)
+
+
+def test_strided_quantizer_rejects_bad_row_stride():
+    L = qgd.lib()
+    P = ctypes.c_void_p
+    # ldx below K, or not a multiple of 8: refused before any launch
+    assert L.quant_act_per_token_strided(P(16), 4, 512, 500, 0, P(16), P(16), None) == -1
+    assert L.quant_act_per_token_strided(P(16), 4, 512, 516, 0, P(16), P(16), None) == -1
+    assert L.quant_act_group128_strided(P(16), 4, 512, 256, P(16), P(16), None) == -1
+    # an empty call with a valid stride is fine
+    assert L.quant_act_per_token_strided(P(16), 0, 512, 1024, 0, P(16), P(16), None) == 0
