@@ -217,7 +217,8 @@ class DecodeSet:
                 sx = torch.empty((M, K // 128) if self.fmt == BLOCK_FP8 else (M,), dtype=torch.float32, device=device)
                 y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
                 self.calls.append(dict(M=M, N=N, K=K, mi=mi, x=xd, x_host=x, xq=xq, sx=sx, y=y))
-                ws_need = max(ws_need, qgd.qgd_workspace_size(self.fmt_id, M, N, K))
+                ws_need = max(ws_need, qgd.qgd_workspace_size(self.fmt_id, M, N, K),
+                              qgd.qgd_layer_workspace_size(self.fmt_id, M, N, K))
         self.ws = qgd.Workspace(ws_need, device)
         torch.cuda.synchronize(device)
 
@@ -238,11 +239,26 @@ class DecodeSet:
               BLOCK_FP8: qgd.qlinear_block_fp8}[self.fmt]
         fn(c["xq"], c["sx"], wq, sw, y=c["y"], ws=self.ws)
 
+    def layer(self, c, copy_idx=None, next_w=None):
+        """The layer call from bf16 activations (quantizer fused into the GEMM
+        where the layer plan says so), warming `next_w` in L2."""
+        copies = self.weights[(c["N"], c["K"])]
+        wq, sw = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
+        self.qgd.qlinear_bf16(self.fmt_id, c["x"], wq, sw, y=c["y"], ws=self.ws, next_w=next_w)
+
+    def weight_of(self, c, copy_idx=None):
+        copies = self.weights[(c["N"], c["K"])]
+        return copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)][0]
+
     def step(self, gemm_only=False):
-        for c in self.calls:
-            if not gemm_only:
-                self.quant(c)
-            self.gemm(c)
+        """One pass: every call in order, each warming the next call's weights
+        in L2 (the last one the first call's, which the next step runs first)."""
+        n = len(self.calls)
+        for i, c in enumerate(self.calls):
+            if gemm_only:
+                self.gemm(c)
+            else:
+                self.layer(c, next_w=self.weight_of(self.calls[(i + 1) % n]))
 
     def capture(self, fn) -> torch.cuda.CUDAGraph:
         s = torch.cuda.Stream(self.device)
@@ -258,11 +274,33 @@ class DecodeSet:
         return g
 
     def launches_per_step(self, gemm_only=False) -> int:
+        """Kernels of one step: per call the GEMM, a second reduction kernel
+        for two-pass Split-K, and (layer calls) the quantizer unless fused."""
         n = 0
         for c in self.calls:
-            p = self.qgd.qgd_get_plan(self.fmt_id, c["M"], c["N"], c["K"])
-            n += (0 if gemm_only else 1) + 1 + (1 if p["split_k"] > 1 and p["reduce"] == 1 else 0)
+            get = self.qgd.qgd_get_plan if gemm_only else self.qgd.qgd_get_layer_plan
+            p = get(self.fmt_id, c["M"], c["N"], c["K"])
+            n += (0 if gemm_only or p["fused"] else 1) + 1 + (1 if p["split_k"] > 1 and p["reduce"] == 1 else 0)
         return n
+
+    def gemm_kernels(self):
+        """The step's GEMM kernels alone: for each call the GEMM on the
+        quantized activations, or -- where the layer plan fuses the quantizer
+        -- the fused kernel on the bf16 activations (the same kernel the step
+        runs).  Returns the algorithmic bytes those launches must move."""
+        b = 0
+        n = len(self.calls)
+        for i, c in enumerate(self.calls):
+            if self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"]:
+                self.layer(c, next_w=self.weight_of(self.calls[(i + 1) % n]))
+                b += path_bytes(self.fmt, c["M"], c["N"], c["K"])
+            else:
+                self.gemm(c)
+                b += workloads.algorithmic_bytes(self.fmt, c["M"], c["N"], c["K"])
+        return b
+
+    def fused_calls(self) -> int:
+        return sum(self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"] for c in self.calls)
 
     def bytes_per_step(self):
         gemm = sum(workloads.algorithmic_bytes(self.fmt, c["M"], c["N"], c["K"]) for c in self.calls)
@@ -318,8 +356,7 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
 
         def layer(c=c, ncop=ncop):
             for j in range(ncop):
-                ds.quant(c)
-                ds.gemm(c, copy_idx=j)
+                ds.layer(c, copy_idx=j, next_w=ds.weight_of(c, j + 1))
 
         g = ds.capture(body)
         times = replay_times(g, reps)
@@ -333,6 +370,7 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
         b = workloads.algorithmic_bytes(ds.fmt, c["M"], c["N"], c["K"])
         f = workloads.flops(c["M"], c["N"], c["K"])
         p = ds.qgd.qgd_get_plan(ds.fmt_id, c["M"], c["N"], c["K"])
+        fused = ds.qgd.qgd_get_layer_plan(ds.fmt_id, c["M"], c["N"], c["K"])["fused"]
         pb = path_bytes(ds.fmt, c["M"], c["N"], c["K"])
         rows.append({"M": c["M"], "N": c["N"], "K": c["K"], "us": round(ms * 1e3, 3), "median_us": round(med * 1e3, 3),
                      "p90_us": round(p90 * 1e3, 3),
@@ -342,7 +380,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
                      "layer_gbs": round(pb / (ms_layer * 1e-3) / 1e9, 1),
                      "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
                               f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
-                              f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}")})
+                              f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}"),
+                     "layer_fused": fused})
     return rows
 
 
@@ -661,8 +700,8 @@ def headline(out: dict) -> dict:
             "vs_baseline", "dtype", "data", "tflops", "frac_of_hbm_peak", "frac_of_8tbs", "gpu_launches")
     line = {k: out[k] for k in keep if k in out}
     cfg = out.get("config", {})
-    line["config"] = {k: cfg[k] for k in ("workload", "format", "shapes", "ms", "calls_per_step", "l2", "parallelism")
-                      if k in cfg}
+    line["config"] = {k: cfg[k] for k in ("workload", "format", "shapes", "ms", "calls_per_step", "fused_calls", "l2",
+                                          "parallelism") if k in cfg}
     rf = out.get("roofline")
     if rf:
         line["roofline"] = {k: rf[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source",
@@ -847,10 +886,12 @@ def main():
     clk = clocks.stop()
     value, ms_step = aggregate_throughput(path_b, ms_step_local, dist)
 
-    # ---- the dominant kernel (GEMM alone), same calls --------------------
-    g_gemm = ds.capture(lambda: ds.step(gemm_only=True))
+    # ---- the dominant kernel (the GEMM, fused or not), same calls ---------
+    kern_b = [0]
+    g_gemm = ds.capture(lambda: kern_b.__setitem__(0, ds.gemm_kernels()))
     ms_gemm = dist.max(time_graph(g_gemm, max(args.steps, 50), args.warmup, dist))
     del g_gemm
+    gemm_b = kern_b[0]
 
     # ---- e2e: the public layer API with pinned host buffers ---------------
     # every step copies its activations in from pinned host memory and its
@@ -897,7 +938,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
         "config": {"workload": wl.name, "format": wl.fmt, "shapes": [list(s) for s in wl.shapes], "ms": list(wl.ms),
-                   "calls_per_step": len(ds.calls), "graph": "one CUDA graph per step (quantize + GEMM per call)",
+                   "calls_per_step": len(ds.calls), "fused_calls": ds.fused_calls(),
+                   "graph": "one CUDA graph per step (one layer call per (M, N, K): quantize + GEMM, "
+                            "fused into one kernel where the tuned plan says so)",
                    "l2": f"inputs larger than L2: each call reads its own weight copy; "
                          f"{sum(len(v) for v in ds.weights.values())} copies, "
                          f"{path_b * 1e-9:.3f} GB streamed per step vs 126 MB L2",
@@ -905,7 +948,9 @@ def main():
         "tflops": round(flops * world / (ms_step * 1e-3) / 1e12, 3),
         "frac_of_hbm_peak": round(value / world / pk["hbm_gbs"], 4),
         "frac_of_8tbs": round(value / world / 8000.0, 4),
-        "roofline": {"bound": "hbm", "kernel": "GEMM (swapab/standard, all calls of the sweep)",
+        "roofline": {"bound": "hbm",
+                     "kernel": f"GEMM (swapab/standard, all calls of the sweep; {ds.fused_calls()} of {len(ds.calls)} "
+                               f"with the activation quantizer fused in, counted with bf16 activations in)",
                      "achieved": round(gemm_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gemm_gbs / pk["hbm_gbs"], 4), "peak_source": pk["source"],
                      # DRAM bytes per launch: the captured case's DRAM/algorithmic ratio

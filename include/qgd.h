@@ -105,6 +105,13 @@ typedef struct {
   int k_slices;  /* Swap-AB: 128-wide K slices per pipeline stage (1 or 2); Standard: 1.  Each stage
                     costs a fixed hand-off between the copy engine and the MMA, so one CTA per SM
                     keeps up with HBM only with two slices (32 KB of weights) per stage */
+  int fused;     /* layer calls (qlinear_*_bf16) only: 1 = the activation quantizer runs inside the
+                    Swap-AB GEMM kernel, 0 = a separate quantizer kernel first.  Always 0 in the plan
+                    of the qlinear_* calls, which take quantized activations */
+  int l2_ahead;  /* Swap-AB: how many weight units (a pipeline stage's worth of weight tiles) each
+                    CTA prefetches into L2 ahead of its shared-memory ring, 0..64 (0 = none; always 0
+                    for Standard).  The L2 holds what the ring cannot, so more of the weight stream
+                    is in flight than shared memory alone allows */
 } qgd_plan;
 
 /* ---------------------------------------------------------------------
@@ -167,6 +174,52 @@ QGD_API qgd_status qlinear_w8a8_int8(const void* xq, const float* sx, const void
 QGD_API qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void* wq, const float* sw, void* y_bf16,
                              int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------
+ * Layer calls from bf16 activations: dynamic activation quantization and
+ * the GEMM in one call ("Fused Quantization Ops" of the explore.n1n.ai
+ * page's architecture diagram; the formats as above).
+ *     y_bf16 [M,N] = qlinear_*(quantize(x_bf16 [M,K]), wq, sw)
+ * with exactly the codes and scales quant_act_per_token /
+ * quant_act_group128 would produce.  x rows are `ldx` elements apart (ldx
+ * >= K, ldx % 8 == 0; 16-byte aligned base), so x may be the first K
+ * columns of a wider activation.  The layer plan (qgd_get_layer_plan)
+ * decides how:
+ *   fused = 1  one Swap-AB kernel: its epilogue warps read x, quantize it
+ *              into the shared-memory stages the MMA consumes (per-token
+ *              scales: every CTA first takes each row's maximum over all of
+ *              K; Block_FP8: per 1x128 group inside the K slice).  No
+ *              activation codes reach global memory.
+ *   fused = 0  the quantizer kernel writes codes and scales into the
+ *              workspace, then the GEMM runs as qlinear_* would.
+ * Workspace: >= qgd_layer_workspace_size() bytes (same rules as for
+ * qlinear_*: zero-filled once after allocation; calls sharing it must not
+ * overlap), ws may be NULL when that size is 0.  Shapes as qlinear_*, and
+ * K <= 65536.  Errors as qlinear_*; ldx < K or not a multiple of 8 ->
+ * QGD_ERR_INVALID.
+ * next_w / next_bytes (optional; NULL / 0 for none): a device range -- for
+ *   example the next layer's weight codes -- that the Swap-AB GEMM warms in
+ *   L2: once a CTA has issued all of its own weight loads it prefetches its
+ *   share of the range, so HBM keeps streaming through this call's tail and
+ *   the next call's start instead of idling.  Only a hint: no result
+ *   depends on it; bytes beyond a multiple of 16 are ignored.  next_w must
+ *   be 16-byte aligned and the whole range readable device memory (else
+ *   QGD_ERR_INVALID for a misaligned pointer; an unreadable range is
+ *   undefined behaviour).  Standard plans ignore it.
+ * ------------------------------------------------------------------- */
+QGD_API qgd_status qlinear_fp8_dynamic_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
+                                            void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
+                                            const void* next_w, size_t next_bytes, void* stream);
+QGD_API qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
+                                          void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
+                                          const void* next_w, size_t next_bytes, void* stream);
+QGD_API qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
+                                          void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
+                                          const void* next_w, size_t next_bytes, void* stream);
+
+/* Bytes of workspace a layer call for (fmt, M, N, K) needs under the layer
+ * plan in force (0 when none). */
+QGD_API size_t qgd_layer_workspace_size(int fmt, int M, int N, int K);
+
 /* Test hook: the W8A8_INT8 mainloop and Split-K reduction of the plan in
  * force, writing the exact int32 accumulator acc[M][N] instead of Y. */
 QGD_API qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
@@ -215,6 +268,9 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
  * concurrent qlinear_* calls. */
 QGD_API qgd_status qgd_load_dispatch_table(const char* path);
 
+/* (Optional 13th and 14th fields: fused = 0 or 1, the layer plan's `fused`;
+ * l2_ahead = 0..64.) */
+
 /* Drop the table in force; the built-in defaults apply again. */
 QGD_API qgd_status qgd_clear_dispatch_table(void);
 
@@ -226,6 +282,19 @@ QGD_API qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduc
 
 /* The plan a qlinear_* call with these arguments would run. */
 QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);
+
+/* The plan a layer call (qlinear_*_bf16) with these arguments would run: the
+ * same table entry, with its `fused` field in effect. */
+QGD_API qgd_status qgd_get_layer_plan(int fmt, int M, int N, int K, qgd_plan* plan);
+
+/* Force the plan fields qgd_set_override does not cover, for one format
+ * (tests and the tuner); -1 keeps the table / default for that field.
+ *   fused     layer plans: 0 = quantizer kernel first, 1 = fused (Swap-AB
+ *             plans only; others stay unfused)
+ *   l2_ahead  Swap-AB L2 run-ahead in weight units, 0..64
+ * Independent of qgd_set_override; qgd_set_override_ext(fmt, -1, -1)
+ * removes it.  Out-of-range values -> QGD_ERR_INVALID. */
+QGD_API qgd_status qgd_set_override_ext(int fmt, int fused, int l2_ahead);
 
 /* M-bucket of a token count: the smallest tuned count >= M among
  * 1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192 (the last one beyond). */
@@ -267,6 +336,13 @@ QGD_API qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void*
  * No other kernel is affected.  Host-global, for tests only; not
  * thread-safe against concurrent qlinear_* calls.  Always QGD_OK. */
 QGD_API qgd_status qgd_test_withhold_accumulator(int on);
+
+/* Test hook for the fused layer calls (the pages have no counterpart):
+ * while xq (device, [M][K] bytes) and sx (device, [M] or [M][K/128] fp32)
+ * are non-null, every fused launch also writes the activation codes and
+ * scales it made there, so they can be compared with the oracle's; both
+ * NULL turns it off.  Host-global, for tests only.  Always QGD_OK. */
+QGD_API qgd_status qgd_test_capture_fused(void* xq, float* sx);
 
 /* Library version, "major.minor.patch". */
 QGD_API const char* qgd_version(void);

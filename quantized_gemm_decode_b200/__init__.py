@@ -33,6 +33,9 @@ __all__ = [
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
     "qgd_mma_peak_probe", "qgd_test_withhold_accumulator",
+    "qlinear_bf16", "qgd_layer_workspace_size", "qgd_get_layer_plan", "qgd_set_fused_override",
+    "qgd_set_override_ext",
+    "qgd_test_capture_fused",
     "Workspace", "DEFAULT_TABLE",
 ]
 
@@ -62,7 +65,8 @@ class QGDError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
                 ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("schedule", ctypes.c_int),
-                ("occupancy", ctypes.c_int), ("source", ctypes.c_int), ("k_slices", ctypes.c_int)]
+                ("occupancy", ctypes.c_int), ("source", ctypes.c_int), ("k_slices", ctypes.c_int),
+                ("fused", ctypes.c_int), ("l2_ahead", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -94,6 +98,12 @@ def lib() -> ctypes.CDLL:
             "qgd_clear_device_error": [],
             "qgd_mma_peak_probe": [I, I, ctypes.POINTER(ctypes.c_double), P],
             "qgd_test_withhold_accumulator": [I],
+            "qlinear_fp8_dynamic_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
+            "qlinear_w8a8_int8_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
+            "qlinear_block_fp8_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
+            "qgd_get_layer_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
+            "qgd_set_override_ext": [I, I, I],
+            "qgd_test_capture_fused": [P, P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -101,6 +111,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = ctypes.c_int
         L.qgd_workspace_size.argtypes = [I, I, I, I]
         L.qgd_workspace_size.restype = S
+        L.qgd_layer_workspace_size.argtypes = [I, I, I, I]
+        L.qgd_layer_workspace_size.restype = S
         L.qgd_m_bucket.argtypes = [I]
         L.qgd_m_bucket.restype = I
         L.qgd_status_string.argtypes = [I]
@@ -326,6 +338,54 @@ def qlinear_block_fp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
     return _qlinear("qlinear_block_fp8", FMT_BLOCK_FP8, xq, sx, wq, sw, y, ws, stream)
 
 
+_LAYER_FN = {FMT_FP8_DYNAMIC: "qlinear_fp8_dynamic_bf16", FMT_W8A8_INT8: "qlinear_w8a8_int8_bf16",
+             FMT_BLOCK_FP8: "qlinear_block_fp8_bf16"}
+
+
+def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None, next_w=None):
+    """Layer call from bf16 activations: dynamic quantization and the GEMM,
+    fused into one kernel when the layer plan says so (qgd_get_layer_plan).
+    x [M, K] bf16 may be a column slice of a wider matrix.  next_w (a CUDA
+    tensor, e.g. the next layer's weight codes) is warmed in L2 while this
+    call finishes; it changes no result."""
+    ldx = _activation_rows(x)
+    M, K = x.shape
+    want_w = (torch.int8,) if fmt == FMT_W8A8_INT8 else (torch.uint8, torch.float8_e4m3fn)
+    if not isinstance(wq, torch.Tensor) or wq.dim() != 2 or wq.shape[1] != K or wq.dtype not in want_w:
+        raise ValueError(f"wq must be a 2-D {want_w} tensor with K={K} columns")
+    N = wq.shape[0]
+    sw_n = (N // 128) * (K // 128) if fmt == FMT_BLOCK_FP8 else N
+    if not isinstance(sw, torch.Tensor) or sw.dtype != torch.float32 or sw.numel() < sw_n or not sw.is_contiguous():
+        raise ValueError(f"sw must be a contiguous float32 tensor of at least {sw_n} scales")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous bfloat16 tensor of shape {(M, N)}")
+    for t, name in ((wq, "wq"), (sw, "sw"), (y, "y")):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    need = qgd_layer_workspace_size(fmt, M, N, K)
+    if ws is None:
+        key = (x.device.index if x.device.index is not None else torch.cuda.current_device())
+        ws = _default_ws.get(key)
+        if ws is None:
+            ws = _default_ws[key] = Workspace(need, x.device)
+    if isinstance(ws, Workspace):
+        ws.ensure(need)
+        wsp, wsn = ws.buf.data_ptr(), ws.nbytes
+    else:
+        wsp, wsn = ws.data_ptr(), ws.numel() * ws.element_size()
+    nb = 0
+    if next_w is not None:
+        if not isinstance(next_w, torch.Tensor) or not next_w.is_cuda or not next_w.is_contiguous():
+            raise ValueError("next_w must be a contiguous CUDA tensor")
+        nb = next_w.numel() * next_w.element_size()
+    fn = _LAYER_FN[fmt]
+    _check(getattr(lib(), fn)(_ptr(x), ldx, _ptr(wq), _ptr(sw), _ptr(y), M, N, K, ctypes.c_void_p(wsp), wsn,
+                              _ptr(next_w), nb, _stream(stream)), fn)
+    return y
+
+
 def qlinear_fp8_dynamic_noalloc(xq, sx, wq, sw, y, stream=None):
     """FP8_Dynamic GEMM into a caller-provided y that allocates nothing: no
     workspace argument, no allocation by the binding or the library (the
@@ -380,6 +440,34 @@ def qgd_get_plan(fmt: int, M: int, N: int, K: int) -> dict:
     p = _Plan()
     _check(lib().qgd_get_plan(fmt, M, N, K, ctypes.byref(p)), "qgd_get_plan")
     return {f: getattr(p, f) for f, _ in _Plan._fields_}
+
+
+def qgd_layer_workspace_size(fmt: int, M: int, N: int, K: int) -> int:
+    return int(lib().qgd_layer_workspace_size(fmt, M, N, K))
+
+
+def qgd_get_layer_plan(fmt: int, M: int, N: int, K: int) -> dict:
+    p = _Plan()
+    _check(lib().qgd_get_layer_plan(fmt, M, N, K, ctypes.byref(p)), "qgd_get_layer_plan")
+    return {f: getattr(p, f) for f, _ in _Plan._fields_}
+
+
+def qgd_set_override_ext(fmt: int, fused: int = -1, l2_ahead: int = -1) -> None:
+    """Force the `fused` (layer plans) and `l2_ahead` plan fields for one
+    format; -1 keeps the table / default."""
+    _check(lib().qgd_set_override_ext(fmt, fused, l2_ahead), "qgd_set_override_ext")
+
+
+def qgd_set_fused_override(fmt: int, fused: int = -1) -> None:
+    """Force layer plans' `fused` field for one format (-1 = table /
+    default), leaving l2_ahead to the table."""
+    qgd_set_override_ext(fmt, fused, -1)
+
+
+def qgd_test_capture_fused(xq=None, sx=None) -> None:
+    """Test hook: fused launches also write their activation codes / scales
+    into these device tensors (None, None turns it off)."""
+    _check(lib().qgd_test_capture_fused(_ptr(xq), _ptr(sx)), "qgd_test_capture_fused")
 
 
 def qgd_m_bucket(M: int) -> int:

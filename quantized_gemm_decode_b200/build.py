@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqgd.so")
 SOURCES = ["api.cu", "gemm.cu", "quant.cu", "probe.cu"]
-HEADERS = ["qgd_internal.h", "sm100.cuh"]
+HEADERS = ["qgd_internal.h", "sm100.cuh", "quantcore.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -112,18 +112,21 @@ const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
 constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;   // decode token counts: Swap-AB by default
 constexpr int kSwapMaxM = 128;    // largest token count the Swap-AB kernel covers (FP8_Dynamic, W8A8_INT8)
+constexpr int kMaxL2Ahead = 64;   // most weight units a Swap-AB CTA prefetches into L2 ahead of its ring
 
 // Token columns of the Swap-AB MMA (its N): the next of 16, 32, 64, 128.
 int swap_mpad(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
 struct Entry {
-  int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices;
+  int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices, fused, l2_ahead;
 };
 using Key = std::tuple<int, int, int, int>;
 std::mutex g_mu;
 std::map<Key, Entry> g_table;
 struct Override {
   int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1, occupancy = 0, k_slices = 0;
+  int fused = -1;     // layer calls: -1 = table/default, 0/1 forced
+  int l2_ahead = -1;  // -1 = table/default, else forced
 } g_override[3];
 
 int bucket_of(int M) {
@@ -165,10 +168,14 @@ int reduce_from_name(const std::string& s) {
   return -1;
 }
 
-qgd_plan make_plan(int fmt, int M, int N, int K) {
+// layer: the plan of a layer call from bf16 activations (the qlinear_*_bf16
+// entry points), the only calls that can fuse the activation quantizer.
+qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   const int nkt = (K + kTileK - 1) / kTileK;
   qgd_plan p;
   p.source = 0;
+  p.fused = 0;
+  p.l2_ahead = 0;
   p.reduce = kLastCta;
   p.stages = 0;
   p.schedule = kGrid;
@@ -205,6 +212,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       p.schedule = e.schedule;
       p.occupancy = e.occupancy;
       p.k_slices = e.k_slices;
+      p.fused = e.fused;
+      p.l2_ahead = e.l2_ahead;
       p.source = 1;
     }
     const Override& o = g_override[fmt];
@@ -218,6 +227,14 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
       if (o.schedule >= 0) p.schedule = o.schedule;
       if (o.occupancy > 0) p.occupancy = o.occupancy;
       if (o.k_slices > 0) p.k_slices = o.k_slices;
+      p.source = 2;
+    }
+    if (o.fused >= 0) {
+      p.fused = o.fused;
+      p.source = 2;
+    }
+    if (o.l2_ahead >= 0) {
+      p.l2_ahead = o.l2_ahead;
       p.source = 2;
     }
   }
@@ -249,8 +266,16 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
                              : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
     if (tiles > kMaxTickets) p.reduce = kTwoPass;  // more tiles than arrival counters
   }
+  // the fused quantizer exists in the Swap-AB kernel only; its two-pass
+  // reduction would need the activation scales in memory, so it takes the
+  // last-arriving CTA instead
+  if (!layer || p.variant != kSwapAB) p.fused = 0;
+  if (p.variant != kSwapAB || p.l2_ahead < 0) p.l2_ahead = 0;
+  if (p.l2_ahead > kMaxL2Ahead) p.l2_ahead = kMaxL2Ahead;
+  p.fused = p.fused ? 1 : 0;
+  if (p.fused && p.reduce == kTwoPass) p.reduce = kLastCta;
   const int mpad = swap_mpad(M);
-  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster)
+  const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster, p.fused != 0)
                                           : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
@@ -258,7 +283,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K) {
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;
   if (p.schedule == kPersistent) {
-    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices, false)
+    const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices, false, p.fused != 0)
                                                : standard_smem_bytes(p.tile_n, p.stages)) + 1024;
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
@@ -356,22 +381,24 @@ qgd_status check_shape(int fmt, int M, int N, int K) {
   return QGD_OK;
 }
 
+std::atomic<void*> g_capture_xq{nullptr};    // qgd_test_capture_fused
+std::atomic<float*> g_capture_sx{nullptr};
+
+// One GEMM launch (plus its memset / second reduction kernel) for a plan.
+// xbf != null: the fused layer call -- the kernel quantizes the bf16
+// activations (rows ldxb elements apart) itself and xq/sx are unused.
 // follows_memset: the caller has just enqueued a memset on `stream`, so the
 // GEMM is launched without a programmatic dependency (that relaxation is
 // defined between two kernels only).
-qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, const float* sw, void* y, void* raw,
-                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream, bool follows_memset = false) {
-  qgd_status st = check_shape(fmt, M, N, K);
-  if (st != QGD_OK) return st;
-  if (M == 0) return QGD_OK;
-  if (!xq || !wq || (!y && !raw)) return fail(QGD_ERR_INVALID, "null operand pointer");
-  if (!raw && (!sx || !sw)) return fail(QGD_ERR_INVALID, "null scale pointer");
-  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(raw) || !aligned16(sx) || !aligned16(sw))
-    return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
+qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float* sx, const uint16_t* xbf, int ldxb,
+                         const void* wq, const float* sw, void* y, void* raw, int M, int N, int K, void* ws,
+                         size_t ws_bytes, void* stream, bool follows_memset, const void* pf = nullptr,
+                         size_t pf_bytes = 0) {
+  qgd_status st;
   if ((st = check_device()) != QGD_OK) return st;
   if ((st = get_encoder()) != QGD_OK) return st;
-
-  const qgd_plan p = make_plan(fmt, M, N, K);
+  const bool fused = xbf != nullptr;
+  if (fused && (!p.fused || p.variant != kSwapAB)) return fail(QGD_ERR_INVALID, "internal: fused launch without a fused plan");
   const Exec ex = make_exec(fmt, p, M, N, K);
   if (ex.total > 0 && (!ws || ws_bytes < ex.total))
     return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", ex.total, ws ? ws_bytes : 0);
@@ -405,9 +432,18 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   a.pdl = (pdl_enabled() && !follows_memset) ? 1 : 0;
   a.trace_tag = g_call_seq.fetch_add(1, std::memory_order_relaxed) & 0x7fffffff;
   a.withhold_acc = g_withhold_acc.load(std::memory_order_relaxed);
+  a.xbf = xbf;
+  a.ldxb = ldxb;
+  a.xq_out = fused ? static_cast<uint8_t*>(g_capture_xq.load()) : nullptr;
+  a.sx_out = fused ? g_capture_sx.load() : nullptr;
+  // (the Standard kernel does not warm L2; its calls are compute-bound)
+  a.l2_ahead = p.l2_ahead;
+  a.pf = static_cast<const uint8_t*>(pf);
+  a.pf_bytes = p.variant == kSwapAB ? pf_bytes : 0;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
+  memset(&tx, 0, sizeof tx);
   cudaError_t e;
   if (a.accum) {
     e = cudaMemsetAsync(a.accum, 0, static_cast<size_t>(M) * N * 4, s);
@@ -416,8 +452,8 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
   }
   if (p.variant == kSwapAB) {
     if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;
-    if ((st = encode_kmajor(&tx, xq, M, K, ex.mpad)) != QGD_OK) return st;
-    e = launch_swapab(fmt, ex.mpad, tw, tx, a, s);
+    if (!fused && (st = encode_kmajor(&tx, xq, M, K, ex.mpad)) != QGD_OK) return st;
+    e = launch_swapab(fmt, ex.mpad, fused, tw, tx, a, s);
   } else {
     if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
     if ((st = encode_kmajor(&tw, wq, N, K, p.tile_n)) != QGD_OK) return st;
@@ -430,6 +466,79 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
     if (e != cudaSuccess) return cuda_fail(e, "Split-K reduce launch");
   }
   return QGD_OK;
+}
+
+qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, const float* sw, void* y, void* raw,
+                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream, bool follows_memset = false) {
+  qgd_status st = check_shape(fmt, M, N, K);
+  if (st != QGD_OK) return st;
+  if (M == 0) return QGD_OK;
+  if (!xq || !wq || (!y && !raw)) return fail(QGD_ERR_INVALID, "null operand pointer");
+  if (!raw && (!sx || !sw)) return fail(QGD_ERR_INVALID, "null scale pointer");
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(raw) || !aligned16(sx) || !aligned16(sw))
+    return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
+  return run_gemm_plan(fmt, make_plan(fmt, M, N, K), xq, sx, nullptr, 0, wq, sw, y, raw, M, N, K, ws, ws_bytes,
+                       stream, follows_memset);
+}
+
+// Workspace of a layer call from bf16 activations: the GEMM's own part first
+// (its counter header must lead), then -- unless the plan fuses the
+// quantizer -- the activation codes and their scales.  The codes never go
+// into the counter header, even when this call's GEMM needs no workspace:
+// a workspace serves calls of every shape and plan, and the header must stay
+// zero between them.
+struct LayerWs {
+  qgd_plan plan;
+  Exec ex;
+  size_t xq_off = 0, sx_off = 0, total = 0;
+};
+
+LayerWs layer_ws(int fmt, int M, int N, int K) {
+  LayerWs l;
+  l.plan = make_plan(fmt, M, N, K, true);
+  l.ex = make_exec(fmt, l.plan, M, N, K);
+  l.total = l.ex.total;
+  if (!l.plan.fused && M > 0) {
+    l.xq_off = align256(l.total > kTicketBytes ? l.total : kTicketBytes);
+    l.sx_off = align256(l.xq_off + static_cast<size_t>(M) * K);
+    const size_t nsx = fmt == kFmtBlock ? static_cast<size_t>(M) * (K / kTileK) : static_cast<size_t>(M);
+    l.total = align256(l.sx_off + nsx * 4);
+  }
+  return l;
+}
+
+qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const float* sw, void* y, int M, int N,
+                     int K, void* ws, size_t ws_bytes, const void* next_w, size_t next_bytes, void* stream) {
+  qgd_status st = check_shape(fmt, M, N, K);
+  if (st != QGD_OK) return st;
+  if (next_bytes && (!next_w || !aligned16(next_w)))
+    return fail(QGD_ERR_INVALID, "next_w must be a 16-byte aligned device pointer when next_bytes > 0");
+  if (ldx < K || ldx % 8 != 0)
+    return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
+  if (K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be <= 65536", K);
+  if (M == 0) return QGD_OK;
+  if (!x_bf16 || !wq || !sw || !y) return fail(QGD_ERR_INVALID, "null operand pointer");
+  if (!aligned16(x_bf16) || !aligned16(wq) || !aligned16(y) || !aligned16(sw))
+    return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
+  const LayerWs l = layer_ws(fmt, M, N, K);
+  if (l.total > 0 && (!ws || ws_bytes < l.total))
+    return fail(QGD_ERR_WORKSPACE, "layer workspace of %zu bytes needed, %zu given", l.total, ws ? ws_bytes : 0);
+  if (l.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
+  const uint16_t* xb = static_cast<const uint16_t*>(x_bf16);
+  if (l.plan.fused)
+    return run_gemm_plan(fmt, l.plan, nullptr, nullptr, xb, ldx, wq, sw, y, nullptr, M, N, K, ws, ws_bytes, stream,
+                         false, next_w, next_bytes);
+  if ((st = check_device()) != QGD_OK) return st;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  void* xq = wsb + l.xq_off;
+  float* sx = reinterpret_cast<float*>(wsb + l.sx_off);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fmt == kFmtBlock
+                      ? launch_quant_group128(xb, M, K, ldx, static_cast<uint8_t*>(xq), sx, s)
+                      : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
+  if (e != cudaSuccess) return cuda_fail(e, "activation quantizer launch");
+  return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false,
+                       next_w, next_bytes);
 }
 
 // ---------------------------------------------------------------------------
@@ -541,6 +650,54 @@ qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void* wq, co
   return run_gemm(kFmtBlock, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream);
 }
 
+qgd_status qlinear_fp8_dynamic_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
+                                    int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
+                                    size_t next_bytes, void* stream) {
+  return run_layer(kFmtFP8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+}
+
+qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
+                                  int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
+                                  size_t next_bytes, void* stream) {
+  return run_layer(kFmtINT8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+}
+
+qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
+                                  int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
+                                  size_t next_bytes, void* stream) {
+  return run_layer(kFmtBlock, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+}
+
+size_t qgd_layer_workspace_size(int fmt, int M, int N, int K) {
+  if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
+  return layer_ws(fmt, M, N, K).total;
+}
+
+qgd_status qgd_get_layer_plan(int fmt, int M, int N, int K, qgd_plan* plan) {
+  if (!plan) return fail(QGD_ERR_INVALID, "null plan");
+  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "bad sizes");
+  *plan = make_plan(fmt, M < 1 ? 1 : M, N, K, true);
+  return QGD_OK;
+}
+
+qgd_status qgd_set_override_ext(int fmt, int fused, int l2_ahead) {
+  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (fused < -1 || fused > 1) return fail(QGD_ERR_INVALID, "fused must be -1, 0 or 1");
+  if (l2_ahead < -1 || l2_ahead > kMaxL2Ahead)
+    return fail(QGD_ERR_INVALID, "l2_ahead must be -1 or 0..%d", kMaxL2Ahead);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_override[fmt].fused = fused;
+  g_override[fmt].l2_ahead = l2_ahead;
+  return QGD_OK;
+}
+
+qgd_status qgd_test_capture_fused(void* xq, float* sx) {
+  g_capture_xq.store(xq);
+  g_capture_sx.store(sx);
+  return QGD_OK;
+}
+
 qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
                                size_t ws_bytes, void* stream) {
   if (M > 0 && !acc) return fail(QGD_ERR_INVALID, "null accumulator pointer");
@@ -595,16 +752,28 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (!(ls >> fmt_s)) continue;  // blank line
     if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s >> occ))
       return fail(QGD_ERR_TABLE,
-                  "%s:%d: expected 11 or 12 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
-                  "occupancy [k_slices]",
+                  "%s:%d: expected 11 to 14 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
+                  "occupancy [k_slices [fused [l2_ahead]]]",
                   path, lineno);
     std::string extra;
+    int fused = 0, l2a = 0;
     if (ls >> extra) {
       char* end = nullptr;
       const long v = strtol(extra.c_str(), &end, 10);
       if (*end != '\0' || v < 0 || v > 2) return fail(QGD_ERR_TABLE, "%s:%d: bad k_slices '%s'", path, lineno, extra.c_str());
       kslices = static_cast<int>(v);
-      if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
+      if (ls >> extra) {
+        const long f = strtol(extra.c_str(), &end, 10);
+        if (*end != '\0' || f < 0 || f > 1) return fail(QGD_ERR_TABLE, "%s:%d: bad fused '%s'", path, lineno, extra.c_str());
+        fused = static_cast<int>(f);
+        if (ls >> extra) {
+          const long a2 = strtol(extra.c_str(), &end, 10);
+          if (*end != '\0' || a2 < 0 || a2 > kMaxL2Ahead)
+            return fail(QGD_ERR_TABLE, "%s:%d: bad l2_ahead '%s'", path, lineno, extra.c_str());
+          l2a = static_cast<int>(a2);
+          if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
+        }
+      }
     }
     const int fmt = fmt_from_name(fmt_s), var = variant_from_name(var_s), red = reduce_from_name(red_s);
     const int sch = schedule_from_name(sch_s);
@@ -617,7 +786,7 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
         occ > 2)
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
-    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ, kslices};
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ, kslices, fused, l2a};
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_table.swap(t);

@@ -29,6 +29,7 @@
 #include <utility>
 
 #include "qgd_internal.h"
+#include "quantcore.cuh"
 #include "sm100.cuh"
 
 namespace qgd {
@@ -79,6 +80,7 @@ constexpr uint32_t kBarBytes = 1024;  // mbarriers, flags and staged token scale
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
+  uint64_t xfull[kMaxStages];  // fused Swap-AB: the stage's activation codes are written (one arrival per warp)
   uint64_t empty[kMaxStages];
   uint64_t tfull[4];
   uint64_t tempty[4];
@@ -92,6 +94,13 @@ struct SmemCtl {
   float sx_s[128];  // Swap-AB, per-token formats: the M token scales, staged once
 };
 static_assert(sizeof(SmemCtl) <= kBarBytes, "control block too large");
+
+// Fused Swap-AB: shared memory after the control block (and the cluster
+// receive buffer) for the per-row maxima of the per-token pre-pass (128 rows
+// x 4 warps) and a ring of Block_FP8 group scales, kScaleRing K slices deep
+// (the quantizer runs at most (stages + 1) x 2 slices ahead of the promotion).
+constexpr int kScaleRing = 36;
+constexpr uint32_t kFusedBytes = 128 * 4 * 4 + kScaleRing * 32 * 4;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -439,7 +448,16 @@ __device__ __forceinline__ void fixup_sum(const GemmArgs& a, int t, int row, int
 
 // Two CTAs per SM must always fit (the persistent grid size assumes it), so
 // the register budget is capped at 65536 / (2 * 192) per thread.
-template <int kFmt, int kMpad>
+//
+// kFused: the activation quantizer runs inside the kernel.  The epilogue
+// warps, idle while the weights stream, read the bf16 activations, quantize
+// them with the stand-alone quantizers' arithmetic (per token: every CTA
+// first takes each row's maximum over all of K; Block_FP8: one scale per
+// 1x128 group, inside the K slice) and write the codes into each stage's
+// activation tile in the layout the TMA would have written (128-byte rows,
+// 16-byte chunk c of row m at chunk c ^ (m % 8)), staying far enough ahead of
+// the MMA that neither waits on the other in a cycle (see quant_until).
+template <int kFmt, int kMpad, bool kFused>
 __global__ void __launch_bounds__(kGemmThreads, 2)
     swapab_kernel(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx,
                   const GemmArgs a) {
@@ -467,6 +485,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   uint8_t* x_ring = base + stages * stage_w;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * stage_x);
   uint8_t* recv_buf = reinterpret_cast<uint8_t*>(ctl) + kBarBytes;  // cluster Split-K: 128 x kMpad words
+  // fused: per-row maxima [128][4] and the Block_FP8 group-scale ring [kScaleRing][kMpad]
+  float* row_red = reinterpret_cast<float*>(recv_buf + (a.reduce == kCluster ? kSwapTileN * kMpad * 4 : 0));
+  float* scale_ring = row_red + 128 * 4;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkt = (a.K + kTileK - 1) / kTileK;
@@ -490,9 +511,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tw);
-    tma_prefetch_desc(&tx);
+    if (!kFused) tma_prefetch_desc(&tx);
     for (int i = 0; i < stages; ++i) {
       mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->xfull[i], 4);  // fused: one arrival per quantizing (epilogue) warp
       mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < kSlots; ++i) {
@@ -529,24 +551,39 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       const uint64_t pol_x = policy_evict_last();
       // Weights do not depend on the preceding kernel: start streaming them
       // before waiting for it, then fetch the activations.
+      // (fused: the stage's activation half is written by the epilogue warps)
+      const uint32_t x_tx = kFused ? 0u : kXBytes;
       const int pre = nk < stages ? nk : stages;
+      // L2 run-ahead: the weight tiles of units [pre, pre + l2_ahead) go to L2
+      // now and each later unit's as the ring advances, so more of the stream
+      // is in flight than the shared-memory ring can hold
+      auto prefetch_unit = [&](int i) {
+        const long long u = ub + i;
+        const int k0 = static_cast<int>(u % nku) * kps;
+        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+        for (int j = 0; j < ns; ++j) tma_prefetch_2d(&tw, (k0 + j) * kTileK, static_cast<int>(u / nku) * kSwapTileN);
+      };
+      const int ahead = a.l2_ahead;
       for (int i = 0; i < pre; ++i) {
         const long long u = ub + i;
         const int k0 = static_cast<int>(u % nku) * kps;   // first K slice of the unit
         const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
-        mbar_arrive_expect_tx(&ctl->full[i], ns * (kWBytes + kXBytes));
+        mbar_arrive_expect_tx(&ctl->full[i], ns * (kWBytes + x_tx));
         for (int j = 0; j < ns; ++j)
           tma_load_2d(w_ring + i * stage_w + j * kWBytes, &tw, &ctl->full[i], (k0 + j) * kTileK,
                       static_cast<int>(u / nku) * kSwapTileN, pol_w);
       }
+      for (int i = pre; i < nk && i < pre + ahead; ++i) prefetch_unit(i);
       QGD_STAMP(13);
-      griddep_wait();
-      QGD_STAMP(14);
-      for (int i = 0; i < pre; ++i) {
-        const int k0 = static_cast<int>((ub + i) % nku) * kps;
-        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
-        for (int j = 0; j < ns; ++j)
-          tma_load_2d(x_ring + i * stage_x + j * kXBytes, &tx, &ctl->full[i], (k0 + j) * kTileK, 0, pol_x);
+      if (!kFused) {
+        griddep_wait();
+        QGD_STAMP(14);
+        for (int i = 0; i < pre; ++i) {
+          const int k0 = static_cast<int>((ub + i) % nku) * kps;
+          const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+          for (int j = 0; j < ns; ++j)
+            tma_load_2d(x_ring + i * stage_x + j * kXBytes, &tx, &ctl->full[i], (k0 + j) * kTileK, 0, pol_x);
+        }
       }
       issued = pre;
       QGD_STAMP(2);
@@ -562,14 +599,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const long long u = ub + i;
         const int k0 = static_cast<int>(u % nku) * kps;
         const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
-        mbar_arrive_expect_tx(&ctl->full[s], ns * (kWBytes + kXBytes));
+        mbar_arrive_expect_tx(&ctl->full[s], ns * (kWBytes + x_tx));
         for (int j = 0; j < ns; ++j) {
           tma_load_2d(w_ring + s * stage_w + j * kWBytes, &tw, &ctl->full[s], (k0 + j) * kTileK,
                       static_cast<int>(u / nku) * kSwapTileN, pol_w);
-          tma_load_2d(x_ring + s * stage_x + j * kXBytes, &tx, &ctl->full[s], (k0 + j) * kTileK, 0, pol_x);
+          if (!kFused)
+            tma_load_2d(x_ring + s * stage_x + j * kXBytes, &tx, &ctl->full[s], (k0 + j) * kTileK, 0, pol_x);
         }
         issued = i + 1;
+        if (ahead > 0 && i + ahead < nk) prefetch_unit(i + ahead);
       }
+      // every load of this CTA is in flight: warm L2 with its share of the
+      // next layer's weights, so HBM keeps streaming through this layer's
+      // tail and the next layer's start
+      if (a.pf_bytes && issued == nk) prefetch_share_l2(a.pf, a.pf_bytes);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -581,7 +624,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       for (int i = 0; i < nk && !stop; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
-        if (!mbar_wait(&ctl->full[s], round & 1)) {
+        if (!mbar_wait(&ctl->full[s], round & 1) || (kFused && !mbar_wait(&ctl->xfull[s], round & 1))) {
           record_error(kErrWaitMma);
           ctl->abort_flag = 1;
           break;
@@ -644,9 +687,117 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int KB = a.K / kTileK;
     const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
     const bool scaled = (kFmt != kFmtBlock) && !a.raw;
-    if (scaled)
-      for (int m = static_cast<int>(threadIdx.x) - 64; m < M; m += kSwapTileN) ctl->sx_s[m] = __ldg(a.sx + m);
+    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 among the epilogue threads
+    if constexpr (kFused && !kBlock) {
+      // per-token scales: every CTA takes each row's maximum over all of K
+      // (four rows at a time, the loads of a row group in flight together)
+      const int nv8 = a.K / 8;
+      for (int m0 = 0; m0 < M; m0 += 4) {
+        float am[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int v = et; v < nv8; v += 128) {
+          uint4 r[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (m0 + k < M) r[k] = __ldg(reinterpret_cast<const uint4*>(a.xbf + static_cast<size_t>(m0 + k) * a.ldxb) + v);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (m0 + k < M) am[k] = fmaxf(am[k], absmax8(r[k]));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float w = warp_max(am[k]);
+          if (lane == 0 && m0 + k < M) row_red[(m0 + k) * 4 + q] = w;
+        }
+      }
+      epi_sync();
+      for (int m = et; m < M; m += 128) {
+        const float* rr = row_red + m * 4;
+        const float amax = fmaxf(fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3])), kAmaxFloor);
+        const float sc = __fdiv_rn(amax, kInt ? kInt8Max : kE4M3Max);
+        ctl->sx_s[m] = sc;
+        if (a.sx_out && ub == 0) a.sx_out[m] = sc;  // the CTA owning unit 0
+      }
+    } else if (scaled) {
+      for (int m = et; m < M; m += kSwapTileN) ctl->sx_s[m] = __ldg(a.sx + m);
+    }
     epi_sync();
+    // Fused: write the activation codes of stages [qnext, limit) into the
+    // ring.  Quantizing stage q needs the MMA to have released the ring slot,
+    // i.e. consumed stage q - stages; callers keep q - stages inside segments
+    // whose accumulator slot is already free (non-Block: the segment after
+    // the one being drained; Block_FP8: K slices at most 4 past the one being
+    // promoted), so the quantizer and the MMA never wait on each other in a
+    // cycle.  Each warp arrives on the stage's xfull barrier after its share;
+    // a warp whose wait gives up records the error and stops quantizing.
+    int qnext = 0, qslice = 0;
+    bool qdead = false;
+    auto quant_until = [&](int limit) {
+      if constexpr (kFused) {
+        if (limit > nk) limit = nk;
+        for (; qnext < limit && !qdead; ++qnext) {
+          const int s = qnext % stages;
+          const uint32_t round = qnext / stages;
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag) || !warp_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+            if (lane == 0) {
+              record_error(kErrWaitEpilogue);
+              ctl->abort_flag = 1;
+            }
+            qdead = true;
+            break;
+          }
+          const long long u = ub + qnext;
+          const int t = static_cast<int>(u / nku);
+          const int k0 = static_cast<int>(u % nku) * kps;
+          const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+          const int rows_w = round == 0 ? kMpad : M;  // the padding rows are zeroed once
+          for (int j = 0; j < ns; ++j, ++qslice) {
+            uint8_t* xs = x_ring + s * stage_x + j * kXBytes;
+            const int kk0 = (k0 + j) * kTileK;
+            for (int base = 0; base < rows_w * 8; base += 128) {
+              const int item = base + et;  // (row, 16-byte chunk); a row's 8 chunks are 8 adjacent lanes
+              const bool valid = item < rows_w * 8;
+              const int m = item >> 3, c = item & 7;
+              // past K (the last slice of a K that is not a multiple of 128;
+              // K % 16 == 0, so a chunk is all in or all out): zero codes, as
+              // the TMA's out-of-range fill gives the weights there
+              const bool live = valid && m < M && kk0 + c * 16 < a.K;
+              uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+              if (live) {
+                const uint4* src = reinterpret_cast<const uint4*>(a.xbf + static_cast<size_t>(m) * a.ldxb + kk0 + c * 16);
+                v0 = __ldg(src);
+                v1 = __ldg(src + 1);
+              }
+              float sc;
+              if constexpr (kBlock) {
+                float am = fmaxf(absmax8(v0), absmax8(v1));
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+                sc = __fdiv_rn(fmaxf(am, kAmaxFloor), kE4M3Max);
+                if (live && c == 0) {
+                  scale_ring[(qslice % kScaleRing) * kMpad + m] = sc;
+                  if (a.sx_out && t == 0) a.sx_out[static_cast<size_t>(m) * KB + k0 + j] = sc;
+                }
+              } else {
+                sc = live ? ctl->sx_s[m] : 1.f;
+              }
+              uint4 code = make_uint4(0, 0, 0, 0);
+              if (live) {
+                const uint2 lo = encode8<kInt ? 1 : 0>(v0, sc), hi = encode8<kInt ? 1 : 0>(v1, sc);
+                code = make_uint4(lo.x, lo.y, hi.x, hi.y);
+              }
+              if (valid) st_shared_v4(xs + m * 128 + ((c ^ (m & 7)) << 4), code);
+              if (live && a.xq_out && t == 0)
+                *reinterpret_cast<uint4*>(a.xq_out + static_cast<size_t>(m) * a.K + kk0 + c * 16) = code;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->xfull[s]);
+        }
+      }
+    };
     int i = 0, seg = 0;
     int sl = 0;  // Block_FP8: K slices consumed so far (same sequence as the MMA issuer's)
     while (i < nk) {
@@ -667,6 +818,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int kb_end = (kp_first + len) * kps < nkt ? (kp_first + len) * kps : nkt;
         for (int kb = kb_first; kb < kb_end; ++kb, ++sl) {
           const int slot = sl % kSlots;
+          const int kstage = i + kb / kps - kp_first;  // the stage holding this K slice
+          quant_until(kstage + stages);
           if (!warp_wait(&ctl->tfull[slot], (sl / kSlots) & 1)) {
             if (lane == 0) {
               record_error(kErrWaitEpilogue);
@@ -680,15 +833,33 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           tmem_wait_ld();
           warp_release(&ctl->tempty[slot]);
           const float swv = __ldg(a.sw + static_cast<size_t>(t) * KB + kb);  // one weight block per tile
+          if constexpr (kFused) {
+            // the slice's group scales, written by all four warps before their
+            // arrivals on the stage's xfull barrier (whose phase is still this
+            // one: the quantizer stays less than `stages` stages ahead)
+            if (!warp_wait(&ctl->xfull[kstage % stages], (kstage / stages) & 1)) {
+              if (lane == 0) {
+                record_error(kErrWaitEpilogue);
+                ctl->abort_flag = 1;
+              }
+              break;
+            }
+            const float* sxs = scale_ring + (sl % kScaleRing) * kMpad;
 #pragma unroll
-          for (int m = 0; m < kMpad; ++m) {
-            if (m < M)
-              facc[m] = fmaf(__uint_as_float(r[m]), __ldg(a.sx + static_cast<size_t>(m) * KB + kb) * swv, facc[m]);
+            for (int m = 0; m < kMpad; ++m)
+              if (m < M) facc[m] = fmaf(__uint_as_float(r[m]), sxs[m] * swv, facc[m]);
+          } else {
+#pragma unroll
+            for (int m = 0; m < kMpad; ++m) {
+              if (m < M)
+                facc[m] = fmaf(__uint_as_float(r[m]), __ldg(a.sx + static_cast<size_t>(m) * KB + kb) * swv, facc[m]);
+            }
           }
         }
 #pragma unroll
         for (int m = 0; m < kMpad; ++m) acc[m] = __float_as_uint(facc[m]);
       } else {
+        quant_until(i + len + nku);  // this segment and the next one
         if (!warp_wait(&ctl->tfull[slot_nb], (seg >> 1) & 1)) {
           if (lane == 0) {
             record_error(kErrWaitEpilogue);
@@ -1347,17 +1518,18 @@ cudaError_t set_smem_attr(Kern kernel, bool& done) {
 
 }  // namespace
 
-size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster) {
+size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused) {
   return 1024 + static_cast<size_t>(stages) * kps * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes +
-         (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0);
+         (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0) + (fused ? kFusedBytes : 0);
 }
 
 size_t standard_smem_bytes(int tile_n, int stages) {
   return 1024 + static_cast<size_t>(stages) * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
 }
 
-int swapab_max_stages(int mpad, int kps, bool cluster) {
-  const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0);
+int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
+  const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0) +
+                       (fused ? kFusedBytes : 0);
   int s = static_cast<int>((smem_budget() - fixed) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
@@ -1367,18 +1539,44 @@ int standard_max_stages(int tile_n) {
   return s > kMaxStages ? kMaxStages : s;
 }
 
-template <int kFmt, int kMpad>
+template <int kFmt, int kMpad, bool kFused>
 static cudaError_t launch_swapab_t(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                                    cudaStream_t stream) {
   static bool attr_done = false;
-  cudaError_t e = set_smem_attr(swapab_kernel<kFmt, kMpad>, attr_done);
+  cudaError_t e = set_smem_attr(swapab_kernel<kFmt, kMpad, kFused>, attr_done);
   if (e != cudaSuccess) return e;
   const dim3 grid = a.persistent ? dim3(a.ctas, 1, 1)
                                  : dim3((a.N + kSwapTileN - 1) / kSwapTileN, a.splits, 1);
   const bool cluster = a.reduce == kCluster;
-  return launch_ex_cluster(swapab_kernel<kFmt, kMpad>, grid, dim3(kGemmThreads),
-                           swapab_smem_bytes(kMpad, a.stages, a.kps, cluster), stream, a.pdl != 0,
+  return launch_ex_cluster(swapab_kernel<kFmt, kMpad, kFused>, grid, dim3(kGemmThreads),
+                           swapab_smem_bytes(kMpad, a.stages, a.kps, cluster, kFused), stream, a.pdl != 0,
                            cluster ? a.splits : 1, tw, tx, a);
+}
+
+template <bool kFused>
+static cudaError_t launch_swapab_f(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx,
+                                   const GemmArgs& a, cudaStream_t stream) {
+  if (fmt == kFmtFP8) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtFP8, 16, kFused>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtFP8, 32, kFused>(tw, tx, a, stream);
+      case 64: return launch_swapab_t<kFmtFP8, 64, kFused>(tw, tx, a, stream);
+      case 128: return launch_swapab_t<kFmtFP8, 128, kFused>(tw, tx, a, stream);
+    }
+  } else if (fmt == kFmtINT8) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtINT8, 16, kFused>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtINT8, 32, kFused>(tw, tx, a, stream);
+      case 64: return launch_swapab_t<kFmtINT8, 64, kFused>(tw, tx, a, stream);
+      case 128: return launch_swapab_t<kFmtINT8, 128, kFused>(tw, tx, a, stream);
+    }
+  } else if (fmt == kFmtBlock) {
+    switch (mpad) {
+      case 16: return launch_swapab_t<kFmtBlock, 16, kFused>(tw, tx, a, stream);
+      case 32: return launch_swapab_t<kFmtBlock, 32, kFused>(tw, tx, a, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int kFmt, int kTileN>
@@ -1394,29 +1592,10 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
                    stream, a.pdl != 0, tx, tw, a);
 }
 
-cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
-                          cudaStream_t stream) {
-  if (fmt == kFmtFP8) {
-    switch (mpad) {
-      case 16: return launch_swapab_t<kFmtFP8, 16>(tw, tx, a, stream);
-      case 32: return launch_swapab_t<kFmtFP8, 32>(tw, tx, a, stream);
-      case 64: return launch_swapab_t<kFmtFP8, 64>(tw, tx, a, stream);
-      case 128: return launch_swapab_t<kFmtFP8, 128>(tw, tx, a, stream);
-    }
-  } else if (fmt == kFmtINT8) {
-    switch (mpad) {
-      case 16: return launch_swapab_t<kFmtINT8, 16>(tw, tx, a, stream);
-      case 32: return launch_swapab_t<kFmtINT8, 32>(tw, tx, a, stream);
-      case 64: return launch_swapab_t<kFmtINT8, 64>(tw, tx, a, stream);
-      case 128: return launch_swapab_t<kFmtINT8, 128>(tw, tx, a, stream);
-    }
-  } else if (fmt == kFmtBlock) {
-    switch (mpad) {
-      case 16: return launch_swapab_t<kFmtBlock, 16>(tw, tx, a, stream);
-      case 32: return launch_swapab_t<kFmtBlock, 32>(tw, tx, a, stream);
-    }
-  }
-  return cudaErrorInvalidValue;
+cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,
+                          const GemmArgs& a, cudaStream_t stream) {
+  return fused ? launch_swapab_f<true>(fmt, mpad, tw, tx, a, stream)
+               : launch_swapab_f<false>(fmt, mpad, tw, tx, a, stream);
 }
 
 cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,

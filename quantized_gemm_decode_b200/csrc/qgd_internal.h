@@ -46,20 +46,32 @@ struct GemmArgs {
   int pdl;         // launch with a programmatic dependency on the preceding kernel
   int trace_tag;   // sequence number of the call (developer timeline builds file stamps by it)
   int withhold_acc;  // failure-detection test: Swap-AB never signals a finished accumulator
+  // Swap-AB with the activation quantizer fused in: the kernel reads bf16
+  // activations and writes their codes into its shared-memory stages itself.
+  const uint16_t* xbf;  // bf16 activations [M] rows, ldxb elements apart
+  int ldxb;
+  uint8_t* xq_out;      // test capture (may be null): the codes [M][K] the kernel made
+  float* sx_out;        // test capture (may be null): their scales, [M] or [M][K/128]
+  // L2 warm-up of the next layer's weights: once a CTA has issued all of its
+  // own loads it prefetches its share of [pf, pf + pf_bytes) into L2
+  const uint8_t* pf;
+  size_t pf_bytes;
+  int l2_ahead;  // Swap-AB: weight units prefetched into L2 ahead of the shared-memory ring
 };
 
 // Launchers (gemm.cu).  Each returns the cudaError_t of the launch.
-cudaError_t launch_swapab(int fmt, int mpad, const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
-                          cudaStream_t stream);
+// fused: the kernel quantizes a.xbf itself (tx unused)
+cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,
+                          const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();
-size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster);
+size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused);
 size_t standard_smem_bytes(int tile_n, int stages);
-int swapab_max_stages(int mpad, int kps, bool cluster);
+int swapab_max_stages(int mpad, int kps, bool cluster, bool fused);
 int standard_max_stages(int tile_n);
 
 // Tensor-core peak probe (probe.cu).

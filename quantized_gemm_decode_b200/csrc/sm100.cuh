@@ -159,6 +159,37 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Bring [p, p + bytes) into L2 (no shared memory, no completion to wait
+// for).  p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
+// This CTA's share of an L2 warm-up range: the range is cut into equal
+// 16-byte-aligned pieces, one per CTA of the grid, issued 64 KB at a time.
+__device__ __forceinline__ void prefetch_share_l2(const uint8_t* base, size_t bytes) {
+  const size_t ncta = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
+  const size_t cid = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  const size_t total = bytes & ~static_cast<size_t>(15);
+  const size_t share = ((total + ncta - 1) / ncta + 15) & ~static_cast<size_t>(15);
+  const size_t b0 = cid * share;
+  const size_t b1 = b0 + share < total ? b0 + share : total;
+  for (size_t b = b0; b < b1; b += 65536) {
+    const size_t n = b1 - b < 65536 ? b1 - b : 65536;
+    prefetch_l2_bulk(base + b, static_cast<uint32_t>(n));
+  }
+}
+
+// Bring one TMA box of a tensor into L2 only (no shared memory, nothing to
+// wait for); coordinates as tma_load_2d.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -280,6 +311,19 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Make this thread's generic-proxy writes to shared memory visible to the
+// async proxy (the tensor core reading an operand tile), before the mbarrier
+// arrival that hands the tile over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(void* p, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
 
 // Named barrier among `nthreads` threads (multiple of 32) of this CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {

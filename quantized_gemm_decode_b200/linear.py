@@ -37,7 +37,8 @@ class QuantizedLinear:
                 qt = qgd.QTYPE_INT8 if fmt == "w8a8_int8" else qgd.QTYPE_E4M3
                 wq, sw = qgd.quant_weight_per_channel(w, qt)
         self.wq, self.sw = wq, sw
-        need = max(qgd.qgd_workspace_size(self.fmt_id, m, self.N, self.K) for m in DECODE_BUCKETS)
+        need = max(max(qgd.qgd_workspace_size(self.fmt_id, m, self.N, self.K),
+                       qgd.qgd_layer_workspace_size(self.fmt_id, m, self.N, self.K)) for m in DECODE_BUCKETS)
         self.ws = qgd.Workspace(need, self.device)
         self._graphs: dict = {}
 
@@ -54,9 +55,17 @@ class QuantizedLinear:
         self.ws.ensure(qgd.qgd_workspace_size(self.fmt_id, xq.shape[0], self.N, self.K))
         return fn(xq, sx, self.wq, self.sw, y=y, ws=self.ws)
 
+    def layer(self, x: torch.Tensor, y=None, next_layer: "QuantizedLinear | None" = None) -> torch.Tensor:
+        """The whole layer call from bf16 x (possibly a column slice of a
+        wider matrix): quantization and GEMM, fused into one kernel when the
+        layer plan says so.  With `next_layer`, its weight codes are warmed
+        in L2 while this call finishes."""
+        self.ws.ensure(qgd.qgd_layer_workspace_size(self.fmt_id, x.shape[0], self.N, self.K))
+        return qgd.qlinear_bf16(self.fmt_id, x, self.wq, self.sw, y=y, ws=self.ws,
+                                next_w=None if next_layer is None else next_layer.wq)
+
     def forward_eager(self, x: torch.Tensor, y=None) -> torch.Tensor:
-        xq, sx = self.quantize(x)
-        return self.gemm(xq, sx, y=y)
+        return self.layer(x, y=y)
 
     # ---- graph path ---------------------------------------------------
     def capture(self, buckets=DECODE_BUCKETS) -> None:
@@ -68,17 +77,15 @@ class QuantizedLinear:
                              device=self.device)
             sx = torch.empty((mb, self.K // 128) if self.fmt == "block_fp8" else (mb,), dtype=torch.float32,
                              device=self.device)
-            self.ws.ensure(qgd.qgd_workspace_size(self.fmt_id, mb, self.N, self.K))
+            self.ws.ensure(qgd.qgd_layer_workspace_size(self.fmt_id, mb, self.N, self.K))
             s = torch.cuda.Stream(self.device)
             s.wait_stream(torch.cuda.current_stream(self.device))
             with torch.cuda.stream(s):
-                self.quantize(x, xq, sx)
-                self.gemm(xq, sx, y)
+                self.layer(x, y)
             torch.cuda.current_stream(self.device).wait_stream(s)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                self.quantize(x, xq, sx)
-                self.gemm(xq, sx, y)
+                self.layer(x, y)
             self._graphs[mb] = (g, x, y)
 
     def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
@@ -133,16 +140,11 @@ class DecodeStep:
         self.out_every = max(1, int(out_every))
         self.calls = list(calls)
         dev = self.calls[0][0].device
-        self.x_dev, self.y_dev, self.q = [], [], []
+        self.x_dev, self.y_dev = [], []
         for (layer, M) in self.calls:
             self.x_dev.append(torch.empty((M, layer.K), dtype=torch.bfloat16, device=dev))
             self.y_dev.append(torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev))
-            qdt = torch.int8 if layer.fmt == "w8a8_int8" else torch.float8_e4m3fn
-            xq = torch.empty((M, layer.K), dtype=qdt, device=dev)
-            sx = torch.empty((M, layer.K // 128) if layer.fmt == "block_fp8" else (M,), dtype=torch.float32,
-                             device=dev)
-            layer.ws.ensure(qgd.qgd_workspace_size(layer.fmt_id, M, layer.N, layer.K))
-            self.q.append((xq, sx))
+            layer.ws.ensure(qgd.qgd_layer_workspace_size(layer.fmt_id, M, layer.N, layer.K))
         self.x_host, self.y_host = list(x_host), list(y_host)
         self.graph = torch.cuda.CUDAGraph()
         main = torch.cuda.Stream(dev)
@@ -159,9 +161,7 @@ class DecodeStep:
         if copy_in is None:
             for i, (layer, M) in enumerate(self.calls):
                 self.x_dev[i].copy_(self.x_host[i], non_blocking=True)
-                xq, sx = self.q[i]
-                layer.quantize(self.x_dev[i], xq, sx)
-                layer.gemm(xq, sx, self.y_dev[i])
+                layer.layer(self.x_dev[i], self.y_dev[i])
                 self.y_host[i].copy_(self.y_dev[i], non_blocking=True)
             return
         landed = {}
@@ -178,9 +178,7 @@ class DecodeStep:
         for i, (layer, M) in enumerate(self.calls):
             if i % self.join_every == 0:
                 main.wait_event(landed[i // self.join_every])
-            xq, sx = self.q[i]
-            layer.quantize(self.x_dev[i], xq, sx)
-            layer.gemm(xq, sx, self.y_dev[i])
+            layer.layer(self.x_dev[i], self.y_dev[i], next_layer=self.calls[(i + 1) % n][0])
             # results leave in groups too: one fork from the compute stream per group
             if (i + 1) % self.out_every == 0 or i == n - 1:
                 done = torch.cuda.Event()
@@ -208,16 +206,16 @@ LAYER_8B = (("qkv", -1, 4096), ("o", 0, 4096), ("gate_up", 1, 4096), ("down", 2,
 
 class DecodeChain:
     """Dependent linear layers of one decode step, captured as one CUDA graph
-    per token count: each layer dynamically quantizes its input -- a column
-    slice of an earlier layer's bf16 output, read in place through the
-    quantizer's row stride -- and runs its GEMM, so every kernel waits for the
-    one before it (the conditions of a model's forward pass, unlike
-    independent calls).
+    per token count: each layer call quantizes its input -- a column slice of
+    an earlier layer's bf16 output, read in place through the row stride --
+    and runs its GEMM (one fused kernel when the layer plan says so), so every
+    kernel waits for the one before it (the conditions of a model's forward
+    pass, unlike independent calls).
 
     `layers` is a list of QuantizedLinear in chain order; `wiring` a list of
     (name, source, columns) as LAYER_8B.  capture(M) builds the graph for M
     tokens; run(M, x) copies x into the chain input and replays it; outputs(M)
-    are the layers' bf16 outputs and quantized(M) their (xq, sx) inputs.
+    are the layers' bf16 outputs and inputs(M) the bf16 inputs they read.
     """
 
     def __init__(self, layers, wiring=LAYER_8B):
@@ -232,32 +230,37 @@ class DecodeChain:
                 raise ValueError(f"layer {i}: input of {cols} columns from source {src} does not fit")
         self._bufs: dict = {}
         self._graphs: dict = {}
+        # each layer warms the next one's weights in L2; the last one warms
+        # the layer that runs after the chain (by default its own first)
+        self.successor: QuantizedLinear | None = self.layers[0]
+
+    def then(self, layer) -> None:
+        """The layer whose weights the chain's last layer warms in L2 (for
+        example the first layer of the next decoder block); None for none.
+        Takes effect at the next capture."""
+        self.successor = layer
+        self._graphs.clear()
 
     def _buffers(self, M: int):
         if M not in self._bufs:
             x = torch.zeros((M, self.layers[0].K), dtype=torch.bfloat16, device=self.device)
-            ys, qs = [], []
+            ys = []
             for layer in self.layers:
                 ys.append(torch.empty((M, layer.N), dtype=torch.bfloat16, device=self.device))
-                qdt = torch.int8 if layer.fmt == "w8a8_int8" else torch.float8_e4m3fn
-                qs.append((torch.empty((M, layer.K), dtype=qdt, device=self.device),
-                           torch.empty((M, layer.K // 128) if layer.fmt == "block_fp8" else (M,),
-                                       dtype=torch.float32, device=self.device)))
-                layer.ws.ensure(qgd.qgd_workspace_size(layer.fmt_id, M, layer.N, layer.K))
-            self._bufs[M] = (x, ys, qs)
+                layer.ws.ensure(qgd.qgd_layer_workspace_size(layer.fmt_id, M, layer.N, layer.K))
+            self._bufs[M] = (x, ys)
         return self._bufs[M]
 
     def _input(self, M: int, i: int) -> torch.Tensor:
-        x, ys, _ = self._buffers(M)
+        x, ys = self._buffers(M)
         _, src, cols = self.wiring[i]
         return x if src < 0 else ys[src][:, :cols]
 
     def _body(self, M: int):
-        _, ys, qs = self._buffers(M)
+        _, ys = self._buffers(M)
         for i, layer in enumerate(self.layers):
-            xq, sx = qs[i]
-            layer.quantize(self._input(M, i), xq, sx)
-            layer.gemm(xq, sx, ys[i])
+            nxt = self.layers[i + 1] if i + 1 < len(self.layers) else self.successor
+            layer.layer(self._input(M, i), ys[i], next_layer=nxt)
 
     def capture(self, M: int) -> None:
         self._buffers(M)
@@ -291,9 +294,6 @@ class DecodeChain:
 
     def outputs(self, M: int) -> list:
         return self._buffers(M)[1]
-
-    def quantized(self, M: int) -> list:
-        return self._buffers(M)[2]
 
     def inputs(self, M: int) -> list:
         """The bf16 input each layer quantized (views into earlier outputs)."""

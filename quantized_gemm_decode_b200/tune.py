@@ -65,28 +65,49 @@ def swap_mpad(M: int) -> int:
     return 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
 
 
-def two_per_sm_stages(M: int, kps: int, cluster: bool) -> int:
+FUSED_BYTES = 128 * 4 * 4 + 36 * 32 * 4  # the fused kernel's row maxima and group-scale ring
+
+
+def two_per_sm_stages(M: int, kps: int, cluster: bool, fused: bool = False) -> int:
     """Deepest Swap-AB ring (at least 2 stages) that still lets two CTAs share an SM; 0 (the
     deepest ring, one CTA per SM) when no such ring exists."""
     mpad = swap_mpad(M)
     per_stage = kps * (128 * 128 + mpad * 128)
-    fixed = 1024 + 1024 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
+    fixed = (1024 + 1024 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
+             + (FUSED_BYTES if fused else 0))
     st = min(16, (SMEM_PER_SM // 2 - fixed) // per_stage)
     return st if st >= 2 else 0
 
 
-def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
-    """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices, stages) tuples legal for the
-    shape; stages 0 = the deepest ring.  A Swap-AB grid with more CTAs than SMs, and the persistent
-    schedule sized for two CTAs per SM, are tried at the ring depth that fits two CTAs per SM."""
+def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148, fused: bool = True):
+    """(variant, split_k, reduce, tile_n, schedule, occupancy, k_slices, stages, fused) tuples legal
+    for the shape; stages 0 = the deepest ring.  A Swap-AB grid with more CTAs than SMs, and the
+    persistent schedule sized for two CTAs per SM, are tried at the ring depth that fits two CTAs per
+    SM; a Swap-AB grid of at most one CTA per SM is tried at the deepest ring and at that shallower
+    one (which leaves room for the next layer's CTAs to start streaming beside it).  At decode token
+    counts every Swap-AB candidate is also tried with the activation quantizer fused in."""
+    if fused and M <= 32:
+        # the fused quantizer has no two-pass reduction (it would need the scales in memory)
+        base = _candidates(fmt, M, N, K, num_sms, False)
+        return [c + (0,) for c in base] + [c + (1,) for c in _candidates(fmt, M, N, K, num_sms, True)
+                                           if c[0] == 1 and c[2] != 1]
+    return [c + (0,) for c in _candidates(fmt, M, N, K, num_sms, False)]
+
+
+def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
     nkt = (K + 127) // 128
     n_tiles = (N + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
     out = []
 
     def swap_grid(s, r, kps):
-        st = two_per_sm_stages(M, kps, r == 3) if n_tiles * s > num_sms else 0
-        out.append((1, s, r, 128, 0, 0, kps, st))
+        st2 = two_per_sm_stages(M, kps, r == 3, fz)
+        if n_tiles * s > num_sms:
+            out.append((1, s, r, 128, 0, 0, kps, st2))
+        else:
+            out.append((1, s, r, 128, 0, 0, kps, 0))
+            if st2:
+                out.append((1, s, r, 128, 0, 0, kps, st2))
 
     # Swap-AB: decode token counts, and up to 128 tokens for the per-token formats (the two-pass
     # reduction covers at most 32)
@@ -97,7 +118,7 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148):
             for r in reduces:
                 # Swap-AB, persistent: one CTA per SM at the deepest ring, or two at a ring that fits
                 out.append((1, 1, r, 128, 1, 1, kps, 0))
-                st2 = two_per_sm_stages(M, kps, False)
+                st2 = two_per_sm_stages(M, kps, False, fz)
                 if st2:
                     out.append((1, 1, r, 128, 1, 2, kps, st2))
         for s in splits:
@@ -145,13 +166,12 @@ class Problem:
         return self.fn(self.xq, self.sx, wq, sw, y=self.y, ws=self.ws)
 
     def layer_call(self, j=0):
-        """What the layer runs per call: quantize the activations, then the GEMM."""
-        if self.fmt == BLOCK_FP8:
-            qgd.quant_act_group128(self.x, xq=self.xq, sx=self.sx)
-        else:
-            qgd.quant_act_per_token(self.x, qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3,
-                                    xq=self.xq, sx=self.sx)
-        return self.run(j)
+        """What the layer runs per call: the layer call from bf16 activations
+        (quantizer kernel + GEMM, or one fused kernel, as the layer plan says),
+        warming the next call's weights in L2 as a decode step does."""
+        wq, sw = self.copies[j % len(self.copies)]
+        nxt = self.copies[(j + 1) % len(self.copies)][0]
+        return qgd.qlinear_bf16(self.fid, self.x, wq, sw, y=self.y, ws=self.ws, next_w=nxt)
 
     def acc32(self):
         return qgd.qgd_w8a8_int8_acc32(self.xq, self.copies[0][0], ws=self.ws)
@@ -161,7 +181,8 @@ class Problem:
         GEMM alone), each on its own weight copy."""
         n = len(self.copies)
         call = self.layer_call if with_quant else self.run
-        self.ws.ensure(qgd.qgd_workspace_size(self.fid, self.M, self.N, self.K))
+        self.ws.ensure(max(qgd.qgd_workspace_size(self.fid, self.M, self.N, self.K),
+                           qgd.qgd_layer_workspace_size(self.fid, self.M, self.N, self.K)))
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
@@ -187,7 +208,12 @@ class Problem:
 
 
 def tune_problem(p: Problem, log=None):
+    """Time every candidate (L2 run-ahead off), then refine the three fastest:
+    their ring depth, and for Swap-AB their L2 run-ahead.  Returns the best
+    (us, variant, split_k, reduce, stages, tile_n, schedule, occupancy,
+    k_slices, fused, l2_ahead) and the first pass's results."""
     fid = p.fid
+    qgd.qgd_set_override_ext(fid, 0, 0)
     qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0,
                          qgd.SCHEDULE_GRID, 0, 1)
     p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
@@ -196,35 +222,47 @@ def tune_problem(p: Problem, log=None):
     scale = ref.abs().max().item() + 1e-30
     results = []
     num_sms = torch.cuda.get_device_properties(p.y.device).multi_processor_count
-    for var, s, r, t, sch, occ, kps, st0 in candidates(p.fmt, p.M, p.N, p.K, num_sms):
+
+    def ensure_ws():
+        p.ws.ensure(max(qgd.qgd_workspace_size(fid, p.M, p.N, p.K),
+                        qgd.qgd_layer_workspace_size(fid, p.M, p.N, p.K)))
+
+    def timed(var, s, r, st, t, sch, occ, kps, fz, l2a):
+        qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
+        qgd.qgd_set_override_ext(fid, fz, l2a)
+        ensure_ws()
+        us = p.time_plan()
+        pl = qgd.qgd_get_layer_plan(fid, p.M, p.N, p.K)
+        return (us, var, pl["split_k"], r, pl["stages"], t, sch, pl["occupancy"], pl["k_slices"], pl["fused"],
+                pl["l2_ahead"])
+
+    for var, s, r, t, sch, occ, kps, st0, fz in candidates(p.fmt, p.M, p.N, p.K, num_sms):
         qgd.qgd_set_override(fid, var, s, r, st0, t, sch, occ, kps)
-        p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
-        y = p.run().float()
+        qgd.qgd_set_override_ext(fid, fz, 0)
+        ensure_ws()
+        y = p.layer_call().float()
         ok = (y - ref).abs().max().item() <= 2e-2 * scale
         if ok and ref_acc is not None:
-            ok = torch.equal(p.acc32(), ref_acc)
+            # exact int32 sums: every plan, fused or not, gives the same bits
+            ok = torch.equal(y, ref) and torch.equal(p.acc32(), ref_acc)
         if not ok:
             if log:
                 log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]} occ={occ} "
-                    f"kps={kps}: differs from the split-free result")
+                    f"kps={kps} fused={fz}: differs from the split-free result")
             continue
-        us = p.time_plan()
-        pl = qgd.qgd_get_plan(fid, p.M, p.N, p.K)
-        results.append((us, var, pl["split_k"], r, pl["stages"], t, sch, occ, pl["k_slices"]))
+        results.append(timed(var, s, r, st0, t, sch, occ, kps, fz, 0))
     results.sort()
-    # refine the pipeline depth of the three fastest
     refined = list(results[:3])
-    for us0, var, s, r, smax, t, sch, occ, kps in results[:3]:
-        for st in (2, 3, 4, 5, 6, 8, 10):
-            if st >= smax:
-                continue
-            qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
-            p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
-            us = p.time_plan()
-            occ_eff = qgd.qgd_get_plan(fid, p.M, p.N, p.K)["occupancy"]
-            refined.append((us, var, s, r, st, t, sch, occ_eff, kps))
+    for us0, var, s, r, smax, t, sch, occ, kps, fz, _ in results[:3]:
+        for st in (2, 3, 4, 5, 6, 8, 10):  # shallower rings
+            if st < smax:
+                refined.append(timed(var, s, r, st, t, sch, occ, kps, fz, 0))
+        if var == qgd.VARIANT_SWAP_AB:  # L2 run-ahead
+            for l2a in (2, 4, 8, 16):
+                refined.append(timed(var, s, r, smax, t, sch, occ, kps, fz, l2a))
     refined.sort()
     qgd.qgd_set_override(fid)
+    qgd.qgd_set_override_ext(fid, -1, -1)
     return refined[0], results
 
 
@@ -249,7 +287,7 @@ def main(argv=None):
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
             f = ln.split("#")[0].split()
-            if len(f) in (11, 12):
+            if len(f) in (11, 12, 13, 14):
                 done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
     only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
     t_start = time.time()
@@ -262,8 +300,8 @@ def main(argv=None):
         tmp = args.out + ".tmp"
         with open(tmp, "w") as f:
             f.write("# Dispatch table for B200 (sm_100a), measured by quantized_gemm_decode_b200.tune\n")
-            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy k_slices"
-                    "   # us per layer call (quantize + GEMM)\n")
+            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy k_slices fused "
+                    "l2_ahead   # us per layer call (quantize + GEMM)\n")
             for k in sorted(lines):
                 f.write(lines[k] + "\n")
         os.replace(tmp, args.out)
@@ -279,13 +317,13 @@ def main(argv=None):
                 t0 = time.time()
                 p = Problem(wl.fmt, M, N, K, wl.seed, device)
                 best, allres = tune_problem(p, log)
-                us, var, s, r, st, t, sch, occ, kps = best
+                us, var, s, r, st, t, sch, occ, kps, fz, l2a = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
                 lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "
-                              f"{occ} {kps}   # {us:.2f} us, {gbs:.0f} GB/s")
+                              f"{occ} {kps} {fz} {l2a}   # {us:.2f} us, {gbs:.0f} GB/s")
                 log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
-                    f"{SCHED_NAME[sch]} occ={occ} kps={kps} {us:.2f} us {gbs:.0f} GB/s ({len(allres)} candidates, "
-                    f"{time.time() - t0:.1f} s)")
+                    f"{SCHED_NAME[sch]} occ={occ} kps={kps} fused={fz} l2_ahead={l2a} {us:.2f} us {gbs:.0f} GB/s "
+                    f"({len(allres)} candidates, {time.time() - t0:.1f} s)")
                 del p
                 torch.cuda.empty_cache()
                 flush()

@@ -30,6 +30,7 @@ def clean_state():
     qgd.qgd_clear_dispatch_table()
     for f in range(3):
         qgd.qgd_set_override(f)
+        qgd.qgd_set_fused_override(f)
     yield
 
 
@@ -330,20 +331,64 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
     from quantized_gemm_decode_b200 import tune
 
     fid = tune.FMT_ID[fmt]
-    for var, s, r, t, sch, occ, kps, st in tune.candidates(fmt, M, N, K, 148):
+    cands = tune.candidates(fmt, M, N, K, 148)
+    assert any(c[8] for c in cands) == (M <= 32)  # fused candidates at decode token counts
+    for var, s, r, t, sch, occ, kps, st, fz in cands:
         qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
-        p = qgd.qgd_get_plan(fid, M, N, K)
-        assert (p["variant"], p["reduce"], p["schedule"], p["k_slices"]) == (var, r, sch, kps), (var, s, r, sch, kps)
+        qgd.qgd_set_fused_override(fid, fz)
+        p = qgd.qgd_get_layer_plan(fid, M, N, K)
+        assert (p["variant"], p["reduce"], p["schedule"], p["k_slices"], p["fused"]) == (var, r, sch, kps, fz), \
+            (var, s, r, sch, kps, fz)
         if sch == qgd.SCHEDULE_PERSISTENT and var == qgd.VARIANT_SWAP_AB:
             assert p["occupancy"] == occ
         if sch == qgd.SCHEDULE_GRID:
             assert p["split_k"] == s
         if st:
             assert p["stages"] == st
-            if var == qgd.VARIANT_SWAP_AB and (sch == qgd.SCHEDULE_GRID or occ == 2):
+            if var == qgd.VARIANT_SWAP_AB and (sch == qgd.SCHEDULE_GRID or occ == 2) and not fz:
                 mpad = tune.swap_mpad(M)
                 smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + (128 * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
+    qgd.qgd_set_fused_override(fid)
+
+
+def test_fused_plan_field():
+    G, P = qgd.SCHEDULE_GRID, qgd.SCHEDULE_PERSISTENT
+    fid = qgd.FMT_FP8_DYNAMIC
+    # not fused by default; the qlinear_* plan never is
+    assert qgd.qgd_get_layer_plan(fid, 4, 4096, 4096)["fused"] == 0
+    qgd.qgd_set_fused_override(fid, 1)
+    qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB, 4, qgd.REDUCE_TWO_PASS, 0, 0, G, 0, 2)
+    lp = qgd.qgd_get_layer_plan(fid, 4, 4096, 4096)
+    assert lp["fused"] == 1 and lp["source"] == 2
+    # the fused kernel has no two-pass reduction: the last CTA adds instead
+    assert lp["reduce"] == qgd.REDUCE_LAST_CTA
+    assert qgd.qgd_get_plan(fid, 4, 4096, 4096)["fused"] == 0
+    # a fused layer call needs only the GEMM's workspace; unfused it also holds codes and scales
+    assert qgd.qgd_layer_workspace_size(fid, 4, 4096, 4096) == qgd.qgd_workspace_size(fid, 4, 4096, 4096)
+    qgd.qgd_set_fused_override(fid, 0)
+    ws0 = qgd.qgd_layer_workspace_size(fid, 4, 4096, 4096)
+    assert ws0 >= qgd.qgd_workspace_size(fid, 4, 4096, 4096) + 4 * 4096 + 4 * 4
+    # Standard plans are never fused
+    qgd.qgd_set_fused_override(fid, 1)
+    qgd.qgd_set_override(fid, qgd.VARIANT_STANDARD, 1, 0, 0, 128, P)
+    assert qgd.qgd_get_layer_plan(fid, 64, 4096, 4096)["fused"] == 0
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_fused_override(fid, 2)
+    qgd.qgd_set_fused_override(fid)
+
+
+def test_table_fused_column(tmp_path):
+    t = tmp_path / "t.tsv"
+    t.write_text("fp8_dynamic 4096 4096 1 swap_ab 8 cluster 2 128 grid 0 2 1\n"
+                 "fp8_dynamic 4096 4096 2 swap_ab 8 cluster 2 128 grid 0 2 0\n")
+    qgd.qgd_load_dispatch_table(str(t))
+    assert qgd.qgd_get_layer_plan(0, 1, 4096, 4096)["fused"] == 1
+    assert qgd.qgd_get_layer_plan(0, 2, 4096, 4096)["fused"] == 0
+    assert qgd.qgd_get_plan(0, 1, 4096, 4096)["fused"] == 0
+    t.write_text("fp8_dynamic 4096 4096 1 swap_ab 8 cluster 2 128 grid 0 2 3\n")
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_load_dispatch_table(str(t))
 
 
 
@@ -428,3 +473,15 @@ def test_strided_quantizer_rejects_bad_row_stride():
     assert L.quant_act_group128_strided(P(16), 4, 512, 256, P(16), P(16), None) == -1
     # an empty call with a valid stride is fine
     assert L.quant_act_per_token_strided(P(16), 0, 512, 1024, 0, P(16), P(16), None) == 0
+
+
+def test_layer_call_rejects_bad_arguments():
+    L = qgd.lib()
+    P = ctypes.c_void_p
+    # misaligned warm-up range, row stride below K, null operands: refused before any launch
+    assert L.qlinear_fp8_dynamic_bf16(P(16), 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, P(17), 4096, None) == -1
+    assert L.qlinear_fp8_dynamic_bf16(P(16), 512, P(16), P(16), P(16), 4, 512, 1024, None, 0, None, 0, None) == -1
+    assert L.qlinear_w8a8_int8_bf16(None, 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, None, 0, None) == -1
+    assert L.qlinear_block_fp8_bf16(P(16), 1000, P(16), P(16), P(16), 4, 512, 1000, None, 0, None, 0, None) == -2
+    # an empty call is fine
+    assert L.qlinear_fp8_dynamic_bf16(None, 1024, None, None, None, 0, 512, 1024, None, 0, None, 0, None) == 0
