@@ -67,6 +67,10 @@ def load_library(path: str) -> ctypes.CDLL:
     L.orc_num_threads.argtypes = []
     L.orc_set_num_threads.restype = ctypes.c_int
     L.orc_set_num_threads.argtypes = [ctypes.c_int]
+    L.orc_quant_mx.restype = None
+    L.orc_quant_mx.argtypes = [P, lg, lg, P, P]
+    L.orc_gemm_mx.restype = None
+    L.orc_gemm_mx.argtypes = [P, P, P, P, lg, lg, lg, P, P]
     return L
 
 
@@ -176,6 +180,34 @@ def gemm_blockscaled(xq, sx, wq, sw, G: int = 128):
     bound = np.empty((M, N), dtype=np.float64)
     lib().orc_gemm_blockscaled(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, G,
                                _ptr(y), _ptr(bound))
+    return y, bound
+
+
+def quant_mx(x):
+    """MXFP8 (OCP MX v1.0): x [R, K] bf16, K % 32 == 0 -> (e4m3 codes [R, K],
+    E8M0 scale bytes [R, K/32])."""
+    xb = _bf16_bits(x)
+    R, K = xb.shape
+    assert K % 32 == 0
+    q = np.empty((R, K), dtype=np.uint8)
+    se = np.empty((R, K // 32), dtype=np.uint8)
+    lib().orc_quant_mx(_ptr(xb), R, K, _ptr(q), _ptr(se))
+    return q, se
+
+
+def gemm_mx(xq, sx, wq, sw):
+    """MXFP8 product: Y [M, N] fp64 and bound from e4m3 codes and E8M0 block
+    scales (sx [M, K/32], sw [N, K/32])."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.uint8)
+    M, K = xq.shape
+    N, _ = wq.shape
+    assert sx.shape == (M, K // 32) and sw.shape == (N, K // 32)
+    y = np.empty((M, N), dtype=np.float64)
+    bound = np.empty((M, N), dtype=np.float64)
+    lib().orc_gemm_mx(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), _ptr(bound))
     return y, bound
 
 

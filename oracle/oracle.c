@@ -343,6 +343,96 @@ int64_t orc_dot_split(const void *xq, long m, const void *wq, long n, long K,
     return total;
 }
 
+/* ------------------------------------------------------------------ */
+/* MXFP8: OCP Microscaling Formats (MX) v1.0 block scaling             */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The fourth format, beside Block_FP8: Blackwell tensor cores scale FP8
+ * operands in hardware with MX block scales (the pages list further vLLM
+ * formats and name Blackwell as the next target; the format itself is the
+ * OCP MX v1.0 specification).  A block of 32 consecutive values along K
+ * shares one scale X = 2^e, stored as an E8M0 byte e + 127 (e in -127..127;
+ * the byte 255 would be NaN and is never produced).  The elements are E4M3.
+ *
+ * Conversion of a block (the specification's rule):
+ *   e = floor(log2(max |v|)) - 8       (8: exponent of E4M3's largest
+ *                                        normal, 448 = 1.75 * 2^8)
+ *   clamped to [-127, 127];  code_i = E4M3(v_i / 2^e), round to nearest
+ *   even, magnitudes above 448 saturate to 448.
+ * Reading where the specification leaves it open: an all-zero block gets
+ * the smallest scale, e = -127 (every code +-0).
+ */
+static int mx_block_exp(double amax)
+{
+    int ex;
+    if (amax == 0.0)
+        return -127;
+    frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1): floor(log2) = ex - 1 */
+    ex = ex - 1 - 8;
+    if (ex < -127)
+        ex = -127;
+    if (ex > 127)
+        ex = 127;
+    return ex;
+}
+
+/* x [rows, K] bf16 (K % 32 == 0) -> e4m3 codes q [rows, K] and E8M0 scale
+ * bytes se [rows, K/32]. */
+void orc_quant_mx(const uint16_t *x, long rows, long K, uint8_t *q, uint8_t *se)
+{
+    long r, b, k, nb = K / 32;
+    for (r = 0; r < rows; r++)
+        for (b = 0; b < nb; b++) {
+            double amax = 0.0, unit;
+            int e;
+            for (k = 0; k < 32; k++) {
+                double a = fabs((double)bf16_to_float(x[r * K + b * 32 + k]));
+                if (a > amax)
+                    amax = a;
+            }
+            e = mx_block_exp(amax);
+            se[r * nb + b] = (uint8_t)(e + 127);
+            unit = ldexp(1.0, e);
+            for (k = 0; k < 32; k++) /* division by a power of two: exact */
+                q[r * K + b * 32 + k] =
+                    orc_e4m3_encode((double)bf16_to_float(x[r * K + b * 32 + k]) / unit);
+        }
+}
+
+/*
+ * MXFP8 product: one exact partial sum per 32-wide K block, weighted by the
+ * two blocks' scales:
+ *   y[m,n] = sum_b acc_b[m,n] * 2^-18 * 2^(sx[m,b]-127) * 2^(sw[n,b]-127)
+ * sx [M, K/32], sw [N, K/32] E8M0 bytes.  bound (nullable) = sum |x^||w^|.
+ */
+void orc_gemm_mx(const uint8_t *xq, const uint8_t *sx, const uint8_t *wq,
+                 const uint8_t *sw, long M, long N, long K, double *y,
+                 double *bound)
+{
+    long n, nb = K / 32;
+    double unit = acc_unit(ORC_E4M3);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < N; n++) {
+        long m, b;
+        for (m = 0; m < M; m++) {
+            double s = 0.0, bb = 0.0;
+            for (b = 0; b < nb; b++) {
+                int64_t aabs;
+                int64_t a = dot_range(xq, m, wq, n, K, b * 32, (b + 1) * 32,
+                                      ORC_E4M3, &aabs);
+                double scale = ldexp(1.0, (int)sx[m * nb + b] - 127 +
+                                              (int)sw[n * nb + b] - 127);
+                s += (double)a * unit * scale;
+                bb += (double)aabs * unit * scale;
+            }
+            y[m * N + n] = s;
+            if (bound)
+                bound[m * N + n] = bb;
+        }
+    }
+}
+
 /* Number of OpenMP threads the GEMMs above run on (1 without OpenMP). */
 int orc_num_threads(void)
 {

@@ -15,6 +15,7 @@ import pytest
 import oracle
 import test_oracle_codec as codec
 import test_oracle_gemm as gemm
+import test_oracle_mx as mx
 import test_oracle_quant as quant
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -48,6 +49,12 @@ MUTANTS = {
     "block row pitch": ("quant_group(w + nb * B * K + kb * B, B, B, K, ORC_E4M3,",
                         "quant_group(w + nb * B * K + kb * B, B, B, B, ORC_E4M3,"),
     "split chunk drops tail": ("if (k1 > K)\n            k1 = K;", "if (k1 >= K)\n            k1 = K - 1;"),
+    "mx exponent off by one": ("ex = ex - 1 - 8;", "ex = ex - 8;"),
+    "mx emax of 7": ("ex = ex - 1 - 8;", "ex = ex - 1 - 7;"),
+    "mx zero block scale": ("        return -127;\n    frexp", "        return 0;\n    frexp"),
+    "mx weight scale of the next block": ("(int)sw[n * nb + b] - 127);", "(int)sw[n * nb + (b + 1) % nb] - 127);"),
+    "mx scales added to exponent bias once": ("double scale = ldexp(1.0, (int)sx[m * nb + b] - 127 +",
+                                              "double scale = ldexp(1.0, (int)sx[m * nb + b] +"),
 }
 
 
@@ -75,6 +82,13 @@ def pin_suite():
     gemm.test_identity_weight_returns_dequantized_activations()
     gemm.test_one_hot_rows_select_columns()
     gemm.test_zero_activation_row_gives_zero_output()
+    mx.test_block_exponent_closed_form()
+    mx.test_zero_block_and_exponent_clamp()
+    mx.test_codes_match_torch_cast_of_scaled_values()
+    mx.test_dequantized_error_within_half_an_e4m3_step()
+    for shape in ((3, 17, 96), (1, 40, 256), (5, 8, 64)):
+        mx.test_mx_gemm_matches_brute_force(*shape)
+    mx.test_mx_gemm_scales_belong_to_their_own_block()
 
 
 @pytest.fixture
