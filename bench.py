@@ -35,7 +35,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from quantized_gemm_decode_b200 import synth, workloads  # noqa: E402
-from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8  # noqa: E402
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, W8A8_INT8  # noqa: E402
 
 METRIC = "achieved HBM GB/s & TFLOP/s (fraction of roofline) per format, M=1..32"
 L2_BYTES = 126 * 1024 * 1024
@@ -60,7 +60,7 @@ def peaks():
 def path_bytes(fmt: str, M: int, N: int, K: int) -> int:
     """Algorithmic bytes of quantize+GEMM: bf16 X in, weight codes and scales,
     bf16 Y out (the intermediate activation codes are not counted)."""
-    wscale = 4 * (N // 128) * (K // 128) if fmt == BLOCK_FP8 else 4 * N
+    wscale = 4 * (N // 128) * (K // 128) if fmt == BLOCK_FP8 else (N * (K // 32) if fmt == MXFP8 else 4 * N)
     return N * K + 2 * M * K + wscale + 2 * M * N
 
 
@@ -187,7 +187,7 @@ class DecodeSet:
 
         self.qgd = qgd
         self.wl, self.fmt, self.device = wl, wl.fmt, device
-        self.fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}[wl.fmt]
+        self.fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}[wl.fmt]
         self.ms = list(wl.ms)
         self.host_w = {}
         self.weights = {}  # (N, K) -> list of (wq, sw) copies
@@ -198,6 +198,8 @@ class DecodeSet:
             wd = w.to(device)
             if self.fmt == BLOCK_FP8:
                 wq, sw = qgd.quant_weight_block128(wd)
+            elif self.fmt == MXFP8:
+                wq, sw = qgd.quant_mx(wd)
             else:
                 wq, sw = qgd.quant_weight_per_channel(wd, qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
             del wd
@@ -214,11 +216,15 @@ class DecodeSet:
                 xd = x.to(device)
                 qdt = torch.int8 if self.fmt == W8A8_INT8 else torch.float8_e4m3fn
                 xq = torch.empty((M, K), dtype=qdt, device=device)
-                sx = torch.empty((M, K // 128) if self.fmt == BLOCK_FP8 else (M,), dtype=torch.float32, device=device)
+                if self.fmt == MXFP8:
+                    sx = torch.empty((M, K // 32), dtype=torch.uint8, device=device)
+                else:
+                    sx = torch.empty((M, K // 128) if self.fmt == BLOCK_FP8 else (M,), dtype=torch.float32,
+                                     device=device)
                 y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
                 self.calls.append(dict(M=M, N=N, K=K, mi=mi, x=xd, x_host=x, xq=xq, sx=sx, y=y))
                 ws_need = max(ws_need, qgd.qgd_workspace_size(self.fmt_id, M, N, K),
-                              qgd.qgd_layer_workspace_size(self.fmt_id, M, N, K))
+                              0 if self.fmt == MXFP8 else qgd.qgd_layer_workspace_size(self.fmt_id, M, N, K))
         self.ws = qgd.Workspace(ws_need, device)
         torch.cuda.synchronize(device)
 
@@ -227,6 +233,8 @@ class DecodeSet:
         qgd = self.qgd
         if self.fmt == BLOCK_FP8:
             qgd.quant_act_group128(c["x"], xq=c["xq"], sx=c["sx"])
+        elif self.fmt == MXFP8:
+            qgd.quant_mx(c["x"], xq=c["xq"], sx=c["sx"])
         else:
             qgd.quant_act_per_token(c["x"], qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3,
                                     xq=c["xq"], sx=c["sx"])
@@ -236,29 +244,27 @@ class DecodeSet:
         copies = self.weights[(c["N"], c["K"])]
         wq, sw = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
         fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
-              BLOCK_FP8: qgd.qlinear_block_fp8}[self.fmt]
+              BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8}[self.fmt]
         fn(c["xq"], c["sx"], wq, sw, y=c["y"], ws=self.ws)
 
-    def layer(self, c, copy_idx=None, next_w=None):
+    def layer(self, c, copy_idx=None):
         """The layer call from bf16 activations (quantizer fused into the GEMM
-        where the layer plan says so), warming `next_w` in L2."""
+        where the layer plan says so).  (MXFP8 has no layer call: its
+        quantizer kernel, then its GEMM.)"""
+        if self.fmt == MXFP8:
+            self.quant(c)
+            self.gemm(c, copy_idx)
+            return
         copies = self.weights[(c["N"], c["K"])]
         wq, sw = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
-        self.qgd.qlinear_bf16(self.fmt_id, c["x"], wq, sw, y=c["y"], ws=self.ws, next_w=next_w)
-
-    def weight_of(self, c, copy_idx=None):
-        copies = self.weights[(c["N"], c["K"])]
-        return copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)][0]
+        self.qgd.qlinear_bf16(self.fmt_id, c["x"], wq, sw, y=c["y"], ws=self.ws)
 
     def step(self, gemm_only=False):
-        """One pass: every call in order, each warming the next call's weights
-        in L2 (the last one the first call's, which the next step runs first)."""
-        n = len(self.calls)
-        for i, c in enumerate(self.calls):
+        for c in self.calls:
             if gemm_only:
                 self.gemm(c)
             else:
-                self.layer(c, next_w=self.weight_of(self.calls[(i + 1) % n]))
+                self.layer(c)
 
     def capture(self, fn) -> torch.cuda.CUDAGraph:
         s = torch.cuda.Stream(self.device)
@@ -278,7 +284,7 @@ class DecodeSet:
         for two-pass Split-K, and (layer calls) the quantizer unless fused."""
         n = 0
         for c in self.calls:
-            get = self.qgd.qgd_get_plan if gemm_only else self.qgd.qgd_get_layer_plan
+            get = self.qgd.qgd_get_plan if (gemm_only or self.fmt == MXFP8) else self.qgd.qgd_get_layer_plan
             p = get(self.fmt_id, c["M"], c["N"], c["K"])
             n += (0 if gemm_only or p["fused"] else 1) + 1 + (1 if p["split_k"] > 1 and p["reduce"] == 1 else 0)
         return n
@@ -289,10 +295,9 @@ class DecodeSet:
         -- the fused kernel on the bf16 activations (the same kernel the step
         runs).  Returns the algorithmic bytes those launches must move."""
         b = 0
-        n = len(self.calls)
-        for i, c in enumerate(self.calls):
-            if self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"]:
-                self.layer(c, next_w=self.weight_of(self.calls[(i + 1) % n]))
+        for c in self.calls:
+            if self.fmt != MXFP8 and self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"]:
+                self.layer(c)
                 b += path_bytes(self.fmt, c["M"], c["N"], c["K"])
             else:
                 self.gemm(c)
@@ -300,6 +305,8 @@ class DecodeSet:
         return b
 
     def fused_calls(self) -> int:
+        if self.fmt == MXFP8:
+            return 0
         return sum(self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"] for c in self.calls)
 
     def bytes_per_step(self):
@@ -356,7 +363,7 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
 
         def layer(c=c, ncop=ncop):
             for j in range(ncop):
-                ds.layer(c, copy_idx=j, next_w=ds.weight_of(c, j + 1))
+                ds.layer(c, copy_idx=j)
 
         g = ds.capture(body)
         times = replay_times(g, reps)
@@ -387,7 +394,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
 
 def quant_bytes(fmt: str, M: int, K: int) -> int:
     """Algorithmic bytes of the activation quantizer: bf16 X in, codes and scales out."""
-    return 2 * M * K + M * K + (4 * M * (K // 128) if fmt == BLOCK_FP8 else 4 * M)
+    scales = 4 * M * (K // 128) if fmt == BLOCK_FP8 else (M * (K // 32) if fmt == MXFP8 else 4 * M)
+    return 2 * M * K + M * K + scales
 
 
 def quantizer_summary(ds: DecodeSet, reps: int = 20):
@@ -976,7 +984,7 @@ def main():
                              "frac": round(value / world / pk["hbm_gbs"], 4),
                              "quantizer": quantizer_summary(ds)}
         keep = ds
-        for wl2 in (workloads.INT8_DECODE, workloads.BLOCK_DECODE):
+        for wl2 in (workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE):
             ds2 = DecodeSet(wl2, device, per_call_rotation=True)
             fmts[wl2.fmt] = format_summary(ds2, args.steps, args.warmup, pk["hbm_gbs"])
             fmts[wl2.fmt]["quantizer"] = quantizer_summary(ds2)

@@ -64,7 +64,7 @@ typedef enum {
   QGD_ERR_DEVICE = -6       /* current device is not an sm_100 part */
 } qgd_status;
 
-typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8 = 2 } qgd_format;
+typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8 = 2, QGD_FMT_MXFP8 = 3 } qgd_format;
 typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
 /* Standard: X is the MMA's A operand (128-token tiles).  Swap-AB: Y^T = W X^T, the weight rows fill
  * the MMA's 128-row slot and the tokens its N (16/32/64/128); up to 32 tokens for Block_FP8 and up
@@ -108,10 +108,6 @@ typedef struct {
   int fused;     /* layer calls (qlinear_*_bf16) only: 1 = the activation quantizer runs inside the
                     Swap-AB GEMM kernel, 0 = a separate quantizer kernel first.  Always 0 in the plan
                     of the qlinear_* calls, which take quantized activations */
-  int l2_ahead;  /* Swap-AB: how many weight units (a pipeline stage's worth of weight tiles) each
-                    CTA prefetches into L2 ahead of its shared-memory ring, 0..64 (0 = none; always 0
-                    for Standard).  The L2 holds what the ring cannot, so more of the weight stream
-                    is in flight than shared memory alone allows */
 } qgd_plan;
 
 /* ---------------------------------------------------------------------
@@ -196,29 +192,48 @@ QGD_API qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void
  * overlap), ws may be NULL when that size is 0.  Shapes as qlinear_*, and
  * K <= 65536.  Errors as qlinear_*; ldx < K or not a multiple of 8 ->
  * QGD_ERR_INVALID.
- * next_w / next_bytes (optional; NULL / 0 for none): a device range -- for
- *   example the next layer's weight codes -- that the Swap-AB GEMM warms in
- *   L2: once a CTA has issued all of its own weight loads it prefetches its
- *   share of the range, so HBM keeps streaming through this call's tail and
- *   the next call's start instead of idling.  Only a hint: no result
- *   depends on it; bytes beyond a multiple of 16 are ignored.  next_w must
- *   be 16-byte aligned and the whole range readable device memory (else
- *   QGD_ERR_INVALID for a misaligned pointer; an unreadable range is
- *   undefined behaviour).  Standard plans ignore it.
  * ------------------------------------------------------------------- */
 QGD_API qgd_status qlinear_fp8_dynamic_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
                                             void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
-                                            const void* next_w, size_t next_bytes, void* stream);
+                                            void* stream);
 QGD_API qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
                                           void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
-                                          const void* next_w, size_t next_bytes, void* stream);
+                                          void* stream);
 QGD_API qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
                                           void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
-                                          const void* next_w, size_t next_bytes, void* stream);
+                                          void* stream);
 
 /* Bytes of workspace a layer call for (fmt, M, N, K) needs under the layer
  * plan in force (0 when none). */
 QGD_API size_t qgd_layer_workspace_size(int fmt, int M, int N, int K);
+
+/* ---------------------------------------------------------------------
+ * MXFP8, a fourth format beside Block_FP8 for Blackwell's block-scaled
+ * tensor cores (the pages list further vLLM formats and name Blackwell as
+ * the next target; the format is the OCP Microscaling (MX) v1.0 definition):
+ * every 32 consecutive values of a row along K share one power-of-two scale
+ * 2^e, stored as an E8M0 byte e + 127; the values are e4m3.
+ *     e = clamp(floor(log2(max |x| over the block)) - 8, -127, 127)
+ *         (8: the exponent of e4m3's largest normal; an all-zero block
+ *          takes e = -127),   q = e4m3_rne_satfinite(x * 2^-e).
+ * The GEMM multiplies in hardware (tcgen05.mma kind::mxf8f6f4 with E8M0
+ * block scales read from tensor memory): Y = sum over 32-wide K blocks of
+ * (Xq . Wq^T)_block * 2^(ex + ew), fp32 accumulation, bf16 out.
+ * ------------------------------------------------------------------- */
+
+/* MX quantizer: x_bf16 [M,K] (rows ldx elements apart, ldx >= K, ldx % 8 ==
+ * 0) -> xq e4m3 [M,K], s_e8m0 [M][K/32] bytes.  Also the weight quantizer
+ * (rows = N).  Requires K % 32 == 0; x and xq 16-byte aligned. */
+QGD_API qgd_status quant_act_mx(const void* x_bf16, int M, int K, int ldx, void* xq, void* s_e8m0, void* stream);
+
+/* MXFP8 GEMM: y_bf16 [M,N] from xq [M,K], sx_e8m0 [M][K/32], wq [N,K],
+ * sw_e8m0 [N][K/32].  Swap-AB kernel only: 0 <= M <= 64 (more ->
+ * QGD_ERR_UNSUPPORTED); K % 128 == 0, N % 16 == 0; all pointers 16-byte
+ * aligned.  The block scales sit in tensor memory beside the accumulators
+ * (at most 256 columns per CTA, which caps the ring depth).  Workspace as qlinear_fp8_dynamic (same plans; no two-pass
+ * reduction, whose requests take the last-arriving CTA). */
+QGD_API qgd_status qlinear_mxfp8(const void* xq, const void* sx_e8m0, const void* wq, const void* sw_e8m0,
+                                 void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
 /* Test hook: the W8A8_INT8 mainloop and Split-K reduction of the plan in
  * force, writing the exact int32 accumulator acc[M][N] instead of Y. */
@@ -260,7 +275,7 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
 /* Load a dispatch table: a text file with one line per (format, N, K,
  * M-bucket) and '#' comments,
  *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy [k_slices]
- * fmt in {fp8_dynamic, w8a8_int8, block_fp8}; variant in {standard, swap_ab};
+ * fmt in {fp8_dynamic, w8a8_int8, block_fp8, mxfp8}; variant in {standard, swap_ab};
  * reduce in {last_cta, two_pass, atomic, cluster}; schedule in {grid, persistent};
  * stages/tile_n/occupancy/k_slices 0 (or k_slices absent) = default.
  * Replaces the table in force.  On
@@ -268,8 +283,7 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
  * concurrent qlinear_* calls. */
 QGD_API qgd_status qgd_load_dispatch_table(const char* path);
 
-/* (Optional 13th and 14th fields: fused = 0 or 1, the layer plan's `fused`;
- * l2_ahead = 0..64.) */
+/* (An optional 13th field, fused = 0 or 1, sets the layer plan's `fused`.) */
 
 /* Drop the table in force; the built-in defaults apply again. */
 QGD_API qgd_status qgd_clear_dispatch_table(void);
@@ -287,14 +301,11 @@ QGD_API qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan);
  * same table entry, with its `fused` field in effect. */
 QGD_API qgd_status qgd_get_layer_plan(int fmt, int M, int N, int K, qgd_plan* plan);
 
-/* Force the plan fields qgd_set_override does not cover, for one format
- * (tests and the tuner); -1 keeps the table / default for that field.
- *   fused     layer plans: 0 = quantizer kernel first, 1 = fused (Swap-AB
- *             plans only; others stay unfused)
- *   l2_ahead  Swap-AB L2 run-ahead in weight units, 0..64
- * Independent of qgd_set_override; qgd_set_override_ext(fmt, -1, -1)
- * removes it.  Out-of-range values -> QGD_ERR_INVALID. */
-QGD_API qgd_status qgd_set_override_ext(int fmt, int fused, int l2_ahead);
+/* Force the `fused` field of layer plans for one format (tests and the
+ * tuner): -1 = table / default (not fused), 0 = quantizer kernel first,
+ * 1 = fused (Swap-AB plans only; others stay unfused).  Independent of
+ * qgd_set_override.  Other values -> QGD_ERR_INVALID. */
+QGD_API qgd_status qgd_set_fused_override(int fmt, int fused);
 
 /* M-bucket of a token count: the smallest tuned count >= M among
  * 1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192 (the last one beyond). */

@@ -27,14 +27,13 @@ __all__ = [
     "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC", "REDUCE_CLUSTER",
     "SCHEDULE_GRID", "SCHEDULE_PERSISTENT",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
-    "quant_act_per_token_strided", "quant_act_group128_strided",
+    "quant_act_per_token_strided", "quant_act_group128_strided", "quant_mx", "qlinear_mxfp8", "FMT_MXFP8",
     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
     "qgd_mma_peak_probe", "qgd_test_withhold_accumulator",
     "qlinear_bf16", "qgd_layer_workspace_size", "qgd_get_layer_plan", "qgd_set_fused_override",
-    "qgd_set_override_ext",
     "qgd_test_capture_fused",
     "Workspace", "DEFAULT_TABLE",
 ]
@@ -45,12 +44,12 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("QGD_LIBRARY") or os.path.join(_PKG, "libqgd.so")
 DEFAULT_TABLE = os.path.join(_PKG, "tables", "b200.tsv")
 
-FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8 = 0, 1, 2
+FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8, FMT_MXFP8 = 0, 1, 2, 3
 QTYPE_E4M3, QTYPE_INT8 = 0, 1
 VARIANT_STANDARD, VARIANT_SWAP_AB = 0, 1
 REDUCE_LAST_CTA, REDUCE_TWO_PASS, REDUCE_ATOMIC, REDUCE_CLUSTER = 0, 1, 2, 3
 SCHEDULE_GRID, SCHEDULE_PERSISTENT = 0, 1
-FORMAT_NAMES = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2}
+FORMAT_NAMES = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "mxfp8": 3}
 
 _lock = threading.Lock()
 _lib = None
@@ -66,7 +65,7 @@ class _Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int), ("split_k", ctypes.c_int), ("reduce", ctypes.c_int),
                 ("stages", ctypes.c_int), ("tile_n", ctypes.c_int), ("schedule", ctypes.c_int),
                 ("occupancy", ctypes.c_int), ("source", ctypes.c_int), ("k_slices", ctypes.c_int),
-                ("fused", ctypes.c_int), ("l2_ahead", ctypes.c_int)]
+                ("fused", ctypes.c_int)]
 
 
 def lib() -> ctypes.CDLL:
@@ -98,12 +97,14 @@ def lib() -> ctypes.CDLL:
             "qgd_clear_device_error": [],
             "qgd_mma_peak_probe": [I, I, ctypes.POINTER(ctypes.c_double), P],
             "qgd_test_withhold_accumulator": [I],
-            "qlinear_fp8_dynamic_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
-            "qlinear_w8a8_int8_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
-            "qlinear_block_fp8_bf16": [P, I, P, P, P, I, I, I, P, S, P, S, P],
+            "qlinear_fp8_dynamic_bf16": [P, I, P, P, P, I, I, I, P, S, P],
+            "qlinear_w8a8_int8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
+            "qlinear_block_fp8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
             "qgd_get_layer_plan": [I, I, I, I, ctypes.POINTER(_Plan)],
-            "qgd_set_override_ext": [I, I, I],
+            "qgd_set_fused_override": [I, I],
             "qgd_test_capture_fused": [P, P],
+            "quant_act_mx": [P, I, I, I, P, P, P],
+            "qlinear_mxfp8": [P, P, P, P, P, I, I, I, P, S, P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -218,6 +219,20 @@ def quant_act_group128(x: torch.Tensor, xq=None, sx=None, stream=None):
         sx = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
     _check(lib().quant_act_group128_strided(_ptr(x), M, K, ldx, _ptr(xq), _ptr(sx), _stream(stream)),
            "quant_act_group128")
+    return xq, sx
+
+
+def quant_mx(x: torch.Tensor, xq=None, sx=None, stream=None):
+    """MXFP8 quantization (OCP MX v1.0): x bf16 [R, K] -> (e4m3 codes [R, K],
+    E8M0 scale bytes uint8 [R, K/32]).  Activations and weights alike; x may
+    be a column slice of a wider matrix."""
+    ldx = _activation_rows(x)
+    R, K = x.shape
+    if xq is None:
+        xq = torch.empty((R, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if sx is None:
+        sx = torch.empty((R, K // 32), dtype=torch.uint8, device=x.device)
+    _check(lib().quant_act_mx(_ptr(x), R, K, ldx, _ptr(xq), _ptr(sx), _stream(stream)), "quant_act_mx")
     return xq, sx
 
 
@@ -342,12 +357,10 @@ _LAYER_FN = {FMT_FP8_DYNAMIC: "qlinear_fp8_dynamic_bf16", FMT_W8A8_INT8: "qlinea
              FMT_BLOCK_FP8: "qlinear_block_fp8_bf16"}
 
 
-def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None, next_w=None):
+def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None):
     """Layer call from bf16 activations: dynamic quantization and the GEMM,
     fused into one kernel when the layer plan says so (qgd_get_layer_plan).
-    x [M, K] bf16 may be a column slice of a wider matrix.  next_w (a CUDA
-    tensor, e.g. the next layer's weight codes) is warmed in L2 while this
-    call finishes; it changes no result."""
+    x [M, K] bf16 may be a column slice of a wider matrix."""
     ldx = _activation_rows(x)
     M, K = x.shape
     want_w = (torch.int8,) if fmt == FMT_W8A8_INT8 else (torch.uint8, torch.float8_e4m3fn)
@@ -375,14 +388,36 @@ def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None
         wsp, wsn = ws.buf.data_ptr(), ws.nbytes
     else:
         wsp, wsn = ws.data_ptr(), ws.numel() * ws.element_size()
-    nb = 0
-    if next_w is not None:
-        if not isinstance(next_w, torch.Tensor) or not next_w.is_cuda or not next_w.is_contiguous():
-            raise ValueError("next_w must be a contiguous CUDA tensor")
-        nb = next_w.numel() * next_w.element_size()
     fn = _LAYER_FN[fmt]
     _check(getattr(lib(), fn)(_ptr(x), ldx, _ptr(wq), _ptr(sw), _ptr(y), M, N, K, ctypes.c_void_p(wsp), wsn,
-                              _ptr(next_w), nb, _stream(stream)), fn)
+                              _stream(stream)), fn)
+    return y
+
+
+def qlinear_mxfp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
+    """Y bf16 [M, N] from MXFP8 operands: e4m3 codes with E8M0 block scales
+    (uint8 [M, K/32] and [N, K/32]), scaled by the tensor core."""
+    for t, name in ((xq, "xq"), (wq, "wq")):
+        if not isinstance(t, torch.Tensor) or t.dim() != 2 or t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise ValueError(f"{name} must be a 2-D e4m3 tensor")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"K mismatch: xq {tuple(xq.shape)} vs wq {tuple(wq.shape)}")
+    for t, name, rows in ((sx, "sx", M), (sw, "sw", N)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or tuple(t.shape) != (rows, K // 32) \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous uint8 tensor of shape {(rows, K // 32)}")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    elif y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous bfloat16 tensor of shape {(M, N)}")
+    for t, name in ((xq, "xq"), (wq, "wq"), (sx, "sx"), (sw, "sw"), (y, "y")):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    wsp, wsn = _workspace(FMT_MXFP8, M, N, K, ws, xq.device)
+    _check(lib().qlinear_mxfp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K, ctypes.c_void_p(wsp), wsn,
+                               _stream(stream)), "qlinear_mxfp8")
     return y
 
 
@@ -452,16 +487,9 @@ def qgd_get_layer_plan(fmt: int, M: int, N: int, K: int) -> dict:
     return {f: getattr(p, f) for f, _ in _Plan._fields_}
 
 
-def qgd_set_override_ext(fmt: int, fused: int = -1, l2_ahead: int = -1) -> None:
-    """Force the `fused` (layer plans) and `l2_ahead` plan fields for one
-    format; -1 keeps the table / default."""
-    _check(lib().qgd_set_override_ext(fmt, fused, l2_ahead), "qgd_set_override_ext")
-
-
 def qgd_set_fused_override(fmt: int, fused: int = -1) -> None:
-    """Force layer plans' `fused` field for one format (-1 = table /
-    default), leaving l2_ahead to the table."""
-    qgd_set_override_ext(fmt, fused, -1)
+    """Force layer plans' `fused` field for one format (-1 = table / default)."""
+    _check(lib().qgd_set_fused_override(fmt, fused), "qgd_set_fused_override")
 
 
 def qgd_test_capture_fused(xq=None, sx=None) -> None:

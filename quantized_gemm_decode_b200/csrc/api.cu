@@ -112,22 +112,25 @@ const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
 constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;   // decode token counts: Swap-AB by default
 constexpr int kSwapMaxM = 128;    // largest token count the Swap-AB kernel covers (FP8_Dynamic, W8A8_INT8)
-constexpr int kMaxL2Ahead = 64;   // most weight units a Swap-AB CTA prefetches into L2 ahead of its ring
+// MXFP8: at most 64 tokens, and at most 256 tensor-memory columns per CTA, so
+// that two CTAs always fit in an SM's 512 columns (a CTA whose allocation had
+// to wait for a cluster peer on the same SM would never be released)
+constexpr int kMxMaxM = 64;
+constexpr unsigned kMxMaxCols = 256;
 
 // Token columns of the Swap-AB MMA (its N): the next of 16, 32, 64, 128.
 int swap_mpad(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
 struct Entry {
-  int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices, fused, l2_ahead;
+  int variant, split_k, reduce, stages, tile_n, schedule, occupancy, k_slices, fused;
 };
 using Key = std::tuple<int, int, int, int>;
 std::mutex g_mu;
 std::map<Key, Entry> g_table;
 struct Override {
   int variant = -1, split_k = -1, reduce = -1, stages = 0, tile_n = 0, schedule = -1, occupancy = 0, k_slices = 0;
-  int fused = -1;     // layer calls: -1 = table/default, 0/1 forced
-  int l2_ahead = -1;  // -1 = table/default, else forced
-} g_override[3];
+  int fused = -1;  // layer calls: -1 = table/default, 0/1 forced
+} g_override[kNumFmts];
 
 int bucket_of(int M) {
   for (int i = 0; i < kNumBuckets; ++i)
@@ -145,6 +148,7 @@ int fmt_from_name(const std::string& s) {
   if (s == "fp8_dynamic" || s == "fp8") return kFmtFP8;
   if (s == "w8a8_int8" || s == "int8") return kFmtINT8;
   if (s == "block_fp8" || s == "block") return kFmtBlock;
+  if (s == "mxfp8" || s == "mx") return kFmtMX;
   return -1;
 }
 
@@ -175,7 +179,6 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   qgd_plan p;
   p.source = 0;
   p.fused = 0;
-  p.l2_ahead = 0;
   p.reduce = kLastCta;
   p.stages = 0;
   p.schedule = kGrid;
@@ -213,7 +216,6 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
       p.occupancy = e.occupancy;
       p.k_slices = e.k_slices;
       p.fused = e.fused;
-      p.l2_ahead = e.l2_ahead;
       p.source = 1;
     }
     const Override& o = g_override[fmt];
@@ -233,12 +235,14 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
       p.fused = o.fused;
       p.source = 2;
     }
-    if (o.l2_ahead >= 0) {
-      p.l2_ahead = o.l2_ahead;
-      p.source = 2;
-    }
+
   }
-  // Make the plan legal for this shape.
+  // Make the plan legal for this shape.  (MXFP8 runs in the Swap-AB kernel
+  // only, up to 128 tokens, and has no two-pass reduction kernel.)
+  if (fmt == kFmtMX) {
+    p.variant = kSwapAB;
+    if (p.reduce == kTwoPass) p.reduce = kLastCta;
+  }
   if (p.variant == kSwapAB && M > (fmt == kFmtBlock ? kDecodeMaxM : kSwapMaxM)) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
@@ -269,9 +273,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   // the fused quantizer exists in the Swap-AB kernel only; its two-pass
   // reduction would need the activation scales in memory, so it takes the
   // last-arriving CTA instead
-  if (!layer || p.variant != kSwapAB) p.fused = 0;
-  if (p.variant != kSwapAB || p.l2_ahead < 0) p.l2_ahead = 0;
-  if (p.l2_ahead > kMaxL2Ahead) p.l2_ahead = kMaxL2Ahead;
+  if (!layer || p.variant != kSwapAB || fmt == kFmtMX) p.fused = 0;
   p.fused = p.fused ? 1 : 0;
   if (p.fused && p.reduce == kTwoPass) p.reduce = kLastCta;
   const int mpad = swap_mpad(M);
@@ -279,6 +281,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
                                           : standard_max_stages(p.tile_n);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
+  if (fmt == kFmtMX)
+    while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices) > kMxMaxCols) --p.stages;
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;
@@ -288,6 +292,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
     if (p.variant == kStandard && (p.tile_n == 256 || fmt == kFmtBlock)) fit = 1;  // all 512 TMEM columns
+
   }
   if (p.occupancy <= 0 || p.occupancy > fit) p.occupancy = fit;
   if (p.schedule != kPersistent) p.occupancy = 1;
@@ -377,6 +382,9 @@ qgd_status check_shape(int fmt, int M, int N, int K) {
   if (K % 16 != 0) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 16", K);
   if (fmt == kFmtBlock && (K % 128 != 0 || N % 128 != 0))
     return fail(QGD_ERR_UNSUPPORTED, "Block_FP8 needs N and K multiples of 128 (N=%d K=%d)", N, K);
+  if (fmt == kFmtMX && K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128 (K=%d)", K);
+  if (fmt == kFmtMX && M > kMxMaxM)
+    return fail(QGD_ERR_UNSUPPORTED, "MXFP8 covers at most %d tokens (M=%d)", kMxMaxM, M);
   if (static_cast<long long>(M) * N > (1LL << 31)) return fail(QGD_ERR_UNSUPPORTED, "M*N too large");
   return QGD_OK;
 }
@@ -392,8 +400,7 @@ std::atomic<float*> g_capture_sx{nullptr};
 // defined between two kernels only).
 qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float* sx, const uint16_t* xbf, int ldxb,
                          const void* wq, const float* sw, void* y, void* raw, int M, int N, int K, void* ws,
-                         size_t ws_bytes, void* stream, bool follows_memset, const void* pf = nullptr,
-                         size_t pf_bytes = 0) {
+                         size_t ws_bytes, void* stream, bool follows_memset) {
   qgd_status st;
   if ((st = check_device()) != QGD_OK) return st;
   if ((st = get_encoder()) != QGD_OK) return st;
@@ -436,10 +443,8 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
   a.ldxb = ldxb;
   a.xq_out = fused ? static_cast<uint8_t*>(g_capture_xq.load()) : nullptr;
   a.sx_out = fused ? g_capture_sx.load() : nullptr;
-  // (the Standard kernel does not warm L2; its calls are compute-bound)
-  a.l2_ahead = p.l2_ahead;
-  a.pf = static_cast<const uint8_t*>(pf);
-  a.pf_bytes = p.variant == kSwapAB ? pf_bytes : 0;
+  a.sx8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sx) : nullptr;
+  a.sw8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sw) : nullptr;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
@@ -508,11 +513,9 @@ LayerWs layer_ws(int fmt, int M, int N, int K) {
 }
 
 qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const float* sw, void* y, int M, int N,
-                     int K, void* ws, size_t ws_bytes, const void* next_w, size_t next_bytes, void* stream) {
+                     int K, void* ws, size_t ws_bytes, void* stream) {
   qgd_status st = check_shape(fmt, M, N, K);
   if (st != QGD_OK) return st;
-  if (next_bytes && (!next_w || !aligned16(next_w)))
-    return fail(QGD_ERR_INVALID, "next_w must be a 16-byte aligned device pointer when next_bytes > 0");
   if (ldx < K || ldx % 8 != 0)
     return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
   if (K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be <= 65536", K);
@@ -527,7 +530,7 @@ qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const
   const uint16_t* xb = static_cast<const uint16_t*>(x_bf16);
   if (l.plan.fused)
     return run_gemm_plan(fmt, l.plan, nullptr, nullptr, xb, ldx, wq, sw, y, nullptr, M, N, K, ws, ws_bytes, stream,
-                         false, next_w, next_bytes);
+                         false);
   if ((st = check_device()) != QGD_OK) return st;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* xq = wsb + l.xq_off;
@@ -537,8 +540,7 @@ qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const
                       ? launch_quant_group128(xb, M, K, ldx, static_cast<uint8_t*>(xq), sx, s)
                       : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
   if (e != cudaSuccess) return cuda_fail(e, "activation quantizer launch");
-  return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false,
-                       next_w, next_bytes);
+  return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -622,6 +624,21 @@ qgd_status quant_act_group128(const void* x_bf16, int M, int K, void* xq, float*
   return quant_act_group128_strided(x_bf16, M, K, K, xq, sx, stream);
 }
 
+qgd_status quant_act_mx(const void* x_bf16, int M, int K, int ldx, void* xq, void* s_e8m0, void* stream) {
+  if (M < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (M=%d K=%d)", M, K);
+  if (K % 32 != 0) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 32", K);
+  if (ldx < K || ldx % 8 != 0)
+    return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
+  if (M == 0) return QGD_OK;
+  if (!x_bf16 || !xq || !s_e8m0) return fail(QGD_ERR_INVALID, "null pointer");
+  if (!aligned16(x_bf16) || !aligned16(xq)) return fail(QGD_ERR_INVALID, "x and xq must be 16-byte aligned");
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  cudaError_t e = launch_quant_mx(static_cast<const uint16_t*>(x_bf16), M, K, ldx, static_cast<uint8_t*>(xq),
+                                  static_cast<uint8_t*>(s_e8m0), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_mx launch");
+}
+
 qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream) {
   if (N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (N=%d K=%d)", N, K);
   if (N % 128 != 0 || K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "N=%d and K=%d must be multiples of 128", N, K);
@@ -650,45 +667,48 @@ qgd_status qlinear_block_fp8(const void* xq, const float* sx, const void* wq, co
   return run_gemm(kFmtBlock, xq, sx, wq, sw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream);
 }
 
+qgd_status qlinear_mxfp8(const void* xq, const void* sx_e8m0, const void* wq, const void* sw_e8m0, void* y_bf16,
+                         int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  // the E8M0 scale rows are read as 32-bit words (4 blocks = one 128-wide K slice)
+  if ((reinterpret_cast<uintptr_t>(sx_e8m0) & 3u) || (reinterpret_cast<uintptr_t>(sw_e8m0) & 3u))
+    return fail(QGD_ERR_INVALID, "MXFP8 scale arrays must be 4-byte aligned");
+  return run_gemm(kFmtMX, xq, static_cast<const float*>(sx_e8m0), wq, static_cast<const float*>(sw_e8m0), y_bf16,
+                  nullptr, M, N, K, ws, ws_bytes, stream);
+}
+
 qgd_status qlinear_fp8_dynamic_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
-                                    int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
-                                    size_t next_bytes, void* stream) {
-  return run_layer(kFmtFP8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+                                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_layer(kFmtFP8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, stream);
 }
 
 qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
-                                  int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
-                                  size_t next_bytes, void* stream) {
-  return run_layer(kFmtINT8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+                                  int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_layer(kFmtINT8, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, stream);
 }
 
 qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
-                                  int M, int N, int K, void* ws, size_t ws_bytes, const void* next_w,
-                                  size_t next_bytes, void* stream) {
-  return run_layer(kFmtBlock, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, next_w, next_bytes, stream);
+                                  int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_layer(kFmtBlock, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, stream);
 }
 
 size_t qgd_layer_workspace_size(int fmt, int M, int N, int K) {
-  if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
+  if (fmt < 0 || fmt >= kNumFmts || M <= 0 || N <= 0 || K <= 0) return 0;
   return layer_ws(fmt, M, N, K).total;
 }
 
 qgd_status qgd_get_layer_plan(int fmt, int M, int N, int K, qgd_plan* plan) {
   if (!plan) return fail(QGD_ERR_INVALID, "null plan");
-  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "bad sizes");
   *plan = make_plan(fmt, M < 1 ? 1 : M, N, K, true);
   return QGD_OK;
 }
 
-qgd_status qgd_set_override_ext(int fmt, int fused, int l2_ahead) {
-  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+qgd_status qgd_set_fused_override(int fmt, int fused) {
+  if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (fused < -1 || fused > 1) return fail(QGD_ERR_INVALID, "fused must be -1, 0 or 1");
-  if (l2_ahead < -1 || l2_ahead > kMaxL2Ahead)
-    return fail(QGD_ERR_INVALID, "l2_ahead must be -1 or 0..%d", kMaxL2Ahead);
   std::lock_guard<std::mutex> lk(g_mu);
   g_override[fmt].fused = fused;
-  g_override[fmt].l2_ahead = l2_ahead;
   return QGD_OK;
 }
 
@@ -731,7 +751,7 @@ qgd_status qlinear_fp8_dynamic_noalloc(const void* xq, const float* sx, const vo
 }
 
 size_t qgd_workspace_size(int fmt, int M, int N, int K) {
-  if (fmt < 0 || fmt > 2 || M <= 0 || N <= 0 || K <= 0) return 0;
+  if (fmt < 0 || fmt >= kNumFmts || M <= 0 || N <= 0 || K <= 0) return 0;
   return make_exec(fmt, make_plan(fmt, M, N, K), M, N, K).total;
 }
 
@@ -752,11 +772,11 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (!(ls >> fmt_s)) continue;  // blank line
     if (!(ls >> N >> K >> Mb >> var_s >> split >> red_s >> stages >> tile_n >> sch_s >> occ))
       return fail(QGD_ERR_TABLE,
-                  "%s:%d: expected 11 to 14 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
-                  "occupancy [k_slices [fused [l2_ahead]]]",
+                  "%s:%d: expected 11 to 13 fields: fmt N K M_bucket variant split_k reduce stages tile_n schedule "
+                  "occupancy [k_slices [fused]]",
                   path, lineno);
     std::string extra;
-    int fused = 0, l2a = 0;
+    int fused = 0;
     if (ls >> extra) {
       char* end = nullptr;
       const long v = strtol(extra.c_str(), &end, 10);
@@ -766,13 +786,7 @@ qgd_status qgd_load_dispatch_table(const char* path) {
         const long f = strtol(extra.c_str(), &end, 10);
         if (*end != '\0' || f < 0 || f > 1) return fail(QGD_ERR_TABLE, "%s:%d: bad fused '%s'", path, lineno, extra.c_str());
         fused = static_cast<int>(f);
-        if (ls >> extra) {
-          const long a2 = strtol(extra.c_str(), &end, 10);
-          if (*end != '\0' || a2 < 0 || a2 > kMaxL2Ahead)
-            return fail(QGD_ERR_TABLE, "%s:%d: bad l2_ahead '%s'", path, lineno, extra.c_str());
-          l2a = static_cast<int>(a2);
-          if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
-        }
+        if (ls >> extra) return fail(QGD_ERR_TABLE, "%s:%d: trailing field '%s'", path, lineno, extra.c_str());
       }
     }
     const int fmt = fmt_from_name(fmt_s), var = variant_from_name(var_s), red = reduce_from_name(red_s);
@@ -786,7 +800,7 @@ qgd_status qgd_load_dispatch_table(const char* path) {
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
         occ > 2)
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
-    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ, kslices, fused, l2a};
+    t[Key(fmt, N, K, Mb)] = Entry{var, split, red, stages, tile_n, sch, occ, kslices, fused};
   }
   std::lock_guard<std::mutex> lk(g_mu);
   g_table.swap(t);
@@ -801,7 +815,7 @@ qgd_status qgd_clear_dispatch_table(void) {
 
 qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule,
                             int occupancy, int k_slices) {
-  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (variant > 1 || reduce > 3 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
       occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
@@ -822,7 +836,7 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
 
 qgd_status qgd_get_plan(int fmt, int M, int N, int K, qgd_plan* plan) {
   if (!plan) return fail(QGD_ERR_INVALID, "null plan");
-  if (fmt < 0 || fmt > 2) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
   if (M < 0 || N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "bad sizes");
   *plan = make_plan(fmt, M < 1 ? 1 : M, N, K);
   return QGD_OK;

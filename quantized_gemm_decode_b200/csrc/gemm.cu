@@ -143,8 +143,8 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 // Accumulator word (fp32 bits, or int32 for INT8) -> final fp32 value.
 template <int kFmt>
 __device__ __forceinline__ float scale_out(uint32_t accbits, int m, int n, const GemmArgs& a) {
-  if constexpr (kFmt == kFmtBlock) {
-    return __uint_as_float(accbits);  // scales were applied per K block
+  if constexpr (kFmt == kFmtBlock || kFmt == kFmtMX) {
+    return __uint_as_float(accbits);  // scales were applied per K block (MXFP8: by the tensor core)
   } else if constexpr (kFmt == kFmtINT8) {
     return (static_cast<float>(static_cast<int32_t>(accbits)) * __ldg(a.sx + m)) * __ldg(a.sw + n);
   } else {
@@ -188,7 +188,7 @@ __device__ __forceinline__ void store_swap_final(uint32_t accbits, int m, int n,
   const size_t idx = static_cast<size_t>(m) * a.N + n;
   if (a.raw) {
     static_cast<uint32_t*>(a.raw)[idx] = accbits;
-  } else if constexpr (kFmt == kFmtBlock) {
+  } else if constexpr (kFmt == kFmtBlock || kFmt == kFmtMX) {
     a.y[idx] = bf16_bits(__uint_as_float(accbits));
   } else if constexpr (kFmt == kFmtINT8) {
     a.y[idx] = bf16_bits((static_cast<float>(static_cast<int32_t>(accbits)) * sx_s[m]) * swv);
@@ -463,11 +463,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
                   const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
+  // MXFP8: the tensor core applies the E8M0 block scales, which the epilogue
+  // warps write into tensor memory stage by stage
+  constexpr bool kMX = (kFmt == kFmtMX);
   // Block_FP8: a ring of per-K-block accumulators; otherwise one accumulator
   // per segment, double-buffered so the next segment's MMAs overlap the drain.
   constexpr int kSlots = kBlock ? 4 : 2;
   constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : (kSlots * kMpad <= 128 ? 128 : 256));
   static_assert(!kBlock || kMpad <= 32, "Block_FP8 Swap-AB covers at most 32 tokens");
+  static_assert(!(kMX && kFused), "MXFP8 takes quantized activations");
+  // MXFP8 scale-factor columns per ring slot: a 4-column group for the
+  // weights (lane quadrant q reads column q), then one for the tokens (token m
+  // in lane m % 32 of every quadrant, column m / 32; kSFB columns used)
+  constexpr uint32_t kSFB = kMpad > 32 ? kMpad / 32 : 1;
+  constexpr uint32_t kSFSlot = kMxSlotCols;
+  static_assert(kSFB <= 4, "token scales fit one 4-column group");
   // the epilogue walks the accumulator row in chunks of at most 32 token columns
   constexpr int kAcc = kMpad > 32 ? 32 : kMpad;
   constexpr int kChunks = kMpad / kAcc;
@@ -507,6 +517,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     ue = t0 + static_cast<long long>(blockIdx.y + 1) * nku / a.splits;
   }
   const int nk = static_cast<int>(ue - ub);
+  const uint32_t ncols = kMX ? mx_tmem_cols(kMpad, stages, kps) : kCols;
   if (threadIdx.x == 0) QGD_STAMP(0);
 
   if (warp == 0 && lane == 0) {
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, kCols);
+    tmem_alloc(&ctl->tmem_base, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -554,16 +565,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       // (fused: the stage's activation half is written by the epilogue warps)
       const uint32_t x_tx = kFused ? 0u : kXBytes;
       const int pre = nk < stages ? nk : stages;
-      // L2 run-ahead: the weight tiles of units [pre, pre + l2_ahead) go to L2
-      // now and each later unit's as the ring advances, so more of the stream
-      // is in flight than the shared-memory ring can hold
-      auto prefetch_unit = [&](int i) {
-        const long long u = ub + i;
-        const int k0 = static_cast<int>(u % nku) * kps;
-        const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
-        for (int j = 0; j < ns; ++j) tma_prefetch_2d(&tw, (k0 + j) * kTileK, static_cast<int>(u / nku) * kSwapTileN);
-      };
-      const int ahead = a.l2_ahead;
       for (int i = 0; i < pre; ++i) {
         const long long u = ub + i;
         const int k0 = static_cast<int>(u % nku) * kps;   // first K slice of the unit
@@ -573,7 +574,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           tma_load_2d(w_ring + i * stage_w + j * kWBytes, &tw, &ctl->full[i], (k0 + j) * kTileK,
                       static_cast<int>(u / nku) * kSwapTileN, pol_w);
       }
-      for (int i = pre; i < nk && i < pre + ahead; ++i) prefetch_unit(i);
       QGD_STAMP(13);
       if (!kFused) {
         griddep_wait();
@@ -607,12 +607,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
             tma_load_2d(x_ring + s * stage_x + j * kXBytes, &tx, &ctl->full[s], (k0 + j) * kTileK, 0, pol_x);
         }
         issued = i + 1;
-        if (ahead > 0 && i + ahead < nk) prefetch_unit(i + ahead);
       }
-      // every load of this CTA is in flight: warm L2 with its share of the
-      // next layer's weights, so HBM keeps streaming through this layer's
-      // tail and the next layer's start
-      if (a.pf_bytes && issued == nk) prefetch_share_l2(a.pf, a.pf_bytes);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -624,7 +619,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       for (int i = 0; i < nk && !stop; ++i) {
         const int s = i % stages;
         const uint32_t round = i / stages;
-        if (!mbar_wait(&ctl->full[s], round & 1) || (kFused && !mbar_wait(&ctl->xfull[s], round & 1))) {
+        if (!mbar_wait(&ctl->full[s], round & 1) ||
+            ((kFused || kMX) && !mbar_wait(&ctl->xfull[s], round & 1))) {
           record_error(kErrWaitMma);
           ctl->abort_flag = 1;
           break;
@@ -655,12 +651,28 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           }
           tc_fence_after();
           const uint32_t d = tmem + slot * kMpad;
+          // MXFP8: this slot's scale-factor columns.  Both groups start on a
+          // multiple of 4 columns (by construction; checked, so that a mistake
+          // aborts the CTA instead of faulting)
+          const uint32_t sfa = tmem + 2 * kMpad + static_cast<uint32_t>(s * kps + j) * kSFSlot;
+          if (kMX && (sfa & 3u) != 0u) {
+            record_error(kErrBadOperand);
+            ctl->abort_flag = 1;
+            stop = true;
+            break;
+          }
 #pragma unroll
           for (int kk = 0; kk < kTileK / 32; ++kk) {
             const uint64_t ad = sdesc_kmajor_sw128(w_base + s * stage_w + j * kWBytes + kk * 32);
             const uint64_t bd = sdesc_kmajor_sw128(x_base + s * stage_x + j * kXBytes + kk * 32);
             const uint32_t accumulate = kBlock ? (kk > 0) : !(seg_start && j == 0 && kk == 0);
-            mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+            if constexpr (kMX) {
+              const uint32_t sel = static_cast<uint32_t>(kk) << 30;  // the 32-wide K block's byte
+              mma_issue_mx(d, ad, bd, idesc_mx(kSwapTileN, kMpad, kk, kk), sfa | sel, (sfa + 4) | sel,
+                           accumulate);
+            } else {
+              mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+            }
           }
           if (kBlock) {
             if (!a.withhold_acc) mma_commit(&ctl->tfull[slot]);
@@ -686,7 +698,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int M = a.M, N = a.N;
     const int KB = a.K / kTileK;
     const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
-    const bool scaled = (kFmt != kFmtBlock) && !a.raw;
+    const bool scaled = (kFmt != kFmtBlock) && !kMX && !a.raw;
     const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 among the epilogue threads
     if constexpr (kFused && !kBlock) {
       // per-token scales: every CTA takes each row's maximum over all of K
@@ -733,7 +745,49 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     int qnext = 0, qslice = 0;
     bool qdead = false;
     auto quant_until = [&](int limit) {
-      if constexpr (kFused) {
+      if constexpr (kMX) {
+        // MXFP8: write each stage's block scales into its tensor-memory slot
+        // once the MMA has released the stage (its empty barrier)
+        if (limit > nk) limit = nk;
+        const int KB32 = a.K / 32;
+        for (; qnext < limit && !qdead; ++qnext) {
+          const int s = qnext % stages;
+          const uint32_t round = qnext / stages;
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag) || !warp_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+            if (lane == 0) {
+              record_error(kErrWaitEpilogue);
+              ctl->abort_flag = 1;
+            }
+            qdead = true;
+            break;
+          }
+          const long long u = ub + qnext;
+          const int t = static_cast<int>(u / nku);
+          const int k0 = static_cast<int>(u % nku) * kps;
+          const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+          tc_fence_after();
+          for (int j = 0; j < ns; ++j) {
+            const uint32_t col = 2 * kMpad + static_cast<uint32_t>(s * kps + j) * kSFSlot;
+            const uint32_t lanes = static_cast<uint32_t>(q * 32) << 16;
+            // weight rows of this lane quadrant: 4 E8M0 bytes (the 128-wide K slice) per row
+            const int n = t * kSwapTileN + q * 32 + lane;
+            const uint32_t wsf = n < N ? __ldg(reinterpret_cast<const unsigned*>(a.sw8 + static_cast<size_t>(n) * KB32) + (k0 + j))
+                                       : 0u;
+            tmem_st32(tmem + lanes + col + q, wsf);
+#pragma unroll
+            for (uint32_t w = 0; w < kSFB; ++w) {
+              const int m = static_cast<int>(w) * 32 + lane;
+              const uint32_t xsf =
+                  m < M ? __ldg(reinterpret_cast<const unsigned*>(a.sx8 + static_cast<size_t>(m) * KB32) + (k0 + j)) : 0u;
+              tmem_st32(tmem + lanes + col + 4 + w, xsf);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->xfull[s]);
+        }
+      } else if constexpr (kFused) {
         if (limit > nk) limit = nk;
         for (; qnext < limit && !qdead; ++qnext) {
           const int s = qnext % stages;
@@ -1014,7 +1068,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     if (threadIdx.x == 64) QGD_STAMP(6);
   }
 
-  teardown(ctl, warp, lane, issued, stages, tmem, kCols);
+  teardown(ctl, warp, lane, issued, stages, tmem, ncols);
   if (threadIdx.x == 32) QGD_STAMP(7);
 }
 
@@ -1574,6 +1628,15 @@ static cudaError_t launch_swapab_f(int fmt, int mpad, const CUtensorMap& tw, con
     switch (mpad) {
       case 16: return launch_swapab_t<kFmtBlock, 16, kFused>(tw, tx, a, stream);
       case 32: return launch_swapab_t<kFmtBlock, 32, kFused>(tw, tx, a, stream);
+    }
+  } else if (fmt == kFmtMX) {
+    if constexpr (!kFused) {
+      switch (mpad) {
+        case 16: return launch_swapab_t<kFmtMX, 16, false>(tw, tx, a, stream);
+        case 32: return launch_swapab_t<kFmtMX, 32, false>(tw, tx, a, stream);
+        case 64: return launch_swapab_t<kFmtMX, 64, false>(tw, tx, a, stream);
+        case 128: return launch_swapab_t<kFmtMX, 128, false>(tw, tx, a, stream);
+      }
     }
   }
   return cudaErrorInvalidValue;

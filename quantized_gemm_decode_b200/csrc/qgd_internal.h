@@ -8,7 +8,8 @@
 
 namespace qgd {
 
-enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2 };
+enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2, kFmtMX = 3 };
+constexpr int kNumFmts = 4;
 enum Variant : int { kStandard = 0, kSwapAB = 1 };
 enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2, kCluster = 3 };
 constexpr int kMaxClusterSplit = 8;  // portable thread-block cluster size
@@ -52,12 +53,23 @@ struct GemmArgs {
   int ldxb;
   uint8_t* xq_out;      // test capture (may be null): the codes [M][K] the kernel made
   float* sx_out;        // test capture (may be null): their scales, [M] or [M][K/128]
-  // L2 warm-up of the next layer's weights: once a CTA has issued all of its
-  // own loads it prefetches its share of [pf, pf + pf_bytes) into L2
-  const uint8_t* pf;
-  size_t pf_bytes;
-  int l2_ahead;  // Swap-AB: weight units prefetched into L2 ahead of the shared-memory ring
+  // MXFP8: E8M0 block-scale bytes, one per 32 values along K
+  const uint8_t* sx8;  // [M][K/32]
+  const uint8_t* sw8;  // [N][K/32]
 };
+
+// Tensor-memory columns of the MXFP8 Swap-AB kernel: two accumulators of mpad
+// columns, then per ring slot (stage, K slice) a group of 4 columns of weight
+// scales and a group of 4 of token scales (a scale-factor operand spans a
+// 4-column, 128-bit group and starts on a multiple of 4); rounded up to a
+// power of two.
+constexpr unsigned kMxSlotCols = 8;
+__host__ __device__ inline unsigned mx_tmem_cols(int mpad, int stages, int kps) {
+  const unsigned need = 2u * mpad + static_cast<unsigned>(stages * kps) * kMxSlotCols;
+  unsigned c = 32;
+  while (c < need) c *= 2;
+  return c;
+}
 
 // Launchers (gemm.cu).  Each returns the cudaError_t of the launch.
 // fused: the kernel quantizes a.xbf itself (tx unused)
@@ -87,5 +99,8 @@ cudaError_t launch_quant_rows(const uint16_t* x, int rows, int K, int ldx, int q
 cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, int ldx, uint8_t* q, float* s,
                                   cudaStream_t stream);
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream);
+// MXFP8: rows of 32-value blocks -> e4m3 codes q [rows][K], E8M0 bytes s [rows][K/32]
+cudaError_t launch_quant_mx(const uint16_t* x, int rows, int K, int ldx, uint8_t* q, uint8_t* s,
+                            cudaStream_t stream);
 
 }  // namespace qgd

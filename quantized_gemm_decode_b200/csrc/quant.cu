@@ -103,6 +103,32 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const uint16_t* __r
 }
 
 // ---------------------------------------------------------------------------
+// MXFP8 blocks of 32 along a row: four lanes per block, 8 values per lane.
+// x rows are ldx elements apart; q [rows][K] codes, s [rows][K/32] E8M0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_mx_kernel(const uint16_t* __restrict__ x, int rows, int K, int ldx,
+                                                       uint8_t* __restrict__ q, uint8_t* __restrict__ s) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
+  const int KB = K / 32;
+  const long long b = static_cast<long long>(blockIdx.x) * 64 + (threadIdx.x >> 2);  // block index (row, kb)
+  const int sub = threadIdx.x & 3;
+  const bool valid = b < static_cast<long long>(rows) * KB;
+  const long long bb = valid ? b : 0;
+  const long long r = bb / KB, kb = bb % KB;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (valid) v = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * ldx + kb * 32 + sub * 8));
+  float amax = absmax8(v);
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  const int e = mx_block_exp(amax);
+  if (valid) {
+    *reinterpret_cast<uint2*>(q + static_cast<size_t>(r) * K + kb * 32 + sub * 8) = encode8_mx(v, mx_inv_scale(e));
+    if (sub == 0) s[static_cast<size_t>(r) * KB + kb] = static_cast<uint8_t>(e + 127);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 128x128 weight blocks: one CTA of 256 threads per block, 8 vectors each.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_block128_kernel(const uint16_t* __restrict__ w, int K,
@@ -178,6 +204,13 @@ cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, int ldx, uint
   const long long groups = static_cast<long long>(M) * (K / 128);
   const unsigned blocks = static_cast<unsigned>((groups + 15) / 16);
   return launch_q(quant_group128_kernel, dim3(blocks), dim3(256), stream, x, M, K, ldx, q, s);
+}
+
+cudaError_t launch_quant_mx(const uint16_t* x, int rows, int K, int ldx, uint8_t* q, uint8_t* s,
+                            cudaStream_t stream) {
+  const long long blocks = static_cast<long long>(rows) * (K / 32);
+  const unsigned grid = static_cast<unsigned>((blocks + 63) / 64);
+  return launch_q(quant_mx_kernel, dim3(grid), dim3(256), stream, x, rows, K, ldx, q, s);
 }
 
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream) {

@@ -60,6 +60,33 @@ __device__ __forceinline__ uint2 encode8(const uint4& v, float s) {
   return out;
 }
 
+// MXFP8 (OCP Microscaling v1.0): a 32-value block shares the scale 2^e,
+// e = floor(log2(amax)) - 8 clamped to [-127, 127] (8: the exponent of
+// e4m3's largest normal, 448 = 1.75 * 2^8), stored as the E8M0 byte e + 127;
+// an all-zero block takes e = -127.  Codes are e4m3(v * 2^-e), round to
+// nearest even, saturating: multiplying by a power of two is exact.
+__device__ __forceinline__ int mx_block_exp(float amax) {
+  if (amax == 0.f) return -127;
+  const uint32_t bits = __float_as_uint(amax);
+  const int ef = static_cast<int>((bits >> 23) & 0xFFu);
+  const int fl = ef ? ef - 127 : (31 - __clz(static_cast<int>(bits & 0x7FFFFFu))) - 149;  // floor(log2(amax))
+  const int e = fl - 8;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^-e as an fp32 (exact; 2^-127 is subnormal).
+__device__ __forceinline__ float mx_inv_scale(int e) {
+  return e >= 127 ? __uint_as_float(0x00400000u) : __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+// 8 bf16 values * inv -> 8 e4m3 codes.
+__device__ __forceinline__ uint2 encode8_mx(const uint4& v, float inv) {
+  uint2 out;
+  out.x = e4m3x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv) | (e4m3x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv) << 16);
+  out.y = e4m3x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv) | (e4m3x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv) << 16);
+  return out;
+}
+
 // Maximum over the 32 lanes of a warp.
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

@@ -21,6 +21,7 @@ enum : unsigned int {
   kErrWaitMma = 2,        // MMA issuer gave up waiting for a filled stage / TMEM slot
   kErrWaitEpilogue = 3,   // epilogue gave up waiting for the accumulator
   kErrWaitDrain = 4,      // teardown gave up waiting for copies or MMAs in flight
+  kErrBadOperand = 5,     // an operand address failed its alignment check; the MMA was skipped
 };
 
 // Wait budget: about one second of wall time (globaltimer is in ns).
@@ -159,37 +160,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Bring [p, p + bytes) into L2 (no shared memory, no completion to wait
-// for).  p 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
-// This CTA's share of an L2 warm-up range: the range is cut into equal
-// 16-byte-aligned pieces, one per CTA of the grid, issued 64 KB at a time.
-__device__ __forceinline__ void prefetch_share_l2(const uint8_t* base, size_t bytes) {
-  const size_t ncta = static_cast<size_t>(gridDim.x) * gridDim.y * gridDim.z;
-  const size_t cid = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-  const size_t total = bytes & ~static_cast<size_t>(15);
-  const size_t share = ((total + ncta - 1) / ncta + 15) & ~static_cast<size_t>(15);
-  const size_t b0 = cid * share;
-  const size_t b1 = b0 + share < total ? b0 + share : total;
-  for (size_t b = b0; b < b1; b += 65536) {
-    const size_t n = b1 - b < 65536 ? b1 - b : 65536;
-    prefetch_l2_bulk(base + b, static_cast<uint32_t>(n));
-  }
-}
-
-// Bring one TMA box of a tensor into L2 only (no shared memory, nothing to
-// wait for); coordinates as tma_load_2d.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -271,6 +241,36 @@ __device__ __forceinline__ void mma_issue(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
   }
 }
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale: e4m3 x
+// e4m3 -> f32, both K-major, E8M0 scale factors, K = 32 per instruction.
+// a_sf_id / b_sf_id pick the byte of the scale-factor word the instruction
+// reads (the 32-wide K block inside a 128-wide K slice).
+__host__ __device__ constexpr uint32_t idesc_mx(uint32_t m, uint32_t n, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4) | (0u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) |
+         (a_sf_id << 29);
+}
+
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T with E8M0 block scales read from tensor
+// memory: tsfa / tsfb are TMEM addresses whose top two bits carry the byte
+// id (the same as the descriptor's sf ids).
+__device__ __forceinline__ void mma_issue_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Each lane of a warp writes one 32-bit word into its TMEM lane (the warp's
+// lane quadrant) at the address's column.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {

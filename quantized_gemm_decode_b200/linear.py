@@ -55,14 +55,12 @@ class QuantizedLinear:
         self.ws.ensure(qgd.qgd_workspace_size(self.fmt_id, xq.shape[0], self.N, self.K))
         return fn(xq, sx, self.wq, self.sw, y=y, ws=self.ws)
 
-    def layer(self, x: torch.Tensor, y=None, next_layer: "QuantizedLinear | None" = None) -> torch.Tensor:
+    def layer(self, x: torch.Tensor, y=None) -> torch.Tensor:
         """The whole layer call from bf16 x (possibly a column slice of a
         wider matrix): quantization and GEMM, fused into one kernel when the
-        layer plan says so.  With `next_layer`, its weight codes are warmed
-        in L2 while this call finishes."""
+        layer plan says so."""
         self.ws.ensure(qgd.qgd_layer_workspace_size(self.fmt_id, x.shape[0], self.N, self.K))
-        return qgd.qlinear_bf16(self.fmt_id, x, self.wq, self.sw, y=y, ws=self.ws,
-                                next_w=None if next_layer is None else next_layer.wq)
+        return qgd.qlinear_bf16(self.fmt_id, x, self.wq, self.sw, y=y, ws=self.ws)
 
     def forward_eager(self, x: torch.Tensor, y=None) -> torch.Tensor:
         return self.layer(x, y=y)
@@ -178,7 +176,7 @@ class DecodeStep:
         for i, (layer, M) in enumerate(self.calls):
             if i % self.join_every == 0:
                 main.wait_event(landed[i // self.join_every])
-            layer.layer(self.x_dev[i], self.y_dev[i], next_layer=self.calls[(i + 1) % n][0])
+            layer.layer(self.x_dev[i], self.y_dev[i])
             # results leave in groups too: one fork from the compute stream per group
             if (i + 1) % self.out_every == 0 or i == n - 1:
                 done = torch.cuda.Event()
@@ -230,16 +228,6 @@ class DecodeChain:
                 raise ValueError(f"layer {i}: input of {cols} columns from source {src} does not fit")
         self._bufs: dict = {}
         self._graphs: dict = {}
-        # each layer warms the next one's weights in L2; the last one warms
-        # the layer that runs after the chain (by default its own first)
-        self.successor: QuantizedLinear | None = self.layers[0]
-
-    def then(self, layer) -> None:
-        """The layer whose weights the chain's last layer warms in L2 (for
-        example the first layer of the next decoder block); None for none.
-        Takes effect at the next capture."""
-        self.successor = layer
-        self._graphs.clear()
 
     def _buffers(self, M: int):
         if M not in self._bufs:
@@ -259,8 +247,7 @@ class DecodeChain:
     def _body(self, M: int):
         _, ys = self._buffers(M)
         for i, layer in enumerate(self.layers):
-            nxt = self.layers[i + 1] if i + 1 < len(self.layers) else self.successor
-            layer.layer(self._input(M, i), ys[i], next_layer=nxt)
+            layer.layer(self._input(M, i), ys[i])
 
     def capture(self, M: int) -> None:
         self._buffers(M)

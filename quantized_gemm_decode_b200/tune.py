@@ -34,10 +34,10 @@ import torch
 
 import quantized_gemm_decode_b200 as qgd
 from quantized_gemm_decode_b200 import synth, workloads
-from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, W8A8_INT8
 
 L2_BYTES = 126 * 1024 * 1024
-FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}
+FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}
 VAR_NAME = {0: "standard", 1: "swap_ab"}
 RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
 
@@ -45,12 +45,16 @@ RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
 def _quant_w(fmt, w):
     if fmt == BLOCK_FP8:
         return qgd.quant_weight_block128(w)
+    if fmt == MXFP8:
+        return qgd.quant_mx(w)
     return qgd.quant_weight_per_channel(w, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
 
 
 def _quant_x(fmt, x):
     if fmt == BLOCK_FP8:
         return qgd.quant_act_group128(x)
+    if fmt == MXFP8:
+        return qgd.quant_mx(x)
     return qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
 
 
@@ -86,6 +90,9 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148, fused: bool
     SM; a Swap-AB grid of at most one CTA per SM is tried at the deepest ring and at that shallower
     one (which leaves room for the next layer's CTAs to start streaming beside it).  At decode token
     counts every Swap-AB candidate is also tried with the activation quantizer fused in."""
+    if fmt == MXFP8:
+        # the Swap-AB kernel only, no two-pass reduction, no fused quantizer
+        return [c + (0,) for c in _candidates(fmt, M, N, K, num_sms, False) if c[0] == 1 and c[2] != 1]
     if fused and M <= 32:
         # the fused quantizer has no two-pass reduction (it would need the scales in memory)
         base = _candidates(fmt, M, N, K, num_sms, False)
@@ -159,7 +166,7 @@ class Problem:
         self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         self.ws = qgd.Workspace(0, device)
         self.fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
-                   BLOCK_FP8: qgd.qlinear_block_fp8}[fmt]
+                   BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8}[fmt]
 
     def run(self, j=0):
         wq, sw = self.copies[j % len(self.copies)]
@@ -167,11 +174,12 @@ class Problem:
 
     def layer_call(self, j=0):
         """What the layer runs per call: the layer call from bf16 activations
-        (quantizer kernel + GEMM, or one fused kernel, as the layer plan says),
-        warming the next call's weights in L2 as a decode step does."""
+        (quantizer kernel + GEMM, or one fused kernel, as the layer plan says)."""
         wq, sw = self.copies[j % len(self.copies)]
-        nxt = self.copies[(j + 1) % len(self.copies)][0]
-        return qgd.qlinear_bf16(self.fid, self.x, wq, sw, y=self.y, ws=self.ws, next_w=nxt)
+        if self.fmt == MXFP8:  # no layer call: the quantizer kernel, then the GEMM
+            qgd.quant_mx(self.x, xq=self.xq, sx=self.sx)
+            return self.run(j)
+        return qgd.qlinear_bf16(self.fid, self.x, wq, sw, y=self.y, ws=self.ws)
 
     def acc32(self):
         return qgd.qgd_w8a8_int8_acc32(self.xq, self.copies[0][0], ws=self.ws)
@@ -208,12 +216,11 @@ class Problem:
 
 
 def tune_problem(p: Problem, log=None):
-    """Time every candidate (L2 run-ahead off), then refine the three fastest:
-    their ring depth, and for Swap-AB their L2 run-ahead.  Returns the best
-    (us, variant, split_k, reduce, stages, tile_n, schedule, occupancy,
-    k_slices, fused, l2_ahead) and the first pass's results."""
+    """Time every candidate, then the ring depth of the three fastest.
+    Returns the best (us, variant, split_k, reduce, stages, tile_n, schedule,
+    occupancy, k_slices, fused) and the first pass's results."""
     fid = p.fid
-    qgd.qgd_set_override_ext(fid, 0, 0)
+    qgd.qgd_set_fused_override(fid, 0)
     qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0,
                          qgd.SCHEDULE_GRID, 0, 1)
     p.ws.ensure(qgd.qgd_workspace_size(fid, p.M, p.N, p.K))
@@ -227,18 +234,17 @@ def tune_problem(p: Problem, log=None):
         p.ws.ensure(max(qgd.qgd_workspace_size(fid, p.M, p.N, p.K),
                         qgd.qgd_layer_workspace_size(fid, p.M, p.N, p.K)))
 
-    def timed(var, s, r, st, t, sch, occ, kps, fz, l2a):
+    def timed(var, s, r, st, t, sch, occ, kps, fz):
         qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
-        qgd.qgd_set_override_ext(fid, fz, l2a)
+        qgd.qgd_set_fused_override(fid, fz)
         ensure_ws()
         us = p.time_plan()
         pl = qgd.qgd_get_layer_plan(fid, p.M, p.N, p.K)
-        return (us, var, pl["split_k"], r, pl["stages"], t, sch, pl["occupancy"], pl["k_slices"], pl["fused"],
-                pl["l2_ahead"])
+        return (us, var, pl["split_k"], r, pl["stages"], t, sch, pl["occupancy"], pl["k_slices"], pl["fused"])
 
     for var, s, r, t, sch, occ, kps, st0, fz in candidates(p.fmt, p.M, p.N, p.K, num_sms):
         qgd.qgd_set_override(fid, var, s, r, st0, t, sch, occ, kps)
-        qgd.qgd_set_override_ext(fid, fz, 0)
+        qgd.qgd_set_fused_override(fid, fz)
         ensure_ws()
         y = p.layer_call().float()
         ok = (y - ref).abs().max().item() <= 2e-2 * scale
@@ -250,25 +256,22 @@ def tune_problem(p: Problem, log=None):
                 log(f"  reject {VAR_NAME[var]} s={s} r={RED_NAME[r]} t={t} {SCHED_NAME[sch]} occ={occ} "
                     f"kps={kps} fused={fz}: differs from the split-free result")
             continue
-        results.append(timed(var, s, r, st0, t, sch, occ, kps, fz, 0))
+        results.append(timed(var, s, r, st0, t, sch, occ, kps, fz))
     results.sort()
     refined = list(results[:3])
-    for us0, var, s, r, smax, t, sch, occ, kps, fz, _ in results[:3]:
+    for us0, var, s, r, smax, t, sch, occ, kps, fz in results[:3]:
         for st in (2, 3, 4, 5, 6, 8, 10):  # shallower rings
             if st < smax:
-                refined.append(timed(var, s, r, st, t, sch, occ, kps, fz, 0))
-        if var == qgd.VARIANT_SWAP_AB:  # L2 run-ahead
-            for l2a in (2, 4, 8, 16):
-                refined.append(timed(var, s, r, smax, t, sch, occ, kps, fz, l2a))
+                refined.append(timed(var, s, r, st, t, sch, occ, kps, fz))
     refined.sort()
     qgd.qgd_set_override(fid)
-    qgd.qgd_set_override_ext(fid, -1, -1)
+    qgd.qgd_set_fused_override(fid)
     return refined[0], results
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--formats", default="fp8_dynamic,w8a8_int8,block_fp8")
+    ap.add_argument("--formats", default="fp8_dynamic,w8a8_int8,block_fp8,mxfp8")
     ap.add_argument("--out", default=qgd.DEFAULT_TABLE)
     ap.add_argument("--large-m", action="store_true", help="also tune the larger-M buckets")
     ap.add_argument("--resume", action="store_true")
@@ -280,14 +283,15 @@ def main(argv=None):
     qgd.qgd_clear_dispatch_table()
     device = torch.device("cuda")
     fmts = args.formats.split(",")
-    wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE) if w.fmt in fmts]
+    wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE)
+           if w.fmt in fmts]
     if args.large_m:
         wls += [w for w in workloads.LARGE if w.fmt in fmts]
     done = {}
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
             f = ln.split("#")[0].split()
-            if len(f) in (11, 12, 13, 14):
+            if len(f) in (11, 12, 13):
                 done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
     only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
     t_start = time.time()
@@ -300,8 +304,8 @@ def main(argv=None):
         tmp = args.out + ".tmp"
         with open(tmp, "w") as f:
             f.write("# Dispatch table for B200 (sm_100a), measured by quantized_gemm_decode_b200.tune\n")
-            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy k_slices fused "
-                    "l2_ahead   # us per layer call (quantize + GEMM)\n")
+            f.write("# fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy k_slices fused"
+                    "   # us per layer call (quantize + GEMM)\n")
             for k in sorted(lines):
                 f.write(lines[k] + "\n")
         os.replace(tmp, args.out)
@@ -317,12 +321,12 @@ def main(argv=None):
                 t0 = time.time()
                 p = Problem(wl.fmt, M, N, K, wl.seed, device)
                 best, allres = tune_problem(p, log)
-                us, var, s, r, st, t, sch, occ, kps, fz, l2a = best
+                us, var, s, r, st, t, sch, occ, kps, fz = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
                 lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "
-                              f"{occ} {kps} {fz} {l2a}   # {us:.2f} us, {gbs:.0f} GB/s")
+                              f"{occ} {kps} {fz}   # {us:.2f} us, {gbs:.0f} GB/s")
                 log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
-                    f"{SCHED_NAME[sch]} occ={occ} kps={kps} fused={fz} l2_ahead={l2a} {us:.2f} us {gbs:.0f} GB/s "
+                    f"{SCHED_NAME[sch]} occ={occ} kps={kps} fused={fz} {us:.2f} us {gbs:.0f} GB/s "
                     f"({len(allres)} candidates, {time.time() - t0:.1f} s)")
                 del p
                 torch.cuda.empty_cache()

@@ -11,7 +11,8 @@ from dataclasses import dataclass, field
 FP8_DYNAMIC = "fp8_dynamic"
 W8A8_INT8 = "w8a8_int8"
 BLOCK_FP8 = "block_fp8"
-FORMATS = (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)
+MXFP8 = "mxfp8"
+FORMATS = (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)  # the three formats of the method; MXFP8 is the Blackwell addition
 
 DECODE_M = (1, 2, 4, 8, 16, 24, 32)
 LARGE_M = (64, 128, 512, 2048, 8192)
@@ -46,12 +47,15 @@ INT8_DECODE = Workload("w8a8_int8_decode_sweep_14b_shapes", W8A8_INT8, SHAPES_14
                        "W8A8_INT8, 14B-class shapes x M in 1..32")
 BLOCK_DECODE = Workload("block_fp8_decode_sweep_32b_shapes", BLOCK_FP8, SHAPES_32B, DECODE_M, 1003, True,
                         "Block_FP8, 32B-class shapes x M in 1..32, 1% x20 outlier channels")
+MX_DECODE = Workload("mxfp8_decode_sweep_8b_shapes", MXFP8, SHAPES_8B, DECODE_M, 1005, True,
+                     "MXFP8 (E8M0 scales per 32 values along K), 8B-class shapes x M in 1..32, "
+                     "1% x20 outlier channels")
 LARGE = tuple(
     Workload(f"{fmt}_large_m_8b_shapes", fmt, SHAPES_8B, LARGE_M, 1004, fmt != W8A8_INT8,
              f"{fmt}, 8B-class shapes x M in 64..8192")
     for fmt in FORMATS)
 
-ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE) + LARGE
+ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE, MX_DECODE) + LARGE
 
 
 def algorithmic_bytes(fmt: str, M: int, N: int, K: int) -> int:
@@ -59,6 +63,8 @@ def algorithmic_bytes(fmt: str, M: int, N: int, K: int) -> int:
     codes, fp32 scales, bf16 output."""
     if fmt == BLOCK_FP8:
         scales = 4 * (N // 128) * (K // 128) + 4 * M * (K // 128)
+    elif fmt == MXFP8:
+        scales = N * (K // 32) + M * (K // 32)  # one E8M0 byte per 32 values
     else:
         scales = 4 * N + 4 * M
     return N * K + M * K + scales + 2 * M * N

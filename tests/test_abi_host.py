@@ -323,7 +323,8 @@ def test_table_cluster_reduce_name(tmp_path):
 @pytest.mark.parametrize("fmt,M,N,K", [("fp8_dynamic", 1, 4096, 4096), ("w8a8_int8", 16, 34816, 5120),
                                        ("block_fp8", 32, 5120, 25600), ("fp8_dynamic", 512, 6144, 4096),
                                        ("fp8_dynamic", 64, 24576, 4096), ("w8a8_int8", 128, 4096, 12288),
-                                       ("block_fp8", 64, 6144, 4096)])
+                                       ("block_fp8", 64, 6144, 4096), ("mxfp8", 16, 4096, 4096),
+                                       ("mxfp8", 64, 6144, 4096)])
 def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
     # every plan the tuner times is one the library runs as asked (no silent
     # legalization), and a grid-schedule Swap-AB candidate with more CTAs than
@@ -332,7 +333,8 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
 
     fid = tune.FMT_ID[fmt]
     cands = tune.candidates(fmt, M, N, K, 148)
-    assert any(c[8] for c in cands) == (M <= 32)  # fused candidates at decode token counts
+    # fused candidates at decode token counts (MXFP8 has no fused quantizer)
+    assert any(c[8] for c in cands) == (M <= 32 and fmt != "mxfp8")
     for var, s, r, t, sch, occ, kps, st, fz in cands:
         qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
         qgd.qgd_set_fused_override(fid, fz)
@@ -478,10 +480,10 @@ def test_strided_quantizer_rejects_bad_row_stride():
 def test_layer_call_rejects_bad_arguments():
     L = qgd.lib()
     P = ctypes.c_void_p
-    # misaligned warm-up range, row stride below K, null operands: refused before any launch
-    assert L.qlinear_fp8_dynamic_bf16(P(16), 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, P(17), 4096, None) == -1
-    assert L.qlinear_fp8_dynamic_bf16(P(16), 512, P(16), P(16), P(16), 4, 512, 1024, None, 0, None, 0, None) == -1
-    assert L.qlinear_w8a8_int8_bf16(None, 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, None, 0, None) == -1
-    assert L.qlinear_block_fp8_bf16(P(16), 1000, P(16), P(16), P(16), 4, 512, 1000, None, 0, None, 0, None) == -2
+    # row stride below K, misaligned x, null operands: refused before any launch
+    assert L.qlinear_fp8_dynamic_bf16(P(16), 512, P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
+    assert L.qlinear_fp8_dynamic_bf16(P(17), 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
+    assert L.qlinear_w8a8_int8_bf16(None, 1024, P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
+    assert L.qlinear_block_fp8_bf16(P(16), 1000, P(16), P(16), P(16), 4, 512, 1000, None, 0, None) == -2
     # an empty call is fine
-    assert L.qlinear_fp8_dynamic_bf16(None, 1024, None, None, None, 0, 512, 1024, None, 0, None, 0, None) == 0
+    assert L.qlinear_fp8_dynamic_bf16(None, 1024, None, None, None, 0, 512, 1024, None, 0, None) == 0

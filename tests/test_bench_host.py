@@ -17,6 +17,10 @@ def test_gemm_algorithmic_bytes():
     assert workloads.algorithmic_bytes(BLOCK_FP8, 8, 10240, 5120) == (
         10240 * 5120 + 8 * 5120 + 4 * (10240 // 128) * kb + 4 * 8 * kb + 2 * 8 * 10240)
     assert workloads.flops(8, 10240, 5120) == 2 * 8 * 10240 * 5120
+    # MXFP8: one E8M0 byte per 32 values of each operand row
+    assert workloads.algorithmic_bytes(workloads.MXFP8, 4, 4096, 4096) == (
+        4096 * 4096 + 4 * 4096 + 4096 * 128 + 4 * 128 + 2 * 4 * 4096)
+    assert bench.path_bytes(workloads.MXFP8, 4, 4096, 4096) == 4096 * 4096 + 2 * 4 * 4096 + 4096 * 128 + 2 * 4 * 4096
 
 
 def test_path_and_quantizer_bytes():

@@ -154,22 +154,6 @@ def test_layer_workspace_covers_the_unfused_path():
     case.check_output(y, yref, bound, "unfused layer call")
 
 
-@pytest.mark.parametrize("fused", [0, 1])
-def test_l2_warmup_changes_no_result(fused):
-    # the next layer's weights warmed in L2 are only a hint: same bits out
-    case = Case(FP8_DYNAMIC, 8, 4096, 4096, seed=13)
-    nxt = Case(FP8_DYNAMIC, 8, 6144, 4096, seed=14)
-    fid = FMT_ID[FP8_DYNAMIC]
-    qgd.qgd_set_fused_override(fid, fused)
-    y0 = qgd.qlinear_bf16(fid, case.xd, case.wq, case.sw)
-    y1 = qgd.qlinear_bf16(fid, case.xd, case.wq, case.sw, next_w=nxt.wq)
-    torch.cuda.synchronize()
-    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
-    yref, bound = case.oracle_gemm(*case.oracle_quant())
-    case.check_output(y1, yref, bound, "with L2 warm-up")
-    assert qgd.qgd_device_error() == 0
-
-
 def test_layer_calls_leave_the_counter_header_zero():
     # an unfused layer call whose GEMM needs no workspace still keeps its
     # activation codes out of the counter header, so a Split-K call sharing
