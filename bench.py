@@ -842,6 +842,68 @@ def run_case(args):
 
 
 # ---------------------------------------------------------------------------
+# markdown rendering of a detail record (python bench.py --report DETAIL.json)
+# ---------------------------------------------------------------------------
+def render_report(d: dict) -> str:
+    """Markdown tables of a full run's detail record: the headline, each
+    format's decode sweep, the FP8 per-call table, the larger-M results, the
+    Split-K reductions, the dependent chain and the CPU baseline."""
+    out = []
+    rf, e2e, clk = d.get("roofline", {}), d.get("e2e", {}), d.get("clocks", {})
+    out.append("| quantity | value |\n|---|---:|")
+    out.append(f"| {d['config']['workload']}: whole path (quantize + GEMM per call, one graph per step) | "
+               f"{d['value']:.0f} GB/s, {d['ms_per_step'] * 1e3:.0f} us per step |")
+    out.append(f"| of measured HBM copy peak ({rf.get('peak')} GB/s) / of 8 TB/s | "
+               f"{d.get('frac_of_hbm_peak', 0):.3f} / {d.get('frac_of_8tbs', 0):.3f} |")
+    out.append(f"| GEMM kernels alone (roofline.achieved, {rf.get('avg_launch_us')} us per launch) | "
+               f"{rf.get('achieved')} GB/s = {rf.get('frac')} of measured |")
+    out.append(f"| end to end (pinned host X in, Y out, inside the graph) | {e2e.get('value')} GB/s |")
+    out.append(f"| SM clock under load (max) / throttle reasons | {clk.get('sm_mhz')} ({clk.get('sm_max_mhz')}) MHz / "
+               f"{', '.join(clk.get('reasons') or []) or 'none'} |")
+    if "formats" in d:
+        out.append("\n| format | workload | step | whole path | of measured HBM | quantizer alone |\n"
+                   "|---|---|---:|---:|---:|---:|")
+        for f, v in d["formats"].items():
+            q = v.get("quantizer", {})
+            out.append(f"| {f} | {v.get('workload', '')} | {v['ms_per_step'] * 1e3:.0f} us | {v['gbs']:.0f} GB/s | "
+                       f"{v['frac']:.3f} | {q.get('us_per_call', '')} us/call |")
+    if "per_call" in d:
+        out.append("\nFP8_Dynamic per call (GEMM alone: mean / p90; layer call = quantizer + GEMM):\n")
+        out.append("| M | N x K | GEMM us | p90 | GB/s | of HBM | layer us | plan |\n|---:|---|---:|---:|---:|---:|---:|---|")
+        for r in d["per_call"]:
+            out.append(f"| {r['M']} | {r['N']} x {r['K']} | {r['us']} | {r['p90_us']} | {r['gbs']} | {r['frac']} | "
+                       f"{r['layer_us']} | {r['plan']} |")
+    if "large_m" in d:
+        out.append("\nLarger M (one GEMM per call; frac against 2 x bf16, frac_probe against the tcgen05 probe):\n")
+        out.append("| format | M | mean frac | mean frac_probe | best TFLOP/s |\n|---|---:|---:|---:|---:|")
+        for f, rows in d["large_m"].items():
+            for M in sorted({r["M"] for r in rows}):
+                rr = [r for r in rows if r["M"] == M]
+                fp = [r["frac_probe"] for r in rr if "frac_probe" in r]
+                out.append(f"| {f} | {M} | {statistics.mean(r['frac'] for r in rr):.3f} | "
+                           f"{(statistics.mean(fp) if fp else float('nan')):.3f} | {max(r['tflops'] for r in rr)} |")
+    if "splitk_modes" in d:
+        out.append("\nSplit-K reductions at one split (GEMM alone, us per call):\n")
+        out.append("| M | N x K | split | atomic | last CTA | two-pass | cluster |\n|---:|---|---:|---:|---:|---:|---:|")
+        for r in d["splitk_modes"]:
+            out.append(f"| {r['M']} | {r['N']} x {r['K']} | {r['split_k']} | {r.get('atomic')} | {r.get('last_cta')} | "
+                       f"{r.get('two_pass')} | {r.get('cluster')} |")
+    if "chain" in d:
+        out.append("\nDependent decode-layer chain (qkv -> o -> gate_up -> down, 8B-class, FP8_Dynamic):\n")
+        out.append("| M | us per chain | whole-path GB/s |\n|---:|---:|---:|")
+        for r in d["chain"]:
+            out.append(f"| {r['M']} | {r['us_per_chain']} | {r['gbs']} |")
+    if "cpu_baseline" in d:
+        cb = d["cpu_baseline"]
+        st = cb.get("single_thread", {})
+        lm = cb.get("large_m", {})
+        out.append(f"\nCPU baseline (the oracle, {cb.get('cpu_model', '')}): {cb['value']} GB/s on {cb['cores']} threads, "
+                   f"{st.get('value')} GB/s on one; {lm.get('call', '')}: {lm.get('full_s_extrapolated')} s on all threads "
+                   f"({lm.get('label', '')}).")
+    return "\n".join(out) + "\n"
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -854,12 +916,18 @@ def main():
     ap.add_argument("--out", default=None, help="also write the JSON line to this file")
     ap.add_argument("--detail-out", default=None, metavar="PATH",
                     help="write the full record (per-call tables, larger-M rows, CPU baseline) to this JSON file")
+    ap.add_argument("--report", default=None, metavar="DETAIL.json",
+                    help="print a detail record (from --detail-out) as markdown tables and exit")
     ap.add_argument("--case", default=None, metavar="FMT:M:N:K",
                     help="time one GEMM shape (eager launches, for profilers) instead of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
+    if args.report:
+        with open(args.report) as f:
+            sys.stdout.write(render_report(json.load(f)))
+        return 0
     dist = Dist()
     if args.impl == "reference":
         return run_reference(args, dist)
