@@ -30,8 +30,9 @@
  *     16-byte aligned.  The library never allocates device memory, never
  *     frees caller memory and never synchronizes the stream.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
- *     enqueued asynchronously; calls can be captured into a CUDA graph
- *     (nothing inside a call allocates or synchronizes).
+ *     enqueued asynchronously.  The quantizers and the qlinear_* calls that
+ *     take a workspace can be captured into a CUDA graph (nothing inside them
+ *     allocates or synchronizes).
  *   - Errors are returned as a qgd_status and nothing is launched when the
  *     arguments are rejected.  qgd_last_error_message() describes the last
  *     failure on the calling thread.  A device-side wait that gives up (about
@@ -202,6 +203,12 @@ QGD_API qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const voi
 QGD_API qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw,
                                           void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
                                           void* stream);
+
+/* MXFP8 layer call: quant_act_mx into the workspace, then qlinear_mxfp8
+ * (there is no fused MXFP8 kernel).  sw_e8m0 [N][K/32] bytes, 16-byte
+ * aligned; otherwise as the calls above. */
+QGD_API qgd_status qlinear_mxfp8_bf16(const void* x_bf16, int ldx, const void* wq, const void* sw_e8m0,
+                                      void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of workspace a layer call for (fmt, M, N, K) needs under the layer
  * plan in force (0 when none). */

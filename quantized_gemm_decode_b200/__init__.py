@@ -105,6 +105,7 @@ def lib() -> ctypes.CDLL:
             "qgd_test_capture_fused": [P, P],
             "quant_act_mx": [P, I, I, I, P, P, P],
             "qlinear_mxfp8": [P, P, P, P, P, I, I, I, P, S, P],
+            "qlinear_mxfp8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -354,7 +355,7 @@ def qlinear_block_fp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
 
 
 _LAYER_FN = {FMT_FP8_DYNAMIC: "qlinear_fp8_dynamic_bf16", FMT_W8A8_INT8: "qlinear_w8a8_int8_bf16",
-             FMT_BLOCK_FP8: "qlinear_block_fp8_bf16"}
+             FMT_BLOCK_FP8: "qlinear_block_fp8_bf16", FMT_MXFP8: "qlinear_mxfp8_bf16"}
 
 
 def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None):
@@ -367,9 +368,10 @@ def qlinear_bf16(fmt: int, x: torch.Tensor, wq, sw, y=None, ws=None, stream=None
     if not isinstance(wq, torch.Tensor) or wq.dim() != 2 or wq.shape[1] != K or wq.dtype not in want_w:
         raise ValueError(f"wq must be a 2-D {want_w} tensor with K={K} columns")
     N = wq.shape[0]
-    sw_n = (N // 128) * (K // 128) if fmt == FMT_BLOCK_FP8 else N
-    if not isinstance(sw, torch.Tensor) or sw.dtype != torch.float32 or sw.numel() < sw_n or not sw.is_contiguous():
-        raise ValueError(f"sw must be a contiguous float32 tensor of at least {sw_n} scales")
+    sw_n = (N // 128) * (K // 128) if fmt == FMT_BLOCK_FP8 else (N * (K // 32) if fmt == FMT_MXFP8 else N)
+    sw_t = torch.uint8 if fmt == FMT_MXFP8 else torch.float32
+    if not isinstance(sw, torch.Tensor) or sw.dtype != sw_t or sw.numel() < sw_n or not sw.is_contiguous():
+        raise ValueError(f"sw must be a contiguous {sw_t} tensor of at least {sw_n} scales")
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     elif y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) or not y.is_contiguous():

@@ -506,7 +506,10 @@ LayerWs layer_ws(int fmt, int M, int N, int K) {
   if (!l.plan.fused && M > 0) {
     l.xq_off = align256(l.total > kTicketBytes ? l.total : kTicketBytes);
     l.sx_off = align256(l.xq_off + static_cast<size_t>(M) * K);
-    const size_t nsx = fmt == kFmtBlock ? static_cast<size_t>(M) * (K / kTileK) : static_cast<size_t>(M);
+    // scales: fp32 per row or per 1x128 group; MXFP8: one byte per 32 values
+    const size_t nsx = fmt == kFmtBlock ? static_cast<size_t>(M) * (K / kTileK)
+                       : fmt == kFmtMX  ? (static_cast<size_t>(M) * (K / 32) + 3) / 4
+                                        : static_cast<size_t>(M);
     l.total = align256(l.sx_off + nsx * 4);
   }
   return l;
@@ -536,9 +539,10 @@ qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const
   void* xq = wsb + l.xq_off;
   float* sx = reinterpret_cast<float*>(wsb + l.sx_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = fmt == kFmtBlock
-                      ? launch_quant_group128(xb, M, K, ldx, static_cast<uint8_t*>(xq), sx, s)
-                      : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
+  cudaError_t e = fmt == kFmtBlock ? launch_quant_group128(xb, M, K, ldx, static_cast<uint8_t*>(xq), sx, s)
+                 : fmt == kFmtMX  ? launch_quant_mx(xb, M, K, ldx, static_cast<uint8_t*>(xq),
+                                                    reinterpret_cast<uint8_t*>(sx), s)
+                                  : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
   if (e != cudaSuccess) return cuda_fail(e, "activation quantizer launch");
   return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false);
 }
@@ -689,6 +693,12 @@ qgd_status qlinear_w8a8_int8_bf16(const void* x_bf16, int ldx, const void* wq, c
 qgd_status qlinear_block_fp8_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,
                                   int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
   return run_layer(kFmtBlock, x_bf16, ldx, wq, sw, y_bf16, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qlinear_mxfp8_bf16(const void* x_bf16, int ldx, const void* wq, const void* sw_e8m0, void* y_bf16,
+                              int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_layer(kFmtMX, x_bf16, ldx, wq, static_cast<const float*>(sw_e8m0), y_bf16, M, N, K, ws, ws_bytes,
+                   stream);
 }
 
 size_t qgd_layer_workspace_size(int fmt, int M, int N, int K) {

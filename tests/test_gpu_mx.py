@@ -85,6 +85,24 @@ def test_mx_gemm_matches_oracle(shape, plan):
     check_fp8_tolerance(bf16_to_f64(y), yref, bound, K, f"MXFP8 M={M} N={N} K={K} plan={p}")
 
 
+@pytest.mark.parametrize("M", [1, 7, 32])
+def test_mx_layer_call_from_bf16(M):
+    # quantizer into the workspace, then the GEMM: the same codes and output
+    N, K = 1024, 2048
+    x = synth.activations(M, K, 40 + M, outliers=True)
+    w = synth.weights(N, K, 40 + M)
+    wq, sw, owq, osw = _quant_check(w)
+    y = qgd.qlinear_bf16(F, x.cuda(), wq, sw)
+    torch.cuda.synchronize()
+    oxq, osx = oracle.quant_mx(x)
+    yref, bound = oracle.gemm_mx(oxq, osx, owq, osw)
+    check_fp8_tolerance(bf16_to_f64(y), yref, bound, K, f"MXFP8 layer call M={M}")
+    xq, sx = qgd.quant_mx(x.cuda())
+    y2 = qgd.qlinear_mxfp8(xq, sx, wq, sw)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
 def test_mx_rejects_what_it_does_not_cover():
     L = qgd.lib()
     import ctypes
