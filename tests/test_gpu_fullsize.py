@@ -19,19 +19,20 @@ import torch
 import oracle
 import quantized_gemm_decode_b200 as qgd
 from quantized_gemm_decode_b200 import synth, workloads
-from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, W8A8_INT8
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, W8A8_INT8
 from paritylib import as_u8, bf16_to_f64, check_fp8_tolerance, check_within_one_ulp
 
 pytestmark = pytest.mark.gpu
 
-DECODE = (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE)
+DECODE = (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE)
+FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}
 CASES = [(wl, n, k, m) for wl in DECODE for (n, k) in wl.shapes for m in (1, 17, 32)]
 
 
 @pytest.fixture(scope="module", autouse=True)
 def shipped_table():
     qgd.lib()
-    for f in range(3):
+    for f in range(4):
         qgd.qgd_set_override(f)
     if qgd.DEFAULT_TABLE:
         qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
@@ -49,6 +50,8 @@ def _weights_for(wl, N, K):
         wd = w.cuda()
         if wl.fmt == BLOCK_FP8:
             wq, sw = qgd.quant_weight_block128(wd)
+        elif wl.fmt == MXFP8:
+            wq, sw = qgd.quant_mx(wd)
         else:
             wq, sw = qgd.quant_weight_per_channel(wd, qgd.QTYPE_INT8 if wl.fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
         del wd
@@ -59,12 +62,14 @@ def _weights_for(wl, N, K):
 def _quant_x(fmt, x):
     if fmt == BLOCK_FP8:
         return qgd.quant_act_group128(x)
+    if fmt == MXFP8:
+        return qgd.quant_mx(x)
     return qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
 
 
 def _gemm(fmt, xq, sx, wq, sw):
     fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
-          BLOCK_FP8: qgd.qlinear_block_fp8}[fmt]
+          BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8}[fmt]
     return fn(xq, sx, wq, sw)
 
 
@@ -78,12 +83,17 @@ def _oracle_sample(fmt, x_rows, w_rows, wkey):
         _oracle_w.clear()
         if fmt == BLOCK_FP8:
             _oracle_w[wkey] = oracle.quant_blocks(w_rows, 128)
+        elif fmt == MXFP8:
+            _oracle_w[wkey] = oracle.quant_mx(w_rows)
         else:
             _oracle_w[wkey] = oracle.quant_rows(w_rows, oracle.INT8 if fmt == W8A8_INT8 else oracle.E4M3)
     wq, sw = _oracle_w[wkey]
     if fmt == BLOCK_FP8:
         xq, sx = oracle.quant_groups(x_rows, 128)
         y, bound = oracle.gemm_blockscaled(xq, sx, wq, sw, 128)
+    elif fmt == MXFP8:
+        xq, sx = oracle.quant_mx(x_rows)
+        y, bound = oracle.gemm_mx(xq, sx, wq, sw)
     else:
         qt = oracle.INT8 if fmt == W8A8_INT8 else oracle.E4M3
         xq, sx = oracle.quant_rows(x_rows, qt)
@@ -130,7 +140,7 @@ def test_decode_full_size_sampled(wl, N, K, M):
     xq, sx = _quant_x(wl.fmt, x.cuda())
     y = bf16_to_f64(_gemm(wl.fmt, xq, sx, wq, sw))
     torch.cuda.synchronize()
-    plan = qgd.qgd_get_plan({FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}[wl.fmt], M, N, K)
+    plan = qgd.qgd_get_plan(FMT_ID[wl.fmt], M, N, K)
     bands = sorted(set([0, N // 128 - 1] + _interior_bands(plan, M, N, K)))
     rows = np.concatenate([np.arange(b * 128, (b + 1) * 128) for b in bands])
     oxq, owq, y_ref, bound = _oracle_sample(wl.fmt, x, w[torch.from_numpy(rows)],
