@@ -17,7 +17,9 @@
  * The GEMM comes in the article's algorithm variants (section "Como se
  * implementa el kernel?" and its matmul listing): Standard (each CTA owns an
  * output tile and reduces all of K), Split-K (K is cut into split_k parts,
- * split_k a power of two from 1 to 256, whose partial sums are then added)
+ * split_k a power of two from 1 to 256 -- any count from 2 to 8 when the
+ * splits reduce inside a thread-block cluster -- whose partial sums are then
+ * added)
  * and Swap-AB (the product is computed as (W . X^T)^T so the wide N dimension
  * fills the MMA's M slot).  Which one runs for a shape is chosen from a
  * measured dispatch table (section "Hybrid dispatch" / "Despacho hibrido":
@@ -77,7 +79,8 @@ typedef enum {
   QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order
                               (Swap-AB: at most 32 tokens, else the last CTA adds them) */
   QGD_REDUCE_ATOMIC = 2,   /* split partials added atomically into a zeroed workspace (fp32 order varies) */
-  QGD_REDUCE_CLUSTER = 3   /* Swap-AB grid schedule, 2 <= split_k <= 8: the splits of a tile form one
+  QGD_REDUCE_CLUSTER = 3   /* Swap-AB grid schedule, 2 <= split_k <= 8 (not only powers of two): the
+                              splits of a tile form one
                               thread-block cluster and add their partials in split order through
                               distributed shared memory (no workspace) */
 } qgd_reduce;
@@ -94,7 +97,8 @@ typedef enum {
 /* The execution plan for one (format, M, N, K). */
 typedef struct {
   int variant;  /* qgd_variant (never AUTO here) */
-  int split_k;  /* grid schedule: CTAs along K, power of two, 1..256, at most ceil(K/128) */
+  int split_k;  /* grid schedule: CTAs along K, 1..256, at most ceil(K/128); a power of two
+                   except with QGD_REDUCE_CLUSTER, which takes any 2..8 */
   int reduce;   /* qgd_reduce, used when several CTAs share an output tile */
   int stages;   /* depth of the shared-memory operand ring */
   int tile_n;   /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */

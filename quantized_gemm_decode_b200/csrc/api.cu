@@ -255,7 +255,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   if (smax < 1) smax = 1;
   if (p.split_k < 1) p.split_k = 1;
   if (p.split_k > smax) p.split_k = smax;
-  p.split_k = floor_pow2(p.split_k);
+  // a power of two, except in a cluster, whose reduction takes any 2..8
+  if (p.reduce != kCluster) p.split_k = floor_pow2(p.split_k);
   if (p.reduce < kLastCta || p.reduce > kCluster) p.reduce = kLastCta;
   // the two-pass reduction kernel covers at most 32 tokens
   if (p.variant == kSwapAB && M > kDecodeMaxM && p.reduce == kTwoPass) p.reduce = kLastCta;
@@ -264,6 +265,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   if (p.reduce == kCluster &&
       (p.variant != kSwapAB || p.schedule != kGrid || p.split_k < 2 || p.split_k > kMaxClusterSplit))
     p.reduce = kLastCta;
+  if (p.reduce != kCluster) p.split_k = floor_pow2(p.split_k);
   if (p.reduce != kTwoPass) {
     const size_t tiles = p.variant == kSwapAB
                              ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
@@ -805,8 +807,9 @@ qgd_status qgd_load_dispatch_table(const char* path) {
       return fail(QGD_ERR_TABLE, "%s:%d: unknown format/variant/reduce/schedule name", path, lineno);
     if (N <= 0 || K <= 0 || bucket_of(Mb) != Mb)
       return fail(QGD_ERR_TABLE, "%s:%d: bad N/K or M bucket %d", path, lineno, Mb);
-    if (split < 1 || split > 256 || (split & (split - 1)) != 0)
-      return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256", path, lineno, split);
+    if (split < 1 || split > 256 || ((split & (split - 1)) != 0 && !(red == kCluster && split <= kMaxClusterSplit)))
+      return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256 (or 2..8 with cluster)", path,
+                  lineno, split);
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
         occ > 2)
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
@@ -830,7 +833,8 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
       occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");
-  if (split_k > 0 && (split_k & (split_k - 1)) != 0) return fail(QGD_ERR_INVALID, "split_k must be a power of two");
+  if (split_k > 0 && (split_k & (split_k - 1)) != 0 && !(reduce == kCluster && split_k <= kMaxClusterSplit))
+    return fail(QGD_ERR_INVALID, "split_k must be a power of two (any 2..8 with the cluster reduction)");
   std::lock_guard<std::mutex> lk(g_mu);
   Override& o = g_override[fmt];
   o.variant = variant < 0 ? -1 : variant;

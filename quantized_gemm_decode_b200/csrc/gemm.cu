@@ -494,9 +494,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   uint8_t* w_ring = base;
   uint8_t* x_ring = base + stages * stage_w;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(x_ring + stages * stage_x);
-  uint8_t* recv_buf = reinterpret_cast<uint8_t*>(ctl) + kBarBytes;  // cluster Split-K: 128 x kMpad words
+  // cluster Split-K: S x ceil(128 / S) <= 128 + 7 rows of kMpad words
+  uint8_t* recv_buf = reinterpret_cast<uint8_t*>(ctl) + kBarBytes;
   // fused: per-row maxima [128][4] and the Block_FP8 group-scale ring [kScaleRing][kMpad]
-  float* row_red = reinterpret_cast<float*>(recv_buf + (a.reduce == kCluster ? kSwapTileN * kMpad * 4 : 0));
+  float* row_red = reinterpret_cast<float*>(recv_buf + (a.reduce == kCluster ? (kSwapTileN + 8) * kMpad * 4 : 0));
   float* scale_ring = row_red + 128 * 4;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -534,7 +535,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     }
     mbar_init(&ctl->accfull, 1);
     mbar_init(&ctl->drain, 1);
-    mbar_init(&ctl->recv_bar, kSwapTileN);  // cluster Split-K: one arrival per weight row of the tile
+    {
+      // cluster Split-K: one arrival per (owned weight row, contributor)
+      const int S = a.splits > 0 ? a.splits : 1;
+      const int j = blockIdx.y;
+      const int lo = (j * kSwapTileN + S - 1) / S, hi = ((j + 1) * kSwapTileN + S - 1) / S;
+      const int cnt = (a.reduce == kCluster && !a.persistent && S > 1) ? (hi - lo) * S : kSwapTileN;
+      mbar_init(&ctl->recv_bar, cnt > 0 ? cnt : 1);
+    }
     ctl->abort_flag = 0;
     ctl->last_flag = 0;
     ctl->epi_ok = 0;
@@ -955,13 +963,16 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         if (threadIdx.x == 64 && last_seg) QGD_STAMP(8);
       } else if (a.reduce == kCluster) {
         // Split-K inside a thread-block cluster (the grid schedule's S splits
-        // of one tile): CTA j owns weight rows [j*R, (j+1)*R) of the tile,
-        // R = 128 / S.  Every CTA writes each of its partial rows into the
-        // owner's shared memory and arrives on the owner's barrier; each owner
+        // of one tile, 2 <= S <= 8, any S): CTA j owns weight rows
+        // [ceil(128 j / S), ceil(128 (j + 1) / S)) of the tile, i.e. row r
+        // belongs to CTA floor(r S / 128).  Every CTA writes each of its
+        // partial rows into the owner's shared memory (at most ceil(128 / S)
+        // rows per contributor) and arrives on the owner's barrier; each owner
         // then adds the S contributions of its rows in CTA order.
         const int S = ncontrib;
-        const int R = kSwapTileN / S;
-        const int owner = row / R, lr = row % R;
+        const int Rm = (kSwapTileN + S - 1) / S;  // most rows any owner holds
+        const int owner = (row * S) / kSwapTileN;
+        const int lr = row - (owner * kSwapTileN + S - 1) / S;
         const uint32_t dst = mapa_shared(smem_u32(recv_buf), static_cast<uint32_t>(owner));
         // owner's layout: [contributor][vector][row], 16 bytes each
         for (int cc = 0; cc < kChunks; ++cc) {
@@ -970,7 +981,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           for (int v = 0; v < kAcc / 4; ++v) {
             const int vg = cc * (kAcc / 4) + v;
             if (vg < nvec)
-              st_cluster_v4(dst + static_cast<uint32_t>(((jslot * nvec + vg) * R + lr) * 16), acc[4 * v],
+              st_cluster_v4(dst + static_cast<uint32_t>(((jslot * nvec + vg) * Rm + lr) * 16), acc[4 * v],
                             acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
           }
         }
@@ -980,17 +991,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           ctl->abort_flag = 1;
         } else {
           const uint4* rb = reinterpret_cast<const uint4*>(recv_buf);
+          const int my_lo = (jslot * kSwapTileN + S - 1) / S;
+          const int R = ((jslot + 1) * kSwapTileN + S - 1) / S - my_lo;
           for (int idx = row; idx < R * nvec; idx += kSwapTileN) {
             const int v = idx / R, r = idx % R;
-            uint4 s4 = rb[v * R + r];
+            uint4 s4 = rb[v * Rm + r];
             for (int j = 1; j < S; ++j) {
-              const uint4 w4 = rb[(j * nvec + v) * R + r];
+              const uint4 w4 = rb[(j * nvec + v) * Rm + r];
               s4.x = add_acc<kFmt>(s4.x, w4.x);
               s4.y = add_acc<kFmt>(s4.y, w4.y);
               s4.z = add_acc<kFmt>(s4.z, w4.z);
               s4.w = add_acc<kFmt>(s4.w, w4.w);
             }
-            const int nn = t * kSwapTileN + jslot * R + r;
+            const int nn = t * kSwapTileN + my_lo + r;
             if (nn < N) {
               const float swn = scaled ? __ldg(a.sw + nn) : 0.f;
               const uint32_t vals[4] = {s4.x, s4.y, s4.z, s4.w};
@@ -1574,7 +1587,7 @@ cudaError_t set_smem_attr(Kern kernel, bool& done) {
 
 size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused) {
   return 1024 + static_cast<size_t>(stages) * kps * (kSwapTileN * kTileK + mpad * kTileK) + kBarBytes +
-         (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0) + (fused ? kFusedBytes : 0);
+         (cluster ? static_cast<size_t>(kSwapTileN + 8) * mpad * 4 : 0) + (fused ? kFusedBytes : 0);
 }
 
 size_t standard_smem_bytes(int tile_n, int stages) {
@@ -1582,7 +1595,7 @@ size_t standard_smem_bytes(int tile_n, int stages) {
 }
 
 int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
-  const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN) * mpad * 4 : 0) +
+  const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN + 8) * mpad * 4 : 0) +
                        (fused ? kFusedBytes : 0);
   int s = static_cast<int>((smem_budget() - fixed) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
   return s > kMaxStages ? kMaxStages : s;

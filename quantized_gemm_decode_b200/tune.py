@@ -9,7 +9,9 @@ Portable vLLM Linear Backend with Helion", sections "Put algorithm selection
 inside the search space", "Hybrid dispatch addresses runtime overhead" and
 "Autoajuste de los kernels").  Here the space is small and discrete, so it is
 searched exhaustively: variant x tile x split_k x reduction x schedule x
-occupancy x K slices per stage at the deepest pipeline, then the pipeline
+occupancy x K slices per stage at the deepest pipeline (and, for the
+thread-block-cluster reduction, every split count from 2 to 8, which can fill
+the SMs more evenly than a power of two), then the pipeline
 depth of the best few.  Each candidate is first checked against the
 split-free result (bit-exact int32 accumulators for W8A8_INT8, a relative
 bound for the fp32-accumulating formats), then timed as a graph of layer
@@ -133,7 +135,9 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 swap_grid(s, r, 1)
             if nkt >= 2 and s <= (nkt + 1) // 2:
                 swap_grid(s, 0, 2)  # two K slices per stage
-            if 2 <= s <= 8:  # the splits of a tile as one thread-block cluster (DSMEM reduction)
+        # the splits of a tile as one thread-block cluster (DSMEM reduction): any count 2..8
+        for s in range(2, 9):
+            if s <= nkt:
                 swap_grid(s, 3, 1)
                 if nkt >= 2 and s <= (nkt + 1) // 2:
                     swap_grid(s, 3, 2)

@@ -98,6 +98,18 @@ def test_override_and_clamping():
     with pytest.raises(qgd.QGDError):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 3, 0, 0, 0)  # split not a power of two
     with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 9, qgd.REDUCE_CLUSTER, 0, 0)  # cluster of 9: too many
+    # the cluster reduction takes any split count from 2 to 8, capped at the K units
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 6, qgd.REDUCE_CLUSTER, 0, 0, qgd.SCHEDULE_GRID, 0, 2)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 6144, 4096)
+    assert (p["variant"], p["split_k"], p["reduce"], p["schedule"]) == (1, 6, qgd.REDUCE_CLUSTER, qgd.SCHEDULE_GRID)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 6144, 640)  # 5 K slices -> 3 units of two
+    assert (p["split_k"], p["reduce"]) == (3, qgd.REDUCE_CLUSTER)
+    # another reduction cannot take a split of 6: it is rounded down to a power of two
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 6, qgd.REDUCE_CLUSTER, 0, 0, qgd.SCHEDULE_PERSISTENT)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 6144, 4096)
+    assert p["reduce"] != qgd.REDUCE_CLUSTER and p["split_k"] in (1, 2, 4)
+    with pytest.raises(qgd.QGDError):
         qgd.qgd_set_override(7, 1, 2, 0, 0, 0)
 
 
@@ -168,6 +180,7 @@ def test_table_load_and_lookup(tmp_path):
 
 @pytest.mark.parametrize("bad", [
     "fp8_dynamic 4096 4096 4 standard 3 two_pass 4 256 grid 0\n",      # split not a power of two
+    "fp8_dynamic 4096 4096 4 swap_ab 9 cluster 2 128 grid 1\n",        # cluster of 9 CTAs
     "fp8_dynamic 4096 4096 5 standard 2 two_pass 4 256 grid 0\n",      # 5 is not a bucket
     "fp9 4096 4096 4 standard 2 two_pass 4 256 grid 0\n",              # unknown format
     "fp8_dynamic 4096 4096 4 standard 2 two_pass 4 256 grid\n",        # missing field
@@ -296,7 +309,7 @@ def test_table_k_slices_column(tmp_path):
 def test_cluster_reduction_plan_rules():
     G, P = qgd.SCHEDULE_GRID, qgd.SCHEDULE_PERSISTENT
     C = qgd.REDUCE_CLUSTER
-    for split in (2, 4, 8):
+    for split in (2, 3, 4, 5, 6, 7, 8):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, split, C, 0, 0, G, 0, 1)
         p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)
         assert p["reduce"] == C and p["split_k"] == split
@@ -314,10 +327,13 @@ def test_cluster_reduction_plan_rules():
 
 def test_table_cluster_reduce_name(tmp_path):
     t = tmp_path / "t.tsv"
-    t.write_text("w8a8_int8 5120 5120 8 swap_ab 4 cluster 0 0 grid 0 2\n")
+    t.write_text("w8a8_int8 5120 5120 8 swap_ab 4 cluster 0 0 grid 0 2\n"
+                 "w8a8_int8 5120 5120 16 swap_ab 5 cluster 0 0 grid 0 2\n")
     qgd.qgd_load_dispatch_table(str(t))
     p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 8, 5120, 5120)
     assert (p["reduce"], p["split_k"], p["k_slices"], p["source"]) == (qgd.REDUCE_CLUSTER, 4, 2, 1)
+    p = qgd.qgd_get_plan(qgd.FMT_W8A8_INT8, 16, 5120, 5120)
+    assert (p["reduce"], p["split_k"], p["k_slices"], p["source"]) == (qgd.REDUCE_CLUSTER, 5, 2, 1)
 
 
 @pytest.mark.parametrize("fmt,M,N,K", [("fp8_dynamic", 1, 4096, 4096), ("w8a8_int8", 16, 34816, 5120),

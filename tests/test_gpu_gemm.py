@@ -316,17 +316,17 @@ def test_two_slices_partial_last_slice(fmt, sched):
 # Split-K inside a thread-block cluster: partial rows travel through
 # distributed shared memory to the CTA that owns them.
 @pytest.mark.parametrize("fmt", ALL_FMTS)
-@pytest.mark.parametrize("split,kps", [(2, 1), (4, 1), (8, 1), (4, 2), (8, 2)])
+# Any split count from 2 to 8: with 3, 5, 6 or 7 the 128 weight rows of a tile
+# do not divide evenly among the owners (ceil(128 j / S) row boundaries).
+@pytest.mark.parametrize("split,kps", [(2, 1), (4, 1), (8, 1), (4, 2), (8, 2), (3, 1), (5, 2), (6, 1), (7, 2)])
 @pytest.mark.parametrize("M,N,K", [(1, 1024, 4096), (17, 384, 2048), (32, 2048, 1152), (5, 256, 1024)])
 def test_cluster_split_reduction(fmt, split, kps, M, N, K):
     case = Case(fmt, M, N, K, seed=split * 31 + M, outliers=True)
     yref, bound = _oracle(case)[:2]
     qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_SWAP_AB, split, qgd.REDUCE_CLUSTER, 0, 0, GRID, 0, kps)
     p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
-    nku = -(-(-(-K // 128)) // kps)  # K units of kps slices: the split is at most that, a power of two
-    expect = split
-    while expect > nku:
-        expect //= 2
+    nku = -(-(-(-K // 128)) // kps)  # K units of kps slices: the split is at most that
+    expect = min(split, nku)
     assert p["reduce"] == qgd.REDUCE_CLUSTER and p["split_k"] == expect
     y1 = case.run()
     case.check_output(y1, yref, bound, f"{fmt} cluster s={split} k={kps} M={M} N={N} K={K}")

@@ -61,6 +61,8 @@ PLANS = [
     (SW, 1, LAST, 0, 0, GRID, 1, 2),
     (SW, 4, LAST, 2, 0, GRID, 1, 2),
     (SW, 4, CLUS, 2, 0, GRID, 1, 1),
+    (SW, 3, CLUS, 2, 0, GRID, 1, 2),
+    (SW, 7, CLUS, 2, 0, GRID, 1, 1),
     (SW, 8, ATOM, 2, 0, GRID, 1, 1),
     (SW, 1, LAST, 2, 0, PERS, 1, 2),
     (SW, 1, LAST, 3, 0, PERS, 2, 1),
