@@ -107,9 +107,11 @@ typedef struct {
                     ring under half the SM's shared memory, the next GEMM's CTA can be resident
                     beside this one and do its set-up and first weight loads before this one ends */
   int source;    /* 0 = built-in default, 1 = dispatch table, 2 = override */
-  int k_slices;  /* Swap-AB: 128-wide K slices per pipeline stage (1 or 2); Standard: 1.  Each stage
-                    costs a fixed hand-off between the copy engine and the MMA, so one CTA per SM
-                    keeps up with HBM only with two slices (32 KB of weights) per stage */
+  int k_slices;  /* 128-wide K slices (K blocks) per pipeline stage, 1 or 2, in both kernels.  Each
+                    stage costs a fixed hand-off between the copy engine and the MMA (and one MMA
+                    commit), so one Swap-AB CTA per SM keeps up with HBM only with two slices
+                    (32 KB of weights) per stage, and the Standard kernel's tensor pipe idles
+                    between one-block stages */
   int fused;     /* layer calls (qlinear_*_bf16) only: 1 = the activation quantizer runs inside the
                     Swap-AB GEMM kernel, 0 = a separate quantizer kernel first.  Always 0 in the plan
                     of the qlinear_* calls, which take quantized activations */

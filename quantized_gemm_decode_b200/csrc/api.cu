@@ -247,8 +247,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
   if (p.schedule != kPersistent) p.schedule = kGrid;
-  // K slices per stage (Swap-AB only): 1 or 2, at most the K extent
-  if (p.variant != kSwapAB || p.k_slices < 1 || nkt < 2) p.k_slices = 1;
+  // 128-wide K slices (K blocks) per pipeline stage: 1 or 2, at most the K extent
+  if (p.k_slices < 1 || nkt < 2) p.k_slices = 1;
   if (p.k_slices > 2) p.k_slices = 2;
   const int nku = (nkt + p.k_slices - 1) / p.k_slices;  // K units per tile
   int smax = nku < 256 ? nku : 256;
@@ -280,7 +280,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   if (p.fused && p.reduce == kTwoPass) p.reduce = kLastCta;
   const int mpad = swap_mpad(M);
   const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster, p.fused != 0)
-                                          : standard_max_stages(p.tile_n);
+                                          : standard_max_stages(p.tile_n, p.k_slices);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
   if (fmt == kFmtMX)
@@ -290,7 +290,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   int fit = 1;
   if (p.schedule == kPersistent) {
     const size_t bytes = (p.variant == kSwapAB ? swapab_smem_bytes(mpad, p.stages, p.k_slices, false, p.fused != 0)
-                                               : standard_smem_bytes(p.tile_n, p.stages)) + 1024;
+                                               : standard_smem_bytes(p.tile_n, p.stages, p.k_slices)) + 1024;
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
     if (p.variant == kStandard && (p.tile_n == 256 || fmt == kFmtBlock)) fit = 1;  // all 512 TMEM columns

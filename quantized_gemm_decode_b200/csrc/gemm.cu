@@ -1189,9 +1189,13 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const int stages = a.stages;
+  // K blocks per pipeline stage (1 or 2): one full/empty hand-off and one
+  // MMA commit per stage, so two blocks per stage halve those per FLOP
+  const int kps = a.kps > 1 ? 2 : 1;
+  const uint32_t stage_x = kps * kXBytes, stage_w = kps * kWBytes;
   uint8_t* x_ring = base;
-  uint8_t* w_ring = base + stages * kXBytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * kWBytes);
+  uint8_t* w_ring = base + stages * stage_x;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * stage_w);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkt = (a.K + kTileK - 1) / kTileK;
@@ -1242,7 +1246,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
         const int m_tile = tile % m_tiles, n_tile = tile / m_tiles;
         const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
         const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
-        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+        for (int kt = kt0; kt < kt1; kt += kps, ++i) {
           const int s = i % stages;
           const uint32_t round = i / stages;
           if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
@@ -1255,9 +1259,14 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[s], kXBytes + kWBytes);
-          tma_load_2d(x_ring + s * kXBytes, &tx, &ctl->full[s], kt * kTileK, m_tile * kStdTileM, pol_x);
-          tma_load_2d(w_ring + s * kWBytes, &tw, &ctl->full[s], kt * kTileK, n_tile * kTileN, pol_w);
+          const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;  // K blocks in this stage
+          mbar_arrive_expect_tx(&ctl->full[s], ns * (kXBytes + kWBytes));
+          for (int h = 0; h < ns; ++h) {
+            tma_load_2d(x_ring + s * stage_x + h * kXBytes, &tx, &ctl->full[s], (kt + h) * kTileK,
+                        m_tile * kStdTileM, pol_x);
+            tma_load_2d(w_ring + s * stage_w + h * kWBytes, &tw, &ctl->full[s], (kt + h) * kTileK,
+                        n_tile * kTileN, pol_w);
+          }
           issued = i + 1;
         }
       }
@@ -1266,7 +1275,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t x_base = smem_u32(x_ring), w_base = smem_u32(w_ring);
-      int i = 0, li = 0;
+      int i = 0, li = 0, ib = 0;  // stages, items and (Block_FP8) K blocks consumed
       bool stop = false;
       for (long long w = blockIdx.x; w < items && !stop; w += gridDim.x, ++li) {
         const int split = static_cast<int>(w % S);
@@ -1280,7 +1289,7 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             break;
           }
         }
-        for (int kt = kt0; kt < kt1; ++kt, ++i) {
+        for (int kt = kt0; kt < kt1 && !stop; kt += kps, ++i) {
           const int s = i % stages;
           const uint32_t round = i / stages;
           if (!mbar_wait(&ctl->full[s], round & 1)) {
@@ -1289,31 +1298,37 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             stop = true;
             break;
           }
-          uint32_t d = tmem + buf * kTileN;
-          if constexpr (kBlock) {
-            const int slot = i % kSlots;
-            if (!mbar_wait(&ctl->tempty[slot], ((i / kSlots) & 1) ^ 1)) {
-              record_error(kErrWaitMma);
-              ctl->abort_flag = 1;
+          const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;
+          for (int h = 0; h < ns; ++h) {
+            uint32_t d = tmem + buf * kTileN;
+            if constexpr (kBlock) {
+              // every K block accumulates into its own TMEM slot
+              const int slot = ib % kSlots;
+              if (!mbar_wait(&ctl->tempty[slot], ((ib / kSlots) & 1) ^ 1)) {
+                record_error(kErrWaitMma);
+                ctl->abort_flag = 1;
+                stop = true;
+                break;
+              }
+              d = tmem + slot * kTileN;
+            }
+            if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) {
               stop = true;
               break;
             }
-            d = tmem + slot * kTileN;
-          }
-          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) {
-            stop = true;
-            break;
-          }
-          tc_fence_after();
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 32; ++kk) {
-            const uint64_t ad = sdesc_kmajor_sw128(x_base + s * kXBytes + kk * 32);
-            const uint64_t bd = sdesc_kmajor_sw128(w_base + s * kWBytes + kk * 32);
-            const uint32_t accumulate = kBlock ? (kk > 0) : (kt > kt0 || kk > 0);
-            mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+            for (int kk = 0; kk < kTileK / 32; ++kk) {
+              const uint64_t ad = sdesc_kmajor_sw128(x_base + s * stage_x + h * kXBytes + kk * 32);
+              const uint64_t bd = sdesc_kmajor_sw128(w_base + s * stage_w + h * kWBytes + kk * 32);
+              const uint32_t accumulate = kBlock ? (kk > 0) : (kt + h > kt0 || kk > 0);
+              mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
+            }
+            if constexpr (kBlock) mma_commit(&ctl->tfull[ib % kSlots]);
+            ++ib;
           }
+          if (stop) break;
           mma_commit(&ctl->empty[s]);
-          if constexpr (kBlock) mma_commit(&ctl->tfull[i % kSlots]);
         }
         if (stop) break;
         if constexpr (!kBlock) mma_commit(&ctl->tfull[buf]);
@@ -1590,8 +1605,8 @@ size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused
          (cluster ? static_cast<size_t>(kSwapTileN + 8) * mpad * 4 : 0) + (fused ? kFusedBytes : 0);
 }
 
-size_t standard_smem_bytes(int tile_n, int stages) {
-  return 1024 + static_cast<size_t>(stages) * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
+size_t standard_smem_bytes(int tile_n, int stages, int kps) {
+  return 1024 + static_cast<size_t>(stages) * kps * (kStdTileM * kTileK + tile_n * kTileK) + kBarBytes;
 }
 
 int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
@@ -1601,8 +1616,8 @@ int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
   return s > kMaxStages ? kMaxStages : s;
 }
 
-int standard_max_stages(int tile_n) {
-  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kStdTileM * kTileK + tile_n * kTileK));
+int standard_max_stages(int tile_n, int kps) {
+  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) / (kps * (kStdTileM * kTileK + tile_n * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -1664,8 +1679,8 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
   const long long items = static_cast<long long>((a.N + kTileN - 1) / kTileN) *
                           ((a.M + kStdTileM - 1) / kStdTileM) * a.splits;
   const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
-  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(std_threads<kFmt>()), standard_smem_bytes(kTileN, a.stages),
-                   stream, a.pdl != 0, tx, tw, a);
+  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(std_threads<kFmt>()),
+                   standard_smem_bytes(kTileN, a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, tx, tw, a);
 }
 
 cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,

@@ -82,9 +82,9 @@ cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStrea
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();
 size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused);
-size_t standard_smem_bytes(int tile_n, int stages);
+size_t standard_smem_bytes(int tile_n, int stages, int kps);
 int swapab_max_stages(int mpad, int kps, bool cluster, bool fused);
-int standard_max_stages(int tile_n);
+int standard_max_stages(int tile_n, int kps);
 
 // Tensor-core peak probe (probe.cu).
 cudaError_t launch_mma_probe(int qtype, int iters, int ctas, cudaStream_t stream);

@@ -142,16 +142,21 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 if nkt >= 2 and s <= (nkt + 1) // 2:
                     swap_grid(s, 3, 2)
     tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
+    # Standard: one K block per stage, and two (half the hand-offs and MMA commits) where the
+    # tensor pipe is the bound
+    kps_std = (1, 2) if (M > 32 and nkt >= 2) else (1,)
     for t in tiles:
-        for s in splits:
-            if M <= 32 and s > 16:
-                continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
-            for r in ((0,) if s == 1 else (0, 1, 2)):
-                out.append((0, s, r, t, 0, 0, 1, 0))
-        for s in (1, 2):
-            if s <= nkt:
-                for r in ((0,) if s == 1 else (0, 1)):
-                    out.append((0, s, r, t, 1, 0, 1, 0))  # Standard, persistent
+        for kps in kps_std:
+            nku = (nkt + kps - 1) // kps
+            for s in splits:
+                if (M <= 32 and s > 16) or s > nku:
+                    continue  # Standard at decode sizes wastes 3/4 of each tile; prune deep splits
+                for r in ((0,) if s == 1 else (0, 1, 2)):
+                    out.append((0, s, r, t, 0, 0, kps, 0))
+            for s in (1, 2):
+                if s <= nku:
+                    for r in ((0,) if s == 1 else (0, 1)):
+                        out.append((0, s, r, t, 1, 0, kps, 0))  # Standard, persistent
     return out
 
 

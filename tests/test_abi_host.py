@@ -261,10 +261,16 @@ def test_k_slices_plan_field():
     assert p["k_slices"] == 2 and p["occupancy"] == 1
     # deepest ring with two 16 KB weight slices + 2 KB activation slices per stage
     assert p["stages"] == (232448 - 1024 - 1024) // (2 * (16384 + 16 * 128))
-    # a single-slice K, or the Standard kernel, has one slice per stage
+    # a single-slice K has one slice per stage
     assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 128)["k_slices"] == 1
-    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 1, 0, 0, 128, P, 0, 2)
-    assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)["k_slices"] == 1
+    # the Standard kernel takes two K blocks per stage too: 128 x 256 tiles then fit two stages
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 1, 0, 0, 256, P, 0, 2)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 64, 4096, 4096)
+    assert p["k_slices"] == 2 and p["stages"] == (232448 - 1024 - 1024) // (2 * (16384 + 32768))
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_STANDARD, 1, 0, 0, 128, P, 0, 2)
+    p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 64, 4096, 4096)
+    assert p["k_slices"] == 2 and p["stages"] == 3
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8)
     # grid Split-K counts units of two slices: at most ceil(nkt / 2) splits
     qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_SWAP_AB, 32, 0, 0, 0, qgd.SCHEDULE_GRID, 0, 2)
     assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 4096, 4096)["split_k"] == 16

@@ -278,6 +278,34 @@ def test_persistent_standard_many_tiles_per_cta(fmt, M, N, K, split):
         check_fp8_tolerance(y[rows], yref, bound, K, f"{fmt} M={M}")
 
 
+# Two K blocks per pipeline stage in the Standard kernel: a stage carries two
+# 128-wide K blocks of X and W, with one hand-off and one commit; a split
+# whose K range is odd ends in a one-block stage.  Block_FP8 still gives every
+# K block its own TMEM slot.
+STD_TWO_BLOCK_PLANS = [(GRID, 1, 0, 128), (GRID, 2, 1, 256), (GRID, 2, 2, 128), (PERSISTENT, 1, 0, 256),
+                       (PERSISTENT, 2, 1, 128), (PERSISTENT, 1, 0, 128)]
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("plan", STD_TWO_BLOCK_PLANS, ids=[f"sch{p[0]}-s{p[1]}-r{p[2]}-t{p[3]}" for p in STD_TWO_BLOCK_PLANS])
+@pytest.mark.parametrize("M,N,K", [(40, 384, 1152), (130, 512, 1408), (300, 256, 640), (33, 1280, 256)])
+def test_standard_two_blocks_per_stage(fmt, plan, M, N, K):
+    sched, split, red, tile = plan
+    case = Case(fmt, M, N, K, seed=M + N + K, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD, split, red, 0, tile, sched, 0, 2)
+    p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
+    assert p["variant"] == qgd.VARIANT_STANDARD and p["k_slices"] == 2
+    y = case.run()
+    case.check_output(y, yref, bound, f"{fmt} Standard two blocks M={M} N={N} K={K} plan={p}")
+    if fmt == W8A8_INT8 and red != qgd.REDUCE_ATOMIC:
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+    assert qgd.qgd_device_error() == 0
+
+
 # Two 128-wide K slices per pipeline stage (Swap-AB): units are pairs of
 # slices, and a tile with an odd slice count ends in a one-slice unit.
 TWO_SLICE_PLANS = [(GRID, 1, 0, 0), (GRID, 2, 0, 0), (GRID, 4, 1, 0), (GRID, 4, 2, 0),
