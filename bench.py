@@ -385,7 +385,7 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
                      "tflops": round(f / (ms * 1e-3) / 1e12, 2),
                      "layer_us": round(ms_layer * 1e3, 3),
                      "layer_gbs": round(pb / (ms_layer * 1e-3) / 1e9, 1),
-                     "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
+                     "plan": (f"{('std', 'swap', 'pair')[p['variant']]}/"
                               f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
                               f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}"),
                      "layer_fused": fused})
@@ -504,7 +504,7 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict |
                    "frac": round(t_roof / (ms * 1e-3), 4),
                    "frac_spec": round(max(b / (peaks_["hbm_gbs"] * 1e9), f / (SPEC_TENSOR_TFLOPS * 1e12))
                                       / (ms * 1e-3), 4),
-                   "plan": (f"{'swap' if p['variant'] == 1 else 'std'}/"
+                   "plan": (f"{('std', 'swap', 'pair')[p['variant']]}/"
                             f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
                             f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}")}
             if probe:

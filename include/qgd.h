@@ -71,8 +71,18 @@ typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8
 typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
 /* Standard: X is the MMA's A operand (128-token tiles).  Swap-AB: Y^T = W X^T, the weight rows fill
  * the MMA's 128-row slot and the tokens its N (16/32/64/128); up to 32 tokens for Block_FP8 and up
- * to 128 for FP8_Dynamic / W8A8_INT8 (a plan asking for more gets Standard). */
-typedef enum { QGD_VARIANT_AUTO = -1, QGD_VARIANT_STANDARD = 0, QGD_VARIANT_SWAP_AB = 1 } qgd_variant;
+ * to 128 for FP8_Dynamic / W8A8_INT8 (a plan asking for more gets Standard).  Standard pair: the
+ * Standard orientation with 256-token x 256-weight-row tiles, each computed by two CTAs on two SMs
+ * (one 2-CTA cluster, tcgen05 cta_group::2): each CTA loads half of the tile's token rows and half
+ * of its weight rows, so operand traffic per FLOP is two thirds of a one-CTA 128 x 256 tile's.
+ * FP8_Dynamic and W8A8_INT8 only (other formats get Standard), no Split-K, table name
+ * "standard_pair". */
+typedef enum {
+  QGD_VARIANT_AUTO = -1,
+  QGD_VARIANT_STANDARD = 0,
+  QGD_VARIANT_SWAP_AB = 1,
+  QGD_VARIANT_STANDARD_PAIR = 2
+} qgd_variant;
 typedef enum {
   QGD_REDUCE_AUTO = -1,
   QGD_REDUCE_LAST_CTA = 0, /* split partials to workspace; the last CTA of each tile adds them in split order */

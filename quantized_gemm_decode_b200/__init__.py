@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "QGDError", "lib", "FMT_FP8_DYNAMIC", "FMT_W8A8_INT8", "FMT_BLOCK_FP8", "QTYPE_E4M3", "QTYPE_INT8",
-    "VARIANT_STANDARD", "VARIANT_SWAP_AB", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC", "REDUCE_CLUSTER",
+    "VARIANT_STANDARD", "VARIANT_SWAP_AB", "VARIANT_STANDARD_PAIR", "REDUCE_LAST_CTA", "REDUCE_TWO_PASS", "REDUCE_ATOMIC", "REDUCE_CLUSTER",
     "SCHEDULE_GRID", "SCHEDULE_PERSISTENT",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
     "quant_act_per_token_strided", "quant_act_group128_strided", "quant_mx", "qlinear_mxfp8", "FMT_MXFP8",
@@ -46,7 +46,7 @@ DEFAULT_TABLE = os.path.join(_PKG, "tables", "b200.tsv")
 
 FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8, FMT_MXFP8 = 0, 1, 2, 3
 QTYPE_E4M3, QTYPE_INT8 = 0, 1
-VARIANT_STANDARD, VARIANT_SWAP_AB = 0, 1
+VARIANT_STANDARD, VARIANT_SWAP_AB, VARIANT_STANDARD_PAIR = 0, 1, 2
 REDUCE_LAST_CTA, REDUCE_TWO_PASS, REDUCE_ATOMIC, REDUCE_CLUSTER = 0, 1, 2, 3
 SCHEDULE_GRID, SCHEDULE_PERSISTENT = 0, 1
 FORMAT_NAMES = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "mxfp8": 3}

@@ -155,6 +155,7 @@ int fmt_from_name(const std::string& s) {
 int variant_from_name(const std::string& s) {
   if (s == "standard") return kStandard;
   if (s == "swap_ab" || s == "swapab") return kSwapAB;
+  if (s == "standard_pair") return kStandardPair;
   return -1;
 }
 
@@ -244,8 +245,16 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
     if (p.reduce == kTwoPass) p.reduce = kLastCta;
   }
   if (p.variant == kSwapAB && M > (fmt == kFmtBlock ? kDecodeMaxM : kSwapMaxM)) p.variant = kStandard;
+  // CTA-pair tiles: the per-token / per-channel formats, no Split-K
+  if (p.variant == kStandardPair && fmt != kFmtFP8 && fmt != kFmtINT8) p.variant = kStandard;
+  if (p.variant < kStandard || p.variant > kStandardPair) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
+  else if (p.variant == kStandardPair) p.tile_n = 256;
   else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+  if (p.variant == kStandardPair) {
+    p.split_k = 1;
+    p.reduce = kLastCta;
+  }
   if (p.schedule != kPersistent) p.schedule = kGrid;
   // 128-wide K slices (K blocks) per pipeline stage: 1 or 2, at most the K extent
   if (p.k_slices < 1 || nkt < 2) p.k_slices = 1;
@@ -280,7 +289,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   if (p.fused && p.reduce == kTwoPass) p.reduce = kLastCta;
   const int mpad = swap_mpad(M);
   const int max_st = p.variant == kSwapAB ? swapab_max_stages(mpad, p.k_slices, p.reduce == kCluster, p.fused != 0)
-                                          : standard_max_stages(p.tile_n, p.k_slices);
+                     : p.variant == kStandardPair ? pair_max_stages(p.k_slices)
+                                                  : standard_max_stages(p.tile_n, p.k_slices);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
   if (fmt == kFmtMX)
@@ -294,6 +304,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
     fit = static_cast<int>(kSmemPerSM / bytes);
     fit = fit < 1 ? 1 : (fit > 2 ? 2 : fit);
     if (p.variant == kStandard && (p.tile_n == 256 || fmt == kFmtBlock)) fit = 1;  // all 512 TMEM columns
+    if (p.variant == kStandardPair) fit = 1;
 
   }
   if (p.occupancy <= 0 || p.occupancy > fit) p.occupancy = fit;
@@ -302,6 +313,22 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
 }
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// How many CTA-pair clusters fit on the current device at once, per
+// (format, stages, K blocks per stage); queried once each (0 if unknown).
+int pair_clusters_that_fit(int fmt, int stages, int kps) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const auto key = std::make_tuple(dev, fmt, stages, kps);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  const int n = pair_max_active_clusters(fmt, stages, kps);
+  cache[key] = n;
+  return n;
+}
 
 long long sk_owner(long long u, long long G, long long U) { return ((u + 1) * G - 1) / U; }
 
@@ -347,6 +374,16 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
       e.data_bytes = p.reduce == kAtomic
                          ? align256(static_cast<size_t>(M) * N * 4)
                          : align256(static_cast<size_t>(n_tiles) * e.maxc * kSwapTileN * e.mstride * 4);
+  } else if (p.variant == kStandardPair) {
+    // 256 x 256 pair tiles dealt to CTA pairs (two CTAs each, one per SM);
+    // the launch lowers the pair count to what fits on the GPU at once
+    e.maxc = 1;
+    e.tiles = static_cast<size_t>((N + 255) / 256) * ((M + 255) / 256);
+    if (p.schedule == kPersistent) {
+      const long long pairs = g_num_sms / 2;
+      e.persistent = true;
+      e.ctas = static_cast<int>(2 * (static_cast<long long>(e.tiles) < pairs ? static_cast<long long>(e.tiles) : pairs));
+    }
   } else {
     e.maxc = p.split_k;
     e.tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
@@ -461,6 +498,15 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
     if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;
     if (!fused && (st = encode_kmajor(&tx, xq, M, K, ex.mpad)) != QGD_OK) return st;
     e = launch_swapab(fmt, ex.mpad, fused, tw, tx, a, s);
+  } else if (p.variant == kStandardPair) {
+    // each CTA of a pair loads 128 token rows and 128 weight rows per K block
+    if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
+    if ((st = encode_kmajor(&tw, wq, N, K, 128)) != QGD_OK) return st;
+    if (a.persistent) {
+      const int fit = pair_clusters_that_fit(fmt, p.stages, p.k_slices);
+      if (fit > 0 && a.ctas > 2 * fit) a.ctas = 2 * fit;
+    }
+    e = launch_standard_pair(fmt, tx, tw, a, s);
   } else {
     if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
     if ((st = encode_kmajor(&tw, wq, N, K, p.tile_n)) != QGD_OK) return st;
@@ -829,7 +875,7 @@ qgd_status qgd_clear_dispatch_table(void) {
 qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int stages, int tile_n, int schedule,
                             int occupancy, int k_slices) {
   if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
-  if (variant > 1 || reduce > 3 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
+  if (variant > 2 || reduce > 3 || split_k > 256 || stages > kMaxStages || stages < 0 || schedule > 1 ||
       occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");

@@ -1513,6 +1513,265 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
 }
 
 // ===========================================================================
+// Standard tiles of 256 tokens x 256 weight rows computed by a CTA pair (a
+// 2-CTA cluster, tcgen05 .cta_group::2), FP8_Dynamic and W8A8_INT8.
+//
+// CTA r of the pair loads X rows [256 mt + 128 r, +128) and W rows
+// [256 nt + 128 r, +128) into its own shared memory; the leader (r = 0)
+// issues one M = 256, N = 256 MMA per 32-wide K step that reads both CTAs'
+// tiles, and each CTA's tensor memory receives its 128 token rows x 256
+// weight columns.  Per CTA and K block that is 32 KB of operands for the
+// same 8.4 MFLOP a one-CTA 128 x 256 tile does with 48 KB: the L2-to-SM
+// traffic per FLOP -- what bounds the one-CTA kernel at large M -- drops by a
+// third.  Both CTAs' copies complete on the leader's `full` barrier (its
+// expect-tx counts both); the leader's commits arrive on `empty` / `tfull` in
+// both CTAs; both CTAs' epilogue warps hand the accumulator back on the
+// leader's `tempty`.  Work items are pair tiles, token-tile fastest, dealt
+// to the pairs round-robin.  A failed (bounded) wait in either CTA sets both
+// CTAs' abort flags.
+// ===========================================================================
+constexpr int kPairTileM = 256;  // tokens per pair tile (MMA M)
+constexpr int kPairTileN = 256;  // weight rows per pair tile (MMA N)
+
+template <int kFmt>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    standard_pair_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+                         const GemmArgs a) {
+  constexpr bool kInt = (kFmt == kFmtINT8);
+  static_assert(kFmt == kFmtFP8 || kFmt == kFmtINT8, "per-token / per-channel formats only");
+  constexpr uint32_t kXBytes = (kPairTileM / 2) * kTileK;  // this CTA's 128 token rows of a K block
+  constexpr uint32_t kWBytes = (kPairTileN / 2) * kTileK;  // this CTA's 128 weight rows of a K block
+  constexpr uint32_t kCols = 2 * kPairTileN;               // double-buffered 128 x 256 accumulator
+  constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kPairTileM, kPairTileN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  const int stages = a.stages;
+  const int kps = a.kps > 1 ? 2 : 1;
+  const uint32_t stage_x = kps * kXBytes, stage_w = kps * kWBytes;
+  uint8_t* x_ring = base;
+  uint8_t* w_ring = base + stages * stage_x;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * stage_w);
+
+  const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkt = (a.K + kTileK - 1) / kTileK;
+  const int m_tiles = (a.M + kPairTileM - 1) / kPairTileM;
+  const int n_tiles = (a.N + kPairTileN - 1) / kPairTileN;
+  const long long items = static_cast<long long>(m_tiles) * n_tiles;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tx);
+    tma_prefetch_desc(&tw);
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->tfull[i], 1);
+      mbar_init(&ctl->tempty[i], 8);  // the 4 epilogue warps of each CTA of the pair
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    ctl->last_flag = 0;
+    ctl->epi_ok = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&ctl->tmem_base, kCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers and tensor memory exist before any traffic between them
+  tc_fence_after();
+  griddep_launch_dependents();
+  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t partner_abort = mapa_shared(smem_u32(&ctl->abort_flag), rank ^ 1u);
+  auto fail = [&](unsigned int code) {
+    record_error(code);
+    ctl->abort_flag = 1;
+    st_cluster_u32(partner_abort, 1u);
+  };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&ctl->abort_flag) != 0; };
+  int issued = 0;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs): this CTA's halves ----------------
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_w = policy_evict_last();
+      const uint32_t full0 = mapa_shared(smem_u32(&ctl->full[0]), 0);  // the leader's barriers
+      griddep_wait();  // activations come from the preceding kernel
+      int i = 0;
+      bool stop = false;
+      for (long long w = pair; w < items && !stop; w += npairs) {
+        const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
+        const int xrow = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2);
+        const int wrow = nt * kPairTileN + static_cast<int>(rank) * (kPairTileN / 2);
+        for (int kt = 0; kt < nkt; kt += kps, ++i) {
+          const int s = i % stages;
+          const uint32_t round = i / stages;
+          if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+            fail(kErrWaitProducer);
+            stop = true;
+            break;
+          }
+          if (aborted()) {
+            stop = true;
+            break;
+          }
+          const int ns = (nkt - kt) < kps ? (nkt - kt) : kps;
+          // the leader's barrier expects both CTAs' bytes (a copy may land first)
+          if (rank == 0) mbar_arrive_expect_tx(&ctl->full[s], 2u * ns * (kXBytes + kWBytes));
+          const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
+          for (int h = 0; h < ns; ++h) {
+            tma_load_2d_pair(x_ring + s * stage_x + h * kXBytes, &tx, fb, (kt + h) * kTileK, xrow, pol_x);
+            tma_load_2d_pair(w_ring + s * stage_w + h * kWBytes, &tw, fb, (kt + h) * kTileK, wrow, pol_w);
+          }
+          issued = i + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the leader only ----------------
+    if (rank == 0 && lane == 0) {
+      const uint32_t x_base = smem_u32(x_ring), w_base = smem_u32(w_ring);
+      int i = 0, li = 0;
+      bool stop = false;
+      for (long long w = pair; w < items && !stop; w += npairs, ++li) {
+        const int buf = li & 1;
+        if (!mbar_wait(&ctl->tempty[buf], ((li >> 1) & 1) ^ 1)) {
+          fail(kErrWaitMma);
+          break;
+        }
+        const uint32_t d = tmem + buf * kPairTileN;
+        for (int kt = 0; kt < nkt && !stop; kt += kps, ++i) {
+          const int s = i % stages;
+          const uint32_t round = i / stages;
+          if (!mbar_wait(&ctl->full[s], round & 1)) {
+            fail(kErrWaitMma);
+            stop = true;
+            break;
+          }
+          if (aborted()) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const int ns = (nkt - kt) < kps ? (nkt - kt) : kps;
+          for (int h = 0; h < ns; ++h) {
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 32; ++kk) {
+              const uint64_t ad = sdesc_kmajor_sw128(x_base + s * stage_x + h * kXBytes + kk * 32);
+              const uint64_t bd = sdesc_kmajor_sw128(w_base + s * stage_w + h * kWBytes + kk * 32);
+              mma_issue_pair<kInt>(d, ad, bd, kIdesc, (kt + h > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit_pair(&ctl->empty[s], 0x3);
+        }
+        if (stop) break;
+        mma_commit_pair(&ctl->tfull[buf], 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    griddep_wait();  // scales and outputs: only after the preceding kernel is done
+    const int q = warp & 3;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tempty0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);  // the leader's
+    const int M = a.M, N = a.N;
+    int li = 0;
+    for (long long w = pair; w < items; w += npairs, ++li) {
+      const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
+      const int buf = li & 1;
+      const bool ok = warp_wait(&ctl->tfull[buf], (li >> 1) & 1);
+      if (!ok && lane == 0) fail(kErrWaitEpilogue);
+      if (ok) tc_fence_after();
+      if (!epi_agree_ok(ctl)) break;
+      const int m = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2) + q * 32 + lane;
+      const bool in_m = m < M;
+      const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
+      const uint32_t tbuf = taddr + buf * kPairTileN;
+#pragma unroll 1
+      for (int c = 0; c < kPairTileN / 16; ++c) {
+        const int nc = nt * kPairTileN + c * 16;
+        uint32_t r[16];
+        __syncwarp();
+        tmem_ld16(tbuf + c * 16, r);
+        tmem_wait_ld();
+        if (c == kPairTileN / 16 - 1) {
+          // the whole accumulator row is in registers: hand the buffer back to the leader
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(tempty0 + static_cast<uint32_t>(buf) * 8u);
+        }
+        if (!in_m || nc >= N) continue;
+        const size_t idx = static_cast<size_t>(m) * N + nc;
+        if (a.raw) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+        } else {
+          const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+          float sw16[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 t4 = __ldg(swv + v);
+            sw16[4 * v] = t4.x;
+            sw16[4 * v + 1] = t4.y;
+            sw16[4 * v + 2] = t4.z;
+            sw16[4 * v + 3] = t4.w;
+          }
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float v0, v1;
+            if constexpr (kInt) {
+              v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
+              v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+            } else {
+              v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
+              v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+            }
+            pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  // one answer for every thread (the partner may set the flag at any time)
+  if (__syncthreads_or(ctl->abort_flag != 0)) {
+    if (rank == 0 && warp == 0 && lane == 0) {
+      // the last copies issued into each stage (both CTAs') must land before either CTA exits
+      for (int i = issued > stages ? issued - stages : 0; i < issued; ++i) {
+        if (!mbar_wait(&ctl->full[i % stages], (i / stages) & 1)) {
+          record_error(kErrWaitDrain);
+          break;
+        }
+      }
+    }
+    if (rank == 0 && warp == 1 && lane == 0) {
+      mma_commit_pair(&ctl->drain, 0x1);  // arrives once every MMA issued so far is done
+      if (!mbar_wait(&ctl->drain, 0)) record_error(kErrWaitDrain);
+    }
+    __syncthreads();
+  }
+  cluster_sync_all();  // neither CTA leaves while its partner may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kCols);
+  }
+}
+
+// ===========================================================================
 // Two-pass Split-K reduction: one thread per output element, partials added
 // in split order s = 0, 1, ..., splits-1.
 // ===========================================================================
@@ -1553,10 +1812,11 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const GemmArgs a) {
 }
 
 // Launch with dynamic shared memory and, when `pdl` is set, a programmatic
-// dependency on the preceding kernel in the stream.
+// dependency on the preceding kernel in the stream; clusters of
+// cluster_x x cluster_y CTAs when either is above 1.
 template <typename... Params, typename... Args>
-cudaError_t launch_ex_cluster(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                              bool pdl, int cluster_y, Args&&... args) {
+cudaError_t launch_ex_cluster_xy(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 bool pdl, int cluster_x, int cluster_y, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -1569,9 +1829,9 @@ cudaError_t launch_ex_cluster(void (*kernel)(Params...), dim3 grid, dim3 block, 
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
   }
-  if (cluster_y > 1) {
+  if (cluster_x > 1 || cluster_y > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
-    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster_x);
     attr[n].val.clusterDim.y = static_cast<unsigned>(cluster_y);
     attr[n].val.clusterDim.z = 1;
     ++n;
@@ -1581,6 +1841,12 @@ cudaError_t launch_ex_cluster(void (*kernel)(Params...), dim3 grid, dim3 block, 
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_ex_cluster(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              bool pdl, int cluster_y, Args&&... args) {
+  return launch_ex_cluster_xy(kernel, grid, block, smem, stream, pdl, 1, cluster_y, std::forward<Args>(args)...);
 }
 
 template <typename... Params, typename... Args>
@@ -1613,6 +1879,22 @@ int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
   const size_t fixed = 1024 + kBarBytes + (cluster ? static_cast<size_t>(kSwapTileN + 8) * mpad * 4 : 0) +
                        (fused ? kFusedBytes : 0);
   int s = static_cast<int>((smem_budget() - fixed) / (kps * (kSwapTileN * kTileK + mpad * kTileK)));
+  return s > kMaxStages ? kMaxStages : s;
+}
+
+// At least half an SM's shared memory, so that no two CTAs of this kernel share
+// an SM: each allocates all 512 tensor-memory columns together with its
+// partner, and a CTA whose allocation waited on another pair's CTA on its SM
+// could wait for good.
+size_t pair_smem_bytes(int stages, int kps) {
+  const size_t need =
+      1024 + static_cast<size_t>(stages) * kps * ((kPairTileM / 2) * kTileK + (kPairTileN / 2) * kTileK) + kBarBytes;
+  return need > kSmemPerSM / 2 ? need : kSmemPerSM / 2;
+}
+
+int pair_max_stages(int kps) {
+  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) /
+                           (kps * ((kPairTileM / 2) * kTileK + (kPairTileN / 2) * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
 
@@ -1681,6 +1963,58 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
   const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
   return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(std_threads<kFmt>()),
                    standard_smem_bytes(kTileN, a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, tx, tw, a);
+}
+
+template <int kFmt>
+static cudaError_t launch_standard_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                                          cudaStream_t stream) {
+  static bool attr_done = false;
+  cudaError_t e = set_smem_attr(standard_pair_kernel<kFmt>, attr_done);
+  if (e != cudaSuccess) return e;
+  const long long items = static_cast<long long>((a.N + kPairTileN - 1) / kPairTileN) *
+                          ((a.M + kPairTileM - 1) / kPairTileM);
+  const long long pairs = a.persistent && a.ctas / 2 < items ? a.ctas / 2 : items;
+  return launch_ex_cluster_xy(standard_pair_kernel<kFmt>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads),
+                              pair_smem_bytes(a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, 2, 1, tx, tw, a);
+}
+
+cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                                 cudaStream_t stream) {
+  if (fmt == kFmtFP8) return launch_standard_pair_t<kFmtFP8>(tx, tw, a, stream);
+  if (fmt == kFmtINT8) return launch_standard_pair_t<kFmtINT8>(tx, tw, a, stream);
+  return cudaErrorInvalidValue;
+}
+
+// Pair clusters that fit on the GPU at once with this shared memory (0 if the
+// query fails): the persistent pair schedule launches no more than that.
+int pair_max_active_clusters(int fmt, int stages, int kps) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = pair_smem_bytes(stages, kps);
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e;
+  if (fmt == kFmtINT8) {
+    static bool done = false;
+    if ((e = set_smem_attr(standard_pair_kernel<kFmtINT8>, done)) != cudaSuccess) return 0;
+    e = cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmtINT8>, &cfg);
+  } else {
+    static bool done = false;
+    if ((e = set_smem_attr(standard_pair_kernel<kFmtFP8>, done)) != cudaSuccess) return 0;
+    e = cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmtFP8>, &cfg);
+  }
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,

@@ -10,7 +10,8 @@ namespace qgd {
 
 enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2, kFmtMX = 3 };
 constexpr int kNumFmts = 4;
-enum Variant : int { kStandard = 0, kSwapAB = 1 };
+// kStandardPair: Standard tiles of 256 x 256 computed by a CTA pair (FP8_Dynamic, W8A8_INT8)
+enum Variant : int { kStandard = 0, kSwapAB = 1, kStandardPair = 2 };
 enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2, kCluster = 3 };
 constexpr int kMaxClusterSplit = 8;  // portable thread-block cluster size
 enum Schedule : int { kGrid = 0, kPersistent = 1 };
@@ -77,6 +78,9 @@ cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, 
                           const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmArgs& a, cudaStream_t stream);
+cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                                 cudaStream_t stream);
+int pair_max_active_clusters(int fmt, int stages, int kps);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
@@ -85,6 +89,8 @@ size_t swapab_smem_bytes(int mpad, int stages, int kps, bool cluster, bool fused
 size_t standard_smem_bytes(int tile_n, int stages, int kps);
 int swapab_max_stages(int mpad, int kps, bool cluster, bool fused);
 int standard_max_stages(int tile_n, int kps);
+size_t pair_smem_bytes(int stages, int kps);
+int pair_max_stages(int kps);
 
 // Tensor-core peak probe (probe.cu).
 cudaError_t launch_mma_probe(int qtype, int iters, int ctas, cudaStream_t stream);

@@ -40,7 +40,7 @@ from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, 
 
 L2_BYTES = 126 * 1024 * 1024
 FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}
-VAR_NAME = {0: "standard", 1: "swap_ab"}
+VAR_NAME = {0: "standard", 1: "swap_ab", 2: "standard_pair"}
 RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
 
 
@@ -79,7 +79,7 @@ def two_per_sm_stages(M: int, kps: int, cluster: bool, fused: bool = False) -> i
     deepest ring, one CTA per SM) when no such ring exists."""
     mpad = swap_mpad(M)
     per_stage = kps * (128 * 128 + mpad * 128)
-    fixed = (1024 + 1024 + (128 * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
+    fixed = (1024 + 1024 + ((128 + 8) * mpad * 4 if cluster else 0) + 1024  # alignment, control, receive buffer, reserve
              + (FUSED_BYTES if fused else 0))
     st = min(16, (SMEM_PER_SM // 2 - fixed) // per_stage)
     return st if st >= 2 else 0
@@ -157,6 +157,11 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 if s <= nku:
                     for r in ((0,) if s == 1 else (0, 1)):
                         out.append((0, s, r, t, 1, 0, kps, 0))  # Standard, persistent
+    # Standard pair tiles (256 x 256 on two SMs): the per-token formats past 128 tokens
+    if fmt in (FP8_DYNAMIC, W8A8_INT8) and M > 128:
+        for kps in kps_std:
+            for sched in (0, 1):
+                out.append((2, 1, 0, 256, sched, 0, kps, 0))
     return out
 
 

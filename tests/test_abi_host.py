@@ -312,6 +312,35 @@ def test_table_k_slices_column(tmp_path):
         qgd.qgd_load_dispatch_table(str(bad))
 
 
+def test_standard_pair_plan_rules():
+    P, G = qgd.SCHEDULE_PERSISTENT, qgd.SCHEDULE_GRID
+    for fmt in (qgd.FMT_FP8_DYNAMIC, qgd.FMT_W8A8_INT8):
+        qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 4, qgd.REDUCE_TWO_PASS, 0, 128, P, 0, 2)
+        p = qgd.qgd_get_plan(fmt, 4096, 6144, 4096)
+        # pair tiles are 256 wide and never split K; two K blocks per stage fit three stages
+        assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"], p["stages"], p["occupancy"]) == \
+            (qgd.VARIANT_STANDARD_PAIR, 256, 1, 2, 3, 1)
+        assert qgd.qgd_workspace_size(fmt, 4096, 6144, 4096) == 0
+        qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, G, 0, 1)
+        assert qgd.qgd_get_plan(fmt, 512, 6144, 4096)["stages"] == (232448 - 2048) // 32768
+        qgd.qgd_set_override(fmt)
+    # Block_FP8 and MXFP8 have no pair tiles
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, P)
+    assert qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 4096, 6144, 4096)["variant"] == qgd.VARIANT_STANDARD
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8)
+    with pytest.raises(qgd.QGDError):
+        qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 3, 1, 0, 0, 0)
+
+
+def test_table_standard_pair_name(tmp_path):
+    t = tmp_path / "t.tsv"
+    t.write_text("fp8_dynamic 6144 4096 8192 standard_pair 1 last_cta 3 256 persistent 1 2\n")
+    qgd.qgd_load_dispatch_table(str(t))
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 8192, 6144, 4096)
+    assert (p["variant"], p["stages"], p["k_slices"], p["schedule"], p["source"]) == \
+        (qgd.VARIANT_STANDARD_PAIR, 3, 2, qgd.SCHEDULE_PERSISTENT, 1)
+
+
 def test_cluster_reduction_plan_rules():
     G, P = qgd.SCHEDULE_GRID, qgd.SCHEDULE_PERSISTENT
     C = qgd.REDUCE_CLUSTER
@@ -371,7 +400,7 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
             assert p["stages"] == st
             if var == qgd.VARIANT_SWAP_AB and (sch == qgd.SCHEDULE_GRID or occ == 2) and not fz:
                 mpad = tune.swap_mpad(M)
-                smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + (128 * mpad * 4 if r == 3 else 0)
+                smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + ((128 + 8) * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
     qgd.qgd_set_fused_override(fid)
 
