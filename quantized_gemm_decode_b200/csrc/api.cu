@@ -86,6 +86,21 @@ qgd_status get_encoder() {
 
 // 2-D byte matrix [rows, cols] (cols contiguous), box = box_rows x 128 bytes,
 // 128-byte swizzle; out-of-range rows/columns read as zero.
+// bf16 output [rows, cols] (cols contiguous) for tensor stores: boxes of
+// 32 rows x 64 columns (128 bytes), 128-byte swizzle; parts of a box past the
+// extent are not written.
+qgd_status encode_out_bf16(CUtensorMap* map, void* base, int rows, int cols) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QGD_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d) rows=%d cols=%d", (int)r, rows, cols);
+  return QGD_OK;
+}
+
 qgd_status encode_kmajor(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
@@ -502,11 +517,14 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
     // each CTA of a pair loads 128 token rows and 128 weight rows per K block
     if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
     if ((st = encode_kmajor(&tw, wq, N, K, 128)) != QGD_OK) return st;
+    CUtensorMap ty;
+    memset(&ty, 0, sizeof ty);
+    if (!raw && (st = encode_out_bf16(&ty, y, M, N)) != QGD_OK) return st;
     if (a.persistent) {
       const int fit = pair_clusters_that_fit(fmt, p.stages, p.k_slices);
       if (fit > 0 && a.ctas > 2 * fit) a.ctas = 2 * fit;
     }
-    e = launch_standard_pair(fmt, tx, tw, a, s);
+    e = launch_standard_pair(fmt, tx, tw, ty, a, s);
   } else {
     if ((st = encode_kmajor(&tx, xq, M, K, kStdTileM)) != QGD_OK) return st;
     if ((st = encode_kmajor(&tw, wq, N, K, p.tile_n)) != QGD_OK) return st;

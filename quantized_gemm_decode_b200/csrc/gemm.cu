@@ -1533,10 +1533,16 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
 constexpr int kPairTileM = 256;  // tokens per pair tile (MMA M)
 constexpr int kPairTileN = 256;  // weight rows per pair tile (MMA N)
 
+// Output staging for the tensor stores of Y: per epilogue warp two buffers of
+// 32 rows x 64 bf16 columns (4 KB each), 128-byte swizzled like the tensor
+// map's box, so that a warp's 32 rows are written without bank conflicts and
+// leave as whole 128-byte lines.
+constexpr uint32_t kPairStageBytes = 4 * 2 * 32 * 128;
+
 template <int kFmt>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     standard_pair_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
-                         const GemmArgs a) {
+                         const __grid_constant__ CUtensorMap ty, const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   static_assert(kFmt == kFmtFP8 || kFmt == kFmtINT8, "per-token / per-channel formats only");
   constexpr uint32_t kXBytes = (kPairTileM / 2) * kTileK;  // this CTA's 128 token rows of a K block
@@ -1551,7 +1557,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t stage_x = kps * kXBytes, stage_w = kps * kWBytes;
   uint8_t* x_ring = base;
   uint8_t* w_ring = base + stages * stage_x;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(w_ring + stages * stage_w);
+  uint8_t* y_stage = w_ring + stages * stage_w;  // 1024-aligned: the rings are whole 16 KB blocks
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(y_stage + kPairStageBytes);
 
   const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
   const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
@@ -1564,6 +1571,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tx);
     tma_prefetch_desc(&tw);
+    if (!a.raw) tma_prefetch_desc(&ty);
     for (int i = 0; i < stages; ++i) {
       mbar_init(&ctl->full[i], 1);
       mbar_init(&ctl->empty[i], 1);
@@ -1682,6 +1690,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tempty0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);  // the leader's
     const int M = a.M, N = a.N;
+    uint8_t* ybuf = y_stage + q * (2 * 32 * 128);  // this warp's two 4 KB staging buffers
+    int nstore = 0;                                // tensor stores this warp has issued
     int li = 0;
     for (long long w = pair; w < items; w += npairs, ++li) {
       const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
@@ -1690,7 +1700,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok && lane == 0) fail(kErrWaitEpilogue);
       if (ok) tc_fence_after();
       if (!epi_agree_ok(ctl)) break;
-      const int m = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2) + q * 32 + lane;
+      const int row0 = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2) + q * 32;  // this warp's rows
+      const int m = row0 + lane;
       const bool in_m = m < M;
       const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
       const uint32_t tbuf = taddr + buf * kPairTileN;
@@ -1707,15 +1718,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(tempty0 + static_cast<uint32_t>(buf) * 8u);
         }
-        if (!in_m || nc >= N) continue;
-        const size_t idx = static_cast<size_t>(m) * N + nc;
-        if (a.raw) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
+        if (a.raw) {  // int32 accumulators (test hook): plain stores
+          if (!in_m || nc >= N) continue;
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
 #pragma unroll
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-        } else {
+          continue;
+        }
+        // columns nc .. nc + 15 of row m -> bf16, into the staging buffer of
+        // this 64-column group (the 16-byte chunk j of a row sits at j ^ (row % 8))
+        float sw16[16];
+        if (nc < N) {
           const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
-          float sw16[16];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             const float4 t4 = __ldg(swv + v);
@@ -1724,25 +1738,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             sw16[4 * v + 2] = t4.z;
             sw16[4 * v + 3] = t4.w;
           }
-          uint32_t pk[8];
+        } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float v0, v1;
-            if constexpr (kInt) {
-              v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
-              v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
-            } else {
-              v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
-              v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
-            }
-            pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+          for (int j = 0; j < 16; ++j) sw16[j] = 0.f;
+        }
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v0, v1;
+          if constexpr (kInt) {
+            v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
+            v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+          } else {
+            v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
+            v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
           }
-          uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+        }
+        const int g = c & 3;  // 16-column chunk within the 64-column group
+        uint8_t* sb = ybuf + (nstore & 1) * (32 * 128);
+        if (g == 0 && lane == 0 && nstore >= 2) bulk_wait_group_read<1>();  // this buffer's last store has read it
+        __syncwarp();
+        st_shared_v4(sb + lane * 128 + (((2 * g) ^ (lane & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        st_shared_v4(sb + lane * 128 + (((2 * g + 1) ^ (lane & 7)) << 4), make_uint4(pk[4], pk[5], pk[6], pk[7]));
+        if (g == 3) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // a group per buffer use, empty when the box lies wholly past M or N,
+            // so that "one group still reading" always means the other buffer
+            if (row0 < M && nc - 48 < N) tma_store_2d(&ty, sb, nc - 48, row0);
+            bulk_commit_group();
+          }
+          ++nstore;
         }
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // the stores are done before the CTA ends
   }
 
   // ---------------- teardown ----------------
@@ -1887,13 +1919,14 @@ int swapab_max_stages(int mpad, int kps, bool cluster, bool fused) {
 // partner, and a CTA whose allocation waited on another pair's CTA on its SM
 // could wait for good.
 size_t pair_smem_bytes(int stages, int kps) {
-  const size_t need =
-      1024 + static_cast<size_t>(stages) * kps * ((kPairTileM / 2) * kTileK + (kPairTileN / 2) * kTileK) + kBarBytes;
+  const size_t need = 1024 +
+                      static_cast<size_t>(stages) * kps * ((kPairTileM / 2) * kTileK + (kPairTileN / 2) * kTileK) +
+                      kPairStageBytes + kBarBytes;
   return need > kSmemPerSM / 2 ? need : kSmemPerSM / 2;
 }
 
 int pair_max_stages(int kps) {
-  int s = static_cast<int>((smem_budget() - 1024 - kBarBytes) /
+  int s = static_cast<int>((smem_budget() - 1024 - kPairStageBytes - kBarBytes) /
                            (kps * ((kPairTileM / 2) * kTileK + (kPairTileN / 2) * kTileK)));
   return s > kMaxStages ? kMaxStages : s;
 }
@@ -1966,8 +1999,8 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
 }
 
 template <int kFmt>
-static cudaError_t launch_standard_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
-                                          cudaStream_t stream) {
+static cudaError_t launch_standard_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                                          const GemmArgs& a, cudaStream_t stream) {
   static bool attr_done = false;
   cudaError_t e = set_smem_attr(standard_pair_kernel<kFmt>, attr_done);
   if (e != cudaSuccess) return e;
@@ -1975,13 +2008,13 @@ static cudaError_t launch_standard_pair_t(const CUtensorMap& tx, const CUtensorM
                           ((a.M + kPairTileM - 1) / kPairTileM);
   const long long pairs = a.persistent && a.ctas / 2 < items ? a.ctas / 2 : items;
   return launch_ex_cluster_xy(standard_pair_kernel<kFmt>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads),
-                              pair_smem_bytes(a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, 2, 1, tx, tw, a);
+                              pair_smem_bytes(a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, 2, 1, tx, tw, ty, a);
 }
 
-cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
-                                 cudaStream_t stream) {
-  if (fmt == kFmtFP8) return launch_standard_pair_t<kFmtFP8>(tx, tw, a, stream);
-  if (fmt == kFmtINT8) return launch_standard_pair_t<kFmtINT8>(tx, tw, a, stream);
+cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                                 const GemmArgs& a, cudaStream_t stream) {
+  if (fmt == kFmtFP8) return launch_standard_pair_t<kFmtFP8>(tx, tw, ty, a, stream);
+  if (fmt == kFmtINT8) return launch_standard_pair_t<kFmtINT8>(tx, tw, ty, a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -78,8 +78,9 @@ cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, 
                           const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CUtensorMap& tw,
                             const GemmArgs& a, cudaStream_t stream);
-cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
-                                 cudaStream_t stream);
+// ty: the bf16 output as a tensor map (boxes of 32 rows x 64 columns, 128-byte swizzle)
+cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                                 const GemmArgs& a, cudaStream_t stream);
 int pair_max_active_clusters(int fmt, int stages, int kps);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);

@@ -322,7 +322,8 @@ def test_standard_pair_plan_rules():
             (qgd.VARIANT_STANDARD_PAIR, 256, 1, 2, 3, 1)
         assert qgd.qgd_workspace_size(fmt, 4096, 6144, 4096) == 0
         qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, G, 0, 1)
-        assert qgd.qgd_get_plan(fmt, 512, 6144, 4096)["stages"] == (232448 - 2048) // 32768
+        # one-block stages of 32 KB beside the 32 KB output staging area
+        assert qgd.qgd_get_plan(fmt, 512, 6144, 4096)["stages"] == (232448 - 2048 - 32768) // 32768
         qgd.qgd_set_override(fmt)
     # Block_FP8 and MXFP8 have no pair tiles
     qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, P)
