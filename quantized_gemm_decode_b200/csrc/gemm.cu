@@ -1522,13 +1522,17 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
 // tiles, and each CTA's tensor memory receives its 128 token rows x 256
 // weight columns.  Per CTA and K block that is 32 KB of operands for the
 // same 8.4 MFLOP a one-CTA 128 x 256 tile does with 48 KB: the L2-to-SM
-// traffic per FLOP -- what bounds the one-CTA kernel at large M -- drops by a
-// third.  Both CTAs' copies complete on the leader's `full` barrier (its
-// expect-tx counts both); the leader's commits arrive on `empty` / `tfull` in
-// both CTAs; both CTAs' epilogue warps hand the accumulator back on the
-// leader's `tempty`.  Work items are pair tiles, token-tile fastest, dealt
-// to the pairs round-robin.  A failed (bounded) wait in either CTA sets both
-// CTAs' abort flags.
+// traffic per FLOP, which bounds the one-CTA kernel at large M, drops by a
+// third.  The accumulator is double-buffered in all 512 TMEM columns, so the
+// epilogue of one tile overlaps the next tile's mainloop.  (A 256 x 512 tile,
+// two N = 256 halves sharing each X tile, cuts the traffic further but leaves
+// no second accumulator: measured slower on B200 at every larger-M shape,
+// the drain of each tile no longer hidden.)  Both CTAs' copies complete on
+// the leader's `full` barrier (its expect-tx counts both); the leader's
+// commits arrive on `empty` / `tfull` in both CTAs; both CTAs' epilogue warps
+// hand the accumulator back on the leader's `tempty`.  Work items are pair
+// tiles, token-tile fastest, dealt to the pairs round-robin.  A failed
+// (bounded) wait in either CTA sets both CTAs' abort flags.
 // ===========================================================================
 constexpr int kPairTileM = 256;  // tokens per pair tile (MMA M)
 constexpr int kPairTileN = 256;  // weight rows per pair tile (MMA N)
@@ -1695,79 +1699,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int li = 0;
     for (long long w = pair; w < items; w += npairs, ++li) {
       const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
-      const int buf = li & 1;
-      const bool ok = warp_wait(&ctl->tfull[buf], (li >> 1) & 1);
-      if (!ok && lane == 0) fail(kErrWaitEpilogue);
-      if (ok) tc_fence_after();
-      if (!epi_agree_ok(ctl)) break;
       const int row0 = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2) + q * 32;  // this warp's rows
       const int m = row0 + lane;
       const bool in_m = m < M;
       const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
-      const uint32_t tbuf = taddr + buf * kPairTileN;
+      {
+        const int buf = li & 1;
+        const bool ok = warp_wait(&ctl->tfull[buf], (li >> 1) & 1);
+        if (!ok && lane == 0) fail(kErrWaitEpilogue);
+        if (ok) tc_fence_after();
+        if (!epi_agree_ok(ctl)) break;
+        const uint32_t tbuf = taddr + buf * kPairTileN;
+        const int ncol0 = nt * kPairTileN;  // first weight column of the tile
+        // 64 columns at a time: four TMEM loads, one wait
 #pragma unroll 1
-      for (int c = 0; c < kPairTileN / 16; ++c) {
-        const int nc = nt * kPairTileN + c * 16;
-        uint32_t r[16];
-        __syncwarp();
-        tmem_ld16(tbuf + c * 16, r);
-        tmem_wait_ld();
-        if (c == kPairTileN / 16 - 1) {
-          // the whole accumulator row is in registers: hand the buffer back to the leader
-          tc_fence_before();
+        for (int grp = 0; grp < kPairTileN / 64; ++grp) {
+          const int nc0 = ncol0 + grp * 64;
+          uint32_t r[4][16];
           __syncwarp();
-          if (lane == 0) mbar_arrive_remote(tempty0 + static_cast<uint32_t>(buf) * 8u);
-        }
-        if (a.raw) {  // int32 accumulators (test hook): plain stores
-          if (!in_m || nc >= N) continue;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-          continue;
-        }
-        // columns nc .. nc + 15 of row m -> bf16, into the staging buffer of
-        // this 64-column group (the 16-byte chunk j of a row sits at j ^ (row % 8))
-        float sw16[16];
-        if (nc < N) {
-          const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 t4 = __ldg(swv + v);
-            sw16[4 * v] = t4.x;
-            sw16[4 * v + 1] = t4.y;
-            sw16[4 * v + 2] = t4.z;
-            sw16[4 * v + 3] = t4.w;
+          for (int g = 0; g < 4; ++g) tmem_ld16(tbuf + grp * 64 + g * 16, r[g]);
+          tmem_wait_ld();
+          if (grp == kPairTileN / 64 - 1) {
+            // the whole accumulator row is in registers: hand the buffer back to the leader
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(tempty0 + static_cast<uint32_t>(buf) * 8u);
           }
-        } else {
+          if (a.raw) {  // int32 accumulators (test hook): plain stores
+            if (in_m) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) sw16[j] = 0.f;
-        }
-        uint32_t pk[8];
+              for (int g = 0; g < 4; ++g) {
+                const int nc = nc0 + g * 16;
+                if (nc >= N) break;
+                uint4* dst =
+                    reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float v0, v1;
-          if constexpr (kInt) {
-            v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
-            v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
-          } else {
-            v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
-            v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(r[g][4 * v], r[g][4 * v + 1], r[g][4 * v + 2], r[g][4 * v + 3]);
+              }
+            }
+            continue;
           }
-          pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
-        }
-        const int g = c & 3;  // 16-column chunk within the 64-column group
-        uint8_t* sb = ybuf + (nstore & 1) * (32 * 128);
-        if (g == 0 && lane == 0 && nstore >= 2) bulk_wait_group_read<1>();  // this buffer's last store has read it
-        __syncwarp();
-        st_shared_v4(sb + lane * 128 + (((2 * g) ^ (lane & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
-        st_shared_v4(sb + lane * 128 + (((2 * g + 1) ^ (lane & 7)) << 4), make_uint4(pk[4], pk[5], pk[6], pk[7]));
-        if (g == 3) {
+          // row m, columns nc0 .. nc0 + 63 -> bf16 in a staging buffer (the
+          // 16-byte chunk j of a row sits at j ^ (row % 8)), then one tensor store
+          uint8_t* sb = ybuf + (nstore & 1) * (32 * 128);
+          if (lane == 0 && nstore >= 2) bulk_wait_group_read<1>();  // this buffer's last store has read it
+          __syncwarp();
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int nc = nc0 + g * 16;
+            float sw16[16];
+            if (nc < N) {
+              const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 t4 = __ldg(swv + v);
+                sw16[4 * v] = t4.x;
+                sw16[4 * v + 1] = t4.y;
+                sw16[4 * v + 2] = t4.z;
+                sw16[4 * v + 3] = t4.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sw16[j] = 0.f;
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float v0, v1;
+              if constexpr (kInt) {
+                v0 = (static_cast<float>(static_cast<int32_t>(r[g][2 * j])) * sxm) * sw16[2 * j];
+                v1 = (static_cast<float>(static_cast<int32_t>(r[g][2 * j + 1])) * sxm) * sw16[2 * j + 1];
+              } else {
+                v0 = (__uint_as_float(r[g][2 * j]) * sxm) * sw16[2 * j];
+                v1 = (__uint_as_float(r[g][2 * j + 1]) * sxm) * sw16[2 * j + 1];
+              }
+              pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+            }
+            st_shared_v4(sb + lane * 128 + (((2 * g) ^ (lane & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+            st_shared_v4(sb + lane * 128 + (((2 * g + 1) ^ (lane & 7)) << 4), make_uint4(pk[4], pk[5], pk[6], pk[7]));
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             // a group per buffer use, empty when the box lies wholly past M or N,
             // so that "one group still reading" always means the other buffer
-            if (row0 < M && nc - 48 < N) tma_store_2d(&ty, sb, nc - 48, row0);
+            if (row0 < M && nc0 < N) tma_store_2d(&ty, sb, nc0, row0);
             bulk_commit_group();
           }
           ++nstore;
@@ -2018,6 +2036,18 @@ cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorM
   return cudaErrorInvalidValue;
 }
 
+template <int kFmt>
+static int pair_clusters_t(cudaLaunchConfig_t& cfg) {
+  static bool done = false;
+  if (set_smem_attr(standard_pair_kernel<kFmt>, done) != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmt>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 // Pair clusters that fit on the GPU at once with this shared memory (0 if the
 // query fails): the persistent pair schedule launches no more than that.
 int pair_max_active_clusters(int fmt, int stages, int kps) {
@@ -2032,22 +2062,7 @@ int pair_max_active_clusters(int fmt, int stages, int kps) {
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  int n = 0;
-  cudaError_t e;
-  if (fmt == kFmtINT8) {
-    static bool done = false;
-    if ((e = set_smem_attr(standard_pair_kernel<kFmtINT8>, done)) != cudaSuccess) return 0;
-    e = cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmtINT8>, &cfg);
-  } else {
-    static bool done = false;
-    if ((e = set_smem_attr(standard_pair_kernel<kFmtFP8>, done)) != cudaSuccess) return 0;
-    e = cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmtFP8>, &cfg);
-  }
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return 0;
-  }
-  return n;
+  return fmt == kFmtINT8 ? pair_clusters_t<kFmtINT8>(cfg) : pair_clusters_t<kFmtFP8>(cfg);
 }
 
 cudaError_t launch_swapab(int fmt, int mpad, bool fused, const CUtensorMap& tw, const CUtensorMap& tx,

@@ -310,19 +310,19 @@ def test_standard_two_blocks_per_stage(fmt, plan, M, N, K):
 # cta_group::2): each CTA loads half the token rows and half the weight rows;
 # M = 40 leaves the second CTA's token rows all past M (zero-filled copies),
 # N = 528 a ragged last weight tile, K = 1152 an odd block count.
-PAIR_PLANS = [(GRID, 1), (GRID, 2), (PERSISTENT, 1), (PERSISTENT, 2)]
+PAIR_PLANS = [(GRID, 1, 256), (GRID, 2, 256), (PERSISTENT, 1, 256), (PERSISTENT, 2, 256)]
 
 
 @pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
-@pytest.mark.parametrize("plan", PAIR_PLANS, ids=[f"sch{p[0]}-k{p[1]}" for p in PAIR_PLANS])
+@pytest.mark.parametrize("plan", PAIR_PLANS, ids=[f"sch{p[0]}-k{p[1]}-t{p[2]}" for p in PAIR_PLANS])
 @pytest.mark.parametrize("M,N,K", [(256, 256, 512), (40, 528, 1152), (300, 1024, 128), (520, 784, 2048)])
 def test_standard_pair_tiles(fmt, plan, M, N, K):
-    sched, kps = plan
+    sched, kps, tile = plan
     case = Case(fmt, M, N, K, seed=M * 3 + N + K, outliers=True)
     yref, bound = _oracle(case)[:2]
-    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, sched, 0, kps)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, tile, sched, 0, kps)
     p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
-    assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"]) == (qgd.VARIANT_STANDARD_PAIR, 256, 1,
+    assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"]) == (qgd.VARIANT_STANDARD_PAIR, tile, 1,
                                                                         kps if K > 128 else 1)
     y1 = case.run()
     case.check_output(y1, yref, bound, f"{fmt} pair M={M} N={N} K={K} plan={p}")
@@ -338,12 +338,13 @@ def test_standard_pair_tiles(fmt, plan, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
-def test_standard_pair_persistent_many_tiles(fmt):
+@pytest.mark.parametrize("tile", [256])
+def test_standard_pair_persistent_many_tiles(fmt, tile):
     # 8 x 20 = 160 pair tiles: every pair walks several through the
     # double-buffered accumulator; sampled rows against the oracle
     M, N, K = 2048, 5120, 512
     case = Case(fmt, M, N, K, seed=77, outliers=True)
-    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, PERSISTENT, 0, 2)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, tile, PERSISTENT, 0, 2)
     y = bf16_to_f64(case.run())
     rows = np.unique(np.concatenate([np.arange(0, M, 61), [127, 128, 255, 256, M - 1]]))
     xsub = case.x[torch.from_numpy(rows)]
