@@ -1169,7 +1169,7 @@ __host__ __device__ constexpr int std_threads() {
   return kFmt == kFmtBlock ? 64 + 128 * kBlockEpiGroups : kGemmThreads;
 }
 
-template <int kFmt, int kTileN>
+template <int kFmt, int kTileN, int kKps>
 __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     standard_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                     const GemmArgs a) {
@@ -1189,9 +1189,11 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const int stages = a.stages;
-  // K blocks per pipeline stage (1 or 2): one full/empty hand-off and one
-  // MMA commit per stage, so two blocks per stage halve those per FLOP
-  const int kps = a.kps > 1 ? 2 : 1;
+  // K blocks per pipeline stage (1 or 2, a compile-time constant so that the
+  // stage loops are straight-line code): one full/empty hand-off and one MMA
+  // commit per stage, so two blocks per stage halve those per FLOP
+  static_assert(kKps == 1 || kKps == 2, "one or two K blocks per stage");
+  constexpr int kps = kKps;
   const uint32_t stage_x = kps * kXBytes, stage_w = kps * kWBytes;
   uint8_t* x_ring = base;
   uint8_t* w_ring = base + stages * stage_x;
@@ -1261,7 +1263,9 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
           }
           const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;  // K blocks in this stage
           mbar_arrive_expect_tx(&ctl->full[s], ns * (kXBytes + kWBytes));
-          for (int h = 0; h < ns; ++h) {
+#pragma unroll
+          for (int h = 0; h < kps; ++h) {
+            if (h >= ns) break;
             tma_load_2d(x_ring + s * stage_x + h * kXBytes, &tx, &ctl->full[s], (kt + h) * kTileK,
                         m_tile * kStdTileM, pol_x);
             tma_load_2d(w_ring + s * stage_w + h * kWBytes, &tw, &ctl->full[s], (kt + h) * kTileK,
@@ -1299,7 +1303,9 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             break;
           }
           const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;
-          for (int h = 0; h < ns; ++h) {
+#pragma unroll
+          for (int h = 0; h < kps; ++h) {
+            if (h >= ns) break;
             uint32_t d = tmem + buf * kTileN;
             if constexpr (kBlock) {
               // every K block accumulates into its own TMEM slot
@@ -2003,17 +2009,24 @@ static cudaError_t launch_swapab_f(int fmt, int mpad, const CUtensorMap& tw, con
   return cudaErrorInvalidValue;
 }
 
-template <int kFmt, int kTileN>
-static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+template <int kFmt, int kTileN, int kKps>
+static cudaError_t launch_standard_k(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
                                      cudaStream_t stream) {
   static bool attr_done = false;
-  cudaError_t e = set_smem_attr(standard_kernel<kFmt, kTileN>, attr_done);
+  cudaError_t e = set_smem_attr(standard_kernel<kFmt, kTileN, kKps>, attr_done);
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>((a.N + kTileN - 1) / kTileN) *
                           ((a.M + kStdTileM - 1) / kStdTileM) * a.splits;
   const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
-  return launch_ex(standard_kernel<kFmt, kTileN>, grid, dim3(std_threads<kFmt>()),
-                   standard_smem_bytes(kTileN, a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, tx, tw, a);
+  return launch_ex(standard_kernel<kFmt, kTileN, kKps>, grid, dim3(std_threads<kFmt>()),
+                   standard_smem_bytes(kTileN, a.stages, kKps), stream, a.pdl != 0, tx, tw, a);
+}
+
+template <int kFmt, int kTileN>
+static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& tw, const GemmArgs& a,
+                                     cudaStream_t stream) {
+  return a.kps > 1 ? launch_standard_k<kFmt, kTileN, 2>(tx, tw, a, stream)
+                   : launch_standard_k<kFmt, kTileN, 1>(tx, tw, a, stream);
 }
 
 template <int kFmt>
