@@ -71,6 +71,14 @@ def load_library(path: str) -> ctypes.CDLL:
     L.orc_quant_mx.argtypes = [P, lg, lg, P, P]
     L.orc_gemm_mx.restype = None
     L.orc_gemm_mx.argtypes = [P, P, P, P, lg, lg, lg, P, P]
+    L.orc_e2m1_decode.restype = ctypes.c_double
+    L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e2m1_encode.restype = ctypes.c_uint8
+    L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+    L.orc_quant_nv.restype = None
+    L.orc_quant_nv.argtypes = [P, lg, lg, P, P, P]
+    L.orc_gemm_nv.restype = None
+    L.orc_gemm_nv.argtypes = [P, P, P, P, P, P, lg, lg, lg, P, P]
     return L
 
 
@@ -208,6 +216,47 @@ def gemm_mx(xq, sx, wq, sw):
     y = np.empty((M, N), dtype=np.float64)
     bound = np.empty((M, N), dtype=np.float64)
     lib().orc_gemm_mx(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), _ptr(bound))
+    return y, bound
+
+
+def e2m1_decode(code: int) -> float:
+    return lib().orc_e2m1_decode(code)
+
+
+def e2m1_encode(v: float) -> int:
+    return lib().orc_e2m1_encode(float(v))
+
+
+def quant_nv(x):
+    """NVFP4: x [R, K] bf16, K % 16 == 0 -> (packed E2M1 codes [R, K/2], two per
+    byte with element 2i in the low nibble; E4M3 block scales [R, K/16]; fp32
+    row scales [R])."""
+    xb = _bf16_bits(x)
+    R, K = xb.shape
+    assert K % 16 == 0
+    q = np.empty((R, K // 2), dtype=np.uint8)
+    s = np.empty((R, K // 16), dtype=np.uint8)
+    g = np.empty((R,), dtype=np.float32)
+    lib().orc_quant_nv(_ptr(xb), R, K, _ptr(q), _ptr(s), _ptr(g))
+    return q, s, g
+
+
+def gemm_nv(xq, sx, gx, wq, sw, gw):
+    """NVFP4 product: Y [M, N] fp64 and bound from packed codes, block scales
+    and row scales of both operands."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.uint8)
+    gx = np.ascontiguousarray(gx, dtype=np.float32)
+    gw = np.ascontiguousarray(gw, dtype=np.float32)
+    M, K2 = xq.shape
+    N, _ = wq.shape
+    K = 2 * K2
+    assert sx.shape == (M, K // 16) and sw.shape == (N, K // 16) and gx.shape == (M,) and gw.shape == (N,)
+    y = np.empty((M, N), dtype=np.float64)
+    bound = np.empty((M, N), dtype=np.float64)
+    lib().orc_gemm_nv(_ptr(xq), _ptr(sx), _ptr(gx), _ptr(wq), _ptr(sw), _ptr(gw), M, N, K, _ptr(y), _ptr(bound))
     return y, bound
 
 

@@ -433,6 +433,162 @@ void orc_gemm_mx(const uint8_t *xq, const uint8_t *sx, const uint8_t *wq,
     }
 }
 
+/* ------------------------------------------------------------------ */
+/* NVFP4: E2M1 values, an E4M3 scale per 16 values along K, and an fp32 */
+/* second-level scale per row                                           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * A fifth format, the 4-bit one the pages list among vLLM's formats
+ * ("NVFP4").  The pages define no recipe; this oracle follows the format's
+ * published definition (4-bit E2M1 elements, one E4M3 scale per 16
+ * consecutive values along K, one fp32 scale above those) and the plainest
+ * reading for what the format leaves open, listed in the design notes:
+ *   - the fp32 scale is per row: per token for the activations (dynamic, as
+ *     the pages' FP8_Dynamic) and per output channel for the weights;
+ *   - row r with amax_r = max |x| (at least 1e-12f):
+ *       g_r  = fp32(amax_r / 2688)              (2688 = 6 * 448: the largest
+ *                                                E2M1 value times E4M3's)
+ *     block b of 16 with amax_b:
+ *       s_b  = E4M3(fp32(amax_b / fp32(6 * g_r)))       (round to nearest
+ *                                                even, saturate at 448)
+ *       d_b  = fp32(dec(s_b) * g_r)
+ *       code = E2M1(fp32(x / d_b))                (nearest even, saturate
+ *                                                at 6; +-0 when d_b is 0)
+ *   - storage: two codes per byte, element 2i in the low nibble of byte i.
+ * E2M1 (OCP Microscaling Formats v1.0, FP4): 1 sign bit, 2 exponent bits
+ * with bias 1, 1 mantissa bit, no infinities or NaN: magnitudes 0, 0.5
+ * (subnormal), 1, 1.5, 2, 3, 4, 6.  The sign of zero is kept.
+ */
+double orc_e2m1_decode(uint8_t code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 0x3;
+    int m = code & 0x1;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m / 2.0, 1 - 1); /* subnormal: 0.m * 2^(1-bias) */
+    else
+        v = ldexp(1.0 + (double)m / 2.0, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest E2M1 code to v; ties to the even mantissa; above 6 saturates. */
+uint8_t orc_e2m1_encode(double v)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0, lo = 0, hi, best;
+    double a = fabs(v), dlo, dhi;
+    if (a >= 6.0)
+        return (uint8_t)(sign | 0x7);
+    while (lo < 0x7 && orc_e2m1_decode((uint8_t)(lo + 1)) <= a)
+        lo++;
+    hi = (uint8_t)(lo + 1);
+    dlo = a - orc_e2m1_decode(lo);
+    dhi = orc_e2m1_decode(hi) - a;
+    if (dlo < dhi)
+        best = lo;
+    else if (dhi < dlo)
+        best = hi;
+    else
+        best = (lo % 2 == 0) ? lo : hi; /* an exact tie goes to the even mantissa */
+    return (uint8_t)(sign | best);
+}
+
+static float mul_rn_f32(float a, float b)
+{
+    return (float)((double)a * (double)b); /* exact in fp64, then one rounding */
+}
+
+/* x [rows, K] bf16 (K % 16 == 0) -> packed codes q [rows, K/2], E4M3 block
+ * scales s [rows, K/16], row scales g [rows]. */
+void orc_quant_nv(const uint16_t *x, long rows, long K, uint8_t *q, uint8_t *s, float *g)
+{
+    long r, b, k, nb = K / 16;
+    memset(q, 0, (size_t)(rows * K / 2));
+    for (r = 0; r < rows; r++) {
+        float amax = 0.0f, gr, six_g;
+        for (k = 0; k < K; k++) {
+            float a = fabsf(bf16_to_float(x[r * K + k]));
+            if (a > amax)
+                amax = a;
+        }
+        if (amax < ORC_AMAX_FLOOR)
+            amax = ORC_AMAX_FLOOR;
+        gr = div_rn_f32(amax, 2688.0f);
+        g[r] = gr;
+        six_g = mul_rn_f32(6.0f, gr);
+        for (b = 0; b < nb; b++) {
+            float bmax = 0.0f, d;
+            uint8_t sc;
+            for (k = 0; k < 16; k++) {
+                float a = fabsf(bf16_to_float(x[r * K + b * 16 + k]));
+                if (a > bmax)
+                    bmax = a;
+            }
+            sc = orc_e4m3_encode((double)div_rn_f32(bmax, six_g));
+            s[r * nb + b] = sc;
+            d = mul_rn_f32((float)orc_e4m3_decode(sc), gr);
+            for (k = 0; k < 16; k++) {
+                long i = b * 16 + k;
+                float xv = bf16_to_float(x[r * K + i]);
+                uint8_t c = (d == 0.0f) ? (uint8_t)(signbit(xv) ? 0x8 : 0x0)
+                                        : orc_e2m1_encode((double)div_rn_f32(xv, d));
+                q[r * (K / 2) + i / 2] |= (uint8_t)((i & 1) ? (c << 4) : c);
+            }
+        }
+    }
+}
+
+/* E2M1 code of element k of a packed row, as an integer number of halves. */
+static int64_t e2m1_halves(const uint8_t *row, long k)
+{
+    uint8_t c = (uint8_t)((k & 1) ? (row[k / 2] >> 4) : (row[k / 2] & 0xF));
+    return (int64_t)ldexp(orc_e2m1_decode(c), 1);
+}
+
+/* E4M3 scale as an integer number of 2^-9 units (every E4M3 value is one). */
+static int64_t e4m3_units(uint8_t code)
+{
+    return (int64_t)(orc_e4m3_decode(code) * 512.0);
+}
+
+/*
+ * NVFP4 product, exact: with codes in halves and scales in 2^-9 units every
+ * term of
+ *   y[m,n] = gx[m] gw[n] sum_b dec(sx[m,b]) dec(sw[n,b]) sum_{k in b} c_x c_w
+ * is an integer multiple of 2^-20 and the sum fits in int64 (at most
+ * 9216 * 229376^2 per block, 2^15 blocks would be 2^63.4; K <= 25600 gives
+ * 1600 blocks, under 2^60).  xq [M, K/2], sx [M, K/16], gx [M]; likewise w.
+ * bound (nullable) = sum |x^||w^|.
+ */
+void orc_gemm_nv(const uint8_t *xq, const uint8_t *sx, const float *gx, const uint8_t *wq,
+                 const uint8_t *sw, const float *gw, long M, long N, long K, double *y, double *bound)
+{
+    long n, nb = K / 16;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (n = 0; n < N; n++) {
+        long m, b, k;
+        for (m = 0; m < M; m++) {
+            int64_t tot = 0, totabs = 0;
+            double unit = ldexp((double)gx[m] * (double)gw[n], -20);
+            for (b = 0; b < nb; b++) {
+                int64_t blk = 0, blkabs = 0, sc;
+                for (k = b * 16; k < b * 16 + 16; k++) {
+                    int64_t p = e2m1_halves(xq + m * (K / 2), k) * e2m1_halves(wq + n * (K / 2), k);
+                    blk += p;
+                    blkabs += p < 0 ? -p : p;
+                }
+                sc = e4m3_units(sx[m * nb + b]) * e4m3_units(sw[n * nb + b]);
+                tot += blk * sc;
+                totabs += blkabs * sc;
+            }
+            y[m * N + n] = (double)tot * unit;
+            if (bound)
+                bound[m * N + n] = (double)totabs * unit;
+        }
+    }
+}
+
 /* Number of OpenMP threads the GEMMs above run on (1 without OpenMP). */
 int orc_num_threads(void)
 {

@@ -16,6 +16,7 @@ import oracle
 import test_oracle_codec as codec
 import test_oracle_gemm as gemm
 import test_oracle_mx as mx
+import test_oracle_nv as nv
 import test_oracle_quant as quant
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -55,6 +56,21 @@ MUTANTS = {
     "mx weight scale of the next block": ("(int)sw[n * nb + b] - 127);", "(int)sw[n * nb + (b + 1) % nb] - 127);"),
     "mx scales added to exponent bias once": ("double scale = ldexp(1.0, (int)sx[m * nb + b] - 127 +",
                                               "double scale = ldexp(1.0, (int)sx[m * nb + b] +"),
+    "e2m1 exponent bias 2": ("v = ldexp(1.0 + (double)m / 2.0, e - 1);", "v = ldexp(1.0 + (double)m / 2.0, e - 2);"),
+    "e2m1 ties to odd": ("best = (lo % 2 == 0) ? lo : hi;", "best = (lo % 2 == 0) ? hi : lo;"),
+    "e2m1 saturation loses sign": ("return (uint8_t)(sign | 0x7);", "return (uint8_t)0x7;"),
+    "nv row scale over 448": ("gr = div_rn_f32(amax, 2688.0f);", "gr = div_rn_f32(amax, 448.0f);"),
+    "nv block maximum over half the block": (
+        "for (k = 0; k < 16; k++) {\n                float a = fabsf(bf16_to_float(x[r * K + b * 16 + k]));",
+        "for (k = 0; k < 8; k++) {\n                float a = fabsf(bf16_to_float(x[r * K + b * 16 + k]));"),
+    # (the nibble order of the product alone is no mistake: swapping both
+    # operands' pairs inside a block leaves every block sum unchanged)
+    "nv nibble order of the codes": ("q[r * (K / 2) + i / 2] |= (uint8_t)((i & 1) ? (c << 4) : c);",
+                                     "q[r * (K / 2) + i / 2] |= (uint8_t)((i & 1) ? c : (c << 4));"),
+    "nv weight row scale dropped": ("double unit = ldexp((double)gx[m] * (double)gw[n], -20);",
+                                    "double unit = ldexp((double)gx[m], -20);"),
+    "nv weight block scale of the token": ("sc = e4m3_units(sx[m * nb + b]) * e4m3_units(sw[n * nb + b]);",
+                                           "sc = e4m3_units(sx[m * nb + b]) * e4m3_units(sw[m * nb + b]);"),
 }
 
 
@@ -89,6 +105,16 @@ def pin_suite():
     for shape in ((3, 17, 96), (1, 40, 256), (5, 8, 64)):
         mx.test_mx_gemm_matches_brute_force(*shape)
     mx.test_mx_gemm_scales_belong_to_their_own_block()
+    nv.test_e2m1_decode_matches_spec_table()
+    nv.test_e2m1_round_trip_midpoints_and_saturation()
+    for seed in (1, 2):
+        nv.test_row_and_block_scales_follow_ieee_fp32_and_torch_cast(seed)
+        nv.test_row_maximum_lands_on_six_with_scale_448(seed + 2)
+        nv.test_dequantized_error_within_half_an_e2m1_step(seed + 4)
+    nv.test_zero_row_zero_block_and_signed_zero()
+    for shape in ((3, 17, 64), (1, 40, 256), (5, 8, 512)):
+        nv.test_nv_gemm_matches_brute_force(*shape)
+    nv.test_nv_gemm_block_scales_belong_to_their_own_block()
 
 
 @pytest.fixture
