@@ -35,7 +35,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from quantized_gemm_decode_b200 import synth, workloads  # noqa: E402
-from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, W8A8_INT8  # noqa: E402
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, NVFP4, W8A8_INT8  # noqa: E402
 
 METRIC = "achieved HBM GB/s & TFLOP/s (fraction of roofline) per format, M=1..32"
 L2_BYTES = 126 * 1024 * 1024
@@ -60,6 +60,8 @@ def peaks():
 def path_bytes(fmt: str, M: int, N: int, K: int) -> int:
     """Algorithmic bytes of quantize+GEMM: bf16 X in, weight codes and scales,
     bf16 Y out (the intermediate activation codes are not counted)."""
+    if fmt == NVFP4:  # half a byte per weight value, an E4M3 byte per 16, an fp32 per row
+        return N * K // 2 + N * (K // 16) + 4 * N + 2 * M * K + 2 * M * N
     wscale = 4 * (N // 128) * (K // 128) if fmt == BLOCK_FP8 else (N * (K // 32) if fmt == MXFP8 else 4 * N)
     return N * K + 2 * M * K + wscale + 2 * M * N
 
@@ -187,7 +189,8 @@ class DecodeSet:
 
         self.qgd = qgd
         self.wl, self.fmt, self.device = wl, wl.fmt, device
-        self.fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}[wl.fmt]
+        self.fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3, NVFP4: 4}[wl.fmt]
+        self.block_scaled = wl.fmt in (MXFP8, NVFP4)  # no fused quantizer
         self.ms = list(wl.ms)
         self.host_w = {}
         self.weights = {}  # (N, K) -> list of (wq, sw) copies
@@ -197,16 +200,18 @@ class DecodeSet:
                 self.host_w[(N, K)] = w
             wd = w.to(device)
             if self.fmt == BLOCK_FP8:
-                wq, sw = qgd.quant_weight_block128(wd)
+                wt = qgd.quant_weight_block128(wd)
             elif self.fmt == MXFP8:
-                wq, sw = qgd.quant_mx(wd)
+                wt = qgd.quant_mx(wd)
+            elif self.fmt == NVFP4:
+                wt = qgd.quant_nv(wd)  # (codes, block scales, row scales)
             else:
-                wq, sw = qgd.quant_weight_per_channel(wd, qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
+                wt = qgd.quant_weight_per_channel(wd, qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
             del wd
             ncopies = len(self.ms)
             if per_call_rotation:
-                ncopies = max(ncopies, math.ceil(ROTATION_BYTES / (N * K)))
-            copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(ncopies - 1)]
+                ncopies = max(ncopies, math.ceil(ROTATION_BYTES / (N * K // (2 if self.fmt == NVFP4 else 1))))
+            copies = [wt] + [tuple(t.clone() for t in wt) for _ in range(ncopies - 1)]
             self.weights[(N, K)] = copies
         self.calls = []  # per (M, N, K): dict of buffers
         ws_need = 0
@@ -215,14 +220,20 @@ class DecodeSet:
                 x = synth.activations(M, K, wl.seed, outliers=wl.outliers)
                 xd = x.to(device)
                 qdt = torch.int8 if self.fmt == W8A8_INT8 else torch.float8_e4m3fn
-                xq = torch.empty((M, K), dtype=qdt, device=device)
-                if self.fmt == MXFP8:
+                gx = None
+                if self.fmt == NVFP4:
+                    xq = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+                    sx = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
+                    gx = torch.empty((M,), dtype=torch.float32, device=device)
+                elif self.fmt == MXFP8:
+                    xq = torch.empty((M, K), dtype=qdt, device=device)
                     sx = torch.empty((M, K // 32), dtype=torch.uint8, device=device)
                 else:
+                    xq = torch.empty((M, K), dtype=qdt, device=device)
                     sx = torch.empty((M, K // 128) if self.fmt == BLOCK_FP8 else (M,), dtype=torch.float32,
                                      device=device)
                 y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-                self.calls.append(dict(M=M, N=N, K=K, mi=mi, x=xd, x_host=x, xq=xq, sx=sx, y=y))
+                self.calls.append(dict(M=M, N=N, K=K, mi=mi, x=xd, x_host=x, xq=xq, sx=sx, gx=gx, y=y))
                 ws_need = max(ws_need, qgd.qgd_workspace_size(self.fmt_id, M, N, K),
                               0 if self.fmt == MXFP8 else qgd.qgd_layer_workspace_size(self.fmt_id, M, N, K))
         self.ws = qgd.Workspace(ws_need, device)
@@ -235,6 +246,8 @@ class DecodeSet:
             qgd.quant_act_group128(c["x"], xq=c["xq"], sx=c["sx"])
         elif self.fmt == MXFP8:
             qgd.quant_mx(c["x"], xq=c["xq"], sx=c["sx"])
+        elif self.fmt == NVFP4:
+            qgd.quant_nv(c["x"], q=c["xq"], s=c["sx"], g=c["gx"])
         else:
             qgd.quant_act_per_token(c["x"], qgd.QTYPE_INT8 if self.fmt == W8A8_INT8 else qgd.QTYPE_E4M3,
                                     xq=c["xq"], sx=c["sx"])
@@ -242,10 +255,13 @@ class DecodeSet:
     def gemm(self, c, copy_idx=None):
         qgd = self.qgd
         copies = self.weights[(c["N"], c["K"])]
-        wq, sw = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
+        wt = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
+        if self.fmt == NVFP4:
+            qgd.qlinear_nvfp4(c["xq"], c["sx"], c["gx"], *wt, y=c["y"], ws=self.ws)
+            return
         fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
               BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8}[self.fmt]
-        fn(c["xq"], c["sx"], wq, sw, y=c["y"], ws=self.ws)
+        fn(c["xq"], c["sx"], *wt, y=c["y"], ws=self.ws)
 
     def layer(self, c, copy_idx=None):
         """The layer call from bf16 activations (quantizer fused into the GEMM
@@ -256,8 +272,11 @@ class DecodeSet:
             self.gemm(c, copy_idx)
             return
         copies = self.weights[(c["N"], c["K"])]
-        wq, sw = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
-        self.qgd.qlinear_bf16(self.fmt_id, c["x"], wq, sw, y=c["y"], ws=self.ws)
+        wt = copies[(c["mi"] if copy_idx is None else copy_idx) % len(copies)]
+        if self.fmt == NVFP4:
+            self.qgd.qlinear_nvfp4_bf16(c["x"], *wt, y=c["y"], ws=self.ws)
+            return
+        self.qgd.qlinear_bf16(self.fmt_id, c["x"], *wt, y=c["y"], ws=self.ws)
 
     def step(self, gemm_only=False):
         for c in self.calls:
@@ -284,7 +303,7 @@ class DecodeSet:
         for two-pass Split-K, and (layer calls) the quantizer unless fused."""
         n = 0
         for c in self.calls:
-            get = self.qgd.qgd_get_plan if (gemm_only or self.fmt == MXFP8) else self.qgd.qgd_get_layer_plan
+            get = self.qgd.qgd_get_plan if (gemm_only or self.block_scaled) else self.qgd.qgd_get_layer_plan
             p = get(self.fmt_id, c["M"], c["N"], c["K"])
             n += (0 if gemm_only or p["fused"] else 1) + 1 + (1 if p["split_k"] > 1 and p["reduce"] == 1 else 0)
         return n
@@ -296,7 +315,7 @@ class DecodeSet:
         runs).  Returns the algorithmic bytes those launches must move."""
         b = 0
         for c in self.calls:
-            if self.fmt != MXFP8 and self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"]:
+            if not self.block_scaled and self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"]:
                 self.layer(c)
                 b += path_bytes(self.fmt, c["M"], c["N"], c["K"])
             else:
@@ -305,7 +324,7 @@ class DecodeSet:
         return b
 
     def fused_calls(self) -> int:
-        if self.fmt == MXFP8:
+        if self.block_scaled:
             return 0
         return sum(self.qgd.qgd_get_layer_plan(self.fmt_id, c["M"], c["N"], c["K"])["fused"] for c in self.calls)
 
@@ -394,6 +413,8 @@ def per_call_table(ds: DecodeSet, peak_gbs: float, reps: int = 20):
 
 def quant_bytes(fmt: str, M: int, K: int) -> int:
     """Algorithmic bytes of the activation quantizer: bf16 X in, codes and scales out."""
+    if fmt == NVFP4:  # half a byte per code, an E4M3 byte per 16, an fp32 per row
+        return 2 * M * K + M * K // 2 + M * (K // 16) + 4 * M
     scales = 4 * M * (K // 128) if fmt == BLOCK_FP8 else (M * (K // 32) if fmt == MXFP8 else 4 * M)
     return 2 * M * K + M * K + scales
 
@@ -520,9 +541,10 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict |
 def splitk_modes_table(device, ms=(1, 8, 32), reps: int = 10) -> list:
     """The Split-K reductions side by side: for each FP8_Dynamic decode shape
     and token count, the GEMM alone (a graph of calls over >= 3x L2 of weight
-    copies) at one split -- the shipped plan's if it splits, else 8 -- under
-    each reduction: atomic (zeroed accumulator + atomic adds, the pages'
-    scheme with fp32 partials), last arriving CTA, a second kernel, and the
+    copies) at one split -- the shipped plan's if it splits, else 8, rounded
+    down to a power of two so that every reduction takes it -- under each
+    reduction: atomic (zeroed accumulator + atomic adds, the pages' scheme
+    with fp32 partials), last arriving CTA, a second kernel, and the
     thread-block cluster.  Same tile, ring and K slices for all four."""
     import quantized_gemm_decode_b200 as qgd
     from quantized_gemm_decode_b200.tune import Problem
@@ -535,6 +557,7 @@ def splitk_modes_table(device, ms=(1, 8, 32), reps: int = 10) -> list:
             p = Problem(FP8_DYNAMIC, M, N, K, 1001, device)
             base = qgd.qgd_get_plan(0, M, N, K)
             split = base["split_k"] if (base["variant"] == 1 and base["schedule"] == 0 and base["split_k"] > 1) else 8
+            split = 1 << (split.bit_length() - 1)
             row = {"M": M, "N": N, "K": K, "split_k": split}
             for red, name in names.items():
                 qgd.qgd_set_override(0, qgd.VARIANT_SWAP_AB, split, red, 2, 0, qgd.SCHEDULE_GRID, 1, 2)
@@ -1052,7 +1075,7 @@ def main():
                              "frac": round(value / world / pk["hbm_gbs"], 4),
                              "quantizer": quantizer_summary(ds)}
         keep = ds
-        for wl2 in (workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE):
+        for wl2 in (workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE, workloads.NV_DECODE):
             ds2 = DecodeSet(wl2, device, per_call_rotation=True)
             fmts[wl2.fmt] = format_summary(ds2, args.steps, args.warmup, pk["hbm_gbs"])
             fmts[wl2.fmt]["quantizer"] = quantizer_summary(ds2)

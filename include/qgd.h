@@ -67,7 +67,13 @@ typedef enum {
   QGD_ERR_DEVICE = -6       /* current device is not an sm_100 part */
 } qgd_status;
 
-typedef enum { QGD_FMT_FP8_DYNAMIC = 0, QGD_FMT_W8A8_INT8 = 1, QGD_FMT_BLOCK_FP8 = 2, QGD_FMT_MXFP8 = 3 } qgd_format;
+typedef enum {
+  QGD_FMT_FP8_DYNAMIC = 0,
+  QGD_FMT_W8A8_INT8 = 1,
+  QGD_FMT_BLOCK_FP8 = 2,
+  QGD_FMT_MXFP8 = 3,
+  QGD_FMT_NVFP4 = 4
+} qgd_format;
 typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
 /* Standard: X is the MMA's A operand (128-token tiles).  Swap-AB: Y^T = W X^T, the weight rows fill
  * the MMA's 128-row slot and the tokens its N (16/32/64/128); up to 32 tokens for Block_FP8 and up
@@ -258,6 +264,52 @@ QGD_API qgd_status quant_act_mx(const void* x_bf16, int M, int K, int ldx, void*
 QGD_API qgd_status qlinear_mxfp8(const void* xq, const void* sx_e8m0, const void* wq, const void* sw_e8m0,
                                  void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------
+ * NVFP4, the 4-bit format the pages list among vLLM's ("NVFP4"): E2M1
+ * values (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one E4M3 scale per 16
+ * consecutive values of a row along K, and one fp32 scale per row -- per
+ * token for the activations (computed at run time, as FP8_Dynamic's) and
+ * per output channel for the weights.  For a row with
+ * amax = max(max |x|, 1e-12f):
+ *     g = amax / 2688                     (6 * 448: the largest E2M1 value
+ *                                          times the largest E4M3)
+ *     per block of 16 with maximum b:
+ *     s = e4m3(b / (6 g)),  d = dec(s) * g,  q = e2m1(x / d)   (q = +-0
+ *                                          where d is 0)
+ * each operation one IEEE fp32 round-to-nearest step; E4M3 and E2M1 round to
+ * nearest even and saturate.  Codes are packed two per byte, value 2i in the
+ * low nibble of byte i.  The GEMM multiplies in hardware (tcgen05.mma
+ * kind::mxf4nvf4 with E4M3 scale factors read from tensor memory, K = 64 per
+ * instruction) and the epilogue applies the row scales:
+ *     Y[m,n] = bf16( gx[m] gw[n] sum_b dec(sx[m,b]) dec(sw[n,b]) sum_{k in b} q_x q_w )
+ * ------------------------------------------------------------------- */
+
+/* NVFP4 quantizer: x_bf16 [rows,K] (rows ldx elements apart, ldx >= K, ldx %
+ * 8 == 0) -> q [rows][K/2] packed codes, s_e4m3 [rows][K/16] block scales,
+ * g [rows] fp32 row scales.  For activations (rows = M) and weights (rows =
+ * N).  Requires K % 16 == 0, K <= 65536; x 16-byte, q 8-byte and g 4-byte
+ * aligned. */
+QGD_API qgd_status quant_nvfp4(const void* x_bf16, int rows, int K, int ldx, void* q, void* s_e4m3, float* g,
+                               void* stream);
+
+/* NVFP4 GEMM: y_bf16 [M,N] from xq [M][K/2], sx_e4m3 [M][K/16], gx [M], wq
+ * [N][K/2], sw_e4m3 [N][K/16], gw [N].  Swap-AB kernel only: 0 <= M <= 64
+ * (more -> QGD_ERR_UNSUPPORTED); K % 256 == 0, N % 16 == 0; all pointers
+ * 16-byte aligned.  The block scales sit in tensor memory beside the
+ * accumulators, 32 columns per ring slot (at most 256 columns per CTA, which
+ * caps the ring depth).  Workspace as qlinear_fp8_dynamic (same plans; no
+ * two-pass reduction, whose requests take the last-arriving CTA). */
+QGD_API qgd_status qlinear_nvfp4(const void* xq, const void* sx_e4m3, const float* gx, const void* wq,
+                                 const void* sw_e4m3, const float* gw, void* y_bf16, int M, int N, int K, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* NVFP4 layer call: quant_nvfp4 of x_bf16 into the workspace, then
+ * qlinear_nvfp4.  Workspace: qgd_layer_workspace_size(QGD_FMT_NVFP4, ...);
+ * otherwise as the calls above. */
+QGD_API qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* wq, const void* sw_e4m3,
+                                      const float* gw, void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
+                                      void* stream);
+
 /* Test hook: the W8A8_INT8 mainloop and Split-K reduction of the plan in
  * force, writing the exact int32 accumulator acc[M][N] instead of Y. */
 QGD_API qgd_status qgd_w8a8_int8_acc32(const void* xq, const void* wq, int32_t* acc, int M, int N, int K, void* ws,
@@ -298,7 +350,7 @@ QGD_API size_t qgd_workspace_size(int fmt, int M, int N, int K);
 /* Load a dispatch table: a text file with one line per (format, N, K,
  * M-bucket) and '#' comments,
  *     fmt N K M_bucket variant split_k reduce stages tile_n schedule occupancy [k_slices]
- * fmt in {fp8_dynamic, w8a8_int8, block_fp8, mxfp8}; variant in {standard, swap_ab};
+ * fmt in {fp8_dynamic, w8a8_int8, block_fp8, mxfp8, nvfp4}; variant in {standard, swap_ab, standard_pair};
  * reduce in {last_cta, two_pass, atomic, cluster}; schedule in {grid, persistent};
  * stages/tile_n/occupancy/k_slices 0 (or k_slices absent) = default.
  * Replaces the table in force.  On

@@ -28,6 +28,7 @@ __all__ = [
     "SCHEDULE_GRID", "SCHEDULE_PERSISTENT",
     "quant_act_per_token", "quant_act_group128", "quant_weight_block128", "quant_weight_per_channel",
     "quant_act_per_token_strided", "quant_act_group128_strided", "quant_mx", "qlinear_mxfp8", "FMT_MXFP8",
+    "quant_nv", "qlinear_nvfp4", "qlinear_nvfp4_bf16", "FMT_NVFP4",
     "qlinear_fp8_dynamic", "qlinear_w8a8_int8", "qlinear_block_fp8", "qgd_w8a8_int8_acc32",
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
@@ -44,7 +45,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("QGD_LIBRARY") or os.path.join(_PKG, "libqgd.so")
 DEFAULT_TABLE = os.path.join(_PKG, "tables", "b200.tsv")
 
-FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8, FMT_MXFP8 = 0, 1, 2, 3
+FMT_FP8_DYNAMIC, FMT_W8A8_INT8, FMT_BLOCK_FP8, FMT_MXFP8, FMT_NVFP4 = 0, 1, 2, 3, 4
 QTYPE_E4M3, QTYPE_INT8 = 0, 1
 VARIANT_STANDARD, VARIANT_SWAP_AB, VARIANT_STANDARD_PAIR = 0, 1, 2
 REDUCE_LAST_CTA, REDUCE_TWO_PASS, REDUCE_ATOMIC, REDUCE_CLUSTER = 0, 1, 2, 3
@@ -106,6 +107,9 @@ def lib() -> ctypes.CDLL:
             "quant_act_mx": [P, I, I, I, P, P, P],
             "qlinear_mxfp8": [P, P, P, P, P, I, I, I, P, S, P],
             "qlinear_mxfp8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
+            "quant_nvfp4": [P, I, I, I, P, P, P, P],
+            "qlinear_nvfp4": [P, P, P, P, P, P, P, I, I, I, P, S, P],
+            "qlinear_nvfp4_bf16": [P, I, P, P, P, P, I, I, I, P, S, P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -235,6 +239,36 @@ def quant_mx(x: torch.Tensor, xq=None, sx=None, stream=None):
         sx = torch.empty((R, K // 32), dtype=torch.uint8, device=x.device)
     _check(lib().quant_act_mx(_ptr(x), R, K, ldx, _ptr(xq), _ptr(sx), _stream(stream)), "quant_act_mx")
     return xq, sx
+
+
+def quant_nv(x: torch.Tensor, q=None, s=None, g=None, stream=None):
+    """NVFP4 quantization: x bf16 [R, K] (K % 16 == 0) -> (packed E2M1 codes
+    uint8 [R, K/2], two per byte with value 2i in the low nibble; E4M3 block
+    scales uint8 [R, K/16], one per 16 values; fp32 row scales [R]).
+    Activations and weights alike; x may be a column slice of a wider matrix."""
+    ldx = _activation_rows(x)
+    R, K = x.shape
+    if q is None:
+        q = torch.empty((R, K // 2), dtype=torch.uint8, device=x.device)
+    if s is None:
+        s = torch.empty((R, K // 16), dtype=torch.uint8, device=x.device)
+    if g is None:
+        g = torch.empty((R,), dtype=torch.float32, device=x.device)
+    for t, name, shape, dt in ((q, "q", (R, K // 2), torch.uint8), (s, "s", (R, K // 16), torch.uint8),
+                               (g, "g", (R,), torch.float32)):
+        if not isinstance(t, torch.Tensor) or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() \
+                or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {shape}")
+    _check(lib().quant_nvfp4(_ptr(x), R, K, ldx, _ptr(q), _ptr(s), _ptr(g), _stream(stream)), "quant_nvfp4")
+    return q, s, g
+
+
+def _check_nv(q, s, g, rows, K, name):
+    for t, nm, shape, dt in ((q, name + "q", (rows, K // 2), torch.uint8), (s, "s" + name, (rows, K // 16), torch.uint8),
+                             (g, "g" + name, (rows,), torch.float32)):
+        if not isinstance(t, torch.Tensor) or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() \
+                or not t.is_cuda:
+            raise ValueError(f"{nm} must be a contiguous CUDA {dt} tensor of shape {shape}")
 
 
 def quant_weight_block128(w: torch.Tensor, wq=None, sw=None, stream=None):
@@ -420,6 +454,59 @@ def qlinear_mxfp8(xq, sx, wq, sw, y=None, ws=None, stream=None):
     wsp, wsn = _workspace(FMT_MXFP8, M, N, K, ws, xq.device)
     _check(lib().qlinear_mxfp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(y), M, N, K, ctypes.c_void_p(wsp), wsn,
                                _stream(stream)), "qlinear_mxfp8")
+    return y
+
+
+def qlinear_nvfp4(xq, sx, gx, wq, sw, gw, y=None, ws=None, stream=None):
+    """Y bf16 [M, N] from NVFP4 operands (quant_nv's outputs for X and W):
+    packed E2M1 codes, E4M3 block scales applied by the tensor core, fp32 row
+    scales applied in the epilogue."""
+    if not isinstance(xq, torch.Tensor) or xq.dim() != 2 or not isinstance(wq, torch.Tensor) or wq.dim() != 2:
+        raise ValueError("xq and wq must be 2-D packed uint8 tensors")
+    M, K = xq.shape[0], 2 * xq.shape[1]
+    N = wq.shape[0]
+    if 2 * wq.shape[1] != K:
+        raise ValueError(f"K mismatch: xq {tuple(xq.shape)} vs wq {tuple(wq.shape)} (two values per byte)")
+    _check_nv(xq, sx, gx, M, K, "x")
+    _check_nv(wq, sw, gw, N, K, "w")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    elif not isinstance(y, torch.Tensor) or y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) \
+            or not y.is_contiguous() or not y.is_cuda:
+        raise ValueError(f"y must be a contiguous CUDA bfloat16 tensor of shape {(M, N)}")
+    wsp, wsn = _workspace(FMT_NVFP4, M, N, K, ws, xq.device)
+    _check(lib().qlinear_nvfp4(_ptr(xq), _ptr(sx), _ptr(gx), _ptr(wq), _ptr(sw), _ptr(gw), _ptr(y), M, N, K,
+                               ctypes.c_void_p(wsp), wsn, _stream(stream)), "qlinear_nvfp4")
+    return y
+
+
+def qlinear_nvfp4_bf16(x: torch.Tensor, wq, sw, gw, y=None, ws=None, stream=None):
+    """NVFP4 layer call: x bf16 [M, K] quantized into the workspace, then the
+    GEMM against quant_nv's weight outputs (wq, sw, gw)."""
+    ldx = _activation_rows(x)
+    M, K = x.shape
+    if not isinstance(wq, torch.Tensor) or wq.dim() != 2:
+        raise ValueError("wq must be a 2-D packed uint8 tensor")
+    N = wq.shape[0]
+    _check_nv(wq, sw, gw, N, K, "w")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif not isinstance(y, torch.Tensor) or y.dtype != torch.bfloat16 or tuple(y.shape) != (M, N) \
+            or not y.is_contiguous() or not y.is_cuda:
+        raise ValueError(f"y must be a contiguous CUDA bfloat16 tensor of shape {(M, N)}")
+    need = qgd_layer_workspace_size(FMT_NVFP4, M, N, K)
+    if ws is None:
+        key = (x.device.index if x.device.index is not None else torch.cuda.current_device())
+        ws = _default_ws.get(key)
+        if ws is None:
+            ws = _default_ws[key] = Workspace(need, x.device)
+    if isinstance(ws, Workspace):
+        ws.ensure(need)
+        wsp, wsn = ws.buf.data_ptr(), ws.nbytes
+    else:
+        wsp, wsn = ws.data_ptr(), ws.numel() * ws.element_size()
+    _check(lib().qlinear_nvfp4_bf16(_ptr(x), ldx, _ptr(wq), _ptr(sw), _ptr(gw), _ptr(y), M, N, K,
+                                    ctypes.c_void_p(wsp), wsn, _stream(stream)), "qlinear_nvfp4_bf16")
     return y
 
 

@@ -164,6 +164,7 @@ int fmt_from_name(const std::string& s) {
   if (s == "w8a8_int8" || s == "int8") return kFmtINT8;
   if (s == "block_fp8" || s == "block") return kFmtBlock;
   if (s == "mxfp8" || s == "mx") return kFmtMX;
+  if (s == "nvfp4" || s == "nv") return kFmtNV;
   return -1;
 }
 
@@ -190,8 +191,11 @@ int reduce_from_name(const std::string& s) {
 
 // layer: the plan of a layer call from bf16 activations (the qlinear_*_bf16
 // entry points), the only calls that can fuse the activation quantizer.
+// K as the kernels count it: NVFP4 packs two values per byte
+int kernel_k(int fmt, int K) { return fmt == kFmtNV ? K / 2 : K; }
+
 qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
-  const int nkt = (K + kTileK - 1) / kTileK;
+  const int nkt = (kernel_k(fmt, K) + kTileK - 1) / kTileK;
   qgd_plan p;
   p.source = 0;
   p.fused = 0;
@@ -255,7 +259,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   }
   // Make the plan legal for this shape.  (MXFP8 runs in the Swap-AB kernel
   // only, up to 128 tokens, and has no two-pass reduction kernel.)
-  if (fmt == kFmtMX) {
+  if (fmt == kFmtMX || fmt == kFmtNV) {
     p.variant = kSwapAB;
     if (p.reduce == kTwoPass) p.reduce = kLastCta;
   }
@@ -299,7 +303,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   // the fused quantizer exists in the Swap-AB kernel only; its two-pass
   // reduction would need the activation scales in memory, so it takes the
   // last-arriving CTA instead
-  if (!layer || p.variant != kSwapAB || fmt == kFmtMX) p.fused = 0;
+  if (!layer || p.variant != kSwapAB || fmt == kFmtMX || fmt == kFmtNV) p.fused = 0;
   p.fused = p.fused ? 1 : 0;
   if (p.fused && p.reduce == kTwoPass) p.reduce = kLastCta;
   const int mpad = swap_mpad(M);
@@ -308,8 +312,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
                                                   : standard_max_stages(p.tile_n, p.k_slices);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
-  if (fmt == kFmtMX)
-    while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices) > kMxMaxCols) --p.stages;
+  if (fmt == kFmtMX || fmt == kFmtNV)
+    while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices, fmt) > kMxMaxCols) --p.stages;
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;
@@ -361,7 +365,7 @@ struct Exec {
 
 Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   Exec e;
-  const int nkt = (K + kTileK - 1) / kTileK;
+  const int nkt = (kernel_k(fmt, K) + kTileK - 1) / kTileK;
   e.mpad = swap_mpad(M);
   e.mstride = (M + 3) / 4 * 4;
   if (M <= 0) return e;
@@ -439,6 +443,9 @@ qgd_status check_shape(int fmt, int M, int N, int K) {
   if (fmt == kFmtMX && K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128 (K=%d)", K);
   if (fmt == kFmtMX && M > kMxMaxM)
     return fail(QGD_ERR_UNSUPPORTED, "MXFP8 covers at most %d tokens (M=%d)", kMxMaxM, M);
+  if (fmt == kFmtNV && K % 256 != 0) return fail(QGD_ERR_UNSUPPORTED, "NVFP4 needs K a multiple of 256 (K=%d)", K);
+  if (fmt == kFmtNV && M > kMxMaxM)
+    return fail(QGD_ERR_UNSUPPORTED, "NVFP4 covers at most %d tokens (M=%d)", kMxMaxM, M);
   if (static_cast<long long>(M) * N > (1LL << 31)) return fail(QGD_ERR_UNSUPPORTED, "M*N too large");
   return QGD_OK;
 }
@@ -452,9 +459,11 @@ std::atomic<float*> g_capture_sx{nullptr};
 // follows_memset: the caller has just enqueued a memset on `stream`, so the
 // GEMM is launched without a programmatic dependency (that relaxation is
 // defined between two kernels only).
+// NVFP4: sx / sw are the fp32 row scales, sx8 / sw8 the E4M3 block scales.
 qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float* sx, const uint16_t* xbf, int ldxb,
                          const void* wq, const float* sw, void* y, void* raw, int M, int N, int K, void* ws,
-                         size_t ws_bytes, void* stream, bool follows_memset) {
+                         size_t ws_bytes, void* stream, bool follows_memset, const uint8_t* sx8 = nullptr,
+                         const uint8_t* sw8 = nullptr) {
   qgd_status st;
   if ((st = check_device()) != QGD_OK) return st;
   if ((st = get_encoder()) != QGD_OK) return st;
@@ -481,7 +490,7 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
   }
   a.M = M;
   a.N = N;
-  a.K = K;
+  a.K = kernel_k(fmt, K);  // NVFP4: bytes of packed codes
   a.splits = p.split_k;
   a.reduce = p.reduce;
   a.stages = p.stages;
@@ -497,8 +506,8 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
   a.ldxb = ldxb;
   a.xq_out = fused ? static_cast<uint8_t*>(g_capture_xq.load()) : nullptr;
   a.sx_out = fused ? g_capture_sx.load() : nullptr;
-  a.sx8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sx) : nullptr;
-  a.sw8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sw) : nullptr;
+  a.sx8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sx) : fmt == kFmtNV ? sx8 : nullptr;
+  a.sw8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sw) : fmt == kFmtNV ? sw8 : nullptr;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
@@ -510,8 +519,8 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
     a.pdl = 0;  // the GEMM follows a memset, not a kernel
   }
   if (p.variant == kSwapAB) {
-    if ((st = encode_kmajor(&tw, wq, N, K, kSwapTileN)) != QGD_OK) return st;
-    if (!fused && (st = encode_kmajor(&tx, xq, M, K, ex.mpad)) != QGD_OK) return st;
+    if ((st = encode_kmajor(&tw, wq, N, a.K, kSwapTileN)) != QGD_OK) return st;
+    if (!fused && (st = encode_kmajor(&tx, xq, M, a.K, ex.mpad)) != QGD_OK) return st;
     e = launch_swapab(fmt, ex.mpad, fused, tw, tx, a, s);
   } else if (p.variant == kStandardPair) {
     // each CTA of a pair loads 128 token rows and 128 weight rows per K block
@@ -540,16 +549,19 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
 }
 
 qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, const float* sw, void* y, void* raw,
-                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream, bool follows_memset = false) {
+                    int M, int N, int K, void* ws, size_t ws_bytes, void* stream, bool follows_memset = false,
+                    const uint8_t* sx8 = nullptr, const uint8_t* sw8 = nullptr) {
   qgd_status st = check_shape(fmt, M, N, K);
   if (st != QGD_OK) return st;
   if (M == 0) return QGD_OK;
   if (!xq || !wq || (!y && !raw)) return fail(QGD_ERR_INVALID, "null operand pointer");
   if (!raw && (!sx || !sw)) return fail(QGD_ERR_INVALID, "null scale pointer");
-  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(raw) || !aligned16(sx) || !aligned16(sw))
+  if (fmt == kFmtNV && (!sx8 || !sw8)) return fail(QGD_ERR_INVALID, "null block-scale pointer");
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(raw) || !aligned16(sx) || !aligned16(sw) ||
+      !aligned16(sx8) || !aligned16(sw8))
     return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
   return run_gemm_plan(fmt, make_plan(fmt, M, N, K), xq, sx, nullptr, 0, wq, sw, y, raw, M, N, K, ws, ws_bytes,
-                       stream, follows_memset);
+                       stream, follows_memset, sx8, sw8);
 }
 
 // Workspace of a layer call from bf16 activations: the GEMM's own part first
@@ -561,7 +573,7 @@ qgd_status run_gemm(int fmt, const void* xq, const float* sx, const void* wq, co
 struct LayerWs {
   qgd_plan plan;
   Exec ex;
-  size_t xq_off = 0, sx_off = 0, total = 0;
+  size_t xq_off = 0, sx_off = 0, sb_off = 0, total = 0;
 };
 
 LayerWs layer_ws(int fmt, int M, int N, int K) {
@@ -571,26 +583,31 @@ LayerWs layer_ws(int fmt, int M, int N, int K) {
   l.total = l.ex.total;
   if (!l.plan.fused && M > 0) {
     l.xq_off = align256(l.total > kTicketBytes ? l.total : kTicketBytes);
-    l.sx_off = align256(l.xq_off + static_cast<size_t>(M) * K);
-    // scales: fp32 per row or per 1x128 group; MXFP8: one byte per 32 values
+    l.sx_off = align256(l.xq_off + static_cast<size_t>(M) * kernel_k(fmt, K));
+    // scales: fp32 per row or per 1x128 group; MXFP8: one byte per 32 values;
+    // NVFP4: fp32 per row, then (sb_off) one byte per 16 values
     const size_t nsx = fmt == kFmtBlock ? static_cast<size_t>(M) * (K / kTileK)
                        : fmt == kFmtMX  ? (static_cast<size_t>(M) * (K / 32) + 3) / 4
                                         : static_cast<size_t>(M);
     l.total = align256(l.sx_off + nsx * 4);
+    if (fmt == kFmtNV) {
+      l.sb_off = l.total;
+      l.total = align256(l.sb_off + static_cast<size_t>(M) * (K / 16));
+    }
   }
   return l;
 }
 
 qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const float* sw, void* y, int M, int N,
-                     int K, void* ws, size_t ws_bytes, void* stream) {
+                     int K, void* ws, size_t ws_bytes, void* stream, const uint8_t* sw8 = nullptr) {
   qgd_status st = check_shape(fmt, M, N, K);
   if (st != QGD_OK) return st;
   if (ldx < K || ldx % 8 != 0)
     return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
   if (K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be <= 65536", K);
   if (M == 0) return QGD_OK;
-  if (!x_bf16 || !wq || !sw || !y) return fail(QGD_ERR_INVALID, "null operand pointer");
-  if (!aligned16(x_bf16) || !aligned16(wq) || !aligned16(y) || !aligned16(sw))
+  if (!x_bf16 || !wq || !sw || !y || (fmt == kFmtNV && !sw8)) return fail(QGD_ERR_INVALID, "null operand pointer");
+  if (!aligned16(x_bf16) || !aligned16(wq) || !aligned16(y) || !aligned16(sw) || !aligned16(sw8))
     return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
   const LayerWs l = layer_ws(fmt, M, N, K);
   if (l.total > 0 && (!ws || ws_bytes < l.total))
@@ -605,12 +622,15 @@ qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const
   void* xq = wsb + l.xq_off;
   float* sx = reinterpret_cast<float*>(wsb + l.sx_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* sb = wsb + l.sb_off;  // NVFP4 block scales
   cudaError_t e = fmt == kFmtBlock ? launch_quant_group128(xb, M, K, ldx, static_cast<uint8_t*>(xq), sx, s)
                  : fmt == kFmtMX  ? launch_quant_mx(xb, M, K, ldx, static_cast<uint8_t*>(xq),
                                                     reinterpret_cast<uint8_t*>(sx), s)
+                 : fmt == kFmtNV  ? launch_quant_nv(xb, M, K, ldx, static_cast<uint8_t*>(xq), sb, sx, s)
                                   : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
   if (e != cudaSuccess) return cuda_fail(e, "activation quantizer launch");
-  return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false);
+  return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false,
+                       fmt == kFmtNV ? sb : nullptr, sw8);
 }
 
 // ---------------------------------------------------------------------------
@@ -709,6 +729,22 @@ qgd_status quant_act_mx(const void* x_bf16, int M, int K, int ldx, void* xq, voi
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_act_mx launch");
 }
 
+qgd_status quant_nvfp4(const void* x_bf16, int rows, int K, int ldx, void* q, void* s_e4m3, float* g, void* stream) {
+  if (rows < 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (rows=%d K=%d)", rows, K);
+  if (K % 16 != 0 || K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be a multiple of 16, at most 65536", K);
+  if (ldx < K || ldx % 8 != 0)
+    return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
+  if (rows == 0) return QGD_OK;
+  if (!x_bf16 || !q || !s_e4m3 || !g) return fail(QGD_ERR_INVALID, "null pointer");
+  if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(q) & 7u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(QGD_ERR_INVALID, "x must be 16-byte aligned, q 8-byte and g 4-byte aligned");
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  cudaError_t e = launch_quant_nv(static_cast<const uint16_t*>(x_bf16), rows, K, ldx, static_cast<uint8_t*>(q),
+                                  static_cast<uint8_t*>(s_e4m3), g, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "quant_nvfp4 launch");
+}
+
 qgd_status quant_weight_block128(const void* w_bf16, int N, int K, void* wq, float* sw, void* stream) {
   if (N <= 0 || K <= 0) return fail(QGD_ERR_INVALID, "sizes must be positive (N=%d K=%d)", N, K);
   if (N % 128 != 0 || K % 128 != 0) return fail(QGD_ERR_UNSUPPORTED, "N=%d and K=%d must be multiples of 128", N, K);
@@ -744,6 +780,18 @@ qgd_status qlinear_mxfp8(const void* xq, const void* sx_e8m0, const void* wq, co
     return fail(QGD_ERR_INVALID, "MXFP8 scale arrays must be 4-byte aligned");
   return run_gemm(kFmtMX, xq, static_cast<const float*>(sx_e8m0), wq, static_cast<const float*>(sw_e8m0), y_bf16,
                   nullptr, M, N, K, ws, ws_bytes, stream);
+}
+
+qgd_status qlinear_nvfp4(const void* xq, const void* sx_e4m3, const float* gx, const void* wq, const void* sw_e4m3,
+                         const float* gw, void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_gemm(kFmtNV, xq, gx, wq, gw, y_bf16, nullptr, M, N, K, ws, ws_bytes, stream, false,
+                  static_cast<const uint8_t*>(sx_e4m3), static_cast<const uint8_t*>(sw_e4m3));
+}
+
+qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* wq, const void* sw_e4m3, const float* gw,
+                              void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
+  return run_layer(kFmtNV, x_bf16, ldx, wq, gw, y_bf16, M, N, K, ws, ws_bytes, stream,
+                   static_cast<const uint8_t*>(sw_e4m3));
 }
 
 qgd_status qlinear_fp8_dynamic_bf16(const void* x_bf16, int ldx, const void* wq, const float* sw, void* y_bf16,

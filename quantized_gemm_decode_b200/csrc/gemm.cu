@@ -463,20 +463,24 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
                   const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
-  // MXFP8: the tensor core applies the E8M0 block scales, which the epilogue
-  // warps write into tensor memory stage by stage
+  // MXFP8 / NVFP4: the tensor core applies the block scales (E8M0 per 32 /
+  // E4M3 per 16 values), which the epilogue warps write into tensor memory
+  // stage by stage; NVFP4's operands are E2M1 codes, two per byte, and its K
+  // here counts bytes (K / 2 values), so a 128-byte slice holds 256 values
   constexpr bool kMX = (kFmt == kFmtMX);
+  constexpr bool kNV = (kFmt == kFmtNV);
+  constexpr bool kBS = kMX || kNV;
   // Block_FP8: a ring of per-K-block accumulators; otherwise one accumulator
   // per segment, double-buffered so the next segment's MMAs overlap the drain.
   constexpr int kSlots = kBlock ? 4 : 2;
   constexpr uint32_t kCols = kSlots * kMpad <= 32 ? 32 : (kSlots * kMpad <= 64 ? 64 : (kSlots * kMpad <= 128 ? 128 : 256));
   static_assert(!kBlock || kMpad <= 32, "Block_FP8 Swap-AB covers at most 32 tokens");
-  static_assert(!(kMX && kFused), "MXFP8 takes quantized activations");
+  static_assert(!(kBS && kFused), "the block-scaled formats take quantized activations");
   // MXFP8 scale-factor columns per ring slot: a 4-column group for the
   // weights (lane quadrant q reads column q), then one for the tokens (token m
   // in lane m % 32 of every quadrant, column m / 32; kSFB columns used)
   constexpr uint32_t kSFB = kMpad > 32 ? kMpad / 32 : 1;
-  constexpr uint32_t kSFSlot = kMxSlotCols;
+  constexpr uint32_t kSFSlot = kNV ? kNvSlotCols : kMxSlotCols;
   static_assert(kSFB <= 4, "token scales fit one 4-column group");
   // the epilogue walks the accumulator row in chunks of at most 32 token columns
   constexpr int kAcc = kMpad > 32 ? 32 : kMpad;
@@ -518,7 +522,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     ue = t0 + static_cast<long long>(blockIdx.y + 1) * nku / a.splits;
   }
   const int nk = static_cast<int>(ue - ub);
-  const uint32_t ncols = kMX ? mx_tmem_cols(kMpad, stages, kps) : kCols;
+  const uint32_t ncols = kBS ? mx_tmem_cols(kMpad, stages, kps, kFmt) : kCols;
   if (threadIdx.x == 0) QGD_STAMP(0);
 
   if (warp == 0 && lane == 0) {
@@ -628,7 +632,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int s = i % stages;
         const uint32_t round = i / stages;
         if (!mbar_wait(&ctl->full[s], round & 1) ||
-            ((kFused || kMX) && !mbar_wait(&ctl->xfull[s], round & 1))) {
+            ((kFused || kBS) && !mbar_wait(&ctl->xfull[s], round & 1))) {
           record_error(kErrWaitMma);
           ctl->abort_flag = 1;
           break;
@@ -659,11 +663,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           }
           tc_fence_after();
           const uint32_t d = tmem + slot * kMpad;
-          // MXFP8: this slot's scale-factor columns.  Both groups start on a
-          // multiple of 4 columns (by construction; checked, so that a mistake
-          // aborts the CTA instead of faulting)
+          // MXFP8 / NVFP4: this slot's scale-factor columns.  Every group
+          // starts on a multiple of 4 columns (by construction; checked, so
+          // that a mistake aborts the CTA instead of faulting)
           const uint32_t sfa = tmem + 2 * kMpad + static_cast<uint32_t>(s * kps + j) * kSFSlot;
-          if (kMX && (sfa & 3u) != 0u) {
+          if (kBS && (sfa & 3u) != 0u) {
             record_error(kErrBadOperand);
             ctl->abort_flag = 1;
             stop = true;
@@ -678,6 +682,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
               const uint32_t sel = static_cast<uint32_t>(kk) << 30;  // the 32-wide K block's byte
               mma_issue_mx(d, ad, bd, idesc_mx(kSwapTileN, kMpad, kk, kk), sfa | sel, (sfa + 4) | sel,
                            accumulate);
+            } else if constexpr (kNV) {
+              // 64 values per MMA: weight-scale group kk, token-scale group 4 + kk
+              mma_issue_nv(d, ad, bd, idesc_nv(kSwapTileN, kMpad), sfa + 4 * kk, sfa + 16 + 4 * kk, accumulate);
             } else {
               mma_issue<kInt>(d, ad, bd, kIdesc, accumulate);
             }
@@ -706,7 +713,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const int M = a.M, N = a.N;
     const int KB = a.K / kTileK;
     const int nvec = (M + 3) / 4;  // float4 groups of the M accumulators
-    const bool scaled = (kFmt != kFmtBlock) && !kMX && !a.raw;
+    const bool scaled = (kFmt != kFmtBlock) && !kMX && !a.raw;  // NVFP4: the fp32 row scales
     const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 among the epilogue threads
     if constexpr (kFused && !kBlock) {
       // per-token scales: every CTA takes each row's maximum over all of K
@@ -753,7 +760,59 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     int qnext = 0, qslice = 0;
     bool qdead = false;
     auto quant_until = [&](int limit) {
-      if constexpr (kMX) {
+      if constexpr (kNV) {
+        // NVFP4: each stage's E4M3 block scales into its tensor-memory slot
+        // once the MMA has released the stage: per K slice (256 values) four
+        // MMAs, each reading one 4-column group of weight scales (lane
+        // quadrant q in column q; a word = the 4 blocks of 16 of its 64
+        // values) and one of token scales (token m in lane m % 32 of every
+        // quadrant, column m / 32)
+        if (limit > nk) limit = nk;
+        const int KB16 = a.K / 8;  // block scales per row: (2 K) / 16
+        for (; qnext < limit && !qdead; ++qnext) {
+          const int s = qnext % stages;
+          const uint32_t round = qnext / stages;
+          if (*reinterpret_cast<volatile int*>(&ctl->abort_flag) || !warp_wait(&ctl->empty[s], (round & 1) ^ 1)) {
+            if (lane == 0) {
+              record_error(kErrWaitEpilogue);
+              ctl->abort_flag = 1;
+            }
+            qdead = true;
+            break;
+          }
+          const long long u = ub + qnext;
+          const int t = static_cast<int>(u / nku);
+          const int k0 = static_cast<int>(u % nku) * kps;
+          const int ns = (nkt - k0) < kps ? (nkt - k0) : kps;
+          tc_fence_after();
+          const uint32_t lanes = static_cast<uint32_t>(q * 32) << 16;
+          const int n = t * kSwapTileN + q * 32 + lane;
+          for (int j = 0; j < ns; ++j) {
+            const uint32_t col = 2 * kMpad + static_cast<uint32_t>(s * kps + j) * kSFSlot;
+            const int b0 = (k0 + j) * 16;  // first block of 16 of the slice
+            const uint4 wsf = n < N ? __ldg(reinterpret_cast<const uint4*>(a.sw8 + static_cast<size_t>(n) * KB16 + b0))
+                                    : make_uint4(0, 0, 0, 0);
+            tmem_st32(tmem + lanes + col + 0 + q, wsf.x);
+            tmem_st32(tmem + lanes + col + 4 + q, wsf.y);
+            tmem_st32(tmem + lanes + col + 8 + q, wsf.z);
+            tmem_st32(tmem + lanes + col + 12 + q, wsf.w);
+#pragma unroll
+            for (uint32_t w = 0; w < kSFB; ++w) {
+              const int m = static_cast<int>(w) * 32 + lane;
+              const uint4 xsf = m < M ? __ldg(reinterpret_cast<const uint4*>(a.sx8 + static_cast<size_t>(m) * KB16 + b0))
+                                      : make_uint4(0, 0, 0, 0);
+              tmem_st32(tmem + lanes + col + 16 + w, xsf.x);
+              tmem_st32(tmem + lanes + col + 20 + w, xsf.y);
+              tmem_st32(tmem + lanes + col + 24 + w, xsf.z);
+              tmem_st32(tmem + lanes + col + 28 + w, xsf.w);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->xfull[s]);
+        }
+      } else if constexpr (kMX) {
         // MXFP8: write each stage's block scales into its tensor-memory slot
         // once the MMA has released the stage (its empty barrier)
         if (limit > nk) limit = nk;
@@ -2003,6 +2062,14 @@ static cudaError_t launch_swapab_f(int fmt, int mpad, const CUtensorMap& tw, con
         case 32: return launch_swapab_t<kFmtMX, 32, false>(tw, tx, a, stream);
         case 64: return launch_swapab_t<kFmtMX, 64, false>(tw, tx, a, stream);
         case 128: return launch_swapab_t<kFmtMX, 128, false>(tw, tx, a, stream);
+      }
+    }
+  } else if (fmt == kFmtNV) {
+    if constexpr (!kFused) {
+      switch (mpad) {
+        case 16: return launch_swapab_t<kFmtNV, 16, false>(tw, tx, a, stream);
+        case 32: return launch_swapab_t<kFmtNV, 32, false>(tw, tx, a, stream);
+        case 64: return launch_swapab_t<kFmtNV, 64, false>(tw, tx, a, stream);
       }
     }
   }

@@ -8,8 +8,8 @@
 
 namespace qgd {
 
-enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2, kFmtMX = 3 };
-constexpr int kNumFmts = 4;
+enum Fmt : int { kFmtFP8 = 0, kFmtINT8 = 1, kFmtBlock = 2, kFmtMX = 3, kFmtNV = 4 };
+constexpr int kNumFmts = 5;
 // kStandardPair: Standard tiles of 256 x 256 computed by a CTA pair (FP8_Dynamic, W8A8_INT8)
 enum Variant : int { kStandard = 0, kSwapAB = 1, kStandardPair = 2 };
 enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2, kCluster = 3 };
@@ -29,8 +29,8 @@ inline size_t smem_budget() { return kSmemBudget; }
 
 // Runtime arguments common to both GEMM orientations.
 struct GemmArgs {
-  const float* sx;      // FP8/INT8: [M]; Block: [M][K/128]
-  const float* sw;      // FP8/INT8: [N]; Block: [N/128][K/128]
+  const float* sx;      // FP8/INT8: [M]; Block: [M][K/128]; NVFP4: the fp32 row scales [M]
+  const float* sw;      // FP8/INT8: [N]; Block: [N/128][K/128]; NVFP4: [N]
   uint16_t* y;          // bf16 [M][N]
   void* raw;            // when non-null: fp32/int32 accumulator [M][N] instead of y
   void* partial;        // Split-K partials, 4-byte [splits][M][N]
@@ -54,19 +54,24 @@ struct GemmArgs {
   int ldxb;
   uint8_t* xq_out;      // test capture (may be null): the codes [M][K] the kernel made
   float* sx_out;        // test capture (may be null): their scales, [M] or [M][K/128]
-  // MXFP8: E8M0 block-scale bytes, one per 32 values along K
-  const uint8_t* sx8;  // [M][K/32]
-  const uint8_t* sw8;  // [N][K/32]
+  // MXFP8: E8M0 block-scale bytes, one per 32 values along K ([M][K/32],
+  // [N][K/32]); NVFP4: E4M3 block-scale bytes, one per 16 ([M][K/16],
+  // [N][K/16]; the kernel's K then counts the packed bytes, K/2)
+  const uint8_t* sx8;
+  const uint8_t* sw8;
 };
 
-// Tensor-memory columns of the MXFP8 Swap-AB kernel: two accumulators of mpad
-// columns, then per ring slot (stage, K slice) a group of 4 columns of weight
-// scales and a group of 4 of token scales (a scale-factor operand spans a
-// 4-column, 128-bit group and starts on a multiple of 4); rounded up to a
-// power of two.
+// Tensor-memory columns of the block-scaled Swap-AB kernels: two accumulators
+// of mpad columns, then per ring slot (stage, K slice) the slice's scale
+// factors, in 4-column, 128-bit groups that each start on a multiple of 4:
+// MXFP8 one group of weight scales and one of token scales (the slice's four
+// MMAs each pick one byte of a word); NVFP4 a group of each per MMA (an MMA
+// of 64 values reads all four bytes, one per 16).  Rounded up to a power of two.
 constexpr unsigned kMxSlotCols = 8;
-__host__ __device__ inline unsigned mx_tmem_cols(int mpad, int stages, int kps) {
-  const unsigned need = 2u * mpad + static_cast<unsigned>(stages * kps) * kMxSlotCols;
+constexpr unsigned kNvSlotCols = 32;
+__host__ __device__ inline unsigned slot_cols(int fmt) { return fmt == kFmtNV ? kNvSlotCols : kMxSlotCols; }
+__host__ __device__ inline unsigned mx_tmem_cols(int mpad, int stages, int kps, int fmt = kFmtMX) {
+  const unsigned need = 2u * mpad + static_cast<unsigned>(stages * kps) * slot_cols(fmt);
   unsigned c = 32;
   while (c < need) c *= 2;
   return c;
@@ -107,6 +112,10 @@ cudaError_t launch_quant_group128(const uint16_t* x, int M, int K, int ldx, uint
                                   cudaStream_t stream);
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream);
 // MXFP8: rows of 32-value blocks -> e4m3 codes q [rows][K], E8M0 bytes s [rows][K/32]
+// NVFP4 rows: q [rows][K/2] packed E2M1 codes, s [rows][K/16] E4M3 block
+// scales, g [rows] fp32 row scales
+cudaError_t launch_quant_nv(const uint16_t* x, int rows, int K, int ldx, uint8_t* q, uint8_t* s, float* g,
+                            cudaStream_t stream);
 cudaError_t launch_quant_mx(const uint16_t* x, int rows, int K, int ldx, uint8_t* q, uint8_t* s,
                             cudaStream_t stream);
 

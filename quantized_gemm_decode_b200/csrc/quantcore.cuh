@@ -10,6 +10,7 @@
 // the search space".
 #pragma once
 
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -85,6 +86,43 @@ __device__ __forceinline__ uint2 encode8_mx(const uint4& v, float inv) {
   out.x = e4m3x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv) | (e4m3x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv) << 16);
   out.y = e4m3x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv) | (e4m3x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv) << 16);
   return out;
+}
+
+// NVFP4: E2M1 values (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one E4M3 scale
+// per 16 values along K and an fp32 scale per row.  For a row with
+// amax = max(max|x|, 1e-12f):  g = amax / 2688 (6 * 448, the largest E2M1
+// value times E4M3's);  per block of 16 with maximum b:  s = e4m3(b / (6 g)),
+// d = dec(s) * g,  code = e2m1(x / d) (+-0 when d is 0); every operation is
+// one IEEE fp32 round-to-nearest step, E4M3 and E2M1 round to nearest even
+// and saturate.  Two codes per byte, element 2i in the low nibble.
+constexpr float kNvRowDiv = 2688.0f;
+
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest));
+}
+
+// Value of an E4M3 code (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// 16 bf16 values (two uint4) of one block -> 16 E2M1 codes in a uint2, given
+// the block's fp32 divisor d (d == 0: every code +-0, keeping the sign).
+__device__ __forceinline__ uint2 encode16_nv(const uint4& v0, const uint4& v1, float d) {
+  const float f[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y), bf16_lo(v0.z), bf16_hi(v0.z),
+                       bf16_lo(v0.w), bf16_hi(v0.w), bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
+                       bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (d == 0.f) {
+      b[i] = ((__float_as_uint(f[2 * i]) >> 31) << 3) | ((__float_as_uint(f[2 * i + 1]) >> 31) << 7);
+    } else {
+      b[i] = e2m1x2(__fdiv_rn(f[2 * i], d), __fdiv_rn(f[2 * i + 1], d));
+    }
+  }
+  return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24), b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
 }
 
 // Maximum over the 32 lanes of a warp.

@@ -335,6 +335,25 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4.block_scale with
+// 16-value blocks: E2M1 x E2M1 -> f32, both K-major, E4M3 scale factors, K = 64
+// per instruction; an instruction reads all four bytes of its scale words
+// (scale-factor ids 0).
+__host__ __device__ constexpr uint32_t idesc_nv(uint32_t m, uint32_t n) {
+  return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (0u << 23) | ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_issue_nv(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
 // Each lane of a warp writes one 32-bit word into its TMEM lane (the warp's
 // lane quadrant) at the address's column.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, uint32_t v) {

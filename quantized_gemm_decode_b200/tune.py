@@ -36,27 +36,33 @@ import torch
 
 import quantized_gemm_decode_b200 as qgd
 from quantized_gemm_decode_b200 import synth, workloads
-from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, W8A8_INT8
+from quantized_gemm_decode_b200.workloads import BLOCK_FP8, FP8_DYNAMIC, MXFP8, NVFP4, W8A8_INT8
 
 L2_BYTES = 126 * 1024 * 1024
-FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3}
+FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3, NVFP4: 4}
 VAR_NAME = {0: "standard", 1: "swap_ab", 2: "standard_pair"}
 RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
 
 
 def _quant_w(fmt, w):
+    """The weight operand tuple the GEMM takes: (wq, sw), or NVFP4's (wq, sw, gw)."""
     if fmt == BLOCK_FP8:
         return qgd.quant_weight_block128(w)
     if fmt == MXFP8:
         return qgd.quant_mx(w)
+    if fmt == NVFP4:
+        return qgd.quant_nv(w)
     return qgd.quant_weight_per_channel(w, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
 
 
 def _quant_x(fmt, x):
+    """The activation operand tuple: (xq, sx), or NVFP4's (xq, sx, gx)."""
     if fmt == BLOCK_FP8:
         return qgd.quant_act_group128(x)
     if fmt == MXFP8:
         return qgd.quant_mx(x)
+    if fmt == NVFP4:
+        return qgd.quant_nv(x)
     return qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
 
 
@@ -92,7 +98,7 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148, fused: bool
     SM; a Swap-AB grid of at most one CTA per SM is tried at the deepest ring and at that shallower
     one (which leaves room for the next layer's CTAs to start streaming beside it).  At decode token
     counts every Swap-AB candidate is also tried with the activation quantizer fused in."""
-    if fmt == MXFP8:
+    if fmt in (MXFP8, NVFP4):
         # the Swap-AB kernel only, no two-pass reduction, no fused quantizer
         return [c + (0,) for c in _candidates(fmt, M, N, K, num_sms, False) if c[0] == 1 and c[2] != 1]
     if fused and M <= 32:
@@ -104,7 +110,7 @@ def candidates(fmt: str, M: int, N: int, K: int, num_sms: int = 148, fused: bool
 
 
 def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
-    nkt = (K + 127) // 128
+    nkt = ((K // 2 if fmt == NVFP4 else K) + 127) // 128  # 128-byte K slices (NVFP4: two values per byte)
     n_tiles = (N + 127) // 128
     splits = [s for s in (1, 2, 4, 8, 16, 32, 64, 128, 256) if s <= nkt]
     out = []
@@ -170,30 +176,33 @@ class Problem:
         self.fmt, self.M, self.N, self.K = fmt, M, N, K
         self.fid = FMT_ID[fmt]
         w = synth.weights(N, K, seed).to(device)
-        wq, sw = _quant_w(fmt, w)
+        wt = _quant_w(fmt, w)
         del w
-        ncopies = max(2, math.ceil(3 * L2_BYTES / (N * K)))
-        self.copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(ncopies - 1)]
+        wbytes = N * K // 2 if fmt == NVFP4 else N * K
+        ncopies = max(2, math.ceil(3 * L2_BYTES / wbytes))
+        self.copies = [wt] + [tuple(t.clone() for t in wt) for _ in range(ncopies - 1)]
         x = synth.activations(M, K, seed, outliers=(fmt != W8A8_INT8)).to(device)
         self.x = x
-        self.xq, self.sx = _quant_x(fmt, x)
+        self.xt = _quant_x(fmt, x)
+        self.xq, self.sx = self.xt[0], self.xt[1]
         self.y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
         self.ws = qgd.Workspace(0, device)
         self.fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
-                   BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8}[fmt]
+                   BLOCK_FP8: qgd.qlinear_block_fp8, MXFP8: qgd.qlinear_mxfp8, NVFP4: qgd.qlinear_nvfp4}[fmt]
 
     def run(self, j=0):
-        wq, sw = self.copies[j % len(self.copies)]
-        return self.fn(self.xq, self.sx, wq, sw, y=self.y, ws=self.ws)
+        return self.fn(*self.xt, *self.copies[j % len(self.copies)], y=self.y, ws=self.ws)
 
     def layer_call(self, j=0):
         """What the layer runs per call: the layer call from bf16 activations
         (quantizer kernel + GEMM, or one fused kernel, as the layer plan says)."""
-        wq, sw = self.copies[j % len(self.copies)]
-        if self.fmt == MXFP8:  # no layer call: the quantizer kernel, then the GEMM
+        wt = self.copies[j % len(self.copies)]
+        if self.fmt == MXFP8:  # the quantizer kernel, then the GEMM
             qgd.quant_mx(self.x, xq=self.xq, sx=self.sx)
             return self.run(j)
-        return qgd.qlinear_bf16(self.fid, self.x, wq, sw, y=self.y, ws=self.ws)
+        if self.fmt == NVFP4:
+            return qgd.qlinear_nvfp4_bf16(self.x, *wt, y=self.y, ws=self.ws)
+        return qgd.qlinear_bf16(self.fid, self.x, *wt, y=self.y, ws=self.ws)
 
     def acc32(self):
         return qgd.qgd_w8a8_int8_acc32(self.xq, self.copies[0][0], ws=self.ws)
@@ -285,7 +294,7 @@ def tune_problem(p: Problem, log=None):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--formats", default="fp8_dynamic,w8a8_int8,block_fp8,mxfp8")
+    ap.add_argument("--formats", default="fp8_dynamic,w8a8_int8,block_fp8,mxfp8,nvfp4")
     ap.add_argument("--out", default=qgd.DEFAULT_TABLE)
     ap.add_argument("--large-m", action="store_true", help="also tune the larger-M buckets")
     ap.add_argument("--resume", action="store_true")

@@ -12,7 +12,8 @@ FP8_DYNAMIC = "fp8_dynamic"
 W8A8_INT8 = "w8a8_int8"
 BLOCK_FP8 = "block_fp8"
 MXFP8 = "mxfp8"
-FORMATS = (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)  # the three formats of the method; MXFP8 is the Blackwell addition
+NVFP4 = "nvfp4"
+FORMATS = (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)  # the three formats of the method; MXFP8 and NVFP4 are additions
 
 DECODE_M = (1, 2, 4, 8, 16, 24, 32)
 LARGE_M = (64, 128, 512, 2048, 8192)
@@ -55,7 +56,10 @@ LARGE = tuple(
              f"{fmt}, 8B-class shapes x M in 64..8192")
     for fmt in FORMATS)
 
-ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE, MX_DECODE) + LARGE
+NV_DECODE = Workload("nvfp4_decode_sweep_8b_shapes", NVFP4, SHAPES_8B, DECODE_M, 1006, True,
+                     "NVFP4 (E2M1 values, E4M3 scale per 16 along K, fp32 per row), 8B-class shapes x M in 1..32, "
+                     "1% x20 outlier channels")
+ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE, MX_DECODE, NV_DECODE) + LARGE
 
 
 def algorithmic_bytes(fmt: str, M: int, N: int, K: int) -> int:
@@ -65,6 +69,9 @@ def algorithmic_bytes(fmt: str, M: int, N: int, K: int) -> int:
         scales = 4 * (N // 128) * (K // 128) + 4 * M * (K // 128)
     elif fmt == MXFP8:
         scales = N * (K // 32) + M * (K // 32)  # one E8M0 byte per 32 values
+    elif fmt == NVFP4:
+        # half a byte per value, one E4M3 byte per 16, an fp32 per row
+        return (N * K + M * K) // 2 + (N + M) * (K // 16) + 4 * (N + M) + 2 * M * N
     else:
         scales = 4 * N + 4 * M
     return N * K + M * K + scales + 2 * M * N

@@ -376,7 +376,9 @@ def test_table_cluster_reduce_name(tmp_path):
                                        ("block_fp8", 32, 5120, 25600), ("fp8_dynamic", 512, 6144, 4096),
                                        ("fp8_dynamic", 64, 24576, 4096), ("w8a8_int8", 128, 4096, 12288),
                                        ("block_fp8", 64, 6144, 4096), ("mxfp8", 16, 4096, 4096),
-                                       ("mxfp8", 64, 6144, 4096)])
+                                       ("mxfp8", 64, 6144, 4096), ("nvfp4", 1, 4096, 4096),
+                                       ("nvfp4", 32, 4096, 12288), ("nvfp4", 64, 6144, 4096),
+                                       ("fp8_dynamic", 2048, 6144, 4096)])
 def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
     # every plan the tuner times is one the library runs as asked (no silent
     # legalization), and a grid-schedule Swap-AB candidate with more CTAs than
@@ -385,8 +387,8 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
 
     fid = tune.FMT_ID[fmt]
     cands = tune.candidates(fmt, M, N, K, 148)
-    # fused candidates at decode token counts (MXFP8 has no fused quantizer)
-    assert any(c[8] for c in cands) == (M <= 32 and fmt != "mxfp8")
+    # fused candidates at decode token counts (the block-scaled formats have no fused quantizer)
+    assert any(c[8] for c in cands) == (M <= 32 and fmt not in ("mxfp8", "nvfp4"))
     for var, s, r, t, sch, occ, kps, st, fz in cands:
         qgd.qgd_set_override(fid, var, s, r, st, t, sch, occ, kps)
         qgd.qgd_set_fused_override(fid, fz)
@@ -539,3 +541,29 @@ def test_layer_call_rejects_bad_arguments():
     assert L.qlinear_block_fp8_bf16(P(16), 1000, P(16), P(16), P(16), 4, 512, 1000, None, 0, None) == -2
     # an empty call is fine
     assert L.qlinear_fp8_dynamic_bf16(None, 1024, None, None, None, 0, 512, 1024, None, 0, None) == 0
+
+
+def test_nvfp4_plan_rules_and_rejects():
+    F = qgd.FMT_NVFP4
+    # Swap-AB only, no two-pass reduction, the ring capped by tensor memory:
+    # 2 x 16 accumulator columns + 32 scale-factor columns per (stage, K slice) <= 256
+    qgd.qgd_set_override(F, qgd.VARIANT_STANDARD, 4, qgd.REDUCE_TWO_PASS, 0, 0, qgd.SCHEDULE_GRID, 0, 1)
+    p = qgd.qgd_get_plan(F, 8, 4096, 4096)
+    assert (p["variant"], p["reduce"]) == (qgd.VARIANT_SWAP_AB, qgd.REDUCE_LAST_CTA)
+    assert 2 * 16 + p["stages"] * p["k_slices"] * 32 <= 256
+    qgd.qgd_set_override(F, qgd.VARIANT_SWAP_AB, 1, 0, 0, 0, qgd.SCHEDULE_PERSISTENT, 1, 2)
+    p = qgd.qgd_get_plan(F, 64, 4096, 4096)
+    assert p["k_slices"] == 2 and 2 * 64 + p["stages"] * 2 * 32 <= 256
+    # K units count 128-byte slices of packed codes: K = 4096 values is 16 slices
+    qgd.qgd_set_override(F, qgd.VARIANT_SWAP_AB, 32, 0, 0, 0, qgd.SCHEDULE_GRID, 0, 1)
+    assert qgd.qgd_get_plan(F, 4, 4096, 4096)["split_k"] == 16
+    qgd.qgd_set_override(F)
+    L = qgd.lib()
+    P = ctypes.c_void_p
+    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 4, 512, 1152, None, 0, None) == -2
+    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 65, 512, 1024, None, 0, None) == -2
+    assert L.quant_nvfp4(P(16), 4, 1000, 1000, P(16), P(16), P(16), None) == -2
+    assert L.qlinear_nvfp4(P(16), None, P(16), P(16), P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
+    # the layer workspace holds the packed codes, the row scales and the block scales
+    ws = qgd.qgd_layer_workspace_size(F, 8, 4096, 4096)
+    assert ws >= 8 * 2048 + 8 * 4 + 8 * 256

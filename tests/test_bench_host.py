@@ -21,6 +21,12 @@ def test_gemm_algorithmic_bytes():
     assert workloads.algorithmic_bytes(workloads.MXFP8, 4, 4096, 4096) == (
         4096 * 4096 + 4 * 4096 + 4096 * 128 + 4 * 128 + 2 * 4 * 4096)
     assert bench.path_bytes(workloads.MXFP8, 4, 4096, 4096) == 4096 * 4096 + 2 * 4 * 4096 + 4096 * 128 + 2 * 4 * 4096
+    # NVFP4: half a byte per value, one E4M3 byte per 16 values, one fp32 per row
+    assert workloads.algorithmic_bytes(workloads.NVFP4, 4, 4096, 4096) == (
+        4096 * 2048 + 4 * 2048 + (4096 + 4) * 256 + 4 * (4096 + 4) + 2 * 4 * 4096)
+    assert bench.path_bytes(workloads.NVFP4, 4, 4096, 4096) == (
+        4096 * 2048 + 4096 * 256 + 4 * 4096 + 2 * 4 * 4096 + 2 * 4 * 4096)
+    assert bench.quant_bytes(workloads.NVFP4, 4, 4096) == 2 * 4 * 4096 + 4 * 2048 + 4 * 256 + 4 * 4
 
 
 def test_path_and_quantizer_bytes():
