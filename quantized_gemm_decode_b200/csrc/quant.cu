@@ -129,35 +129,53 @@ __global__ void __launch_bounds__(256) quant_mx_kernel(const uint16_t* __restric
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 rows (activations or weights): one CTA per row.  The row maximum
-// first (the row stays in L1/L2 for the second read), then one thread per
-// block of 16: its maximum, E4M3 scale and 16 E2M1 codes.
-// x rows are ldx elements apart; q [rows][K/2] packed codes, s [rows][K/16]
-// E4M3 scales, g [rows] fp32 row scales.
+// NVFP4 rows (activations or weights): one CTA of 256 threads per row, each
+// thread holding kBPT blocks of 16 values (two 16-byte vectors each) in
+// registers: the row maximum over the CTA, then per block its maximum, E4M3
+// scale and 16 E2M1 codes.  x rows are ldx elements apart; q [rows][K/2]
+// packed codes, s [rows][K/16] E4M3 scales, g [rows] fp32 row scales.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quant_nv_kernel(const uint16_t* __restrict__ x, int K, int ldx,
-                                                       uint8_t* __restrict__ q, uint8_t* __restrict__ s,
-                                                       float* __restrict__ g) {
+constexpr int kNvThreads = 256;
+
+template <int kBPT>
+__global__ void __launch_bounds__(kNvThreads) quant_nv_kernel(const uint16_t* __restrict__ x, int K, int ldx,
+                                                              uint8_t* __restrict__ q, uint8_t* __restrict__ s,
+                                                              float* __restrict__ g) {
   __shared__ float red[33];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // x comes from the preceding kernel
   const size_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * static_cast<size_t>(ldx));
+  const int nb = K / 16;
+  uint4 v[kBPT][2];
+  float bm[kBPT];
   float amax = 0.f;
-  for (int i = threadIdx.x; i < K / 8; i += blockDim.x) amax = fmaxf(amax, absmax8(__ldg(xr + i)));
+#pragma unroll
+  for (int j = 0; j < kBPT; ++j) {
+    const int b = threadIdx.x + j * kNvThreads;
+    bm[j] = 0.f;
+    if (b < nb) {
+      v[j][0] = __ldg(xr + 2 * b);
+      v[j][1] = __ldg(xr + 2 * b + 1);
+      bm[j] = fmaxf(absmax8(v[j][0]), absmax8(v[j][1]));
+      amax = fmaxf(amax, bm[j]);
+    }
+  }
   amax = fmaxf(block_max(amax, red), kAmaxFloor);
   const float gr = __fdiv_rn(amax, kNvRowDiv);
   const float six_g = __fmul_rn(6.0f, gr);
   if (threadIdx.x == 0) g[row] = gr;
   uint2* qr = reinterpret_cast<uint2*>(q + row * static_cast<size_t>(K / 2));
-  uint8_t* sr = s + row * static_cast<size_t>(K / 16);
-  for (int b = threadIdx.x; b < K / 16; b += blockDim.x) {
-    const uint4 v0 = __ldg(xr + 2 * b), v1 = __ldg(xr + 2 * b + 1);
-    const float bmax = fmaxf(absmax8(v0), absmax8(v1));
-    const uint32_t sc = e4m3x2(__fdiv_rn(bmax, six_g), 0.f) & 0xFFu;
-    const float d = __fmul_rn(e4m3_value(sc), gr);
-    qr[b] = encode16_nv(v0, v1, d);
-    sr[b] = static_cast<uint8_t>(sc);
+  uint8_t* sr = s + row * static_cast<size_t>(nb);
+#pragma unroll
+  for (int j = 0; j < kBPT; ++j) {
+    const int b = threadIdx.x + j * kNvThreads;
+    if (b < nb) {
+      const uint32_t sc = e4m3x2(__fdiv_rn(bm[j], six_g), 0.f) & 0xFFu;
+      const float d = __fmul_rn(e4m3_value(sc), gr);
+      qr[b] = encode16_nv(v[j][0], v[j][1], d);
+      sr[b] = static_cast<uint8_t>(sc);
+    }
   }
 }
 
@@ -248,7 +266,13 @@ cudaError_t launch_quant_mx(const uint16_t* x, int rows, int K, int ldx, uint8_t
 
 cudaError_t launch_quant_nv(const uint16_t* x, int rows, int K, int ldx, uint8_t* q, uint8_t* s, float* g,
                             cudaStream_t stream) {
-  return launch_q(quant_nv_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), stream, x, K, ldx, q, s, g);
+  const int per = (K / 16 + kNvThreads - 1) / kNvThreads;  // blocks of 16 per thread (K <= 65536: <= 16)
+  const dim3 grid(static_cast<unsigned>(rows)), block(kNvThreads);
+  if (per <= 1) return launch_q(quant_nv_kernel<1>, grid, block, stream, x, K, ldx, q, s, g);
+  if (per <= 2) return launch_q(quant_nv_kernel<2>, grid, block, stream, x, K, ldx, q, s, g);
+  if (per <= 4) return launch_q(quant_nv_kernel<4>, grid, block, stream, x, K, ldx, q, s, g);
+  if (per <= 8) return launch_q(quant_nv_kernel<8>, grid, block, stream, x, K, ldx, q, s, g);
+  return launch_q(quant_nv_kernel<16>, grid, block, stream, x, K, ldx, q, s, g);
 }
 
 cudaError_t launch_quant_block128(const uint16_t* w, int N, int K, uint8_t* q, float* s, cudaStream_t stream) {

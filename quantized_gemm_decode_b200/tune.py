@@ -306,8 +306,8 @@ def main(argv=None):
     qgd.qgd_clear_dispatch_table()
     device = torch.device("cuda")
     fmts = args.formats.split(",")
-    wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE)
-           if w.fmt in fmts]
+    wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE,
+                       workloads.NV_DECODE) if w.fmt in fmts]
     if args.large_m:
         wls += [w for w in workloads.LARGE if w.fmt in fmts]
     done = {}
