@@ -29,8 +29,9 @@
  *   - All matrices are row-major with K contiguous ("K-major"): X/Xq [M,K],
  *     W/Wq [N,K], Y [M,N].  bf16 is passed as its 16-bit storage.
  *   - Data pointers are DEVICE pointers owned by the caller and must be
- *     16-byte aligned.  The library never allocates device memory, never
- *     frees caller memory and never synchronizes the stream.
+ *     16-byte aligned.  The library never allocates device memory (except
+ *     qgd_ipc_malloc, on request), never frees caller memory and never
+ *     synchronizes the stream.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
  *     enqueued asynchronously.  The quantizers and the qlinear_* calls that
  *     take a workspace can be captured into a CUDA graph (nothing inside them
@@ -309,6 +310,97 @@ QGD_API qgd_status qlinear_nvfp4(const void* xq, const void* sx_e4m3, const floa
 QGD_API qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* wq, const void* sw_e4m3,
                                       const float* gw, void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes,
                                       void* stream);
+
+/* ---------------------------------------------------------------------
+ * Column-parallel (tensor-parallel) layer call with the all-gather fused
+ * into the GEMM's output stores.  The pages run one GPU only (tensor
+ * parallelism of one: "Building a High-Performance and Portable vLLM Linear
+ * Backend with Helion", section "Preserve the conditions when moving from
+ * kernels to serving"); this is the library's own extension of the same
+ * operation to G GPUs.  The full layer Y[M, ldy] = dequant(Xq) . dequant(W)^T
+ * has its weight rows (output columns) split over G ranks: rank r holds the
+ * rows [col0_r, col0_r + N_r) of W, quantized as for the layer calls above,
+ * and the replicated activations x_bf16 [M,K].  Each rank's call quantizes x
+ * as the layer call would and computes its Y columns with the Swap-AB kernel,
+ * whose epilogue stores every finished element to ALL ranks' full outputs
+ * (peer memory over NVLink), so that after qgd_tp_wait every rank holds the
+ * whole Y.  The numbers are exactly those of a single-GPU layer call on the
+ * shard with the same plan.
+ *
+ *   ranks      G, 1..QGD_MAX_TP_RANKS
+ *   rank       this rank, 0..G-1 (the index of its own entries below)
+ *   col0, ldy  this shard's first column in the full output, and the full
+ *              output's width (its row stride in elements; ldy % 8 == 0,
+ *              col0 + N <= ldy)
+ *   y[r]       rank r's full bf16 output [M, ldy] as addressed from this
+ *              process (this GPU's own buffer at y[rank]; the others opened
+ *              with qgd_ipc_open, or plain pointers when every "rank" runs on
+ *              one GPU), 16-byte aligned
+ *   flags[r]   rank r's flag array: G uint32 entries, zero-filled before the
+ *              first call, as addressed from this process
+ *   epoch      nonzero, one more than the previous call's (every rank uses
+ *              the same sequence 1, 2, 3, ... on the same flags; it may wrap,
+ *              skipping 0)
+ *
+ * After the last of this call's CTAs has stored its output, the kernel sets
+ * entry `rank` of every rank's flag array to `epoch` (a system-scope
+ * release).  A rank reads the full Y only after qgd_tp_wait on its own flags
+ * in stream order after its own call.  Because another rank may already run
+ * its next call and write into this rank's Y while this rank still reads the
+ * previous result, alternate between two output buffers (by epoch parity);
+ * the flags need no second copy.
+ *
+ * Plan: the layer plan for (fmt, M, N, K) forced to Swap-AB (the Standard
+ * kernels have no such epilogue) and to a reduction inside the GEMM kernel
+ * (a two-pass request takes the last-arriving CTA).  M <= 128 (FP8_Dynamic,
+ * W8A8_INT8), <= 64 (MXFP8, NVFP4), <= 32 (Block_FP8); more ->
+ * QGD_ERR_UNSUPPORTED.  M == 0 launches nothing and sets no flag: skip the
+ * wait for such a call.  sw: the weight scales of the format (fp32 per
+ * channel or per block; MXFP8 E8M0 bytes; NVFP4 the fp32 row scales), and
+ * sw_block the NVFP4 E4M3 block scales (NULL otherwise).  Workspace:
+ * qgd_tp_workspace_size() bytes, never NULL (the 64 KiB counter header is
+ * always present; its last word counts this call's finished CTAs), the usual
+ * rules otherwise.  Errors as the layer calls; a bad descriptor ->
+ * QGD_ERR_INVALID.
+ * ------------------------------------------------------------------- */
+#define QGD_MAX_TP_RANKS 8
+typedef struct {
+  int ranks;
+  int rank;
+  int col0;
+  int ldy;
+  void* y[QGD_MAX_TP_RANKS];
+  unsigned int* flags[QGD_MAX_TP_RANKS];
+  unsigned int epoch;
+} qgd_tp;
+
+QGD_API size_t qgd_tp_workspace_size(int fmt, int M, int N, int K);
+QGD_API qgd_status qlinear_tp_bf16(int fmt, const void* x_bf16, int ldx, const void* wq, const void* sw,
+                                   const void* sw_block, int M, int N, int K, const qgd_tp* tp, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Enqueue, on `stream`, a one-thread kernel that waits until every one of
+ * flags[0..ranks-1] (this rank's own flag array) holds `epoch` or a later
+ * value (compared modulo 2^32), with acquire semantics at system scope, so
+ * that kernels after it on the stream see every rank's output.  A flag still
+ * behind after about one second makes the kernel record device error 6
+ * (qgd_device_error) and return; the output is then incomplete.  Launch it
+ * only after this rank's own qlinear_tp_bf16 in the same stream: it must
+ * never wait for a kernel of its own GPU. */
+QGD_API qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, unsigned int epoch, void* stream);
+
+/* Buffers shared between processes (CUDA IPC).  qgd_ipc_malloc allocates
+ * `bytes` of device memory on the current device, zero-fills it
+ * (synchronously) and writes its QGD_IPC_HANDLE_BYTES-byte handle to
+ * `handle`; free it with qgd_ipc_free after every importer has closed it.
+ * qgd_ipc_open maps another process's buffer from its handle (peer access
+ * enabled on demand) and qgd_ipc_close unmaps it.  A process cannot open its
+ * own handles. */
+#define QGD_IPC_HANDLE_BYTES 64
+QGD_API qgd_status qgd_ipc_malloc(size_t bytes, void** dptr, void* handle);
+QGD_API qgd_status qgd_ipc_open(const void* handle, void** dptr);
+QGD_API qgd_status qgd_ipc_close(void* dptr);
+QGD_API qgd_status qgd_ipc_free(void* dptr);
 
 /* Test hook: the W8A8_INT8 mainloop and Split-K reduction of the plan in
  * force, writing the exact int32 accumulator acc[M][N] instead of Y. */

@@ -36,6 +36,8 @@ __all__ = [
     "qgd_mma_peak_probe", "qgd_test_withhold_accumulator",
     "qlinear_bf16", "qgd_layer_workspace_size", "qgd_get_layer_plan", "qgd_set_fused_override",
     "qgd_test_capture_fused",
+    "MAX_TP_RANKS", "qlinear_tp_bf16", "qgd_tp_workspace_size", "qgd_tp_wait", "ipc_malloc", "ipc_open",
+    "ipc_close", "ipc_free", "tensor_at",
     "Workspace", "DEFAULT_TABLE",
 ]
 
@@ -60,6 +62,16 @@ class QGDError(RuntimeError):
     def __init__(self, status: int, where: str, message: str):
         super().__init__(f"{where}: {message} (status {status})")
         self.status = status
+
+
+MAX_TP_RANKS = 8
+IPC_HANDLE_BYTES = 64
+
+
+class _Tp(ctypes.Structure):
+    _fields_ = [("ranks", ctypes.c_int), ("rank", ctypes.c_int), ("col0", ctypes.c_int), ("ldy", ctypes.c_int),
+                ("y", ctypes.c_void_p * MAX_TP_RANKS), ("flags", ctypes.c_void_p * MAX_TP_RANKS),
+                ("epoch", ctypes.c_uint)]
 
 
 class _Plan(ctypes.Structure):
@@ -110,6 +122,12 @@ def lib() -> ctypes.CDLL:
             "quant_nvfp4": [P, I, I, I, P, P, P, P],
             "qlinear_nvfp4": [P, P, P, P, P, P, P, I, I, I, P, S, P],
             "qlinear_nvfp4_bf16": [P, I, P, P, P, P, I, I, I, P, S, P],
+            "qlinear_tp_bf16": [I, P, I, P, P, P, I, I, I, ctypes.POINTER(_Tp), P, S, P],
+            "qgd_tp_wait": [P, I, ctypes.c_uint, P],
+            "qgd_ipc_malloc": [S, ctypes.POINTER(ctypes.c_void_p), P],
+            "qgd_ipc_open": [P, ctypes.POINTER(ctypes.c_void_p)],
+            "qgd_ipc_close": [P],
+            "qgd_ipc_free": [P],
         }
         for name, args in sigs.items():
             fn = getattr(L, name)
@@ -119,6 +137,8 @@ def lib() -> ctypes.CDLL:
         L.qgd_workspace_size.restype = S
         L.qgd_layer_workspace_size.argtypes = [I, I, I, I]
         L.qgd_layer_workspace_size.restype = S
+        L.qgd_tp_workspace_size.argtypes = [I, I, I, I]
+        L.qgd_tp_workspace_size.restype = S
         L.qgd_m_bucket.argtypes = [I]
         L.qgd_m_bucket.restype = I
         L.qgd_status_string.argtypes = [I]
@@ -508,6 +528,120 @@ def qlinear_nvfp4_bf16(x: torch.Tensor, wq, sw, gw, y=None, ws=None, stream=None
     _check(lib().qlinear_nvfp4_bf16(_ptr(x), ldx, _ptr(wq), _ptr(sw), _ptr(gw), _ptr(y), M, N, K,
                                     ctypes.c_void_p(wsp), wsn, _stream(stream)), "qlinear_nvfp4_bf16")
     return y
+
+
+# ---------------------------------------------------------------------------
+# Column-parallel layer call (all-gather fused into the output stores)
+# ---------------------------------------------------------------------------
+def _layer_weight_operands(fmt: int, wq, sw, sw_block, K: int) -> int:
+    """Check a layer call's weight operands for format fmt; returns N."""
+    if not isinstance(wq, torch.Tensor) or wq.dim() != 2 or not wq.is_cuda or not wq.is_contiguous():
+        raise ValueError("wq must be a contiguous 2-D CUDA tensor")
+    N = wq.shape[0]
+    if fmt == FMT_NVFP4:
+        _check_nv(wq, sw_block, sw, N, K, "w")
+        return N
+    if sw_block is not None:
+        raise ValueError("sw_block is for NVFP4 weights only")
+    want_w = (torch.int8,) if fmt == FMT_W8A8_INT8 else (torch.uint8, torch.float8_e4m3fn)
+    if wq.shape[1] != K or wq.dtype not in want_w:
+        raise ValueError(f"wq must be a {want_w} tensor with K={K} columns")
+    sw_n = (N // 128) * (K // 128) if fmt == FMT_BLOCK_FP8 else (N * (K // 32) if fmt == FMT_MXFP8 else N)
+    sw_t = torch.uint8 if fmt == FMT_MXFP8 else torch.float32
+    if not isinstance(sw, torch.Tensor) or sw.dtype != sw_t or sw.numel() < sw_n or not sw.is_contiguous() \
+            or not sw.is_cuda:
+        raise ValueError(f"sw must be a contiguous CUDA {sw_t} tensor of at least {sw_n} scales")
+    return N
+
+
+def qgd_tp_workspace_size(fmt: int, M: int, N: int, K: int) -> int:
+    return int(lib().qgd_tp_workspace_size(fmt, M, N, K))
+
+
+def qlinear_tp_bf16(fmt: int, x: torch.Tensor, wq, sw, sw_block, *, ranks: int, rank: int, col0: int, ldy: int,
+                    ys, flags, epoch: int, ws, stream=None) -> None:
+    """Column-parallel layer call: this rank's weight shard (wq [N, K] with
+    its scales; NVFP4: sw = fp32 row scales, sw_block = E4M3 block scales)
+    against the replicated bf16 activations x [M, K].  Every finished output
+    element goes to columns [col0, col0 + N) of all ranks' full outputs
+    ys[r] (bf16 [>= M, ldy], device pointers or tensors as addressed from this
+    process), and entry `rank` of every rank's flag array flags[r] is set to
+    `epoch` when the call is done.  Follow with qgd_tp_wait on this rank's
+    own flags before reading its full output."""
+    ldx = _activation_rows(x)
+    M, K = x.shape
+    N = _layer_weight_operands(fmt, wq, sw, sw_block, K)
+    if len(ys) != ranks or len(flags) != ranks or not 1 <= ranks <= MAX_TP_RANKS:
+        raise ValueError(f"need one output and one flag array per rank (1..{MAX_TP_RANKS} ranks)")
+    if not (0 <= epoch < 2 ** 32):
+        raise ValueError("epoch must fit in 32 bits")
+    tp = _Tp()
+    tp.ranks, tp.rank, tp.col0, tp.ldy, tp.epoch = ranks, rank, col0, ldy, epoch
+    for r in range(ranks):
+        tp.y[r] = _ptr(ys[r]).value
+        tp.flags[r] = _ptr(flags[r]).value
+    if isinstance(ws, Workspace):
+        ws.ensure(qgd_tp_workspace_size(fmt, M, N, K))
+        wsp, wsn = ws.buf.data_ptr(), ws.nbytes
+    else:
+        wsp, wsn = ws.data_ptr(), ws.numel() * ws.element_size()
+    _check(lib().qlinear_tp_bf16(fmt, _ptr(x), ldx, _ptr(wq), _ptr(sw), _ptr(sw_block), M, N, K, ctypes.byref(tp),
+                                 ctypes.c_void_p(wsp), wsn, _stream(stream)), "qlinear_tp_bf16")
+
+
+def qgd_tp_wait(flags, ranks: int, epoch: int, stream=None) -> None:
+    """Enqueue the wait for every rank's flag in this rank's own flag array
+    (a tensor or a device pointer) to reach `epoch`."""
+    _check(lib().qgd_tp_wait(_ptr(flags), ranks, epoch, _stream(stream)), "qgd_tp_wait")
+
+
+def ipc_malloc(nbytes: int) -> tuple:
+    """A zero-filled device buffer on the current device that other processes
+    can map: returns (device pointer, handle bytes)."""
+    ptr = ctypes.c_void_p(0)
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().qgd_ipc_malloc(nbytes, ctypes.byref(ptr), handle), "qgd_ipc_malloc")
+    return int(ptr.value), handle.raw
+
+
+def ipc_open(handle: bytes) -> int:
+    """Map another process's buffer from its handle; returns the pointer."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes")
+    ptr = ctypes.c_void_p(0)
+    _check(lib().qgd_ipc_open(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES), ctypes.byref(ptr)),
+           "qgd_ipc_open")
+    return int(ptr.value)
+
+
+def ipc_close(ptr: int) -> None:
+    _check(lib().qgd_ipc_close(ctypes.c_void_p(ptr)), "qgd_ipc_close")
+
+
+def ipc_free(ptr: int) -> None:
+    _check(lib().qgd_ipc_free(ctypes.c_void_p(ptr)), "qgd_ipc_free")
+
+
+class _DeviceArray:
+    """__cuda_array_interface__ of a raw device pointer (no ownership)."""
+
+    def __init__(self, ptr: int, shape: tuple, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 2, "strides": None}
+
+
+_TYPESTR = {torch.bfloat16: ("<i2", torch.int16), torch.int16: ("<i2", torch.int16),
+            torch.int32: ("<i4", torch.int32), torch.uint8: ("|u1", torch.uint8)}
+
+
+def tensor_at(ptr: int, shape: tuple, dtype: torch.dtype, device) -> torch.Tensor:
+    """A tensor over device memory this library allocated or mapped (no copy,
+    no ownership: the memory must outlive the tensor)."""
+    typestr, carrier = _TYPESTR[dtype]
+    with torch.cuda.device(device):
+        t = torch.as_tensor(_DeviceArray(ptr, shape, typestr), device=device)
+    assert t.dtype == carrier and t.data_ptr() == ptr
+    return t.view(dtype)
 
 
 def qlinear_fp8_dynamic_noalloc(xq, sx, wq, sw, y, stream=None):

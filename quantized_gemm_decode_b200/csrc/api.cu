@@ -194,7 +194,9 @@ int reduce_from_name(const std::string& s) {
 // K as the kernels count it: NVFP4 packs two values per byte
 int kernel_k(int fmt, int K) { return fmt == kFmtNV ? K / 2 : K; }
 
-qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
+// tp: a column-parallel call (qlinear_tp_bf16), whose output epilogue exists
+// in the Swap-AB kernel only and must be the last kernel of the call.
+qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = false) {
   const int nkt = (kernel_k(fmt, K) + kTileK - 1) / kTileK;
   qgd_plan p;
   p.source = 0;
@@ -259,7 +261,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false) {
   }
   // Make the plan legal for this shape.  (MXFP8 runs in the Swap-AB kernel
   // only, up to 128 tokens, and has no two-pass reduction kernel.)
-  if (fmt == kFmtMX || fmt == kFmtNV) {
+  if (fmt == kFmtMX || fmt == kFmtNV || tp) {
     p.variant = kSwapAB;
     if (p.reduce == kTwoPass) p.reduce = kLastCta;
   }
@@ -460,21 +462,25 @@ std::atomic<float*> g_capture_sx{nullptr};
 // GEMM is launched without a programmatic dependency (that relaxation is
 // defined between two kernels only).
 // NVFP4: sx / sw are the fp32 row scales, sx8 / sw8 the E4M3 block scales.
+// tp != null: a column-parallel call; the output goes to every rank's full Y
+// (tp->y) and tp_done is this rank's completion counter (zero between calls).
 qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float* sx, const uint16_t* xbf, int ldxb,
                          const void* wq, const float* sw, void* y, void* raw, int M, int N, int K, void* ws,
                          size_t ws_bytes, void* stream, bool follows_memset, const uint8_t* sx8 = nullptr,
-                         const uint8_t* sw8 = nullptr) {
+                         const uint8_t* sw8 = nullptr, const qgd_tp* tp = nullptr, unsigned* tp_done = nullptr) {
   qgd_status st;
   if ((st = check_device()) != QGD_OK) return st;
   if ((st = get_encoder()) != QGD_OK) return st;
   const bool fused = xbf != nullptr;
   if (fused && (!p.fused || p.variant != kSwapAB)) return fail(QGD_ERR_INVALID, "internal: fused launch without a fused plan");
+  if (tp && (p.variant != kSwapAB || p.reduce == kTwoPass || raw || !tp_done))
+    return fail(QGD_ERR_INVALID, "internal: column-parallel launch without a one-kernel Swap-AB plan");
   const Exec ex = make_exec(fmt, p, M, N, K);
   if (ex.total > 0 && (!ws || ws_bytes < ex.total))
     return fail(QGD_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", ex.total, ws ? ws_bytes : 0);
   if (ex.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
 
-  GemmArgs a;
+  GemmArgs a{};
   a.sx = sx;
   a.sw = sw;
   a.y = static_cast<uint16_t*>(y);
@@ -508,6 +514,28 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
   a.sx_out = fused ? g_capture_sx.load() : nullptr;
   a.sx8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sx) : fmt == kFmtNV ? sx8 : nullptr;
   a.sw8 = fmt == kFmtMX ? reinterpret_cast<const uint8_t*>(sw) : fmt == kFmtNV ? sw8 : nullptr;
+  a.tp_ranks = 0;  // a plain call unless column-parallel
+  a.tp_rank = 0;
+  a.tp_col0 = 0;
+  a.tp_ldy = 0;
+  a.tp_epoch = 0;
+  a.tp_done = nullptr;
+  for (int r = 0; r < kMaxTpRanks; ++r) {
+    a.tp_y[r] = nullptr;
+    a.tp_flag[r] = nullptr;
+  }
+  if (tp) {
+    a.tp_ranks = tp->ranks;
+    a.tp_rank = tp->rank;
+    a.tp_col0 = tp->col0;
+    a.tp_ldy = tp->ldy;
+    a.tp_epoch = tp->epoch;
+    a.tp_done = tp_done;
+    for (int r = 0; r < tp->ranks; ++r) {
+      a.tp_y[r] = static_cast<uint16_t*>(tp->y[r]);
+      a.tp_flag[r] = tp->flags[r];
+    }
+  }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tw, tx;
@@ -576,11 +604,14 @@ struct LayerWs {
   size_t xq_off = 0, sx_off = 0, sb_off = 0, total = 0;
 };
 
-LayerWs layer_ws(int fmt, int M, int N, int K) {
+// tp: a column-parallel call, whose completion counter lives in the last
+// word of the counter header, so its workspace always holds the header.
+LayerWs layer_ws(int fmt, int M, int N, int K, bool tp = false) {
   LayerWs l;
-  l.plan = make_plan(fmt, M, N, K, true);
+  l.plan = make_plan(fmt, M, N, K, true, tp);
   l.ex = make_exec(fmt, l.plan, M, N, K);
   l.total = l.ex.total;
+  if (tp && l.total < kTicketBytes) l.total = kTicketBytes;
   if (!l.plan.fused && M > 0) {
     l.xq_off = align256(l.total > kTicketBytes ? l.total : kTicketBytes);
     l.sx_off = align256(l.xq_off + static_cast<size_t>(M) * kernel_k(fmt, K));
@@ -598,25 +629,30 @@ LayerWs layer_ws(int fmt, int M, int N, int K) {
   return l;
 }
 
+// tp != null: a column-parallel call (checked by the caller); y is unused.
 qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const float* sw, void* y, int M, int N,
-                     int K, void* ws, size_t ws_bytes, void* stream, const uint8_t* sw8 = nullptr) {
+                     int K, void* ws, size_t ws_bytes, void* stream, const uint8_t* sw8 = nullptr,
+                     const qgd_tp* tp = nullptr) {
   qgd_status st = check_shape(fmt, M, N, K);
   if (st != QGD_OK) return st;
   if (ldx < K || ldx % 8 != 0)
     return fail(QGD_ERR_INVALID, "row stride ldx=%d must be >= K=%d and a multiple of 8", ldx, K);
   if (K > 65536) return fail(QGD_ERR_UNSUPPORTED, "K=%d must be <= 65536", K);
   if (M == 0) return QGD_OK;
-  if (!x_bf16 || !wq || !sw || !y || (fmt == kFmtNV && !sw8)) return fail(QGD_ERR_INVALID, "null operand pointer");
+  if (!x_bf16 || !wq || !sw || (!y && !tp) || (fmt == kFmtNV && !sw8))
+    return fail(QGD_ERR_INVALID, "null operand pointer");
   if (!aligned16(x_bf16) || !aligned16(wq) || !aligned16(y) || !aligned16(sw) || !aligned16(sw8))
     return fail(QGD_ERR_INVALID, "operand pointers must be 16-byte aligned");
-  const LayerWs l = layer_ws(fmt, M, N, K);
+  const LayerWs l = layer_ws(fmt, M, N, K, tp != nullptr);
   if (l.total > 0 && (!ws || ws_bytes < l.total))
     return fail(QGD_ERR_WORKSPACE, "layer workspace of %zu bytes needed, %zu given", l.total, ws ? ws_bytes : 0);
   if (l.total > 0 && !aligned16(ws)) return fail(QGD_ERR_INVALID, "workspace must be 16-byte aligned");
+  // column-parallel: the completion counter is the last word of the header
+  unsigned* tp_done = tp ? static_cast<unsigned*>(ws) + (kMaxTickets - 1) : nullptr;
   const uint16_t* xb = static_cast<const uint16_t*>(x_bf16);
   if (l.plan.fused)
     return run_gemm_plan(fmt, l.plan, nullptr, nullptr, xb, ldx, wq, sw, y, nullptr, M, N, K, ws, ws_bytes, stream,
-                         false);
+                         false, nullptr, nullptr, tp, tp_done);
   if ((st = check_device()) != QGD_OK) return st;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* xq = wsb + l.xq_off;
@@ -630,7 +666,7 @@ qgd_status run_layer(int fmt, const void* x_bf16, int ldx, const void* wq, const
                                   : launch_quant_rows(xb, M, K, ldx, fmt == kFmtINT8 ? 1 : 0, xq, sx, s);
   if (e != cudaSuccess) return cuda_fail(e, "activation quantizer launch");
   return run_gemm_plan(fmt, l.plan, xq, sx, nullptr, 0, wq, sw, y, nullptr, M, N, K, ws, l.ex.total, stream, false,
-                       fmt == kFmtNV ? sb : nullptr, sw8);
+                       fmt == kFmtNV ? sb : nullptr, sw8, tp, tp_done);
 }
 
 // ---------------------------------------------------------------------------
@@ -813,6 +849,101 @@ qgd_status qlinear_mxfp8_bf16(const void* x_bf16, int ldx, const void* wq, const
                               int M, int N, int K, void* ws, size_t ws_bytes, void* stream) {
   return run_layer(kFmtMX, x_bf16, ldx, wq, static_cast<const float*>(sw_e8m0), y_bf16, M, N, K, ws, ws_bytes,
                    stream);
+}
+
+// ---------------------------------------------------------------------------
+// Column-parallel (tensor-parallel) layer call: this rank's N-shard of the
+// weights, its output tile written straight into every rank's full Y.
+size_t qgd_tp_workspace_size(int fmt, int M, int N, int K) {
+  if (fmt < 0 || fmt >= kNumFmts || M <= 0 || N <= 0 || K <= 0) return 0;
+  return layer_ws(fmt, M, N, K, true).total;
+}
+
+qgd_status qlinear_tp_bf16(int fmt, const void* x_bf16, int ldx, const void* wq, const void* sw,
+                           const void* sw_block, int M, int N, int K, const qgd_tp* tp, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (fmt < 0 || fmt >= kNumFmts) return fail(QGD_ERR_INVALID, "bad format %d", fmt);
+  if (!tp) return fail(QGD_ERR_INVALID, "null tensor-parallel descriptor");
+  if (tp->ranks < 1 || tp->ranks > kMaxTpRanks || tp->rank < 0 || tp->rank >= tp->ranks)
+    return fail(QGD_ERR_INVALID, "rank %d of %d ranks (1..%d ranks)", tp->rank, tp->ranks, kMaxTpRanks);
+  if (tp->epoch == 0) return fail(QGD_ERR_INVALID, "epoch 0 is the flags' initial value");
+  if (N <= 0 || tp->col0 < 0 || tp->ldy % 8 != 0 || static_cast<long long>(tp->col0) + N > tp->ldy)
+    return fail(QGD_ERR_INVALID, "shard columns [%d, %d) outside a full output %d wide (a multiple of 8)", tp->col0,
+                tp->col0 + N, tp->ldy);
+  for (int r = 0; r < tp->ranks; ++r) {
+    if (!tp->y[r] || !tp->flags[r]) return fail(QGD_ERR_INVALID, "null output or flag pointer of rank %d", r);
+    if (!aligned16(tp->y[r]) || reinterpret_cast<uintptr_t>(tp->flags[r]) % 4 != 0)
+      return fail(QGD_ERR_INVALID, "rank %d: output must be 16-byte aligned, flags 4-byte aligned", r);
+  }
+  const int max_m = fmt == kFmtBlock ? kDecodeMaxM : (fmt == kFmtMX || fmt == kFmtNV) ? kMxMaxM : kSwapMaxM;
+  if (M > max_m)
+    return fail(QGD_ERR_UNSUPPORTED, "column-parallel calls cover at most %d tokens in this format (M=%d)", max_m, M);
+  if (static_cast<long long>(M) * tp->ldy > (1LL << 31)) return fail(QGD_ERR_UNSUPPORTED, "M*ldy too large");
+  if (static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN) >= kMaxTickets)
+    return fail(QGD_ERR_UNSUPPORTED, "N=%d has more output tiles than the counter header holds", N);
+  if (!ws) return fail(QGD_ERR_WORKSPACE, "column-parallel calls need a workspace");
+  return run_layer(fmt, x_bf16, ldx, wq, static_cast<const float*>(sw), nullptr, M, N, K, ws, ws_bytes, stream,
+                   static_cast<const uint8_t*>(sw_block), tp);
+}
+
+qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, unsigned int epoch, void* stream) {
+  if (!flags || reinterpret_cast<uintptr_t>(flags) % 4 != 0) return fail(QGD_ERR_INVALID, "null or misaligned flags");
+  if (ranks < 1 || ranks > kMaxTpRanks) return fail(QGD_ERR_INVALID, "%d ranks (1..%d)", ranks, kMaxTpRanks);
+  if (epoch == 0) return fail(QGD_ERR_INVALID, "epoch 0 is the flags' initial value");
+  qgd_status st;
+  if ((st = check_device()) != QGD_OK) return st;
+  const cudaError_t e = launch_tp_wait(flags, ranks, epoch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tensor-parallel wait launch");
+  return QGD_OK;
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == QGD_IPC_HANDLE_BYTES, "IPC handle size");
+static_assert(QGD_MAX_TP_RANKS == kMaxTpRanks, "tensor-parallel rank limit");
+
+qgd_status qgd_ipc_malloc(size_t bytes, void** dptr, void* handle) {
+  if (!dptr || !handle || bytes == 0) return fail(QGD_ERR_INVALID, "null pointer or zero size");
+  *dptr = nullptr;
+  qgd_status st;
+  if ((st = check_device()) != QGD_OK) return st;
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc (shared buffer)");
+  e = cudaMemset(p, 0, bytes);
+  cudaIpcMemHandle_t h;
+  if (e == cudaSuccess) e = cudaIpcGetMemHandle(&h, p);
+  if (e != cudaSuccess) {
+    cudaFree(p);
+    return cuda_fail(e, "zeroing or exporting a shared buffer");
+  }
+  memcpy(handle, &h, sizeof h);
+  *dptr = p;
+  return QGD_OK;
+}
+
+qgd_status qgd_ipc_open(const void* handle, void** dptr) {
+  if (!handle || !dptr) return fail(QGD_ERR_INVALID, "null pointer");
+  *dptr = nullptr;
+  qgd_status st;
+  if ((st = check_device()) != QGD_OK) return st;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof h);
+  const cudaError_t e = cudaIpcOpenMemHandle(dptr, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+  return QGD_OK;
+}
+
+qgd_status qgd_ipc_close(void* dptr) {
+  if (!dptr) return fail(QGD_ERR_INVALID, "null pointer");
+  const cudaError_t e = cudaIpcCloseMemHandle(dptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
+  return QGD_OK;
+}
+
+qgd_status qgd_ipc_free(void* dptr) {
+  if (!dptr) return fail(QGD_ERR_INVALID, "null pointer");
+  const cudaError_t e = cudaFree(dptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree (shared buffer)");
+  return QGD_OK;
 }
 
 size_t qgd_layer_workspace_size(int fmt, int M, int N, int K) {

@@ -188,12 +188,43 @@ __device__ __forceinline__ void store_swap_final(uint32_t accbits, int m, int n,
   const size_t idx = static_cast<size_t>(m) * a.N + n;
   if (a.raw) {
     static_cast<uint32_t*>(a.raw)[idx] = accbits;
-  } else if constexpr (kFmt == kFmtBlock || kFmt == kFmtMX) {
-    a.y[idx] = bf16_bits(__uint_as_float(accbits));
+    return;
+  }
+  uint16_t v;
+  if constexpr (kFmt == kFmtBlock || kFmt == kFmtMX) {
+    v = bf16_bits(__uint_as_float(accbits));
   } else if constexpr (kFmt == kFmtINT8) {
-    a.y[idx] = bf16_bits((static_cast<float>(static_cast<int32_t>(accbits)) * sx_s[m]) * swv);
+    v = bf16_bits((static_cast<float>(static_cast<int32_t>(accbits)) * sx_s[m]) * swv);
   } else {
-    a.y[idx] = bf16_bits((__uint_as_float(accbits) * sx_s[m]) * swv);
+    v = bf16_bits((__uint_as_float(accbits) * sx_s[m]) * swv);
+  }
+  if (a.tp_ranks == 0) {
+    a.y[idx] = v;
+  } else {
+    // column-parallel: this element of the full output, on every rank
+    const size_t full = static_cast<size_t>(m) * a.tp_ldy + a.tp_col0 + n;
+    for (int r = 0; r < a.tp_ranks; ++r) a.tp_y[r][full] = v;
+  }
+}
+
+// Column-parallel completion: after every CTA's output is out, the last CTA
+// to finish publishes this rank's epoch in every rank's flag array (system
+// scope: the readers are other GPUs).  Called by all threads of a CTA at its
+// end.
+__device__ __forceinline__ void tp_signal_done(const GemmArgs& a) {
+  if (a.tp_ranks == 0) return;
+  __threadfence_system();  // each thread's output stores, to every rank, before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+    const unsigned prev = atomicAdd(a.tp_done, 1u);
+    if (prev == total - 1) {
+      __threadfence_system();  // every CTA's stores (their fences preceded their arrivals)
+      for (int r = 0; r < a.tp_ranks; ++r)
+        asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(a.tp_flag[r] + a.tp_rank), "r"(a.tp_epoch)
+                     : "memory");
+      *a.tp_done = 0u;  // ready for the next call
+    }
   }
 }
 
@@ -1142,6 +1173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 
   teardown(ctl, warp, lane, issued, stages, tmem, ncols);
   if (threadIdx.x == 32) QGD_STAMP(7);
+  tp_signal_done(a);
 }
 
 // Two-pass reduction for the Swap-AB layout: one CTA per tile, one thread per
@@ -1887,6 +1919,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ===========================================================================
+// Tensor-parallel wait: one thread reads each rank's entry of this rank's
+// flag array (acquire, system scope) until it holds the call's epoch (or a
+// later one: a rank may already have finished its next call), giving
+// up after about kWaitLimitNs per rank (error kErrWaitPeers).  Launched in
+// stream order after this rank's GEMM, so it never waits on a kernel of its
+// own GPU; the kernels after it read the full output.
+// ===========================================================================
+__global__ void __launch_bounds__(32) tp_wait_kernel(const unsigned* flags, int ranks, unsigned epoch) {
+  if (threadIdx.x != 0) return;
+  for (int r = 0; r < ranks; ++r) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+      unsigned v;
+      asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(flags + r) : "memory");
+      if (static_cast<int>(v - epoch) >= 0) break;  // this call's epoch or a later one (wraps)
+      if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_error(kErrWaitPeers);
+        return;
+      }
+    }
+  }
+}
+
+// ===========================================================================
 // Two-pass Split-K reduction: one thread per output element, partials added
 // in split order s = 0, 1, ..., splits-1.
 // ===========================================================================
@@ -2168,6 +2224,11 @@ extern "C" __attribute__((visibility("default"))) int qgd_debug_trace(unsigned l
   return static_cast<int>(cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)));
 }
 #endif
+
+cudaError_t launch_tp_wait(const unsigned* flags, int ranks, unsigned epoch, cudaStream_t stream) {
+  // no programmatic dependency: it starts only after this rank's GEMM is done
+  return launch_ex(tp_wait_kernel, dim3(1), dim3(32), 0, stream, false, flags, ranks, epoch);
+}
 
 cudaError_t read_device_error(unsigned int* code) {
   return cudaMemcpyFromSymbol(code, g_device_error, sizeof(unsigned int));

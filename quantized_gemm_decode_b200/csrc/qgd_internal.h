@@ -14,6 +14,7 @@ constexpr int kNumFmts = 5;
 enum Variant : int { kStandard = 0, kSwapAB = 1, kStandardPair = 2 };
 enum Reduce : int { kLastCta = 0, kTwoPass = 1, kAtomic = 2, kCluster = 3 };
 constexpr int kMaxClusterSplit = 8;  // portable thread-block cluster size
+constexpr int kMaxTpRanks = 8;       // tensor-parallel ranks of one NVLink domain
 enum Schedule : int { kGrid = 0, kPersistent = 1 };
 
 constexpr int kTileK = 128;           // K elements (= bytes) per pipeline stage
@@ -59,6 +60,19 @@ struct GemmArgs {
   // [N][K/16]; the kernel's K then counts the packed bytes, K/2)
   const uint8_t* sx8;
   const uint8_t* sw8;
+  // Column-parallel tensor parallelism (Swap-AB): this rank's output columns
+  // (its weight shard's N) go to columns [tp_col0, tp_col0 + N) of every
+  // rank's full bf16 output, tp_ldy columns wide, through the ranks' pointers
+  // (peer memory); the last CTA to finish then sets entry tp_rank of every
+  // rank's flag array to tp_epoch.  tp_ranks == 0: a plain call.
+  int tp_ranks;
+  int tp_rank;
+  int tp_col0;
+  int tp_ldy;
+  unsigned tp_epoch;
+  unsigned* tp_done;  // CTAs finished this call (zero on entry and exit)
+  uint16_t* tp_y[kMaxTpRanks];
+  unsigned* tp_flag[kMaxTpRanks];
 };
 
 // Tensor-memory columns of the block-scaled Swap-AB kernels: two accumulators
@@ -88,6 +102,8 @@ cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorM
                                  const GemmArgs& a, cudaStream_t stream);
 int pair_max_active_clusters(int fmt, int stages, int kps);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
+// Tensor parallelism: wait (bounded) until flags[0..ranks) all equal epoch
+cudaError_t launch_tp_wait(const unsigned* flags, int ranks, unsigned epoch, cudaStream_t stream);
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();

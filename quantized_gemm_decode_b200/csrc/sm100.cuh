@@ -22,6 +22,7 @@ enum : unsigned int {
   kErrWaitEpilogue = 3,   // epilogue gave up waiting for the accumulator
   kErrWaitDrain = 4,      // teardown gave up waiting for copies or MMAs in flight
   kErrBadOperand = 5,     // an operand address failed its alignment check; the MMA was skipped
+  kErrWaitPeers = 6,      // a tensor-parallel wait gave up on a rank's completion flag
 };
 
 // Wait budget: about one second of wall time (globaltimer is in ns).

@@ -285,3 +285,148 @@ class DecodeChain:
     def inputs(self, M: int) -> list:
         """The bf16 input each layer quantized (views into earlier outputs)."""
         return [self._input(M, i) for i in range(len(self.layers))]
+
+
+# ---------------------------------------------------------------------------
+# Column-parallel (tensor-parallel) layer
+# ---------------------------------------------------------------------------
+_TP_FMT = {"fp8_dynamic": qgd.FMT_FP8_DYNAMIC, "w8a8_int8": qgd.FMT_W8A8_INT8, "block_fp8": qgd.FMT_BLOCK_FP8,
+           "mxfp8": qgd.FMT_MXFP8, "nvfp4": qgd.FMT_NVFP4}
+
+
+def quantize_weight(w: torch.Tensor, fmt: str) -> tuple:
+    """(wq, sw, sw_block) of a bf16 weight [N, K] in a layer format, as the
+    layer calls take them (sw_block: the NVFP4 E4M3 block scales, else None)."""
+    if fmt == "block_fp8":
+        wq, sw = qgd.quant_weight_block128(w)
+        return wq, sw, None
+    if fmt == "mxfp8":
+        wq, sw = qgd.quant_mx(w)
+        return wq, sw, None
+    if fmt == "nvfp4":
+        wq, sb, g = qgd.quant_nv(w)
+        return wq, g, sb
+    qt = qgd.QTYPE_INT8 if fmt == "w8a8_int8" else qgd.QTYPE_E4M3
+    wq, sw = qgd.quant_weight_per_channel(w, qt)
+    return wq, sw, None
+
+
+class _LibraryIpc:
+    malloc = staticmethod(qgd.ipc_malloc)
+    open = staticmethod(qgd.ipc_open)
+    close = staticmethod(qgd.ipc_close)
+    free = staticmethod(qgd.ipc_free)
+
+
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
+class ColumnParallelLinear:
+    """y = x @ W^T with W's rows (the output columns) split over the ranks of
+    a torch.distributed group, one GPU per rank, and the all-gather of y fused
+    into the GEMM: each rank's kernel stores its columns straight into every
+    rank's full output over peer memory (NVLink) and then raises one flag per
+    rank, so every rank ends the call holding all of y.
+
+    Each rank owns one shared device buffer, mapped by all ranks (CUDA IPC):
+    two full outputs [max_m, ldy] bf16 (successive calls alternate, so that a
+    rank already running its next call never overwrites the output another
+    rank is still reading) and a flag array of one uint32 per rank.  Shards
+    may differ in width; col0 and ldy come from an all-gather of the widths.
+    """
+
+    def __init__(self, w_shard: torch.Tensor | None, fmt: str = "fp8_dynamic", group=None, max_m: int = 32,
+                 weights: tuple | None = None, ipc=None):
+        import torch.distributed as dist
+
+        if fmt not in _TP_FMT:
+            raise ValueError(f"unknown format {fmt}")
+        self.fmt, self.fmt_id = fmt, _TP_FMT[fmt]
+        self.group = group
+        self._dist = dist if dist.is_available() and dist.is_initialized() else None
+        self.G = self._dist.get_world_size(group) if self._dist else 1
+        self.rank = self._dist.get_rank(group) if self._dist else 0
+        if self.G > qgd.MAX_TP_RANKS:
+            raise ValueError(f"at most {qgd.MAX_TP_RANKS} ranks share one output")
+        self.wq, self.sw, self.sw_block = weights if weights is not None else quantize_weight(w_shard, fmt)
+        self.N = self.wq.shape[0]
+        self.K = self.wq.shape[1] * (2 if fmt == "nvfp4" else 1)
+        self.device = self.wq.device
+        widths = self._all_gather(self.N)
+        self.col0, self.ldy = sum(widths[:self.rank]), sum(widths)
+        self.max_m = max_m
+        self.out_bytes = max_m * self.ldy * 2
+        self.flags_off = 2 * _align(self.out_bytes)
+        self.nbytes = self.flags_off + _align(4 * self.G)
+        self._ipc = ipc if ipc is not None else _LibraryIpc
+        self.own, handle = self._ipc.malloc(self.nbytes)
+        handles = self._all_gather(handle)
+        self.bases = [self.own if r == self.rank else self._ipc.open(handles[r]) for r in range(self.G)]
+        self.ws = qgd.Workspace(qgd.qgd_tp_workspace_size(self.fmt_id, max_m, self.N, self.K), self.device)
+        self.calls = 0
+        self.epoch = 0
+
+    def _all_gather(self, obj) -> list:
+        if self._dist is None:
+            return [obj]
+        out = [None] * self.G
+        self._dist.all_gather_object(out, obj, group=self.group)
+        return out
+
+    def _next_epoch(self) -> int:
+        self.epoch = self.epoch % 0xFFFFFFFF + 1  # 1, 2, ..., 2^32 - 1, 1, ... (0 is the flags' initial value)
+        return self.epoch
+
+    def output_ptr(self, rank: int, buf: int) -> int:
+        return self.bases[rank] + buf * _align(self.out_bytes)
+
+    def flags_ptr(self, rank: int) -> int:
+        return self.bases[rank] + self.flags_off
+
+    def launch(self, x: torch.Tensor, stream=None) -> int:
+        """Enqueue this rank's share of the call; returns the output buffer
+        (0 or 1) it writes.  Every rank must launch the same sequence of calls."""
+        M = x.shape[0]
+        if M > self.max_m:
+            raise ValueError(f"M={M} exceeds the buffers' {self.max_m} rows")
+        buf = self.calls & 1
+        self.calls += 1
+        epoch = self._next_epoch()
+        if M == 0:
+            return buf
+        qgd.qlinear_tp_bf16(self.fmt_id, x, self.wq, self.sw, self.sw_block, ranks=self.G, rank=self.rank,
+                            col0=self.col0, ldy=self.ldy, ys=[self.output_ptr(r, buf) for r in range(self.G)],
+                            flags=[self.flags_ptr(r) for r in range(self.G)], epoch=epoch, ws=self.ws,
+                            stream=stream)
+        return buf
+
+    def wait(self, M: int, buf: int, stream=None) -> torch.Tensor:
+        """Enqueue the wait for every rank's share of the last call and return
+        the full output [M, ldy] (a view of this rank's shared buffer, valid
+        until the call after next)."""
+        if M > 0:
+            qgd.qgd_tp_wait(self.flags_ptr(self.rank), self.G, self.epoch, stream=stream)
+        full = qgd.tensor_at(self.output_ptr(self.rank, buf), (self.max_m, self.ldy), torch.bfloat16, self.device)
+        return full[:M]
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        buf = self.launch(x, stream=stream)
+        return self.wait(x.shape[0], buf, stream=stream)
+
+    def close(self) -> None:
+        """Unmap the peers' buffers and free this rank's (collective: every
+        rank calls it, after its last use of the outputs)."""
+        if self.bases is None:
+            return
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+        if self._dist is not None:
+            self._dist.barrier(group=self.group)  # no rank still writes into another's buffer
+        for r, p in enumerate(self.bases):
+            if r != self.rank:
+                self._ipc.close(p)
+        if self._dist is not None:
+            self._dist.barrier(group=self.group)  # every mapping of this rank's buffer is gone
+        self._ipc.free(self.own)
+        self.bases = None

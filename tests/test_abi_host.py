@@ -567,3 +567,53 @@ def test_nvfp4_plan_rules_and_rejects():
     # the layer workspace holds the packed codes, the row scales and the block scales
     ws = qgd.qgd_layer_workspace_size(F, 8, 4096, 4096)
     assert ws >= 8 * 2048 + 8 * 4 + 8 * 256
+
+
+def _tp_desc(ranks=2, rank=0, col0=0, ldy=512, epoch=1, null_y=False):
+    d = qgd._Tp()
+    d.ranks, d.rank, d.col0, d.ldy, d.epoch = ranks, rank, col0, ldy, epoch
+    for r in range(min(max(ranks, 0), qgd.MAX_TP_RANKS)):
+        d.y[r] = None if null_y and r == ranks - 1 else 4096 * (r + 1)
+        d.flags[r] = 8192 * (r + 1)
+    return d
+
+
+def test_column_parallel_call_rules():
+    L = qgd.lib()
+    P = ctypes.c_void_p
+    for name in ("qlinear_tp_bf16", "qgd_tp_wait", "qgd_tp_workspace_size", "qgd_ipc_malloc", "qgd_ipc_open",
+                 "qgd_ipc_close", "qgd_ipc_free"):
+        assert name in declared_functions()
+    assert ctypes.sizeof(qgd._Tp) == 4 * 4 + 2 * 8 * 8 + 8  # four ints, two pointer arrays, the epoch (padded)
+    # the workspace always holds the 64 KiB counter header (its last word counts finished CTAs)
+    for fmt in range(5):
+        assert qgd.qgd_tp_workspace_size(fmt, 4, 256, 1024) >= 64 * 1024
+        assert qgd.qgd_tp_workspace_size(fmt, 4, 256, 1024) >= qgd.qgd_layer_workspace_size(fmt, 4, 256, 1024)
+
+    def call(desc, fmt=0, M=4, N=256, K=1024, ws=P(1 << 20), wsn=1 << 20):
+        return L.qlinear_tp_bf16(fmt, P(16), K, P(16), P(16), None, M, N, K,
+                                 ctypes.byref(desc) if desc is not None else None, ws, wsn, None)
+
+    assert call(None) == -1
+    assert call(_tp_desc(ranks=0)) == -1
+    assert call(_tp_desc(ranks=9)) == -1
+    assert call(_tp_desc(rank=2)) == -1
+    assert call(_tp_desc(epoch=0)) == -1
+    assert call(_tp_desc(col0=300)) == -1                 # shard past the full output
+    assert call(_tp_desc(ldy=260)) == -1                  # not a multiple of 8
+    assert call(_tp_desc(null_y=True)) == -1
+    assert call(_tp_desc(), fmt=0, M=129) == -2           # beyond the Swap-AB kernel's 128 tokens
+    assert call(_tp_desc(), fmt=2, M=33) == -2            # Block_FP8: 32
+    assert call(_tp_desc(), fmt=4, M=65, K=1024) == -2    # NVFP4: 64
+    assert call(_tp_desc(), ws=None, wsn=0) == -3
+    assert call(_tp_desc(), fmt=5) == -1
+    assert L.qgd_tp_wait(None, 1, 1, None) == -1
+    assert L.qgd_tp_wait(P(16), 0, 1, None) == -1
+    assert L.qgd_tp_wait(P(16), 9, 1, None) == -1
+    assert L.qgd_tp_wait(P(16), 1, 0, None) == -1
+    assert L.qgd_tp_wait(P(18), 1, 1, None) == -1
+    p = ctypes.c_void_p(0)
+    assert L.qgd_ipc_malloc(0, ctypes.byref(p), ctypes.create_string_buffer(64)) == -1
+    assert L.qgd_ipc_malloc(256, None, ctypes.create_string_buffer(64)) == -1
+    assert L.qgd_ipc_open(None, ctypes.byref(p)) == -1
+    assert L.qgd_ipc_close(None) == -1 and L.qgd_ipc_free(None) == -1
