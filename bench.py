@@ -617,6 +617,73 @@ def chain_table(device, reps: int = 20) -> list:
     return rows
 
 
+def tp_table(device, ms=(1, 32), gs=(1, 8), reps: int = 10) -> list:
+    """Column-parallel layer calls on one GPU (FP8_Dynamic, 8B-class shapes):
+    the share of one of G ranks -- an N/G-row weight shard -- as a plain
+    layer call, and as the column-parallel call whose epilogue stores every
+    element to all G full outputs (here G buffers of this GPU standing in for
+    the peers' memory) and raises the flags.  At G = 1 also the call followed
+    by its wait kernel.  Each a graph of calls over >= 3x L2 of weight
+    copies; microseconds per call."""
+    import quantized_gemm_decode_b200 as qgd
+    from quantized_gemm_decode_b200.linear import quantize_weight
+
+    F = qgd.FMT_FP8_DYNAMIC
+    rows = []
+
+    def per_call_us(fn, copies):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for c in range(copies):
+                fn(c)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in range(copies):
+                fn(c)
+        us = time_graph(g, reps, 3) * 1e3 / copies
+        del g
+        return round(us, 2)
+
+    for (N, K) in workloads.SHAPES_8B:
+        for G in gs:
+            n = N // G
+            copies = max(3, -(-3 * L2_BYTES // (n * K)))
+            wq, sw, _ = quantize_weight(synth.weights(n, K, 3001).to(device), FP8_DYNAMIC)
+            wqs = [wq.clone() for _ in range(copies)]
+            for M in ms:
+                x = synth.activations(M, K, 3001, outliers=True).to(device)
+                y = torch.empty((M, n), dtype=torch.bfloat16, device=device)
+                outs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(G)]
+                flags = [torch.zeros(G + 1, dtype=torch.int32, device=device) for _ in range(G)]
+                ws = qgd.Workspace(max(qgd.qgd_tp_workspace_size(F, M, n, K), qgd.qgd_layer_workspace_size(F, M, n, K)),
+                                   device)
+
+                def plain(c):
+                    qgd.qlinear_bf16(F, x, wqs[c], sw, y=y, ws=ws)
+
+                def tp(c):
+                    qgd.qlinear_tp_bf16(F, x, wqs[c], sw, None, ranks=G, rank=0, col0=0, ldy=N, ys=outs,
+                                        flags=flags, ws=ws)
+
+                def tp_wait(c):
+                    tp(c)
+                    qgd.qgd_tp_wait(flags[0], G)
+
+                row = {"M": M, "N": N, "K": K, "ranks": G, "shard_n": n, "layer_us": per_call_us(plain, copies),
+                       "tp_us": per_call_us(tp, copies)}
+                if G == 1:
+                    row["tp_wait_us"] = per_call_us(tp_wait, copies)
+                rows.append(row)
+            del wqs, wq
+            torch.cuda.empty_cache()
+    if qgd.qgd_device_error() != 0:
+        raise RuntimeError(f"device error {qgd.qgd_device_error()} during the column-parallel table")
+    return rows
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
@@ -776,7 +843,7 @@ def emit(out: dict, detail_path: str | None, stream=None) -> str:
     `detail_path` if given, then print the headline as the last line."""
     stream = stream or sys.stdout
     big = {k: out[k] for k in ("per_call", "formats", "large_m", "tensor_probe", "cpu_baseline", "roofline",
-                               "e2e", "splitk_modes", "chain", "fused") if k in out}
+                               "e2e", "splitk_modes", "chain", "fused", "tensor_parallel") if k in out}
     for k, v in big.items():
         stream.write(f"detail {k} {json.dumps(v)}\n")
     if detail_path:
@@ -916,6 +983,13 @@ def render_report(d: dict) -> str:
         out.append("| M | us per chain | whole-path GB/s |\n|---:|---:|---:|")
         for r in d["chain"]:
             out.append(f"| {r['M']} | {r['us_per_chain']} | {r['gbs']} |")
+    if "tensor_parallel" in d:
+        out.append("\nColumn-parallel calls on one GPU (FP8_Dynamic; one rank's N/G shard; us per call):\n")
+        out.append("| M | N x K | ranks G | shard rows | layer call | column-parallel call (G outputs) | + wait |\n"
+                   "|---:|---|---:|---:|---:|---:|---:|")
+        for r in d["tensor_parallel"]:
+            out.append(f"| {r['M']} | {r['N']} x {r['K']} | {r['ranks']} | {r['shard_n']} | {r['layer_us']} | "
+                       f"{r['tp_us']} | {r.get('tp_wait_us', '')} |")
     if "cpu_baseline" in d:
         cb = d["cpu_baseline"]
         st = cb.get("single_thread", {})
@@ -1088,6 +1162,7 @@ def main():
         out["large_m"] = {f: large_m_summary(f, device, pk, probe=probe) for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)}
         out["splitk_modes"] = splitk_modes_table(device)
         out["chain"] = chain_table(device)
+        out["tensor_parallel"] = tp_table(device)
         out.update(extra)
         ds = keep
     if dist.rank == 0 and dist.world == 1 and not args.quick and not args.no_cpu_baseline:

@@ -336,19 +336,21 @@ QGD_API qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* w
  *              process (this GPU's own buffer at y[rank]; the others opened
  *              with qgd_ipc_open, or plain pointers when every "rank" runs on
  *              one GPU), 16-byte aligned
- *   flags[r]   rank r's flag array: G uint32 entries, zero-filled before the
- *              first call, as addressed from this process
- *   epoch      nonzero, one more than the previous call's (every rank uses
- *              the same sequence 1, 2, 3, ... on the same flags; it may wrap,
- *              skipping 0)
+ *   flags[r]   rank r's flag array as addressed from this process: G + 1
+ *              uint32 words, zero-filled before the first call.  Entry j
+ *              holds the number of calls rank j has completed; word G is
+ *              rank r's own call counter
  *
- * After the last of this call's CTAs has stored its output, the kernel sets
- * entry `rank` of every rank's flag array to `epoch` (a system-scope
- * release).  A rank reads the full Y only after qgd_tp_wait on its own flags
- * in stream order after its own call.  Because another rank may already run
- * its next call and write into this rank's Y while this rank still reads the
- * previous result, alternate between two output buffers (by epoch parity);
- * the flags need no second copy.
+ * After the last of this call's CTAs has stored its output, the kernel adds
+ * one to this rank's counter (word G of flags[rank]; 0 is skipped when it
+ * wraps) and writes the new count to entry `rank` of every rank's flag array
+ * (a system-scope release).  The count lives on the device, so the call can
+ * be captured in a CUDA graph and replayed.  Every rank must make the same
+ * sequence of calls on the same flag arrays.  A rank reads the full Y only
+ * after qgd_tp_wait on its own flags in stream order after its own call.
+ * Because another rank may already run its next call and write into this
+ * rank's Y while this rank still reads the previous result, alternate
+ * between two output buffers (the flags need no second copy).
  *
  * Plan: the layer plan for (fmt, M, N, K) forced to Swap-AB (the Standard
  * kernels have no such epilogue) and to a reduction inside the GEMM kernel
@@ -371,7 +373,6 @@ typedef struct {
   int ldy;
   void* y[QGD_MAX_TP_RANKS];
   unsigned int* flags[QGD_MAX_TP_RANKS];
-  unsigned int epoch;
 } qgd_tp;
 
 QGD_API size_t qgd_tp_workspace_size(int fmt, int M, int N, int K);
@@ -379,15 +380,16 @@ QGD_API qgd_status qlinear_tp_bf16(int fmt, const void* x_bf16, int ldx, const v
                                    const void* sw_block, int M, int N, int K, const qgd_tp* tp, void* ws,
                                    size_t ws_bytes, void* stream);
 
-/* Enqueue, on `stream`, a one-thread kernel that waits until every one of
- * flags[0..ranks-1] (this rank's own flag array) holds `epoch` or a later
- * value (compared modulo 2^32), with acquire semantics at system scope, so
- * that kernels after it on the stream see every rank's output.  A flag still
- * behind after about one second makes the kernel record device error 6
- * (qgd_device_error) and return; the output is then incomplete.  Launch it
- * only after this rank's own qlinear_tp_bf16 in the same stream: it must
- * never wait for a kernel of its own GPU. */
-QGD_API qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, unsigned int epoch, void* stream);
+/* Enqueue, on `stream`, a one-thread kernel that reads this rank's call
+ * count e from word `ranks` of its own flag array `flags` and waits until
+ * every one of flags[0..ranks-1] holds e or a later count (compared modulo
+ * 2^32), with acquire semantics at system scope, so that kernels after it on
+ * the stream see every rank's output.  A flag still behind after about one
+ * second makes the kernel record device error 6 (qgd_device_error) and
+ * return; the output is then incomplete.  Launch it only after this rank's
+ * own qlinear_tp_bf16 in the same stream: it must never wait for a kernel of
+ * its own GPU. */
+QGD_API qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, void* stream);
 
 /* Buffers shared between processes (CUDA IPC).  qgd_ipc_malloc allocates
  * `bytes` of device memory on the current device, zero-fills it

@@ -70,8 +70,7 @@ IPC_HANDLE_BYTES = 64
 
 class _Tp(ctypes.Structure):
     _fields_ = [("ranks", ctypes.c_int), ("rank", ctypes.c_int), ("col0", ctypes.c_int), ("ldy", ctypes.c_int),
-                ("y", ctypes.c_void_p * MAX_TP_RANKS), ("flags", ctypes.c_void_p * MAX_TP_RANKS),
-                ("epoch", ctypes.c_uint)]
+                ("y", ctypes.c_void_p * MAX_TP_RANKS), ("flags", ctypes.c_void_p * MAX_TP_RANKS)]
 
 
 class _Plan(ctypes.Structure):
@@ -123,7 +122,7 @@ def lib() -> ctypes.CDLL:
             "qlinear_nvfp4": [P, P, P, P, P, P, P, I, I, I, P, S, P],
             "qlinear_nvfp4_bf16": [P, I, P, P, P, P, I, I, I, P, S, P],
             "qlinear_tp_bf16": [I, P, I, P, P, P, I, I, I, ctypes.POINTER(_Tp), P, S, P],
-            "qgd_tp_wait": [P, I, ctypes.c_uint, P],
+            "qgd_tp_wait": [P, I, P],
             "qgd_ipc_malloc": [S, ctypes.POINTER(ctypes.c_void_p), P],
             "qgd_ipc_open": [P, ctypes.POINTER(ctypes.c_void_p)],
             "qgd_ipc_close": [P],
@@ -559,24 +558,23 @@ def qgd_tp_workspace_size(fmt: int, M: int, N: int, K: int) -> int:
 
 
 def qlinear_tp_bf16(fmt: int, x: torch.Tensor, wq, sw, sw_block, *, ranks: int, rank: int, col0: int, ldy: int,
-                    ys, flags, epoch: int, ws, stream=None) -> None:
+                    ys, flags, ws, stream=None) -> None:
     """Column-parallel layer call: this rank's weight shard (wq [N, K] with
     its scales; NVFP4: sw = fp32 row scales, sw_block = E4M3 block scales)
     against the replicated bf16 activations x [M, K].  Every finished output
     element goes to columns [col0, col0 + N) of all ranks' full outputs
     ys[r] (bf16 [>= M, ldy], device pointers or tensors as addressed from this
-    process), and entry `rank` of every rank's flag array flags[r] is set to
-    `epoch` when the call is done.  Follow with qgd_tp_wait on this rank's
-    own flags before reading its full output."""
+    process); when the call is done, its new call count (word `ranks` of this
+    rank's own flag array, advanced on the device) goes to entry `rank` of
+    every rank's flag array flags[r] (ranks + 1 uint32 words each).  Follow
+    with qgd_tp_wait on this rank's own flags before reading its full output."""
     ldx = _activation_rows(x)
     M, K = x.shape
     N = _layer_weight_operands(fmt, wq, sw, sw_block, K)
     if len(ys) != ranks or len(flags) != ranks or not 1 <= ranks <= MAX_TP_RANKS:
         raise ValueError(f"need one output and one flag array per rank (1..{MAX_TP_RANKS} ranks)")
-    if not (0 <= epoch < 2 ** 32):
-        raise ValueError("epoch must fit in 32 bits")
     tp = _Tp()
-    tp.ranks, tp.rank, tp.col0, tp.ldy, tp.epoch = ranks, rank, col0, ldy, epoch
+    tp.ranks, tp.rank, tp.col0, tp.ldy = ranks, rank, col0, ldy
     for r in range(ranks):
         tp.y[r] = _ptr(ys[r]).value
         tp.flags[r] = _ptr(flags[r]).value
@@ -589,10 +587,10 @@ def qlinear_tp_bf16(fmt: int, x: torch.Tensor, wq, sw, sw_block, *, ranks: int, 
                                  ctypes.c_void_p(wsp), wsn, _stream(stream)), "qlinear_tp_bf16")
 
 
-def qgd_tp_wait(flags, ranks: int, epoch: int, stream=None) -> None:
-    """Enqueue the wait for every rank's flag in this rank's own flag array
-    (a tensor or a device pointer) to reach `epoch`."""
-    _check(lib().qgd_tp_wait(_ptr(flags), ranks, epoch, _stream(stream)), "qgd_tp_wait")
+def qgd_tp_wait(flags, ranks: int, stream=None) -> None:
+    """Enqueue the wait for every rank's entry in this rank's own flag array
+    (a tensor or a device pointer) to reach this rank's call count."""
+    _check(lib().qgd_tp_wait(_ptr(flags), ranks, _stream(stream)), "qgd_tp_wait")
 
 
 def ipc_malloc(nbytes: int) -> tuple:

@@ -518,7 +518,6 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
   a.tp_rank = 0;
   a.tp_col0 = 0;
   a.tp_ldy = 0;
-  a.tp_epoch = 0;
   a.tp_done = nullptr;
   for (int r = 0; r < kMaxTpRanks; ++r) {
     a.tp_y[r] = nullptr;
@@ -529,7 +528,6 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
     a.tp_rank = tp->rank;
     a.tp_col0 = tp->col0;
     a.tp_ldy = tp->ldy;
-    a.tp_epoch = tp->epoch;
     a.tp_done = tp_done;
     for (int r = 0; r < tp->ranks; ++r) {
       a.tp_y[r] = static_cast<uint16_t*>(tp->y[r]);
@@ -866,7 +864,6 @@ qgd_status qlinear_tp_bf16(int fmt, const void* x_bf16, int ldx, const void* wq,
   if (!tp) return fail(QGD_ERR_INVALID, "null tensor-parallel descriptor");
   if (tp->ranks < 1 || tp->ranks > kMaxTpRanks || tp->rank < 0 || tp->rank >= tp->ranks)
     return fail(QGD_ERR_INVALID, "rank %d of %d ranks (1..%d ranks)", tp->rank, tp->ranks, kMaxTpRanks);
-  if (tp->epoch == 0) return fail(QGD_ERR_INVALID, "epoch 0 is the flags' initial value");
   if (N <= 0 || tp->col0 < 0 || tp->ldy % 8 != 0 || static_cast<long long>(tp->col0) + N > tp->ldy)
     return fail(QGD_ERR_INVALID, "shard columns [%d, %d) outside a full output %d wide (a multiple of 8)", tp->col0,
                 tp->col0 + N, tp->ldy);
@@ -886,13 +883,12 @@ qgd_status qlinear_tp_bf16(int fmt, const void* x_bf16, int ldx, const void* wq,
                    static_cast<const uint8_t*>(sw_block), tp);
 }
 
-qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, unsigned int epoch, void* stream) {
+qgd_status qgd_tp_wait(const unsigned int* flags, int ranks, void* stream) {
   if (!flags || reinterpret_cast<uintptr_t>(flags) % 4 != 0) return fail(QGD_ERR_INVALID, "null or misaligned flags");
   if (ranks < 1 || ranks > kMaxTpRanks) return fail(QGD_ERR_INVALID, "%d ranks (1..%d)", ranks, kMaxTpRanks);
-  if (epoch == 0) return fail(QGD_ERR_INVALID, "epoch 0 is the flags' initial value");
   qgd_status st;
   if ((st = check_device()) != QGD_OK) return st;
-  const cudaError_t e = launch_tp_wait(flags, ranks, epoch, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_tp_wait(flags, ranks, pdl_enabled(), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tensor-parallel wait launch");
   return QGD_OK;
 }

@@ -208,20 +208,31 @@ __device__ __forceinline__ void store_swap_final(uint32_t accbits, int m, int n,
 }
 
 // Column-parallel completion: after every CTA's output is out, the last CTA
-// to finish publishes this rank's epoch in every rank's flag array (system
-// scope: the readers are other GPUs).  Called by all threads of a CTA at its
-// end.
+// to finish advances this rank's call counter (word `ranks` of its own flag
+// array; 0 is skipped when it wraps) and publishes the new value in entry
+// `rank` of every rank's flag array (system scope: the readers are other
+// GPUs).  The counter lives on the device, so a captured graph advances it on
+// every replay.  Called by all threads of a CTA at its end.
 __device__ __forceinline__ void tp_signal_done(const GemmArgs& a) {
   if (a.tp_ranks == 0) return;
-  __threadfence_system();  // each thread's output stores, to every rank, before the CTA's arrival
-  __syncthreads();
+  __syncthreads();  // every thread's output stores, to every rank, precede thread 0's fence
   if (threadIdx.x == 0) {
     const unsigned total = gridDim.x * gridDim.y * gridDim.z;
-    const unsigned prev = atomicAdd(a.tp_done, 1u);
+    unsigned prev;
+    // the arrival releases this CTA's stores (the barrier above ordered every
+    // thread's before it); the last arrival acquires every other CTA's, and its
+    // system-scope releases below pass them all on to the other ranks
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.tp_done) : "memory");
     if (prev == total - 1) {
-      __threadfence_system();  // every CTA's stores (their fences preceded their arrivals)
+      unsigned* own = a.tp_flag[a.tp_rank];
+      unsigned epoch = *reinterpret_cast<volatile unsigned*>(own + a.tp_ranks) + 1u;
+      if (epoch == 0u) epoch = 1u;
+      own[a.tp_ranks] = epoch;  // read by this rank's wait, after this kernel in stream order
+      // one system-scope fence releases the output to every rank's flag (a
+      // fence followed by strong stores); a release per store costs a fence each
+      asm volatile("fence.acq_rel.sys;" ::: "memory");
       for (int r = 0; r < a.tp_ranks; ++r)
-        asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(a.tp_flag[r] + a.tp_rank), "r"(a.tp_epoch)
+        asm volatile("st.relaxed.sys.global.u32 [%0], %1;" ::"l"(a.tp_flag[r] + a.tp_rank), "r"(epoch)
                      : "memory");
       *a.tp_done = 0u;  // ready for the next call
     }
@@ -1919,15 +1930,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ===========================================================================
-// Tensor-parallel wait: one thread reads each rank's entry of this rank's
-// flag array (acquire, system scope) until it holds the call's epoch (or a
-// later one: a rank may already have finished its next call), giving
-// up after about kWaitLimitNs per rank (error kErrWaitPeers).  Launched in
-// stream order after this rank's GEMM, so it never waits on a kernel of its
-// own GPU; the kernels after it read the full output.
+// Tensor-parallel wait: one thread takes the epoch of this rank's last call
+// from word `ranks` of its own flag array, then reads each rank's entry
+// (acquire, system scope) until it holds that epoch (or a later one: a rank
+// may already have finished its next call), giving up after about
+// kWaitLimitNs per rank (error kErrWaitPeers).  Launched in stream order after
+// this rank's GEMM, so it never waits on a kernel of its own GPU; the kernels
+// after it read the full output.
 // ===========================================================================
-__global__ void __launch_bounds__(32) tp_wait_kernel(const unsigned* flags, int ranks, unsigned epoch) {
+__global__ void __launch_bounds__(32) tp_wait_kernel(const unsigned* flags, int ranks) {
+  griddep_launch_dependents();  // the next kernel may set up and stream its weights meanwhile
+  griddep_wait();               // this rank's GEMM (which advanced the count) is complete
   if (threadIdx.x != 0) return;
+  const unsigned epoch = *reinterpret_cast<const volatile unsigned*>(flags + ranks);
   for (int r = 0; r < ranks; ++r) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0;; ++i) {
@@ -2225,9 +2240,10 @@ extern "C" __attribute__((visibility("default"))) int qgd_debug_trace(unsigned l
 }
 #endif
 
-cudaError_t launch_tp_wait(const unsigned* flags, int ranks, unsigned epoch, cudaStream_t stream) {
-  // no programmatic dependency: it starts only after this rank's GEMM is done
-  return launch_ex(tp_wait_kernel, dim3(1), dim3(32), 0, stream, false, flags, ranks, epoch);
+cudaError_t launch_tp_wait(const unsigned* flags, int ranks, bool pdl, cudaStream_t stream) {
+  // with a programmatic dependency it starts early and reads the count only
+  // after its griddepcontrol.wait, once this rank's GEMM is complete
+  return launch_ex(tp_wait_kernel, dim3(1), dim3(32), 0, stream, pdl, flags, ranks);
 }
 
 cudaError_t read_device_error(unsigned int* code) {

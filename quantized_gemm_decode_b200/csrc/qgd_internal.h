@@ -63,13 +63,13 @@ struct GemmArgs {
   // Column-parallel tensor parallelism (Swap-AB): this rank's output columns
   // (its weight shard's N) go to columns [tp_col0, tp_col0 + N) of every
   // rank's full bf16 output, tp_ldy columns wide, through the ranks' pointers
-  // (peer memory); the last CTA to finish then sets entry tp_rank of every
-  // rank's flag array to tp_epoch.  tp_ranks == 0: a plain call.
+  // (peer memory); the last CTA to finish then advances this rank's call
+  // counter (word tp_ranks of its own flag array) and writes the new value to
+  // entry tp_rank of every rank's flag array.  tp_ranks == 0: a plain call.
   int tp_ranks;
   int tp_rank;
   int tp_col0;
   int tp_ldy;
-  unsigned tp_epoch;
   unsigned* tp_done;  // CTAs finished this call (zero on entry and exit)
   uint16_t* tp_y[kMaxTpRanks];
   unsigned* tp_flag[kMaxTpRanks];
@@ -102,8 +102,9 @@ cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorM
                                  const GemmArgs& a, cudaStream_t stream);
 int pair_max_active_clusters(int fmt, int stages, int kps);
 cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream);
-// Tensor parallelism: wait (bounded) until flags[0..ranks) all equal epoch
-cudaError_t launch_tp_wait(const unsigned* flags, int ranks, unsigned epoch, cudaStream_t stream);
+// Tensor parallelism: wait (bounded) until flags[0..ranks) all reach the
+// epoch in flags[ranks] (this rank's call counter)
+cudaError_t launch_tp_wait(const unsigned* flags, int ranks, bool pdl, cudaStream_t stream);
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();

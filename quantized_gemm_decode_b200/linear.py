@@ -332,8 +332,10 @@ class ColumnParallelLinear:
     Each rank owns one shared device buffer, mapped by all ranks (CUDA IPC):
     two full outputs [max_m, ldy] bf16 (successive calls alternate, so that a
     rank already running its next call never overwrites the output another
-    rank is still reading) and a flag array of one uint32 per rank.  Shards
-    may differ in width; col0 and ldy come from an all-gather of the widths.
+    rank is still reading) and a flag array of one uint32 per rank plus this
+    rank's call counter, which the kernels advance (so a captured graph of the
+    calls stays in step).  Shards may differ in width; col0 and ldy come from
+    an all-gather of the widths.
     """
 
     def __init__(self, w_shard: torch.Tensor | None, fmt: str = "fp8_dynamic", group=None, max_m: int = 32,
@@ -358,14 +360,13 @@ class ColumnParallelLinear:
         self.max_m = max_m
         self.out_bytes = max_m * self.ldy * 2
         self.flags_off = 2 * _align(self.out_bytes)
-        self.nbytes = self.flags_off + _align(4 * self.G)
+        self.nbytes = self.flags_off + _align(4 * (self.G + 1))
         self._ipc = ipc if ipc is not None else _LibraryIpc
         self.own, handle = self._ipc.malloc(self.nbytes)
         handles = self._all_gather(handle)
         self.bases = [self.own if r == self.rank else self._ipc.open(handles[r]) for r in range(self.G)]
         self.ws = qgd.Workspace(qgd.qgd_tp_workspace_size(self.fmt_id, max_m, self.N, self.K), self.device)
         self.calls = 0
-        self.epoch = 0
 
     def _all_gather(self, obj) -> list:
         if self._dist is None:
@@ -373,10 +374,6 @@ class ColumnParallelLinear:
         out = [None] * self.G
         self._dist.all_gather_object(out, obj, group=self.group)
         return out
-
-    def _next_epoch(self) -> int:
-        self.epoch = self.epoch % 0xFFFFFFFF + 1  # 1, 2, ..., 2^32 - 1, 1, ... (0 is the flags' initial value)
-        return self.epoch
 
     def output_ptr(self, rank: int, buf: int) -> int:
         return self.bases[rank] + buf * _align(self.out_bytes)
@@ -392,13 +389,11 @@ class ColumnParallelLinear:
             raise ValueError(f"M={M} exceeds the buffers' {self.max_m} rows")
         buf = self.calls & 1
         self.calls += 1
-        epoch = self._next_epoch()
         if M == 0:
             return buf
         qgd.qlinear_tp_bf16(self.fmt_id, x, self.wq, self.sw, self.sw_block, ranks=self.G, rank=self.rank,
                             col0=self.col0, ldy=self.ldy, ys=[self.output_ptr(r, buf) for r in range(self.G)],
-                            flags=[self.flags_ptr(r) for r in range(self.G)], epoch=epoch, ws=self.ws,
-                            stream=stream)
+                            flags=[self.flags_ptr(r) for r in range(self.G)], ws=self.ws, stream=stream)
         return buf
 
     def wait(self, M: int, buf: int, stream=None) -> torch.Tensor:
@@ -406,7 +401,7 @@ class ColumnParallelLinear:
         the full output [M, ldy] (a view of this rank's shared buffer, valid
         until the call after next)."""
         if M > 0:
-            qgd.qgd_tp_wait(self.flags_ptr(self.rank), self.G, self.epoch, stream=stream)
+            qgd.qgd_tp_wait(self.flags_ptr(self.rank), self.G, stream=stream)
         full = qgd.tensor_at(self.output_ptr(self.rank, buf), (self.max_m, self.ldy), torch.bfloat16, self.device)
         return full[:M]
 

@@ -238,10 +238,11 @@ class Problem:
         return t0.elapsed_time(t1) / (reps * n) * 1e3  # microseconds per call
 
 
-def tune_problem(p: Problem, log=None):
+def tune_problem(p: Problem, log=None, tp: bool = False):
     """Time every candidate, then the ring depth of the three fastest.
     Returns the best (us, variant, split_k, reduce, stages, tile_n, schedule,
-    occupancy, k_slices, fused) and the first pass's results."""
+    occupancy, k_slices, fused) and the first pass's results.  tp: only the
+    plans a column-parallel call runs (Swap-AB, reduced inside the GEMM)."""
     fid = p.fid
     qgd.qgd_set_fused_override(fid, 0)
     qgd.qgd_set_override(fid, qgd.VARIANT_SWAP_AB if p.M <= 32 else qgd.VARIANT_STANDARD, 1, 0, 0, 0,
@@ -265,7 +266,10 @@ def tune_problem(p: Problem, log=None):
         pl = qgd.qgd_get_layer_plan(fid, p.M, p.N, p.K)
         return (us, var, pl["split_k"], r, pl["stages"], t, sch, pl["occupancy"], pl["k_slices"], pl["fused"])
 
-    for var, s, r, t, sch, occ, kps, st0, fz in candidates(p.fmt, p.M, p.N, p.K, num_sms):
+    cands = candidates(p.fmt, p.M, p.N, p.K, num_sms)
+    if tp:
+        cands = [c for c in cands if c[0] == 1 and c[2] != 1]
+    for var, s, r, t, sch, occ, kps, st0, fz in cands:
         qgd.qgd_set_override(fid, var, s, r, st0, t, sch, occ, kps)
         qgd.qgd_set_fused_override(fid, fz)
         ensure_ws()
@@ -299,6 +303,8 @@ def main(argv=None):
     ap.add_argument("--large-m", action="store_true", help="also tune the larger-M buckets")
     ap.add_argument("--resume", action="store_true")
     ap.add_argument("--only-m", default=None, help="comma-separated M values to tune")
+    ap.add_argument("--tp8", action="store_true",
+                    help="also tune the 8-way column-parallel shards of the 8B-class shapes (FP8_Dynamic)")
     args = ap.parse_args(argv)
 
     os.environ["QGD_NO_TABLE"] = "1"
@@ -310,6 +316,8 @@ def main(argv=None):
                        workloads.NV_DECODE) if w.fmt in fmts]
     if args.large_m:
         wls += [w for w in workloads.LARGE if w.fmt in fmts]
+    if args.tp8:
+        wls.append(workloads.FP8_TP8)
     done = {}
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
@@ -343,7 +351,7 @@ def main(argv=None):
                     continue
                 t0 = time.time()
                 p = Problem(wl.fmt, M, N, K, wl.seed, device)
-                best, allres = tune_problem(p, log)
+                best, allres = tune_problem(p, log, tp=(wl is workloads.FP8_TP8))
                 us, var, s, r, st, t, sch, occ, kps, fz = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
                 lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "

@@ -569,9 +569,9 @@ def test_nvfp4_plan_rules_and_rejects():
     assert ws >= 8 * 2048 + 8 * 4 + 8 * 256
 
 
-def _tp_desc(ranks=2, rank=0, col0=0, ldy=512, epoch=1, null_y=False):
+def _tp_desc(ranks=2, rank=0, col0=0, ldy=512, null_y=False):
     d = qgd._Tp()
-    d.ranks, d.rank, d.col0, d.ldy, d.epoch = ranks, rank, col0, ldy, epoch
+    d.ranks, d.rank, d.col0, d.ldy = ranks, rank, col0, ldy
     for r in range(min(max(ranks, 0), qgd.MAX_TP_RANKS)):
         d.y[r] = None if null_y and r == ranks - 1 else 4096 * (r + 1)
         d.flags[r] = 8192 * (r + 1)
@@ -584,7 +584,7 @@ def test_column_parallel_call_rules():
     for name in ("qlinear_tp_bf16", "qgd_tp_wait", "qgd_tp_workspace_size", "qgd_ipc_malloc", "qgd_ipc_open",
                  "qgd_ipc_close", "qgd_ipc_free"):
         assert name in declared_functions()
-    assert ctypes.sizeof(qgd._Tp) == 4 * 4 + 2 * 8 * 8 + 8  # four ints, two pointer arrays, the epoch (padded)
+    assert ctypes.sizeof(qgd._Tp) == 4 * 4 + 2 * 8 * 8  # four ints, two pointer arrays
     # the workspace always holds the 64 KiB counter header (its last word counts finished CTAs)
     for fmt in range(5):
         assert qgd.qgd_tp_workspace_size(fmt, 4, 256, 1024) >= 64 * 1024
@@ -598,7 +598,6 @@ def test_column_parallel_call_rules():
     assert call(_tp_desc(ranks=0)) == -1
     assert call(_tp_desc(ranks=9)) == -1
     assert call(_tp_desc(rank=2)) == -1
-    assert call(_tp_desc(epoch=0)) == -1
     assert call(_tp_desc(col0=300)) == -1                 # shard past the full output
     assert call(_tp_desc(ldy=260)) == -1                  # not a multiple of 8
     assert call(_tp_desc(null_y=True)) == -1
@@ -607,11 +606,10 @@ def test_column_parallel_call_rules():
     assert call(_tp_desc(), fmt=4, M=65, K=1024) == -2    # NVFP4: 64
     assert call(_tp_desc(), ws=None, wsn=0) == -3
     assert call(_tp_desc(), fmt=5) == -1
-    assert L.qgd_tp_wait(None, 1, 1, None) == -1
-    assert L.qgd_tp_wait(P(16), 0, 1, None) == -1
-    assert L.qgd_tp_wait(P(16), 9, 1, None) == -1
-    assert L.qgd_tp_wait(P(16), 1, 0, None) == -1
-    assert L.qgd_tp_wait(P(18), 1, 1, None) == -1
+    assert L.qgd_tp_wait(None, 1, None) == -1
+    assert L.qgd_tp_wait(P(16), 0, None) == -1
+    assert L.qgd_tp_wait(P(16), 9, None) == -1
+    assert L.qgd_tp_wait(P(18), 1, None) == -1
     p = ctypes.c_void_p(0)
     assert L.qgd_ipc_malloc(0, ctypes.byref(p), ctypes.create_string_buffer(64)) == -1
     assert L.qgd_ipc_malloc(256, None, ctypes.create_string_buffer(64)) == -1

@@ -94,6 +94,9 @@ def _fake_result():
                                          "samples": 40, "reasons": []},
         "formats": fmts, "tensor_probe": {"e4m3_tflops": 4443.0, "int8_tops": 4588.0, "how": "z" * 120},
         "large_m": large, "per_call": per_call,
+        "tensor_parallel": [{"M": 1, "N": 4096, "K": 4096, "ranks": 8, "shard_n": 512, "layer_us": 4.1,
+                             "tp_us": 4.3}, {"M": 1, "N": 4096, "K": 4096, "ranks": 1, "shard_n": 4096,
+                                             "layer_us": 8.4, "tp_us": 8.5, "tp_wait_us": 9.9}],
         "cpu_baseline": {"value": 0.047, "unit": "GB/s", "cores": 16, "kind": "oracle", "sample": "s" * 200,
                          "cpu_model": "Some CPU @ 2.70GHz",
                          "single_thread": {"value": 0.006, "unit": "GB/s", "cores": 1, "seconds": 5.0},
@@ -125,3 +128,10 @@ def test_result_line_is_compact_and_last(tmp_path):
     # the full record went to the detail file
     full = json.loads(detail.read_text())
     assert len(full["per_call"]) == 28 and len(full["large_m"][FP8_DYNAMIC]) == 20
+    assert len(full["tensor_parallel"]) == 2
+
+
+def test_report_renders_every_section():
+    rep = bench.render_report(_fake_result())
+    assert "Column-parallel calls on one GPU" in rep and "| 1 | 4096 x 4096 | 8 | 512 | 4.1 | 4.3 |  |" in rep
+    assert "Larger M" in rep and "CPU baseline" in rep

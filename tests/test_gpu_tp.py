@@ -4,8 +4,8 @@ unsharded layer.
 
 The library's own extension of the pages' single-GPU operation: the weight
 rows (output columns) are split over G ranks, each rank's kernel stores its
-columns into every rank's full output and then raises its flag in every
-rank's flag array.  With one GPU the ranks are emulated in one process: all G
+columns into every rank's full output and then advances its call count
+and writes it into every rank's flag array.  With one GPU the ranks are emulated in one process: all G
 calls run first, one after another, each writing all G outputs and flag
 arrays; only then are the G waits enqueued, so no kernel ever waits for a
 kernel that has not yet finished.  The IPC test runs two processes on the
@@ -72,9 +72,9 @@ def check_layer(fmt: str, y: torch.Tensor, yref: np.ndarray, bound: np.ndarray, 
 
 
 def run_emulated(fmt: str, Ms, widths, K: int, seed: int, max_m: int = None):
-    """G = len(widths) ranks on one GPU, one call per entry of Ms (epochs
-    1, 2, ...; outputs alternate between two buffers).  Returns nothing; every
-    rank's full output is checked against the oracle after every call."""
+    """G = len(widths) ranks on one GPU, one call per entry of Ms (outputs
+    alternate between two buffers).  Every rank's full output is checked
+    against the oracle after every call, and its flags against the count."""
     F = FMTS[fmt]
     G, ldy = len(widths), sum(widths)
     col0 = [sum(widths[:r]) for r in range(G)]
@@ -83,10 +83,10 @@ def run_emulated(fmt: str, Ms, widths, K: int, seed: int, max_m: int = None):
     shards = [quantize_weight(w[c:c + n].cuda(), fmt) for c, n in zip(col0, widths)]
     outs = [[torch.full((max_m, ldy), SENTINEL, dtype=torch.int16, device="cuda") for _ in range(G)]
             for _ in range(2)]
-    flags = [torch.zeros(G, dtype=torch.int32, device="cuda") for _ in range(G)]
+    flags = [torch.zeros(G + 1, dtype=torch.int32, device="cuda") for _ in range(G)]  # + the call counter
     wss = [qgd.Workspace(qgd.qgd_tp_workspace_size(F, max_m, n, K)) for n in widths]
     for call, M in enumerate(Ms):
-        epoch, buf = call + 1, call & 1
+        count, buf = call + 1, call & 1
         for o in outs[buf]:
             o.fill_(SENTINEL)
         x = synth.activations(M, K, seed + 7 * call, outliers=True)
@@ -94,13 +94,13 @@ def run_emulated(fmt: str, Ms, widths, K: int, seed: int, max_m: int = None):
         for r in range(G):
             wq, sw, sb = shards[r]
             qgd.qlinear_tp_bf16(F, xd, wq, sw, sb, ranks=G, rank=r, col0=col0[r], ldy=ldy, ys=outs[buf],
-                                flags=flags, epoch=epoch, ws=wss[r])
+                                flags=flags, ws=wss[r])
         for r in range(G):
-            qgd.qgd_tp_wait(flags[r], G, epoch)
+            qgd.qgd_tp_wait(flags[r], G)
         torch.cuda.synchronize()
         assert qgd.qgd_device_error() == 0
         for r in range(G):
-            assert flags[r].cpu().tolist() == [epoch] * G, f"rank {r} flags after call {call}"
+            assert flags[r].cpu().tolist() == [count] * (G + 1), f"rank {r} flags after call {call}"
             # the completion counter (last word of the 64 KiB header) is back to zero
             assert int(wss[r].buf[65536 - 4:65536].view(torch.int32).item()) == 0
         yref, bound = oracle_layer(fmt, x, w)
@@ -158,30 +158,69 @@ def test_tp_single_rank_is_the_plain_layer_call():
     x = synth.activations(M, K, 5).cuda()
     wq, sw, _ = quantize_weight(synth.weights(N, K, 5).cuda(), "fp8_dynamic")
     y = torch.full((M, N + 64), SENTINEL, dtype=torch.int16, device="cuda")
-    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flags = torch.tensor([2, 2], dtype=torch.int32, device="cuda")  # two calls already made
     ws = qgd.Workspace(qgd.qgd_tp_workspace_size(F, M, N, K))
-    qgd.qlinear_tp_bf16(F, x, wq, sw, None, ranks=1, rank=0, col0=64, ldy=N + 64, ys=[y], flags=[flags], epoch=3,
-                        ws=ws)
-    qgd.qgd_tp_wait(flags, 1, 3)
+    qgd.qlinear_tp_bf16(F, x, wq, sw, None, ranks=1, rank=0, col0=64, ldy=N + 64, ys=[y], flags=[flags], ws=ws)
+    qgd.qgd_tp_wait(flags, 1)
     y_plain = qgd.qlinear_bf16(F, x, wq, sw)
     torch.cuda.synchronize()
-    assert qgd.qgd_device_error() == 0 and flags.item() == 3
+    assert qgd.qgd_device_error() == 0 and flags.tolist() == [3, 3]
     assert torch.equal(y[:, 64:], y_plain.view(torch.int16))
     assert bool((y[:, :64] == SENTINEL).all())
 
 
 def test_tp_wait_gives_up_on_a_flag_nobody_sets():
     # bounded wait: about one second, then device error 6 and the kernel returns
-    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
-    qgd.qgd_tp_wait(flags, 1, 1)
+    flags = torch.tensor([0, 1], dtype=torch.int32, device="cuda")  # count 1, nobody has reached it
+    qgd.qgd_tp_wait(flags, 1)
     torch.cuda.synchronize()
     assert qgd.qgd_device_error() == 6
     qgd.qgd_clear_device_error()
-    # the context is still usable: a later flag value than the epoch also ends the wait
-    flags.fill_(5)
-    qgd.qgd_tp_wait(flags, 1, 4)
+    # the context is still usable: a count past this rank's own also ends the wait
+    flags.copy_(torch.tensor([5, 4], dtype=torch.int32))
+    qgd.qgd_tp_wait(flags, 1)
     torch.cuda.synchronize()
     assert qgd.qgd_device_error() == 0
+
+
+def test_tp_graph_replay_advances_the_count():
+    # the count lives on the device: a captured pair of ranks replays correctly
+    F, M, K, widths = qgd.FMT_FP8_DYNAMIC, 4, 1024, [256, 384]
+    G, ldy = 2, sum(widths)
+    w = synth.weights(ldy, K, 31)
+    shards = [quantize_weight(w[c:c + n].cuda(), "fp8_dynamic") for c, n in ((0, 256), (256, 384))]
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    outs = [torch.zeros((M, ldy), dtype=torch.int16, device="cuda") for _ in range(G)]
+    flags = [torch.zeros(G + 1, dtype=torch.int32, device="cuda") for _ in range(G)]
+    wss = [qgd.Workspace(qgd.qgd_tp_workspace_size(F, M, n, K)) for n in widths]
+
+    def step():
+        for r in range(G):
+            qgd.qlinear_tp_bf16(F, x, *shards[r], ranks=G, rank=r, col0=sum(widths[:r]), ldy=ldy, ys=outs,
+                                flags=flags, ws=wss[r])
+        for r in range(G):
+            qgd.qgd_tp_wait(flags[r], G)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # count 1
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()  # captured, not run
+    for rep in range(3):
+        xr = synth.activations(M, K, 40 + rep)
+        x.copy_(xr.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        assert qgd.qgd_device_error() == 0
+        for r in range(G):
+            assert flags[r].cpu().tolist() == [rep + 2] * (G + 1)
+        yref, bound = oracle_layer("fp8_dynamic", xr, w)
+        for r in range(G):
+            check_layer("fp8_dynamic", outs[r].view(torch.bfloat16), yref, bound, K, f"replay {rep} rank {r}")
 
 
 def test_tp_rejects_bad_descriptors():
@@ -189,13 +228,12 @@ def test_tp_rejects_bad_descriptors():
     x = synth.activations(M, K, 1).cuda()
     wq, sw, _ = quantize_weight(synth.weights(N, K, 1).cuda(), "fp8_dynamic")
     y = torch.zeros((M, 512), dtype=torch.int16, device="cuda")
-    flags = torch.zeros(2, dtype=torch.int32, device="cuda")
+    flags = torch.zeros(3, dtype=torch.int32, device="cuda")
     ws = qgd.Workspace(qgd.qgd_tp_workspace_size(F, M, N, K))
     common = dict(ranks=2, ys=[y, y], flags=[flags, flags], ws=ws)
-    bad = [dict(rank=2, col0=0, ldy=512, epoch=1),       # rank out of range
-           dict(rank=0, col0=300, ldy=512, epoch=1),     # shard past the full output
-           dict(rank=0, col0=0, ldy=500, epoch=1),       # ldy not a multiple of 8
-           dict(rank=0, col0=0, ldy=512, epoch=0)]       # epoch 0
+    bad = [dict(rank=2, col0=0, ldy=512),       # rank out of range
+           dict(rank=0, col0=300, ldy=512),     # shard past the full output
+           dict(rank=0, col0=0, ldy=500)]       # ldy not a multiple of 8
     for kw in bad:
         with pytest.raises(qgd.QGDError) as e:
             qgd.qlinear_tp_bf16(F, x, wq, sw, None, **common, **kw)
@@ -203,7 +241,7 @@ def test_tp_rejects_bad_descriptors():
     xb = synth.activations(40, 1024, 2).cuda()
     wb, swb, _ = quantize_weight(synth.weights(256, 1024, 2).cuda(), "block_fp8")
     with pytest.raises(qgd.QGDError) as e:  # Block_FP8 Swap-AB covers 32 tokens
-        qgd.qlinear_tp_bf16(qgd.FMT_BLOCK_FP8, xb, wb, swb, None, rank=0, col0=0, ldy=512, epoch=1,
+        qgd.qlinear_tp_bf16(qgd.FMT_BLOCK_FP8, xb, wb, swb, None, rank=0, col0=0, ldy=512,
                             **dict(common, ws=qgd.Workspace(1 << 20)))
     assert e.value.status == -2
     torch.cuda.synchronize()

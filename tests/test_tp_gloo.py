@@ -3,7 +3,8 @@ ranks on the CPU: shard offsets and the full width from the ranks' shard
 widths, the exchange of buffer handles (each rank maps every other rank's
 buffer and never its own), the pointers handed to the kernel call (every
 rank's output buffer, alternating between two per call, and every rank's
-flag array), the epoch sequence, and the collective teardown order.  The
+flag array), the alternation of output buffers, and the collective
+teardown order.  The
 shared-memory calls and the kernel call are replaced by recording fakes."""
 import os
 import socket
@@ -63,8 +64,8 @@ def _rank_main(rank, world, port, widths, q):
         x = torch.zeros((4, K), dtype=torch.bfloat16)
         bufs = [layer.launch(x) for _ in range(3)] + [layer.launch(torch.zeros((0, K), dtype=torch.bfloat16))]
         layer.close()
-        q.put((rank, layer.col0, layer.ldy, layer.own, list(ipc.log), bufs, layer.epoch,
-               [(kw["rank"], kw["ranks"], kw["col0"], kw["ldy"], kw["ys"], kw["flags"], kw["epoch"])
+        q.put((rank, layer.col0, layer.ldy, layer.own, list(ipc.log), bufs, layer.calls,
+               [(kw["rank"], kw["ranks"], kw["col0"], kw["ldy"], kw["ys"], kw["flags"])
                 for _, kw in calls], layer.out_bytes, layer.flags_off, None))
     except Exception as exc:
         q.put((rank,) + (None,) * 10 + (repr(exc),))
@@ -84,32 +85,24 @@ def test_column_parallel_plumbing_over_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for r, col0, ldy, own, log, bufs, epoch, calls, out_bytes, flags_off, exc in res:
+    for r, col0, ldy, own, log, bufs, ncalls, calls, out_bytes, flags_off, exc in res:
         assert exc is None, f"rank {r}: {exc}"
         assert col0 == sum(widths[:r]) and ldy == sum(widths)
         assert own == (r + 1) << 32
         peer = 1 - r
         peer_ptr = ((peer + 1) << 32) + (1 << 20)
-        # one buffer of two outputs [8, 640] bf16 and the flags, each 256-byte aligned
+        # one buffer of two outputs [8, 640] bf16 and the flags (2 entries + the counter), each 256-byte aligned
         assert out_bytes == 8 * 640 * 2 and flags_off == 2 * 10240
         assert log[0] == ("malloc", flags_off + 256)
         assert log[1:] == [("open", peer), ("close", peer_ptr), ("free", own)]
-        assert bufs == [0, 1, 0, 1] and epoch == 4          # the empty call takes an epoch, launches nothing
+        assert bufs == [0, 1, 0, 1] and ncalls == 4         # the empty call takes a buffer turn, launches nothing
         assert len(calls) == 3
         base = {r: own, peer: peer_ptr}
-        for i, (rank, ranks, c0, ld, ys, flags, ep) in enumerate(calls):
-            assert (rank, ranks, c0, ld, ep) == (r, 2, col0, ldy, i + 1)
+        for i, (rank, ranks, c0, ld, ys, flags) in enumerate(calls):
+            assert (rank, ranks, c0, ld) == (r, 2, col0, ldy)
             off = (i & 1) * 10240
             assert ys == [base[0] + off, base[1] + off]
             assert flags == [base[0] + flags_off, base[1] + flags_off]
-
-
-def test_epochs_skip_zero_when_they_wrap():
-    from quantized_gemm_decode_b200.linear import ColumnParallelLinear
-
-    layer = ColumnParallelLinear.__new__(ColumnParallelLinear)
-    layer.epoch = 0xFFFFFFFE
-    assert [layer._next_epoch() for _ in range(3)] == [0xFFFFFFFF, 1, 2]
 
 
 def test_single_process_needs_no_group():
