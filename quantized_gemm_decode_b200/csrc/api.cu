@@ -218,9 +218,10 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
     while (tiles * s < g_num_sms && s * 2 <= nkt && s < 256) s *= 2;
     p.split_k = s;  // used by the grid schedule
   } else {
-    // Larger M: Standard tiles, one persistent CTA per SM.
+    // Larger M: Standard tiles, one persistent CTA per SM (Block_FP8: two
+    // weight blocks per tile, which keeps the tensor pipe twice as busy)
     p.variant = kStandard;
-    p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+    p.tile_n = 256;
     p.split_k = 1;
     p.schedule = kPersistent;
   }
@@ -271,7 +272,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
   if (p.variant < kStandard || p.variant > kStandardPair) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (p.variant == kStandardPair) p.tile_n = 256;
-  else if (fmt == kFmtBlock || (p.tile_n != 128 && p.tile_n != 256)) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
+  else if (p.tile_n != 128 && p.tile_n != 256) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
   if (p.variant == kStandardPair) {
     p.split_k = 1;
     p.reduce = kLastCta;

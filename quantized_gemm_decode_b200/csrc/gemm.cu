@@ -1277,13 +1277,14 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
                     const GemmArgs a) {
   constexpr bool kInt = (kFmt == kFmtINT8);
   constexpr bool kBlock = (kFmt == kFmtBlock);
-  static_assert(!kBlock || kTileN == 128, "Block_FP8 tiles are one weight block wide");
   constexpr uint32_t kEpi = std_threads<kFmt>() - 64;  // epilogue threads
   constexpr int kHalf = kBlock ? kTileN / kBlockEpiGroups : kTileN;  // columns per epilogue thread
-  // Block_FP8: a ring of 4 per-K-block accumulators (the MMA runs up to three
-  // K blocks ahead of the promotion); else: a per-tile double buffer.
-  constexpr int kSlots = kBlock ? 4 : 2;
-  constexpr uint32_t kCols = kSlots * kTileN;  // 512 (Block_FP8: 4 x 128; else 2 x 256) or 256
+  // Block_FP8: a ring of per-K-block accumulators (4 x 128 columns, or 2 x
+  // 256 for tiles two weight blocks wide, whose epilogue warp pairs then each
+  // own one weight block); else: a per-tile double buffer.
+  static_assert(!kBlock || kTileN == 128 || kTileN == 256, "Block_FP8 tiles are one or two weight blocks wide");
+  constexpr int kSlots = kBlock ? (kTileN == 128 ? 4 : 2) : 2;
+  constexpr uint32_t kCols = kSlots * kTileN;  // 512 (4 x 128 or 2 x 256) or 256
   constexpr uint32_t kXBytes = kStdTileM * kTileK;
   constexpr uint32_t kWBytes = kTileN * kTileK;
   constexpr uint32_t kIdesc = idesc_mma(kInt ? 2 : 1, kInt ? 1 : 0, kStdTileM, kTileN);
@@ -1465,14 +1466,18 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
         float facc[kHalf];
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) facc[j] = 0.f;
+        // this thread's columns lie in one 128-row weight block (n0 / 128); in
+        // a 256-wide tile past N (N an odd number of blocks) the second half
+        // has no block and no scale
+        const bool live = in_m && n0 < N;
         const float* sxrow = a.sx + static_cast<size_t>(in_m ? m : 0) * KB;
-        const float* swrow = a.sw + static_cast<size_t>(n_tile) * KB;
+        const float* swrow = a.sw + static_cast<size_t>(n0 < N ? n0 / 128 : 0) * KB;
         // scales one K block ahead, so their load latency hides behind a block
-        float sc_next = (in_m && kt0 < kt1) ? __ldg(sxrow + kt0) * __ldg(swrow + kt0) : 0.f;
+        float sc_next = (live && kt0 < kt1) ? __ldg(sxrow + kt0) * __ldg(swrow + kt0) : 0.f;
         for (int kt = kt0; kt < kt1; ++kt, ++i) {
           const int slot = i % kSlots;
           const float sc = sc_next;
-          if (kt + 1 < kt1) sc_next = in_m ? __ldg(sxrow + kt + 1) * __ldg(swrow + kt + 1) : 0.f;
+          if (kt + 1 < kt1) sc_next = live ? __ldg(sxrow + kt + 1) * __ldg(swrow + kt + 1) : 0.f;
           if (!warp_wait(&ctl->tfull[slot], (i / kSlots) & 1)) {
             if (lane == 0) {
               record_error(kErrWaitEpilogue);
@@ -1481,16 +1486,21 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             break;
           }
           tc_fence_after();
-          // this thread's columns: all its TMEM loads issued before one wait
-          {
-            uint32_t r[kHalf / 16][16];
+          // this thread's columns, at most 64 per TMEM wait (a 128-column half
+          // in two rounds: its running sums already hold 128 registers)
+          constexpr int kRound = kHalf < 64 ? kHalf : 64;
 #pragma unroll
-            for (int c = 0; c < kHalf / 16; ++c) tmem_ld16(taddr + slot * kTileN + half * kHalf + c * 16, r[c]);
+          for (int c0 = 0; c0 < kHalf; c0 += kRound) {
+            uint32_t r[kRound / 16][16];
+#pragma unroll
+            for (int c = 0; c < kRound / 16; ++c)
+              tmem_ld16(taddr + slot * kTileN + half * kHalf + c0 + c * 16, r[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kHalf / 16; ++c)
+            for (int c = 0; c < kRound / 16; ++c)
 #pragma unroll
-              for (int j = 0; j < 16; ++j) facc[c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[c * 16 + j]);
+              for (int j = 0; j < 16; ++j)
+                facc[c0 + c * 16 + j] = fmaf(__uint_as_float(r[c][j]), sc, facc[c0 + c * 16 + j]);
           }
           warp_release(&ctl->tempty[slot]);
         }
@@ -2228,7 +2238,8 @@ cudaError_t launch_standard(int fmt, int tile_n, const CUtensorMap& tx, const CU
                                            : launch_standard_t<kFmtFP8, 128>(tx, tw, a, stream);
   if (fmt == kFmtINT8) return tile_n == 256 ? launch_standard_t<kFmtINT8, 256>(tx, tw, a, stream)
                                             : launch_standard_t<kFmtINT8, 128>(tx, tw, a, stream);
-  if (fmt == kFmtBlock && tile_n == 128) return launch_standard_t<kFmtBlock, 128>(tx, tw, a, stream);
+  if (fmt == kFmtBlock) return tile_n == 256 ? launch_standard_t<kFmtBlock, 256>(tx, tw, a, stream)
+                                             : launch_standard_t<kFmtBlock, 128>(tx, tw, a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -147,7 +147,7 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 swap_grid(s, 3, 1)
                 if nkt >= 2 and s <= (nkt + 1) // 2:
                     swap_grid(s, 3, 2)
-    tiles = (128,) if fmt == BLOCK_FP8 else (128, 256)
+    tiles = (128, 256)
     # Standard: one K block per stage, and two (half the hand-offs and MMA commits) where the
     # tensor pipe is the bound
     kps_std = (1, 2) if (M > 32 and nkt >= 2) else (1,)

@@ -81,7 +81,7 @@ def test_default_plans():
     assert p["variant"] == qgd.VARIANT_STANDARD and p["split_k"] == 1 and p["tile_n"] == 256
     assert p["schedule"] == qgd.SCHEDULE_PERSISTENT
     p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 512, 6144, 4096)
-    assert p["tile_n"] == 128
+    assert p["tile_n"] == 256  # two 128-row weight blocks per tile
     # split never exceeds the number of 128-wide K tiles
     p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 1, 128, 256)
     assert p["split_k"] == 2

@@ -62,8 +62,6 @@ def _vid(v):
 @pytest.mark.parametrize("variant", VARIANTS, ids=_vid)
 def test_every_variant_tiny(fmt, variant):
     var, split, red, tile, sched = variant
-    if fmt == BLOCK_FP8 and tile == 256:
-        pytest.skip("Block_FP8 Standard tiles are 128 wide")
     case = Case(fmt, 4, 512, 1024, seed=1, outliers=True)
     yref, bound = _oracle(case)[:2]
     qgd.qgd_set_override(FMT_ID[fmt], var, split, red, 0, tile, sched)
@@ -99,6 +97,27 @@ def test_large_m_standard(fmt, M, N, K):
     yref, bound = _oracle(case)[:2]
     assert qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)["variant"] == qgd.VARIANT_STANDARD
     case.check_output(case.run(), yref, bound, f"{fmt} M={M}")
+
+
+BLOCK_TWO_BLOCK_PLANS = [(1, 0, GRID, 1), (2, 0, GRID, 1), (4, 1, GRID, 2), (2, 2, GRID, 1), (1, 0, PERSISTENT, 2),
+                         (1, 0, PERSISTENT, 1), (2, 0, PERSISTENT, 1)]
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 384, 1024), (257, 640, 2048), (64, 256, 512), (200, 1152, 1536)])
+@pytest.mark.parametrize("plan", BLOCK_TWO_BLOCK_PLANS,
+                         ids=[f"s{p[0]}-r{p[1]}-sch{p[2]}-k{p[3]}" for p in BLOCK_TWO_BLOCK_PLANS])
+def test_block_fp8_two_block_tiles(M, N, K, plan):
+    # 128 x 256 tiles: two 128-row weight blocks, each promoted with its own
+    # scale by one pair of epilogue warps; N an odd number of blocks leaves the
+    # last tile's second block past N
+    split, red, sched, kps = plan
+    case = Case(BLOCK_FP8, M, N, K, seed=M + N + K, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_STANDARD, split, red, 0, 256, sched, 0, kps)
+    p = qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, M, N, K)
+    assert p["tile_n"] == 256 and p["variant"] == qgd.VARIANT_STANDARD and p["k_slices"] == min(kps, K // 128)
+    case.check_output(case.run(), yref, bound, f"Block_FP8 256-wide M={M} N={N} K={K} plan={p}")
+    assert qgd.qgd_device_error() == 0
 
 
 @pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
