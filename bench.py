@@ -448,9 +448,25 @@ def tensor_probe(reps: int = 3, iters: int = 8192) -> dict:
             torch.cuda.synchronize()
             best = max(best, f / (t0.elapsed_time(t1) * 1e-3) / 1e12)
         out[name] = round(best, 1)
+    # the accumulator ring: a group the issuer waits on (a slot's previous
+    # group, before reusing the slot) costs about as long as an N = 256 group
+    ring = {}
+    for n, slots, wait in ((256, 2, 1), (128, 4, 1), (128, 4, 0)):
+        qgd.qgd_mma_ring_probe(n, slots, bool(wait), 64)
+        best = 0.0
+        for _ in range(reps):
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            f = qgd.qgd_mma_ring_probe(n, slots, bool(wait), iters)
+            t1.record()
+            torch.cuda.synchronize()
+            best = max(best, f / (t0.elapsed_time(t1) * 1e-3) / 1e12)
+        ring[f"n{n}_slots{slots}_{'wait' if wait else 'nowait'}_tflops"] = round(best, 1)
+    out["ring"] = ring
     assert qgd.qgd_device_error() == 0
     out["how"] = (f"qgd_mma_peak_probe: one CTA per SM, {iters} x 4 back-to-back tcgen05.mma (128x256x32) "
-                  f"from shared memory, best of {reps}")
+                  f"from shared memory, best of {reps}; ring: qgd_mma_ring_probe")
     return out
 
 

@@ -506,6 +506,16 @@ QGD_API qgd_status qgd_clear_device_error(void);
  * --------------------------------------------------------------------- */
 QGD_API qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream);
 
+/* Measurement aid: the tensor pipe with a ring of accumulators.  One CTA per
+ * SM issues `iters` groups of four e4m3 tcgen05.mma (128 x n x 32 each) into
+ * `slots` TMEM slots of n columns in turn, committing each group to its
+ * slot's mbarrier; with wait = 1 the issuing thread first waits for the
+ * slot's previous group to complete (the hand-off of a kernel whose
+ * accumulators form a ring), with wait = 0 it never waits.  n in {128, 256},
+ * slots in {1, 2, 4}, n * slots <= 512, 1 <= iters <= 200000, else
+ * QGD_ERR_INVALID.  *flops and timing as qgd_mma_peak_probe. */
+QGD_API qgd_status qgd_mma_ring_probe(int n, int slots, int wait, int iters, double* flops, void* stream);
+
 /* Test hook for the failure-detection path (the pages have no counterpart).
  * While on (on != 0), GEMMs launched from then on in the Swap-AB orientation
  * never signal the epilogue that an accumulator is complete -- a flag that

@@ -1138,6 +1138,18 @@ qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void* stream)
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "qgd_mma_peak_probe launch");
 }
 
+qgd_status qgd_mma_ring_probe(int n, int slots, int wait, int iters, double* flops, void* stream) {
+  if ((n != 128 && n != 256) || (slots != 1 && slots != 2 && slots != 4) || n * slots > 512 || (wait != 0 && wait != 1))
+    return fail(QGD_ERR_INVALID, "n=%d slots=%d wait=%d: n in {128, 256}, slots in {1, 2, 4}, n*slots <= 512",
+                n, slots, wait);
+  if (iters < 1 || iters > 200000) return fail(QGD_ERR_INVALID, "iters=%d must be in [1, 200000]", iters);
+  qgd_status st = check_device();
+  if (st != QGD_OK) return st;
+  if (flops) *flops = 2.0 * 128.0 * n * kTileK * static_cast<double>(iters) * g_num_sms;
+  cudaError_t e = launch_mma_ring_probe(n, slots, wait != 0, iters, g_num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QGD_OK : cuda_fail(e, "qgd_mma_ring_probe launch");
+}
+
 qgd_status qgd_test_withhold_accumulator(int on) {
   g_withhold_acc.store(on ? 1 : 0, std::memory_order_relaxed);
   return QGD_OK;

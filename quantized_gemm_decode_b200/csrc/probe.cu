@@ -73,7 +73,97 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters) {
   }
 }
 
+// Ring probe: groups of four K=32 e4m3 MMAs (128 x N x 128 per group) into
+// kSlots TMEM slots in turn, each group committed to its slot's barrier.
+// kWait: before reusing a slot, the issuing thread waits for that slot's
+// previous group to complete (the hand-off a kernel with a ring of
+// accumulators makes); otherwise it never waits.
+template <uint32_t kN, uint32_t kSlots, bool kWait>
+__global__ void __launch_bounds__(128, 1) mma_ring_kernel(int iters) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = probe_align1024(smem_raw);
+  uint8_t* a = base;
+  uint8_t* b = base + kProbeABytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(b + kN * kTileK);  // kSlots slot barriers, then `done`
+  uint64_t* done = bar + kSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  for (uint32_t i = threadIdx.x; i < (kProbeABytes + kN * kTileK) / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(base)[i] = make_uint4(0u, 0u, 0u, 0u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kN * kSlots);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    constexpr uint32_t idesc = idesc_mma(1, 0, 128, kN);
+    const uint64_t ad = sdesc_kmajor_sw128(smem_u32(a));
+    const uint64_t bd = sdesc_kmajor_sw128(smem_u32(b));
+    for (int it = 0; it < iters; ++it) {
+      const uint32_t s = static_cast<uint32_t>(it) % kSlots;
+      if (kWait && it >= static_cast<int>(kSlots) &&
+          !mbar_wait(&bar[s], ((static_cast<uint32_t>(it) / kSlots) - 1) & 1)) {
+        atomicCAS(&g_probe_error, 0u, static_cast<unsigned int>(kErrWaitMma));
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_issue<false>(tmem + s * kN, ad + static_cast<uint64_t>((kk * 32) >> 4),
+                         bd + static_cast<uint64_t>((kk * 32) >> 4), idesc, kk != 0);
+      mma_commit(&bar[s]);
+    }
+    mma_commit(done);
+    if (!mbar_wait(done, 0)) {
+      atomicCAS(&g_probe_error, 0u, static_cast<unsigned int>(kErrWaitDrain));
+      if (!mbar_wait(done, 0)) atomicCAS(&g_probe_error, 0u, static_cast<unsigned int>(kErrWaitDrain));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kN * kSlots);
+  }
+}
+
+template <uint32_t kN, uint32_t kSlots, bool kWait>
+cudaError_t launch_ring(int iters, int ctas, cudaStream_t stream) {
+  // operands, then (kSlots + 1) barriers and the TMEM address (<= 44 bytes), plus alignment slack
+  static_assert((kSlots + 1) * 8 + 4 <= 64, "barrier area");
+  const size_t smem = kProbeABytes + kN * kTileK + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(mma_ring_kernel<kN, kSlots, kWait>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  mma_ring_kernel<kN, kSlots, kWait><<<ctas, 128, smem, stream>>>(iters);
+  return cudaGetLastError();
+}
+
+template <bool kWait>
+cudaError_t launch_ring_w(int n, int slots, int iters, int ctas, cudaStream_t stream) {
+  if (n == 128 && slots == 1) return launch_ring<128, 1, kWait>(iters, ctas, stream);
+  if (n == 128 && slots == 2) return launch_ring<128, 2, kWait>(iters, ctas, stream);
+  if (n == 128 && slots == 4) return launch_ring<128, 4, kWait>(iters, ctas, stream);
+  if (n == 256 && slots == 1) return launch_ring<256, 1, kWait>(iters, ctas, stream);
+  if (n == 256 && slots == 2) return launch_ring<256, 2, kWait>(iters, ctas, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
+
+cudaError_t launch_mma_ring_probe(int n, int slots, bool wait, int iters, int ctas, cudaStream_t stream) {
+  return wait ? launch_ring_w<true>(n, slots, iters, ctas, stream)
+              : launch_ring_w<false>(n, slots, iters, ctas, stream);
+}
 
 size_t mma_probe_smem_bytes() { return kProbeABytes + kProbeBBytes + 64 + 1024; }
 

@@ -118,6 +118,7 @@ int pair_max_stages(int kps);
 // Tensor-core peak probe (probe.cu).
 cudaError_t launch_mma_probe(int qtype, int iters, int ctas, cudaStream_t stream);
 double mma_probe_flops(int iters, int ctas);
+cudaError_t launch_mma_ring_probe(int n, int slots, bool wait, int iters, int ctas, cudaStream_t stream);
 cudaError_t read_probe_error(unsigned int* code);
 cudaError_t clear_probe_error();
 

@@ -250,6 +250,8 @@ def test_mma_peak_probe_rejects_bad_arguments():
     assert L.qgd_mma_peak_probe(2, 16, ctypes.byref(flops), None) == -1  # qtype
     assert L.qgd_mma_peak_probe(qgd.QTYPE_E4M3, 0, ctypes.byref(flops), None) == -1
     assert L.qgd_mma_peak_probe(qgd.QTYPE_INT8, 200001, ctypes.byref(flops), None) == -1
+    for n, slots, wait, iters in ((64, 1, 1, 16), (256, 4, 1, 16), (128, 3, 0, 16), (128, 1, 2, 16), (128, 1, 1, 0)):
+        assert L.qgd_mma_ring_probe(n, slots, wait, iters, ctypes.byref(flops), None) == -1
 
 
 def test_k_slices_plan_field():

@@ -24,3 +24,20 @@ def test_probe_rate_is_plausible(qtype):
     assert qgd.qgd_device_error() == 0
     tflops = flops / (e0.elapsed_time(e1) * 1e-3) / 1e12
     assert 1000.0 < tflops < 6000.0, tflops
+
+
+def test_ring_probe_runs_and_waited_wide_groups_keep_the_rate():
+    qgd.qgd_clear_device_error()
+    rates = {}
+    for n, slots, wait in ((256, 2, True), (128, 4, True), (128, 4, False), (128, 1, True), (256, 1, False)):
+        qgd.qgd_mma_ring_probe(n, slots, wait, 64)  # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        flops = qgd.qgd_mma_ring_probe(n, slots, wait, 4096)
+        e1.record()
+        torch.cuda.synchronize()
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert flops == 2 * 128 * n * 128 * 4096 * sms
+        rates[(n, slots, wait)] = flops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    assert qgd.qgd_device_error() == 0
+    assert all(500.0 < r < 6000.0 for r in rates.values()), rates
