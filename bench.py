@@ -979,6 +979,13 @@ def render_report(d: dict) -> str:
         for r in d["per_call"]:
             out.append(f"| {r['M']} | {r['N']} x {r['K']} | {r['us']} | {r['p90_us']} | {r['gbs']} | {r['frac']} | "
                        f"{r['layer_us']} | {r['plan']} |")
+    if "tensor_probe" in d:
+        tp = d["tensor_probe"]
+        ring = tp.get("ring", {})
+        out.append(f"\nTensor probe (tcgen05 from shared memory, one CTA per SM): {tp.get('e4m3_tflops')} TFLOP/s e4m3, "
+                   f"{tp.get('int8_tops')} TOPS int8" +
+                   ("; accumulator ring: " + ", ".join(f"{k.replace('_tflops', '')} {v}" for k, v in ring.items())
+                    if ring else "") + ".")
     if "large_m" in d:
         out.append("\nLarger M (one GEMM per call; frac against 2 x bf16, frac_probe against the tcgen05 probe):\n")
         out.append("| format | M | mean frac | mean frac_probe | best TFLOP/s |\n|---|---:|---:|---:|---:|")
