@@ -1210,44 +1210,89 @@ __global__ void __launch_bounds__(kSwapTileN) swapab_reduce_kernel(const GemmArg
     if (m < M) store_final<kFmt>(sum[m], m, n, a);
 }
 
-// Last CTA of a Standard tile: add the split partials (or read the atomic
-// sum) for this thread's token row, 16 columns at a time, in split order.
+// Split-K fixup by the last-arriving CTA: this thread's row m, columns
+// [n0, n0 + kCols), 32 at a time, partials added in split order s = 0, 1, ...
+// (or the atomic accumulator read).  Every load of a chunk -- its partials and
+// its channel scales -- is issued before any of its stores, and the stores
+// are vectorised, so a chunk costs one L2 round trip per split rather than
+// one per 16 columns plus one per element's scales.
 template <int kFmt, int kCols>
 __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0, bool in_m) {
   if (!in_m) return;
+  constexpr bool kScaled = !(kFmt == kFmtBlock || kFmt == kFmtMX);
   const int M = a.M, N = a.N;
-  for (int nc = n0; nc < n0 + kCols && nc < N; nc += 16) {
-    const size_t idx = static_cast<size_t>(m) * N + nc;
-    uint32_t v[16];
-    if (a.reduce == kAtomic) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.accum) + idx);
+  const float sxm = (kScaled && !a.raw) ? __ldg(a.sx + m) : 1.f;
+  for (int nc0 = n0; nc0 < n0 + kCols && nc0 < N; nc0 += 32) {
+    const int nq = (N - nc0 < 32 ? N - nc0 : 32) / 4;  // 16-byte groups in this chunk: 4 or 8 (N % 16 == 0)
+    const size_t idx = static_cast<size_t>(m) * N + nc0;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        static_cast<const uint32_t*>(a.reduce == kAtomic ? a.accum : a.partial) + idx);
+    uint4 v[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 t = __ldcg(src + q);
-        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+    for (int q = 0; q < 8; ++q) v[q] = q < nq ? __ldcg(src + q) : make_uint4(0u, 0u, 0u, 0u);
+    float sw32[32];
+    if (kScaled && !a.raw) {
+      const float4* swv = reinterpret_cast<const float4*>(a.sw + nc0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 t4 = q < nq ? __ldg(swv + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sw32[4 * q] = t4.x;
+        sw32[4 * q + 1] = t4.y;
+        sw32[4 * q + 2] = t4.z;
+        sw32[4 * q + 3] = t4.w;
       }
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.partial) + idx);
+    }
+    if (a.reduce != kAtomic) {
+      for (int sp = 1; sp < a.splits; ++sp) {
+        const uint4* ps = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.partial) +
+                                                         static_cast<size_t>(sp) * M * N + idx);
+        uint4 t[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 t = __ldcg(src + q);
-        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
-      }
-      for (int s = 1; s < a.splits; ++s) {
-        const uint4* sp = reinterpret_cast<const uint4*>(static_cast<const uint32_t*>(a.partial) +
-                                                         static_cast<size_t>(s) * M * N + idx);
+        for (int q = 0; q < 8; ++q) t[q] = q < nq ? __ldcg(ps + q) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 t = __ldcg(sp + q);
-          v[4 * q] = add_acc<kFmt>(v[4 * q], t.x);
-          v[4 * q + 1] = add_acc<kFmt>(v[4 * q + 1], t.y);
-          v[4 * q + 2] = add_acc<kFmt>(v[4 * q + 2], t.z);
-          v[4 * q + 3] = add_acc<kFmt>(v[4 * q + 3], t.w);
+        for (int q = 0; q < 8; ++q) {
+          v[q].x = add_acc<kFmt>(v[q].x, t[q].x);
+          v[q].y = add_acc<kFmt>(v[q].y, t[q].y);
+          v[q].z = add_acc<kFmt>(v[q].z, t[q].z);
+          v[q].w = add_acc<kFmt>(v[q].w, t[q].w);
         }
       }
     }
+    if (a.raw) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) store_final<kFmt>(v[j], m, nc + j, a);
+      for (int q = 0; q < 8; ++q)
+        if (q < nq) dst[q] = v[q];
+      continue;
+    }
+    uint32_t w[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      w[4 * q] = v[q].x;
+      w[4 * q + 1] = v[q].y;
+      w[4 * q + 2] = v[q].z;
+      w[4 * q + 3] = v[q].w;
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float f0, f1;
+      if constexpr (kFmt == kFmtINT8) {
+        f0 = (static_cast<float>(static_cast<int32_t>(w[2 * j])) * sxm) * sw32[2 * j];
+        f1 = (static_cast<float>(static_cast<int32_t>(w[2 * j + 1])) * sxm) * sw32[2 * j + 1];
+      } else if constexpr (kScaled) {
+        f0 = (__uint_as_float(w[2 * j]) * sxm) * sw32[2 * j];
+        f1 = (__uint_as_float(w[2 * j + 1]) * sxm) * sw32[2 * j + 1];
+      } else {
+        f0 = __uint_as_float(w[2 * j]);
+        f1 = __uint_as_float(w[2 * j + 1]);
+      }
+      pk[j] = static_cast<uint32_t>(bf16_bits(f0)) | (static_cast<uint32_t>(bf16_bits(f1)) << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (2 * q < nq) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
   }
 }
 
