@@ -292,9 +292,11 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
   // the two-pass reduction kernel covers at most 32 tokens
   if (p.variant == kSwapAB && M > kDecodeMaxM && p.reduce == kTwoPass) p.reduce = kLastCta;
   // cluster Split-K: the S splits of a tile form one thread-block cluster
-  // (Swap-AB, grid schedule, 2 <= S <= 8)
-  if (p.reduce == kCluster &&
-      (p.variant != kSwapAB || p.schedule != kGrid || p.split_k < 2 || p.split_k > kMaxClusterSplit))
+  // (Swap-AB, or the one-CTA Standard kernel for FP8_Dynamic / W8A8_INT8;
+  // grid schedule, 2 <= S <= 8)
+  const bool std_cluster_ok = p.variant == kStandard && (fmt == kFmtFP8 || fmt == kFmtINT8);
+  if (p.reduce == kCluster && ((p.variant != kSwapAB && !std_cluster_ok) || p.schedule != kGrid || p.split_k < 2 ||
+                               p.split_k > kMaxClusterSplit))
     p.reduce = kLastCta;
   if (p.reduce != kCluster) p.split_k = floor_pow2(p.split_k);
   if (p.reduce != kTwoPass) {
@@ -315,6 +317,16 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
                                                   : standard_max_stages(p.tile_n, p.k_slices);
   if (p.stages <= 0 || p.stages > max_st) p.stages = max_st;
   if (p.stages < 2) p.stages = 2;
+  // the Standard cluster reduction receives the other splits' rows in the
+  // ring: (S - 1) ceil(128 / S) rows of tile_n fp32 values must fit there
+  if (p.variant == kStandard && p.reduce == kCluster) {
+    const size_t recv = static_cast<size_t>(p.split_k - 1) * ((kStdTileM + p.split_k - 1) / p.split_k) * p.tile_n * 4;
+    const size_t ring = static_cast<size_t>(p.stages) * p.k_slices * (kStdTileM + p.tile_n) * kTileK;
+    if (recv > ring) {
+      p.reduce = kLastCta;
+      p.split_k = floor_pow2(p.split_k);
+    }
+  }
   if (fmt == kFmtMX || fmt == kFmtNV)
     while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices, fmt) > kMxMaxCols) --p.stages;
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
@@ -418,7 +430,7 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
       e.persistent = true;
       e.ctas = static_cast<int>(items < cap ? items : cap);
     }
-    if (p.split_k > 1)
+    if (p.split_k > 1 && p.reduce != kCluster)  // the cluster reduction needs no workspace
       e.data_bytes = align256(static_cast<size_t>(M) * N * 4 * (p.reduce == kAtomic ? 1 : p.split_k));
   }
   if (e.data_bytes) {

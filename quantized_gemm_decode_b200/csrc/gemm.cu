@@ -1296,6 +1296,143 @@ __device__ __forceinline__ void std_reduce_tile(const GemmArgs& a, int m, int n0
   }
 }
 
+// Split-K of the Standard kernel inside a thread-block cluster (grid schedule:
+// the S = a.splits CTAs of a tile are one cluster, CTA rank = split).  Row r of
+// the tile (TMEM lane r) belongs to CTA floor(r S / 128); after every CTA's
+// MMAs are done (first cluster barrier: each epilogue has waited for its
+// accumulator, so every ring is idle), each CTA writes its partial rows that
+// others own into the owner's ring through distributed shared memory, and
+// after the second barrier each owner adds the S partials of its rows in
+// split order -- its own straight from tensor memory -- and stores them.
+// Called by every thread of the CTA (the barriers need all of them).  The
+// host checks that (S - 1) ceil(128 / S) kTileN * 4 bytes fit in the ring.
+template <int kFmt, int kTileN>
+__device__ __forceinline__ void std_cluster_reduce(const GemmArgs& a, SmemCtl* ctl, uint8_t* ring, uint32_t tmem,
+                                                   int warp, int lane) {
+  const int S = a.splits;
+  const int self = static_cast<int>(cluster_ctarank());
+  const int tile = static_cast<int>(blockIdx.x) / S;
+  const int m_tiles = (a.M + kStdTileM - 1) / kStdTileM;
+  const int m_tile = tile % m_tiles, n_tile = tile / m_tiles;
+  const int Rm = (kStdTileM + S - 1) / S;  // most rows any owner holds
+  tc_fence_before();
+  cluster_sync_all();
+  // an aborted CTA may still have copies landing in its ring: no exchange then
+  bool abort = false;
+  for (int j = 0; j < S; ++j)
+    abort |= ld_cluster_u32(mapa_shared(smem_u32(&ctl->abort_flag), static_cast<uint32_t>(j))) != 0u;
+  const int q = warp & 3, r = q * 32 + lane;  // this thread's tile row (TMEM lane), epilogue warps only
+  const int owner = (r * S) / kStdTileM;     // (an owner's band may start inside a warp: the TMEM
+  const int lr = r - (owner * kStdTileM + S - 1) / S;  // loads stay warp-wide, the rest per lane)
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);  // accumulator buffer 0
+  if (warp >= 2 && !abort) {
+    tc_fence_after();
+    const int jslot = self < owner ? self : self - 1;  // this CTA's slot in the owner's buffer
+    const uint32_t dst = mapa_shared(smem_u32(ring), static_cast<uint32_t>(owner)) +
+                         static_cast<uint32_t>((jslot * Rm + lr) * kTileN * 4);
+#pragma unroll 1
+    for (int c4 = 0; c4 < kTileN / 64; ++c4) {
+      uint32_t vv[4][16];
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 4; ++h) tmem_ld16(taddr + c4 * 64 + h * 16, vv[h]);
+      tmem_wait_ld();
+      if (owner != self) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int ch = (16 * c4 + 4 * h + g) ^ (lr & 7);  // 16-byte chunk, swizzled against bank conflicts
+            st_cluster_v4(dst + static_cast<uint32_t>(ch * 16), vv[h][4 * g], vv[h][4 * g + 1], vv[h][4 * g + 2],
+                          vv[h][4 * g + 3]);
+          }
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp < 2) return;
+  if (abort) {
+    if (lane == 0) record_error(kErrWaitEpilogue);
+    return;
+  }
+  tc_fence_after();
+  const int M = a.M, N = a.N;
+  const int m = m_tile * kStdTileM + r;
+  const int n0 = n_tile * kTileN;
+  const bool mine = owner == self && m < M;
+  const float sxm = (mine && !a.raw) ? __ldg(a.sx + m) : 0.f;
+#pragma unroll 1
+  for (int c4 = 0; c4 < kTileN / 64; ++c4) {
+    uint32_t own4[4][16];
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 4; ++h) tmem_ld16(taddr + c4 * 64 + h * 16, own4[h]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int c = 4 * c4 + h;
+      const int nc = n0 + c * 16;
+      const uint32_t (&own)[16] = own4[h];
+      if (!mine || nc >= N) continue;
+      uint32_t v[16];
+      for (int j = 0; j < S; ++j) {
+        uint32_t p[16];
+        if (j == self) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) p[e] = own[e];
+        } else {
+          const int js = j < self ? j : j - 1;
+          const uint8_t* src = ring + static_cast<size_t>((js * Rm + lr) * kTileN * 4);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint4 t = *reinterpret_cast<const uint4*>(src + (((4 * c + g) ^ (lr & 7)) * 16));
+            p[4 * g] = t.x;
+            p[4 * g + 1] = t.y;
+            p[4 * g + 2] = t.z;
+            p[4 * g + 3] = t.w;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = j == 0 ? p[e] : add_acc<kFmt>(v[e], p[e]);  // split order
+      }
+      const size_t idx = static_cast<size_t>(m) * N + nc;
+      if (a.raw) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) dst[g] = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        continue;
+      }
+      const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+      float sw16[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 t = __ldg(swv + g);
+        sw16[4 * g] = t.x;
+        sw16[4 * g + 1] = t.y;
+        sw16[4 * g + 2] = t.z;
+        sw16[4 * g + 3] = t.w;
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float f0, f1;
+        if constexpr (kFmt == kFmtINT8) {
+          f0 = (static_cast<float>(static_cast<int32_t>(v[2 * j])) * sxm) * sw16[2 * j];
+          f1 = (static_cast<float>(static_cast<int32_t>(v[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+        } else {
+          f0 = (__uint_as_float(v[2 * j]) * sxm) * sw16[2 * j];
+          f1 = (__uint_as_float(v[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+        }
+        pk[j] = static_cast<uint32_t>(bf16_bits(f0)) | (static_cast<uint32_t>(bf16_bits(f1)) << 16);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  }
+}
+
 // ===========================================================================
 // Standard kernel (larger M): D[m, n] over 128 x kTileN output tiles.
 //
@@ -1608,61 +1745,68 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
         }
         if (ok) tc_fence_after();
         if (!epi_agree_ok(ctl)) break;
+        if (a.reduce == kCluster) continue;  // the cluster reduction below reads the accumulator
         const float sxm = (in_m && !a.raw) ? __ldg(a.sx + m) : 0.f;
         const uint32_t tbuf = taddr + buf * kTileN;
+        // 64 columns per TMEM wait: four loads in flight instead of one
 #pragma unroll 1
-        for (int c = 0; c < kTileN / 16; ++c) {
-          const int nc = n0 + c * 16;
-          uint32_t r[16];
+        for (int c4 = 0; c4 < kTileN / 64; ++c4) {
+          uint32_t rr[4][16];
           __syncwarp();
-          tmem_ld16(tbuf + c * 16, r);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) tmem_ld16(tbuf + c4 * 64 + g * 16, rr[g]);
           tmem_wait_ld();
-          if (c == kTileN / 16 - 1) {
+          if (c4 == kTileN / 64 - 1) {
             // the whole accumulator is in registers: hand the buffer back
             warp_release(&ctl->tempty[buf]);
           }
-          if (!in_m || nc >= N) continue;
-          const size_t idx = static_cast<size_t>(m) * N + nc;
-          if (S > 1) {
-            if (a.reduce == kAtomic) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, r[j]);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t (&r)[16] = rr[g];
+            const int nc = n0 + (c4 * 4 + g) * 16;
+            if (!in_m || nc >= N) continue;
+            const size_t idx = static_cast<size_t>(m) * N + nc;
+            if (S > 1) {
+              if (a.reduce == kAtomic) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) atomic_acc<kFmt>(a.accum, idx + j, r[j]);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.partial) + static_cast<size_t>(split) * M * N + idx);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+              }
+            } else if (a.raw) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
 #pragma unroll
               for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            }
-          } else if (a.raw) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + idx);
+            } else {
+              const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
+              float sw16[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-          } else {
-            const float4* swv = reinterpret_cast<const float4*>(a.sw + nc);
-            float sw16[16];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const float4 t = __ldg(swv + v);
-              sw16[4 * v] = t.x;
-              sw16[4 * v + 1] = t.y;
-              sw16[4 * v + 2] = t.z;
-              sw16[4 * v + 3] = t.w;
-            }
-            uint32_t pk[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float v0, v1;
-              if constexpr (kInt) {
-                v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
-                v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
-              } else {
-                v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
-                v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+              for (int v = 0; v < 4; ++v) {
+                const float4 t = __ldg(swv + v);
+                sw16[4 * v] = t.x;
+                sw16[4 * v + 1] = t.y;
+                sw16[4 * v + 2] = t.z;
+                sw16[4 * v + 3] = t.w;
               }
-              pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+              uint32_t pk[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float v0, v1;
+                if constexpr (kInt) {
+                  v0 = (static_cast<float>(static_cast<int32_t>(r[2 * j])) * sxm) * sw16[2 * j];
+                  v1 = (static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * sxm) * sw16[2 * j + 1];
+                } else {
+                  v0 = (__uint_as_float(r[2 * j]) * sxm) * sw16[2 * j];
+                  v1 = (__uint_as_float(r[2 * j + 1]) * sxm) * sw16[2 * j + 1];
+                }
+                pk[j] = static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
-            uint4* dst = reinterpret_cast<uint4*>(a.y + idx);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
         if (S > 1 && a.reduce != kTwoPass && epi_arrive_last(ctl, a, tile, S)) {
@@ -1673,6 +1817,9 @@ __global__ void __launch_bounds__(std_threads<kFmt>(), 1)
     }
   }
 
+  if constexpr (!kBlock) {
+    if (a.reduce == kCluster) std_cluster_reduce<kFmt, kTileN>(a, ctl, x_ring, tmem, warp, lane);
+  }
   teardown(ctl, warp, lane, issued, stages, tmem, kCols);
 }
 
@@ -2212,8 +2359,10 @@ static cudaError_t launch_standard_k(const CUtensorMap& tx, const CUtensorMap& t
   const long long items = static_cast<long long>((a.N + kTileN - 1) / kTileN) *
                           ((a.M + kStdTileM - 1) / kStdTileM) * a.splits;
   const dim3 grid(static_cast<unsigned>(a.persistent && a.ctas < items ? a.ctas : items));
-  return launch_ex(standard_kernel<kFmt, kTileN, kKps>, grid, dim3(std_threads<kFmt>()),
-                   standard_smem_bytes(kTileN, a.stages, kKps), stream, a.pdl != 0, tx, tw, a);
+  // cluster Split-K (grid schedule): the a.splits CTAs of a tile, consecutive along x, are one cluster
+  return launch_ex_cluster_xy(standard_kernel<kFmt, kTileN, kKps>, grid, dim3(std_threads<kFmt>()),
+                              standard_smem_bytes(kTileN, a.stages, kKps), stream, a.pdl != 0,
+                              a.reduce == kCluster ? a.splits : 1, 1, tx, tw, a);
 }
 
 template <int kFmt, int kTileN>

@@ -163,6 +163,11 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 if s <= nku:
                     for r in ((0,) if s == 1 else (0, 1)):
                         out.append((0, s, r, t, 1, 0, kps, 0))  # Standard, persistent
+            # the splits of a tile as one thread-block cluster (DSMEM reduction), per-token formats
+            if fmt in (FP8_DYNAMIC, W8A8_INT8) and M > 32:
+                for s in range(2, 9):
+                    if s <= nku:
+                        out.append((0, s, 3, t, 0, 0, kps, 0))
     # Standard pair tiles (256 x 256 on two SMs): the per-token formats past 128 tokens
     if fmt in (FP8_DYNAMIC, W8A8_INT8) and M > 128:
         for kps in kps_std:

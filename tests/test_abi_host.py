@@ -353,12 +353,30 @@ def test_cluster_reduction_plan_rules():
         assert p["reduce"] == C and p["split_k"] == split
         # the splits exchange partials through shared memory: no workspace
         assert qgd.qgd_workspace_size(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096) == 0
-    # beyond a portable cluster, on the persistent schedule, or for Standard
-    # tiles the reduction falls back to the last-arriving CTA
+    # beyond a portable cluster, on the persistent schedule, or with one split
+    # the reduction falls back to the last-arriving CTA
     for args in ((qgd.VARIANT_SWAP_AB, 16, C, 0, 0, G), (qgd.VARIANT_SWAP_AB, -1, C, 0, 0, P),
-                 (qgd.VARIANT_STANDARD, 4, C, 0, 128, G), (qgd.VARIANT_SWAP_AB, 1, C, 0, 0, G)):
+                 (qgd.VARIANT_STANDARD, 4, C, 0, 128, P), (qgd.VARIANT_SWAP_AB, 1, C, 0, 0, G)):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, *args)
         assert qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 4, 4096, 4096)["reduce"] == qgd.REDUCE_LAST_CTA
+    # Standard tiles of the per-token formats: the splits' rows meet in the owners' rings
+    for fmt in (qgd.FMT_FP8_DYNAMIC, qgd.FMT_W8A8_INT8):
+        for split in (2, 3, 5, 8):
+            qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD, split, C, 0, 256, G, 0, 2)
+            p = qgd.qgd_get_plan(fmt, 512, 4096, 4096)
+            assert (p["variant"], p["reduce"], p["split_k"]) == (qgd.VARIANT_STANDARD, C, split)
+            assert qgd.qgd_workspace_size(fmt, 512, 4096, 4096) == 0
+        qgd.qgd_set_override(fmt)
+    # Block_FP8 promotes into registers: no cluster reduction in its Standard kernel
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8, qgd.VARIANT_STANDARD, 4, C, 0, 256, G, 0, 2)
+    assert qgd.qgd_get_plan(qgd.FMT_BLOCK_FP8, 512, 4096, 4096)["reduce"] == qgd.REDUCE_LAST_CTA
+    qgd.qgd_set_override(qgd.FMT_BLOCK_FP8)
+    # the received rows must fit the ring: two one-block stages of 128 x 256 hold 96 KB,
+    # less than the 7 x 16 rows x 1 KB that eight splits send
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, qgd.VARIANT_STANDARD, 8, C, 2, 256, G, 0, 1)
+    p = qgd.qgd_get_plan(qgd.FMT_FP8_DYNAMIC, 512, 4096, 4096)
+    assert (p["reduce"], p["split_k"]) == (qgd.REDUCE_LAST_CTA, 8)
+    qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC)
     with pytest.raises(qgd.QGDError):
         qgd.qgd_set_override(qgd.FMT_FP8_DYNAMIC, 1, 4, 4, 0, 0, G)
 

@@ -489,3 +489,39 @@ def test_swap_ab_wide_token_counts(fmt, plan, M, N, K):
         torch.cuda.synchronize()
         np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
     assert qgd.qgd_device_error() == 0
+
+
+STD_CLUSTER_PLANS = [(2, 256, 2), (3, 256, 1), (4, 128, 2), (5, 256, 1), (8, 128, 1), (8, 256, 1), (2, 128, 1)]
+
+
+@pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
+@pytest.mark.parametrize("plan", STD_CLUSTER_PLANS, ids=[f"s{p[0]}-t{p[1]}-k{p[2]}" for p in STD_CLUSTER_PLANS])
+@pytest.mark.parametrize("M,N,K", [(130, 528, 2048), (257, 256, 4096), (40, 1040, 1536), (512, 768, 1024)])
+def test_standard_cluster_split(fmt, plan, M, N, K):
+    # Standard tiles whose K splits form one thread-block cluster: every row's
+    # owner adds the splits' partials in split order, so the output equals the
+    # last-arriving-CTA reduction's bit for bit
+    split, tile, kps = plan
+    case = Case(fmt, M, N, K, seed=M + 2 * N + K + split, outliers=True)
+    yref, bound = _oracle(case)[:2]
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD, split, qgd.REDUCE_CLUSTER, 0, tile, GRID, 0, kps)
+    p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
+    if p["reduce"] != qgd.REDUCE_CLUSTER:
+        pytest.skip(f"plan legalised to {p}")
+    assert p["variant"] == qgd.VARIANT_STANDARD and p["tile_n"] == tile
+    y1 = case.run()
+    case.check_output(y1, yref, bound, f"{fmt} Standard cluster M={M} N={N} K={K} plan={p}")
+    assert qgd.qgd_device_error() == 0
+    if p["split_k"] & (p["split_k"] - 1) == 0:  # the other reductions take powers of two only
+        qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD, p["split_k"], qgd.REDUCE_LAST_CTA, p["stages"], tile,
+                             GRID, 0, p["k_slices"])
+        y2 = case.run()
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    if fmt == W8A8_INT8:
+        qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD, split, qgd.REDUCE_CLUSTER, 0, tile, GRID, 0, kps)
+        _, _, acc = _oracle(case, want_acc=True)
+        got = qgd.qgd_w8a8_int8_acc32(case.xq, case.wq)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got.cpu().numpy().astype(np.int64), acc)
+    assert qgd.qgd_device_error() == 0
