@@ -96,10 +96,11 @@ typedef enum {
   QGD_REDUCE_TWO_PASS = 1, /* split partials to workspace; a second kernel adds them in split order
                               (Swap-AB: at most 32 tokens, else the last CTA adds them) */
   QGD_REDUCE_ATOMIC = 2,   /* split partials added atomically into a zeroed workspace (fp32 order varies) */
-  QGD_REDUCE_CLUSTER = 3   /* Swap-AB grid schedule, 2 <= split_k <= 8 (not only powers of two): the
-                              splits of a tile form one
-                              thread-block cluster and add their partials in split order through
-                              distributed shared memory (no workspace) */
+  QGD_REDUCE_CLUSTER = 3   /* grid schedule, 2 <= split_k <= 8 (not only powers of two): the splits of
+                              a tile form one thread-block cluster and add their partials in split
+                              order through distributed shared memory (no workspace).  Swap-AB, and
+                              the one-CTA Standard kernel for FP8_Dynamic / W8A8_INT8 when the other
+                              splits' rows fit the ring (else the last CTA adds them) */
 } qgd_reduce;
 
 typedef enum {
