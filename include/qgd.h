@@ -517,6 +517,14 @@ QGD_API qgd_status qgd_mma_peak_probe(int qtype, int iters, double* flops, void*
  * QGD_ERR_INVALID.  *flops and timing as qgd_mma_peak_probe. */
 QGD_API qgd_status qgd_mma_ring_probe(int n, int slots, int wait, int iters, double* flops, void* stream);
 
+/* Programmatic dependent launch (each kernel starts while the one before it
+ * on the stream finishes, and waits only where it reads that kernel's
+ * output): on = 1 (the default), 0 = plain stream order, -1 = as the
+ * environment variable QGD_PDL says (QGD_PDL=0 turns it off), read at the
+ * next launch.  The setting is read once and then cached, not looked up per
+ * launch.  Other values -> QGD_ERR_INVALID. */
+QGD_API qgd_status qgd_set_pdl(int on);
+
 /* Test hook for the failure-detection path (the pages have no counterpart).
  * While on (on != 0), GEMMs launched from then on in the Swap-AB orientation
  * never signal the epilogue that an accumulator is complete -- a flag that

@@ -33,7 +33,7 @@ __all__ = [
     "qlinear_fp8_dynamic_noalloc",
     "qgd_workspace_size", "qgd_load_dispatch_table", "qgd_clear_dispatch_table", "qgd_set_override",
     "qgd_get_plan", "qgd_m_bucket", "qgd_device_error", "qgd_clear_device_error", "qgd_version",
-    "qgd_mma_peak_probe", "qgd_mma_ring_probe", "qgd_test_withhold_accumulator",
+    "qgd_mma_peak_probe", "qgd_mma_ring_probe", "qgd_test_withhold_accumulator", "qgd_set_pdl",
     "qlinear_bf16", "qgd_layer_workspace_size", "qgd_get_layer_plan", "qgd_set_fused_override",
     "qgd_test_capture_fused",
     "MAX_TP_RANKS", "qlinear_tp_bf16", "qgd_tp_workspace_size", "qgd_tp_wait", "ipc_malloc", "ipc_open",
@@ -110,6 +110,7 @@ def lib() -> ctypes.CDLL:
             "qgd_mma_peak_probe": [I, I, ctypes.POINTER(ctypes.c_double), P],
             "qgd_mma_ring_probe": [I, I, I, I, ctypes.POINTER(ctypes.c_double), P],
             "qgd_test_withhold_accumulator": [I],
+            "qgd_set_pdl": [I],
             "qlinear_fp8_dynamic_bf16": [P, I, P, P, P, I, I, I, P, S, P],
             "qlinear_w8a8_int8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
             "qlinear_block_fp8_bf16": [P, I, P, P, P, I, I, I, P, S, P],
@@ -752,6 +753,11 @@ def qgd_mma_ring_probe(n: int = 256, slots: int = 2, wait: bool = True, iters: i
     _check(lib().qgd_mma_ring_probe(n, slots, 1 if wait else 0, iters, ctypes.byref(flops), _stream(stream)),
            "qgd_mma_ring_probe")
     return float(flops.value)
+
+
+def qgd_set_pdl(on: int = -1) -> None:
+    """Programmatic dependent launch on (1), off (0), or as QGD_PDL says (-1)."""
+    _check(lib().qgd_set_pdl(on), "qgd_set_pdl")
 
 
 def qgd_test_withhold_accumulator(on: bool) -> None:

@@ -440,11 +440,23 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   return e;
 }
 
-// Programmatic dependent launch is on unless QGD_PDL=0.
-bool pdl_enabled() {
-  const char* v = getenv("QGD_PDL");
-  return !(v && v[0] == '0');
+// Programmatic dependent launch: on unless QGD_PDL=0 (read once, at the first
+// launch) or qgd_set_pdl(0).  -1: not yet decided.
+std::atomic<int> g_pdl{-1};
+
+}  // namespace
+
+bool qgd::pdl_enabled() {
+  int v = g_pdl.load(std::memory_order_relaxed);
+  if (v < 0) {
+    const char* e = getenv("QGD_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+    g_pdl.store(v, std::memory_order_relaxed);
+  }
+  return v != 0;
 }
+
+namespace {
 
 std::atomic<int> g_call_seq{0};  // numbers GEMM calls for the developer timeline
 std::atomic<int> g_withhold_acc{0};  // qgd_test_withhold_accumulator
@@ -1160,6 +1172,12 @@ qgd_status qgd_mma_ring_probe(int n, int slots, int wait, int iters, double* flo
   if (flops) *flops = 2.0 * 128.0 * n * kTileK * static_cast<double>(iters) * g_num_sms;
   cudaError_t e = launch_mma_ring_probe(n, slots, wait != 0, iters, g_num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QGD_OK : cuda_fail(e, "qgd_mma_ring_probe launch");
+}
+
+qgd_status qgd_set_pdl(int on) {
+  if (on < -1 || on > 1) return fail(QGD_ERR_INVALID, "on=%d must be -1, 0 or 1", on);
+  g_pdl.store(on, std::memory_order_relaxed);  // -1: QGD_PDL decides again at the next launch
+  return QGD_OK;
 }
 
 qgd_status qgd_test_withhold_accumulator(int on) {

@@ -105,6 +105,9 @@ cudaError_t launch_splitk_reduce(int fmt, const GemmArgs& a, cudaStream_t stream
 // Tensor parallelism: wait (bounded) until flags[0..ranks) all reach the
 // epoch in flags[ranks] (this rank's call counter)
 cudaError_t launch_tp_wait(const unsigned* flags, int ranks, bool pdl, cudaStream_t stream);
+// Programmatic dependent launch for every kernel of the library: on unless
+// QGD_PDL=0 (read once) or qgd_set_pdl(0)
+bool pdl_enabled();
 cudaError_t launch_swapab_reduce(int fmt, int mpad, const GemmArgs& a, cudaStream_t stream);
 cudaError_t read_device_error(unsigned int* code);
 cudaError_t clear_device_error();

@@ -212,8 +212,7 @@ __global__ void __launch_bounds__(256) quant_block128_kernel(const uint16_t* __r
 // QGD_PDL=0): the kernel may start early and waits in griddepcontrol.wait.
 template <typename... Params, typename... Args>
 cudaError_t launch_q(void (*kernel)(Params...), dim3 grid, dim3 block, cudaStream_t stream, Args&&... args) {
-  const char* v = getenv("QGD_PDL");
-  const bool pdl = !(v && v[0] == '0');
+  const bool pdl = pdl_enabled();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

@@ -635,3 +635,11 @@ def test_column_parallel_call_rules():
     assert L.qgd_ipc_malloc(256, None, ctypes.create_string_buffer(64)) == -1
     assert L.qgd_ipc_open(None, ctypes.byref(p)) == -1
     assert L.qgd_ipc_close(None) == -1 and L.qgd_ipc_free(None) == -1
+
+
+def test_pdl_setting_is_validated_and_cached():
+    L = qgd.lib()
+    for bad in (-2, 2, 7):
+        assert L.qgd_set_pdl(bad) == -1
+    for ok in (0, 1, -1):
+        assert L.qgd_set_pdl(ok) == 0

@@ -27,6 +27,7 @@ def _no_override():
     yield
     for f in range(3):
         qgd.qgd_set_override(f)
+    qgd.qgd_set_pdl(-1)
 
 
 def _oracle(case: Case, want_acc=False):
@@ -251,10 +252,10 @@ def test_persistent_shallow_pipelines_one_or_two_ctas_per_sm(stages, occupancy):
 
 
 @pytest.mark.parametrize("pdl", ["0", "1"])
-def test_chained_layers_with_and_without_programmatic_launch(monkeypatch, pdl):
+def test_chained_layers_with_and_without_programmatic_launch(pdl):
     # quantize -> GEMM -> quantize(Y) -> GEMM on one stream: the second layer
     # reads the first layer's output, so any missing dependency shows
-    monkeypatch.setenv("QGD_PDL", pdl)
+    qgd.qgd_set_pdl(int(pdl))
     x = synth.activations(8, 2048, seed=31, outliers=True).cuda()
     w1 = synth.weights(1024, 2048, seed=32).cuda()
     w2 = synth.weights(512, 1024, seed=33).cuda()
