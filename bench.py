@@ -492,33 +492,53 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict |
     frac_spec: against the 4.5 PFLOP/s data-sheet figure."""
     import quantized_gemm_decode_b200 as qgd
 
-    wl = [w for w in workloads.LARGE if w.fmt == fmt][0]
-    fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2}[fmt]
+    wl = [w for w in workloads.LARGE + workloads.LARGE_BS if w.fmt == fmt][0]
+    fmt_id = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3, NVFP4: 4}[fmt]
     peak_tc = 2.0 * peaks_["bf16_tflops"]  # e4m3 / int8 dense rate = 2x bf16 (nominal ratio)
-    fn = {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
-          BLOCK_FP8: qgd.qlinear_block_fp8}[fmt]
+    if fmt == NVFP4:
+        peak_tc *= 2.0  # e2m1: twice the e4m3 rate (nominal ratio)
     rows = []
     for (N, K) in wl.shapes:
         w = synth.weights(N, K, wl.seed).to(device)
         if fmt == BLOCK_FP8:
-            wq, sw = qgd.quant_weight_block128(w)
+            wops = qgd.quant_weight_block128(w)
+        elif fmt == MXFP8:
+            wops = qgd.quant_mx(w)
+        elif fmt == NVFP4:
+            q_, s_, g_ = qgd.quant_nv(w)
+            wops = (q_, s_, g_)
         else:
-            wq, sw = qgd.quant_weight_per_channel(w, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
+            wops = qgd.quant_weight_per_channel(w, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
         del w
-        ncop = max(2, math.ceil(ROTATION_BYTES / (N * K)))
-        copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(ncop - 1)]
+        wbytes = workloads.algorithmic_bytes(fmt, 0, N, K)
+        ncop = max(2, math.ceil(ROTATION_BYTES / max(wbytes, 1)))
+        copies = [wops] + [tuple(t.clone() for t in wops) for _ in range(ncop - 1)]
         for M in wl.ms:
             x = synth.activations(M, K, wl.seed, outliers=wl.outliers).to(device)
             if fmt == BLOCK_FP8:
-                xq, sx = qgd.quant_act_group128(x)
+                xops = qgd.quant_act_group128(x)
+            elif fmt == MXFP8:
+                xops = qgd.quant_mx(x)
+            elif fmt == NVFP4:
+                xops = qgd.quant_nv(x)
             else:
-                xq, sx = qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
+                xops = qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             ws = qgd.Workspace(qgd.qgd_workspace_size(fmt_id, M, N, K), device)
 
+            def call(j):
+                wo = copies[j]
+                if fmt == NVFP4:
+                    qgd.qlinear_nvfp4(xops[0], xops[1], xops[2], wo[0], wo[1], wo[2], y=y, ws=ws)
+                elif fmt == MXFP8:
+                    qgd.qlinear_mxfp8(xops[0], xops[1], wo[0], wo[1], y=y, ws=ws)
+                else:
+                    {FP8_DYNAMIC: qgd.qlinear_fp8_dynamic, W8A8_INT8: qgd.qlinear_w8a8_int8,
+                     BLOCK_FP8: qgd.qlinear_block_fp8}[fmt](xops[0], xops[1], wo[0], wo[1], y=y, ws=ws)
+
             def body():
                 for j in range(ncop):
-                    fn(xq, sx, copies[j][0], copies[j][1], y=y, ws=ws)
+                    call(j)
 
             s_ = torch.cuda.Stream(device)
             s_.wait_stream(torch.cuda.current_stream(device))
@@ -545,11 +565,11 @@ def large_m_summary(fmt: str, device, peaks_: dict, reps: int = 5, probe: dict |
                             f"{'pers' + str(p['occupancy']) if p['schedule'] == 1 else 's' + str(p['split_k'])}"
                             f"/r{p['reduce']}/st{p['stages']}/k{p['k_slices']}")}
             if probe:
-                pk = probe["int8_tops"] if fmt == W8A8_INT8 else probe["e4m3_tflops"]
+                pk = probe["int8_tops"] if fmt == W8A8_INT8 else probe["e4m3_tflops"] * (2.0 if fmt == NVFP4 else 1.0)
                 row["frac_probe"] = round(max(b / (peaks_["hbm_gbs"] * 1e9), f / (pk * 1e12)) / (ms * 1e-3), 4)
             rows.append(row)
-            del x, xq, sx, y, ws
-        del copies, wq, sw
+            del x, xops, y, ws
+        del copies, wops
         torch.cuda.empty_cache()
     return rows
 
@@ -1182,7 +1202,8 @@ def main():
         out["formats"] = fmts
         probe = tensor_probe()
         out["tensor_probe"] = probe
-        out["large_m"] = {f: large_m_summary(f, device, pk, probe=probe) for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8)}
+        out["large_m"] = {f: large_m_summary(f, device, pk, probe=probe)
+                          for f in (FP8_DYNAMIC, W8A8_INT8, BLOCK_FP8, MXFP8, NVFP4)}
         out["splitk_modes"] = splitk_modes_table(device)
         out["chain"] = chain_table(device)
         out["tensor_parallel"] = tp_table(device)

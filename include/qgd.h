@@ -258,11 +258,13 @@ QGD_API size_t qgd_layer_workspace_size(int fmt, int M, int N, int K);
 QGD_API qgd_status quant_act_mx(const void* x_bf16, int M, int K, int ldx, void* xq, void* s_e8m0, void* stream);
 
 /* MXFP8 GEMM: y_bf16 [M,N] from xq [M,K], sx_e8m0 [M][K/32], wq [N,K],
- * sw_e8m0 [N][K/32].  Swap-AB kernel only: 0 <= M <= 64 (more ->
+ * sw_e8m0 [N][K/32].  Swap-AB kernel only: 0 <= M <= 128 (more ->
  * QGD_ERR_UNSUPPORTED); K % 128 == 0, N % 16 == 0; all pointers 16-byte
  * aligned.  The block scales sit in tensor memory beside the accumulators
- * (at most 256 columns per CTA, which caps the ring depth).  Workspace as qlinear_fp8_dynamic (same plans; no two-pass
- * reduction, whose requests take the last-arriving CTA). */
+ * (at most 256 columns per CTA up to 64 tokens, which caps the ring depth;
+ * at 65..128 tokens all 512, with a ring of at least four K slices so that
+ * the CTA has its SM to itself).  Workspace as qlinear_fp8_dynamic (same
+ * plans; no two-pass reduction, whose requests take the last-arriving CTA). */
 QGD_API qgd_status qlinear_mxfp8(const void* xq, const void* sx_e8m0, const void* wq, const void* sw_e8m0,
                                  void* y_bf16, int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
@@ -295,12 +297,13 @@ QGD_API qgd_status quant_nvfp4(const void* x_bf16, int rows, int K, int ldx, voi
                                void* stream);
 
 /* NVFP4 GEMM: y_bf16 [M,N] from xq [M][K/2], sx_e4m3 [M][K/16], gx [M], wq
- * [N][K/2], sw_e4m3 [N][K/16], gw [N].  Swap-AB kernel only: 0 <= M <= 64
+ * [N][K/2], sw_e4m3 [N][K/16], gw [N].  Swap-AB kernel only: 0 <= M <= 128
  * (more -> QGD_ERR_UNSUPPORTED); K % 256 == 0, N % 16 == 0; all pointers
  * 16-byte aligned.  The block scales sit in tensor memory beside the
- * accumulators, 32 columns per ring slot (at most 256 columns per CTA, which
- * caps the ring depth).  Workspace as qlinear_fp8_dynamic (same plans; no
- * two-pass reduction, whose requests take the last-arriving CTA). */
+ * accumulators, 32 columns per ring slot (at most 256 columns per CTA up to
+ * 64 tokens, which caps the ring depth; at 65..128 tokens all 512, as for
+ * MXFP8).  Workspace as qlinear_fp8_dynamic (same plans; no two-pass
+ * reduction, whose requests take the last-arriving CTA). */
 QGD_API qgd_status qlinear_nvfp4(const void* xq, const void* sx_e4m3, const float* gx, const void* wq,
                                  const void* sw_e4m3, const float* gw, void* y_bf16, int M, int N, int K, void* ws,
                                  size_t ws_bytes, void* stream);
@@ -356,7 +359,7 @@ QGD_API qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* w
  * Plan: the layer plan for (fmt, M, N, K) forced to Swap-AB (the Standard
  * kernels have no such epilogue) and to a reduction inside the GEMM kernel
  * (a two-pass request takes the last-arriving CTA).  M <= 128 (FP8_Dynamic,
- * W8A8_INT8), <= 64 (MXFP8, NVFP4), <= 32 (Block_FP8); more ->
+ * W8A8_INT8, MXFP8, NVFP4), <= 32 (Block_FP8); more ->
  * QGD_ERR_UNSUPPORTED.  M == 0 launches nothing and sets no flag: skip the
  * wait for such a call.  sw: the weight scales of the format (fp32 per
  * channel or per block; MXFP8 E8M0 bytes; NVFP4 the fp32 row scales), and

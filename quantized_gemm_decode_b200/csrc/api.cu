@@ -127,11 +127,15 @@ const int kBuckets[] = {1, 2, 4, 8, 16, 24, 32, 64, 128, 512, 2048, 8192};
 constexpr int kNumBuckets = sizeof(kBuckets) / sizeof(kBuckets[0]);
 constexpr int kDecodeMaxM = 32;   // decode token counts: Swap-AB by default
 constexpr int kSwapMaxM = 128;    // largest token count the Swap-AB kernel covers (FP8_Dynamic, W8A8_INT8)
-// MXFP8: at most 64 tokens, and at most 256 tensor-memory columns per CTA, so
-// that two CTAs always fit in an SM's 512 columns (a CTA whose allocation had
-// to wait for a cluster peer on the same SM would never be released)
-constexpr int kMxMaxM = 64;
+// MXFP8 / NVFP4: at most 128 tokens.  Up to 64 tokens a CTA takes at most 256
+// tensor-memory columns, so that two CTAs always fit in an SM's 512 (a CTA
+// whose allocation had to wait for a cluster peer on the same SM would never
+// be released); at 128 tokens it takes all 512 (two 128-column accumulators
+// and the scale slots), and its ring holds at least four K slices, so that
+// its shared memory keeps it alone on its SM.
+constexpr int kMxMaxM = 128;
 constexpr unsigned kMxMaxCols = 256;
+constexpr int kMxWideSlices = 4;  // K slices in the ring of a 128-token CTA, at least
 
 // Token columns of the Swap-AB MMA (its N): the next of 16, 32, 64, 128.
 int swap_mpad(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
@@ -327,8 +331,16 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
       p.split_k = floor_pow2(p.split_k);
     }
   }
-  if (fmt == kFmtMX || fmt == kFmtNV)
-    while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices, fmt) > kMxMaxCols) --p.stages;
+  if (fmt == kFmtMX || fmt == kFmtNV) {
+    if (mpad < 128) {
+      while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices, fmt) > kMxMaxCols) --p.stages;
+    } else {
+      // 128 tokens: all 512 columns, and a ring deep enough to fill more than
+      // half of the SM's shared memory (one CTA per SM)
+      while (p.stages * p.k_slices < kMxWideSlices && p.stages < max_st) ++p.stages;
+      while (p.stages > 2 && mx_tmem_cols(mpad, p.stages, p.k_slices, fmt) > 512u) --p.stages;
+    }
+  }
   // CTAs per SM for the persistent grid: at most what shared memory (and, for
   // the Standard kernel, TMEM) allows, at most 2; 0 asks for that maximum.
   int fit = 1;

@@ -2344,6 +2344,7 @@ static cudaError_t launch_swapab_f(int fmt, int mpad, const CUtensorMap& tw, con
         case 16: return launch_swapab_t<kFmtNV, 16, false>(tw, tx, a, stream);
         case 32: return launch_swapab_t<kFmtNV, 32, false>(tw, tx, a, stream);
         case 64: return launch_swapab_t<kFmtNV, 64, false>(tw, tx, a, stream);
+        case 128: return launch_swapab_t<kFmtNV, 128, false>(tw, tx, a, stream);
       }
     }
   }

@@ -320,7 +320,7 @@ def main(argv=None):
     wls = [w for w in (workloads.FP8_DECODE, workloads.INT8_DECODE, workloads.BLOCK_DECODE, workloads.MX_DECODE,
                        workloads.NV_DECODE) if w.fmt in fmts]
     if args.large_m:
-        wls += [w for w in workloads.LARGE if w.fmt in fmts]
+        wls += [w for w in workloads.LARGE + workloads.LARGE_BS if w.fmt in fmts]
     if args.tp8:
         wls.append(workloads.FP8_TP8)
     done = {}

@@ -59,11 +59,17 @@ LARGE = tuple(
 NV_DECODE = Workload("nvfp4_decode_sweep_8b_shapes", NVFP4, SHAPES_8B, DECODE_M, 1006, True,
                      "NVFP4 (E2M1 values, E4M3 scale per 16 along K, fp32 per row), 8B-class shapes x M in 1..32, "
                      "1% x20 outlier channels")
+# the block-scaled formats past the decode buckets: their kernels cover up to 128 tokens
+MID_M = (64, 128)
+LARGE_BS = tuple(
+    Workload(f"{fmt}_mid_m_8b_shapes", fmt, SHAPES_8B, MID_M, 1008, True, f"{fmt}, 8B-class shapes x M in 64, 128")
+    for fmt in (MXFP8, NVFP4))
+
 # one rank's weight shard of the 8B-class layers split column-parallel over 8 GPUs
 SHAPES_8B_TP8 = tuple((n // 8, k) for (n, k) in SHAPES_8B)
 FP8_TP8 = Workload("fp8_dynamic_decode_tp8_shards_8b", FP8_DYNAMIC, SHAPES_8B_TP8, DECODE_M, 1007, True,
                    "FP8_Dynamic, one of 8 column-parallel shards of the 8B-class shapes x M in 1..32")
-ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE, MX_DECODE, NV_DECODE, FP8_TP8) + LARGE
+ALL = (TINY, FP8_DECODE, INT8_DECODE, BLOCK_DECODE, MX_DECODE, NV_DECODE, FP8_TP8) + LARGE + LARGE_BS
 
 
 def algorithmic_bytes(fmt: str, M: int, N: int, K: int) -> int:

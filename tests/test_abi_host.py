@@ -581,7 +581,7 @@ def test_nvfp4_plan_rules_and_rejects():
     L = qgd.lib()
     P = ctypes.c_void_p
     assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 4, 512, 1152, None, 0, None) == -2
-    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 65, 512, 1024, None, 0, None) == -2
+    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 129, 512, 1024, None, 0, None) == -2
     assert L.quant_nvfp4(P(16), 4, 1000, 1000, P(16), P(16), P(16), None) == -2
     assert L.qlinear_nvfp4(P(16), None, P(16), P(16), P(16), P(16), P(16), 4, 512, 1024, None, 0, None) == -1
     # the layer workspace holds the packed codes, the row scales and the block scales
@@ -623,7 +623,7 @@ def test_column_parallel_call_rules():
     assert call(_tp_desc(null_y=True)) == -1
     assert call(_tp_desc(), fmt=0, M=129) == -2           # beyond the Swap-AB kernel's 128 tokens
     assert call(_tp_desc(), fmt=2, M=33) == -2            # Block_FP8: 32
-    assert call(_tp_desc(), fmt=4, M=65, K=1024) == -2    # NVFP4: 64
+    assert call(_tp_desc(), fmt=4, M=129, K=1024) == -2   # NVFP4: 128
     assert call(_tp_desc(), ws=None, wsn=0) == -3
     assert call(_tp_desc(), fmt=5) == -1
     assert L.qgd_tp_wait(None, 1, None) == -1

@@ -67,7 +67,8 @@ PLANS = [
     (SW, 1, LAST, 2, 0, PERS, 1, 2),
     (SW, 1, LAST, 3, 0, PERS, 2, 1),
 ]
-SHAPES = [(1, 1024, 1024), (5, 768, 2048), (16, 1024, 4096), (32, 512, 1152), (64, 512, 2048)]
+SHAPES = [(1, 1024, 1024), (5, 768, 2048), (16, 1024, 4096), (32, 512, 1152), (64, 512, 2048), (65, 640, 1024),
+          (100, 512, 2048), (128, 1024, 1152)]
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=[f"M{m}-N{n}-K{k}" for m, n, k in SHAPES])
@@ -87,7 +88,7 @@ def test_mx_gemm_matches_oracle(shape, plan):
     check_fp8_tolerance(bf16_to_f64(y), yref, bound, K, f"MXFP8 M={M} N={N} K={K} plan={p}")
 
 
-@pytest.mark.parametrize("M", [1, 7, 32])
+@pytest.mark.parametrize("M", [1, 7, 32, 97, 128])
 def test_mx_layer_call_from_bf16(M):
     # quantizer into the workspace, then the GEMM: the same codes and output
     N, K = 1024, 2048
@@ -111,5 +112,16 @@ def test_mx_rejects_what_it_does_not_cover():
     P = ctypes.c_void_p
     # K not a multiple of 128, more than 128 tokens: refused before any launch
     assert L.qlinear_mxfp8(P(16), P(16), P(16), P(16), P(16), 4, 512, 1056, None, 0, None) == -2
-    assert L.qlinear_mxfp8(P(16), P(16), P(16), P(16), P(16), 65, 512, 1024, None, 0, None) == -2
+    assert L.qlinear_mxfp8(P(16), P(16), P(16), P(16), P(16), 129, 512, 1024, None, 0, None) == -2
     assert L.quant_act_mx(P(16), 4, 1000, 1000, P(16), P(16), None) == -2
+
+
+@pytest.mark.parametrize("fmt", [qgd.FMT_MXFP8, qgd.FMT_NVFP4])
+def test_block_scaled_128_token_plans_take_the_whole_sm(fmt):
+    # 65..128 tokens: 512 tensor-memory columns, and a ring of at least four K
+    # slices, which keeps one CTA per SM whatever the override asks
+    for kps, stages in ((1, 2), (2, 2), (1, 0), (2, 0)):
+        qgd.qgd_set_override(fmt, SW, 1, LAST, stages, 0, GRID, 1, kps)
+        p = qgd.qgd_get_plan(fmt, 100, 4096, 4096)
+        assert p["stages"] * p["k_slices"] >= 4, p
+    qgd.qgd_set_override(fmt)

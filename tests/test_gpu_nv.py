@@ -84,7 +84,8 @@ PLANS = [
     (SW, 1, LAST, 3, 0, PERS, 2, 1),
     (SW, 1, LAST, 0, 0, PERS, 1, 1),
 ]
-SHAPES = [(1, 1024, 1024), (5, 768, 2048), (16, 1024, 4096), (32, 512, 2304), (64, 512, 2048)]
+SHAPES = [(1, 1024, 1024), (5, 768, 2048), (16, 1024, 4096), (32, 512, 2304), (64, 512, 2048), (65, 640, 1024),
+          (100, 512, 2048), (128, 1024, 2304)]
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=[f"M{m}-N{n}-K{k}" for m, n, k in SHAPES])
@@ -104,7 +105,7 @@ def test_nv_gemm_matches_oracle(shape, plan):
     check_fp8_tolerance(bf16_to_f64(y), yref, bound, K, f"NVFP4 M={M} N={N} K={K} plan={p}")
 
 
-@pytest.mark.parametrize("M", [1, 7, 32, 64])
+@pytest.mark.parametrize("M", [1, 7, 32, 64, 97, 128])
 def test_nv_layer_call_from_bf16(M):
     # quantizer into the workspace, then the GEMM: the same output
     N, K = 1024, 2048
@@ -126,7 +127,7 @@ def test_nv_rejects_what_it_does_not_cover():
     L = qgd.lib()
     import ctypes
     P = ctypes.c_void_p
-    # K not a multiple of 256, more than 64 tokens: refused before any launch
+    # K not a multiple of 256, more than 128 tokens: refused before any launch
     assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 4, 512, 1152, None, 0, None) == -2
-    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 65, 512, 1024, None, 0, None) == -2
+    assert L.qlinear_nvfp4(P(16), P(16), P(16), P(16), P(16), P(16), P(16), 129, 512, 1024, None, 0, None) == -2
     assert L.quant_nvfp4(P(16), 4, 1000, 1000, P(16), P(16), P(16), None) == -2
