@@ -1316,6 +1316,7 @@ __device__ __forceinline__ void std_cluster_reduce(const GemmArgs& a, SmemCtl* c
   const int m_tile = tile % m_tiles, n_tile = tile / m_tiles;
   const int Rm = (kStdTileM + S - 1) / S;  // most rows any owner holds
   tc_fence_before();
+  __syncwarp();  // the role branches leave warps diverged; the cluster barrier is warp-aligned
   cluster_sync_all();
   // an aborted CTA may still have copies landing in its ring: no exchange then
   bool abort = false;
@@ -1350,6 +1351,7 @@ __device__ __forceinline__ void std_cluster_reduce(const GemmArgs& a, SmemCtl* c
     }
   }
   tc_fence_before();
+  __syncwarp();
   cluster_sync_all();
   if (warp < 2) return;
   if (abort) {
