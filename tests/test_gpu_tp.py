@@ -119,6 +119,8 @@ CASES = [
     ("block_fp8", [8], [128, 128, 256, 128, 384, 128, 256, 128], 512),
     ("mxfp8", [4, 33], [256, 512], 1024),
     ("nvfp4", [2, 64], [512, 256, 256], 2048),
+    ("nvfp4", [100, 128], [256, 384], 1024),
+    ("mxfp8", [128, 65], [384, 256, 128], 1024),
     ("fp8_dynamic", [100], [256, 256], 1024),
 ]
 
