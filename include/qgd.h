@@ -354,7 +354,10 @@ QGD_API qgd_status qlinear_nvfp4_bf16(const void* x_bf16, int ldx, const void* w
  * after qgd_tp_wait on its own flags in stream order after its own call.
  * Because another rank may already run its next call and write into this
  * rank's Y while this rank still reads the previous result, alternate
- * between two output buffers (the flags need no second copy).
+ * between two output buffers (the flags need no second copy).  A kernel that
+ * gave up on one of its bounded waits still advances and raises its count
+ * (every rank stays in step), so its share of Y is then incomplete: every
+ * rank should check qgd_device_error() before trusting a result.
  *
  * Plan: the layer plan for (fmt, M, N, K) forced to Swap-AB (the Standard
  * kernels have no such epilogue) and to a reduction inside the GEMM kernel
