@@ -18,8 +18,8 @@
  * implementa el kernel?" and its matmul listing): Standard (each CTA owns an
  * output tile and reduces all of K), Split-K (K is cut into split_k parts,
  * split_k a power of two from 1 to 256 -- any count from 2 to 8 when the
- * splits reduce inside a thread-block cluster -- whose partial sums are then
- * added)
+ * splits reduce inside a thread-block cluster, and any count in CTA-pair
+ * tiles -- whose partial sums are then added)
  * and Swap-AB (the product is computed as (W . X^T)^T so the wide N dimension
  * fills the MMA's M slot).  Which one runs for a shape is chosen from a
  * measured dispatch table (section "Hybrid dispatch" / "Despacho hibrido":
@@ -82,8 +82,8 @@ typedef enum { QGD_QTYPE_E4M3 = 0, QGD_QTYPE_INT8 = 1 } qgd_qtype;
  * Standard orientation with 256-token x 256-weight-row tiles, each computed by two CTAs on two SMs
  * (one 2-CTA cluster, tcgen05 cta_group::2): each CTA loads half of the tile's token rows and half
  * of its weight rows, so operand traffic per FLOP is two thirds of a one-CTA 128 x 256 tile's.
- * FP8_Dynamic and W8A8_INT8 only (other formats get Standard), no Split-K, table name
- * "standard_pair". */
+ * FP8_Dynamic and W8A8_INT8 only (other formats get Standard); Split-K only with the two-pass
+ * reduction (any split_k above 1 takes it, not only powers of two), table name "standard_pair". */
 typedef enum {
   QGD_VARIANT_AUTO = -1,
   QGD_VARIANT_STANDARD = 0,
@@ -116,7 +116,8 @@ typedef enum {
 typedef struct {
   int variant;  /* qgd_variant (never AUTO here) */
   int split_k;  /* grid schedule: CTAs along K, 1..256, at most ceil(K/128); a power of two
-                   except with QGD_REDUCE_CLUSTER, which takes any 2..8 */
+                   except with QGD_REDUCE_CLUSTER, which takes any 2..8, and in Standard pair
+                   tiles, which take any count */
   int reduce;   /* qgd_reduce, used when several CTAs share an output tile */
   int stages;   /* depth of the shared-memory operand ring */
   int tile_n;   /* Standard: output columns per CTA (128 or 256); Swap-AB: 128 */

@@ -101,6 +101,24 @@ qgd_status encode_out_bf16(CUtensorMap* map, void* base, int rows, int cols) {
   return QGD_OK;
 }
 
+// Split-K partials as a 3-D tensor [splits][rows][cols] of 32-bit words
+// (fp32 or int32 accumulator bits), boxes of 32 rows x 32 words, 128-byte
+// swizzle: a box clips at `rows` within its own split.
+qgd_status encode_partial_u32(CUtensorMap* map, void* base, int splits, int rows, int cols) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(splits)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4, static_cast<cuuint64_t>(rows) * cols * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(QGD_ERR_CUDA, "cuTensorMapEncodeTiled (partials) failed (%d) splits=%d rows=%d cols=%d", (int)r, splits,
+                rows, cols);
+  return QGD_OK;
+}
+
 qgd_status encode_kmajor(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
@@ -271,16 +289,13 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
     if (p.reduce == kTwoPass) p.reduce = kLastCta;
   }
   if (p.variant == kSwapAB && M > (fmt == kFmtBlock ? kDecodeMaxM : kSwapMaxM)) p.variant = kStandard;
-  // CTA-pair tiles: the per-token / per-channel formats, no Split-K
+  // CTA-pair tiles: the per-token / per-channel formats; Split-K with the
+  // two-pass reduction only
   if (p.variant == kStandardPair && fmt != kFmtFP8 && fmt != kFmtINT8) p.variant = kStandard;
   if (p.variant < kStandard || p.variant > kStandardPair) p.variant = kStandard;
   if (p.variant == kSwapAB) p.tile_n = kSwapTileN;
   else if (p.variant == kStandardPair) p.tile_n = 256;
   else if (p.tile_n != 128 && p.tile_n != 256) p.tile_n = (fmt == kFmtBlock) ? 128 : 256;
-  if (p.variant == kStandardPair) {
-    p.split_k = 1;
-    p.reduce = kLastCta;
-  }
   if (p.schedule != kPersistent) p.schedule = kGrid;
   // 128-wide K slices (K blocks) per pipeline stage: 1 or 2, at most the K extent
   if (p.k_slices < 1 || nkt < 2) p.k_slices = 1;
@@ -290,8 +305,10 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
   if (smax < 1) smax = 1;
   if (p.split_k < 1) p.split_k = 1;
   if (p.split_k > smax) p.split_k = smax;
-  // a power of two, except in a cluster, whose reduction takes any 2..8
-  if (p.reduce != kCluster) p.split_k = floor_pow2(p.split_k);
+  // a power of two, except in a cluster, whose reduction takes any 2..8, and
+  // in pair tiles, whose two-pass reduction takes any count
+  const bool any_split = p.reduce == kCluster || p.variant == kStandardPair;
+  if (!any_split) p.split_k = floor_pow2(p.split_k);
   if (p.reduce < kLastCta || p.reduce > kCluster) p.reduce = kLastCta;
   // the two-pass reduction kernel covers at most 32 tokens
   if (p.variant == kSwapAB && M > kDecodeMaxM && p.reduce == kTwoPass) p.reduce = kLastCta;
@@ -302,7 +319,8 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
   if (p.reduce == kCluster && ((p.variant != kSwapAB && !std_cluster_ok) || p.schedule != kGrid || p.split_k < 2 ||
                                p.split_k > kMaxClusterSplit))
     p.reduce = kLastCta;
-  if (p.reduce != kCluster) p.split_k = floor_pow2(p.split_k);
+  if (p.reduce != kCluster && p.variant != kStandardPair) p.split_k = floor_pow2(p.split_k);
+  if (p.variant == kStandardPair) p.reduce = p.split_k > 1 ? kTwoPass : kLastCta;
   if (p.reduce != kTwoPass) {
     const size_t tiles = p.variant == kSwapAB
                              ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
@@ -423,13 +441,16 @@ Exec make_exec(int fmt, const qgd_plan& p, int M, int N, int K) {
   } else if (p.variant == kStandardPair) {
     // 256 x 256 pair tiles dealt to CTA pairs (two CTAs each, one per SM);
     // the launch lowers the pair count to what fits on the GPU at once
-    e.maxc = 1;
+    // ((tile, split) items with Split-K, whose fp32 partials a second kernel adds)
+    e.maxc = p.split_k;
     e.tiles = static_cast<size_t>((N + 255) / 256) * ((M + 255) / 256);
     if (p.schedule == kPersistent) {
+      const long long items = static_cast<long long>(e.tiles) * p.split_k;
       const long long pairs = g_num_sms / 2;
       e.persistent = true;
-      e.ctas = static_cast<int>(2 * (static_cast<long long>(e.tiles) < pairs ? static_cast<long long>(e.tiles) : pairs));
+      e.ctas = static_cast<int>(2 * (items < pairs ? items : pairs));
     }
+    if (p.split_k > 1) e.data_bytes = align256(static_cast<size_t>(M) * N * 4 * p.split_k);
   } else {
     e.maxc = p.split_k;
     e.tiles = static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);
@@ -591,7 +612,11 @@ qgd_status run_gemm_plan(int fmt, const qgd_plan& p, const void* xq, const float
     if ((st = encode_kmajor(&tw, wq, N, K, 128)) != QGD_OK) return st;
     CUtensorMap ty;
     memset(&ty, 0, sizeof ty);
-    if (!raw && (st = encode_out_bf16(&ty, y, M, N)) != QGD_OK) return st;
+    if (a.splits > 1) {  // fp32 / int32 partials, one plane per split, for the two-pass reduction
+      if ((st = encode_partial_u32(&ty, a.partial, a.splits, M, N)) != QGD_OK) return st;
+    } else if (!raw && (st = encode_out_bf16(&ty, y, M, N)) != QGD_OK) {
+      return st;
+    }
     if (a.persistent) {
       const int fit = pair_clusters_that_fit(fmt, p.stages, p.k_slices);
       if (fit > 0 && a.ctas > 2 * fit) a.ctas = 2 * fit;
@@ -1083,9 +1108,11 @@ qgd_status qgd_load_dispatch_table(const char* path) {
       return fail(QGD_ERR_TABLE, "%s:%d: unknown format/variant/reduce/schedule name", path, lineno);
     if (N <= 0 || K <= 0 || bucket_of(Mb) != Mb)
       return fail(QGD_ERR_TABLE, "%s:%d: bad N/K or M bucket %d", path, lineno, Mb);
-    if (split < 1 || split > 256 || ((split & (split - 1)) != 0 && !(red == kCluster && split <= kMaxClusterSplit)))
-      return fail(QGD_ERR_TABLE, "%s:%d: split_k %d is not a power of two in 1..256 (or 2..8 with cluster)", path,
-                  lineno, split);
+    if (split < 1 || split > 256 ||
+        ((split & (split - 1)) != 0 && !(red == kCluster && split <= kMaxClusterSplit) && var != kStandardPair))
+      return fail(QGD_ERR_TABLE,
+                  "%s:%d: split_k %d is not a power of two in 1..256 (or 2..8 with cluster, any with pair tiles)",
+                  path, lineno, split);
     if (stages < 0 || stages > kMaxStages || (tile_n != 0 && tile_n != 128 && tile_n != 256) || occ < 0 ||
         occ > 2)
       return fail(QGD_ERR_TABLE, "%s:%d: bad stages/tile_n/occupancy", path, lineno);
@@ -1109,8 +1136,10 @@ qgd_status qgd_set_override(int fmt, int variant, int split_k, int reduce, int s
       occupancy < 0 || occupancy > 2 || k_slices < 0 || k_slices > 2 ||
       (tile_n != 0 && tile_n != 128 && tile_n != 256))
     return fail(QGD_ERR_INVALID, "bad override");
-  if (split_k > 0 && (split_k & (split_k - 1)) != 0 && !(reduce == kCluster && split_k <= kMaxClusterSplit))
-    return fail(QGD_ERR_INVALID, "split_k must be a power of two (any 2..8 with the cluster reduction)");
+  if (split_k > 0 && (split_k & (split_k - 1)) != 0 && !(reduce == kCluster && split_k <= kMaxClusterSplit) &&
+      variant != kStandardPair)
+    return fail(QGD_ERR_INVALID,
+                "split_k must be a power of two (any 2..8 with the cluster reduction, any with pair tiles)");
   std::lock_guard<std::mutex> lk(g_mu);
   Override& o = g_override[fmt];
   o.variant = variant < 0 ? -1 : variant;

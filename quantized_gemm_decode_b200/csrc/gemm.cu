@@ -1856,7 +1856,7 @@ constexpr int kPairTileN = 256;  // weight rows per pair tile (MMA N)
 // leave as whole 128-byte lines.
 constexpr uint32_t kPairStageBytes = 4 * 2 * 32 * 128;
 
-template <int kFmt>
+template <int kFmt, bool kSplitK>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     standard_pair_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                          const __grid_constant__ CUtensorMap ty, const GemmArgs a) {
@@ -1883,12 +1883,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nkt = (a.K + kTileK - 1) / kTileK;
   const int m_tiles = (a.M + kPairTileM - 1) / kPairTileM;
   const int n_tiles = (a.N + kPairTileN - 1) / kPairTileN;
-  const long long items = static_cast<long long>(m_tiles) * n_tiles;
+  // work items: (pair tile, K split), the splits of a tile adjacent; with
+  // Split-K (a separate instantiation, so that the one-split kernel keeps its
+  // own code) each split writes its partial for a second kernel to add
+  const int S = kSplitK ? a.splits : 1;
+  const long long items = static_cast<long long>(m_tiles) * n_tiles * S;
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tx);
     tma_prefetch_desc(&tw);
-    if (!a.raw) tma_prefetch_desc(&ty);
+    if (!a.raw || S > 1) tma_prefetch_desc(&ty);
     for (int i = 0; i < stages; ++i) {
       mbar_init(&ctl->full[i], 1);
       mbar_init(&ctl->empty[i], 1);
@@ -1931,10 +1935,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int i = 0;
       bool stop = false;
       for (long long w = pair; w < items && !stop; w += npairs) {
-        const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
+        const long long tile = w / S;
+        const int split = static_cast<int>(w % S);
+        const int mt = static_cast<int>(tile % m_tiles), nt = static_cast<int>(tile / m_tiles);
+        const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
+        const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
         const int xrow = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2);
         const int wrow = nt * kPairTileN + static_cast<int>(rank) * (kPairTileN / 2);
-        for (int kt = 0; kt < nkt; kt += kps, ++i) {
+        for (int kt = kt0; kt < kt1; kt += kps, ++i) {
           const int s = i % stages;
           const uint32_t round = i / stages;
           if (!mbar_wait(&ctl->empty[s], (round & 1) ^ 1)) {
@@ -1946,7 +1954,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             stop = true;
             break;
           }
-          const int ns = (nkt - kt) < kps ? (nkt - kt) : kps;
+          const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;
           // the leader's barrier expects both CTAs' bytes (a copy may land first)
           if (rank == 0) mbar_arrive_expect_tx(&ctl->full[s], 2u * ns * (kXBytes + kWBytes));
           const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
@@ -1965,13 +1973,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int i = 0, li = 0;
       bool stop = false;
       for (long long w = pair; w < items && !stop; w += npairs, ++li) {
+        const int split = static_cast<int>(w % S);
+        const int kt0 = static_cast<int>(static_cast<long long>(split) * nkt / S);
+        const int kt1 = static_cast<int>(static_cast<long long>(split + 1) * nkt / S);
         const int buf = li & 1;
         if (!mbar_wait(&ctl->tempty[buf], ((li >> 1) & 1) ^ 1)) {
           fail(kErrWaitMma);
           break;
         }
         const uint32_t d = tmem + buf * kPairTileN;
-        for (int kt = 0; kt < nkt && !stop; kt += kps, ++i) {
+        for (int kt = kt0; kt < kt1 && !stop; kt += kps, ++i) {
           const int s = i % stages;
           const uint32_t round = i / stages;
           if (!mbar_wait(&ctl->full[s], round & 1)) {
@@ -1984,13 +1995,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const int ns = (nkt - kt) < kps ? (nkt - kt) : kps;
+          const int ns = (kt1 - kt) < kps ? (kt1 - kt) : kps;
           for (int h = 0; h < ns; ++h) {
 #pragma unroll
             for (int kk = 0; kk < kTileK / 32; ++kk) {
               const uint64_t ad = sdesc_kmajor_sw128(x_base + s * stage_x + h * kXBytes + kk * 32);
               const uint64_t bd = sdesc_kmajor_sw128(w_base + s * stage_w + h * kWBytes + kk * 32);
-              mma_issue_pair<kInt>(d, ad, bd, kIdesc, (kt + h > 0 || kk > 0) ? 1u : 0u);
+              mma_issue_pair<kInt>(d, ad, bd, kIdesc, (kt + h > kt0 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit_pair(&ctl->empty[s], 0x3);
@@ -2011,7 +2022,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int nstore = 0;                                // tensor stores this warp has issued
     int li = 0;
     for (long long w = pair; w < items; w += npairs, ++li) {
-      const int mt = static_cast<int>(w % m_tiles), nt = static_cast<int>(w / m_tiles);
+      const long long tile = w / S;
+      const int split = static_cast<int>(w % S);
+      const int mt = static_cast<int>(tile % m_tiles), nt = static_cast<int>(tile / m_tiles);
       const int row0 = mt * kPairTileM + static_cast<int>(rank) * (kPairTileM / 2) + q * 32;  // this warp's rows
       const int m = row0 + lane;
       const bool in_m = m < M;
@@ -2039,14 +2052,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(tempty0 + static_cast<uint32_t>(buf) * 8u);
           }
+          if constexpr (kSplitK) {
+            // Split-K partial (raw accumulator bits) of row m, columns nc0 ..
+            // nc0 + 63: both 4 KB buffers, 32 columns each (the same 128-byte
+            // swizzle), then two tensor stores into split plane `split`
+            if (lane == 0 && nstore >= 1) bulk_wait_group_read<0>();  // the last group has read them
+            __syncwarp();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint8_t* row = ybuf + (g >> 1) * (32 * 128) + lane * 128;
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                st_shared_v4(row + ((((g & 1) * 4 + v) ^ (lane & 7)) << 4),
+                             make_uint4(r[g][4 * v], r[g][4 * v + 1], r[g][4 * v + 2], r[g][4 * v + 3]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < M && nc0 < N) {
+                tma_store_3d(&ty, ybuf, nc0, row0, split);
+                if (nc0 + 32 < N) tma_store_3d(&ty, ybuf + 32 * 128, nc0 + 32, row0, split);
+              }
+              bulk_commit_group();
+            }
+            ++nstore;
+            continue;
+          }
           if (a.raw) {  // int32 accumulators (test hook): plain stores
             if (in_m) {
+              uint32_t* out = static_cast<uint32_t*>(a.raw);
 #pragma unroll
               for (int g = 0; g < 4; ++g) {
                 const int nc = nc0 + g * 16;
                 if (nc >= N) break;
-                uint4* dst =
-                    reinterpret_cast<uint4*>(static_cast<uint32_t*>(a.raw) + static_cast<size_t>(m) * N + nc);
+                uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * N + nc);
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
                   dst[v] = make_uint4(r[g][4 * v], r[g][4 * v + 1], r[g][4 * v + 2], r[g][4 * v + 3]);
@@ -2375,17 +2414,25 @@ static cudaError_t launch_standard_t(const CUtensorMap& tx, const CUtensorMap& t
                    : launch_standard_k<kFmt, kTileN, 1>(tx, tw, a, stream);
 }
 
+template <int kFmt, bool kSplitK>
+static cudaError_t launch_standard_pair_split_t(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                                                const GemmArgs& a, cudaStream_t stream) {
+  static bool attr_done = false;
+  cudaError_t e = set_smem_attr(standard_pair_kernel<kFmt, kSplitK>, attr_done);
+  if (e != cudaSuccess) return e;
+  const long long items = static_cast<long long>((a.N + kPairTileN - 1) / kPairTileN) *
+                          ((a.M + kPairTileM - 1) / kPairTileM) * (kSplitK ? a.splits : 1);
+  const long long pairs = a.persistent && a.ctas / 2 < items ? a.ctas / 2 : items;
+  return launch_ex_cluster_xy(standard_pair_kernel<kFmt, kSplitK>, dim3(static_cast<unsigned>(2 * pairs)),
+                              dim3(kGemmThreads), pair_smem_bytes(a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, 2,
+                              1, tx, tw, ty, a);
+}
+
 template <int kFmt>
 static cudaError_t launch_standard_pair_t(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
                                           const GemmArgs& a, cudaStream_t stream) {
-  static bool attr_done = false;
-  cudaError_t e = set_smem_attr(standard_pair_kernel<kFmt>, attr_done);
-  if (e != cudaSuccess) return e;
-  const long long items = static_cast<long long>((a.N + kPairTileN - 1) / kPairTileN) *
-                          ((a.M + kPairTileM - 1) / kPairTileM);
-  const long long pairs = a.persistent && a.ctas / 2 < items ? a.ctas / 2 : items;
-  return launch_ex_cluster_xy(standard_pair_kernel<kFmt>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads),
-                              pair_smem_bytes(a.stages, a.kps > 1 ? 2 : 1), stream, a.pdl != 0, 2, 1, tx, tw, ty, a);
+  if (a.splits > 1) return launch_standard_pair_split_t<kFmt, true>(tx, tw, ty, a, stream);
+  return launch_standard_pair_split_t<kFmt, false>(tx, tw, ty, a, stream);
 }
 
 cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
@@ -2398,9 +2445,9 @@ cudaError_t launch_standard_pair(int fmt, const CUtensorMap& tx, const CUtensorM
 template <int kFmt>
 static int pair_clusters_t(cudaLaunchConfig_t& cfg) {
   static bool done = false;
-  if (set_smem_attr(standard_pair_kernel<kFmt>, done) != cudaSuccess) return 0;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmt>, &cfg) != cudaSuccess) {
+  if (set_smem_attr(standard_pair_kernel<kFmt, false>, done) != cudaSuccess) return 0;
+  int n = 0;  // (the Split-K instantiation has the same shared memory and block)
+  if (cudaOccupancyMaxActiveClusters(&n, standard_pair_kernel<kFmt, false>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }

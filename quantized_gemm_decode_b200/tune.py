@@ -10,8 +10,8 @@ inside the search space", "Hybrid dispatch addresses runtime overhead" and
 "Autoajuste de los kernels").  Here the space is small and discrete, so it is
 searched exhaustively: variant x tile x split_k x reduction x schedule x
 occupancy x K slices per stage at the deepest pipeline (and, for the
-thread-block-cluster reduction, every split count from 2 to 8, which can fill
-the SMs more evenly than a power of two), then the pipeline
+thread-block-cluster reduction and for CTA-pair tiles, other split counts,
+which can fill the SMs more evenly than a power of two), then the pipeline
 depth of the best few.  Each candidate is first checked against the
 split-free result (bit-exact int32 accumulators for W8A8_INT8, a relative
 bound for the fp32-accumulating formats), then timed as a graph of layer
@@ -168,11 +168,17 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
                 for s in range(2, 9):
                     if s <= nku:
                         out.append((0, s, 3, t, 0, 0, kps, 0))
-    # Standard pair tiles (256 x 256 on two SMs): the per-token formats past 128 tokens
+    # Standard pair tiles (256 x 256 on two SMs): the per-token formats past 128 tokens;
+    # Split-K (two-pass) when the pair tiles are fewer than the SM pairs
     if fmt in (FP8_DYNAMIC, W8A8_INT8) and M > 128:
+        pair_tiles = -(-M // 256) * -(-N // 256)
         for kps in kps_std:
+            nku = -(-nkt // kps)
             for sched in (0, 1):
                 out.append((2, 1, 0, 256, sched, 0, kps, 0))
+            for s in range(2, 7):
+                if s <= nku and pair_tiles < 74:
+                    out.append((2, s, 1, 256, 0, 0, kps, 0))
     return out
 
 

@@ -317,12 +317,22 @@ def test_table_k_slices_column(tmp_path):
 def test_standard_pair_plan_rules():
     P, G = qgd.SCHEDULE_PERSISTENT, qgd.SCHEDULE_GRID
     for fmt in (qgd.FMT_FP8_DYNAMIC, qgd.FMT_W8A8_INT8):
-        qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 4, qgd.REDUCE_TWO_PASS, 0, 128, P, 0, 2)
+        qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, qgd.REDUCE_TWO_PASS, 0, 128, P, 0, 2)
         p = qgd.qgd_get_plan(fmt, 4096, 6144, 4096)
-        # pair tiles are 256 wide and never split K; two K blocks per stage fit three stages
-        assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"], p["stages"], p["occupancy"]) == \
-            (qgd.VARIANT_STANDARD_PAIR, 256, 1, 2, 3, 1)
+        # pair tiles are 256 wide; two K blocks per stage fit three stages
+        assert (p["variant"], p["tile_n"], p["split_k"], p["reduce"], p["k_slices"], p["stages"],
+                p["occupancy"]) == (qgd.VARIANT_STANDARD_PAIR, 256, 1, qgd.REDUCE_LAST_CTA, 2, 3, 1)
         assert qgd.qgd_workspace_size(fmt, 4096, 6144, 4096) == 0
+        # Split-K always takes the two-pass reduction: one fp32 partial per split
+        # after the 64 KiB header, any count up to the K units
+        for split, red in ((4, qgd.REDUCE_LAST_CTA), (4, qgd.REDUCE_ATOMIC), (3, qgd.REDUCE_CLUSTER),
+                           (64, qgd.REDUCE_TWO_PASS)):
+            qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, split, red, 0, 0, G, 0, 2)
+            p = qgd.qgd_get_plan(fmt, 512, 1024, 4096)
+            want = {4: 4, 3: 3, 64: 16}[split]  # 32 K blocks / 2 per stage = 16 K units
+            assert (p["variant"], p["split_k"], p["reduce"]) == (qgd.VARIANT_STANDARD_PAIR, want,
+                                                                 qgd.REDUCE_TWO_PASS), (split, red, p)
+            assert qgd.qgd_workspace_size(fmt, 512, 1024, 4096) == 65536 + 512 * 1024 * 4 * want
         qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, G, 0, 1)
         # one-block stages of 32 KB beside the 32 KB output staging area
         assert qgd.qgd_get_plan(fmt, 512, 6144, 4096)["stages"] == (232448 - 2048 - 32768) // 32768

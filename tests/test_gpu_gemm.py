@@ -329,21 +329,28 @@ def test_standard_two_blocks_per_stage(fmt, plan, M, N, K):
 # Standard pair tiles (256 tokens x 256 weight rows on two SMs, tcgen05
 # cta_group::2): each CTA loads half the token rows and half the weight rows;
 # M = 40 leaves the second CTA's token rows all past M (zero-filled copies),
-# N = 528 a ragged last weight tile, K = 1152 an odd block count.
-PAIR_PLANS = [(GRID, 1, 256), (GRID, 2, 256), (PERSISTENT, 1, 256), (PERSISTENT, 2, 256)]
+# N = 528 a ragged last weight tile, K = 1152 an odd block count.  With
+# Split-K (two-pass) the K blocks split unevenly where the count is odd.
+PAIR_PLANS = [(GRID, 1, 256, 1), (GRID, 2, 256, 1), (PERSISTENT, 1, 256, 1), (PERSISTENT, 2, 256, 1),
+              (GRID, 1, 256, 2), (GRID, 2, 256, 4), (PERSISTENT, 1, 256, 4), (GRID, 1, 256, 3)]
 
 
 @pytest.mark.parametrize("fmt", [FP8_DYNAMIC, W8A8_INT8])
-@pytest.mark.parametrize("plan", PAIR_PLANS, ids=[f"sch{p[0]}-k{p[1]}-t{p[2]}" for p in PAIR_PLANS])
+@pytest.mark.parametrize("plan", PAIR_PLANS, ids=[f"sch{p[0]}-k{p[1]}-t{p[2]}-s{p[3]}" for p in PAIR_PLANS])
 @pytest.mark.parametrize("M,N,K", [(256, 256, 512), (40, 528, 1152), (300, 1024, 128), (520, 784, 2048)])
 def test_standard_pair_tiles(fmt, plan, M, N, K):
-    sched, kps, tile = plan
+    sched, kps, tile, split = plan
     case = Case(fmt, M, N, K, seed=M * 3 + N + K, outliers=True)
     yref, bound = _oracle(case)[:2]
-    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, tile, sched, 0, kps)
+    qgd.qgd_set_override(FMT_ID[fmt], qgd.VARIANT_STANDARD_PAIR, split, qgd.REDUCE_TWO_PASS, 0, tile, sched, 0,
+                         kps)
     p = qgd.qgd_get_plan(FMT_ID[fmt], M, N, K)
-    assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"]) == (qgd.VARIANT_STANDARD_PAIR, tile, 1,
-                                                                        kps if K > 128 else 1)
+    kps = kps if K > 128 else 1
+    nku = -(-(K // 128) // kps)
+    want_split = min(split, nku)
+    assert (p["variant"], p["tile_n"], p["split_k"], p["k_slices"]) == (qgd.VARIANT_STANDARD_PAIR, tile, want_split,
+                                                                        kps)
+    assert p["reduce"] == (qgd.REDUCE_TWO_PASS if want_split > 1 else qgd.REDUCE_LAST_CTA)
     y1 = case.run()
     case.check_output(y1, yref, bound, f"{fmt} pair M={M} N={N} K={K} plan={p}")
     y2 = case.run()

@@ -87,7 +87,8 @@ def test_every_plan_is_legal(table, shape, ov):
     if v == STD:
         assert tile in (128, 256)
     if v == PAIR:
-        assert fmt in (FP8, INT8) and s == 1 and tile == 256
+        assert fmt in (FP8, INT8) and tile == 256
+        assert r == (1 if s > 1 else 0)  # Split-K through the two-pass reduction only
     assert kps in (1, 2) and (kps == 1 or nkt >= 2)
     assert stages >= 2 and occ >= 1 and sched in (0, 1)
     assert 1 <= s <= 256 and s <= -(-nkt // kps)
@@ -99,8 +100,8 @@ def test_every_plan_is_legal(table, shape, ov):
             rows = -(-128 // s)
             assert (s - 1) * rows * tile * 4 <= stages * kps * (128 + tile) * 128  # received rows fit the ring
         assert ws == 0
-    else:
-        assert s & (s - 1) == 0  # a power of two outside a cluster
+    elif v != PAIR:
+        assert s & (s - 1) == 0  # a power of two outside a cluster and pair tiles
     if v == SWAP and M > 32:
         assert r != 1  # the two-pass reduction kernel covers 32 tokens
     if fmt in (MX, NV):
@@ -110,6 +111,8 @@ def test_every_plan_is_legal(table, shape, ov):
             assert cols <= 256
         else:
             assert cols <= 512 and stages * kps >= 4  # a CTA that has its SM to itself
+    if v == PAIR and s > 1:
+        assert ws == 65536 + ((M * N * 4 * s + 255) // 256) * 256  # one fp32 partial per split
     if s == 1 and r != CLUSTER:
         assert ws == 0 or v == SWAP  # (Swap-AB persistent plans may split tiles between CTAs)
     assert ws >= 0
