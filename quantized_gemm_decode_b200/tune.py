@@ -177,7 +177,7 @@ def _candidates(fmt: str, M: int, N: int, K: int, num_sms: int, fz: bool):
             for sched in (0, 1):
                 out.append((2, 1, 0, 256, sched, 0, kps, 0))
             for s in range(2, 7):
-                if s <= nku and pair_tiles < 74:
+                if s <= nku and pair_tiles < num_sms // 2:
                     out.append((2, s, 1, 256, 0, 0, kps, 0))
     return out
 

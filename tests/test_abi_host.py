@@ -408,7 +408,7 @@ def test_table_cluster_reduce_name(tmp_path):
                                        ("block_fp8", 64, 6144, 4096), ("mxfp8", 16, 4096, 4096),
                                        ("mxfp8", 64, 6144, 4096), ("nvfp4", 1, 4096, 4096),
                                        ("nvfp4", 32, 4096, 12288), ("nvfp4", 64, 6144, 4096),
-                                       ("fp8_dynamic", 2048, 6144, 4096)])
+                                       ("fp8_dynamic", 2048, 6144, 4096), ("w8a8_int8", 512, 4096, 12288)])
 def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
     # every plan the tuner times is one the library runs as asked (no silent
     # legalization), and a grid-schedule Swap-AB candidate with more CTAs than
@@ -436,6 +436,11 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
                 smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + ((128 + 8) * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
     qgd.qgd_set_fused_override(fid)
+    # pair tiles split K (any count) only where they are fewer than the SM pairs
+    pair_splits = sorted({c[1] for c in cands if c[0] == qgd.VARIANT_STANDARD_PAIR and c[1] > 1})
+    pair_tiles = -(-M // 256) * -(-N // 256)
+    assert pair_splits == ([2, 3, 4, 5, 6] if fmt in ("fp8_dynamic", "w8a8_int8") and M > 128 and pair_tiles < 74
+                           else [])
 
 
 def test_fused_plan_field():
