@@ -321,7 +321,7 @@ qgd_plan make_plan(int fmt, int M, int N, int K, bool layer = false, bool tp = f
     p.reduce = kLastCta;
   if (p.reduce != kCluster && p.variant != kStandardPair) p.split_k = floor_pow2(p.split_k);
   if (p.variant == kStandardPair) p.reduce = p.split_k > 1 ? kTwoPass : kLastCta;
-  if (p.reduce != kTwoPass) {
+  if (p.reduce != kTwoPass && p.variant != kStandardPair) {  // (pair tiles take no arrival counters)
     const size_t tiles = p.variant == kSwapAB
                              ? static_cast<size_t>((N + kSwapTileN - 1) / kSwapTileN)
                              : static_cast<size_t>((N + p.tile_n - 1) / p.tile_n) * ((M + kStdTileM - 1) / kStdTileM);

@@ -333,6 +333,11 @@ def test_standard_pair_plan_rules():
             assert (p["variant"], p["split_k"], p["reduce"]) == (qgd.VARIANT_STANDARD_PAIR, want,
                                                                  qgd.REDUCE_TWO_PASS), (split, red, p)
             assert qgd.qgd_workspace_size(fmt, 512, 1024, 4096) == 65536 + 512 * 1024 * 4 * want
+        # more 128 x 256 tiles than arrival counters: pair tiles use none, so no split keeps no workspace
+        qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, P, 0, 2)
+        p = qgd.qgd_get_plan(fmt, 8192, 131072, 4096)
+        assert (p["variant"], p["split_k"], p["reduce"]) == (qgd.VARIANT_STANDARD_PAIR, 1, qgd.REDUCE_LAST_CTA)
+        assert qgd.qgd_workspace_size(fmt, 8192, 131072, 4096) == 0
         qgd.qgd_set_override(fmt, qgd.VARIANT_STANDARD_PAIR, 1, 0, 0, 0, G, 0, 1)
         # one-block stages of 32 KB beside the 32 KB output staging area
         assert qgd.qgd_get_plan(fmt, 512, 6144, 4096)["stages"] == (232448 - 2048 - 32768) // 32768
