@@ -522,6 +522,30 @@ def test_shipped_table_covers_every_benchmarked_shape():
                 assert qgd.qgd_workspace_size(fid[wl.fmt], M, N, K) >= 0
 
 
+def test_shipped_table_entries_run_as_written():
+    # every entry of the shipped table is what a call of its bucket's token
+    # count runs, field for field: none is silently legalised into another plan
+    qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
+    fid = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "mxfp8": 3, "nvfp4": 4}
+    var = {"standard": 0, "swap_ab": 1, "standard_pair": 2}
+    red = {"last_cta": 0, "two_pass": 1, "atomic": 2, "cluster": 3}
+    sch = {"grid": 0, "persistent": 1}
+    n = 0
+    for ln in open(qgd.DEFAULT_TABLE):
+        f = ln.split("#")[0].split()
+        if not f:
+            continue
+        fmt, N, K, M = fid[f[0]], int(f[1]), int(f[2]), int(f[3])
+        want = dict(variant=var[f[4]], split_k=int(f[5]), reduce=red[f[6]], stages=int(f[7]), tile_n=int(f[8]),
+                    schedule=sch[f[9]], occupancy=int(f[10]), k_slices=int(f[11]))
+        p = qgd.qgd_get_plan(fmt, M, N, K)
+        got = {k: p[k] for k in want}
+        assert got == want and p["source"] == 1, (ln, got)
+        assert qgd.qgd_get_layer_plan(fmt, M, N, K)["fused"] == int(f[12]), ln
+        n += 1
+    assert n > 200
+
+
 def test_binding_checks_gemm_operands_before_any_launch():
     # CPU tensors: every shape / dtype / size check runs before the device
     # check, so each mistake is reported as what it is, and nothing reaches
