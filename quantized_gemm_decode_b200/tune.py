@@ -19,10 +19,13 @@ calls (activation quantizer + GEMM, as the layer runs) that cycle through at
 least 3x L2 of distinct weight copies.
 
     python -m quantized_gemm_decode_b200.tune [--formats fp8_dynamic,...] [--out tables/b200.tsv]
-        [--large-m] [--resume]
+        [--large-m] [--resume [--recheck PCT]]
 
 Tuning time is reported separately on stderr.  With --resume, keys already in
-the output file are kept and skipped.
+the output file are kept and skipped; with --recheck PCT as well, each kept
+entry's plan is first timed again, and an entry now more than PCT percent
+slower than the time recorded beside it (a plan measured on older kernels) is
+tuned afresh.
 """
 from __future__ import annotations
 
@@ -42,6 +45,40 @@ L2_BYTES = 126 * 1024 * 1024
 FMT_ID = {FP8_DYNAMIC: 0, W8A8_INT8: 1, BLOCK_FP8: 2, MXFP8: 3, NVFP4: 4}
 VAR_NAME = {0: "standard", 1: "swap_ab", 2: "standard_pair"}
 RED_NAME = {0: "last_cta", 1: "two_pass", 2: "atomic", 3: "cluster"}
+SCHED_NAME = {0: "grid", 1: "persistent"}
+
+
+def parse_table_line(ln: str):
+    """(key, plan, recorded us) of one dispatch-table line -- key (fmt, N, K,
+    M bucket), plan (variant, split_k, reduce, stages, tile_n, schedule,
+    occupancy, k_slices, fused) as the override calls take them, the time the
+    tuner wrote beside it (None if absent) -- or None for a comment line."""
+    body, _, note = ln.partition("#")
+    f = body.split()
+    if not f:
+        return None
+    if len(f) not in (11, 12, 13):
+        raise ValueError(f"not a dispatch-table line: {ln!r}")
+    var = {v: k for k, v in VAR_NAME.items()}[f[4]]
+    red = {v: k for k, v in RED_NAME.items()}[f[6]]
+    sch = {v: k for k, v in SCHED_NAME.items()}[f[9]]
+    kps = int(f[11]) if len(f) > 11 else 0
+    fz = int(f[12]) if len(f) > 12 else 0
+    plan = (var, int(f[5]), red, int(f[7]), int(f[8]), sch, int(f[10]), kps, fz)
+    us = None
+    words = note.split()
+    if len(words) >= 2 and words[1].rstrip(",") == "us":
+        try:
+            us = float(words[0])
+        except ValueError:
+            us = None
+    return (f[0], int(f[1]), int(f[2]), int(f[3])), plan, us
+
+
+def is_stale(recorded_us, measured_us: float, pct: float) -> bool:
+    """A table entry is stale when its plan now takes more than pct percent
+    longer than the time recorded for it (no recorded time: stale)."""
+    return recorded_us is None or measured_us > recorded_us * (1.0 + pct / 100.0)
 
 
 def _quant_w(fmt, w):
@@ -64,9 +101,6 @@ def _quant_x(fmt, x):
     if fmt == NVFP4:
         return qgd.quant_nv(x)
     return qgd.quant_act_per_token(x, qgd.QTYPE_INT8 if fmt == W8A8_INT8 else qgd.QTYPE_E4M3)
-
-
-SCHED_NAME = {0: "grid", 1: "persistent"}
 
 
 SMEM_PER_SM = 233472  # bytes of shared memory per SM on sm_100 (228 KB)
@@ -313,6 +347,9 @@ def main(argv=None):
     ap.add_argument("--out", default=qgd.DEFAULT_TABLE)
     ap.add_argument("--large-m", action="store_true", help="also tune the larger-M buckets")
     ap.add_argument("--resume", action="store_true")
+    ap.add_argument("--recheck", type=float, default=None, metavar="PCT",
+                    help="with --resume: time each kept entry's plan again and re-tune it when it is more "
+                         "than PCT percent slower than recorded")
     ap.add_argument("--only-m", default=None, help="comma-separated M values to tune")
     ap.add_argument("--tp8", action="store_true",
                     help="also tune the 8-way column-parallel shards of the 8B-class shapes (FP8_Dynamic)")
@@ -330,11 +367,13 @@ def main(argv=None):
     if args.tp8:
         wls.append(workloads.FP8_TP8)
     done = {}
+    if args.recheck is not None and not args.resume:
+        ap.error("--recheck needs --resume (it re-times the entries of an existing table)")
     if args.resume and os.path.exists(args.out):
         for ln in open(args.out):
-            f = ln.split("#")[0].split()
-            if len(f) in (11, 12, 13):
-                done[(f[0], int(f[1]), int(f[2]), int(f[3]))] = ln.rstrip("\n")
+            parsed = parse_table_line(ln)
+            if parsed is not None:
+                done[parsed[0]] = ln.rstrip("\n")
     only_m = set(int(m) for m in args.only_m.split(",")) if args.only_m else None
     t_start = time.time()
     lines = dict(done)
@@ -358,10 +397,27 @@ def main(argv=None):
                 if only_m and M not in only_m:
                     continue
                 key = (wl.fmt, N, K, M)
+                p = None
                 if key in done:
-                    continue
+                    if args.recheck is None:
+                        continue
+                    _, plan, rec_us = parse_table_line(done[key])
+                    p = Problem(wl.fmt, M, N, K, wl.seed, device)
+                    qgd.qgd_set_override(p.fid, *plan[:8])
+                    qgd.qgd_set_fused_override(p.fid, plan[8])
+                    p.ws.ensure(max(qgd.qgd_workspace_size(p.fid, M, N, K),
+                                    qgd.qgd_layer_workspace_size(p.fid, M, N, K)))
+                    now_us = p.time_plan()
+                    qgd.qgd_set_override(p.fid)
+                    qgd.qgd_set_fused_override(p.fid)
+                    if not is_stale(rec_us, now_us, args.recheck):
+                        log(f"{wl.fmt} N={N} K={K} M={M}: kept ({now_us:.2f} us now, {rec_us} us recorded)")
+                        del p
+                        continue
+                    log(f"{wl.fmt} N={N} K={K} M={M}: stale ({now_us:.2f} us now, {rec_us} us recorded), re-tuning")
                 t0 = time.time()
-                p = Problem(wl.fmt, M, N, K, wl.seed, device)
+                if p is None:
+                    p = Problem(wl.fmt, M, N, K, wl.seed, device)
                 best, allres = tune_problem(p, log, tp=(wl is workloads.FP8_TP8))
                 us, var, s, r, st, t, sch, occ, kps, fz = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9

@@ -440,6 +440,7 @@ def test_tuner_candidates_are_legal_plans(fmt, M, N, K):
                 mpad = tune.swap_mpad(M)
                 smem = 1024 + st * kps * (16384 + mpad * 128) + 1024 + ((128 + 8) * mpad * 4 if r == 3 else 0)
                 assert 2 * (smem + 1024) <= 233472
+    qgd.qgd_set_override(fid)
     qgd.qgd_set_fused_override(fid)
     # pair tiles split K (any count) only where they are fewer than the SM pairs
     pair_splits = sorted({c[1] for c in cands if c[0] == qgd.VARIANT_STANDARD_PAIR and c[1] > 1})
@@ -525,6 +526,9 @@ def test_shipped_table_covers_every_benchmarked_shape():
 def test_shipped_table_entries_run_as_written():
     # every entry of the shipped table is what a call of its bucket's token
     # count runs, field for field: none is silently legalised into another plan
+    for f in range(5):
+        qgd.qgd_set_override(f)
+        qgd.qgd_set_fused_override(f)
     qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
     fid = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "mxfp8": 3, "nvfp4": 4}
     var = {"standard": 0, "swap_ab": 1, "standard_pair": 2}
@@ -544,6 +548,39 @@ def test_shipped_table_entries_run_as_written():
         assert qgd.qgd_get_layer_plan(fmt, M, N, K)["fused"] == int(f[12]), ln
         n += 1
     assert n > 200
+
+
+def test_tuner_reads_back_every_shipped_table_line():
+    # the tuner's table-line parser (used by --resume / --recheck) gives back the
+    # plan each line names, in the override calls' argument order, and its time
+    from quantized_gemm_decode_b200 import tune
+
+    qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
+    for ln in open(qgd.DEFAULT_TABLE):
+        parsed = tune.parse_table_line(ln)
+        if parsed is None:
+            assert ln.startswith("#") or not ln.strip()
+            continue
+        (fmt, N, K, M), plan, us = parsed
+        assert us is not None and us > 0, ln
+        fid = tune.FMT_ID[fmt]
+        qgd.qgd_clear_dispatch_table()
+        qgd.qgd_set_override(fid, *plan[:8])
+        qgd.qgd_set_fused_override(fid, plan[8])
+        try:
+            p = qgd.qgd_get_layer_plan(fid, M, N, K)
+        finally:
+            qgd.qgd_set_override(fid)
+            qgd.qgd_set_fused_override(fid)
+            qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
+        assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["tile_n"], p["schedule"], p["k_slices"],
+                p["fused"]) == (plan[0], plan[1], plan[2], plan[3], plan[4], plan[5], plan[7], plan[8]), ln
+    assert tune.parse_table_line("   # only a comment") is None
+    with pytest.raises(ValueError):
+        tune.parse_table_line("fp8_dynamic 4096 4096 1 swap_ab 1")
+    # stale: more than PCT percent slower than recorded, or nothing recorded
+    assert not tune.is_stale(10.0, 11.4, 15.0) and tune.is_stale(10.0, 11.6, 15.0)
+    assert tune.is_stale(None, 1.0, 15.0)
 
 
 def test_binding_checks_gemm_operands_before_any_launch():
