@@ -75,6 +75,15 @@ def parse_table_line(ln: str):
     return (f[0], int(f[1]), int(f[2]), int(f[3])), plan, us
 
 
+def format_table_line(key, plan, us: float, gbs: float) -> str:
+    """One dispatch-table line: key (fmt, N, K, M bucket), plan as
+    parse_table_line returns it, and the measured time and bandwidth."""
+    fmt, N, K, M = key
+    var, s, r, st, t, sch, occ, kps, fz = plan
+    return (f"{fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} {occ} {kps} {fz}"
+            f"   # {us:.2f} us, {gbs:.0f} GB/s")
+
+
 def is_stale(recorded_us, measured_us: float, pct: float) -> bool:
     """A table entry is stale when its plan now takes more than pct percent
     longer than the time recorded for it (no recorded time: stale)."""
@@ -421,8 +430,7 @@ def main(argv=None):
                 best, allres = tune_problem(p, log, tp=(wl is workloads.FP8_TP8))
                 us, var, s, r, st, t, sch, occ, kps, fz = best
                 gbs = workloads.algorithmic_bytes(wl.fmt, M, N, K) / (us * 1e-6) / 1e9
-                lines[key] = (f"{wl.fmt} {N} {K} {M} {VAR_NAME[var]} {s} {RED_NAME[r]} {st} {t} {SCHED_NAME[sch]} "
-                              f"{occ} {kps} {fz}   # {us:.2f} us, {gbs:.0f} GB/s")
+                lines[key] = format_table_line(key, (var, s, r, st, t, sch, occ, kps, fz), us, gbs)
                 log(f"{wl.fmt} N={N} K={K} M={M}: {VAR_NAME[var]} s={s} {RED_NAME[r]} st={st} t={t} "
                     f"{SCHED_NAME[sch]} occ={occ} kps={kps} fused={fz} {us:.2f} us {gbs:.0f} GB/s "
                     f"({len(allres)} candidates, {time.time() - t0:.1f} s)")

@@ -575,6 +575,9 @@ def test_tuner_reads_back_every_shipped_table_line():
             qgd.qgd_load_dispatch_table(qgd.DEFAULT_TABLE)
         assert (p["variant"], p["split_k"], p["reduce"], p["stages"], p["tile_n"], p["schedule"], p["k_slices"],
                 p["fused"]) == (plan[0], plan[1], plan[2], plan[3], plan[4], plan[5], plan[7], plan[8]), ln
+        # and the writer gives the line back byte for byte from what was read
+        gbs = float(ln.split("#")[1].split(",")[1].split()[0])
+        assert tune.format_table_line((fmt, N, K, M), plan, us, gbs) == ln.rstrip("\n")
     assert tune.parse_table_line("   # only a comment") is None
     with pytest.raises(ValueError):
         tune.parse_table_line("fp8_dynamic 4096 4096 1 swap_ab 1")
