@@ -422,6 +422,7 @@ def main(argv=None):
                     if not is_stale(rec_us, now_us, args.recheck):
                         log(f"{wl.fmt} N={N} K={K} M={M}: kept ({now_us:.2f} us now, {rec_us} us recorded)")
                         del p
+                        torch.cuda.empty_cache()
                         continue
                     log(f"{wl.fmt} N={N} K={K} M={M}: stale ({now_us:.2f} us now, {rec_us} us recorded), re-tuning")
                 t0 = time.time()
